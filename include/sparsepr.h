@@ -1,0 +1,195 @@
+/*
+ * sparsepr.h -- C ABI of the SparsePR attention operator for NVIDIA B200 (sm_100a).
+ *
+ * SparsePR (arXiv 2608.18484) replaces one dense softmax-attention call by
+ *   (a) Response-Coupled Partitioning: keys, with their paired values, are grouped by
+ *       their responses to a sample of queries; queries are then grouped by their
+ *       responses to the key-group centroids, in one asymmetric pass;
+ *   (b) shared block routing: each query block evaluates the key groups with the
+ *       largest centroid score, up to an executed-pair density budget that counts the
+ *       probe rows;
+ *   (c) block-sparse softmax attention over the routed (query block, key group) pairs;
+ *   (d) Probe-Fitted Residual Reconstruction: exact attention on a few probe rows per
+ *       head calibrates a weighted-ridge affine map from sparse output to residual,
+ *       restricted to the top-r subspace of the probe residuals; the predicted residual
+ *       is added to every unprobed row.
+ * Sources: the paper's abstract (English text on the arxivdaily.com page for
+ * 2608.18484; also reprinted on the peercurrent.com digest) and the skillfed.io article
+ * "Partition the Support, Reconstruct the Residual", paragraph on the two components.
+ * The pages give the method in prose only; the readings this library takes where they
+ * are silent are stated at each call below.
+ *
+ * Conventions (all calls):
+ *  - Tensor arguments are DEVICE pointers owned by the caller; the library never
+ *    allocates, frees or synchronises on them.  Scratch space is the caller's
+ *    workspace `ws` of sparsepr_workspace_size() bytes (256-byte aligned), which
+ *    must not be shared by calls that may overlap on the GPU.
+ *  - Every call is asynchronous on `stream` (0 = legacy default stream).
+ *  - Layouts are contiguous row-major: Q, K, V, O are [Bt, H, N, d]; per-head index
+ *    arrays are [Bt, H, ...] as stated.  dtype is SPARSEPR_BF16 or SPARSEPR_F32;
+ *    d is 64 or 128; block B is 64 or 128; indices are int32, pair counts int64.
+ *  - Return value: SPARSEPR_OK or an error code; on error nothing was launched and
+ *    sparsepr_last_error() returns a message (thread-local).  Errors found on the
+ *    device (a NaN reaching a decision, a bounded wait that ran out) are recorded in a
+ *    status word inside `ws`; sparsepr_check() reads it.
+ *  - Partition state never persists between calls: each call's map is call-specific.
+ */
+#ifndef SPARSEPR_H
+#define SPARSEPR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sparsepr_stream_t; /* same type as cudaStream_t */
+
+enum {
+  SPARSEPR_OK = 0,
+  SPARSEPR_ERR_INVALID_ARG = 1,
+  SPARSEPR_ERR_UNSUPPORTED = 2,
+  SPARSEPR_ERR_CUDA = 3,
+  SPARSEPR_ERR_TIMEOUT = 4,   /* a bounded device-side wait gave up */
+  SPARSEPR_ERR_NONFINITE = 5  /* a NaN reached a clustering or routing decision */
+};
+
+enum { SPARSEPR_BF16 = 0, SPARSEPR_F32 = 1 };
+
+enum { SPARSEPR_WEIGHT_INV_NORM = 0, SPARSEPR_WEIGHT_UNIFORM = 1 };
+
+typedef struct sparsepr_params {
+  int32_t block;        /* B: query-block and key-group capacity (64 or 128)            */
+  int32_t n_sampled;    /* S: sampled queries that define key response profiles        */
+  int32_t n_probe;      /* P: exact probe rows per head                                 */
+  int32_t kmeans_iters; /* T: balanced k-means iterations on each side (>= 0)           */
+  int32_t rank;         /* r: residual subspace rank (clamped to d)                    */
+  int32_t weight_mode;  /* SPARSEPR_WEIGHT_*: probe weights when none are supplied      */
+  double density;       /* rho: executed-pair budget / N^2, probe rows counted          */
+  double ridge_lambda;  /* lambda: ridge on the centred weighted Gram (sum w = P)       */
+  float scale;          /* softmax scale tau; <= 0 selects 1/sqrt(d)                    */
+} sparsepr_params;
+
+/* Number of groups G = Gq = ceil(N / B): capacity-B groups that cover all N tokens. */
+int32_t sparsepr_num_groups(int32_t N, int32_t block);
+
+/* Routed key groups per query block (host arithmetic, no device work):
+ * k = clamp(floor((rho*N*N - P*N) / (N*B)), 1, G), evaluated in IEEE double in this
+ * order.  Reading: one uniform k for every block, so that k*N*B + P*N <= rho*N^2
+ * (the budget counts probes, as the abstract's density figure does). */
+int32_t sparsepr_route_k(int32_t N, int32_t block, double density, int32_t n_probe);
+
+/* Bytes of workspace one call sequence needs for these sizes (0 on invalid sizes). */
+size_t sparsepr_workspace_size(int32_t Bt, int32_t H, int32_t N, int32_t d,
+                               const sparsepr_params* params);
+
+/* (a) Response-Coupled Partitioning.
+ *   Q, K        [Bt,H,N,d] dtype.  V is not read: values follow their keys.
+ *   sample_idx  [S] int32 token indices of the sampled queries, or NULL for the
+ *               midpoint stride floor((2m+1)N/(2S)) (reading: the pages do not say
+ *               how queries are sampled).
+ *   Outputs:
+ *   key_perm    [Bt,H,G*B]  member tokens of key group g at [g*B, g*B+size), in
+ *               ascending token order, -1 in the padding slots.
+ *   key_gsize   [Bt,H,G]    members per key group (1..B).
+ *   query_perm  [Bt,H,Gq*B], qblock_size [Bt,H,Gq]: the same for query blocks.
+ *   block_scores[Bt,H,Gq,G] fp32 routing score of (query block b, key group g): the
+ *               mean over b's members of tau * q_i . mu_g, mu_g = mean key of g.
+ * Method: keys are clustered on profiles r_j[m] = tau q_{s_m} . k_j by T iterations of
+ * balanced k-means (start: contiguous chunks of B tokens; assignment: capacity-B
+ * proposal rounds, ties to lower group, then lower token); queries are clustered the
+ * same way on coordinates u_i[g] = tau q_i . mu_g.  Both clusterings run in the
+ * exactly equivalent head-dim form |x - c|_Gamma^2 with Gamma = Q_S^T Q_S (keys) or
+ * mu^T mu (queries), on tensor cores.  Resets the status word in ws. */
+int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int32_t H,
+                       int32_t N, int32_t d, const sparsepr_params* params,
+                       const int32_t* sample_idx, int32_t* key_perm, int32_t* key_gsize,
+                       int32_t* query_perm, int32_t* qblock_size, float* block_scores,
+                       void* ws, sparsepr_stream_t stream);
+
+/* (b) Centroid routing.  For every query block: the k key groups with the largest
+ * block score (ties to the lower group index), written in ascending group order, with
+ * k = sparsepr_route_k(N, B, density, P) (also returned in *k_out, host memory).
+ *   route          [Bt,H,Gq,k] int32
+ *   executed_pairs [Bt,H] int64 = sum_b qblock_size[b] * sum_{g in route(b)} key_gsize[g]
+ *                  + P*N: every evaluated (query, key) pair, probe rows counted.
+ * A NaN score sets SPARSEPR_ERR_NONFINITE in the status word (NaN ranks lowest). */
+int sparsepr_route(const float* block_scores, const int32_t* key_gsize,
+                   const int32_t* qblock_size, int32_t Bt, int32_t H, int32_t N,
+                   const sparsepr_params* params, int32_t* route, int32_t* k_out,
+                   int64_t* executed_pairs, void* ws, sparsepr_stream_t stream);
+
+/* (c) Block-sparse softmax attention.  Row i of query block b attends to the union of
+ * the members of the k routed key groups of b, softmax renormalised over that support:
+ *   S_out[i] = sum_j softmax_j(tau q_i . k_j) v_j,  written fp32 in token order
+ *   [Bt,H,N,d].  bf16 inputs run on tensor cores with fp32 accumulation. */
+int sparsepr_sparse_attn(const void* Q, const void* K, const void* V, int dtype,
+                         int32_t Bt, int32_t H, int32_t N, int32_t d, int32_t block,
+                         const int32_t* key_perm, const int32_t* key_gsize,
+                         const int32_t* query_perm, const int32_t* qblock_size,
+                         const int32_t* route, int32_t k, float scale, float* S_out,
+                         void* ws, sparsepr_stream_t stream);
+
+/* Dense softmax attention of every row against all N keys with the same kernel
+ * family (the comparator the density budget is measured against):
+ *   O_out [Bt,H,N,d] fp32. */
+int sparsepr_dense_attn(const void* Q, const void* K, const void* V, int dtype,
+                        int32_t Bt, int32_t H, int32_t N, int32_t d, int32_t block,
+                        float scale, float* O_out, void* ws, sparsepr_stream_t stream);
+
+/* (d1) Probe rows.  For each probe token p (probe_idx [Bt,H,P], distinct, in [0,N)):
+ *   probe_out    [Bt,H,P,d] fp32: exact attention of p against all N keys;
+ *   probe_sparse [Bt,H,P,d] fp32: p's block-sparse output over its block's route.
+ * Both are computed with the softmax weights carried at ~16-bit precision (split
+ * bf16 hi+lo products), because they are the only inputs of the residual fit. */
+int sparsepr_probe_dense(const void* Q, const void* K, const void* V, int dtype,
+                         int32_t Bt, int32_t H, int32_t N, int32_t d, int32_t block,
+                         const int32_t* probe_idx, int32_t P, const int32_t* key_perm,
+                         const int32_t* key_gsize, const int32_t* query_perm,
+                         const int32_t* route, int32_t k, float scale, float* probe_out,
+                         float* probe_sparse, void* ws, sparsepr_stream_t stream);
+
+/* (d2) Residual fit, per (batch, head), in fp64:
+ *   y_p = probe_out_p - probe_sparse_p;  w_p from `weights` [Bt,H,P] if not NULL,
+ *   else weight_mode (inverse squared norm of probe_out_p, or uniform), then scaled
+ *   so sum_p w_p = P;  U_r = top-r eigenvectors of sum_p w_p y_p y_p^T;
+ *   z_p = U_r^T y_p;  A = (Z_c^T W X_c)(X_c^T W X_c + lambda I)^-1 with X = probe_sparse
+ *   centred at its weighted mean;  b = zbar - A xbar.
+ *   Outputs M = U_r A [Bt,H,d,d] and beta = U_r b [Bt,H,d], fp32. */
+int sparsepr_fit_residual(const float* probe_sparse, const float* probe_out,
+                          const float* weights, int32_t Bt, int32_t H, int32_t d,
+                          int32_t P, double ridge_lambda, int32_t rank,
+                          int32_t weight_mode, float* M, float* beta, void* ws,
+                          sparsepr_stream_t stream);
+
+/* (d3) Apply: O_i = S_i + M S_i + beta for unprobed rows, O_p = probe_out_p for probe
+ * rows.  O [Bt,H,N,d] in out_dtype.  O may alias S_out when out_dtype is F32. */
+int sparsepr_apply_residual(const float* S_out, const float* M, const float* beta,
+                            const int32_t* probe_idx, const float* probe_out,
+                            int32_t Bt, int32_t H, int32_t N, int32_t d, int32_t P,
+                            void* O, int out_dtype, sparsepr_stream_t stream);
+
+/* Wait for `stream` and return the device status word in `ws` (SPARSEPR_OK, or the
+ * first device-side error since the last sparsepr_partition).  This is the only call
+ * that synchronises. */
+int sparsepr_check(const void* ws, sparsepr_stream_t stream);
+
+/* Message of the last host-side error on this thread ("" if none). */
+const char* sparsepr_last_error(void);
+
+/* ---- decision kernels on injected scores (used by the parity tests) ---------------
+ * sparsepr_test_fill: the capacity-B assignment used by every k-means iteration, run
+ *   on caller-supplied fp32 distances D [H, n, G] (device); labels [H, n] int32.
+ * sparsepr_test_topk: the routing selection on caller-supplied scores Sc [H, Gq, G];
+ *   route [H, Gq, k] int32.  Both use the same kernels as the operator. */
+size_t sparsepr_test_fill_workspace_size(int32_t H, int32_t n, int32_t G);
+int sparsepr_test_fill(const float* D, int32_t H, int32_t n, int32_t G, int32_t cap,
+                       int32_t* labels, void* ws, sparsepr_stream_t stream);
+int sparsepr_test_topk(const float* Sc, int32_t H, int32_t Gq, int32_t G, int32_t k,
+                       int32_t* route, void* ws, sparsepr_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPARSEPR_H */
