@@ -1,0 +1,13 @@
+"""SparsePR attention operator for NVIDIA B200 (sm_100a).
+
+The operator (arXiv 2608.18484) runs Response-Coupled Partitioning, centroid block
+routing, block-sparse attention and Probe-Fitted Residual Reconstruction in one call.
+All arithmetic runs in the CUDA library libsparsepr.so behind the C ABI declared in
+include/sparsepr.h; this package is its Python binding.
+"""
+from .sparsepr import (  # noqa: F401
+    BF16, ERR_CUDA, ERR_INVALID_ARG, ERR_NONFINITE, ERR_TIMEOUT, ERR_UNSUPPORTED, EXPORTED_SYMBOLS, F32, OK,
+    WEIGHT_INV_NORM, WEIGHT_UNIFORM, Partition, SparsePRConfig, SparsePRError, apply_residual, attention, check,
+    dense_attn, fit_residual, lib, new_workspace, num_groups, partition, probe_dense, probe_rows, route, route_k,
+    sparse_attn, test_fill, test_topk, workspace_size,
+)

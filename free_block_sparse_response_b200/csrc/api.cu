@@ -1,0 +1,481 @@
+// extern "C" entry points of libsparsepr (see include/sparsepr.h for the contract).
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/sparsepr.h"
+#include "attention.cuh"
+#include "common.cuh"
+#include "fit.cuh"
+#include "partition.cuh"
+#include "route.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(SPARSEPR_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define SPR_CUDA(call, where)                       \
+  do {                                              \
+    cudaError_t e_ = (call);                        \
+    if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+  } while (0)
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Byte offsets of every scratch region inside the caller's workspace.
+struct Layout {
+  size_t header = 0, sample_idx, gamma, gamma_hi, gamma_lo, nrm, cent_k, cent_q, wf, whi, wlo, eg, dmat,
+         prop_g0, prop_v0, labels, room, cnt, offs, cursor, bucket, list0, list1, list_len, prop_g, prop_v,
+         perm_tmp, perm_cursor, qblk, partial, fit, total;
+};
+
+Layout make_layout(int heads, int N, int d, int block, int S, int P) {
+  const size_t H = heads, n = N, G = spr::ceil_div(N, block), D = d;
+  Layout L;
+  size_t off = align_up(sizeof(spr::WorkspaceHeader));
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes);
+    return at;
+  };
+  L.sample_idx = take(sizeof(int) * static_cast<size_t>(S));
+  L.gamma = take(sizeof(float) * H * D * D);
+  L.gamma_hi = take(2 * H * D * D);
+  L.gamma_lo = take(2 * H * D * D);
+  L.nrm = take(sizeof(float) * H * n);
+  L.cent_k = take(sizeof(float) * H * G * D);
+  L.cent_q = take(sizeof(float) * H * G * D);
+  L.wf = take(sizeof(float) * H * G * D);
+  L.whi = take(2 * H * G * D);
+  L.wlo = take(2 * H * G * D);
+  L.eg = take(sizeof(float) * H * G);
+  L.dmat = take(sizeof(float) * H * n * G);
+  L.prop_g0 = take(sizeof(int) * H * n);
+  L.prop_v0 = take(sizeof(float) * H * n);
+  L.labels = take(sizeof(int) * H * n);
+  L.room = take(sizeof(int) * H * G);
+  L.cnt = take(sizeof(int) * H * G);
+  L.offs = take(sizeof(int) * H * G);
+  L.cursor = take(sizeof(int) * H * G);
+  L.bucket = take(sizeof(unsigned long long) * H * n);
+  L.list0 = take(sizeof(int) * H * n);
+  L.list1 = take(sizeof(int) * H * n);
+  L.list_len = take(sizeof(int) * 4);
+  L.prop_g = take(sizeof(int) * H * n);
+  L.prop_v = take(sizeof(float) * H * n);
+  L.perm_tmp = take(sizeof(int) * H * G * block);
+  L.perm_cursor = take(sizeof(int) * H * G);
+  L.qblk = take(sizeof(int) * H * n);
+  L.partial = take(P > 0 ? spr::probe_partial_bytes(heads, P, static_cast<int>(G), d) : 0);
+  L.fit = take(P > 0 ? sizeof(double) * H * spr::fit_scratch_doubles(P, d) : 0);
+  L.total = off;
+  return L;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+spr::WorkspaceHeader* header(void* ws) { return static_cast<spr::WorkspaceHeader*>(ws); }
+
+int check_shape(int32_t Bt, int32_t H, int32_t N, int32_t d) {
+  if (Bt < 1 || H < 1 || N < 1) return fail(SPARSEPR_ERR_INVALID_ARG, "Bt, H and N must be >= 1");
+  if (d != 64 && d != 128) return fail(SPARSEPR_ERR_UNSUPPORTED, "head dim %d: only 64 and 128 are built", d);
+  if (static_cast<long long>(Bt) * H * N > (1ll << 30))
+    return fail(SPARSEPR_ERR_UNSUPPORTED, "Bt*H*N above 2^30 tokens per call");
+  return SPARSEPR_OK;
+}
+
+int check_block(int32_t block) {
+  if (block != 64 && block != 128) return fail(SPARSEPR_ERR_UNSUPPORTED, "block %d: only 64 and 128 are built", block);
+  return SPARSEPR_OK;
+}
+
+int check_dtype(int dtype) {
+  if (dtype != SPARSEPR_BF16 && dtype != SPARSEPR_F32) return fail(SPARSEPR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  return SPARSEPR_OK;
+}
+
+float resolve_scale(float scale, int d) { return scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d)); }
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+}  // namespace
+
+extern "C" {
+
+int32_t sparsepr_num_groups(int32_t N, int32_t block) {
+  if (N < 1 || block < 1) return 0;
+  return spr::ceil_div(N, block);
+}
+
+int32_t sparsepr_route_k(int32_t N, int32_t block, double density, int32_t n_probe) {
+  if (N < 1 || block < 1) return 0;
+  const int32_t G = spr::ceil_div(N, block);
+  const double num = density * static_cast<double>(N) * static_cast<double>(N) -
+                     static_cast<double>(n_probe) * static_cast<double>(N);
+  const double k = std::floor(num / (static_cast<double>(N) * static_cast<double>(block)));
+  if (!(k >= 1.0)) return 1;
+  if (k >= static_cast<double>(G)) return G;
+  return static_cast<int32_t>(k);
+}
+
+size_t sparsepr_workspace_size(int32_t Bt, int32_t H, int32_t N, int32_t d, const sparsepr_params* p) {
+  if (p == nullptr || check_shape(Bt, H, N, d) != SPARSEPR_OK || check_block(p->block) != SPARSEPR_OK) return 0;
+  return make_layout(Bt * H, N, d, p->block, p->n_sampled > 0 ? p->n_sampled : 1, p->n_probe).total;
+}
+
+const char* sparsepr_last_error(void) { return g_last_error.c_str(); }
+
+int sparsepr_check(const void* ws, sparsepr_stream_t stream) {
+  if (ws == nullptr) return fail(SPARSEPR_ERR_INVALID_ARG, "null workspace");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  SPR_CUDA(cudaStreamSynchronize(st), "sparsepr_check: stream");
+  int status = 0;
+  SPR_CUDA(cudaMemcpy(&status, ws, sizeof(int), cudaMemcpyDeviceToHost), "sparsepr_check: read status");
+  if (status != SPARSEPR_OK) return fail(status, "device-side error %d recorded in the workspace", status);
+  return SPARSEPR_OK;
+}
+
+int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int32_t H, int32_t N, int32_t d,
+                       const sparsepr_params* p, const int32_t* sample_idx, int32_t* key_perm,
+                       int32_t* key_gsize, int32_t* query_perm, int32_t* qblock_size, float* block_scores,
+                       void* ws, sparsepr_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(Bt, H, N, d)) || (rc = check_dtype(dtype))) return rc;
+  if (p == nullptr) return fail(SPARSEPR_ERR_INVALID_ARG, "null params");
+  if ((rc = check_block(p->block))) return rc;
+  if (!Q || !K || !key_perm || !key_gsize || !query_perm || !qblock_size || !block_scores || !ws)
+    return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
+  if (p->n_sampled < 1 || p->n_sampled > N) return fail(SPARSEPR_ERR_INVALID_ARG, "n_sampled must be in [1, N]");
+  if (p->kmeans_iters < 0 || p->kmeans_iters > 64) return fail(SPARSEPR_ERR_INVALID_ARG, "kmeans_iters must be in [0, 64]");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int heads = Bt * H, B = p->block, G = spr::ceil_div(N, B), S = p->n_sampled;
+  const bool f32 = dtype == SPARSEPR_F32;
+  const float tau = resolve_scale(p->scale, d);
+  const Layout L = make_layout(heads, N, d, B, S, p->n_probe);
+  spr::WorkspaceHeader* hdr = header(ws);
+  int* status = &hdr->status;
+  SPR_CUDA(cudaMemsetAsync(ws, 0, sizeof(spr::WorkspaceHeader), st), "partition: reset status");
+  const int* sidx = sample_idx;
+  if (sidx == nullptr) {
+    SPR_CUDA(spr::launch_midpoint_stride(at<int>(ws, L.sample_idx), N, S, st), "partition: sample");
+    sidx = at<int>(ws, L.sample_idx);
+  }
+  float* gamma = at<float>(ws, L.gamma);
+  __nv_bfloat16* ghi = at<__nv_bfloat16>(ws, L.gamma_hi);
+  __nv_bfloat16* glo = at<__nv_bfloat16>(ws, L.gamma_lo);
+  float* nrm = at<float>(ws, L.nrm);
+  float* wf = at<float>(ws, L.wf);
+  __nv_bfloat16* whi = at<__nv_bfloat16>(ws, L.whi);
+  __nv_bfloat16* wlo = at<__nv_bfloat16>(ws, L.wlo);
+  float* eg = at<float>(ws, L.eg);
+
+  float* dmat = at<float>(ws, L.dmat);
+  spr::FillArgs fa{};
+  fa.D = dmat;
+  fa.prop_g0 = at<int>(ws, L.prop_g0);
+  fa.prop_v0 = at<float>(ws, L.prop_v0);
+  fa.heads = heads;
+  fa.n = N;
+  fa.G = G;
+  fa.cap = B;
+  fa.labels = at<int>(ws, L.labels);
+  fa.room = at<int>(ws, L.room);
+  fa.cnt = at<int>(ws, L.cnt);
+  fa.offs = at<int>(ws, L.offs);
+  fa.cursor = at<int>(ws, L.cursor);
+  fa.bucket = at<unsigned long long>(ws, L.bucket);
+  fa.list0 = at<int>(ws, L.list0);
+  fa.list1 = at<int>(ws, L.list1);
+  fa.list_len = at<int>(ws, L.list_len);
+  fa.prop_g = at<int>(ws, L.prop_g);
+  fa.prop_v = at<float>(ws, L.prop_v);
+  fa.hdr = hdr;
+
+  // One side of the partition: balanced k-means of the rows of X under metric gamma.
+  auto cluster = [&](const void* X, float* cent, int32_t* perm, int32_t* sizes) -> int {
+    spr::RowGemmArgs ra{};
+    ra.X = X;
+    ra.f32 = f32;
+    ra.heads = heads;
+    ra.n = N;
+    ra.d = d;
+    ra.status = status;
+    if (!f32) SPR_CUDA(spr::launch_split_bf16(gamma, ghi, glo, static_cast<size_t>(heads) * d * d, st), "split gamma");
+    ra.ncols = d;
+    ra.Bhi = ghi;
+    ra.Blo = glo;
+    ra.Bf32 = gamma;
+    ra.nrm_out = nrm;
+    SPR_CUDA(spr::launch_rowgemm(ra, false, st), "row norms");
+    SPR_CUDA(spr::launch_chunk_perm(perm, sizes, N, G, B, heads, st), "chunk start");
+    SPR_CUDA(spr::launch_centroid(X, f32, N, perm, sizes, G, B, heads, d, cent, st), "centroids");
+    for (int t = 0; t < p->kmeans_iters; ++t) {
+      SPR_CUDA(spr::launch_wmat(cent, gamma, G, heads, d, wf, whi, wlo, eg, st), "gamma centroids");
+      ra.ncols = G;
+      ra.Bhi = whi;
+      ra.Blo = wlo;
+      ra.Bf32 = wf;
+      ra.nrm = nrm;
+      ra.ecol = eg;
+      ra.tau2 = tau * tau;
+      ra.Dout = dmat;
+      ra.prop_g = at<int>(ws, L.prop_g0);
+      ra.prop_v = at<float>(ws, L.prop_v0);
+      ra.nrm_out = nullptr;
+      SPR_CUDA(spr::launch_rowgemm(ra, true, st), "distances");
+      SPR_CUDA(spr::launch_fill(fa, st), "capacity fill");
+      SPR_CUDA(spr::launch_build_perm(fa.labels, N, G, B, heads, at<int>(ws, L.perm_cursor), at<int>(ws, L.perm_tmp),
+                                      perm, sizes, status, st),
+               "permutation");
+      SPR_CUDA(spr::launch_centroid(X, f32, N, perm, sizes, G, B, heads, d, cent, st), "centroids");
+    }
+    return SPARSEPR_OK;
+  };
+
+  float* cent_k = at<float>(ws, L.cent_k);
+  float* cent_q = at<float>(ws, L.cent_q);
+  // keys: profiles against the sampled queries -> gamma = Q_S^T Q_S
+  SPR_CUDA(spr::launch_gram(Q, f32, static_cast<size_t>(N) * d, sidx, S, heads, d, gamma, st), "Q_S gram");
+  if ((rc = cluster(K, cent_k, key_perm, key_gsize))) return rc;
+  // queries: coordinates against the key-group mean keys -> gamma = mu^T mu
+  SPR_CUDA(spr::launch_gram(cent_k, true, static_cast<size_t>(G) * d, nullptr, G, heads, d, gamma, st), "mu gram");
+  if ((rc = cluster(Q, cent_q, query_perm, qblock_size))) return rc;
+  SPR_CUDA(spr::launch_block_scores(cent_q, cent_k, G, heads, d, tau, block_scores, st), "block scores");
+  return SPARSEPR_OK;
+}
+
+int sparsepr_route(const float* block_scores, const int32_t* key_gsize, const int32_t* qblock_size, int32_t Bt,
+                   int32_t H, int32_t N, const sparsepr_params* p, int32_t* route, int32_t* k_out,
+                   int64_t* executed_pairs, void* ws, sparsepr_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(Bt, H, N, 64))) return rc;
+  if (p == nullptr) return fail(SPARSEPR_ERR_INVALID_ARG, "null params");
+  if ((rc = check_block(p->block))) return rc;
+  if (!block_scores || !key_gsize || !qblock_size || !route || !ws)
+    return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
+  if (p->n_probe < 0 || p->n_probe > N) return fail(SPARSEPR_ERR_INVALID_ARG, "n_probe must be in [0, N]");
+  const int G = spr::ceil_div(N, p->block);
+  const int k = sparsepr_route_k(N, p->block, p->density, p->n_probe);
+  if (k_out) *k_out = k;
+  SPR_CUDA(spr::launch_route(block_scores, Bt * H, G, G, k, route, key_gsize, qblock_size,
+                             reinterpret_cast<long long*>(executed_pairs),
+                             static_cast<long long>(p->n_probe) * N, &header(ws)->status,
+                             reinterpret_cast<cudaStream_t>(stream)),
+           "route");
+  return SPARSEPR_OK;
+}
+
+static int attention_common(const void* Q, const void* K, const void* V, int dtype, int32_t Bt, int32_t H,
+                            int32_t N, int32_t d, int32_t block, const int32_t* key_perm, const int32_t* key_gsize,
+                            const int32_t* query_perm, const int32_t* qblock_size, const int32_t* route, int32_t k,
+                            float scale, float* out, bool dense, sparsepr_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(Bt, H, N, d)) || (rc = check_dtype(dtype)) || (rc = check_block(block))) return rc;
+  if (!Q || !K || !V || !out) return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
+  const int G = spr::ceil_div(N, block);
+  if (!dense) {
+    if (!key_perm || !key_gsize || !query_perm || !qblock_size || !route)
+      return fail(SPARSEPR_ERR_INVALID_ARG, "null partition or route");
+    if (k < 1 || k > G) return fail(SPARSEPR_ERR_INVALID_ARG, "k=%d outside [1, %d]", k, G);
+  }
+  spr::AttnArgs a{};
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.f32 = dtype == SPARSEPR_F32;
+  a.heads = Bt * H;
+  a.N = N;
+  a.d = d;
+  a.block = block;
+  a.G = G;
+  a.k = dense ? G : k;
+  a.key_perm = key_perm;
+  a.key_gsize = key_gsize;
+  a.query_perm = query_perm;
+  a.qblock_size = qblock_size;
+  a.route = route;
+  a.scale_log2 = resolve_scale(scale, d) * kLog2e;
+  a.out = out;
+  SPR_CUDA(spr::launch_attention(a, dense, reinterpret_cast<cudaStream_t>(stream)), dense ? "dense attention" : "sparse attention");
+  return SPARSEPR_OK;
+}
+
+int sparsepr_sparse_attn(const void* Q, const void* K, const void* V, int dtype, int32_t Bt, int32_t H, int32_t N,
+                         int32_t d, int32_t block, const int32_t* key_perm, const int32_t* key_gsize,
+                         const int32_t* query_perm, const int32_t* qblock_size, const int32_t* route, int32_t k,
+                         float scale, float* S_out, void* ws, sparsepr_stream_t stream) {
+  (void)ws;
+  return attention_common(Q, K, V, dtype, Bt, H, N, d, block, key_perm, key_gsize, query_perm, qblock_size, route, k,
+                          scale, S_out, false, stream);
+}
+
+int sparsepr_dense_attn(const void* Q, const void* K, const void* V, int dtype, int32_t Bt, int32_t H, int32_t N,
+                        int32_t d, int32_t block, float scale, float* O_out, void* ws, sparsepr_stream_t stream) {
+  (void)ws;
+  return attention_common(Q, K, V, dtype, Bt, H, N, d, block, nullptr, nullptr, nullptr, nullptr, nullptr, 0, scale,
+                          O_out, true, stream);
+}
+
+int sparsepr_probe_dense(const void* Q, const void* K, const void* V, int dtype, int32_t Bt, int32_t H, int32_t N,
+                         int32_t d, int32_t block, const int32_t* probe_idx, int32_t P, const int32_t* key_perm,
+                         const int32_t* key_gsize, const int32_t* query_perm, const int32_t* route, int32_t k,
+                         float scale, float* probe_out, float* probe_sparse, void* ws, sparsepr_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(Bt, H, N, d)) || (rc = check_dtype(dtype)) || (rc = check_block(block))) return rc;
+  if (P < 1 || P > N) return fail(SPARSEPR_ERR_INVALID_ARG, "P must be in [1, N]");
+  if (!Q || !K || !V || !probe_idx || !key_perm || !key_gsize || !query_perm || !route || !probe_out ||
+      !probe_sparse || !ws)
+    return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
+  const int G = spr::ceil_div(N, block);
+  if (k < 1 || k > G) return fail(SPARSEPR_ERR_INVALID_ARG, "k=%d outside [1, %d]", k, G);
+  const Layout L = make_layout(Bt * H, N, d, block, 1, P);
+  spr::ProbeArgs a{};
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.f32 = dtype == SPARSEPR_F32;
+  a.heads = Bt * H;
+  a.N = N;
+  a.d = d;
+  a.block = block;
+  a.G = G;
+  a.k = k;
+  a.P = P;
+  a.probe_idx = probe_idx;
+  a.key_perm = key_perm;
+  a.key_gsize = key_gsize;
+  a.query_perm = query_perm;
+  a.route = route;
+  a.scale_log2 = resolve_scale(scale, d) * kLog2e;
+  a.probe_out = probe_out;
+  a.probe_sparse = probe_sparse;
+  a.qblk = at<int>(ws, L.qblk);
+  a.partial = at<float>(ws, L.partial);
+  SPR_CUDA(spr::launch_probe(a, reinterpret_cast<cudaStream_t>(stream)), "probe rows");
+  return SPARSEPR_OK;
+}
+
+int sparsepr_fit_residual(const float* probe_sparse, const float* probe_out, const float* weights, int32_t Bt,
+                          int32_t H, int32_t d, int32_t P, double ridge_lambda, int32_t rank, int32_t weight_mode,
+                          float* M, float* beta, void* ws, sparsepr_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(Bt, H, 1, d))) return rc;
+  if (P < 1) return fail(SPARSEPR_ERR_INVALID_ARG, "P must be >= 1");
+  if (rank < 1) return fail(SPARSEPR_ERR_INVALID_ARG, "rank must be >= 1");
+  if (!(ridge_lambda >= 0.0)) return fail(SPARSEPR_ERR_INVALID_ARG, "ridge_lambda must be >= 0");
+  if (weight_mode != SPARSEPR_WEIGHT_INV_NORM && weight_mode != SPARSEPR_WEIGHT_UNIFORM)
+    return fail(SPARSEPR_ERR_INVALID_ARG, "unknown weight_mode %d", weight_mode);
+  if (!probe_sparse || !probe_out || !M || !beta || !ws) return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
+  if (spr::fit_smem_bytes(d, P) > 220 * 1024) return fail(SPARSEPR_ERR_UNSUPPORTED, "P=%d too large for the fit", P);
+  // The fit's scratch starts right after the header: no partition state is live any more
+  // and sparsepr_workspace_size() covers it.
+  const size_t off = align_up(sizeof(spr::WorkspaceHeader));
+  double* scratch = at<double>(ws, off);
+  SPR_CUDA(spr::launch_fit(probe_sparse, probe_out, weights, Bt * H, d, P, ridge_lambda, rank, weight_mode, scratch, M,
+                           beta, &header(ws)->status, reinterpret_cast<cudaStream_t>(stream)),
+           "fit");
+  return SPARSEPR_OK;
+}
+
+int sparsepr_apply_residual(const float* S_out, const float* M, const float* beta, const int32_t* probe_idx,
+                            const float* probe_out, int32_t Bt, int32_t H, int32_t N, int32_t d, int32_t P, void* O,
+                            int out_dtype, sparsepr_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(Bt, H, N, d)) || (rc = check_dtype(out_dtype))) return rc;
+  if (P < 0 || P > N) return fail(SPARSEPR_ERR_INVALID_ARG, "P must be in [0, N]");
+  if (!S_out || !M || !beta || !O || (P > 0 && (!probe_idx || !probe_out)))
+    return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
+  if (O == static_cast<const void*>(S_out) && out_dtype != SPARSEPR_F32)
+    return fail(SPARSEPR_ERR_INVALID_ARG, "in-place apply needs out_dtype F32");
+  SPR_CUDA(spr::launch_apply(S_out, M, beta, probe_idx, probe_out, Bt * H, N, d, P, O, out_dtype == SPARSEPR_F32,
+                             reinterpret_cast<cudaStream_t>(stream)),
+           "apply");
+  return SPARSEPR_OK;
+}
+
+int sparsepr_probe_rows(int32_t N, int32_t P, int32_t Bt, int32_t H, int32_t* probe_idx,
+                        sparsepr_stream_t stream) {
+  if (N < 1 || P < 1 || P > N || Bt < 1 || H < 1 || !probe_idx)
+    return fail(SPARSEPR_ERR_INVALID_ARG, "bad probe-row arguments");
+  SPR_CUDA(spr::launch_probe_rows(N, P, Bt * H, probe_idx, reinterpret_cast<cudaStream_t>(stream)), "probe rows");
+  return SPARSEPR_OK;
+}
+
+size_t sparsepr_test_fill_workspace_size(int32_t H, int32_t n, int32_t G) {
+  if (H < 1 || n < 1 || G < 1) return 0;
+  const size_t h = H, nn = n, g = G;
+  return align_up(sizeof(spr::WorkspaceHeader)) + align_up(4 * h * g * sizeof(int)) +
+         align_up(h * nn * sizeof(unsigned long long)) + 3 * align_up(h * nn * sizeof(int)) + align_up(4 * sizeof(int)) +
+         align_up(h * nn * sizeof(float));
+}
+
+int sparsepr_test_fill(const float* D, int32_t H, int32_t n, int32_t G, int32_t cap, int32_t* labels, void* ws,
+                       sparsepr_stream_t stream) {
+  if (!D || !labels || !ws || H < 1 || n < 1 || G < 1 || cap < 1)
+    return fail(SPARSEPR_ERR_INVALID_ARG, "bad fill arguments");
+  if (static_cast<long long>(G) * cap < n) return fail(SPARSEPR_ERR_INVALID_ARG, "G * cap < n");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t h = H, nn = n, g = G;
+  size_t off = align_up(sizeof(spr::WorkspaceHeader));
+  auto take = [&](size_t bytes) {
+    const size_t a = off;
+    off += align_up(bytes);
+    return a;
+  };
+  spr::FillArgs fa{};
+  fa.D = D;
+  fa.prop_g0 = nullptr;
+  fa.prop_v0 = nullptr;
+  fa.heads = H;
+  fa.n = n;
+  fa.G = G;
+  fa.cap = cap;
+  fa.labels = labels;
+  const size_t grp = take(4 * h * g * sizeof(int));
+  fa.room = at<int>(ws, grp);
+  fa.cnt = fa.room + h * g;
+  fa.offs = fa.cnt + h * g;
+  fa.cursor = fa.offs + h * g;
+  fa.bucket = at<unsigned long long>(ws, take(h * nn * sizeof(unsigned long long)));
+  fa.list0 = at<int>(ws, take(h * nn * sizeof(int)));
+  fa.list1 = at<int>(ws, take(h * nn * sizeof(int)));
+  fa.prop_g = at<int>(ws, take(h * nn * sizeof(int)));
+  fa.list_len = at<int>(ws, take(4 * sizeof(int)));
+  fa.prop_v = at<float>(ws, take(h * nn * sizeof(float)));
+  fa.hdr = header(ws);
+  SPR_CUDA(cudaMemsetAsync(ws, 0, sizeof(spr::WorkspaceHeader), st), "fill: reset status");
+  SPR_CUDA(spr::launch_fill(fa, st), "fill");
+  return SPARSEPR_OK;
+}
+
+int sparsepr_test_topk(const float* Sc, int32_t H, int32_t Gq, int32_t G, int32_t k, int32_t* route, void* ws,
+                       sparsepr_stream_t stream) {
+  if (!Sc || !route || !ws || H < 1 || Gq < 1 || G < 1 || k < 1 || k > G)
+    return fail(SPARSEPR_ERR_INVALID_ARG, "bad top-k arguments");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  SPR_CUDA(cudaMemsetAsync(ws, 0, sizeof(spr::WorkspaceHeader), st), "topk: reset status");
+  SPR_CUDA(spr::launch_route(Sc, H, Gq, G, k, route, nullptr, nullptr, nullptr, 0, &header(ws)->status, st), "topk");
+  return SPARSEPR_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,47 @@
+// Launch interface of the attention kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace spr {
+
+struct AttnArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  bool f32;
+  int heads, N, d, block, G, k;
+  const int* key_perm;
+  const int* key_gsize;
+  const int* query_perm;
+  const int* qblock_size;
+  const int* route;
+  float scale_log2;  // tau * log2(e)
+  float* out;
+};
+
+struct ProbeArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  bool f32;
+  int heads, N, d, block, G, k, P;
+  const int* probe_idx;
+  const int* key_perm;
+  const int* key_gsize;
+  const int* query_perm;
+  const int* route;
+  float scale_log2;
+  float* probe_out;
+  float* probe_sparse;
+  int* qblk;       // workspace [heads, N]
+  float* partial;  // workspace, probe_partial_bytes()
+};
+
+cudaError_t launch_attention(const AttnArgs& a, bool dense, cudaStream_t st);
+cudaError_t launch_probe(const ProbeArgs& a, cudaStream_t st);
+size_t probe_partial_bytes(int heads, int P, int G, int d);
+cudaError_t launch_probe_rows(int N, int P, int heads, int* probe_idx, cudaStream_t st);
+
+}  // namespace spr

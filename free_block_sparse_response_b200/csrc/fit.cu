@@ -1,0 +1,424 @@
+// Probe-Fitted Residual Reconstruction: the fit and the apply step (sm_100a).
+//
+// Source: SparsePR abstract (arXiv 2608.18484, arxivdaily.com English abstract): exact
+// probe rows calibrate an affine correction from the sparse output to the dense-minus-
+// sparse difference by weighted ridge regression, and the predicted residual is added
+// to every unprobed row; the skillfed.io article's paragraph on the two components adds
+// that the correction lives in the output subspace seen in the probe residuals.
+//
+// Fit, one CTA per (batch, head), fp64 throughout:
+//   w_p (caller / 1/|d_p|^2 / uniform) scaled to sum P;  y_p = d_p - s_p;
+//   C = sum_p w_p y_p y_p^T;  eigenvectors by Jacobi with the round-robin parallel
+//   ordering (d/2 disjoint rotations per step);  U_r = top-r;  z_p = U_r^T y_p;
+//   A = (Z_c^T W X_c)(X_c^T W X_c + lambda I)^-1 by Cholesky;  b = zbar - A xbar;
+//   M = U_r A, beta = U_r b.
+#include "common.cuh"
+#include "fit.cuh"
+
+namespace spr {
+
+constexpr int kFitThreads = 512;
+constexpr int kStageRows = 16;
+
+__device__ double block_sum_d(double v, double* red) {
+  v = warp_sum_d(v);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  double s = 0.0;
+  for (int w = 0; w < kFitThreads / 32; ++w) s += red[w];
+  return s;
+}
+
+__host__ __device__ size_t fit_scratch_doubles(int P, int d) {
+  return static_cast<size_t>(d) * d + static_cast<size_t>(P) * d + static_cast<size_t>(d) * d + 4ull * d;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kFitThreads)
+    fit_kernel(const float* __restrict__ xs_all, const float* __restrict__ dp_all,
+               const float* __restrict__ weights, int P, double lambda, int R, int weight_mode,
+               double* __restrict__ scratch, float* __restrict__ M_out, float* __restrict__ beta_out,
+               int* __restrict__ status) {
+  constexpr int LD = D + 1;
+  extern __shared__ __align__(16) double sm[];
+  double* C = sm;                          // D x LD
+  double* w = C + D * LD;                  // P
+  double* stage = w + P;                   // kStageRows x D
+  __shared__ double red[kFitThreads / 32];
+  __shared__ double pc[D / 2], ps[D / 2];
+  __shared__ int pp[D / 2], pq[D / 2], order[D];
+  __shared__ double xbar[D], zbar[D], bvec[D];
+  __shared__ int s_fail;
+
+  const int head = blockIdx.x, tid = threadIdx.x;
+  const float* xs = xs_all + static_cast<size_t>(head) * P * D;
+  const float* dp = dp_all + static_cast<size_t>(head) * P * D;
+  double* Vt = scratch + static_cast<size_t>(head) * fit_scratch_doubles(P, D);
+  double* Z = Vt + D * D;                  // P x R
+  double* A = Z + static_cast<size_t>(P) * D;  // R x D
+  if (tid == 0) s_fail = 0;
+
+  // ---- weights
+  for (int p = tid; p < P; p += kFitThreads) {
+    double wp = 1.0;
+    if (weights != nullptr) {
+      wp = weights[static_cast<size_t>(head) * P + p];
+    } else if (weight_mode == 0) {
+      double n2 = 0.0;
+      for (int e = 0; e < D; ++e) {
+        const double v = dp[static_cast<size_t>(p) * D + e];
+        n2 += v * v;
+      }
+      wp = 1.0 / fmax(n2, 1e-30);
+    }
+    w[p] = wp;
+  }
+  __syncthreads();
+  double wsum = 0.0;
+  for (int p = tid; p < P; p += kFitThreads) wsum += w[p];
+  wsum = block_sum_d(wsum, red);
+  if (!(wsum > 0.0)) {
+    if (tid == 0) record_error(status, kErrInvalidArg);
+    wsum = P;
+    for (int p = tid; p < P; p += kFitThreads) w[p] = 1.0;
+  }
+  __syncthreads();
+  for (int p = tid; p < P; p += kFitThreads) w[p] *= static_cast<double>(P) / wsum;
+  __syncthreads();
+
+  // ---- C = sum_p w_p y_p y_p^T
+  constexpr int kPer = D * D / kFitThreads;
+  double acc[kPer];
+#pragma unroll
+  for (int x = 0; x < kPer; ++x) acc[x] = 0.0;
+  for (int p0 = 0; p0 < P; p0 += kStageRows) {
+    __syncthreads();
+    for (int x = tid; x < kStageRows * D; x += kFitThreads) {
+      const int p = p0 + x / D, e = x % D;
+      stage[x] = p < P ? (static_cast<double>(dp[static_cast<size_t>(p) * D + e]) -
+                          static_cast<double>(xs[static_cast<size_t>(p) * D + e])) : 0.0;
+    }
+    __syncthreads();
+    for (int r = 0; r < kStageRows && p0 + r < P; ++r) {
+      const double wr = w[p0 + r];
+      const double* y = stage + r * D;
+#pragma unroll
+      for (int x = 0; x < kPer; ++x) {
+        const int ij = tid + x * kFitThreads;
+        acc[x] += wr * y[ij / D] * y[ij % D];
+      }
+    }
+  }
+#pragma unroll
+  for (int x = 0; x < kPer; ++x) {
+    const int ij = tid + x * kFitThreads;
+    C[(ij / D) * LD + ij % D] = acc[x];
+  }
+  for (int x = tid; x < D * D; x += kFitThreads) Vt[x] = (x / D == x % D) ? 1.0 : 0.0;
+  __syncthreads();
+
+  // ---- Jacobi, round-robin parallel ordering
+  double total = 0.0;
+  for (int x = tid; x < D * D; x += kFitThreads) {
+    const double v = C[(x / D) * LD + x % D];
+    total += v * v;
+  }
+  total = block_sum_d(total, red);
+  const double tol2 = 1e-28 * total;
+  for (int sweep = 0; sweep < 40; ++sweep) {
+    double off = 0.0;
+    for (int x = tid; x < D * D; x += kFitThreads) {
+      const int i = x / D, j = x % D;
+      if (i != j) {
+        const double v = C[i * LD + j];
+        off += v * v;
+      }
+    }
+    off = block_sum_d(off, red);
+    if (off <= tol2 || total == 0.0) break;
+    for (int round = 0; round < D - 1; ++round) {
+      if (tid < D / 2) {
+        int p, q;
+        if (tid == 0) {
+          p = round;
+          q = D - 1;
+        } else {
+          p = (round + tid) % (D - 1);
+          q = (round - tid + (D - 1)) % (D - 1);
+        }
+        if (p > q) {
+          const int t = p;
+          p = q;
+          q = t;
+        }
+        const double apq = C[p * LD + q];
+        double c = 1.0, s = 0.0;
+        if (apq != 0.0 && apq * apq > 1e-36 * total) {
+          const double theta = (C[q * LD + q] - C[p * LD + p]) / (2.0 * apq);
+          const double t = (theta >= 0.0 ? 1.0 : -1.0) / (fabs(theta) + sqrt(theta * theta + 1.0));
+          c = 1.0 / sqrt(t * t + 1.0);
+          s = t * c;
+        }
+        pp[tid] = p;
+        pq[tid] = q;
+        pc[tid] = c;
+        ps[tid] = s;
+      }
+      __syncthreads();
+      for (int x = tid; x < (D / 2) * D; x += kFitThreads) {  // rows: J^T C, and V^T rows
+        const int t = x / D, j = x % D;
+        const int p = pp[t], q = pq[t];
+        const double c = pc[t], s = ps[t];
+        if (s != 0.0) {
+          const double cp = C[p * LD + j], cq = C[q * LD + j];
+          C[p * LD + j] = c * cp - s * cq;
+          C[q * LD + j] = s * cp + c * cq;
+          const double vp = Vt[p * D + j], vq = Vt[q * D + j];
+          Vt[p * D + j] = c * vp - s * vq;
+          Vt[q * D + j] = s * vp + c * vq;
+        }
+      }
+      __syncthreads();
+      for (int x = tid; x < (D / 2) * D; x += kFitThreads) {  // columns: (J^T C) J
+        const int t = x % (D / 2), i = x / (D / 2);
+        const int p = pp[t], q = pq[t];
+        const double c = pc[t], s = ps[t];
+        if (s != 0.0) {
+          const double cp = C[i * LD + p], cq = C[i * LD + q];
+          C[i * LD + p] = c * cp - s * cq;
+          C[i * LD + q] = s * cp + c * cq;
+        }
+      }
+      __syncthreads();
+      if (tid < D / 2 && ps[tid] != 0.0) {
+        C[pp[tid] * LD + pq[tid]] = 0.0;
+        C[pq[tid] * LD + pp[tid]] = 0.0;
+      }
+      __syncthreads();
+    }
+  }
+  // ---- eigenvalues descending (stable on ties)
+  for (int i = tid; i < D; i += kFitThreads) {
+    const double li = C[i * LD + i];
+    int rank = 0;
+    for (int j = 0; j < D; ++j) {
+      const double lj = C[j * LD + j];
+      rank += (lj > li) || (lj == li && j < i);
+    }
+    order[rank] = i;
+  }
+  __syncthreads();
+
+  // ---- z_p = U_r^T y_p ; weighted means
+  for (int x = tid; x < P * R; x += kFitThreads) {
+    const int p = x / R, a = x % R;
+    const double* u = Vt + static_cast<size_t>(order[a]) * D;
+    double s = 0.0;
+    for (int e = 0; e < D; ++e)
+      s += u[e] * (static_cast<double>(dp[static_cast<size_t>(p) * D + e]) -
+                   static_cast<double>(xs[static_cast<size_t>(p) * D + e]));
+    Z[x] = s;
+  }
+  __syncthreads();
+  for (int e = tid; e < D; e += kFitThreads) {
+    double s = 0.0;
+    for (int p = 0; p < P; ++p) s += w[p] * xs[static_cast<size_t>(p) * D + e];
+    xbar[e] = s / static_cast<double>(P);
+  }
+  for (int a = tid; a < R; a += kFitThreads) {
+    double s = 0.0;
+    for (int p = 0; p < P; ++p) s += w[p] * Z[p * R + a];
+    zbar[a] = s / static_cast<double>(P);
+  }
+  __syncthreads();
+
+  // ---- Gram = X_c^T W X_c + lambda I  (into C)
+#pragma unroll
+  for (int x = 0; x < kPer; ++x) acc[x] = 0.0;
+  for (int p0 = 0; p0 < P; p0 += kStageRows) {
+    __syncthreads();
+    for (int x = tid; x < kStageRows * D; x += kFitThreads) {
+      const int p = p0 + x / D, e = x % D;
+      stage[x] = p < P ? static_cast<double>(xs[static_cast<size_t>(p) * D + e]) - xbar[e] : 0.0;
+    }
+    __syncthreads();
+    for (int r = 0; r < kStageRows && p0 + r < P; ++r) {
+      const double wr = w[p0 + r];
+      const double* xc = stage + r * D;
+#pragma unroll
+      for (int x = 0; x < kPer; ++x) {
+        const int ij = tid + x * kFitThreads;
+        acc[x] += wr * xc[ij / D] * xc[ij % D];
+      }
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int x = 0; x < kPer; ++x) {
+    const int ij = tid + x * kFitThreads;
+    C[(ij / D) * LD + ij % D] = acc[x] + ((ij / D == ij % D) ? lambda : 0.0);
+  }
+  // cross = Z_c^T W X_c  -> A (R x D), solved in place below
+  for (int x = tid; x < R * D; x += kFitThreads) {
+    const int a = x / D, e = x % D;
+    double s = 0.0;
+    for (int p = 0; p < P; ++p)
+      s += w[p] * (Z[p * R + a] - zbar[a]) * (static_cast<double>(xs[static_cast<size_t>(p) * D + e]) - xbar[e]);
+    A[x] = s;
+  }
+  __syncthreads();
+
+  // ---- Cholesky (lower, in C)
+  for (int j = 0; j < D; ++j) {
+    if (tid < 32) {
+      double s = 0.0;
+      for (int k = tid; k < j; k += 32) s += C[j * LD + k] * C[j * LD + k];
+      s = warp_sum_d(s);
+      if (tid == 0) {
+        const double dj = C[j * LD + j] - s;
+        if (!(dj > 0.0)) {
+          s_fail = 1;
+          C[j * LD + j] = 1.0;
+        } else {
+          C[j * LD + j] = sqrt(dj);
+        }
+      }
+    }
+    __syncthreads();
+    const double ljj = C[j * LD + j];
+    for (int i = j + 1 + tid; i < D; i += kFitThreads) {
+      double s = C[i * LD + j];
+      for (int k = 0; k < j; ++k) s -= C[i * LD + k] * C[j * LD + k];
+      C[i * LD + j] = s / ljj;
+    }
+    __syncthreads();
+  }
+  // ---- solve (L L^T) a_row = cross_row for every a (one warp per right-hand side)
+  const int lane = tid & 31, warp = tid >> 5;
+  for (int a = warp; a < R; a += kFitThreads / 32) {
+    double* x = A + static_cast<size_t>(a) * D;
+    for (int i = 0; i < D; ++i) {
+      double s = 0.0;
+      for (int k = lane; k < i; k += 32) s += C[i * LD + k] * x[k];
+      s = warp_sum_d(s);
+      if (lane == 0) x[i] = (x[i] - s) / C[i * LD + i];
+      __syncwarp();
+    }
+    for (int i = D - 1; i >= 0; --i) {
+      double s = 0.0;
+      for (int k = i + 1 + lane; k < D; k += 32) s += C[k * LD + i] * x[k];
+      s = warp_sum_d(s);
+      if (lane == 0) x[i] = (x[i] - s) / C[i * LD + i];
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  for (int a = tid; a < R; a += kFitThreads) {
+    double s = 0.0;
+    for (int e = 0; e < D; ++e) s += A[static_cast<size_t>(a) * D + e] * xbar[e];
+    bvec[a] = zbar[a] - s;
+  }
+  __syncthreads();
+  // ---- M = U_r A, beta = U_r b
+  const bool failed = s_fail != 0;
+  for (int x = tid; x < D * D; x += kFitThreads) {
+    const int i = x / D, j = x % D;
+    double s = 0.0;
+    for (int a = 0; a < R; ++a) s += Vt[static_cast<size_t>(order[a]) * D + i] * A[static_cast<size_t>(a) * D + j];
+    M_out[static_cast<size_t>(head) * D * D + x] = failed ? 0.f : static_cast<float>(s);
+  }
+  for (int i = tid; i < D; i += kFitThreads) {
+    double s = 0.0;
+    for (int a = 0; a < R; ++a) s += Vt[static_cast<size_t>(order[a]) * D + i] * bvec[a];
+    beta_out[static_cast<size_t>(head) * D + i] = failed ? 0.f : static_cast<float>(s);
+  }
+  if (failed && tid == 0) record_error(status, kErrInvalidArg);
+}
+
+// O = S + S M^T + beta, 32 rows per CTA; M^T and the rows staged in shared memory.
+template <int D, typename TO>
+__global__ void __launch_bounds__(256)
+    apply_kernel(const float* __restrict__ S, const float* __restrict__ M, const float* __restrict__ beta, int N,
+                 TO* __restrict__ O) {
+  constexpr int kRows = 32;
+  extern __shared__ float fsm[];
+  float* Mt = fsm;               // [e][j] = M[j][e]
+  float* rows = Mt + D * D;      // kRows x D
+  const int head = blockIdx.y, row0 = blockIdx.x * kRows, tid = threadIdx.x;
+  const float* m = M + static_cast<size_t>(head) * D * D;
+  for (int x = tid; x < D * D; x += 256) Mt[(x % D) * D + x / D] = m[x];
+  const float* s = S + static_cast<size_t>(head) * N * D;
+  for (int x = tid; x < kRows * D; x += 256) {
+    const int r = row0 + x / D;
+    rows[x] = r < N ? s[static_cast<size_t>(r) * D + x % D] : 0.f;
+  }
+  __syncthreads();
+  const int j = tid % D;
+  const float bj = beta[static_cast<size_t>(head) * D + j];
+  for (int r = tid / D; r < kRows; r += 256 / D) {
+    if (row0 + r >= N) break;
+    const float* sr = rows + r * D;
+    float acc = sr[j] + bj;
+#pragma unroll 8
+    for (int e = 0; e < D; ++e) acc += sr[e] * Mt[e * D + j];
+    O[(static_cast<size_t>(head) * N + row0 + r) * D + j] = from_f32<TO>(acc);
+  }
+}
+
+template <int D, typename TO>
+__global__ void probe_overwrite_kernel(const int* __restrict__ probe_idx, const float* __restrict__ probe_out,
+                                       int N, int P, TO* __restrict__ O) {
+  const int p = blockIdx.x, head = blockIdx.y, e = threadIdx.x;
+  const int tok = probe_idx[static_cast<size_t>(head) * P + p];
+  O[(static_cast<size_t>(head) * N + tok) * D + e] =
+      from_f32<TO>(probe_out[(static_cast<size_t>(head) * P + p) * D + e]);
+}
+
+cudaError_t launch_fit(const float* xs, const float* dp, const float* weights, int heads, int d, int P,
+                       double lambda, int rank, int weight_mode, double* scratch, float* M, float* beta,
+                       int* status, cudaStream_t st) {
+  const int R = rank < d ? rank : d;
+  const size_t smem = (static_cast<size_t>(d) * (d + 1) + P + kStageRows * d) * sizeof(double);
+  if (d == 64) {
+    cudaError_t e = cudaFuncSetAttribute(fit_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    fit_kernel<64><<<heads, kFitThreads, smem, st>>>(xs, dp, weights, P, lambda, R, weight_mode, scratch, M, beta, status);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(fit_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    fit_kernel<128><<<heads, kFitThreads, smem, st>>>(xs, dp, weights, P, lambda, R, weight_mode, scratch, M, beta, status);
+  }
+  return cudaGetLastError();
+}
+
+size_t fit_smem_bytes(int d, int P) {
+  return (static_cast<size_t>(d) * (d + 1) + P + kStageRows * d) * sizeof(double);
+}
+
+template <int D, typename TO>
+static cudaError_t launch_apply_t(const float* S, const float* M, const float* beta, const int* probe_idx,
+                                  const float* probe_out, int heads, int N, int P, TO* O, cudaStream_t st) {
+  const size_t smem = (static_cast<size_t>(D) * D + 32 * D) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(apply_kernel<D, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  apply_kernel<D, TO><<<dim3(ceil_div(N, 32), heads), 256, smem, st>>>(S, M, beta, N, O);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || P == 0) return e;
+  probe_overwrite_kernel<D, TO><<<dim3(P, heads), D, 0, st>>>(probe_idx, probe_out, N, P, O);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_apply(const float* S, const float* M, const float* beta, const int* probe_idx,
+                         const float* probe_out, int heads, int N, int d, int P, void* O, bool out_f32,
+                         cudaStream_t st) {
+  if (d == 64) {
+    if (out_f32) return launch_apply_t<64, float>(S, M, beta, probe_idx, probe_out, heads, N, P, static_cast<float*>(O), st);
+    return launch_apply_t<64, __nv_bfloat16>(S, M, beta, probe_idx, probe_out, heads, N, P, static_cast<__nv_bfloat16*>(O), st);
+  }
+  if (out_f32) return launch_apply_t<128, float>(S, M, beta, probe_idx, probe_out, heads, N, P, static_cast<float*>(O), st);
+  return launch_apply_t<128, __nv_bfloat16>(S, M, beta, probe_idx, probe_out, heads, N, P, static_cast<__nv_bfloat16*>(O), st);
+}
+
+}  // namespace spr

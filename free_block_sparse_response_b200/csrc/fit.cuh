@@ -1,0 +1,18 @@
+// Launch interface of the fit and apply kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace spr {
+
+__host__ __device__ size_t fit_scratch_doubles(int P, int d);
+size_t fit_smem_bytes(int d, int P);
+cudaError_t launch_fit(const float* xs, const float* dp, const float* weights, int heads, int d, int P,
+                       double lambda, int rank, int weight_mode, double* scratch, float* M, float* beta,
+                       int* status, cudaStream_t st);
+cudaError_t launch_apply(const float* S, const float* M, const float* beta, const int* probe_idx,
+                         const float* probe_out, int heads, int N, int d, int P, void* O, bool out_f32,
+                         cudaStream_t st);
+
+}  // namespace spr

@@ -1,0 +1,65 @@
+// Launch interface of the partition kernels (internal to the library).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "common.cuh"
+
+namespace spr {
+
+struct RowGemmArgs {
+  const void* X;  // [heads, n, d] bf16 or f32
+  bool f32;
+  int heads, n, d, ncols;
+  const __nv_bfloat16* Bhi;  // [heads, ncols, d] (bf16 path)
+  const __nv_bfloat16* Blo;  // optional low part (split precision)
+  const float* Bf32;         // [heads, ncols, d] (fp32 path)
+  const float* nrm;          // DIST: [heads, n]
+  const float* ecol;         // DIST: [heads, ncols]
+  float tau2;
+  float* Dout;               // DIST: [heads, n, ncols]
+  int* prop_g;               // DIST: [heads, n]
+  float* prop_v;
+  float* nrm_out;            // NORM: [heads, n]
+  int* status;
+};
+
+struct FillArgs {
+  const float* D;       // [heads, n, G]
+  const int* prop_g0;   // optional first proposals [heads, n]
+  const float* prop_v0;
+  int heads, n, G, cap;
+  int* labels;          // [heads, n]
+  int* room;            // [heads, G]
+  int* cnt;
+  int* offs;
+  int* cursor;
+  unsigned long long* bucket;  // [heads, n]
+  int* list0;           // [heads * n]
+  int* list1;
+  int* list_len;        // [2]
+  int* prop_g;          // [heads, n]
+  float* prop_v;
+  WorkspaceHeader* hdr;
+};
+
+cudaError_t launch_midpoint_stride(int* idx, int n, int count, cudaStream_t st);
+cudaError_t launch_gram(const void* X, bool f32, size_t head_stride, const int* rows, int nrows, int heads,
+                        int d, float* gamma, cudaStream_t st);
+cudaError_t launch_split_bf16(const float* src, __nv_bfloat16* hi, __nv_bfloat16* lo, size_t count,
+                              cudaStream_t st);
+cudaError_t launch_chunk_perm(int* perm, int* sizes, int n, int G, int cap, int heads, cudaStream_t st);
+cudaError_t launch_centroid(const void* X, bool f32, int n, const int* perm, const int* sizes, int G, int cap,
+                            int heads, int d, float* cent, cudaStream_t st);
+cudaError_t launch_wmat(const float* cent, const float* gamma, int G, int heads, int d, float* wf,
+                        __nv_bfloat16* whi, __nv_bfloat16* wlo, float* eg, cudaStream_t st);
+cudaError_t launch_rowgemm(const RowGemmArgs& a, bool dist, cudaStream_t st);
+cudaError_t launch_fill(const FillArgs& a, cudaStream_t st);
+cudaError_t launch_build_perm(const int* labels, int n, int G, int cap, int heads, int* cursor, int* tmp,
+                              int* perm, int* sizes, int* status, cudaStream_t st);
+cudaError_t launch_block_scores(const float* qbar, const float* mu, int G, int heads, int d, float tau,
+                                float* sc, cudaStream_t st);
+
+}  // namespace spr

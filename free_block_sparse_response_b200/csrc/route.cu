@@ -1,0 +1,125 @@
+// Centroid-based block routing (sm_100a).
+//
+// Source: SparsePR abstract (arXiv 2608.18484, arxivdaily.com English abstract): query
+// groups share one sparse route chosen from their responses to the key-group centroids,
+// and the executed-pair density counts the exact probe rows.  Each query block keeps the
+// k key groups with the largest score (ties to the lower group), listed in ascending
+// group order; one warp per block row selects them by radix select on 64-bit keys.
+#include "common.cuh"
+#include "route.cuh"
+
+namespace spr {
+
+// Smaller key = preferred: high word = inverted order key of the score (largest score
+// first; NaN ranks last), low word = group index (lower group first on ties).
+__device__ __forceinline__ unsigned long long route_key(float v, int g) {
+  const uint32_t hi = (v != v) ? 0xffffffffu : ~float_order_key(v);
+  return (static_cast<unsigned long long>(hi) << 32) | static_cast<uint32_t>(g);
+}
+
+__global__ void __launch_bounds__(256)
+    route_topk_kernel(const float* __restrict__ sc, int Gq, int G, int k, int* __restrict__ route,
+                      const int* __restrict__ key_gsize, const int* __restrict__ qblock_size,
+                      unsigned long long* __restrict__ pairs, int* __restrict__ status) {
+  __shared__ unsigned int hist[8][256];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int head = blockIdx.y;
+  const int b = blockIdx.x * 8 + warp;
+  if (b >= Gq) return;
+  const float* row = sc + (static_cast<size_t>(head) * Gq + b) * G;
+  unsigned int* h = hist[warp];
+  // radix select the k-th smallest key
+  unsigned long long prefix = 0;
+  int kth = k;
+  bool saw_nan = false;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int x = lane; x < 256; x += 32) h[x] = 0;
+    __syncwarp();
+    const unsigned long long hmask = shift == 56 ? 0ull : (~0ull << (shift + 8));
+    for (int g = lane; g < G; g += 32) {
+      const float v = row[g];
+      saw_nan |= (v != v);
+      const unsigned long long key = route_key(v, g);
+      if ((key & hmask) == prefix) atomicAdd(&h[(key >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    unsigned int local[8], tot = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      local[j] = h[8 * lane + j];
+      tot += local[j];
+    }
+    unsigned int incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const unsigned int excl = incl - tot;
+    const bool mine = excl < static_cast<unsigned int>(kth) && static_cast<unsigned int>(kth) <= incl;
+    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    int digit = 0;
+    unsigned int before = 0;
+    if (mine) {
+      unsigned int acc = excl;
+      for (int j = 0; j < 8; ++j) {
+        if (acc + local[j] >= static_cast<unsigned int>(kth)) {
+          digit = 8 * lane + j;
+          before = acc;
+          break;
+        }
+        acc += local[j];
+      }
+    }
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    before = __shfl_sync(0xffffffffu, before, src);
+    kth -= static_cast<int>(before);
+    prefix |= static_cast<unsigned long long>(digit) << shift;
+    __syncwarp();
+  }
+  // emit the selected groups in ascending order and count the executed pairs
+  int* out = route + (static_cast<size_t>(head) * Gq + b) * k;
+  int written = 0;
+  long long member_sum = 0;
+  for (int g0 = 0; g0 < G; g0 += 32) {
+    const int g = g0 + lane;
+    const bool sel = g < G && route_key(row[g], g) <= prefix;
+    const unsigned int ball = __ballot_sync(0xffffffffu, sel);
+    const int slot = written + __popc(ball & ((1u << lane) - 1u));
+    if (sel && slot < k) {
+      out[slot] = g;
+      if (key_gsize != nullptr) member_sum += key_gsize[static_cast<size_t>(head) * G + g];
+    }
+    written += __popc(ball);
+  }
+  if (lane == 0 && (saw_nan || written != k)) record_error(status, written != k ? kErrInvalidArg : kErrNonFinite);
+  if (pairs != nullptr) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) member_sum += __shfl_xor_sync(0xffffffffu, member_sum, o);
+    if (lane == 0) {
+      const long long nb = qblock_size[static_cast<size_t>(head) * Gq + b];
+      atomicAdd(pairs + head, static_cast<unsigned long long>(nb * member_sum));
+    }
+  }
+}
+
+__global__ void pairs_init_kernel(unsigned long long* pairs, int heads, long long probe_pairs) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h < heads) pairs[h] = static_cast<unsigned long long>(probe_pairs);
+}
+
+cudaError_t launch_route(const float* sc, int heads, int Gq, int G, int k, int* route, const int* key_gsize,
+                         const int* qblock_size, long long* pairs, long long probe_pairs, int* status,
+                         cudaStream_t st) {
+  unsigned long long* up = reinterpret_cast<unsigned long long*>(pairs);
+  if (up != nullptr) {
+    pairs_init_kernel<<<ceil_div(heads, 256), 256, 0, st>>>(up, heads, probe_pairs);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  route_topk_kernel<<<dim3(ceil_div(Gq, 8), heads), 256, 0, st>>>(sc, Gq, G, k, route, key_gsize, qblock_size,
+                                                                   up, status);
+  return cudaGetLastError();
+}
+
+}  // namespace spr

@@ -1,0 +1,314 @@
+"""Python binding of libsparsepr (the SparsePR C ABI in include/sparsepr.h).
+
+Argument marshalling only: torch provides device memory and the current stream, every
+step of the attention call runs in the library's CUDA kernels.  There is no CPU or
+PyTorch fallback: if the library is not built, or no GPU is present, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import NamedTuple, Optional
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsparsepr.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NONFINITE = range(6)
+BF16, F32 = 0, 1
+WEIGHT_INV_NORM, WEIGHT_UNIFORM = 0, 1
+_DTYPE_CODE = {torch.bfloat16: BF16, torch.float32: F32}
+
+EXPORTED_SYMBOLS = (
+    "sparsepr_num_groups", "sparsepr_route_k", "sparsepr_probe_rows", "sparsepr_workspace_size",
+    "sparsepr_partition", "sparsepr_route", "sparsepr_sparse_attn", "sparsepr_dense_attn",
+    "sparsepr_probe_dense", "sparsepr_fit_residual", "sparsepr_apply_residual", "sparsepr_check",
+    "sparsepr_last_error", "sparsepr_test_fill_workspace_size", "sparsepr_test_fill",
+    "sparsepr_test_topk",
+)
+
+
+class SparsePRError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"[sparsepr error {code}] {message}")
+        self.code = code
+
+
+class _CParams(ctypes.Structure):
+    _fields_ = [("block", ctypes.c_int32), ("n_sampled", ctypes.c_int32), ("n_probe", ctypes.c_int32),
+                ("kmeans_iters", ctypes.c_int32), ("rank", ctypes.c_int32), ("weight_mode", ctypes.c_int32),
+                ("density", ctypes.c_double), ("ridge_lambda", ctypes.c_double), ("scale", ctypes.c_float)]
+
+
+@dataclasses.dataclass(frozen=True)
+class SparsePRConfig:
+    """Parameters of one call: block B, sampled queries S, probe rows P, k-means
+    iterations T, subspace rank r, probe weighting, density rho, ridge lambda, scale."""
+    block: int = 128
+    n_sampled: int = 512
+    n_probe: int = 256
+    kmeans_iters: int = 4
+    rank: int = 32
+    weight_mode: int = WEIGHT_INV_NORM
+    density: float = 0.22
+    ridge_lambda: float = 1e-3
+    scale: float = 0.0
+
+    def c(self) -> _CParams:
+        return _CParams(self.block, self.n_sampled, self.n_probe, self.kmeans_iters, self.rank,
+                        self.weight_mode, self.density, self.ridge_lambda, self.scale)
+
+
+_LIB = None
+_vp, _i32, _i64p, _f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_float
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsparsepr.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is not built; run `python -m free_block_sparse_response_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER(_CParams)
+    sig = {
+        "sparsepr_num_groups": (_i32, [_i32, _i32]),
+        "sparsepr_route_k": (_i32, [_i32, _i32, ctypes.c_double, _i32]),
+        "sparsepr_probe_rows": (ctypes.c_int, [_i32, _i32, _i32, _i32, _vp, _vp]),
+        "sparsepr_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32, _i32, P]),
+        "sparsepr_partition": (ctypes.c_int, [_vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32, P, _vp, _vp, _vp,
+                                              _vp, _vp, _vp, _vp, _vp]),
+        "sparsepr_route": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i32, _i32, P, _vp, ctypes.POINTER(_i32), _vp,
+                                          _vp, _vp]),
+        "sparsepr_sparse_attn": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32, _i32, _vp,
+                                                _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _vp]),
+        "sparsepr_dense_attn": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32, _i32, _f32,
+                                               _vp, _vp, _vp]),
+        "sparsepr_probe_dense": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32, _i32, _vp,
+                                                _i32, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _vp, _vp]),
+        "sparsepr_fit_residual": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, ctypes.c_double, _i32,
+                                                 _i32, _vp, _vp, _vp, _vp]),
+        "sparsepr_apply_residual": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp,
+                                                   ctypes.c_int, _vp]),
+        "sparsepr_check": (ctypes.c_int, [_vp, _vp]),
+        "sparsepr_last_error": (ctypes.c_char_p, []),
+        "sparsepr_test_fill_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32]),
+        "sparsepr_test_fill": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+        "sparsepr_test_topk": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _LIB = L
+    return L
+
+
+def _call(name: str, *args) -> int:
+    rc = getattr(lib(), name)(*args)
+    if rc != OK:
+        msg = lib().sparsepr_last_error().decode(errors="replace")
+        raise SparsePRError(rc, f"{name}: {msg}")
+    return rc
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _need_cuda(*ts: torch.Tensor) -> None:
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("SparsePR tensors must live on a CUDA device")
+        if not t.is_contiguous():
+            raise ValueError("SparsePR tensors must be contiguous")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype not in _DTYPE_CODE:
+        raise ValueError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+    return _DTYPE_CODE[t.dtype]
+
+
+# ------------------------------------------------------------------------ host helpers
+
+def num_groups(n: int, block: int) -> int:
+    return int(lib().sparsepr_num_groups(n, block))
+
+
+def route_k(n: int, block: int, density: float, n_probe: int) -> int:
+    return int(lib().sparsepr_route_k(n, block, density, n_probe))
+
+
+def workspace_size(batch: int, heads: int, n: int, d: int, cfg: SparsePRConfig) -> int:
+    size = int(lib().sparsepr_workspace_size(batch, heads, n, d, ctypes.byref(cfg.c())))
+    if size == 0:
+        raise SparsePRError(ERR_INVALID_ARG, "invalid sizes for the workspace")
+    return size
+
+
+def new_workspace(batch: int, heads: int, n: int, d: int, cfg: SparsePRConfig, device) -> torch.Tensor:
+    return torch.empty(workspace_size(batch, heads, n, d, cfg), dtype=torch.uint8, device=device)
+
+
+def check(ws: torch.Tensor) -> None:
+    """Wait for the current stream and raise if a device-side error was recorded."""
+    _call("sparsepr_check", _p(ws), _stream(ws))
+
+
+# ----------------------------------------------------------------------------- stages
+
+class Partition(NamedTuple):
+    key_perm: torch.Tensor      # [Bt, H, G*B] int32, -1 pads
+    key_gsize: torch.Tensor     # [Bt, H, G] int32
+    query_perm: torch.Tensor    # [Bt, H, G*B] int32
+    qblock_size: torch.Tensor   # [Bt, H, G] int32
+    block_scores: torch.Tensor  # [Bt, H, G, G] fp32
+
+
+def partition(q, k, cfg: SparsePRConfig, ws: torch.Tensor, sample_idx: Optional[torch.Tensor] = None) -> Partition:
+    _need_cuda(q, k, ws, sample_idx)
+    bt, h, n, d = q.shape
+    g = num_groups(n, cfg.block)
+    dev = q.device
+    out = Partition(
+        torch.empty(bt, h, g * cfg.block, dtype=torch.int32, device=dev),
+        torch.empty(bt, h, g, dtype=torch.int32, device=dev),
+        torch.empty(bt, h, g * cfg.block, dtype=torch.int32, device=dev),
+        torch.empty(bt, h, g, dtype=torch.int32, device=dev),
+        torch.empty(bt, h, g, g, dtype=torch.float32, device=dev))
+    _call("sparsepr_partition", _p(q), _p(k), _dtype_code(q), bt, h, n, d, ctypes.byref(cfg.c()),
+          _p(sample_idx), *(_p(t) for t in out), _p(ws), _stream(q))
+    return out
+
+
+def route(part: Partition, n: int, cfg: SparsePRConfig, ws: torch.Tensor):
+    """Returns (route [Bt,H,G,k] int32, k, executed_pairs [Bt,H] int64)."""
+    bt, h, g, _ = part.block_scores.shape
+    kk = route_k(n, cfg.block, cfg.density, cfg.n_probe)
+    rt = torch.empty(bt, h, g, kk, dtype=torch.int32, device=ws.device)
+    pairs = torch.empty(bt, h, dtype=torch.int64, device=ws.device)
+    k_out = _i32(0)
+    _call("sparsepr_route", _p(part.block_scores), _p(part.key_gsize), _p(part.qblock_size), bt, h, n,
+          ctypes.byref(cfg.c()), _p(rt), ctypes.byref(k_out), _p(pairs), _p(ws), _stream(ws))
+    assert k_out.value == kk
+    return rt, kk, pairs
+
+
+def sparse_attn(q, k, v, part: Partition, rt: torch.Tensor, kk: int, cfg: SparsePRConfig,
+                out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need_cuda(q, k, v, rt)
+    bt, h, n, d = q.shape
+    s_out = torch.empty(bt, h, n, d, dtype=torch.float32, device=q.device) if out is None else out
+    _call("sparsepr_sparse_attn", _p(q), _p(k), _p(v), _dtype_code(q), bt, h, n, d, cfg.block,
+          _p(part.key_perm), _p(part.key_gsize), _p(part.query_perm), _p(part.qblock_size), _p(rt), kk,
+          cfg.scale, _p(s_out), _p(ws), _stream(q))
+    return s_out
+
+
+def dense_attn(q, k, v, block: int = 128, scale: float = 0.0, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Dense softmax attention of every row with the same kernel family (fp32 out)."""
+    _need_cuda(q, k, v)
+    bt, h, n, d = q.shape
+    o = torch.empty(bt, h, n, d, dtype=torch.float32, device=q.device) if out is None else out
+    _call("sparsepr_dense_attn", _p(q), _p(k), _p(v), _dtype_code(q), bt, h, n, d, block, scale, _p(o), None,
+          _stream(q))
+    return o
+
+
+def probe_rows(n: int, p: int, batch: int, heads: int, device) -> torch.Tensor:
+    idx = torch.empty(batch, heads, p, dtype=torch.int32, device=device)
+    _call("sparsepr_probe_rows", n, p, batch, heads, _p(idx), ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream))
+    return idx
+
+
+def probe_dense(q, k, v, probe_idx, part: Partition, rt, kk: int, cfg: SparsePRConfig, ws: torch.Tensor):
+    """Returns (probe_out, probe_sparse), each [Bt,H,P,d] fp32."""
+    _need_cuda(q, k, v, probe_idx, rt, ws)
+    bt, h, n, d = q.shape
+    p = probe_idx.shape[-1]
+    po = torch.empty(bt, h, p, d, dtype=torch.float32, device=q.device)
+    ps = torch.empty_like(po)
+    _call("sparsepr_probe_dense", _p(q), _p(k), _p(v), _dtype_code(q), bt, h, n, d, cfg.block, _p(probe_idx), p,
+          _p(part.key_perm), _p(part.key_gsize), _p(part.query_perm), _p(rt), kk, cfg.scale, _p(po), _p(ps),
+          _p(ws), _stream(q))
+    return po, ps
+
+
+def fit_residual(probe_sparse, probe_out, cfg: SparsePRConfig, ws: torch.Tensor,
+                 weights: Optional[torch.Tensor] = None):
+    """Returns (M [Bt,H,d,d], beta [Bt,H,d]) fp32."""
+    _need_cuda(probe_sparse, probe_out, ws, weights)
+    bt, h, p, d = probe_out.shape
+    m = torch.empty(bt, h, d, d, dtype=torch.float32, device=probe_out.device)
+    beta = torch.empty(bt, h, d, dtype=torch.float32, device=probe_out.device)
+    _call("sparsepr_fit_residual", _p(probe_sparse), _p(probe_out), _p(weights), bt, h, d, p, cfg.ridge_lambda,
+          cfg.rank, cfg.weight_mode, _p(m), _p(beta), _p(ws), _stream(probe_out))
+    return m, beta
+
+
+def apply_residual(s_out, m, beta, probe_idx, probe_out, out_dtype=torch.bfloat16,
+                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _need_cuda(s_out, m, beta, probe_idx, probe_out)
+    bt, h, n, d = s_out.shape
+    p = probe_idx.shape[-1]
+    o = torch.empty(bt, h, n, d, dtype=out_dtype, device=s_out.device) if out is None else out
+    _call("sparsepr_apply_residual", _p(s_out), _p(m), _p(beta), _p(probe_idx), _p(probe_out), bt, h, n, d, p,
+          _p(o), _DTYPE_CODE[o.dtype], _stream(s_out))
+    return o
+
+
+# --------------------------------------------------------------------------- the call
+
+def attention(q, k, v, cfg: SparsePRConfig, ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+              return_parts: bool = False):
+    """One SparsePR attention call: partition, route, sparse attention, probes, fit,
+    apply.  Returns O [Bt,H,N,d] in q's dtype (and the intermediates if asked).
+    Asynchronous on the current stream; ``check(ws)`` surfaces device-side errors."""
+    _need_cuda(q, k, v)
+    bt, h, n, d = q.shape
+    if ws is None:
+        ws = new_workspace(bt, h, n, d, cfg, q.device)
+    part = partition(q, k, cfg, ws)
+    rt, kk, pairs = route(part, n, cfg, ws)
+    s_out = sparse_attn(q, k, v, part, rt, kk, cfg, ws=ws)
+    pidx = probe_rows(n, cfg.n_probe, bt, h, q.device)
+    p_out, p_sparse = probe_dense(q, k, v, pidx, part, rt, kk, cfg, ws)
+    m, beta = fit_residual(p_sparse, p_out, cfg, ws)
+    o = apply_residual(s_out, m, beta, pidx, p_out, out_dtype=q.dtype, out=out)
+    if not return_parts:
+        return o
+    return o, {"partition": part, "route": rt, "k": kk, "executed_pairs": pairs, "S": s_out, "probe_idx": pidx,
+               "probe_out": p_out, "probe_sparse": p_sparse, "M": m, "beta": beta, "ws": ws}
+
+
+# ------------------------------------------------------- decision kernels, injected input
+
+def test_fill(dist: torch.Tensor, cap: int) -> torch.Tensor:
+    """Capacity fill on injected fp32 distances [H, n, G] -> labels [H, n] int32."""
+    _need_cuda(dist)
+    h, n, g = dist.shape
+    ws = torch.empty(int(lib().sparsepr_test_fill_workspace_size(h, n, g)), dtype=torch.uint8, device=dist.device)
+    labels = torch.empty(h, n, dtype=torch.int32, device=dist.device)
+    _call("sparsepr_test_fill", _p(dist), h, n, g, cap, _p(labels), _p(ws), _stream(dist))
+    check(ws)
+    return labels
+
+
+def test_topk(scores: torch.Tensor, k: int) -> torch.Tensor:
+    """Routing selection on injected fp32 scores [H, Gq, G] -> route [H, Gq, k] int32."""
+    _need_cuda(scores)
+    h, gq, g = scores.shape
+    ws = torch.zeros(256, dtype=torch.uint8, device=scores.device)
+    rt = torch.empty(h, gq, k, dtype=torch.int32, device=scores.device)
+    _call("sparsepr_test_topk", _p(scores), h, gq, g, k, _p(rt), _p(ws), _stream(scores))
+    check(ws)
+    return rt

@@ -44,6 +44,12 @@
 extern "C" {
 #endif
 
+#if defined(__GNUC__)
+#define SPARSEPR_API __attribute__((visibility("default")))
+#else
+#define SPARSEPR_API
+#endif
+
 typedef struct CUstream_st* sparsepr_stream_t; /* same type as cudaStream_t */
 
 enum {
@@ -72,16 +78,22 @@ typedef struct sparsepr_params {
 } sparsepr_params;
 
 /* Number of groups G = Gq = ceil(N / B): capacity-B groups that cover all N tokens. */
-int32_t sparsepr_num_groups(int32_t N, int32_t block);
+SPARSEPR_API int32_t sparsepr_num_groups(int32_t N, int32_t block);
 
 /* Routed key groups per query block (host arithmetic, no device work):
  * k = clamp(floor((rho*N*N - P*N) / (N*B)), 1, G), evaluated in IEEE double in this
  * order.  Reading: one uniform k for every block, so that k*N*B + P*N <= rho*N^2
  * (the budget counts probes, as the abstract's density figure does). */
-int32_t sparsepr_route_k(int32_t N, int32_t block, double density, int32_t n_probe);
+SPARSEPR_API int32_t sparsepr_route_k(int32_t N, int32_t block, double density, int32_t n_probe);
+
+/* Probe rows of every (batch, head): the midpoint stride floor((2p+1)N/(2P)), p < P,
+ * in raster token order (reading: the pages do not say how probe rows are chosen; a
+ * stride spreads them over all frames).  probe_idx [Bt,H,P] int32, device. */
+SPARSEPR_API int sparsepr_probe_rows(int32_t N, int32_t P, int32_t Bt, int32_t H, int32_t* probe_idx,
+                        sparsepr_stream_t stream);
 
 /* Bytes of workspace one call sequence needs for these sizes (0 on invalid sizes). */
-size_t sparsepr_workspace_size(int32_t Bt, int32_t H, int32_t N, int32_t d,
+SPARSEPR_API size_t sparsepr_workspace_size(int32_t Bt, int32_t H, int32_t N, int32_t d,
                                const sparsepr_params* params);
 
 /* (a) Response-Coupled Partitioning.
@@ -102,7 +114,7 @@ size_t sparsepr_workspace_size(int32_t Bt, int32_t H, int32_t N, int32_t d,
  * same way on coordinates u_i[g] = tau q_i . mu_g.  Both clusterings run in the
  * exactly equivalent head-dim form |x - c|_Gamma^2 with Gamma = Q_S^T Q_S (keys) or
  * mu^T mu (queries), on tensor cores.  Resets the status word in ws. */
-int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int32_t H,
+SPARSEPR_API int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int32_t H,
                        int32_t N, int32_t d, const sparsepr_params* params,
                        const int32_t* sample_idx, int32_t* key_perm, int32_t* key_gsize,
                        int32_t* query_perm, int32_t* qblock_size, float* block_scores,
@@ -115,7 +127,7 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
  *   executed_pairs [Bt,H] int64 = sum_b qblock_size[b] * sum_{g in route(b)} key_gsize[g]
  *                  + P*N: every evaluated (query, key) pair, probe rows counted.
  * A NaN score sets SPARSEPR_ERR_NONFINITE in the status word (NaN ranks lowest). */
-int sparsepr_route(const float* block_scores, const int32_t* key_gsize,
+SPARSEPR_API int sparsepr_route(const float* block_scores, const int32_t* key_gsize,
                    const int32_t* qblock_size, int32_t Bt, int32_t H, int32_t N,
                    const sparsepr_params* params, int32_t* route, int32_t* k_out,
                    int64_t* executed_pairs, void* ws, sparsepr_stream_t stream);
@@ -124,7 +136,7 @@ int sparsepr_route(const float* block_scores, const int32_t* key_gsize,
  * the members of the k routed key groups of b, softmax renormalised over that support:
  *   S_out[i] = sum_j softmax_j(tau q_i . k_j) v_j,  written fp32 in token order
  *   [Bt,H,N,d].  bf16 inputs run on tensor cores with fp32 accumulation. */
-int sparsepr_sparse_attn(const void* Q, const void* K, const void* V, int dtype,
+SPARSEPR_API int sparsepr_sparse_attn(const void* Q, const void* K, const void* V, int dtype,
                          int32_t Bt, int32_t H, int32_t N, int32_t d, int32_t block,
                          const int32_t* key_perm, const int32_t* key_gsize,
                          const int32_t* query_perm, const int32_t* qblock_size,
@@ -134,7 +146,7 @@ int sparsepr_sparse_attn(const void* Q, const void* K, const void* V, int dtype,
 /* Dense softmax attention of every row against all N keys with the same kernel
  * family (the comparator the density budget is measured against):
  *   O_out [Bt,H,N,d] fp32. */
-int sparsepr_dense_attn(const void* Q, const void* K, const void* V, int dtype,
+SPARSEPR_API int sparsepr_dense_attn(const void* Q, const void* K, const void* V, int dtype,
                         int32_t Bt, int32_t H, int32_t N, int32_t d, int32_t block,
                         float scale, float* O_out, void* ws, sparsepr_stream_t stream);
 
@@ -143,7 +155,7 @@ int sparsepr_dense_attn(const void* Q, const void* K, const void* V, int dtype,
  *   probe_sparse [Bt,H,P,d] fp32: p's block-sparse output over its block's route.
  * Both are computed with the softmax weights carried at ~16-bit precision (split
  * bf16 hi+lo products), because they are the only inputs of the residual fit. */
-int sparsepr_probe_dense(const void* Q, const void* K, const void* V, int dtype,
+SPARSEPR_API int sparsepr_probe_dense(const void* Q, const void* K, const void* V, int dtype,
                          int32_t Bt, int32_t H, int32_t N, int32_t d, int32_t block,
                          const int32_t* probe_idx, int32_t P, const int32_t* key_perm,
                          const int32_t* key_gsize, const int32_t* query_perm,
@@ -157,7 +169,7 @@ int sparsepr_probe_dense(const void* Q, const void* K, const void* V, int dtype,
  *   z_p = U_r^T y_p;  A = (Z_c^T W X_c)(X_c^T W X_c + lambda I)^-1 with X = probe_sparse
  *   centred at its weighted mean;  b = zbar - A xbar.
  *   Outputs M = U_r A [Bt,H,d,d] and beta = U_r b [Bt,H,d], fp32. */
-int sparsepr_fit_residual(const float* probe_sparse, const float* probe_out,
+SPARSEPR_API int sparsepr_fit_residual(const float* probe_sparse, const float* probe_out,
                           const float* weights, int32_t Bt, int32_t H, int32_t d,
                           int32_t P, double ridge_lambda, int32_t rank,
                           int32_t weight_mode, float* M, float* beta, void* ws,
@@ -165,7 +177,7 @@ int sparsepr_fit_residual(const float* probe_sparse, const float* probe_out,
 
 /* (d3) Apply: O_i = S_i + M S_i + beta for unprobed rows, O_p = probe_out_p for probe
  * rows.  O [Bt,H,N,d] in out_dtype.  O may alias S_out when out_dtype is F32. */
-int sparsepr_apply_residual(const float* S_out, const float* M, const float* beta,
+SPARSEPR_API int sparsepr_apply_residual(const float* S_out, const float* M, const float* beta,
                             const int32_t* probe_idx, const float* probe_out,
                             int32_t Bt, int32_t H, int32_t N, int32_t d, int32_t P,
                             void* O, int out_dtype, sparsepr_stream_t stream);
@@ -173,20 +185,20 @@ int sparsepr_apply_residual(const float* S_out, const float* M, const float* bet
 /* Wait for `stream` and return the device status word in `ws` (SPARSEPR_OK, or the
  * first device-side error since the last sparsepr_partition).  This is the only call
  * that synchronises. */
-int sparsepr_check(const void* ws, sparsepr_stream_t stream);
+SPARSEPR_API int sparsepr_check(const void* ws, sparsepr_stream_t stream);
 
 /* Message of the last host-side error on this thread ("" if none). */
-const char* sparsepr_last_error(void);
+SPARSEPR_API const char* sparsepr_last_error(void);
 
 /* ---- decision kernels on injected scores (used by the parity tests) ---------------
  * sparsepr_test_fill: the capacity-B assignment used by every k-means iteration, run
  *   on caller-supplied fp32 distances D [H, n, G] (device); labels [H, n] int32.
  * sparsepr_test_topk: the routing selection on caller-supplied scores Sc [H, Gq, G];
  *   route [H, Gq, k] int32.  Both use the same kernels as the operator. */
-size_t sparsepr_test_fill_workspace_size(int32_t H, int32_t n, int32_t G);
-int sparsepr_test_fill(const float* D, int32_t H, int32_t n, int32_t G, int32_t cap,
+SPARSEPR_API size_t sparsepr_test_fill_workspace_size(int32_t H, int32_t n, int32_t G);
+SPARSEPR_API int sparsepr_test_fill(const float* D, int32_t H, int32_t n, int32_t G, int32_t cap,
                        int32_t* labels, void* ws, sparsepr_stream_t stream);
-int sparsepr_test_topk(const float* Sc, int32_t H, int32_t Gq, int32_t G, int32_t k,
+SPARSEPR_API int sparsepr_test_topk(const float* Sc, int32_t H, int32_t Gq, int32_t G, int32_t k,
                        int32_t* route, void* ws, sparsepr_stream_t stream);
 
 #ifdef __cplusplus

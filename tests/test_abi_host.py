@@ -1,0 +1,76 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+function include/sparsepr.h declares, and its host arithmetic and argument checks
+behave (no kernel is launched here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import free_block_sparse_response_b200 as spr
+from oracle import sparsepr_oracle as O
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "sparsepr.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from free_block_sparse_response_b200.build import build
+    build()
+    return spr.lib()
+
+
+def test_header_declarations_are_exported(L):
+    text = open(HEADER).read()
+    declared = set(re.findall(r"SPARSEPR_API\s+[\w\s\*]+?\b(sparsepr_\w+)\s*\(", text))
+    assert declared == set(spr.EXPORTED_SYMBOLS)
+    for name in declared:
+        assert getattr(L, name) is not None
+
+
+def test_route_k_and_groups_match_oracle(L):
+    for n, b, rho, p in [(1024, 64, 0.25, 32), (8192, 128, 0.22, 64), (75600, 128, 0.22, 256),
+                         (118800, 128, 0.22, 256), (32760, 128, 0.26, 512), (1000, 64, 0.0, 3),
+                         (1000, 64, 5.0, 3), (777, 64, 0.3, 0), (128, 128, 1.0, 0)]:
+        assert spr.route_k(n, b, rho, p) == O.route_k(n, b, rho, p)
+        assert spr.num_groups(n, b) == O.n_groups(n, b)
+
+
+def test_workspace_size_positive_and_rejects_bad_sizes(L):
+    cfg = spr.SparsePRConfig()
+    assert spr.workspace_size(1, 40, 75600, 128, cfg) > 40 * 75600 * 591 * 4
+    assert L.sparsepr_workspace_size(1, 1, 100, 96, ctypes.byref(cfg.c())) == 0
+    bad = spr.SparsePRConfig(block=48)
+    assert L.sparsepr_workspace_size(1, 1, 100, 64, ctypes.byref(bad.c())) == 0
+
+
+def test_argument_errors_return_codes_without_launching(L):
+    cfg = spr.SparsePRConfig(block=128).c()
+    # unsupported head dim: rejected before any device work
+    rc = L.sparsepr_partition(None, None, spr.BF16, 1, 1, 100, 96, ctypes.byref(cfg), None, None, None, None,
+                              None, None, None, None)
+    assert rc == spr.ERR_UNSUPPORTED
+    assert b"head dim" in L.sparsepr_last_error()
+    rc = L.sparsepr_partition(None, None, 7, 1, 1, 100, 128, ctypes.byref(cfg), None, None, None, None, None,
+                              None, None, None)
+    assert rc == spr.ERR_INVALID_ARG
+    rc = L.sparsepr_sparse_attn(None, None, None, spr.BF16, 1, 1, 100, 128, 128, None, None, None, None, None, 1,
+                                0.0, None, None, None)
+    assert rc == spr.ERR_INVALID_ARG
+    rc = L.sparsepr_fit_residual(None, None, None, 1, 1, 128, 64, -1.0, 8, 0, None, None, None, None)
+    assert rc == spr.ERR_INVALID_ARG
+    rc = L.sparsepr_test_topk(None, 1, 4, 4, 5, None, None, None)
+    assert rc == spr.ERR_INVALID_ARG
+
+
+def test_params_struct_layout():
+    assert ctypes.sizeof(spr.sparsepr._CParams) == 48
+    assert spr.sparsepr._CParams.density.offset == 24
+    assert spr.sparsepr._CParams.scale.offset == 40
+
+
+def test_python_wrappers_refuse_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 1, 64, 64)
+    with pytest.raises(ValueError):
+        spr.dense_attn(q, q, q, block=64)

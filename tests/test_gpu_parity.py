@@ -1,0 +1,302 @@
+"""GPU parity of the SparsePR CUDA path against the fp64 oracle.
+
+Decisions (capacity fill, routing, pair counts) must be bit-exact when both sides get
+the same fp32 scores.  Outputs are compared with the oracle run on the GPU's own
+decisions (partition, routes, probe rows injected): rel-L2 <= 3e-3 per head for bf16
+inputs with fp32 accumulation, fitted maps within 1e-3 relative Frobenius.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import free_block_sparse_response_b200 as spr
+from oracle import sparsepr_oracle as O
+from synthetic import CONFIGS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_BF16 = 3e-3     # per-head output rel-L2, bf16 inputs / fp32 accumulation
+TOL_F32 = 2e-5      # fp32 inputs, fp32 SIMT arithmetic
+TOL_MAP = 1e-3      # fitted M and beta, relative Frobenius
+TOL_PROBE = 2e-4    # probe rows: softmax weights carried at ~16 bits
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from free_block_sparse_response_b200.build import build
+    build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    spr.lib()
+
+
+def rel(a, b):
+    return float(np.linalg.norm(np.asarray(a, np.float64) - np.asarray(b, np.float64)) /
+                 max(np.linalg.norm(np.asarray(b, np.float64)), 1e-300))
+
+
+def spr_cfg(w, **kw):
+    base = dict(block=w.block, n_sampled=w.n_sampled, n_probe=w.n_probe, kmeans_iters=w.kmeans_iters,
+                rank=w.rank, density=w.density, ridge_lambda=w.ridge_lambda)
+    base.update(kw)
+    return spr.SparsePRConfig(**base)
+
+
+def perm_labels(perm, sizes, n, block):
+    perm = np.asarray(perm)
+    sizes = np.asarray(sizes)
+    labels = np.full(n, -1, dtype=np.int64)
+    for g in range(sizes.size):
+        members = perm[g * block: g * block + sizes[g]]
+        assert (members >= 0).all() and (perm[g * block + sizes[g]:(g + 1) * block] == -1).all()
+        assert (np.diff(members) > 0).all(), "members must be in ascending token order"
+        labels[members] = g
+    assert (labels >= 0).all() and sizes.sum() == n and sizes.max() <= block
+    return labels
+
+
+def run_call(w, q, k, v, cfg):
+    dev = torch.device("cuda")
+    qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    o, parts = spr.attention(qd, kd, vd, cfg, return_parts=True)
+    spr.check(parts["ws"])
+    return o, parts
+
+
+def oracle_on_gpu_decisions(q, k, v, parts, h, cfg, n):
+    part = parts["partition"]
+    kl = perm_labels(part.key_perm[0, h].cpu().numpy(), part.key_gsize[0, h].cpu().numpy(), n, cfg.block)
+    ql = perm_labels(part.query_perm[0, h].cpu().numpy(), part.qblock_size[0, h].cpu().numpy(), n, cfg.block)
+    return O.sparsepr_head(*(t[0, h].double().numpy() for t in (q, k, v)), block=cfg.block,
+                           n_sampled=cfg.n_sampled, n_probe=cfg.n_probe, density=cfg.density,
+                           ridge_lambda=cfg.ridge_lambda, rank=cfg.rank, kmeans_iters=cfg.kmeans_iters,
+                           inject={"key_labels": kl, "query_labels": ql,
+                                   "routes": parts["route"][0, h].cpu().numpy(),
+                                   "probe_idx": parts["probe_idx"][0, h].cpu().numpy()})
+
+
+# ----------------------------------------------------------------- decisions, bit-exact
+
+def test_fill_bit_exact_on_oracle_kmeans_distances():
+    """Every fp32 distance matrix the oracle's balanced k-means hands to its fill
+    (keys and queries, Tiny head 0 and a Small head) gives identical labels on GPU."""
+    for name, heads in (("tiny", 1), ("small", 1)):
+        w = CONFIGS[name]
+        q, k, _ = make_inputs(w, 0, heads=heads)
+        dump = {}
+        O.partition(q[0, 0].double().numpy(), k[0, 0].double().numpy(), 1 / math.sqrt(w.head_dim), w.block,
+                    w.n_sampled, w.kmeans_iters, dump=dump)
+        for dmat in dump["key_dist"] + dump["query_dist"]:
+            gpu = spr.test_fill(torch.from_numpy(dmat)[None].cuda(), w.block)[0].cpu().numpy()
+            assert np.array_equal(gpu, O.fill(dmat, w.block))
+
+
+@pytest.mark.parametrize("heads,n,g,cap,levels", [(1, 1000, 16, 64, 4), (3, 300, 7, 50, 3), (2, 4096, 33, 128, 1000),
+                                                  (1, 64, 64, 1, 2), (2, 777, 13, 64, 0)])
+def test_fill_bit_exact_random_with_ties(heads, n, g, cap, levels):
+    rng = np.random.default_rng(n + g)
+    if levels == 0:   # signed zeros and infinities
+        dmat = rng.choice(np.array([0.0, -0.0, 1.0, np.inf], dtype=np.float32), size=(heads, n, g))
+    else:
+        dmat = rng.integers(0, levels, size=(heads, n, g)).astype(np.float32) * np.float32(0.5)
+    gpu = spr.test_fill(torch.from_numpy(dmat).cuda(), cap).cpu().numpy()
+    for h in range(heads):
+        assert np.array_equal(gpu[h], O.fill(dmat[h], cap))
+
+
+@pytest.mark.parametrize("gq,g,k", [(16, 16, 3), (64, 64, 13), (591, 591, 127), (40, 40, 40), (9, 30, 1)])
+def test_topk_bit_exact_with_ties(gq, g, k):
+    rng = np.random.default_rng(gq * g + k)
+    sc = rng.integers(-4, 4, size=(2, gq, g)).astype(np.float32)
+    sc[0, 0, :4] = [0.0, -0.0, 0.0, -0.0]
+    gpu = spr.test_topk(torch.from_numpy(sc).cuda(), k).cpu().numpy()
+    for h in range(2):
+        assert np.array_equal(gpu[h], O.route(sc[h], k))
+
+
+def test_nan_scores_are_reported():
+    sc = np.zeros((1, 4, 8), dtype=np.float32)
+    sc[0, 1, 2] = np.nan
+    with pytest.raises(spr.SparsePRError) as ei:
+        spr.test_topk(torch.from_numpy(sc).cuda(), 2)
+    assert ei.value.code == spr.ERR_NONFINITE
+    dmat = np.ones((1, 10, 4), dtype=np.float32)
+    dmat[0, 3, 1] = np.nan
+    with pytest.raises(spr.SparsePRError) as ei:
+        spr.test_fill(torch.from_numpy(dmat).cuda(), 4)
+    assert ei.value.code == spr.ERR_NONFINITE
+
+
+# ------------------------------------------------------------------- whole-call parity
+
+def _check_call(w, cfg, seed=0, heads=None, tol=TOL_BF16, map_tol=TOL_MAP):
+    q, k, v = make_inputs(w, seed, heads=heads)
+    n = w.n_tokens
+    o, parts = run_call(w, q, k, v, cfg)
+    gpu_pairs = parts["executed_pairs"].cpu().numpy()
+    for h in range(q.shape[1]):
+        ref = oracle_on_gpu_decisions(q, k, v, parts, h, cfg, n)
+        assert int(gpu_pairs[0, h]) == ref["executed_pairs"]
+        s_gpu = parts["S"][0, h].cpu().numpy()
+        assert rel(s_gpu, ref["S"]) <= tol, f"head {h}: sparse output"
+        pidx = ref["probe_idx"]
+        assert rel(parts["probe_out"][0, h].cpu().numpy(), ref["probe_out"]) <= TOL_PROBE
+        assert rel(parts["probe_sparse"][0, h].cpu().numpy(), ref["S"][pidx]) <= TOL_PROBE
+        m_gpu, b_gpu = parts["M"][0, h].cpu().numpy(), parts["beta"][0, h].cpu().numpy()
+        fit = ref["fit"]
+        if fit["eigengap"] > 1e-6:
+            assert rel(m_gpu, fit["M"]) <= map_tol, f"head {h}: M"
+            assert rel(b_gpu, fit["beta"]) <= map_tol, f"head {h}: beta"
+        o_gpu = o[0, h].double().cpu().numpy()
+        assert rel(o_gpu, ref["O"]) <= tol, f"head {h}: final output"
+        # probe rows of O are the probe outputs, cast to the output dtype
+        want = parts["probe_out"][0, h].to(o.dtype)
+        assert torch.equal(o[0, h][parts["probe_idx"][0, h].long()].cpu(), want.cpu())
+    return o, parts
+
+
+def test_call_tiny_fp32():
+    w = CONFIGS["tiny"]
+    _check_call(w, spr_cfg(w), tol=TOL_F32, map_tol=1e-4)
+
+
+def test_call_small_bf16():
+    w = CONFIGS["small"]
+    _check_call(w, spr_cfg(w), heads=3)
+
+
+def test_call_bf16_d64_block64_ragged():
+    """bf16 tensor-core path at d=64, B=64 on a ragged N (last group and block short)."""
+    w = CONFIGS["tiny"].with_(grid=(3, 15, 22), dtype="bf16")     # N = 990
+    _check_call(w, spr_cfg(w, n_probe=40))
+
+
+def test_call_bf16_d128_ragged_long_tail():
+    w = CONFIGS["small"].with_(grid=(5, 9, 23), heads=2)           # N = 1035, last group 11 tokens
+    _check_call(w, spr_cfg(w, n_sampled=128, n_probe=80, rank=8))
+
+
+def test_full_density_equals_dense():
+    """k = G: sparse output is dense attention; the fitted map is ~0."""
+    w = CONFIGS["small"].with_(grid=(2, 16, 32), heads=2)
+    cfg = spr_cfg(w, density=10.0, n_sampled=128)
+    q, k, v = make_inputs(w, 1)
+    o, parts = run_call(w, q, k, v, cfg)
+    assert parts["k"] == spr.num_groups(w.n_tokens, w.block)
+    dense = spr.dense_attn(*(t.cuda() for t in (q, k, v)), block=w.block)
+    for h in range(2):
+        ref = O.dense_attention_rows(*(t[0, h].double().numpy() for t in (q, k, v)), 1 / math.sqrt(128),
+                                     np.arange(w.n_tokens))
+        assert rel(dense[0, h].cpu().numpy(), ref) <= TOL_BF16
+        assert rel(parts["S"][0, h].cpu().numpy(), ref) <= TOL_BF16
+        assert rel(o[0, h].double().cpu().numpy(), ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("overrides", [dict(kmeans_iters=0), dict(density=0.01), dict(n_probe=4, rank=8),
+                                       dict(weight_mode=spr.WEIGHT_UNIFORM)])
+def test_degenerate_and_variant_settings(overrides):
+    """T = 0 (chunk partition), k = 1, rank above the probe count, uniform weights."""
+    w = CONFIGS["tiny"].with_(dtype="bf16")
+    cfg = spr_cfg(w, **overrides)
+    q, k, v = make_inputs(w, 2)
+    o, parts = run_call(w, q, k, v, cfg)
+    n = w.n_tokens
+    if cfg.kmeans_iters == 0:
+        kp = parts["partition"].key_perm[0, 0].cpu().numpy()
+        assert np.array_equal(kp[kp >= 0], np.arange(n))
+    for h in range(2):
+        ref = oracle_on_gpu_decisions(q, k, v, parts, h, cfg, n)
+        if cfg.weight_mode == spr.WEIGHT_UNIFORM:
+            ref_fit = O.fit_residual(ref["S"][ref["probe_idx"]], ref["probe_out"], cfg.ridge_lambda, cfg.rank,
+                                     weight_mode="uniform")
+            ref["O"] = O.apply_residual(ref["S"], ref_fit["M"], ref_fit["beta"], ref["probe_idx"], ref["probe_out"])
+        assert rel(o[0, h].double().cpu().numpy(), ref["O"]) <= TOL_BF16
+
+
+def test_fit_kernel_matches_oracle_on_identical_inputs():
+    """The fp64 fit kernel alone: the GPU's probe outputs fed to both sides."""
+    w = CONFIGS["small"]
+    q, k, v = make_inputs(w, 0, heads=2)
+    cfg = spr_cfg(w)
+    _, parts = run_call(w, q, k, v, cfg)
+    for h in range(2):
+        xs = parts["probe_sparse"][0, h].double().cpu().numpy()
+        dp = parts["probe_out"][0, h].double().cpu().numpy()
+        fit = O.fit_residual(xs, dp, cfg.ridge_lambda, cfg.rank)
+        assert rel(parts["M"][0, h].cpu().numpy(), fit["M"]) <= 1e-5
+        assert rel(parts["beta"][0, h].cpu().numpy(), fit["beta"]) <= 1e-5
+
+
+def test_partition_label_agreement_with_oracle():
+    """Uninjected: the GPU partition is valid and agrees with the oracle's on most
+    tokens (near-ties may differ: distances are evaluated in bf16 on the GPU)."""
+    w = CONFIGS["small"]
+    q, k, v = make_inputs(w, 0, heads=1)
+    cfg = spr_cfg(w)
+    _, parts = run_call(w, q, k, v, cfg)
+    n = w.n_tokens
+    part = parts["partition"]
+    kl = perm_labels(part.key_perm[0, 0].cpu().numpy(), part.key_gsize[0, 0].cpu().numpy(), n, w.block)
+    ql = perm_labels(part.query_perm[0, 0].cpu().numpy(), part.qblock_size[0, 0].cpu().numpy(), n, w.block)
+    ref = O.partition(q[0, 0].double().numpy(), k[0, 0].double().numpy(), 1 / math.sqrt(w.head_dim), w.block,
+                      w.n_sampled, w.kmeans_iters)
+    key_agree = float((kl == ref["key_labels"]).mean())
+    print(f"key label agreement {key_agree:.3f}, query {(ql == ref['query_labels']).mean():.3f}")
+    assert key_agree > 0.5
+
+
+def test_nonfinite_input_is_reported():
+    w = CONFIGS["tiny"].with_(dtype="bf16")
+    q, k, v = make_inputs(w, 0)
+    q[0, 0, 5, 3] = float("nan")
+    with pytest.raises(spr.SparsePRError) as ei:
+        run_call(w, q, k, v, spr_cfg(w))
+    assert ei.value.code == spr.ERR_NONFINITE
+
+
+# ----------------------------------------------------- full size, sampled outputs (bench)
+
+def test_video_config_sampled_rows():
+    """75,600 tokens x 40 heads in the bench's launch configuration.  All heads: valid
+    partitions and exact pair counts; heads 0 and 39: sampled rows of the sparse
+    output, every probe row, and the final output on sampled rows against the oracle."""
+    w = CONFIGS["video"]
+    cfg = spr_cfg(w)
+    q, k, v = make_inputs(w, 0)
+    o, parts = run_call(w, q, k, v, cfg)
+    n, B = w.n_tokens, w.block
+    kk = parts["k"]
+    assert kk == 127
+    part = parts["partition"]
+    pairs = parts["executed_pairs"].cpu().numpy()
+    ks_all, bs_all = part.key_gsize.cpu().numpy(), part.qblock_size.cpu().numpy()
+    rt_all = parts["route"].cpu().numpy()
+    for h in range(w.heads):
+        assert ks_all[0, h].sum() == n and bs_all[0, h].sum() == n
+        assert int(pairs[0, h]) == O.executed_pairs(rt_all[0, h], ks_all[0, h], bs_all[0, h], w.n_probe, n)
+        assert pairs[0, h] / n ** 2 <= w.density
+    rng = np.random.default_rng(7)
+    tau = 1 / math.sqrt(w.head_dim)
+    for h in (0, w.heads - 1):
+        qh, kh, vh = (t[0, h].double().numpy() for t in (q, k, v))
+        kl = perm_labels(part.key_perm[0, h].cpu().numpy(), ks_all[0, h], n, B)
+        ql = perm_labels(part.query_perm[0, h].cpu().numpy(), bs_all[0, h], n, B)
+        pidx = parts["probe_idx"][0, h].cpu().numpy()
+        rows = np.sort(rng.choice(np.setdiff1d(np.arange(n), pidx), size=96, replace=False))
+        s_ref = np.stack([O.sparse_attention(qh[[i]], kh, vh, tau, kl, np.zeros(1, np.int64),
+                                             rt_all[0, h][[ql[i]]])[0] for i in rows])
+        s_gpu = parts["S"][0, h][torch.from_numpy(rows).cuda()].cpu().numpy()
+        assert rel(s_gpu, s_ref) <= TOL_BF16
+        d_ref = O.dense_attention_rows(qh, kh, vh, tau, pidx)
+        assert rel(parts["probe_out"][0, h].cpu().numpy(), d_ref) <= TOL_PROBE
+        sp_ref = np.stack([O.sparse_attention(qh[[i]], kh, vh, tau, kl, np.zeros(1, np.int64),
+                                              rt_all[0, h][[ql[i]]])[0] for i in pidx])
+        assert rel(parts["probe_sparse"][0, h].cpu().numpy(), sp_ref) <= TOL_PROBE
+        fit = O.fit_residual(sp_ref, d_ref, w.ridge_lambda, w.rank)
+        if fit["eigengap"] > 1e-6:
+            assert rel(parts["M"][0, h].cpu().numpy(), fit["M"]) <= TOL_MAP
+            assert rel(parts["beta"][0, h].cpu().numpy(), fit["beta"]) <= TOL_MAP
+        o_ref = s_ref + s_ref @ fit["M"].T + fit["beta"]
+        o_gpu = o[0, h][torch.from_numpy(rows).cuda()].double().cpu().numpy()
+        assert rel(o_gpu, o_ref) <= TOL_BF16
