@@ -1,0 +1,416 @@
+#!/usr/bin/env python
+"""Benchmark of the SparsePR attention call on one B200 per rank.
+
+A step is one whole SparsePR call (partition, routing, block-sparse attention, probe
+rows, fit, apply) on the video-DiT 720p-like workload: 40 heads x 75,600 tokens
+(21x45x80 grid), head dim 128, bf16, synthetic seeded latents.  Each rank runs its own
+independent call (weak scaling, no data-path collective).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle on a
+bounded sample of the same workload instead (the reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SparsePR ms/call & eff. TFLOP/s at 22% pair density; mean rel-L2 err vs dense"
+UNIT = "TFLOP/s (dense-equivalent, 4*d*N^2*H per call)"
+
+# DRAM bytes per launch of the dominant kernel from an ncu capture of the same kernel
+# build (profiles/); None until a capture of the current kernel exists.
+DOMINANT_TRAFFIC_BYTES = None
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="video")
+    ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+def workload(args):
+    from synthetic import CONFIGS
+    w = CONFIGS[args.config]
+    if args.heads:
+        w = w.with_(heads=args.heads)
+    return w
+
+
+def config_block(w, args):
+    t, y, x = w.grid
+    return {"workload": f"{w.name}: {w.heads} heads x {w.n_tokens} tokens ({t}x{y}x{x} grid), d={w.head_dim}, "
+                        f"{w.dtype}, B={w.block}, S={w.n_sampled}, P={w.n_probe}, density={w.density}, "
+                        f"lambda={w.ridge_lambda}, r={w.rank}, T={w.kmeans_iters}",
+            "batch": w.batch, "heads": w.heads, "tokens": w.n_tokens, "head_dim": w.head_dim,
+            "parallelism": f"independent call per rank x{args.gpus}", "seed": args.seed,
+            "l2": "inputs (3 x 774 MB bf16) larger than the 126 MB L2; no flush needed"}
+
+
+def dense_flops(w):
+    return 4.0 * w.head_dim * float(w.n_tokens) ** 2 * w.heads * w.batch
+
+
+# ------------------------------------------------------------------- CPU oracle sample
+
+def oracle_sample(w, seed=0):
+    """Time the fp64 oracle's stages on one head of the workload restricted to its
+    first frame and extrapolate to the full call by each stage's cost order.
+    Returns (seconds per full call, description, threads)."""
+    import numpy as np
+
+    from oracle import sparsepr_oracle as O
+    from synthetic import make_inputs
+    t_frames, gy, gx = w.grid
+    sub = w.with_(grid=(1, gy, gx), heads=1)
+    q, k, v = make_inputs(sub, seed)
+    q, k, v = (x[0, 0].double().numpy() for x in (q, k, v))
+    n_s, n = sub.n_tokens, w.n_tokens
+    tau = 1.0 / math.sqrt(w.head_dim)
+    s_count = min(w.n_sampled, n_s)
+    tm = {}
+    t0 = time.perf_counter()
+    part = O.partition(q, k, tau, w.block, s_count, w.kmeans_iters)
+    tm["partition"] = time.perf_counter() - t0
+    kk = O.route_k(n_s, w.block, w.density, w.n_probe)
+    t0 = time.perf_counter()
+    routes = O.route(part["block_scores"], kk)
+    tm["route"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    s = O.sparse_attention(q, k, v, tau, part["key_labels"], part["query_labels"], routes)
+    tm["sparse"] = time.perf_counter() - t0
+    pidx = O.midpoint_stride(n_s, w.n_probe)
+    t0 = time.perf_counter()
+    d_probe = O.dense_attention_rows(q, k, v, tau, pidx)
+    tm["probes"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    fit = O.fit_residual(s[pidx], d_probe, w.ridge_lambda, w.rank)
+    tm["fit"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.apply_residual(s, fit["M"], fit["beta"], pidx, d_probe)
+    tm["apply"] = time.perf_counter() - t0
+    r = n / n_s
+    # partition: N*G*dims with G ~ N and dims S (keys) / G (queries) -> between N^2 and N^3;
+    # take N^2 (keys dominate at S fixed).  sparse ~ N*k*B ~ N^2.  probes ~ P*N.  apply ~ N.
+    scale = {"partition": r * r, "route": r * r, "sparse": r * r, "probes": r, "fit": 1.0, "apply": r}
+    per_head = sum(tm[x] * scale[x] for x in tm)
+    full = per_head * w.heads * w.batch
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        threads = 1
+    desc = (f"fp64 oracle, 1 head, first frame ({n_s} tokens, S={s_count}, P={w.n_probe}); stage times "
+            + ", ".join(f"{x} {tm[x]:.2f}s" for x in tm)
+            + f"; extrapolated per stage (partition, route, sparse x(N/n)^2; probes, apply x N/n; fit x1) "
+              f"and x{w.heads * w.batch} heads")
+    return full, desc, threads
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    times = []
+    desc = threads = None
+    for i in range(args.warmup + args.steps):
+        full, desc, threads = oracle_sample(w, args.seed)
+        if i >= args.warmup:
+            times.append(full)
+    sec = statistics.mean(times)
+    value = dense_flops(w) / sec / 1e12
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_block(w, args),
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------- GPU helpers
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index):
+        import torch
+        self.proc = None
+        self.sel = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.sel = ["-i", uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"]
+        except Exception:
+            self.sel = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", *self.sel, f"--query-gpu={','.join(self.FIELDS)}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in out.strip().splitlines():
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[3:]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["bf16_tflops_sustained"]), "measured (cuBLAS bf16, sustained)"
+    except Exception:
+        return 1400.0, "fallback (1.4 PFLOP/s sustained bf16)"
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    import free_block_sparse_response_b200 as spr
+    from free_block_sparse_response_b200.build import build
+    from synthetic import make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        build()
+    if world > 1:
+        dist.barrier()
+    spr.lib()
+
+    cpu_base = None
+    if rank == 0 and world == 1:
+        cpu_sec, cpu_desc, cpu_threads = oracle_sample(w, args.seed)
+        cpu_base = {"value": dense_flops(w) / cpu_sec / 1e12, "unit": UNIT, "cores": cpu_threads,
+                    "kind": "oracle", "sample": cpu_desc}
+
+    q_h, k_h, v_h = make_inputs(w, args.seed + rank)
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    bt, h, n, d = q.shape
+    sc = spr.SparsePRConfig(block=w.block, n_sampled=w.n_sampled, n_probe=w.n_probe, kmeans_iters=w.kmeans_iters,
+                            rank=w.rank, density=w.density, ridge_lambda=w.ridge_lambda)
+    ws = spr.new_workspace(bt, h, n, d, sc, dev)
+    o = torch.empty_like(q)
+    stages = ["partition", "route", "sparse_attn", "probe_dense", "fit_residual", "apply_residual"]
+
+    def step(record=None):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] if record is not None else None
+        if ev:
+            ev[0].record()
+        part = spr.partition(q, k, sc, ws)
+        if ev:
+            ev[1].record()
+        rt, kk, pairs = spr.route(part, n, sc, ws)
+        if ev:
+            ev[2].record()
+        s_out = spr.sparse_attn(q, k, v, part, rt, kk, sc, ws=ws)
+        if ev:
+            ev[3].record()
+        pidx = spr.probe_rows(n, sc.n_probe, bt, h, dev)
+        p_out, p_sparse = spr.probe_dense(q, k, v, pidx, part, rt, kk, sc, ws)
+        if ev:
+            ev[4].record()
+        m, beta = spr.fit_residual(p_sparse, p_out, sc, ws)
+        if ev:
+            ev[5].record()
+        spr.apply_residual(s_out, m, beta, pidx, p_out, out_dtype=q.dtype, out=o)
+        if ev:
+            ev[6].record()
+            record.append(ev)
+        return {"S": s_out, "pidx": pidx, "pairs": pairs, "k": kk}
+
+    for _ in range(args.warmup):
+        step()
+    spr.check(ws)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    launches0 = spr.launch_count()
+    events = []
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t_start.record()
+    for _ in range(args.steps):
+        last = step(events)
+    t_end.record()
+    torch.cuda.synchronize()
+    launches = spr.launch_count() - launches0
+    clk = clocks.stop()
+    spr.check(ws)
+    elapsed = t_start.elapsed_time(t_end) / 1e3
+    if world > 1:
+        tt = torch.tensor([elapsed], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed = float(tt.item())
+        dist.barrier()
+    ms_step = elapsed / args.steps * 1e3
+    stage_ms = {s: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in events) for i, s in enumerate(stages)}
+
+    # ---- dominant kernel roofline (block-sparse attention: 4*d flops per routed pair)
+    pairs = last["pairs"].to(torch.float64).sum().item()
+    sparse_pairs = pairs - float(w.n_probe) * n * h * bt
+    sparse_flops = 4.0 * d * sparse_pairs
+    t_sparse = stage_ms["sparse_attn"] / 1e3
+    peak, peak_src = measured_peak()
+    achieved = sparse_flops / t_sparse / 1e12
+    roofline = {"kernel": "attn_mma_kernel (block-sparse attention)", "bound": "tensor", "achieved": achieved,
+                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": DOMINANT_TRAFFIC_BYTES,
+                "peak_source": peak_src,
+                "per_launch_flops": sparse_flops}
+
+    # ---- e2e through host buffers (pinned), same call, copies inside the timed region
+    qp, kp, vp = (t.pin_memory() for t in (q_h, k_h, v_h))
+    op = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    for _ in range(1):
+        q.copy_(qp, non_blocking=True), k.copy_(kp, non_blocking=True), v.copy_(vp, non_blocking=True)
+        spr.attention(q, k, v, sc, ws=ws, out=o)
+        op.copy_(o, non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        q.copy_(qp, non_blocking=True)
+        k.copy_(kp, non_blocking=True)
+        v.copy_(vp, non_blocking=True)
+        spr.attention(q, k, v, sc, ws=ws, out=o)
+        op.copy_(o, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_s = e0.elapsed_time(e1) / 1e3
+    if world > 1:
+        tt = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_s = float(tt.item())
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
+    d2h = o.numel() * o.element_size()
+
+    # ---- dense comparators and the error metric (outside the timed regions)
+    s_last = last["S"]
+    dense = torch.empty(bt, h, n, d, dtype=torch.float32, device=dev)
+    spr.dense_attn(q, k, v, block=w.block, out=dense)
+    torch.cuda.synchronize()
+    de0, de1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    de0.record()
+    for _ in range(2):
+        spr.dense_attn(q, k, v, block=w.block, out=dense)
+    de1.record()
+    torch.cuda.synchronize()
+    dense_ms = de0.elapsed_time(de1) / 2
+    sdpa_ms = None
+    try:
+        import torch.nn.functional as F
+        F.scaled_dot_product_attention(q, k, v)
+        torch.cuda.synchronize()
+        se0, se1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        se0.record()
+        for _ in range(2):
+            F.scaled_dot_product_attention(q, k, v)
+        se1.record()
+        torch.cuda.synchronize()
+        sdpa_ms = se0.elapsed_time(se1) / 2
+    except Exception:
+        sdpa_ms = None
+    pidx = spr.probe_rows(n, sc.n_probe, bt, h, dev)
+    err = spr.row_errors(o, dense, pidx)
+    err_s = spr.row_errors(s_last, dense, pidx)
+
+    def summary(e):
+        means, p99s = [], []
+        for hh in range(h):
+            x = e[0, hh]
+            x = x[~torch.isnan(x)]
+            xs, _ = torch.sort(x)
+            means.append(float(xs.double().mean()))
+            p99s.append(float(xs[max(math.ceil(0.99 * xs.numel()) - 1, 0)]))
+        return statistics.mean(means), statistics.mean(p99s)
+
+    err_mean, err_p99 = summary(err)
+    s_mean, s_p99 = summary(err_s)
+    spr.check(ws)
+
+    total_flops = dense_flops(w) * world
+    value = total_flops * args.steps / elapsed / 1e12
+    e2e_value = total_flops * args.steps / e2e_s / 1e12
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded video-token latents)",
+                "config": config_block(w, args),
+                "err": {"mean_rel_l2_unprobed": err_mean, "p99_rel_l2_unprobed": err_p99,
+                        "uncorrected_sparse_mean": s_mean, "uncorrected_sparse_p99": s_p99,
+                        "reference": "same-family dense attention, fp32 output"},
+                "density": pairs / (float(n) ** 2 * h * bt), "k": last["k"],
+                "stage_ms": stage_ms, "dense_ms": dense_ms, "sdpa_ms": sdpa_ms,
+                "speedup_vs_dense": dense_ms / ms_step,
+                "roofline": roofline, "cpu_baseline": cpu_base,
+                "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                        "ms_per_step": e2e_s / args.steps * 1e3},
+                "gpu_launches": launches, "clocks": clk}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    w = workload(args)
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -2,6 +2,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <atomic>
 #include <cstring>
 #include <string>
 
@@ -11,6 +12,13 @@
 #include "fit.cuh"
 #include "partition.cuh"
 #include "route.cuh"
+
+namespace spr {
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}
+void note_launches(int n) { g_launches.fetch_add(static_cast<unsigned long long>(n), std::memory_order_relaxed); }
+}  // namespace spr
 
 namespace {
 
@@ -418,6 +426,19 @@ int sparsepr_probe_rows(int32_t N, int32_t P, int32_t Bt, int32_t H, int32_t* pr
   if (N < 1 || P < 1 || P > N || Bt < 1 || H < 1 || !probe_idx)
     return fail(SPARSEPR_ERR_INVALID_ARG, "bad probe-row arguments");
   SPR_CUDA(spr::launch_probe_rows(N, P, Bt * H, probe_idx, reinterpret_cast<cudaStream_t>(stream)), "probe rows");
+  return SPARSEPR_OK;
+}
+
+uint64_t sparsepr_launch_count(void) { return spr::g_launches.load(std::memory_order_relaxed); }
+
+int sparsepr_row_errors(const void* O, int o_dtype, const float* O_ref, const int32_t* probe_idx, int32_t Bt,
+                        int32_t H, int32_t N, int32_t d, int32_t P, float* err, sparsepr_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(Bt, H, N, d)) || (rc = check_dtype(o_dtype))) return rc;
+  if (!O || !O_ref || !err || (P > 0 && !probe_idx)) return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
+  SPR_CUDA(spr::launch_row_errors(O, o_dtype == SPARSEPR_F32, O_ref, Bt * H, N, d, probe_idx, P, err,
+                                  reinterpret_cast<cudaStream_t>(stream)),
+           "row errors");
   return SPARSEPR_OK;
 }
 

@@ -578,7 +578,7 @@ __global__ void probe_rows_kernel(int N, int P, int heads, int* __restrict__ pro
 
 cudaError_t launch_probe_rows(int N, int P, int heads, int* probe_idx, cudaStream_t st) {
   probe_rows_kernel<<<ceil_div(heads * P, 256), 256, 0, st>>>(N, P, heads, probe_idx);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 // token -> query block, from query_perm.
@@ -605,7 +605,7 @@ static cudaError_t launch_attn_mma_t(const AttnArgs& a, cudaStream_t st) {
   kern<<<grid, BQ * 2, smem, st>>>(static_cast<const __nv_bfloat16*>(a.Q), static_cast<const __nv_bfloat16*>(a.K),
                                    static_cast<const __nv_bfloat16*>(a.V), a.N, a.G, a.k, a.key_perm,
                                    a.key_gsize, a.query_perm, a.qblock_size, a.route, a.scale_log2, a.out);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 template <int D, bool DENSE>
@@ -614,7 +614,7 @@ static cudaError_t launch_attn_f32_t(const AttnArgs& a, cudaStream_t st) {
   attn_f32_kernel<D, DENSE><<<grid, 256, 0, st>>>(
       static_cast<const float*>(a.Q), static_cast<const float*>(a.K), static_cast<const float*>(a.V), a.N,
       a.block, a.G, a.k, a.key_perm, a.key_gsize, a.query_perm, a.qblock_size, a.route, a.scale_log2, a.out);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 cudaError_t launch_attention(const AttnArgs& a, bool dense, cudaStream_t st) {
@@ -647,7 +647,7 @@ static cudaError_t launch_probe_t(const ProbeArgs& a, cudaStream_t st) {
         static_cast<const float*>(a.Q), static_cast<const float*>(a.K), static_cast<const float*>(a.V), a.N,
         a.block, a.G, a.k, a.probe_idx, a.P, a.key_perm, a.key_gsize, a.route, a.qblk, a.scale_log2,
         a.probe_out, a.probe_sparse);
-    return cudaGetLastError();
+    return counted(cudaGetLastError(), 2);
   }
   const int gps = probe_groups_per_split(a.G);
   const int nsplit = ceil_div(a.G, gps);
@@ -662,7 +662,7 @@ static cudaError_t launch_probe_t(const ProbeArgs& a, cudaStream_t st) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   probe_combine_kernel<D><<<dim3(a.P, a.heads), D, 0, st>>>(a.partial, a.P, nsplit, a.probe_out, a.probe_sparse);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 3);
 }
 
 cudaError_t launch_probe(const ProbeArgs& a, cudaStream_t st) {

@@ -123,4 +123,11 @@ __device__ __forceinline__ float float_from_order_key(uint32_t k) {
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Host-side count of kernels this library has enqueued (all devices, all threads).
+void note_launches(int n);
+inline cudaError_t counted(cudaError_t e, int n) {
+  if (e == cudaSuccess) note_launches(n);
+  return e;
+}
+
 }  // namespace spr

@@ -376,6 +376,45 @@ __global__ void probe_overwrite_kernel(const int* __restrict__ probe_idx, const 
       from_f32<TO>(probe_out[(static_cast<size_t>(head) * P + p) * D + e]);
 }
 
+// e_i = |o_i - o*_i| / |o*_i| per row (one warp per row); probe rows get NaN so that
+// the mean over unprobed rows the pages report can skip them.
+template <typename TO>
+__global__ void row_errors_kernel(const TO* __restrict__ O, const float* __restrict__ ref, int N, int d,
+                                  const int* __restrict__ probe_idx, int P, float* __restrict__ err) {
+  const int head = blockIdx.y;
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= N) return;
+  const size_t off = (static_cast<size_t>(head) * N + row) * d;
+  float num = 0.f, den = 0.f;
+  for (int e = lane; e < d; e += 32) {
+    const float r = ref[off + e];
+    const float diff = to_f32(O[off + e]) - r;
+    num += diff * diff;
+    den += r * r;
+  }
+  num = warp_sum(num);
+  den = warp_sum(den);
+  if (lane == 0) err[static_cast<size_t>(head) * N + row] = sqrtf(num) / sqrtf(den);
+}
+
+__global__ void mark_probe_rows_kernel(const int* __restrict__ probe_idx, int N, int P, float* __restrict__ err) {
+  const int head = blockIdx.y;
+  const int p = blockIdx.x * blockDim.x + threadIdx.x;
+  if (p < P) err[static_cast<size_t>(head) * N + probe_idx[static_cast<size_t>(head) * P + p]] = __int_as_float(0x7fc00000);
+}
+
+cudaError_t launch_row_errors(const void* O, bool o_f32, const float* ref, int heads, int N, int d,
+                              const int* probe_idx, int P, float* err, cudaStream_t st) {
+  dim3 grid(ceil_div(N, 8), heads);
+  if (o_f32) row_errors_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(O), ref, N, d, probe_idx, P, err);
+  else row_errors_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(O), ref, N, d, probe_idx, P, err);
+  cudaError_t e = counted(cudaGetLastError(), 1);
+  if (e != cudaSuccess || P == 0 || probe_idx == nullptr) return e;
+  mark_probe_rows_kernel<<<dim3(ceil_div(P, 256), heads), 256, 0, st>>>(probe_idx, N, P, err);
+  return counted(cudaGetLastError(), 1);
+}
+
 cudaError_t launch_fit(const float* xs, const float* dp, const float* weights, int heads, int d, int P,
                        double lambda, int rank, int weight_mode, double* scratch, float* M, float* beta,
                        int* status, cudaStream_t st) {
@@ -390,7 +429,7 @@ cudaError_t launch_fit(const float* xs, const float* dp, const float* weights, i
     if (e != cudaSuccess) return e;
     fit_kernel<128><<<heads, kFitThreads, smem, st>>>(xs, dp, weights, P, lambda, R, weight_mode, scratch, M, beta, status);
   }
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 size_t fit_smem_bytes(int d, int P) {
@@ -404,10 +443,10 @@ static cudaError_t launch_apply_t(const float* S, const float* M, const float* b
   cudaError_t e = cudaFuncSetAttribute(apply_kernel<D, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   apply_kernel<D, TO><<<dim3(ceil_div(N, 32), heads), 256, smem, st>>>(S, M, beta, N, O);
-  e = cudaGetLastError();
+  e = counted(cudaGetLastError(), 1);
   if (e != cudaSuccess || P == 0) return e;
   probe_overwrite_kernel<D, TO><<<dim3(P, heads), D, 0, st>>>(probe_idx, probe_out, N, P, O);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 cudaError_t launch_apply(const float* S, const float* M, const float* beta, const int* probe_idx,

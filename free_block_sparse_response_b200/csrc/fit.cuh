@@ -15,4 +15,7 @@ cudaError_t launch_apply(const float* S, const float* M, const float* beta, cons
                          const float* probe_out, int heads, int N, int d, int P, void* O, bool out_f32,
                          cudaStream_t st);
 
+cudaError_t launch_row_errors(const void* O, bool o_f32, const float* ref, int heads, int N, int d,
+                              const int* probe_idx, int P, float* err, cudaStream_t st);
+
 }  // namespace spr

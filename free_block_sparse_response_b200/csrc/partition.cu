@@ -475,20 +475,24 @@ __global__ void __launch_bounds__(kFillThreads) fill_coop_kernel(FillArgs a) {
         const float* drow = a.D + static_cast<size_t>(item) * G;
         const int* room = a.room + static_cast<size_t>(h) * G;
         unsigned long long best = ~0ull;
+        bool saw_nan = false;
         for (int g = lane; g < G; g += 32) {
           if (__ldcg(room + g) > 0) {
-            const unsigned long long key = decision_key(__ldcg(drow + g), g);
+            const float v = __ldcg(drow + g);
+            saw_nan |= (v != v);
+            const unsigned long long key = decision_key(v, g);
             best = key < best ? key : best;
           }
         }
         best = warp_min_u64(best);
+        saw_nan = __any_sync(0xffffffffu, saw_nan);
         if (lane == 0) {
+          if (saw_nan) record_error(&a.hdr->status, kErrNonFinite);
           if (best == ~0ull) {
             record_error(&a.hdr->status, kErrInvalidArg);
           } else {
             const int g = static_cast<int>(best & 0xffffffffu);
             const float v = __ldcg(drow + g);
-            if (v != v) record_error(&a.hdr->status, kErrNonFinite);
             a.prop_g[item] = g;
             a.prop_v[item] = v;
             atomicAdd(a.cnt + static_cast<size_t>(h) * G + g, 1);
@@ -645,7 +649,7 @@ __global__ void block_score_kernel(const float* __restrict__ qbar, const float* 
 
 cudaError_t launch_midpoint_stride(int* idx, int n, int count, cudaStream_t st) {
   midpoint_stride_kernel<<<ceil_div(count, 256), 256, 0, st>>>(idx, n, count);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 cudaError_t launch_gram(const void* X, bool f32, size_t head_stride, const int* rows, int nrows, int heads,
@@ -658,18 +662,18 @@ cudaError_t launch_gram(const void* X, bool f32, size_t head_stride, const int* 
     if (d == 64) gram_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), head_stride, rows, nrows, gamma);
     else gram_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), head_stride, rows, nrows, gamma);
   }
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 cudaError_t launch_split_bf16(const float* src, __nv_bfloat16* hi, __nv_bfloat16* lo, size_t count, cudaStream_t st) {
   const int blocks = static_cast<int>(std::min<size_t>(4096, (count + 255) / 256));
   split_bf16_kernel<<<blocks, 256, 0, st>>>(src, hi, lo, count);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 cudaError_t launch_chunk_perm(int* perm, int* sizes, int n, int G, int cap, int heads, cudaStream_t st) {
   chunk_perm_kernel<<<dim3(ceil_div(G * cap, 256), heads), 256, 0, st>>>(perm, sizes, n, G, cap);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 cudaError_t launch_centroid(const void* X, bool f32, int n, const int* perm, const int* sizes, int G, int cap,
@@ -682,7 +686,7 @@ cudaError_t launch_centroid(const void* X, bool f32, int n, const int* perm, con
     if (d == 64) centroid_kernel<__nv_bfloat16, 64><<<grid, 64, 0, st>>>(static_cast<const __nv_bfloat16*>(X), n, perm, sizes, G, cap, cent);
     else centroid_kernel<__nv_bfloat16, 128><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(X), n, perm, sizes, G, cap, cent);
   }
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 cudaError_t launch_wmat(const float* cent, const float* gamma, int G, int heads, int d, float* wf,
@@ -690,7 +694,7 @@ cudaError_t launch_wmat(const float* cent, const float* gamma, int G, int heads,
   dim3 grid(ceil_div(G, 8), heads);
   if (d == 64) wmat_kernel<64><<<grid, 64, 0, st>>>(cent, gamma, G, wf, whi, wlo, eg);
   else wmat_kernel<128><<<grid, 128, 0, st>>>(cent, gamma, G, wf, whi, wlo, eg);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 template <int D, bool DIST, bool SPLIT>
@@ -702,7 +706,7 @@ static cudaError_t launch_rowgemm_mma_t(const RowGemmArgs& a, cudaStream_t st) {
   kern<<<dim3(ceil_div(a.n, kGemmRows), a.heads), 256, smem, st>>>(
       static_cast<const __nv_bfloat16*>(a.X), a.n, a.Bhi, a.Blo, a.ncols, a.nrm, a.ecol, a.tau2, a.Dout,
       a.prop_g, a.prop_v, a.nrm_out, a.status);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 cudaError_t launch_rowgemm(const RowGemmArgs& a, bool dist, cudaStream_t st) {
@@ -716,7 +720,7 @@ cudaError_t launch_rowgemm(const RowGemmArgs& a, bool dist, cudaStream_t st) {
       if (dist) rowgemm_f32_kernel<128, true><<<grid, 256, 0, st>>>(X, a.n, a.Bf32, a.ncols, a.nrm, a.ecol, a.tau2, a.Dout, a.prop_g, a.prop_v, a.nrm_out, a.status);
       else rowgemm_f32_kernel<128, false><<<grid, 256, 0, st>>>(X, a.n, a.Bf32, a.ncols, a.nrm, a.ecol, a.tau2, a.Dout, a.prop_g, a.prop_v, a.nrm_out, a.status);
     }
-    return cudaGetLastError();
+    return counted(cudaGetLastError(), 1);
   }
   const bool split = a.Blo != nullptr;
   if (a.d == 64) {
@@ -741,8 +745,9 @@ cudaError_t launch_fill(const FillArgs& a, cudaStream_t st) {
   const int blocks = sms * std::min(per_sm, 2);
   FillArgs args = a;
   void* params[] = {&args};
-  return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(fill_coop_kernel), dim3(blocks), dim3(kFillThreads),
-                                     params, 0, st);
+  e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(fill_coop_kernel), dim3(blocks), dim3(kFillThreads),
+                                  params, 0, st);
+  return counted(e, 2);
 }
 
 cudaError_t launch_build_perm(const int* labels, int n, int G, int cap, int heads, int* cursor, int* tmp,
@@ -753,7 +758,7 @@ cudaError_t launch_build_perm(const int* labels, int n, int G, int cap, int head
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   perm_sort_kernel<<<dim3(G, heads), cap, cap * sizeof(int), st>>>(cursor, tmp, G, cap, perm, sizes);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 2);
 }
 
 cudaError_t launch_block_scores(const float* qbar, const float* mu, int G, int heads, int d, float tau,
@@ -761,7 +766,7 @@ cudaError_t launch_block_scores(const float* qbar, const float* mu, int G, int h
   dim3 grid(ceil_div(G, 16), ceil_div(G, 16), heads);
   if (d == 64) block_score_kernel<64><<<grid, 256, 0, st>>>(qbar, mu, G, tau, sc);
   else block_score_kernel<128><<<grid, 256, 0, st>>>(qbar, mu, G, tau, sc);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 }  // namespace spr

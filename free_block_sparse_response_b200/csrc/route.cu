@@ -92,6 +92,7 @@ __global__ void __launch_bounds__(256)
     }
     written += __popc(ball);
   }
+  saw_nan = __any_sync(0xffffffffu, saw_nan);
   if (lane == 0 && (saw_nan || written != k)) record_error(status, written != k ? kErrInvalidArg : kErrNonFinite);
   if (pairs != nullptr) {
 #pragma unroll
@@ -119,7 +120,7 @@ cudaError_t launch_route(const float* sc, int heads, int Gq, int G, int k, int* 
   }
   route_topk_kernel<<<dim3(ceil_div(Gq, 8), heads), 256, 0, st>>>(sc, Gq, G, k, route, key_gsize, qblock_size,
                                                                    up, status);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), up != nullptr ? 2 : 1);
 }
 
 }  // namespace spr

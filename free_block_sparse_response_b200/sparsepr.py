@@ -25,7 +25,7 @@ EXPORTED_SYMBOLS = (
     "sparsepr_partition", "sparsepr_route", "sparsepr_sparse_attn", "sparsepr_dense_attn",
     "sparsepr_probe_dense", "sparsepr_fit_residual", "sparsepr_apply_residual", "sparsepr_check",
     "sparsepr_last_error", "sparsepr_test_fill_workspace_size", "sparsepr_test_fill",
-    "sparsepr_test_topk",
+    "sparsepr_test_topk", "sparsepr_row_errors", "sparsepr_launch_count",
 )
 
 
@@ -97,6 +97,8 @@ def lib() -> ctypes.CDLL:
         "sparsepr_test_fill_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32]),
         "sparsepr_test_fill": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
         "sparsepr_test_topk": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+        "sparsepr_row_errors": (ctypes.c_int, [_vp, ctypes.c_int, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
+        "sparsepr_launch_count": (ctypes.c_uint64, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -288,6 +290,24 @@ def attention(q, k, v, cfg: SparsePRConfig, ws: Optional[torch.Tensor] = None, o
         return o
     return o, {"partition": part, "route": rt, "k": kk, "executed_pairs": pairs, "S": s_out, "probe_idx": pidx,
                "probe_out": p_out, "probe_sparse": p_sparse, "M": m, "beta": beta, "ws": ws}
+
+
+# ------------------------------------------------------------------------ measurement
+
+def row_errors(o: torch.Tensor, o_ref: torch.Tensor, probe_idx: Optional[torch.Tensor]) -> torch.Tensor:
+    """Per-row relative L2 error of o against o_ref ([Bt,H,N] fp32, NaN on probe rows)."""
+    _need_cuda(o, o_ref, probe_idx)
+    bt, h, n, d = o.shape
+    p = 0 if probe_idx is None else probe_idx.shape[-1]
+    err = torch.empty(bt, h, n, dtype=torch.float32, device=o.device)
+    _call("sparsepr_row_errors", _p(o), _DTYPE_CODE[o.dtype], _p(o_ref), _p(probe_idx), bt, h, n, d, p, _p(err),
+          _stream(o))
+    return err
+
+
+def launch_count() -> int:
+    """Kernels the library has enqueued since it was loaded."""
+    return int(lib().sparsepr_launch_count())
 
 
 # ------------------------------------------------------- decision kernels, injected input

@@ -182,6 +182,19 @@ SPARSEPR_API int sparsepr_apply_residual(const float* S_out, const float* M, con
                             int32_t Bt, int32_t H, int32_t N, int32_t d, int32_t P,
                             void* O, int out_dtype, sparsepr_stream_t stream);
 
+/* Measurement: per-row relative L2 error against a reference output (the metric the
+ * abstract reports, averaged there over unprobed queries):
+ *   err[b,h,i] = |O_i - O_ref_i|_2 / |O_ref_i|_2, and NaN for the P probe rows listed in
+ *   probe_idx [Bt,H,P] (NULL or P = 0: no row is marked).
+ *   O [Bt,H,N,d] in o_dtype; O_ref [Bt,H,N,d] fp32; err [Bt,H,N] fp32. */
+SPARSEPR_API int sparsepr_row_errors(const void* O, int o_dtype, const float* O_ref,
+                                     const int32_t* probe_idx, int32_t Bt, int32_t H,
+                                     int32_t N, int32_t d, int32_t P, float* err,
+                                     sparsepr_stream_t stream);
+
+/* Number of kernels this library has enqueued since it was loaded (host counter). */
+SPARSEPR_API uint64_t sparsepr_launch_count(void);
+
 /* Wait for `stream` and return the device status word in `ws` (SPARSEPR_OK, or the
  * first device-side error since the last sparsepr_partition).  This is the only call
  * that synchronises. */

@@ -18,7 +18,7 @@ from synthetic import CONFIGS, make_inputs
 pytestmark = pytest.mark.gpu
 
 TOL_BF16 = 3e-3     # per-head output rel-L2, bf16 inputs / fp32 accumulation
-TOL_F32 = 2e-5      # fp32 inputs, fp32 SIMT arithmetic
+TOL_F32 = 1e-4      # fp32 inputs, fp32 SIMT arithmetic; the fit at P < d+1 amplifies rounding
 TOL_MAP = 1e-3      # fitted M and beta, relative Frobenius
 TOL_PROBE = 2e-4    # probe rows: softmax weights carried at ~16 bits
 
