@@ -158,7 +158,10 @@ def workspace_size(batch: int, heads: int, n: int, d: int, cfg: SparsePRConfig) 
 
 
 def new_workspace(batch: int, heads: int, n: int, d: int, cfg: SparsePRConfig, device) -> torch.Tensor:
-    return torch.empty(workspace_size(batch, heads, n, d, cfg), dtype=torch.uint8, device=device)
+    """Workspace for calls of these sizes; its 256-byte status header starts at zero."""
+    ws = torch.empty(workspace_size(batch, heads, n, d, cfg), dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
 
 
 def check(ws: torch.Tensor) -> None:

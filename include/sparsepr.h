@@ -23,7 +23,9 @@
  *  - Tensor arguments are DEVICE pointers owned by the caller; the library never
  *    allocates, frees or synchronises on them.  Scratch space is the caller's
  *    workspace `ws` of sparsepr_workspace_size() bytes (256-byte aligned), which
- *    must not be shared by calls that may overlap on the GPU.
+ *    must not be shared by calls that may overlap on the GPU.  Its first 256 bytes
+ *    are a status header that must be zero before the first call on a new workspace
+ *    (sparsepr_partition zeroes it again at the start of every call sequence).
  *  - Every call is asynchronous on `stream` (0 = legacy default stream).
  *  - Layouts are contiguous row-major: Q, K, V, O are [Bt, H, N, d]; per-head index
  *    arrays are [Bt, H, ...] as stated.  dtype is SPARSEPR_BF16 or SPARSEPR_F32;
