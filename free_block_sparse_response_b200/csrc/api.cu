@@ -4,6 +4,7 @@
 #include <cstdio>
 #include <atomic>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "../../include/sparsepr.h"
@@ -500,3 +501,73 @@ int sparsepr_test_topk(const float* Sc, int32_t H, int32_t Gq, int32_t G, int32_
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Allocation-free variant of the residual fit.
+//
+// Some callers cannot call cudaMalloc: an inference-engine plugin must run inside the
+// memory plan its host engine fixed before execution, and a latency-critical serving loop
+// cannot take cudaMalloc's implicit device synchronisation and unbounded latency.  This
+// entry point takes its scratch from a fixed array compiled into the library instead of a
+// caller workspace.  The array is file-scope and static: every GPU that loads the library
+// holds it until the process exits.  Its host-side name is only a stand-in for the device
+// array, so the device address is looked up once per device (with that device current)
+// and that address is what the kernel receives.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 32ull << 20;  // 32 MiB
+constexpr size_t kNoAllocStatusBytes = 256;            // status word, cleared every call
+constexpr int kNoAllocMaxDevices = 64;
+
+__device__ __align__(256) unsigned char g_fit_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_base[kNoAllocMaxDevices] = {};
+
+// Device address of the static scratch array on the current device (looked up once).
+int noalloc_scratch(void** base) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "fit_noalloc: current device");
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(SPARSEPR_ERR_UNSUPPORTED, "device index %d too large", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_base[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_fit_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "fit_noalloc: scratch address");
+    g_noalloc_base[dev] = ptr;
+  }
+  *base = g_noalloc_base[dev];
+  return SPARSEPR_OK;
+}
+
+}  // namespace
+
+extern "C" int sparsepr_fit_residual_noalloc(const float* probe_sparse, const float* probe_out, const float* weights,
+                                             int32_t Bt, int32_t H, int32_t d, int32_t P, double ridge_lambda,
+                                             int32_t rank, int32_t weight_mode, float* M, float* beta,
+                                             sparsepr_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(Bt, H, 1, d))) return rc;
+  if (P < 1) return fail(SPARSEPR_ERR_INVALID_ARG, "P must be >= 1");
+  if (rank < 1) return fail(SPARSEPR_ERR_INVALID_ARG, "rank must be >= 1");
+  if (!(ridge_lambda >= 0.0)) return fail(SPARSEPR_ERR_INVALID_ARG, "ridge_lambda must be >= 0");
+  if (weight_mode != SPARSEPR_WEIGHT_INV_NORM && weight_mode != SPARSEPR_WEIGHT_UNIFORM)
+    return fail(SPARSEPR_ERR_INVALID_ARG, "unknown weight_mode %d", weight_mode);
+  if (!probe_sparse || !probe_out || !M || !beta) return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
+  if (spr::fit_smem_bytes(d, P) > 220 * 1024) return fail(SPARSEPR_ERR_UNSUPPORTED, "P=%d too large for the fit", P);
+  const size_t need = kNoAllocStatusBytes + sizeof(double) * static_cast<size_t>(Bt) * H * spr::fit_scratch_doubles(P, d);
+  if (need > kNoAllocScratchBytes)
+    return fail(SPARSEPR_ERR_UNSUPPORTED,
+                "fit_noalloc: Bt*H=%d heads at d=%d, P=%d need %zu bytes of scratch; the fixed array holds %zu",
+                Bt * H, d, P, need, kNoAllocScratchBytes);
+  void* base = nullptr;
+  if ((rc = noalloc_scratch(&base))) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  SPR_CUDA(cudaMemsetAsync(base, 0, kNoAllocStatusBytes, st), "fit_noalloc: clear status");
+  double* scratch = reinterpret_cast<double*>(static_cast<char*>(base) + kNoAllocStatusBytes);
+  SPR_CUDA(spr::launch_fit(probe_sparse, probe_out, weights, Bt * H, d, P, ridge_lambda, rank, weight_mode, scratch, M,
+                           beta, static_cast<int*>(base), st),
+           "fit_noalloc");
+  return SPARSEPR_OK;
+}

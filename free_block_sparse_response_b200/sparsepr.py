@@ -25,7 +25,7 @@ EXPORTED_SYMBOLS = (
     "sparsepr_partition", "sparsepr_route", "sparsepr_sparse_attn", "sparsepr_dense_attn",
     "sparsepr_probe_dense", "sparsepr_fit_residual", "sparsepr_apply_residual", "sparsepr_check",
     "sparsepr_last_error", "sparsepr_test_fill_workspace_size", "sparsepr_test_fill",
-    "sparsepr_test_topk", "sparsepr_row_errors", "sparsepr_launch_count",
+    "sparsepr_test_topk", "sparsepr_row_errors", "sparsepr_launch_count", "sparsepr_fit_residual_noalloc",
 )
 
 
@@ -99,6 +99,8 @@ def lib() -> ctypes.CDLL:
         "sparsepr_test_topk": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
         "sparsepr_row_errors": (ctypes.c_int, [_vp, ctypes.c_int, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
         "sparsepr_launch_count": (ctypes.c_uint64, []),
+        "sparsepr_fit_residual_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, ctypes.c_double,
+                                                         _i32, _i32, _vp, _vp, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -257,6 +259,18 @@ def fit_residual(probe_sparse, probe_out, cfg: SparsePRConfig, ws: torch.Tensor,
     beta = torch.empty(bt, h, d, dtype=torch.float32, device=probe_out.device)
     _call("sparsepr_fit_residual", _p(probe_sparse), _p(probe_out), _p(weights), bt, h, d, p, cfg.ridge_lambda,
           cfg.rank, cfg.weight_mode, _p(m), _p(beta), _p(ws), _stream(probe_out))
+    return m, beta
+
+
+def fit_residual_noalloc(probe_sparse, probe_out, cfg: SparsePRConfig, m: torch.Tensor, beta: torch.Tensor,
+                         weights: Optional[torch.Tensor] = None):
+    """The fit through the allocation-free entry point, for callers that cannot
+    allocate device memory during the call: results go to the caller's m [Bt,H,d,d]
+    and beta [Bt,H,d]; scratch is the library's fixed static array (no workspace)."""
+    _need_cuda(probe_sparse, probe_out, m, beta, weights)
+    bt, h, p, d = probe_out.shape
+    _call("sparsepr_fit_residual_noalloc", _p(probe_sparse), _p(probe_out), _p(weights), bt, h, d, p,
+          cfg.ridge_lambda, cfg.rank, cfg.weight_mode, _p(m), _p(beta), _stream(probe_out))
     return m, beta
 
 

@@ -177,6 +177,26 @@ SPARSEPR_API int sparsepr_fit_residual(const float* probe_sparse, const float* p
                           int32_t weight_mode, float* M, float* beta, void* ws,
                           sparsepr_stream_t stream);
 
+/* Allocation-free variant of sparsepr_fit_residual (no counterpart in the paper: it is
+ * an interface for callers that cannot allocate device memory, such as an inference-
+ * engine plugin bound to a memory plan fixed before execution, or a latency-critical
+ * loop that cannot take cudaMalloc's implicit synchronisation).  Same arguments, layout
+ * and result as sparsepr_fit_residual, but no workspace: the scratch is a 32 MiB static
+ * device array inside the library, held by every GPU that loads it until the process
+ * exits.  Limit: 256 + 8 * Bt*H * (2 d^2 + P d + 4 d) bytes <= 32 MiB (d = 128, P = 256:
+ * 63 heads); larger calls return SPARSEPR_ERR_UNSUPPORTED without launching.  The call
+ * allocates nothing (no cudaMalloc/cudaFree).  The first call on each device looks up the
+ * array's device address; make that first call before any stream capture.  Every call
+ * shares the one array (it keeps the last call's contents; the kernel rewrites all of it
+ * before reading it), so calls that overlap on the GPU race: serialise them, e.g. on one
+ * stream.  Device-side failures (non-positive weight sum, a failed Cholesky) write M = 0
+ * and beta = 0 for the head. */
+SPARSEPR_API int sparsepr_fit_residual_noalloc(const float* probe_sparse, const float* probe_out,
+                                               const float* weights, int32_t Bt, int32_t H,
+                                               int32_t d, int32_t P, double ridge_lambda,
+                                               int32_t rank, int32_t weight_mode, float* M,
+                                               float* beta, sparsepr_stream_t stream);
+
 /* (d3) Apply: O_i = S_i + M S_i + beta for unprobed rows, O_p = probe_out_p for probe
  * rows.  O [Bt,H,N,d] in out_dtype.  O may alias S_out when out_dtype is F32. */
 SPARSEPR_API int sparsepr_apply_residual(const float* S_out, const float* M, const float* beta,
