@@ -302,7 +302,7 @@ def run_ours(args, w):
     t_sparse = stage_ms["sparse_attn"] / 1e3
     peak, peak_src = measured_peak()
     achieved = sparse_flops / t_sparse / 1e12
-    roofline = {"kernel": "attn_mma_kernel (block-sparse attention)", "bound": "tensor", "achieved": achieved,
+    roofline = {"kernel": "attn_tc_kernel<false> (block-sparse attention, tcgen05)", "bound": "tensor", "achieved": achieved,
                 "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": DOMINANT_TRAFFIC_BYTES,
                 "peak_source": peak_src,
                 "per_launch_flops": sparse_flops}

@@ -294,10 +294,13 @@ int sparsepr_route(const float* block_scores, const int32_t* key_gsize, const in
   return SPARSEPR_OK;
 }
 
+// Status word for attention calls made without a workspace (the dense comparator).
+__device__ int g_attention_status_sink;
+
 static int attention_common(const void* Q, const void* K, const void* V, int dtype, int32_t Bt, int32_t H,
                             int32_t N, int32_t d, int32_t block, const int32_t* key_perm, const int32_t* key_gsize,
                             const int32_t* query_perm, const int32_t* qblock_size, const int32_t* route, int32_t k,
-                            float scale, float* out, bool dense, sparsepr_stream_t stream) {
+                            float scale, float* out, bool dense, void* ws, sparsepr_stream_t stream) {
   int rc;
   if ((rc = check_shape(Bt, H, N, d)) || (rc = check_dtype(dtype)) || (rc = check_block(block))) return rc;
   if (!Q || !K || !V || !out) return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
@@ -325,6 +328,11 @@ static int attention_common(const void* Q, const void* K, const void* V, int dty
   a.route = route;
   a.scale_log2 = resolve_scale(scale, d) * kLog2e;
   a.out = out;
+  if (ws != nullptr) {
+    a.status = &header(ws)->status;
+  } else {
+    SPR_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&a.status), g_attention_status_sink), "status sink");
+  }
   SPR_CUDA(spr::launch_attention(a, dense, reinterpret_cast<cudaStream_t>(stream)), dense ? "dense attention" : "sparse attention");
   return SPARSEPR_OK;
 }
@@ -333,16 +341,14 @@ int sparsepr_sparse_attn(const void* Q, const void* K, const void* V, int dtype,
                          int32_t d, int32_t block, const int32_t* key_perm, const int32_t* key_gsize,
                          const int32_t* query_perm, const int32_t* qblock_size, const int32_t* route, int32_t k,
                          float scale, float* S_out, void* ws, sparsepr_stream_t stream) {
-  (void)ws;
   return attention_common(Q, K, V, dtype, Bt, H, N, d, block, key_perm, key_gsize, query_perm, qblock_size, route, k,
-                          scale, S_out, false, stream);
+                          scale, S_out, false, ws, stream);
 }
 
 int sparsepr_dense_attn(const void* Q, const void* K, const void* V, int dtype, int32_t Bt, int32_t H, int32_t N,
                         int32_t d, int32_t block, float scale, float* O_out, void* ws, sparsepr_stream_t stream) {
-  (void)ws;
   return attention_common(Q, K, V, dtype, Bt, H, N, d, block, nullptr, nullptr, nullptr, nullptr, nullptr, 0, scale,
-                          O_out, true, stream);
+                          O_out, true, ws, stream);
 }
 
 int sparsepr_probe_dense(const void* Q, const void* K, const void* V, int dtype, int32_t Bt, int32_t H, int32_t N,

@@ -618,6 +618,7 @@ static cudaError_t launch_attn_f32_t(const AttnArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_attention(const AttnArgs& a, bool dense, cudaStream_t st) {
+  if (!a.f32 && a.d == 128 && a.block == 128) return launch_attention_tc(a, dense, a.status, st);
   if (a.f32) {
     if (a.d == 64) return dense ? launch_attn_f32_t<64, true>(a, st) : launch_attn_f32_t<64, false>(a, st);
     return dense ? launch_attn_f32_t<128, true>(a, st) : launch_attn_f32_t<128, false>(a, st);

@@ -19,6 +19,7 @@ struct AttnArgs {
   const int* route;
   float scale_log2;  // tau * log2(e)
   float* out;
+  int* status;       // device status word (bounded waits of the tensor-core kernel)
 };
 
 struct ProbeArgs {
@@ -40,6 +41,8 @@ struct ProbeArgs {
 };
 
 cudaError_t launch_attention(const AttnArgs& a, bool dense, cudaStream_t st);
+cudaError_t launch_attention_tc(const AttnArgs& a, bool dense, int* status, cudaStream_t st);
+size_t attn_tc_smem_bytes();
 cudaError_t launch_probe(const ProbeArgs& a, cudaStream_t st);
 size_t probe_partial_bytes(int heads, int P, int G, int d);
 cudaError_t launch_probe_rows(int N, int P, int heads, int* probe_idx, cudaStream_t st);

@@ -221,12 +221,13 @@ def sparse_attn(q, k, v, part: Partition, rt: torch.Tensor, kk: int, cfg: Sparse
     return s_out
 
 
-def dense_attn(q, k, v, block: int = 128, scale: float = 0.0, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+def dense_attn(q, k, v, block: int = 128, scale: float = 0.0, out: Optional[torch.Tensor] = None,
+               ws: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Dense softmax attention of every row with the same kernel family (fp32 out)."""
-    _need_cuda(q, k, v)
+    _need_cuda(q, k, v, ws)
     bt, h, n, d = q.shape
     o = torch.empty(bt, h, n, d, dtype=torch.float32, device=q.device) if out is None else out
-    _call("sparsepr_dense_attn", _p(q), _p(k), _p(v), _dtype_code(q), bt, h, n, d, block, scale, _p(o), None,
+    _call("sparsepr_dense_attn", _p(q), _p(k), _p(v), _dtype_code(q), bt, h, n, d, block, scale, _p(o), _p(ws),
           _stream(q))
     return o
 
