@@ -42,7 +42,7 @@ struct ProbeArgs {
 
 cudaError_t launch_attention(const AttnArgs& a, bool dense, cudaStream_t st);
 cudaError_t launch_attention_tc(const AttnArgs& a, bool dense, int* status, cudaStream_t st);
-size_t attn_tc_smem_bytes();
+size_t attn_tc_smem_bytes(int n_tiles);
 cudaError_t launch_probe(const ProbeArgs& a, cudaStream_t st);
 size_t probe_partial_bytes(int heads, int P, int G, int d);
 cudaError_t launch_probe_rows(int N, int P, int heads, int* probe_idx, cudaStream_t st);

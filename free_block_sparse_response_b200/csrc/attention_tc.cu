@@ -112,38 +112,58 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int* kperm = DENSE ? nullptr : key_perm + goff * 128;
   const int n_tiles = DENSE ? G : k;
   const int* my_route = DENSE ? nullptr : route + (goff + b) * k;
-  auto group_of = [&](int j) { return DENSE ? j : __ldg(my_route + j); };
-  auto group_size = [&](int g) { return DENSE ? min(128, N - g * 128) : __ldg(key_gsize + goff + g); };
+  // per-tile key group and its size, staged once (the producers and the softmax read them)
+  int* s_group = reinterpret_cast<int*>(dsmem + (sbase - tc::saddr(dsmem)) + 5 * kTile);
+  int* s_size = s_group + n_tiles;
+  for (int j = tid; j < n_tiles; j += kTcThreads) {
+    const int g = DENSE ? j : __ldg(my_route + j);
+    s_group[j] = g;
+    s_size[j] = DENSE ? min(128, N - g * 128) : __ldg(key_gsize + goff + g);
+  }
+  __syncthreads();
   volatile int* abort_v = &abort_flag;
 
   if (warp < 2) {
     // ------------------------------------------------------------------ producers
-    const int pt = tid;
-    for (int x = pt; x < 128 * 16; x += kTcProducers) {
-      const int r = x >> 4, ch = x & 15;
-      const int tok = r < nq ? (DENSE ? b * 128 + r : __ldg(qperm + r)) : -1;
-      cp_async_16(sQ + tc::sw128_offset(r, ch), tok >= 0 ? Q + static_cast<size_t>(tok) * 128 + ch * 8 : Q,
-                  tok >= 0 ? 16 : 0);
+    // Thread pt copies 16-byte chunk (pt & 15) of rows (pt >> 4) + 4 i, i < 32: 16 threads
+    // cover one 256-byte row.  The 32 row indices are fetched before any copy is issued.
+    const int pt = tid, ch = pt & 15, r0 = pt >> 4;
+    int toks[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int r = r0 + 4 * i;
+      toks[i] = r < nq ? (DENSE ? b * 128 + r : __ldg(qperm + r)) : -1;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int r = r0 + 4 * i;
+      cp_async_16(sQ + tc::sw128_offset(r, ch), toks[i] >= 0 ? Q + static_cast<size_t>(toks[i]) * 128 + ch * 8 : Q,
+                  toks[i] >= 0 ? 16 : 0);
     }
     tc::cp_async_arrive_noinc(bar(kQFull));
     for (int j = 0; j < n_tiles; ++j) {
       const int s = j & 1;
-      const int g = group_of(j);
-      const int gs = group_size(g);
+      const int g = s_group[j];
+      const int gs = s_size[j];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = r0 + 4 * i;
+        toks[i] = r < gs ? (DENSE ? g * 128 + r : __ldg(kperm + g * 128 + r)) : -1;
+      }
       if (j >= 2 && !tc::mbar_wait(bar(kKEmpty0 + s), ((j >> 1) - 1) & 1, abort_v, status)) break;
-      for (int x = pt; x < 128 * 16; x += kTcProducers) {
-        const int r = x >> 4, ch = x & 15;
-        const int tok = r < gs ? (DENSE ? g * 128 + r : __ldg(kperm + g * 128 + r)) : -1;
-        cp_async_16(sK[s] + tc::sw128_offset(r, ch), tok >= 0 ? K + static_cast<size_t>(tok) * 128 + ch * 8 : K,
-                    tok >= 0 ? 16 : 0);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = r0 + 4 * i;
+        cp_async_16(sK[s] + tc::sw128_offset(r, ch),
+                    toks[i] >= 0 ? K + static_cast<size_t>(toks[i]) * 128 + ch * 8 : K, toks[i] >= 0 ? 16 : 0);
       }
       tc::cp_async_arrive_noinc(bar(kKFull0 + s));
       if (j >= 2 && !tc::mbar_wait(bar(kVEmpty0 + s), ((j >> 1) - 1) & 1, abort_v, status)) break;
-      for (int x = pt; x < 128 * 16; x += kTcProducers) {
-        const int r = x >> 4, ch = x & 15;
-        const int tok = r < gs ? (DENSE ? g * 128 + r : __ldg(kperm + g * 128 + r)) : -1;
-        cp_async_16(sV[s] + tc::sw128_offset(r, ch), tok >= 0 ? V + static_cast<size_t>(tok) * 128 + ch * 8 : V,
-                    tok >= 0 ? 16 : 0);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = r0 + 4 * i;
+        cp_async_16(sV[s] + tc::sw128_offset(r, ch),
+                    toks[i] >= 0 ? V + static_cast<size_t>(toks[i]) * 128 + ch * 8 : V, toks[i] >= 0 ? 16 : 0);
       }
       tc::cp_async_arrive_noinc(bar(kVFull0 + s));
     }
@@ -213,14 +233,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc::tmem_ld32(sbuf + 64, *reinterpret_cast<uint32_t(*)[32]>(&u[64]));
       tc::tmem_ld32(sbuf + 96, *reinterpret_cast<uint32_t(*)[32]>(&u[96]));
       tc::tmem_wait_ld();
-      const int nvalid = group_size(group_of(j));
+      const int nvalid = s_size[j];
       float mx = -kInf;
 #pragma unroll
       for (int c = 0; c < 128; ++c) {
-        const float x = c < nvalid ? __uint_as_float(u[c]) * scale_log2 : -kInf;
+        const float x = c < nvalid ? __uint_as_float(u[c]) : -kInf;
         u[c] = __float_as_uint(x);
         mx = fmaxf(mx, x);
       }
+      mx *= scale_log2;
       const bool grow = mx > m_run + kRescaleLog2;
       const bool need_o = grow && m_run != -kInf;
       float alpha = 1.f;
@@ -253,8 +274,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2(__uint_as_float(u[half * 64 + 2 * i]) - msafe);
-          const float p1 = ex2(__uint_as_float(u[half * 64 + 2 * i + 1]) - msafe);
+          const float p0 = ex2(fmaf(__uint_as_float(u[half * 64 + 2 * i]), scale_log2, -msafe));
+          const float p1 = ex2(fmaf(__uint_as_float(u[half * 64 + 2 * i + 1]), scale_log2, -msafe));
           sum += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
@@ -296,10 +317,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 }  // namespace
 
-size_t attn_tc_smem_bytes() { return 5ull * kTile + 1024; }
+size_t attn_tc_smem_bytes(int n_tiles) { return 5ull * kTile + 1024 + 8ull * n_tiles; }
 
 cudaError_t launch_attention_tc(const AttnArgs& a, bool dense, int* status, cudaStream_t st) {
-  const size_t smem = attn_tc_smem_bytes();
+  const size_t smem = attn_tc_smem_bytes(dense ? a.G : a.k);
+  if (smem > 227 * 1024) return cudaErrorInvalidValue;
   auto kern = dense ? attn_tc_kernel<true> : attn_tc_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
