@@ -51,7 +51,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 // Byte offsets of every scratch region inside the caller's workspace.
 struct Layout {
   size_t header = 0, sample_idx, gamma, gamma_hi, gamma_lo, nrm, cent_k, cent_q, wf, whi, wlo, eg, dmat,
-         prop_g0, prop_v0, labels, room, cnt, offs, cursor, bucket, list0, list1, list_len, prop_g, prop_v,
+         prop_g0, prop_v0, labels, room, cnt, offs, cursor, closed, bucket, list0, list1, list_len, prop_g, prop_v,
          perm_tmp, perm_cursor, qblk, partial, fit, total;
 };
 
@@ -83,6 +83,7 @@ Layout make_layout(int heads, int N, int d, int block, int S, int P) {
   L.cnt = take(sizeof(int) * H * G);
   L.offs = take(sizeof(int) * H * G);
   L.cursor = take(sizeof(int) * H * G);
+  L.closed = take(sizeof(unsigned int) * H * ((G + 31) / 32));
   L.bucket = take(sizeof(unsigned long long) * H * n);
   L.list0 = take(sizeof(int) * H * n);
   L.list1 = take(sizeof(int) * H * n);
@@ -212,6 +213,7 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
   fa.cnt = at<int>(ws, L.cnt);
   fa.offs = at<int>(ws, L.offs);
   fa.cursor = at<int>(ws, L.cursor);
+  fa.closed = at<unsigned int>(ws, L.closed);
   fa.bucket = at<unsigned long long>(ws, L.bucket);
   fa.list0 = at<int>(ws, L.list0);
   fa.list1 = at<int>(ws, L.list1);
@@ -453,6 +455,7 @@ size_t sparsepr_test_fill_workspace_size(int32_t H, int32_t n, int32_t G) {
   if (H < 1 || n < 1 || G < 1) return 0;
   const size_t h = H, nn = n, g = G;
   return align_up(sizeof(spr::WorkspaceHeader)) + align_up(4 * h * g * sizeof(int)) +
+         align_up(h * ((g + 31) / 32) * sizeof(unsigned int)) +
          align_up(h * nn * sizeof(unsigned long long)) + 3 * align_up(h * nn * sizeof(int)) + align_up(4 * sizeof(int)) +
          align_up(h * nn * sizeof(float));
 }
@@ -484,6 +487,7 @@ int sparsepr_test_fill(const float* D, int32_t H, int32_t n, int32_t G, int32_t 
   fa.cnt = fa.room + h * g;
   fa.offs = fa.cnt + h * g;
   fa.cursor = fa.offs + h * g;
+  fa.closed = at<unsigned int>(ws, take(h * ((g + 31) / 32) * sizeof(unsigned int)));
   fa.bucket = at<unsigned long long>(ws, take(h * nn * sizeof(unsigned long long)));
   fa.list0 = at<int>(ws, take(h * nn * sizeof(int)));
   fa.list1 = at<int>(ws, take(h * nn * sizeof(int)));

@@ -365,16 +365,36 @@ __global__ void __launch_bounds__(256)
 // --------------------------------------------------------------- capacity-constrained fill
 // Rounds: every unplaced item proposes to its nearest group with room (ties -> lower
 // group); each group accepts its proposers in ascending (distance, token) order while
-// it has room.  One cooperative launch runs every round for every head.
+// it has room.  One cooperative launch runs every round for every head.  Full groups
+// are tracked in a per-head bitmap so a proposal reads only its distance row.
 
+// Key of the kth smallest (1-based) of `count` distinct 64-bit keys, by a warp: radix
+// select on 8-bit digits, starting below the bits all keys share and stopping as soon
+// as the selected digit bin holds a single key.
 __device__ unsigned long long warp_select_kth(const unsigned long long* keys, int count, int kth,
                                               unsigned int* hist) {
   const int lane = threadIdx.x & 31;
-  unsigned long long prefix = 0;
-  for (int shift = 56; shift >= 0; shift -= 8) {
+  unsigned long long kmin = ~0ull, kmax = 0ull;
+  for (int e = lane; e < count; e += 32) {
+    const unsigned long long key = __ldcg(keys + e);
+    kmin = key < kmin ? key : kmin;
+    kmax = key > kmax ? key : kmax;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin, o);
+    const unsigned long long b = __shfl_xor_sync(0xffffffffu, kmax, o);
+    kmin = a < kmin ? a : kmin;
+    kmax = b > kmax ? b : kmax;
+  }
+  if (kmin == kmax) return kmin;
+  const int top = 63 - __clzll(static_cast<long long>(kmin ^ kmax));  // highest differing bit
+  int shift = (top / 8) * 8;
+  unsigned long long prefix = shift + 8 >= 64 ? 0ull : (kmin & (~0ull << (shift + 8)));
+  for (; shift >= 0; shift -= 8) {
     for (int b = lane; b < 256; b += 32) hist[b] = 0;
     __syncwarp();
-    const unsigned long long hmask = shift == 56 ? 0ull : (~0ull << (shift + 8));
+    const unsigned long long hmask = shift + 8 >= 64 ? 0ull : (~0ull << (shift + 8));
     for (int e = lane; e < count; e += 32) {
       const unsigned long long key = __ldcg(keys + e);
       if ((key & hmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
@@ -395,10 +415,9 @@ __device__ unsigned long long warp_select_kth(const unsigned long long* keys, in
     }
     const unsigned int excl = incl - tot;
     const bool mine = excl < static_cast<unsigned int>(kth) && static_cast<unsigned int>(kth) <= incl;
-    const unsigned int ball = __ballot_sync(0xffffffffu, mine);
-    const int src = __ffs(ball) - 1;
+    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
     int digit = 0;
-    unsigned int before = 0;
+    unsigned int before = 0, in_bin = 0;
     if (mine) {
       unsigned int acc = excl;
 #pragma unroll
@@ -406,6 +425,7 @@ __device__ unsigned long long warp_select_kth(const unsigned long long* keys, in
         if (acc + local[j] >= static_cast<unsigned int>(kth)) {
           digit = 8 * lane + j;
           before = acc;
+          in_bin = local[j];
           break;
         }
         acc += local[j];
@@ -413,9 +433,25 @@ __device__ unsigned long long warp_select_kth(const unsigned long long* keys, in
     }
     digit = __shfl_sync(0xffffffffu, digit, src);
     before = __shfl_sync(0xffffffffu, before, src);
+    in_bin = __shfl_sync(0xffffffffu, in_bin, src);
     kth -= static_cast<int>(before);
     prefix |= static_cast<unsigned long long>(digit) << shift;
     __syncwarp();
+    if (in_bin == 1 || shift == 0) {
+      // the kth key is the only key with this prefix: fetch it
+      const unsigned long long pmask = ~0ull << shift;
+      unsigned long long found = ~0ull;
+      for (int e = lane; e < count; e += 32) {
+        const unsigned long long key = __ldcg(keys + e);
+        if ((key & pmask) == prefix) found = key;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long y = __shfl_xor_sync(0xffffffffu, found, o);
+        found = y < found ? y : found;
+      }
+      return found;
+    }
   }
   return prefix;
 }
@@ -423,6 +459,7 @@ __device__ unsigned long long warp_select_kth(const unsigned long long* keys, in
 __global__ void fill_init_kernel(FillArgs a) {
   const size_t items = static_cast<size_t>(a.heads) * a.n;
   const size_t groups = static_cast<size_t>(a.heads) * a.G;
+  const size_t words = static_cast<size_t>(a.heads) * ((a.G + 31) / 32);
   for (size_t x = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; x < items;
        x += static_cast<size_t>(gridDim.x) * blockDim.x) {
     a.labels[x] = -1;
@@ -434,6 +471,9 @@ __global__ void fill_init_kernel(FillArgs a) {
     a.cnt[x] = 0;
     a.cursor[x] = 0;
   }
+  for (size_t x = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; x < words;
+       x += static_cast<size_t>(gridDim.x) * blockDim.x)
+    a.closed[x] = 0u;
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     a.list_len[0] = static_cast<int>(items);
     a.list_len[1] = 0;
@@ -452,6 +492,7 @@ __global__ void __launch_bounds__(kFillThreads) fill_coop_kernel(FillArgs a) {
   const int gwarp = gthread >> 5;
   const int nwarps = nthreads >> 5;
   const int n = a.n, G = a.G;
+  const int words = (G + 31) / 32;
   int* lists[2] = {a.list0, a.list1};
   int cur = 0;
   const int max_rounds = n + 2;
@@ -473,15 +514,26 @@ __global__ void __launch_bounds__(kFillThreads) fill_coop_kernel(FillArgs a) {
         const int item = __ldcg(L + x);
         const int h = item / n;
         const float* drow = a.D + static_cast<size_t>(item) * G;
-        const int* room = a.room + static_cast<size_t>(h) * G;
+        const unsigned int* closed = a.closed + static_cast<size_t>(h) * words;
         unsigned long long best = ~0ull;
         bool saw_nan = false;
-        for (int g = lane; g < G; g += 32) {
-          if (__ldcg(room + g) > 0) {
-            const float v = __ldcg(drow + g);
-            saw_nan |= (v != v);
-            const unsigned long long key = decision_key(v, g);
-            best = key < best ? key : best;
+        for (int w0 = 0; w0 < words; w0 += 4) {
+          float v[4];
+          unsigned int cw[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int g = (w0 + u) * 32 + lane;
+            cw[u] = w0 + u < words ? __ldcg(closed + w0 + u) : ~0u;
+            v[u] = g < G ? __ldcg(drow + g) : 0.f;
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int g = (w0 + u) * 32 + lane;
+            if (g < G && !((cw[u] >> lane) & 1u)) {
+              saw_nan |= (v[u] != v[u]);
+              const unsigned long long key = decision_key(v[u], g);
+              best = key < best ? key : best;
+            }
           }
         }
         best = warp_min_u64(best);
@@ -492,9 +544,8 @@ __global__ void __launch_bounds__(kFillThreads) fill_coop_kernel(FillArgs a) {
             record_error(&a.hdr->status, kErrInvalidArg);
           } else {
             const int g = static_cast<int>(best & 0xffffffffu);
-            const float v = __ldcg(drow + g);
             a.prop_g[item] = g;
-            a.prop_v[item] = v;
+            a.prop_v[item] = __ldcg(drow + g);
             atomicAdd(a.cnt + static_cast<size_t>(h) * G + g, 1);
           }
         }
@@ -562,9 +613,11 @@ __global__ void __launch_bounds__(kFillThreads) fill_coop_kernel(FillArgs a) {
       }
       __syncwarp();
       if (lane == 0) {
-        a.room[x] = r - min(c, r);
+        const int left = r - min(c, r);
+        a.room[x] = left;
         a.cnt[x] = 0;
         a.cursor[x] = 0;
+        if (left == 0) atomicOr(a.closed + static_cast<size_t>(h) * words + g / 32, 1u << (g % 32));
       }
     }
     if (!grid_barrier(a.hdr, nblocks)) return;
@@ -742,7 +795,7 @@ cudaError_t launch_fill(const FillArgs& a, cudaStream_t st) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fill_coop_kernel, kFillThreads, 0);
   if (e != cudaSuccess) return e;
-  const int blocks = sms * std::min(per_sm, 2);
+  const int blocks = sms * std::min(per_sm, 4);
   FillArgs args = a;
   void* params[] = {&args};
   e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(fill_coop_kernel), dim3(blocks), dim3(kFillThreads),

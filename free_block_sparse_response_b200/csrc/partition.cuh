@@ -36,6 +36,7 @@ struct FillArgs {
   int* cnt;
   int* offs;
   int* cursor;
+  unsigned int* closed;  // [heads, ceil(G/32)] bit g set once group g is full
   unsigned long long* bucket;  // [heads, n]
   int* list0;           // [heads * n]
   int* list1;
