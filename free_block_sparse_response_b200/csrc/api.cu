@@ -75,7 +75,7 @@ Layout make_layout(int heads, int N, int d, int block, int S, int P) {
   L.whi = take(2 * H * G * D);
   L.wlo = take(2 * H * G * D);
   L.eg = take(sizeof(float) * H * G);
-  L.dmat = take(sizeof(float) * H * n * G);
+  L.dmat = take(sizeof(float) * H * n * ((G + 3) / 4 * 4));
   L.prop_g0 = take(sizeof(int) * H * n);
   L.prop_v0 = take(sizeof(float) * H * n);
   L.labels = take(sizeof(int) * H * n);
@@ -202,6 +202,7 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
   float* dmat = at<float>(ws, L.dmat);
   spr::FillArgs fa{};
   fa.D = dmat;
+  fa.ldd = (G + 3) / 4 * 4;
   fa.prop_g0 = at<int>(ws, L.prop_g0);
   fa.prop_v0 = at<float>(ws, L.prop_v0);
   fa.heads = heads;
@@ -250,6 +251,7 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
       ra.ecol = eg;
       ra.tau2 = tau * tau;
       ra.Dout = dmat;
+      ra.ldd = fa.ldd;
       ra.prop_g = at<int>(ws, L.prop_g0);
       ra.prop_v = at<float>(ws, L.prop_v0);
       ra.nrm_out = nullptr;
@@ -475,6 +477,7 @@ int sparsepr_test_fill(const float* D, int32_t H, int32_t n, int32_t G, int32_t 
   };
   spr::FillArgs fa{};
   fa.D = D;
+  fa.ldd = G;
   fa.prop_g0 = nullptr;
   fa.prop_v0 = nullptr;
   fa.heads = H;

@@ -166,7 +166,7 @@ template <int D, bool DIST, bool SPLIT>
 __global__ void __launch_bounds__(256)
     rowgemm_mma_kernel(const __nv_bfloat16* __restrict__ X, int n, const __nv_bfloat16* __restrict__ Bhi,
                        const __nv_bfloat16* __restrict__ Blo, int ncols, const float* __restrict__ nrm,
-                       const float* __restrict__ ecol, float tau2, float* __restrict__ Dout,
+                       const float* __restrict__ ecol, float tau2, float* __restrict__ Dout, int ldd,
                        int* __restrict__ prop_g, float* __restrict__ prop_v, float* __restrict__ nrm_out,
                        int* __restrict__ status) {
   constexpr int kCh = D / 8;
@@ -274,11 +274,11 @@ __global__ void __launch_bounds__(256)
       for (int h = 0; h < 2; ++h) {
         const int row = row0 + rloc[h];
         if (row >= n) continue;
-        float* drow = Dout + (static_cast<size_t>(head) * n + row) * ncols;
+        float* drow = Dout + (static_cast<size_t>(head) * n + row) * ldd;
 #pragma unroll
         for (int nt = 0; nt < kGemmCols / 8; ++nt) {
           const int col = t * kGemmCols + nt * 8 + 2 * t4;
-          if (col + 1 < ncols && (ncols % 2 == 0)) {
+          if (col + 1 < ncols && (ldd % 2 == 0)) {
             *reinterpret_cast<float2*>(drow + col) = make_float2(acc[nt][2 * h], acc[nt][2 * h + 1]);
           } else {
             if (col < ncols) drow[col] = acc[nt][2 * h];
@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(256)
         const size_t o = static_cast<size_t>(head) * n + row;
         const int col = static_cast<int>(b & 0xffffffffu);
         prop_g[o] = col;
-        prop_v[o] = Dout[o * ncols + col];
+        prop_v[o] = Dout[o * ldd + col];
       }
     } else {
       float p = part[h];
@@ -320,7 +320,7 @@ template <int D, bool DIST>
 __global__ void __launch_bounds__(256)
     rowgemm_f32_kernel(const float* __restrict__ X, int n, const float* __restrict__ B, int ncols,
                        const float* __restrict__ nrm, const float* __restrict__ ecol, float tau2,
-                       float* __restrict__ Dout, int* __restrict__ prop_g, float* __restrict__ prop_v,
+                       float* __restrict__ Dout, int ldd, int* __restrict__ prop_g, float* __restrict__ prop_v,
                        float* __restrict__ nrm_out, int* __restrict__ status) {
   const int head = blockIdx.y;
   const int lane = threadIdx.x & 31;
@@ -341,7 +341,7 @@ __global__ void __launch_bounds__(256)
     dot = warp_sum(dot);
     if (DIST) {
       const float v = tau2 * (nrm[static_cast<size_t>(head) * n + row] - 2.f * dot + ecol[static_cast<size_t>(head) * ncols + c]);
-      if (lane == 0) Dout[(static_cast<size_t>(head) * n + row) * ncols + c] = v;
+      if (lane == 0) Dout[(static_cast<size_t>(head) * n + row) * ldd + c] = v;
       saw_nan |= (v != v);
       const unsigned long long key = decision_key(v, c);
       best = key < best ? key : best;
@@ -354,7 +354,7 @@ __global__ void __launch_bounds__(256)
     if (DIST) {
       const int col = static_cast<int>(best & 0xffffffffu);
       prop_g[o] = col;
-      prop_v[o] = Dout[o * ncols + col];
+      prop_v[o] = Dout[o * ldd + col];
       if (saw_nan) record_error(status, kErrNonFinite);
     } else {
       nrm_out[o] = nsum;
@@ -513,7 +513,7 @@ __global__ void __launch_bounds__(kFillThreads) fill_coop_kernel(FillArgs a) {
       for (int x = gwarp; x < ncur; x += nwarps) {
         const int item = __ldcg(L + x);
         const int h = item / n;
-        const float* drow = a.D + static_cast<size_t>(item) * G;
+        const float* drow = a.D + static_cast<size_t>(item) * a.ldd;
         const unsigned int* closed = a.closed + static_cast<size_t>(h) * words;
         unsigned long long best = ~0ull;
         bool saw_nan = false;
@@ -757,7 +757,7 @@ static cudaError_t launch_rowgemm_mma_t(const RowGemmArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   kern<<<dim3(ceil_div(a.n, kGemmRows), a.heads), 256, smem, st>>>(
-      static_cast<const __nv_bfloat16*>(a.X), a.n, a.Bhi, a.Blo, a.ncols, a.nrm, a.ecol, a.tau2, a.Dout,
+      static_cast<const __nv_bfloat16*>(a.X), a.n, a.Bhi, a.Blo, a.ncols, a.nrm, a.ecol, a.tau2, a.Dout, a.ldd,
       a.prop_g, a.prop_v, a.nrm_out, a.status);
   return counted(cudaGetLastError(), 1);
 }
@@ -767,15 +767,16 @@ cudaError_t launch_rowgemm(const RowGemmArgs& a, bool dist, cudaStream_t st) {
     dim3 grid(ceil_div(a.n, 8), a.heads);
     const float* X = static_cast<const float*>(a.X);
     if (a.d == 64) {
-      if (dist) rowgemm_f32_kernel<64, true><<<grid, 256, 0, st>>>(X, a.n, a.Bf32, a.ncols, a.nrm, a.ecol, a.tau2, a.Dout, a.prop_g, a.prop_v, a.nrm_out, a.status);
-      else rowgemm_f32_kernel<64, false><<<grid, 256, 0, st>>>(X, a.n, a.Bf32, a.ncols, a.nrm, a.ecol, a.tau2, a.Dout, a.prop_g, a.prop_v, a.nrm_out, a.status);
+      if (dist) rowgemm_f32_kernel<64, true><<<grid, 256, 0, st>>>(X, a.n, a.Bf32, a.ncols, a.nrm, a.ecol, a.tau2, a.Dout, a.ldd, a.prop_g, a.prop_v, a.nrm_out, a.status);
+      else rowgemm_f32_kernel<64, false><<<grid, 256, 0, st>>>(X, a.n, a.Bf32, a.ncols, a.nrm, a.ecol, a.tau2, a.Dout, a.ldd, a.prop_g, a.prop_v, a.nrm_out, a.status);
     } else {
-      if (dist) rowgemm_f32_kernel<128, true><<<grid, 256, 0, st>>>(X, a.n, a.Bf32, a.ncols, a.nrm, a.ecol, a.tau2, a.Dout, a.prop_g, a.prop_v, a.nrm_out, a.status);
-      else rowgemm_f32_kernel<128, false><<<grid, 256, 0, st>>>(X, a.n, a.Bf32, a.ncols, a.nrm, a.ecol, a.tau2, a.Dout, a.prop_g, a.prop_v, a.nrm_out, a.status);
+      if (dist) rowgemm_f32_kernel<128, true><<<grid, 256, 0, st>>>(X, a.n, a.Bf32, a.ncols, a.nrm, a.ecol, a.tau2, a.Dout, a.ldd, a.prop_g, a.prop_v, a.nrm_out, a.status);
+      else rowgemm_f32_kernel<128, false><<<grid, 256, 0, st>>>(X, a.n, a.Bf32, a.ncols, a.nrm, a.ecol, a.tau2, a.Dout, a.ldd, a.prop_g, a.prop_v, a.nrm_out, a.status);
     }
     return counted(cudaGetLastError(), 1);
   }
   const bool split = a.Blo != nullptr;
+  if (dist && a.d == 128) return launch_dist_tc(a, a.ldd, st);
   if (a.d == 64) {
     if (dist) return split ? launch_rowgemm_mma_t<64, true, true>(a, st) : launch_rowgemm_mma_t<64, true, false>(a, st);
     return split ? launch_rowgemm_mma_t<64, false, true>(a, st) : launch_rowgemm_mma_t<64, false, false>(a, st);

@@ -19,7 +19,8 @@ struct RowGemmArgs {
   const float* nrm;          // DIST: [heads, n]
   const float* ecol;         // DIST: [heads, ncols]
   float tau2;
-  float* Dout;               // DIST: [heads, n, ncols]
+  float* Dout;               // DIST: [heads, n, ldd]
+  int ldd;                   // DIST: row stride of Dout (>= ncols)
   int* prop_g;               // DIST: [heads, n]
   float* prop_v;
   float* nrm_out;            // NORM: [heads, n]
@@ -27,7 +28,8 @@ struct RowGemmArgs {
 };
 
 struct FillArgs {
-  const float* D;       // [heads, n, G]
+  const float* D;       // [heads, n, ldd]
+  int ldd;              // row stride of D (>= G)
   const int* prop_g0;   // optional first proposals [heads, n]
   const float* prop_v0;
   int heads, n, G, cap;
@@ -57,6 +59,7 @@ cudaError_t launch_centroid(const void* X, bool f32, int n, const int* perm, con
 cudaError_t launch_wmat(const float* cent, const float* gamma, int G, int heads, int d, float* wf,
                         __nv_bfloat16* whi, __nv_bfloat16* wlo, float* eg, cudaStream_t st);
 cudaError_t launch_rowgemm(const RowGemmArgs& a, bool dist, cudaStream_t st);
+cudaError_t launch_dist_tc(const RowGemmArgs& a, int ldd, cudaStream_t st);
 cudaError_t launch_fill(const FillArgs& a, cudaStream_t st);
 cudaError_t launch_build_perm(const int* labels, int n, int G, int cap, int heads, int* cursor, int* tmp,
                               int* perm, int* sizes, int* status, cudaStream_t st);
