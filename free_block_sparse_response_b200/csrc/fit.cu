@@ -46,6 +46,7 @@ __global__ void __launch_bounds__(kFitThreads)
   double* C = sm;                          // D x LD
   double* w = C + D * LD;                  // P
   double* stage = w + P;                   // kStageRows x D
+  float* Vt = reinterpret_cast<float*>(stage + kStageRows * D);  // D x D eigenvectors (rows), fp32
   __shared__ double red[kFitThreads / 32];
   __shared__ double pc[D / 2], ps[D / 2];
   __shared__ int pp[D / 2], pq[D / 2], order[D];
@@ -55,8 +56,7 @@ __global__ void __launch_bounds__(kFitThreads)
   const int head = blockIdx.x, tid = threadIdx.x;
   const float* xs = xs_all + static_cast<size_t>(head) * P * D;
   const float* dp = dp_all + static_cast<size_t>(head) * P * D;
-  double* Vt = scratch + static_cast<size_t>(head) * fit_scratch_doubles(P, D);
-  double* Z = Vt + D * D;                  // P x R
+  double* Z = scratch + static_cast<size_t>(head) * fit_scratch_doubles(P, D) + D * D;  // P x R
   double* A = Z + static_cast<size_t>(P) * D;  // R x D
   if (tid == 0) s_fail = 0;
 
@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kFitThreads)
     const int ij = tid + x * kFitThreads;
     C[(ij / D) * LD + ij % D] = acc[x];
   }
-  for (int x = tid; x < D * D; x += kFitThreads) Vt[x] = (x / D == x % D) ? 1.0 : 0.0;
+  for (int x = tid; x < D * D; x += kFitThreads) Vt[x] = (x / D == x % D) ? 1.f : 0.f;
   __syncthreads();
 
   // ---- Jacobi, round-robin parallel ordering
@@ -126,7 +126,12 @@ __global__ void __launch_bounds__(kFitThreads)
     total += v * v;
   }
   total = block_sum_d(total, red);
-  const double tol2 = 1e-28 * total;
+  const double tol2 = 1e-20 * total;  // stop at off-diagonal norm <= 1e-10 |C|
+  if (tid < D / 2) {
+    pp[tid] = 0;
+    pq[tid] = 0;
+    ps[tid] = 0.0;
+  }
   for (int sweep = 0; sweep < 40; ++sweep) {
     double off = 0.0;
     for (int x = tid; x < D * D; x += kFitThreads) {
@@ -140,6 +145,11 @@ __global__ void __launch_bounds__(kFitThreads)
     if (off <= tol2 || total == 0.0) break;
     for (int round = 0; round < D - 1; ++round) {
       if (tid < D / 2) {
+        // the previous round's pair of this slot was annihilated: store exact zeros
+        if (ps[tid] != 0.0) {
+          C[pp[tid] * LD + pq[tid]] = 0.0;
+          C[pq[tid] * LD + pp[tid]] = 0.0;
+        }
         int p, q;
         if (tid == 0) {
           p = round;
@@ -154,51 +164,55 @@ __global__ void __launch_bounds__(kFitThreads)
           q = t;
         }
         const double apq = C[p * LD + q];
-        double c = 1.0, s = 0.0;
-        if (apq != 0.0 && apq * apq > 1e-36 * total) {
-          const double theta = (C[q * LD + q] - C[p * LD + p]) / (2.0 * apq);
+        const double app = C[p * LD + p], aqq = C[q * LD + q];
+        double c = 1.0, sn = 0.0;
+        if (apq != 0.0 && apq * apq > 1e-30 * fabs(app * aqq) && apq * apq > 1e-36 * total) {
+          const double theta = (aqq - app) / (2.0 * apq);
           const double t = (theta >= 0.0 ? 1.0 : -1.0) / (fabs(theta) + sqrt(theta * theta + 1.0));
           c = 1.0 / sqrt(t * t + 1.0);
-          s = t * c;
+          sn = t * c;
         }
         pp[tid] = p;
         pq[tid] = q;
         pc[tid] = c;
-        ps[tid] = s;
+        ps[tid] = sn;
       }
       __syncthreads();
       for (int x = tid; x < (D / 2) * D; x += kFitThreads) {  // rows: J^T C, and V^T rows
         const int t = x / D, j = x % D;
-        const int p = pp[t], q = pq[t];
-        const double c = pc[t], s = ps[t];
-        if (s != 0.0) {
+        const double sn = ps[t];
+        if (sn != 0.0) {
+          const int p = pp[t], q = pq[t];
+          const double c = pc[t];
           const double cp = C[p * LD + j], cq = C[q * LD + j];
-          C[p * LD + j] = c * cp - s * cq;
-          C[q * LD + j] = s * cp + c * cq;
-          const double vp = Vt[p * D + j], vq = Vt[q * D + j];
-          Vt[p * D + j] = c * vp - s * vq;
-          Vt[q * D + j] = s * vp + c * vq;
+          C[p * LD + j] = c * cp - sn * cq;
+          C[q * LD + j] = sn * cp + c * cq;
+          const float cf = static_cast<float>(c), sf = static_cast<float>(sn);
+          const float vp = Vt[p * D + j], vq = Vt[q * D + j];
+          Vt[p * D + j] = cf * vp - sf * vq;
+          Vt[q * D + j] = sf * vp + cf * vq;
         }
       }
       __syncthreads();
       for (int x = tid; x < (D / 2) * D; x += kFitThreads) {  // columns: (J^T C) J
         const int t = x % (D / 2), i = x / (D / 2);
-        const int p = pp[t], q = pq[t];
-        const double c = pc[t], s = ps[t];
-        if (s != 0.0) {
+        const double sn = ps[t];
+        if (sn != 0.0) {
+          const int p = pp[t], q = pq[t];
+          const double c = pc[t];
           const double cp = C[i * LD + p], cq = C[i * LD + q];
-          C[i * LD + p] = c * cp - s * cq;
-          C[i * LD + q] = s * cp + c * cq;
+          C[i * LD + p] = c * cp - sn * cq;
+          C[i * LD + q] = sn * cp + c * cq;
         }
-      }
-      __syncthreads();
-      if (tid < D / 2 && ps[tid] != 0.0) {
-        C[pp[tid] * LD + pq[tid]] = 0.0;
-        C[pq[tid] * LD + pp[tid]] = 0.0;
       }
       __syncthreads();
     }
   }
+  if (tid < D / 2 && ps[tid] != 0.0) {
+    C[pp[tid] * LD + pq[tid]] = 0.0;
+    C[pq[tid] * LD + pp[tid]] = 0.0;
+  }
+  __syncthreads();
   // ---- eigenvalues descending (stable on ties)
   for (int i = tid; i < D; i += kFitThreads) {
     const double li = C[i * LD + i];
@@ -214,7 +228,7 @@ __global__ void __launch_bounds__(kFitThreads)
   // ---- z_p = U_r^T y_p ; weighted means
   for (int x = tid; x < P * R; x += kFitThreads) {
     const int p = x / R, a = x % R;
-    const double* u = Vt + static_cast<size_t>(order[a]) * D;
+    const float* u = Vt + static_cast<size_t>(order[a]) * D;
     double s = 0.0;
     for (int e = 0; e < D; ++e)
       s += u[e] * (static_cast<double>(dp[static_cast<size_t>(p) * D + e]) -
@@ -326,44 +340,86 @@ __global__ void __launch_bounds__(kFitThreads)
   for (int x = tid; x < D * D; x += kFitThreads) {
     const int i = x / D, j = x % D;
     double s = 0.0;
-    for (int a = 0; a < R; ++a) s += Vt[static_cast<size_t>(order[a]) * D + i] * A[static_cast<size_t>(a) * D + j];
+    for (int a = 0; a < R; ++a)
+      s += static_cast<double>(Vt[static_cast<size_t>(order[a]) * D + i]) * A[static_cast<size_t>(a) * D + j];
     M_out[static_cast<size_t>(head) * D * D + x] = failed ? 0.f : static_cast<float>(s);
   }
   for (int i = tid; i < D; i += kFitThreads) {
     double s = 0.0;
-    for (int a = 0; a < R; ++a) s += Vt[static_cast<size_t>(order[a]) * D + i] * bvec[a];
+    for (int a = 0; a < R; ++a) s += static_cast<double>(Vt[static_cast<size_t>(order[a]) * D + i]) * bvec[a];
     beta_out[static_cast<size_t>(head) * D + i] = failed ? 0.f : static_cast<float>(s);
   }
   if (failed && tid == 0) record_error(status, kErrInvalidArg);
 }
 
-// O = S + S M^T + beta, 32 rows per CTA; M^T and the rows staged in shared memory.
+// O = S + S M^T + beta.  CTA: 8 tiles of 64 rows (M^T staged once), 256 threads; thread
+// (ty, tx) computes rows 4 ty .. 4 ty + 3 and columns (D / 16) tx .. + D / 16 of a tile
+// (register tiling: 4 + D/16 shared loads per 4 D/16 FMAs).  M^T rows are padded by 4
+// floats so the staging transpose and the vector reads avoid most bank conflicts.
+constexpr int kApplyTile = 64;
+constexpr int kApplyTiles = 8;
+
 template <int D, typename TO>
 __global__ void __launch_bounds__(256)
     apply_kernel(const float* __restrict__ S, const float* __restrict__ M, const float* __restrict__ beta, int N,
                  TO* __restrict__ O) {
-  constexpr int kRows = 32;
-  extern __shared__ float fsm[];
-  float* Mt = fsm;               // [e][j] = M[j][e]
-  float* rows = Mt + D * D;      // kRows x D
-  const int head = blockIdx.y, row0 = blockIdx.x * kRows, tid = threadIdx.x;
+  constexpr int kCols = D / 16;  // columns per thread: 8 (D = 128) or 4 (D = 64)
+  constexpr int LDM = D + 4;
+  extern __shared__ __align__(16) float fsm[];
+  float* Mt = fsm;                // [e][j] = M[j][e], row stride LDM
+  float* rows = Mt + D * LDM;     // kApplyTile x D
+  const int head = blockIdx.y, tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
   const float* m = M + static_cast<size_t>(head) * D * D;
-  for (int x = tid; x < D * D; x += 256) Mt[(x % D) * D + x / D] = m[x];
+  for (int x = tid; x < D * D; x += 256) Mt[(x % D) * LDM + x / D] = m[x];
   const float* s = S + static_cast<size_t>(head) * N * D;
-  for (int x = tid; x < kRows * D; x += 256) {
-    const int r = row0 + x / D;
-    rows[x] = r < N ? s[static_cast<size_t>(r) * D + x % D] : 0.f;
-  }
-  __syncthreads();
-  const int j = tid % D;
-  const float bj = beta[static_cast<size_t>(head) * D + j];
-  for (int r = tid / D; r < kRows; r += 256 / D) {
-    if (row0 + r >= N) break;
-    const float* sr = rows + r * D;
-    float acc = sr[j] + bj;
-#pragma unroll 8
-    for (int e = 0; e < D; ++e) acc += sr[e] * Mt[e * D + j];
-    O[(static_cast<size_t>(head) * N + row0 + r) * D + j] = from_f32<TO>(acc);
+  float bt[kCols];
+#pragma unroll
+  for (int c = 0; c < kCols; ++c) bt[c] = beta[static_cast<size_t>(head) * D + tx * kCols + c];
+  for (int tile = 0; tile < kApplyTiles; ++tile) {
+    const int row0 = (blockIdx.x * kApplyTiles + tile) * kApplyTile;
+    if (row0 >= N) break;
+    __syncthreads();  // previous tile's reads of `rows` are done (and Mt is staged)
+    for (int x = tid * 4; x < kApplyTile * D; x += 256 * 4) {
+      const int r = row0 + x / D;
+      const float4 v = r < N ? *reinterpret_cast<const float4*>(s + static_cast<size_t>(r) * D + x % D)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(rows + x) = v;
+    }
+    __syncthreads();
+    float acc[4][kCols];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int c = 0; c < kCols; ++c) acc[i][c] = rows[(ty * 4 + i) * D + tx * kCols + c] + bt[c];
+    }
+#pragma unroll 4
+    for (int e = 0; e < D; ++e) {
+      float sv[4], mv[kCols];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sv[i] = rows[(ty * 4 + i) * D + e];
+#pragma unroll
+      for (int c = 0; c < kCols; c += 4) {
+        const float4 q = *reinterpret_cast<const float4*>(Mt + e * LDM + tx * kCols + c);
+        mv[c] = q.x;
+        mv[c + 1] = q.y;
+        mv[c + 2] = q.z;
+        mv[c + 3] = q.w;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int c = 0; c < kCols; ++c) acc[i][c] = fmaf(sv[i], mv[c], acc[i][c]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = row0 + ty * 4 + i;
+      if (r >= N) break;
+      TO* dst = O + (static_cast<size_t>(head) * N + r) * D + tx * kCols;
+#pragma unroll
+      for (int c = 0; c < kCols; ++c) dst[c] = from_f32<TO>(acc[i][c]);
+    }
   }
 }
 
@@ -419,7 +475,7 @@ cudaError_t launch_fit(const float* xs, const float* dp, const float* weights, i
                        double lambda, int rank, int weight_mode, double* scratch, float* M, float* beta,
                        int* status, cudaStream_t st) {
   const int R = rank < d ? rank : d;
-  const size_t smem = (static_cast<size_t>(d) * (d + 1) + P + kStageRows * d) * sizeof(double);
+  const size_t smem = fit_smem_bytes(d, P);
   if (d == 64) {
     cudaError_t e = cudaFuncSetAttribute(fit_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
@@ -433,16 +489,17 @@ cudaError_t launch_fit(const float* xs, const float* dp, const float* weights, i
 }
 
 size_t fit_smem_bytes(int d, int P) {
-  return (static_cast<size_t>(d) * (d + 1) + P + kStageRows * d) * sizeof(double);
+  return (static_cast<size_t>(d) * (d + 1) + P + kStageRows * d) * sizeof(double) +
+         static_cast<size_t>(d) * d * sizeof(float);
 }
 
 template <int D, typename TO>
 static cudaError_t launch_apply_t(const float* S, const float* M, const float* beta, const int* probe_idx,
                                   const float* probe_out, int heads, int N, int P, TO* O, cudaStream_t st) {
-  const size_t smem = (static_cast<size_t>(D) * D + 32 * D) * sizeof(float);
+  const size_t smem = (static_cast<size_t>(D) * (D + 4) + kApplyTile * D) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(apply_kernel<D, TO>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  apply_kernel<D, TO><<<dim3(ceil_div(N, 32), heads), 256, smem, st>>>(S, M, beta, N, O);
+  apply_kernel<D, TO><<<dim3(ceil_div(N, kApplyTile * kApplyTiles), heads), 256, smem, st>>>(S, M, beta, N, O);
   e = counted(cudaGetLastError(), 1);
   if (e != cudaSuccess || P == 0) return e;
   probe_overwrite_kernel<D, TO><<<dim3(P, heads), D, 0, st>>>(probe_idx, probe_out, N, P, O);
