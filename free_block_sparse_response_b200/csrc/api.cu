@@ -177,6 +177,8 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
     return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
   if (p->n_sampled < 1 || p->n_sampled > N) return fail(SPARSEPR_ERR_INVALID_ARG, "n_sampled must be in [1, N]");
   if (p->kmeans_iters < 0 || p->kmeans_iters > 64) return fail(SPARSEPR_ERR_INVALID_ARG, "kmeans_iters must be in [0, 64]");
+  if (spr::ceil_div(N, p->block) > 1024)
+    return fail(SPARSEPR_ERR_UNSUPPORTED, "more than 1024 groups per head (N / block) is not built");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int heads = Bt * H, B = p->block, G = spr::ceil_div(N, B), S = p->n_sampled;
   const bool f32 = dtype == SPARSEPR_F32;
@@ -467,6 +469,7 @@ int sparsepr_test_fill(const float* D, int32_t H, int32_t n, int32_t G, int32_t 
   if (!D || !labels || !ws || H < 1 || n < 1 || G < 1 || cap < 1)
     return fail(SPARSEPR_ERR_INVALID_ARG, "bad fill arguments");
   if (static_cast<long long>(G) * cap < n) return fail(SPARSEPR_ERR_INVALID_ARG, "G * cap < n");
+  if (G > 1024) return fail(SPARSEPR_ERR_UNSUPPORTED, "more than 1024 groups is not built");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const size_t h = H, nn = n, g = G;
   size_t off = align_up(sizeof(spr::WorkspaceHeader));

@@ -375,10 +375,20 @@ __device__ unsigned long long warp_select_kth(const unsigned long long* keys, in
                                               unsigned int* hist) {
   const int lane = threadIdx.x & 31;
   unsigned long long kmin = ~0ull, kmax = 0ull;
-  for (int e = lane; e < count; e += 32) {
-    const unsigned long long key = __ldcg(keys + e);
-    kmin = key < kmin ? key : kmin;
-    kmax = key > kmax ? key : kmax;
+  for (int e0 = 0; e0 < count; e0 += 256) {
+    unsigned long long kb[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int e = e0 + u * 32 + lane;
+      kb[u] = e < count ? __ldcg(keys + e) : 0ull;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (e0 + u * 32 + lane < count) {
+        kmin = kb[u] < kmin ? kb[u] : kmin;
+        kmax = kb[u] > kmax ? kb[u] : kmax;
+      }
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -395,9 +405,17 @@ __device__ unsigned long long warp_select_kth(const unsigned long long* keys, in
     for (int b = lane; b < 256; b += 32) hist[b] = 0;
     __syncwarp();
     const unsigned long long hmask = shift + 8 >= 64 ? 0ull : (~0ull << (shift + 8));
-    for (int e = lane; e < count; e += 32) {
-      const unsigned long long key = __ldcg(keys + e);
-      if ((key & hmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    for (int e0 = 0; e0 < count; e0 += 256) {
+      unsigned long long kb[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int e = e0 + u * 32 + lane;
+        kb[u] = e < count ? __ldcg(keys + e) : ~0ull;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (e0 + u * 32 + lane < count && (kb[u] & hmask) == prefix) atomicAdd(&hist[(kb[u] >> shift) & 255u], 1u);
+      }
     }
     __syncwarp();
     unsigned int local[8];
@@ -441,9 +459,17 @@ __device__ unsigned long long warp_select_kth(const unsigned long long* keys, in
       // the kth key is the only key with this prefix: fetch it
       const unsigned long long pmask = ~0ull << shift;
       unsigned long long found = ~0ull;
-      for (int e = lane; e < count; e += 32) {
-        const unsigned long long key = __ldcg(keys + e);
-        if ((key & pmask) == prefix) found = key;
+      for (int e0 = 0; e0 < count; e0 += 256) {
+        unsigned long long kb[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int e = e0 + u * 32 + lane;
+          kb[u] = e < count ? __ldcg(keys + e) : ~0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (e0 + u * 32 + lane < count && (kb[u] & pmask) == prefix) found = kb[u];
+        }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
@@ -481,10 +507,14 @@ __global__ void fill_init_kernel(FillArgs a) {
 }
 
 constexpr int kFillThreads = 256;
+constexpr size_t kFillStageLimit = 64 * 1024;  // bytes of full-group bitmaps staged per block
 
-__global__ void __launch_bounds__(kFillThreads) fill_coop_kernel(FillArgs a) {
+// MAXW = 32-group words of a distance row held per lane (G <= 32 MAXW).
+template <int MAXW>
+__global__ void __launch_bounds__(kFillThreads, 3) fill_coop_kernel(FillArgs a) {
   __shared__ unsigned int hist[kFillThreads / 32][256];
   __shared__ int scan_tmp[kFillThreads];
+  extern __shared__ unsigned int s_closed[];  // [heads * words] when a.stage_closed
   const unsigned int nblocks = gridDim.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gthread = blockIdx.x * kFillThreads + tid;
@@ -510,30 +540,36 @@ __global__ void __launch_bounds__(kFillThreads) fill_coop_kernel(FillArgs a) {
         atomicAdd(a.cnt + static_cast<size_t>(h) * G + g, 1);
       }
     } else {
+      // The full-group bitmaps of all heads are staged in shared memory once per round
+      // (when they fit), so a proposal waits only for its own distance row.
+      const unsigned int* closed_all = a.closed;
+      if (a.stage_closed) {
+        for (int x = tid; x < a.heads * words; x += kFillThreads) s_closed[x] = __ldcg(a.closed + x);
+        __syncthreads();
+        closed_all = s_closed;
+      }
+      // One item per warp, with the item's whole distance row (up to MAXW values per
+      // lane) requested before any is used; full-group bitmap words are warp-uniform.
       for (int x = gwarp; x < ncur; x += nwarps) {
         const int item = __ldcg(L + x);
         const int h = item / n;
         const float* drow = a.D + static_cast<size_t>(item) * a.ldd;
-        const unsigned int* closed = a.closed + static_cast<size_t>(h) * words;
+        const unsigned int* closed = closed_all + static_cast<size_t>(h) * words;
+        float v[MAXW];
+#pragma unroll
+        for (int u = 0; u < MAXW; ++u) {
+          const int g = u * 32 + lane;
+          v[u] = g < G ? __ldcg(drow + g) : 0.f;
+        }
         unsigned long long best = ~0ull;
         bool saw_nan = false;
-        for (int w0 = 0; w0 < words; w0 += 4) {
-          float v[4];
-          unsigned int cw[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int g = (w0 + u) * 32 + lane;
-            cw[u] = w0 + u < words ? __ldcg(closed + w0 + u) : ~0u;
-            v[u] = g < G ? __ldcg(drow + g) : 0.f;
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int g = (w0 + u) * 32 + lane;
-            if (g < G && !((cw[u] >> lane) & 1u)) {
-              saw_nan |= (v[u] != v[u]);
-              const unsigned long long key = decision_key(v[u], g);
-              best = key < best ? key : best;
-            }
+        for (int u = 0; u < MAXW; ++u) {
+          const int g = u * 32 + lane;
+          if (u < words && g < G && !(((a.stage_closed ? closed[u] : __ldcg(closed + u)) >> lane) & 1u)) {
+            saw_nan |= (v[u] != v[u]);
+            const unsigned long long key = decision_key(v[u], g);
+            best = key < best ? key : best;
           }
         }
         best = warp_min_u64(best);
@@ -596,14 +632,19 @@ __global__ void __launch_bounds__(kFillThreads) fill_coop_kernel(FillArgs a) {
       const int r = __ldcg(a.room + x);
       const unsigned long long* bk = a.bucket + static_cast<size_t>(h) * n + __ldcg(a.offs + x);
       int* lab = a.labels + static_cast<size_t>(h) * n;
-      if (c <= r) {
-        for (int e = lane; e < c; e += 32) lab[__ldcg(bk + e) & 0xffffffffu] = g;
-      } else {
-        const unsigned long long thr = warp_select_kth(bk, c, r, hist[warp]);
-        for (int e = lane; e < c; e += 32) {
-          const unsigned long long key = __ldcg(bk + e);
-          const int i = static_cast<int>(key & 0xffffffffu);
-          if (key <= thr) {
+      const unsigned long long thr = c <= r ? ~0ull : warp_select_kth(bk, c, r, hist[warp]);
+      for (int e0 = 0; e0 < c; e0 += 256) {
+        unsigned long long kb[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int e = e0 + u * 32 + lane;
+          kb[u] = e < c ? __ldcg(bk + e) : ~0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (e0 + u * 32 + lane >= c) continue;
+          const int i = static_cast<int>(kb[u] & 0xffffffffu);
+          if (kb[u] <= thr) {
             lab[i] = g;
           } else {
             const int pos = atomicAdd(a.list_len + next, 1);
@@ -794,13 +835,24 @@ cudaError_t launch_fill(const FillArgs& a, cudaStream_t st) {
   int dev = 0, sms = 0, per_sm = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fill_coop_kernel, kFillThreads, 0);
+  const int words = ceil_div(a.G, 32);
+  if (words > 32) return cudaErrorInvalidValue;
+  void* kern = words <= 8 ? reinterpret_cast<void*>(fill_coop_kernel<8>)
+               : words <= 20 ? reinterpret_cast<void*>(fill_coop_kernel<20>)
+                             : reinterpret_cast<void*>(fill_coop_kernel<32>);
+  FillArgs args = a;
+  const size_t closed_bytes = sizeof(unsigned int) * static_cast<size_t>(a.heads) * words;
+  args.stage_closed = closed_bytes <= kFillStageLimit ? 1 : 0;
+  const size_t smem = args.stage_closed ? closed_bytes : 0;
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFillThreads, smem);
   if (e != cudaSuccess) return e;
   const int blocks = sms * std::min(per_sm, 4);
-  FillArgs args = a;
   void* params[] = {&args};
-  e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(fill_coop_kernel), dim3(blocks), dim3(kFillThreads),
-                                  params, 0, st);
+  e = cudaLaunchCooperativeKernel(kern, dim3(blocks), dim3(kFillThreads), params, smem, st);
   return counted(e, 2);
 }
 

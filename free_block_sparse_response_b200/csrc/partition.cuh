@@ -46,6 +46,7 @@ struct FillArgs {
   int* prop_g;          // [heads, n]
   float* prop_v;
   WorkspaceHeader* hdr;
+  int stage_closed;     // set by the launcher: bitmaps fit in shared memory
 };
 
 cudaError_t launch_midpoint_stride(int* idx, int n, int count, cudaStream_t st);
