@@ -234,13 +234,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc::tmem_ld32(sbuf + 96, *reinterpret_cast<uint32_t(*)[32]>(&u[96]));
       tc::tmem_wait_ld();
       const int nvalid = s_size[j];
-      float mx = -kInf;
+      if (nvalid < 128) {  // short group (warp-uniform): mask the padding keys
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const float x = c < nvalid ? __uint_as_float(u[c]) : -kInf;
-        u[c] = __float_as_uint(x);
-        mx = fmaxf(mx, x);
+        for (int c = 0; c < 128; ++c)
+          if (c >= nvalid) u[c] = __float_as_uint(-kInf);
       }
+      // row max as a tree of 8 independent chains
+      float mx8[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) mx8[t] = __uint_as_float(u[t]);
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(u[c]));
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       mx *= scale_log2;
       const bool grow = mx > m_run + kRescaleLog2;
       const bool need_o = grow && m_run != -kInf;
@@ -268,7 +274,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       const float msafe = m_run == -kInf ? 0.f : m_run;
-      float sum = 0.f;
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
@@ -276,12 +282,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int i = 0; i < 32; ++i) {
           const float p0 = ex2(fmaf(__uint_as_float(u[half * 64 + 2 * i]), scale_log2, -msafe));
           const float p1 = ex2(fmaf(__uint_as_float(u[half * 64 + 2 * i + 1]), scale_log2, -msafe));
-          sum += p0 + p1;
+          sum4[i & 3] += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
         tc::tmem_st32(sbuf + half * 32, pk);
       }
-      l_run += sum;
+      l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       tc::tmem_wait_st();
       tc::fence_before_sync();
       tc::mbar_arrive(bar(kPFull));
