@@ -29,9 +29,9 @@ METRIC = "SparsePR ms/call & eff. TFLOP/s at 22% pair density; mean rel-L2 err v
 UNIT = "TFLOP/s (dense-equivalent, 4*d*N^2*H per call)"
 
 # DRAM bytes per launch of the dominant kernel from an ncu capture of the same kernel
-# build (profiles/attn_tc_kernel_video_4h.md: 375.9 MB on 4 heads, scaled by heads to
-# the 40-head launch); set back to None whenever that kernel changes.
-DOMINANT_TRAFFIC_BYTES = 3.759e9
+# build (profiles/), scaled by heads to the 40-head launch; None whenever that kernel
+# has changed since the capture.
+DOMINANT_TRAFFIC_BYTES = None
 
 
 def parse_args():

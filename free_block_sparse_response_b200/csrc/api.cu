@@ -52,7 +52,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct Layout {
   size_t header = 0, sample_idx, gamma, gamma_hi, gamma_lo, nrm, cent_k, cent_q, wf, whi, wlo, eg, dmat,
          prop_g0, prop_v0, labels, room, cnt, offs, cursor, closed, bucket, list0, list1, list_len, prop_g, prop_v,
-         perm_tmp, perm_cursor, qblk, partial, fit, total;
+         perm_tmp, perm_cursor, qblk, partial, fit, kv_grouped, total;
 };
 
 Layout make_layout(int heads, int N, int d, int block, int S, int P) {
@@ -64,6 +64,11 @@ Layout make_layout(int heads, int N, int d, int block, int S, int P) {
     off = align_up(off + bytes);
     return at;
   };
+  // Regions read by the calls after partition come first, so that their offsets depend
+  // only on the shapes (and P) each of those calls knows.
+  L.kv_grouped = take(2 * 2 * H * G * block * D);  // K and V in key-group order, bf16
+  L.partial = take(P > 0 ? spr::probe_partial_bytes(heads, P, static_cast<int>(G), d) : 0);
+  L.fit = take(P > 0 ? sizeof(double) * H * spr::fit_scratch_doubles(P, d) : 0);
   L.sample_idx = take(sizeof(int) * static_cast<size_t>(S));
   L.gamma = take(sizeof(float) * H * D * D);
   L.gamma_hi = take(2 * H * D * D);
@@ -93,8 +98,6 @@ Layout make_layout(int heads, int N, int d, int block, int S, int P) {
   L.perm_tmp = take(sizeof(int) * H * G * block);
   L.perm_cursor = take(sizeof(int) * H * G);
   L.qblk = take(sizeof(int) * H * n);
-  L.partial = take(P > 0 ? spr::probe_partial_bytes(heads, P, static_cast<int>(G), d) : 0);
-  L.fit = take(P > 0 ? sizeof(double) * H * spr::fit_scratch_doubles(P, d) : 0);
   L.total = off;
   return L;
 }
@@ -334,6 +337,12 @@ static int attention_common(const void* Q, const void* K, const void* V, int dty
   a.route = route;
   a.scale_log2 = resolve_scale(scale, d) * kLog2e;
   a.out = out;
+  if (!dense && !a.f32 && d == 128 && block == 128) {
+    if (ws == nullptr) return fail(SPARSEPR_ERR_INVALID_ARG, "sparse attention needs the workspace");
+    const Layout L = make_layout(Bt * H, N, d, block, 1, 0);
+    a.k_grouped = at<char>(ws, L.kv_grouped);
+    a.v_grouped = at<char>(ws, L.kv_grouped) + static_cast<size_t>(Bt) * H * G * block * d * 2;
+  }
   if (ws != nullptr) {
     a.status = &header(ws)->status;
   } else {

@@ -20,6 +20,10 @@ struct AttnArgs {
   float scale_log2;  // tau * log2(e)
   float* out;
   int* status;       // device status word (bounded waits of the tensor-core kernel)
+  // Group-ordered copies of K and V ([heads, G * 128, 128] bf16 each, pad rows zero),
+  // written by the sparse tensor-core path before its attention kernel; null otherwise.
+  void* k_grouped;
+  void* v_grouped;
 };
 
 struct ProbeArgs {

@@ -4,19 +4,36 @@
 // query block attends only to its routed key groups, softmax renormalised over that
 // support.  One CTA per (query block of 128 rows, head); head dim 128; key groups of 128.
 //
-// Warp roles (256 threads, one CTA per SM):
-//   warps 0-1  producers: gather the block's Q rows and each routed group's K and V rows
-//              (through the permutations) with cp.async into 128B-swizzled UMMA tiles;
-//              K and V double-buffered; arrival on mbarriers when the copies land.
-//   warp 2     MMA issuer (one lane): S_j = Q K_j^T into TMEM (double-buffered, so S_{j+1}
-//              overlaps the softmax of tile j), O += P_j V_j with P read from TMEM.
-//   warps 4-7  softmax: thread i owns TMEM lane i (query row i); reads S_j, keeps the
-//              running max / sum, writes P_j (bf16) back over S_j, rescales O only when
-//              the row max grew by more than 2^8 (stale maxima are exact after the final
-//              division), and writes the normalised row at the end.
-// TMEM (512 columns): S0 [0,128), S1 [128,256), O [256,384).
+// The routed tiles j = 0 .. n-1 of a block are split into two streams, even and odd j.
+// Each stream keeps its own S tile, running max / sum and O accumulator, so that the
+// two softmax warpgroups work on different tiles at the same time (one keeps the MUFU
+// busy while the other loads, reduces or stores); the two partial results are merged
+// at the end like a split-K softmax: O = (2^(m0-m) O0 + 2^(m1-m) O1) / (2^(m0-m) l0 +
+// 2^(m1-m) l1), m = max(m0, m1).
+//
+// Warp roles (384 threads, one CTA per SM):
+//   warps 0-1   producers, warp x feeds stream x: TMA loads of its routed groups as two
+//               64-column x 128-row boxes of the group-ordered K and V copies (sparse) or
+//               of K and V themselves (dense), into that stream's own K and V buffers;
+//               warp 0 also gathers the block's Q rows through the query permutation
+//               (tile::gather4, 4 token rows per instruction; pad rows of a short block
+//               repeat its first member).
+//   warps 2-3   MMA issuers, lane 0 of warp 2 + x drives stream x: S_x = Q K_j^T into
+//               TMEM, then O_x += P_j V_j with P read from TMEM, then S_x for the next
+//               tile of the stream.  With one issuer per stream, one stream's waits and
+//               commits overlap the other stream's MMAs.
+//   warps 4-7   softmax, stream 0; warps 8-11 softmax, stream 1.  Thread i of a
+//               warpgroup owns TMEM lane i (query row i); it reads S, keeps the running
+//               max / sum, writes P (bf16) back over S, rescales its O only when the row
+//               max grew by more than 2^8 (stale maxima are exact after the final
+//               division), and at the end merges the two streams for half the columns.
+// Warps 0-3 give registers to the softmax warpgroups (setmaxnreg).
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 // Every wait is bounded; on timeout the CTA records kErrTimeout, drains its MMAs and
 // frees TMEM before exiting.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "attention.cuh"
 #include "common.cuh"
 #include "tcgen05.cuh"
@@ -25,16 +42,22 @@
 namespace spr {
 namespace {
 
-constexpr int kTcThreads = 256;
-constexpr int kTcProducers = 64;
+constexpr int kTcThreads = 384;
+constexpr int kRegLow = 80;       // warps 0-3 after the re-split
+constexpr int kRegSoftmax = 208;  // warps 4-11 after the re-split
 constexpr uint32_t kTile = 128 * 128 * 2;  // one 128 x 128 bf16 tile
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr float kInf = __builtin_huge_valf();
 
+// Barriers: Q landed; per stream x (index + x): K / V tile landed, S ready (which also
+// frees the stream's K buffer), P ready, PV done (which frees the V buffer and means
+// O_x holds every finished tile), drain; the last PV of both streams.
+// kTok0 + x: the other stream's exponentials for the tile before stream x's next one
+// are done (the two softmax warpgroups take turns on the MUFU).
 enum : int {
-  kQFull = 0, kKFull0 = 1, kVFull0 = 3, kKEmpty0 = 5, kVEmpty0 = 7, kSFull0 = 9,
-  kPFull = 11, kOReady = 12, kOFinal = 13, kDrain = 14, kNumBars = 15
+  kQFull = 0, kKFull0 = 1, kVFull0 = 3, kSFull0 = 5, kPFull0 = 7, kVEmpty0 = 9, kDrain0 = 11,
+  kTok0 = 13, kOFinal = 15, kNumBars = 16
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -58,8 +81,8 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 
 template <bool DENSE>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    attn_tc_kernel(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
-                   const __nv_bfloat16* __restrict__ V, int N, int G, int k, const int* __restrict__ key_perm,
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, int N, int G, int k, const int* __restrict__ key_perm,
                    const int* __restrict__ key_gsize, const int* __restrict__ query_perm,
                    const int* __restrict__ qblock_size, const int* __restrict__ route, float scale_log2,
                    float* __restrict__ out, int* __restrict__ status) {
@@ -67,28 +90,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ __align__(8) uint64_t bars[kNumBars];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  __shared__ float2 s_ml[2][128];  // per stream and row: final (max, sum)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = blockIdx.x, head = blockIdx.y;
   const uint32_t sbase = (tc::saddr(dsmem) + 1023u) & ~1023u;
   const uint32_t sQ = sbase;
-  const uint32_t sK[2] = {sbase + kTile, sbase + 2 * kTile};
-  const uint32_t sV[2] = {sbase + 3 * kTile, sbase + 4 * kTile};
+  const uint32_t sK0 = sbase + kTile;      // K buffer of stream x: sK0 + x kTile
+  const uint32_t sV0 = sbase + 3 * kTile;  // V buffer of stream x: sV0 + x kTile
   auto bar = [&](int i) { return tc::saddr(&bars[i]); };
 
   if (tid == 0) {
-    tc::mbar_init(bar(kQFull), kTcProducers);
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(bar(kKFull0 + s), kTcProducers);
-      tc::mbar_init(bar(kVFull0 + s), kTcProducers);
-      tc::mbar_init(bar(kKEmpty0 + s), 1);
-      tc::mbar_init(bar(kVEmpty0 + s), 1);
-      tc::mbar_init(bar(kSFull0 + s), 1);
+    tc::mbar_init(bar(kQFull), 1);
+    for (int x = 0; x < 2; ++x) {
+      tc::mbar_init(bar(kKFull0 + x), 1);
+      tc::mbar_init(bar(kVFull0 + x), 1);
+      tc::mbar_init(bar(kSFull0 + x), 1);
+      tc::mbar_init(bar(kPFull0 + x), 128);
+      tc::mbar_init(bar(kVEmpty0 + x), 1);
+      tc::mbar_init(bar(kDrain0 + x), 1);
+      tc::mbar_init(bar(kTok0 + x), 128);
     }
-    tc::mbar_init(bar(kPFull), 128);
-    tc::mbar_init(bar(kOReady), 1);
-    tc::mbar_init(bar(kOFinal), 1);
-    tc::mbar_init(bar(kDrain), 1);
+    tc::mbar_init(bar(kOFinal), 2);
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -101,15 +124,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc::fence_after_sync();
   const uint32_t tbase = tmem_slot;
 
-  const size_t hoff = static_cast<size_t>(head) * N * 128;
-  Q += hoff;
-  K += hoff;
-  V += hoff;
-  out += hoff;
+  const int row0 = head * N;  // first row of this head in the [heads * N, 128] tensor maps
+  out += static_cast<size_t>(head) * N * 128;
   const size_t goff = static_cast<size_t>(head) * G;
   const int nq = DENSE ? min(128, N - b * 128) : qblock_size[goff + b];
   const int* qperm = DENSE ? nullptr : query_perm + (goff + b) * 128;
-  const int* kperm = DENSE ? nullptr : key_perm + goff * 128;
   const int n_tiles = DENSE ? G : k;
   const int* my_route = DENSE ? nullptr : route + (goff + b) * k;
   // per-tile key group and its size, staged once (the producers and the softmax read them)
@@ -123,110 +142,129 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   volatile int* abort_v = &abort_flag;
 
-  if (warp < 2) {
-    // ------------------------------------------------------------------ producers
-    // Thread pt copies 16-byte chunk (pt & 15) of rows (pt >> 4) + 4 i, i < 32: 16 threads
-    // cover one 256-byte row.  The 32 row indices are fetched before any copy is issued.
-    const int pt = tid, ch = pt & 15, r0 = pt >> 4;
-    int toks[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int r = r0 + 4 * i;
-      toks[i] = r < nq ? (DENSE ? b * 128 + r : __ldg(qperm + r)) : -1;
-    }
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int r = r0 + 4 * i;
-      cp_async_16(sQ + tc::sw128_offset(r, ch), toks[i] >= 0 ? Q + static_cast<size_t>(toks[i]) * 128 + ch * 8 : Q,
-                  toks[i] >= 0 ? 16 : 0);
-    }
-    tc::cp_async_arrive_noinc(bar(kQFull));
-    for (int j = 0; j < n_tiles; ++j) {
-      const int s = j & 1;
-      const int g = s_group[j];
-      const int gs = s_size[j];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = r0 + 4 * i;
-        toks[i] = r < gs ? (DENSE ? g * 128 + r : __ldg(kperm + g * 128 + r)) : -1;
+  if (warp < 4) {
+    tc::setmaxnreg_dec<kRegLow>();
+    if (warp < 2) {
+      // ------------------------------------------------------------------ producers
+      // Q: lane l gathers rows 4 l .. 4 l + 3 through the query permutation (two gather4
+      // per lane, one per 64-column half of the swizzled tile).  K / V: one lane loads
+      // each routed group as two 64-column x 128-row boxes.
+      const int rq = 4 * lane;
+      auto gather_tile = [&](const CUtensorMap* tm, uint32_t dst, const int4& t, uint32_t full) {
+        tc::tma_gather4(dst + rq * 128, tm, 0, t.x, t.y, t.z, t.w, full);
+        tc::tma_gather4(dst + 128 * 128 + rq * 128, tm, 64, t.x, t.y, t.z, t.w, full);
+      };
+      const int x = warp;  // stream whose K and V tiles this warp loads
+      if (x == 0) {
+        int4 t;
+        if (DENSE) {
+          const int base = row0 + b * 128;
+          t = make_int4(base + min(rq, nq - 1), base + min(rq + 1, nq - 1), base + min(rq + 2, nq - 1),
+                        base + min(rq + 3, nq - 1));
+        } else {
+          const int4 v = __ldg(reinterpret_cast<const int4*>(qperm + rq));
+          const int first = __shfl_sync(0xffffffffu, v.x, 0);
+          t = make_int4(row0 + (rq < nq ? v.x : first), row0 + (rq + 1 < nq ? v.y : first),
+                        row0 + (rq + 2 < nq ? v.z : first), row0 + (rq + 3 < nq ? v.w : first));
+        }
+        if (lane == 0) tc::mbar_arrive_expect_tx(bar(kQFull), kTile);
+        __syncwarp();
+        gather_tile(&tmQ, sQ, t, bar(kQFull));
       }
-      if (j >= 2 && !tc::mbar_wait(bar(kKEmpty0 + s), ((j >> 1) - 1) & 1, abort_v, status)) break;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = r0 + 4 * i;
-        cp_async_16(sK[s] + tc::sw128_offset(r, ch),
-                    toks[i] >= 0 ? K + static_cast<size_t>(toks[i]) * 128 + ch * 8 : K, toks[i] >= 0 ? 16 : 0);
+      // first row of key group g in the K / V maps: the token order itself (dense) or the
+      // group-ordered copies (sparse)
+      const int kvrow0 = DENSE ? row0 : head * G * 128;
+      const uint32_t sK = sK0 + x * kTile, sV = sV0 + x * kTile;
+      int issued = 0;  // tiles of this stream whose copies were issued
+      for (int j = x; j < n_tiles; j += 2) {
+        const int it = j >> 1;
+        const int row = kvrow0 + s_group[j] * 128;
+        // K buffer free once S of the stream's previous tile is ready
+        if (it >= 1 && !warp_wait(bar(kSFull0 + x), (it - 1) & 1, abort_v, status)) break;
+        if (lane == 0) {
+          tc::mbar_arrive_expect_tx(bar(kKFull0 + x), kTile);
+          tc::tma_load_2d(sK, &tmK, 0, row, bar(kKFull0 + x));
+          tc::tma_load_2d(sK + 128 * 128, &tmK, 64, row, bar(kKFull0 + x));
+        }
+        // V buffer free once the stream's previous PV is done
+        if (it >= 1 && !warp_wait(bar(kVEmpty0 + x), (it - 1) & 1, abort_v, status)) {
+          issued = -(it + 1);  // K of this tile is in flight, V is not
+          break;
+        }
+        if (lane == 0) {
+          tc::mbar_arrive_expect_tx(bar(kVFull0 + x), kTile);
+          tc::tma_load_2d(sV, &tmV, 0, row, bar(kVFull0 + x));
+          tc::tma_load_2d(sV + 128 * 128, &tmV, 64, row, bar(kVFull0 + x));
+        }
+        __syncwarp();
+        issued = it + 1;
       }
-      tc::cp_async_arrive_noinc(bar(kKFull0 + s));
-      if (j >= 2 && !tc::mbar_wait(bar(kVEmpty0 + s), ((j >> 1) - 1) & 1, abort_v, status)) break;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = r0 + 4 * i;
-        cp_async_16(sV[s] + tc::sw128_offset(r, ch),
-                    toks[i] >= 0 ? V + static_cast<size_t>(toks[i]) * 128 + ch * 8 : V, toks[i] >= 0 ? 16 : 0);
+      // Copies still in flight after an abort must land before the CTA exits: wait
+      // (bounded) for the stream's last K and V phases and for Q.  On the normal path
+      // these phases completed long ago and the waits return at once.
+      if (lane == 0) {
+        const int nk = issued >= 0 ? issued : -issued, nv = issued >= 0 ? issued : -issued - 1;
+        if (nk > 0) drain_wait(bar(kKFull0 + x), (nk - 1) & 1);
+        if (nv > 0) drain_wait(bar(kVFull0 + x), (nv - 1) & 1);
+        if (x == 0) drain_wait(bar(kQFull), 0);
       }
-      tc::cp_async_arrive_noinc(bar(kVFull0 + s));
-    }
-    cp_async_wait<0>();
-  } else if (warp == 2) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+      __syncwarp();
+    } else if (lane == 0) {
+      // ------------------------------------------------------------------ MMA issuers
+      // warp 2 lane 0 drives stream 0, warp 3 lane 0 stream 1: while one waits or
+      // commits, the other's MMAs keep the tensor pipe busy.
+      const int x = warp - 2;
       constexpr uint32_t kIdQK = tc::idesc_bf16(128, 128, false, false);
       constexpr uint32_t kIdPV = tc::idesc_bf16(128, 128, false, true);
-      const uint32_t tS[2] = {tbase, tbase + 128};
-      const uint32_t tO = tbase + 256;
+      const uint32_t tS = tbase + 128 * x, tO = tbase + 256 + 128 * x;
+      const uint32_t sK = sK0 + x * kTile, sV = sV0 + x * kTile;
       bool ok = tc::mbar_wait(bar(kQFull), 0, abort_v, status);
-      tc::fence_proxy_async();
-      auto issue_s = [&](int j) -> bool {
-        const int s = j & 1;
-        if (!tc::mbar_wait(bar(kKFull0 + s), (j >> 1) & 1, abort_v, status)) return false;
-        tc::fence_proxy_async();
+      auto issue_s = [&](int it) -> bool {
+        if (!tc::mbar_wait(bar(kKFull0 + x), it & 1, abort_v, status)) return false;
+        tc::fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          tc::mma_ss(tS[s], tc::sdesc_sw128(sQ + koff, 16, 1024), tc::sdesc_sw128(sK[s] + koff, 16, 1024), kIdQK,
+          tc::mma_ss(tS, tc::sdesc_sw128(sQ + koff, 16, 1024), tc::sdesc_sw128(sK + koff, 16, 1024), kIdQK,
                      kk > 0 ? 1u : 0u);
         }
-        tc::mma_commit(bar(kKEmpty0 + s));
-        tc::mma_commit(bar(kSFull0 + s));
+        tc::mma_commit(bar(kSFull0 + x));
         return true;
       };
-      if (ok) ok = issue_s(0);
-      if (ok && n_tiles > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j & 1;
-        if (!tc::mbar_wait(bar(kPFull), j & 1, abort_v, status)) break;
+      if (ok && x < n_tiles) ok = issue_s(0);
+      for (int j = x, it = 0; ok && j < n_tiles; j += 2, ++it) {
+        if (!tc::mbar_wait(bar(kPFull0 + x), it & 1, abort_v, status)) break;
         tc::fence_after_sync();
-        if (!tc::mbar_wait(bar(kVFull0 + s), (j >> 1) & 1, abort_v, status)) break;
-        tc::fence_proxy_async();
+        if (!tc::mbar_wait(bar(kVFull0 + x), it & 1, abort_v, status)) break;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          tc::mma_ts(tO, tS[s] + kk * 8, tc::sdesc_sw128(sV[s] + kk * 2048, 128 * 128, 1024), kIdPV,
-                     (j > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_ts(tO, tS + kk * 8, tc::sdesc_sw128(sV + kk * 2048, 128 * 128, 1024), kIdPV,
+                     (it > 0 || kk > 0) ? 1u : 0u);
         }
-        tc::mma_commit(bar(kVEmpty0 + s));
-        tc::mma_commit(bar(kOReady));
-        if (j + 2 < n_tiles && !issue_s(j + 2)) break;
-        if (j == n_tiles - 1) tc::mma_commit(bar(kOFinal));
+        tc::mma_commit(bar(kVEmpty0 + x));
+        if (j + 2 < n_tiles && !issue_s(it + 1)) break;
       }
-      tc::mma_commit(bar(kDrain));
-      drain_wait(bar(kDrain), 0);
+      tc::mma_commit(bar(kOFinal));
+      tc::mma_commit(bar(kDrain0 + x));
+      drain_wait(bar(kDrain0 + x), 0);
     }
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------------------------ softmax
-    const int r = tid - 128;
-    const uint32_t lane_off = static_cast<uint32_t>(32 * (warp - 4)) << 16;
+    tc::setmaxnreg_inc<kRegSoftmax>();
+    const int x = (warp - 4) >> 2;  // stream: tiles x, x + 2, x + 4, ...
+    const int r = 32 * (warp & 3) + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const uint32_t sbuf = tbase + lane_off + x * 128;
     const int tok = r < nq ? (DENSE ? b * 128 + r : __ldg(qperm + r)) : -1;
     float m_run = -kInf, l_run = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      const int s = j & 1;
-      if (!warp_wait(bar(kSFull0 + s), (j >> 1) & 1, abort_v, status)) {
+    for (int j = x; j < n_tiles; j += 2) {
+      const int it = j >> 1;  // index of this tile within the stream
+      if (!warp_wait(bar(kSFull0 + x), it & 1, abort_v, status)) {
         ok = false;
         break;
       }
       tc::fence_after_sync();
-      const uint32_t sbuf = tbase + lane_off + s * 128;
       uint32_t u[128];
       tc::tmem_ld32(sbuf, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
       tc::tmem_ld32(sbuf + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
@@ -257,12 +295,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         m_run = mx;
       }
       if (__any_sync(0xffffffffu, need_o)) {
-        if (!warp_wait(bar(kOReady), (j - 1) & 1, abort_v, status)) {
+        // O_x holds tiles up to j - 2 once that tile's PV has completed
+        if (!warp_wait(bar(kVEmpty0 + x), (it - 1) & 1, abort_v, status)) {
           ok = false;
           break;
         }
         tc::fence_after_sync();
-        const uint32_t obuf = tbase + lane_off + 256;
+        const uint32_t obuf = tbase + lane_off + 256 + x * 128;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t o[32];
@@ -272,6 +311,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           tc::tmem_st32(obuf + q * 32, o);
         }
+      }
+      // Take turns with the other stream: tile j starts its exponentials once tile j - 1
+      // (the other stream's) has finished them, so that one warpgroup's MUFU phase runs
+      // while the other stream's MMAs do.
+      if (j >= 1 && !warp_wait(bar(kTok0 + x), (x == 1 ? it : it - 1) & 1, abort_v, status)) {
+        ok = false;
+        break;
       }
       const float msafe = m_run == -kInf ? 0.f : m_run;
       float sum4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -287,26 +333,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tc::tmem_st32(sbuf + half * 32, pk);
       }
+      if (j + 1 < n_tiles) tc::mbar_arrive(bar(kTok0 + (x ^ 1)));
       l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       tc::tmem_wait_st();
       tc::fence_before_sync();
-      tc::mbar_arrive(bar(kPFull));
+      tc::mbar_arrive(bar(kPFull0 + x));
     }
+    // ---- merge the two streams; warpgroup x writes columns [64 x, 64 x + 64)
+    s_ml[x][r] = make_float2(m_run, l_run);
+    tc::named_bar_sync(1, 256);  // every softmax thread reaches this exactly once
+    const float2 a0 = s_ml[0][r], a1 = s_ml[1][r];
+    const float mm = fmaxf(a0.x, a1.x);
+    const float f0 = a0.x == -kInf ? 0.f : ex2(a0.x - mm);
+    const float f1 = a1.x == -kInf ? 0.f : ex2(a1.x - mm);
+    const float den = a0.y * f0 + a1.y * f1;
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    const float g0 = f0 * inv, g1 = f1 * inv;
+    const bool has1 = n_tiles > 1;  // stream 1 never wrote O1 otherwise
     if (ok && warp_wait(bar(kOFinal), 0, abort_v, status)) {
       tc::fence_after_sync();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      const uint32_t obuf = tbase + lane_off + 256;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t o[32];
-        tc::tmem_ld32(obuf + q * 32, o);
+      for (int q = 0; q < 2; ++q) {
+        const int col = 64 * x + 32 * q;
+        uint32_t o0[32], o1[32];
+        tc::tmem_ld32(tbase + lane_off + 256 + col, o0);
+        if (has1) tc::tmem_ld32(tbase + lane_off + 384 + col, o1);
         tc::tmem_wait_ld();
-        if (tok >= 0) {
-          float4* dst = reinterpret_cast<float4*>(out + static_cast<size_t>(tok) * 128 + q * 32);
+        if (!has1) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv, __uint_as_float(o[4 * i + 1]) * inv,
-                                 __uint_as_float(o[4 * i + 2]) * inv, __uint_as_float(o[4 * i + 3]) * inv);
+          for (int i = 0; i < 32; ++i) o1[i] = 0u;
+        }
+        if (tok >= 0) {
+          float4* dst = reinterpret_cast<float4*>(out + static_cast<size_t>(tok) * 128 + col);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float v[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+              v[t] = fmaf(__uint_as_float(o0[4 * i + t]), g0, __uint_as_float(o1[4 * i + t]) * g1);
+            dst[i] = make_float4(v[0], v[1], v[2], v[3]);
+          }
         }
       }
     }
@@ -321,20 +387,98 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
+// K and V rows of every key group, in group order: row r of group g of head h lands at
+// row (h G + g) 128 + r of the copies; rows past the group's size are zero.  One CTA per
+// (group, head); 16 threads copy one 256-byte row with 16-byte accesses.
+__global__ void __launch_bounds__(256) kv_group_kernel(const uint4* __restrict__ K, const uint4* __restrict__ V,
+                                                       int N, int G, const int* __restrict__ key_perm,
+                                                       const int* __restrict__ key_gsize, uint4* __restrict__ Kg,
+                                                       uint4* __restrict__ Vg) {
+  const int g = blockIdx.x, head = blockIdx.y;
+  const size_t grp = static_cast<size_t>(head) * G + g;
+  const int gs = __ldg(key_gsize + grp);
+  const int ch = threadIdx.x & 15;
+#pragma unroll 4
+  for (int r = threadIdx.x >> 4; r < 128; r += 16) {
+    const int tok = r < gs ? __ldg(key_perm + grp * 128 + r) : -1;
+    const size_t dst = (grp * 128 + r) * 16 + ch;
+    uint4 kv = make_uint4(0, 0, 0, 0), vv = kv;
+    if (tok >= 0 && tok < N) {
+      const size_t src = (static_cast<size_t>(head) * N + tok) * 16 + ch;
+      kv = __ldg(K + src);
+      vv = __ldg(V + src);
+    }
+    Kg[dst] = kv;
+    Vg[dst] = vv;
+  }
+}
+
 }  // namespace
 
 size_t attn_tc_smem_bytes(int n_tiles) { return 5ull * kTile + 1024 + 8ull * n_tiles; }
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// Map over a [rows, 128] bf16 tensor with 128-byte swizzle and a box of 64 columns x
+// box_rows rows (1 for row gathers).
+bool bf16_map(CUtensorMap* m, const void* base, long long rows, int box_rows) {
+  auto fn = encode_tiled();
+  if (fn == nullptr || (reinterpret_cast<uintptr_t>(base) & 15u) != 0 || rows <= 0) return false;
+  cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {128 * sizeof(__nv_bfloat16)};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
 
 cudaError_t launch_attention_tc(const AttnArgs& a, bool dense, int* status, cudaStream_t st) {
   const size_t smem = attn_tc_smem_bytes(dense ? a.G : a.k);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   auto kern = dense ? attn_tc_kernel<true> : attn_tc_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  // The register re-split must fit in what the block is launched with, or the
+  // setmaxnreg.inc of the softmax warpgroups would never be granted.
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(a.G, a.heads), kTcThreads, smem, st>>>(
-      static_cast<const __nv_bfloat16*>(a.Q), static_cast<const __nv_bfloat16*>(a.K),
-      static_cast<const __nv_bfloat16*>(a.V), a.N, a.G, a.k, a.key_perm, a.key_gsize, a.query_perm, a.qblock_size,
-      a.route, a.scale_log2, a.out, status);
+  if (128 * kRegLow + 256 * kRegSoftmax > fa.numRegs * kTcThreads) return cudaErrorInvalidConfiguration;
+  const long long rows = static_cast<long long>(a.heads) * a.N;
+  const long long grows = static_cast<long long>(a.heads) * a.G * 128;
+  if (rows > 0x7fffffffLL || grows > 0x7fffffffLL) return cudaErrorInvalidValue;  // TMA coordinates are int32
+  if (!dense && (a.k_grouped == nullptr || a.v_grouped == nullptr)) return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, tv;
+  const bool maps = bf16_map(&tq, a.Q, rows, 1) &&
+                    (dense ? bf16_map(&tk, a.K, rows, 128) && bf16_map(&tv, a.V, rows, 128)
+                           : bf16_map(&tk, a.k_grouped, grows, 128) && bf16_map(&tv, a.v_grouped, grows, 128));
+  if (!maps) return cudaErrorInvalidValue;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  if (!dense) {
+    kv_group_kernel<<<dim3(a.G, a.heads), 256, 0, st>>>(
+        static_cast<const uint4*>(a.K), static_cast<const uint4*>(a.V), a.N, a.G, a.key_perm, a.key_gsize,
+        static_cast<uint4*>(a.k_grouped), static_cast<uint4*>(a.v_grouped));
+    e = counted(cudaGetLastError(), 1);
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<dim3(a.G, a.heads), kTcThreads, smem, st>>>(tq, tk, tv, a.N, a.G, a.k, a.key_perm, a.key_gsize,
+                                                       a.query_perm, a.qblock_size, a.route, a.scale_log2, a.out,
+                                                       status);
   return counted(cudaGetLastError(), 1);
 }
 
