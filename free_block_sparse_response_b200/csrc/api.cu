@@ -453,6 +453,20 @@ int sparsepr_probe_rows(int32_t N, int32_t P, int32_t Bt, int32_t H, int32_t* pr
 
 uint64_t sparsepr_launch_count(void) { return spr::g_launches.load(std::memory_order_relaxed); }
 
+int sparsepr_kernel_timing(int enable) {
+  spr::attn_timing_enable(enable != 0);
+  return SPARSEPR_OK;
+}
+
+int sparsepr_kernel_timing_read(double* ms_total, int64_t* launches) {
+  long long n = 0;
+  double ms = 0.0;
+  SPR_CUDA(spr::attn_timing_read(&ms, &n), "kernel timing read");
+  if (ms_total) *ms_total = ms;
+  if (launches) *launches = n;
+  return SPARSEPR_OK;
+}
+
 int sparsepr_row_errors(const void* O, int o_dtype, const float* O_ref, const int32_t* probe_idx, int32_t Bt,
                         int32_t H, int32_t N, int32_t d, int32_t P, float* err, sparsepr_stream_t stream) {
   int rc;

@@ -46,6 +46,9 @@ struct ProbeArgs {
 
 cudaError_t launch_attention(const AttnArgs& a, bool dense, cudaStream_t st);
 cudaError_t launch_attention_tc(const AttnArgs& a, bool dense, int* status, cudaStream_t st);
+// Event pairs around the tensor-core attention kernel (measurement hook).
+void attn_timing_enable(bool on);
+cudaError_t attn_timing_read(double* ms_total, long long* launches);
 size_t attn_tc_smem_bytes(int n_tiles);
 cudaError_t launch_probe(const ProbeArgs& a, cudaStream_t st);
 size_t probe_partial_bytes(int heads, int P, int G, int d);

@@ -34,6 +34,10 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <mutex>
+#include <utility>
+#include <vector>
+
 #include "attention.cuh"
 #include "common.cuh"
 #include "tcgen05.cuh"
@@ -43,27 +47,80 @@ namespace spr {
 namespace {
 
 constexpr int kTcThreads = 384;
-constexpr int kRegLow = 80;       // warps 0-3 after the re-split
-constexpr int kRegSoftmax = 208;  // warps 4-11 after the re-split
+constexpr int kRegLow = 72;       // warps 0-3 after the re-split
+constexpr int kRegSoftmax = 216;  // warps 4-11 after the re-split
 constexpr uint32_t kTile = 128 * 128 * 2;  // one 128 x 128 bf16 tile
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr float kInf = __builtin_huge_valf();
 
-// Barriers: Q landed; per stream x (index + x): K / V tile landed, S ready (which also
-// frees the stream's K buffer), P ready, PV done (which frees the V buffer and means
-// O_x holds every finished tile), drain; the last PV of both streams.
-// kTok0 + x: the other stream's exponentials for the tile before stream x's next one
-// are done (the two softmax warpgroups take turns on the MUFU).
+// Barriers: Q landed; per stream x (index + x): K / V tile landed, S ready (QK done,
+// which also frees the stream's K buffer), S loaded by the softmax (S may be
+// overwritten), P written to shared memory, PV done (which frees the stream's V and P
+// buffers and means O_x holds every finished tile), the other stream's exponentials
+// for the preceding tile done (kTok0: the two softmax warpgroups take turns on the
+// MUFU), drain; and the last PV of both streams.
 enum : int {
-  kQFull = 0, kKFull0 = 1, kVFull0 = 3, kSFull0 = 5, kPFull0 = 7, kVEmpty0 = 9, kDrain0 = 11,
-  kTok0 = 13, kOFinal = 15, kNumBars = 16
+  kQFull = 0, kKFull0 = 1, kVFull0 = 3, kSFull0 = 5, kSFree0 = 7, kPFull0 = 9, kVEmpty0 = 11, kTok0 = 13,
+  kDrain0 = 15, kOFinal = 17, kNumBars = 18
 };
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^y on the FMA pipe (a share of the exponentials, so that the MUFU is not the only
+// unit doing them).  Range reduction y = j + f, j = round(y) by the round-to-nearest
+// add of 1.5 * 2^23 (exact for |y| < 2^22), f = y - j in [-1/2, 1/2]; 2^f by a cubic
+// with p(0) = 1 whose three coefficients are a least-squares minimax fit of 2^f on
+// [-1/2, 1/2] (max relative error 1.0e-4, below the bf16 rounding of P); j is added to
+// the exponent field.  y is clamped at -127: there j = -127, f = 0, p = 1 and the
+// exponent add gives +0 exactly, so masked keys (y = -inf) still weigh nothing.
+constexpr float kExp2C1 = 0.6932829022407532f;
+constexpr float kExp2C2 = 0.2422109693288803f;
+constexpr float kExp2C3 = 0.05500893294811249f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+__device__ __forceinline__ float exp2_fma(float y) {
+  y = fmaxf(y, -127.0f);
+  const float t = __fadd_rn(y, kRoundMagic);
+  const float f = __fsub_rn(y, __fsub_rn(t, kRoundMagic));
+  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, 1.0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+// Of every 8 column pairs of a row, this many take exp2_fma, the rest the MUFU.
+constexpr int kFmaExpPairs = 0;
+// The two softmax warpgroups take turns on their exponentials (else they overlap).
+constexpr bool kAlternateExp = false;
+
+// Packed pairs of fp32 (one f32x2 instruction does two lanes' worth of FMA / add).
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f32x2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
@@ -82,7 +139,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 template <bool DENSE>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, int N, int G, int k, const int* __restrict__ key_perm,
+                   const __grid_constant__ CUtensorMap tmV, int N, int G, int k,
                    const int* __restrict__ key_gsize, const int* __restrict__ query_perm,
                    const int* __restrict__ qblock_size, const int* __restrict__ route, float scale_log2,
                    float* __restrict__ out, int* __restrict__ status) {
@@ -90,14 +147,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ __align__(8) uint64_t bars[kNumBars];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
-  __shared__ float2 s_ml[2][128];  // per stream and row: final (max, sum)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = blockIdx.x, head = blockIdx.y;
+  // shared memory: Q, then per stream x a K, a V and a P tile (128 x 128 bf16 each,
+  // 128B-swizzled, 1024-byte aligned)
   const uint32_t sbase = (tc::saddr(dsmem) + 1023u) & ~1023u;
   const uint32_t sQ = sbase;
-  const uint32_t sK0 = sbase + kTile;      // K buffer of stream x: sK0 + x kTile
-  const uint32_t sV0 = sbase + 3 * kTile;  // V buffer of stream x: sV0 + x kTile
+  auto sK = [&](int x) { return sbase + (1 + x) * kTile; };
+  auto sV = [&](int x) { return sbase + (3 + x) * kTile; };
+  auto sP = [&](int x) { return sbase + (5 + x) * kTile; };
+  uint8_t* const gsP0 = dsmem + (sP(0) - tc::saddr(dsmem));  // generic pointer to stream 0's P tile
   auto bar = [&](int i) { return tc::saddr(&bars[i]); };
 
   if (tid == 0) {
@@ -106,10 +166,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc::mbar_init(bar(kKFull0 + x), 1);
       tc::mbar_init(bar(kVFull0 + x), 1);
       tc::mbar_init(bar(kSFull0 + x), 1);
+      tc::mbar_init(bar(kSFree0 + x), 128);
       tc::mbar_init(bar(kPFull0 + x), 128);
       tc::mbar_init(bar(kVEmpty0 + x), 1);
-      tc::mbar_init(bar(kDrain0 + x), 1);
       tc::mbar_init(bar(kTok0 + x), 128);
+      tc::mbar_init(bar(kDrain0 + x), 1);
     }
     tc::mbar_init(bar(kOFinal), 2);
     abort_flag = 0;
@@ -131,31 +192,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int* qperm = DENSE ? nullptr : query_perm + (goff + b) * 128;
   const int n_tiles = DENSE ? G : k;
   const int* my_route = DENSE ? nullptr : route + (goff + b) * k;
-  // per-tile key group and its size, staged once (the producers and the softmax read them)
-  int* s_group = reinterpret_cast<int*>(dsmem + (sbase - tc::saddr(dsmem)) + 5 * kTile);
-  int* s_size = s_group + n_tiles;
-  for (int j = tid; j < n_tiles; j += kTcThreads) {
-    const int g = DENSE ? j : __ldg(my_route + j);
-    s_group[j] = g;
-    s_size[j] = DENSE ? min(128, N - g * 128) : __ldg(key_gsize + goff + g);
-  }
-  __syncthreads();
+  // key group of routed tile j and its number of members
+  auto group_of = [&](int j) { return DENSE ? j : __ldg(my_route + j); };
+  auto size_of = [&](int g) { return DENSE ? min(128, N - g * 128) : __ldg(key_gsize + goff + g); };
   volatile int* abort_v = &abort_flag;
 
   if (warp < 4) {
     tc::setmaxnreg_dec<kRegLow>();
     if (warp < 2) {
       // ------------------------------------------------------------------ producers
-      // Q: lane l gathers rows 4 l .. 4 l + 3 through the query permutation (two gather4
-      // per lane, one per 64-column half of the swizzled tile).  K / V: one lane loads
-      // each routed group as two 64-column x 128-row boxes.
-      const int rq = 4 * lane;
-      auto gather_tile = [&](const CUtensorMap* tm, uint32_t dst, const int4& t, uint32_t full) {
-        tc::tma_gather4(dst + rq * 128, tm, 0, t.x, t.y, t.z, t.w, full);
-        tc::tma_gather4(dst + 128 * 128 + rq * 128, tm, 64, t.x, t.y, t.z, t.w, full);
-      };
-      const int x = warp;  // stream whose K and V tiles this warp loads
-      if (x == 0) {
+      if (warp == 0) {
+        // Q: lane l gathers rows 4 l .. 4 l + 3 through the query permutation (two
+        // gather4 per lane, one per 64-column half of the swizzled tile).
+        const int rq = 4 * lane;
         int4 t;
         if (DENSE) {
           const int base = row0 + b * 128;
@@ -169,55 +218,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         if (lane == 0) tc::mbar_arrive_expect_tx(bar(kQFull), kTile);
         __syncwarp();
-        gather_tile(&tmQ, sQ, t, bar(kQFull));
+        tc::tma_gather4(sQ + rq * 128, &tmQ, 0, t.x, t.y, t.z, t.w, bar(kQFull));
+        tc::tma_gather4(sQ + 128 * 128 + rq * 128, &tmQ, 64, t.x, t.y, t.z, t.w, bar(kQFull));
       }
-      // first row of key group g in the K / V maps: the token order itself (dense) or the
-      // group-ordered copies (sparse)
+      // K (warp 0) and V (warp 1) of each routed group, tile after tile, into the buffer
+      // of the tile's stream: two 64-column x 128-row boxes of the group-ordered copies
+      // (sparse) or of K and V in token order (dense).  K of a stream's next tile waits
+      // only for the stream's previous QK, V only for its previous PV.
+      const bool isK = warp == 0;
       const int kvrow0 = DENSE ? row0 : head * G * 128;
-      const uint32_t sK = sK0 + x * kTile, sV = sV0 + x * kTile;
-      int issued = 0;  // tiles of this stream whose copies were issued
-      for (int j = x; j < n_tiles; j += 2) {
-        const int it = j >> 1;
-        const int row = kvrow0 + s_group[j] * 128;
-        // K buffer free once S of the stream's previous tile is ready
-        if (it >= 1 && !warp_wait(bar(kSFull0 + x), (it - 1) & 1, abort_v, status)) break;
+      const CUtensorMap* tm = isK ? &tmK : &tmV;
+      const int full0 = isK ? kKFull0 : kVFull0;
+      // the stream's buffer is free once its previous QK (K) or PV (V) is done
+      const int free0 = isK ? kSFull0 : kVEmpty0;
+      int issued = 0;  // tiles whose copies were issued
+      int g_next = n_tiles > 0 ? group_of(0) : 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int xs = j & 1, it = j >> 1;
+        const int row = kvrow0 + g_next * 128;
+        if (j + 1 < n_tiles) g_next = group_of(j + 1);
+        if (it >= 1 && !warp_wait(bar(free0 + xs), (it - 1) & 1, abort_v, status)) break;
         if (lane == 0) {
-          tc::mbar_arrive_expect_tx(bar(kKFull0 + x), kTile);
-          tc::tma_load_2d(sK, &tmK, 0, row, bar(kKFull0 + x));
-          tc::tma_load_2d(sK + 128 * 128, &tmK, 64, row, bar(kKFull0 + x));
+          const uint32_t dst = isK ? sK(xs) : sV(xs);
+          tc::mbar_arrive_expect_tx(bar(full0 + xs), kTile);
+          tc::tma_load_2d(dst, tm, 0, row, bar(full0 + xs));
+          tc::tma_load_2d(dst + 128 * 128, tm, 64, row, bar(full0 + xs));
         }
-        // V buffer free once the stream's previous PV is done
-        if (it >= 1 && !warp_wait(bar(kVEmpty0 + x), (it - 1) & 1, abort_v, status)) {
-          issued = -(it + 1);  // K of this tile is in flight, V is not
-          break;
-        }
-        if (lane == 0) {
-          tc::mbar_arrive_expect_tx(bar(kVFull0 + x), kTile);
-          tc::tma_load_2d(sV, &tmV, 0, row, bar(kVFull0 + x));
-          tc::tma_load_2d(sV + 128 * 128, &tmV, 64, row, bar(kVFull0 + x));
-        }
-        __syncwarp();
-        issued = it + 1;
+        issued = j + 1;
       }
       // Copies still in flight after an abort must land before the CTA exits: wait
-      // (bounded) for the stream's last K and V phases and for Q.  On the normal path
-      // these phases completed long ago and the waits return at once.
+      // (bounded) for the last phase of each stream's buffer and for Q.  On the normal
+      // path these phases completed long ago and the waits return at once.
       if (lane == 0) {
-        const int nk = issued >= 0 ? issued : -issued, nv = issued >= 0 ? issued : -issued - 1;
-        if (nk > 0) drain_wait(bar(kKFull0 + x), (nk - 1) & 1);
-        if (nv > 0) drain_wait(bar(kVFull0 + x), (nv - 1) & 1);
-        if (x == 0) drain_wait(bar(kQFull), 0);
+        for (int j = max(0, issued - 2); j < issued; ++j) drain_wait(bar(full0 + (j & 1)), (j >> 1) & 1);
+        if (isK) drain_wait(bar(kQFull), 0);
       }
       __syncwarp();
     } else if (lane == 0) {
       // ------------------------------------------------------------------ MMA issuers
-      // warp 2 lane 0 drives stream 0, warp 3 lane 0 stream 1: while one waits or
-      // commits, the other's MMAs keep the tensor pipe busy.
+      // Lane 0 of warp 2 + x drives stream x.  Per tile: as soon as the softmax has
+      // loaded S, S of the stream's next tile is computed (it overlaps the softmax);
+      // then O_x += P V with P from shared memory.
       const int x = warp - 2;
-      constexpr uint32_t kIdQK = tc::idesc_bf16(128, 128, false, false);
+      constexpr uint32_t kIdMma = tc::idesc_bf16(128, 128, false, false);
       constexpr uint32_t kIdPV = tc::idesc_bf16(128, 128, false, true);
       const uint32_t tS = tbase + 128 * x, tO = tbase + 256 + 128 * x;
-      const uint32_t sK = sK0 + x * kTile, sV = sV0 + x * kTile;
+      const int n_x = n_tiles > x ? (n_tiles - x + 1) / 2 : 0;  // tiles of this stream
       bool ok = tc::mbar_wait(bar(kQFull), 0, abort_v, status);
       auto issue_s = [&](int it) -> bool {
         if (!tc::mbar_wait(bar(kKFull0 + x), it & 1, abort_v, status)) return false;
@@ -225,24 +271,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          tc::mma_ss(tS, tc::sdesc_sw128(sQ + koff, 16, 1024), tc::sdesc_sw128(sK + koff, 16, 1024), kIdQK,
+          tc::mma_ss(tS, tc::sdesc_sw128(sQ + koff, 16, 1024), tc::sdesc_sw128(sK(x) + koff, 16, 1024), kIdMma,
                      kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(bar(kSFull0 + x));
         return true;
       };
-      if (ok && x < n_tiles) ok = issue_s(0);
-      for (int j = x, it = 0; ok && j < n_tiles; j += 2, ++it) {
+      if (ok && n_x > 0) ok = issue_s(0);
+      for (int it = 0; ok && it < n_x; ++it) {
+        if (it + 1 < n_x) {
+          // S_x may be overwritten once the softmax holds tile it's scores in registers
+          if (!tc::mbar_wait(bar(kSFree0 + x), it & 1, abort_v, status)) break;
+          tc::fence_after_sync();
+          if (!issue_s(it + 1)) break;
+        }
         if (!tc::mbar_wait(bar(kPFull0 + x), it & 1, abort_v, status)) break;
         tc::fence_after_sync();
         if (!tc::mbar_wait(bar(kVFull0 + x), it & 1, abort_v, status)) break;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          tc::mma_ts(tO, tS + kk * 8, tc::sdesc_sw128(sV + kk * 2048, 128 * 128, 1024), kIdPV,
-                     (it > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          tc::mma_ss(tO, tc::sdesc_sw128(sP(x) + koff, 16, 1024),
+                     tc::sdesc_sw128(sV(x) + kk * 2048, 128 * 128, 1024), kIdPV, (it > 0 || kk > 0) ? 1u : 0u);
         }
         tc::mma_commit(bar(kVEmpty0 + x));
-        if (j + 2 < n_tiles && !issue_s(it + 1)) break;
       }
       tc::mma_commit(bar(kOFinal));
       tc::mma_commit(bar(kDrain0 + x));
@@ -255,11 +307,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int r = 32 * (warp & 3) + lane;
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     const uint32_t sbuf = tbase + lane_off + x * 128;
+    const uint32_t obuf = tbase + lane_off + 256 + x * 128;
     const int tok = r < nq ? (DENSE ? b * 128 + r : __ldg(qperm + r)) : -1;
     float m_run = -kInf, l_run = 0.f;
     bool ok = true;
-    for (int j = x; j < n_tiles; j += 2) {
-      const int it = j >> 1;  // index of this tile within the stream
+    int nv_next = x < n_tiles ? size_of(group_of(x)) : 0;
+    for (int j = x, it = 0; j < n_tiles; j += 2, ++it) {
+      const int nvalid = nv_next;
+      if (j + 2 < n_tiles) nv_next = size_of(group_of(j + 2));  // in flight during this tile
       if (!warp_wait(bar(kSFull0 + x), it & 1, abort_v, status)) {
         ok = false;
         break;
@@ -271,20 +326,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc::tmem_ld32(sbuf + 64, *reinterpret_cast<uint32_t(*)[32]>(&u[64]));
       tc::tmem_ld32(sbuf + 96, *reinterpret_cast<uint32_t(*)[32]>(&u[96]));
       tc::tmem_wait_ld();
-      const int nvalid = s_size[j];
+      tc::fence_before_sync();
+      tc::mbar_arrive(bar(kSFree0 + x));  // S_x may now take the stream's next tile
       if (nvalid < 128) {  // short group (warp-uniform): mask the padding keys
 #pragma unroll
         for (int c = 0; c < 128; ++c)
           if (c >= nvalid) u[c] = __float_as_uint(-kInf);
       }
-      // row max as a tree of 8 independent chains
+      // row max: 8 independent chains of 3-input maxima
       float mx8[8];
 #pragma unroll
       for (int t = 0; t < 8; ++t) mx8[t] = __uint_as_float(u[t]);
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(u[c]));
-      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      for (int c = 8; c < 128; c += 2)
+        mx8[(c >> 1) & 7] = fmax3(mx8[(c >> 1) & 7], __uint_as_float(u[c]), __uint_as_float(u[c + 1]));
+      float mx = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
       mx *= scale_log2;
       const bool grow = mx > m_run + kRescaleLog2;
       const bool need_o = grow && m_run != -kInf;
@@ -294,14 +350,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         l_run *= alpha;
         m_run = mx;
       }
+      // Take turns with the other stream: tile j starts its exponentials once tile j - 1
+      // (the other stream's) has finished them, so that one warpgroup's MUFU phase runs
+      // while the other stream's MMAs do.
+      if (kAlternateExp && j >= 1 && !warp_wait(bar(kTok0 + x), (x == 1 ? it : it - 1) & 1, abort_v, status)) {
+        ok = false;
+        break;
+      }
+      // The P tile is free, and O_x holds every earlier tile, once the previous PV is done.
+      if (it >= 1 && !warp_wait(bar(kVEmpty0 + x), (it - 1) & 1, abort_v, status)) {
+        ok = false;
+        break;
+      }
       if (__any_sync(0xffffffffu, need_o)) {
-        // O_x holds tiles up to j - 2 once that tile's PV has completed
-        if (!warp_wait(bar(kVEmpty0 + x), (it - 1) & 1, abort_v, status)) {
-          ok = false;
-          break;
-        }
         tc::fence_after_sync();
-        const uint32_t obuf = tbase + lane_off + 256 + x * 128;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t o[32];
@@ -311,47 +373,61 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
           tc::tmem_st32(obuf + q * 32, o);
         }
-      }
-      // Take turns with the other stream: tile j starts its exponentials once tile j - 1
-      // (the other stream's) has finished them, so that one warpgroup's MUFU phase runs
-      // while the other stream's MMAs do.
-      if (j >= 1 && !warp_wait(bar(kTok0 + x), (x == 1 ? it : it - 1) & 1, abort_v, status)) {
-        ok = false;
-        break;
+        tc::tmem_wait_st();
       }
       const float msafe = m_run == -kInf ? 0.f : m_run;
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint64_t sc2 = f32x2(scale_log2, scale_log2), nm2 = f32x2(-msafe, -msafe);
+      uint64_t acc2[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2(fmaf(__uint_as_float(u[half * 64 + 2 * i]), scale_log2, -msafe));
-          const float p1 = ex2(fmaf(__uint_as_float(u[half * 64 + 2 * i + 1]), scale_log2, -msafe));
-          sum4[i & 3] += p0 + p1;
+          const int c = half * 64 + 2 * i;
+          float y0, y1;
+          f32x2_split(ffma2(f32x2(__uint_as_float(u[c]), __uint_as_float(u[c + 1])), sc2, nm2), y0, y1);
+          float p0, p1;
+          if ((i & 7) < kFmaExpPairs) {
+            p0 = exp2_fma(y0);
+            p1 = exp2_fma(y1);
+          } else {
+            p0 = ex2(y0);
+            p1 = ex2(y1);
+          }
+          acc2[i & 1] = fadd2(acc2[i & 1], f32x2(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
-        tc::tmem_st32(sbuf + half * 32, pk);
+        // row r of the 128B-swizzled P tile (K-major A operand of the PV MMA)
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8)
+          st_shared_v4(sP(x) + tc::sw128_offset(r, half * 8 + c8), pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2],
+                       pk[4 * c8 + 3]);
       }
-      if (j + 1 < n_tiles) tc::mbar_arrive(bar(kTok0 + (x ^ 1)));
+      if (kAlternateExp && j + 1 < n_tiles) tc::mbar_arrive(bar(kTok0 + (x ^ 1)));
+      float sum4[4];
+      f32x2_split(acc2[0], sum4[0], sum4[1]);
+      f32x2_split(acc2[1], sum4[2], sum4[3]);
       l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-      tc::tmem_wait_st();
+      tc::fence_proxy_async();  // P (generic-proxy stores) visible to the tensor core
       tc::fence_before_sync();
       tc::mbar_arrive(bar(kPFull0 + x));
     }
     // ---- merge the two streams; warpgroup x writes columns [64 x, 64 x + 64)
-    s_ml[x][r] = make_float2(m_run, l_run);
+    const bool fin = ok && warp_wait(bar(kOFinal), 0, abort_v, status);
+    // every PV is done: the P tiles are free and hold each row's (max, sum) per stream
+    float2* s_ml = reinterpret_cast<float2*>(gsP0);
+    if (fin) s_ml[x * 128 + r] = make_float2(m_run, l_run);
     tc::named_bar_sync(1, 256);  // every softmax thread reaches this exactly once
-    const float2 a0 = s_ml[0][r], a1 = s_ml[1][r];
-    const float mm = fmaxf(a0.x, a1.x);
-    const float f0 = a0.x == -kInf ? 0.f : ex2(a0.x - mm);
-    const float f1 = a1.x == -kInf ? 0.f : ex2(a1.x - mm);
-    const float den = a0.y * f0 + a1.y * f1;
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    const float g0 = f0 * inv, g1 = f1 * inv;
-    const bool has1 = n_tiles > 1;  // stream 1 never wrote O1 otherwise
-    if (ok && warp_wait(bar(kOFinal), 0, abort_v, status)) {
+    if (fin) {
       tc::fence_after_sync();
+      const float2 a0 = s_ml[r], a1 = s_ml[128 + r];
+      const float mm = fmaxf(a0.x, a1.x);
+      const float f0 = a0.x == -kInf ? 0.f : ex2(a0.x - mm);
+      const float f1 = a1.x == -kInf ? 0.f : ex2(a1.x - mm);
+      const float den = a0.y * f0 + a1.y * f1;
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      const float g0 = f0 * inv, g1 = f1 * inv;
+      const bool has1 = n_tiles > 1;  // stream 1 never wrote O1 otherwise
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         const int col = 64 * x + 32 * q;
@@ -415,7 +491,8 @@ __global__ void __launch_bounds__(256) kv_group_kernel(const uint4* __restrict__
 
 }  // namespace
 
-size_t attn_tc_smem_bytes(int n_tiles) { return 5ull * kTile + 1024 + 8ull * n_tiles; }
+// Q, and a K, a V and a P tile per stream, plus the 1024-byte alignment slack.
+size_t attn_tc_smem_bytes(int) { return 7ull * kTile + 1024; }
 
 namespace {
 
@@ -448,6 +525,36 @@ bool bf16_map(CUtensorMap* m, const void* base, long long rows, int box_rows) {
 
 }  // namespace
 
+namespace {
+std::mutex g_timing_mu;
+bool g_timing_on = false;
+std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_timing_pairs;  // recorded, not yet read
+std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_timing_free;   // reusable
+}  // namespace
+
+void attn_timing_enable(bool on) {
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  g_timing_on = on;
+}
+
+cudaError_t attn_timing_read(double* ms_total, long long* launches) {
+  std::lock_guard<std::mutex> lk(g_timing_mu);
+  double total = 0.0;
+  cudaError_t err = cudaSuccess;
+  for (auto& pr : g_timing_pairs) {
+    cudaError_t e = cudaEventSynchronize(pr.second);
+    float ms = 0.f;
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, pr.first, pr.second);
+    if (e != cudaSuccess && err == cudaSuccess) err = e;
+    total += ms;
+    g_timing_free.push_back(pr);
+  }
+  if (launches) *launches = static_cast<long long>(g_timing_pairs.size());
+  g_timing_pairs.clear();
+  if (ms_total) *ms_total = total;
+  return err;
+}
+
 cudaError_t launch_attention_tc(const AttnArgs& a, bool dense, int* status, cudaStream_t st) {
   const size_t smem = attn_tc_smem_bytes(dense ? a.G : a.k);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
@@ -476,10 +583,30 @@ cudaError_t launch_attention_tc(const AttnArgs& a, bool dense, int* status, cuda
     e = counted(cudaGetLastError(), 1);
     if (e != cudaSuccess) return e;
   }
-  kern<<<dim3(a.G, a.heads), kTcThreads, smem, st>>>(tq, tk, tv, a.N, a.G, a.k, a.key_perm, a.key_gsize,
+  std::pair<cudaEvent_t, cudaEvent_t> ev{nullptr, nullptr};
+  {
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    if (g_timing_on) {
+      if (!g_timing_free.empty()) {
+        ev = g_timing_free.back();
+        g_timing_free.pop_back();
+      } else if (cudaEventCreate(&ev.first) != cudaSuccess || cudaEventCreate(&ev.second) != cudaSuccess) {
+        return cudaErrorMemoryAllocation;
+      }
+    }
+  }
+  if (ev.first != nullptr && (e = cudaEventRecord(ev.first, st)) != cudaSuccess) return e;
+  kern<<<dim3(a.G, a.heads), kTcThreads, smem, st>>>(tq, tk, tv, a.N, a.G, a.k, a.key_gsize,
                                                        a.query_perm, a.qblock_size, a.route, a.scale_log2, a.out,
                                                        status);
-  return counted(cudaGetLastError(), 1);
+  e = counted(cudaGetLastError(), 1);
+  if (ev.first != nullptr) {
+    cudaError_t e2 = cudaEventRecord(ev.second, st);
+    std::lock_guard<std::mutex> lk(g_timing_mu);
+    g_timing_pairs.push_back(ev);
+    if (e == cudaSuccess) e = e2;
+  }
+  return e;
 }
 
 }  // namespace spr

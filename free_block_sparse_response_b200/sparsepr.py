@@ -26,6 +26,7 @@ EXPORTED_SYMBOLS = (
     "sparsepr_probe_dense", "sparsepr_fit_residual", "sparsepr_apply_residual", "sparsepr_check",
     "sparsepr_last_error", "sparsepr_test_fill_workspace_size", "sparsepr_test_fill",
     "sparsepr_test_topk", "sparsepr_row_errors", "sparsepr_launch_count", "sparsepr_fit_residual_noalloc",
+    "sparsepr_kernel_timing", "sparsepr_kernel_timing_read",
 )
 
 
@@ -99,6 +100,8 @@ def lib() -> ctypes.CDLL:
         "sparsepr_test_topk": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
         "sparsepr_row_errors": (ctypes.c_int, [_vp, ctypes.c_int, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
         "sparsepr_launch_count": (ctypes.c_uint64, []),
+        "sparsepr_kernel_timing": (ctypes.c_int, [ctypes.c_int]),
+        "sparsepr_kernel_timing_read": (ctypes.c_int, [_vp, _vp]),
         "sparsepr_fit_residual_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, ctypes.c_double,
                                                          _i32, _i32, _vp, _vp, _vp]),
     }
@@ -321,6 +324,19 @@ def row_errors(o: torch.Tensor, o_ref: torch.Tensor, probe_idx: Optional[torch.T
     _call("sparsepr_row_errors", _p(o), _DTYPE_CODE[o.dtype], _p(o_ref), _p(probe_idx), bt, h, n, d, p, _p(err),
           _stream(o))
     return err
+
+
+def kernel_timing(enable: bool) -> None:
+    """Record CUDA events around every later attention kernel (measurement hook)."""
+    _call("sparsepr_kernel_timing", 1 if enable else 0)
+
+
+def kernel_timing_read():
+    """(summed ms, launches) of the attention kernels timed since the last read."""
+    ms = ctypes.c_double(0.0)
+    n = ctypes.c_int64(0)
+    _call("sparsepr_kernel_timing_read", ctypes.byref(ms), ctypes.byref(n))
+    return ms.value, n.value
 
 
 def launch_count() -> int:

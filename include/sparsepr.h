@@ -217,6 +217,16 @@ SPARSEPR_API int sparsepr_row_errors(const void* O, int o_dtype, const float* O_
 /* Number of kernels this library has enqueued since it was loaded (host counter). */
 SPARSEPR_API uint64_t sparsepr_launch_count(void);
 
+/* Measurement hook for the tensor-core attention kernels.  sparsepr_kernel_timing(1)
+ * makes every later sparse or dense attention call record a CUDA event pair on its
+ * stream immediately around the attention kernel itself (the sparse path's copy of K
+ * and V into group order is outside the pair); sparsepr_kernel_timing(0) stops it.
+ * sparsepr_kernel_timing_read waits for the recorded pairs, returns their summed device
+ * time in milliseconds and their number, and forgets them.  Process-wide state meant
+ * for timing runs (not for concurrent callers); errors: SPARSEPR_ERR_CUDA. */
+SPARSEPR_API int sparsepr_kernel_timing(int enable);
+SPARSEPR_API int sparsepr_kernel_timing_read(double* ms_total, int64_t* launches);
+
 /* Wait for `stream` and return the device status word in `ws` (SPARSEPR_OK, or the
  * first device-side error since the last sparsepr_partition).  This is the only call
  * that synchronises. */
