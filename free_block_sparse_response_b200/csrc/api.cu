@@ -52,7 +52,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct Layout {
   size_t header = 0, sample_idx, gamma, gamma_hi, gamma_lo, nrm, cent_k, cent_q, wf, whi, wlo, eg, dmat,
          prop_g0, prop_v0, labels, room, cnt, offs, cursor, closed, bucket, list0, list1, list_len, prop_g, prop_v,
-         perm_tmp, perm_cursor, qblk, partial, fit, kv_grouped, total;
+         perm_tmp, perm_cursor, qblk, partial, fit, kv_grouped, segmin, total;
 };
 
 Layout make_layout(int heads, int N, int d, int block, int S, int P) {
@@ -81,6 +81,7 @@ Layout make_layout(int heads, int N, int d, int block, int S, int P) {
   L.wlo = take(2 * H * G * D);
   L.eg = take(sizeof(float) * H * G);
   L.dmat = take(sizeof(float) * H * n * ((G + 3) / 4 * 4));
+  L.segmin = take(sizeof(unsigned long long) * H * n * 2 * ((G + 127) / 128));
   L.prop_g0 = take(sizeof(int) * H * n);
   L.prop_v0 = take(sizeof(float) * H * n);
   L.labels = take(sizeof(int) * H * n);
@@ -210,6 +211,10 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
   fa.ldd = (G + 3) / 4 * 4;
   fa.prop_g0 = at<int>(ws, L.prop_g0);
   fa.prop_v0 = at<float>(ws, L.prop_v0);
+  // segment minima come from the tensor-core distance kernel (bf16, d = 128)
+  const bool seg = !f32 && d == 128;
+  fa.nseg = 2 * spr::ceil_div(G, 128);
+  fa.seg_min = seg ? at<unsigned long long>(ws, L.segmin) : nullptr;
   fa.heads = heads;
   fa.n = N;
   fa.G = G;
@@ -259,6 +264,8 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
       ra.ldd = fa.ldd;
       ra.prop_g = at<int>(ws, L.prop_g0);
       ra.prop_v = at<float>(ws, L.prop_v0);
+      ra.seg_min = seg ? at<unsigned long long>(ws, L.segmin) : nullptr;
+      ra.nseg = fa.nseg;
       ra.nrm_out = nullptr;
       SPR_CUDA(spr::launch_rowgemm(ra, true, st), "distances");
       SPR_CUDA(spr::launch_fill(fa, st), "capacity fill");
@@ -484,11 +491,11 @@ size_t sparsepr_test_fill_workspace_size(int32_t H, int32_t n, int32_t G) {
   return align_up(sizeof(spr::WorkspaceHeader)) + align_up(4 * h * g * sizeof(int)) +
          align_up(h * ((g + 31) / 32) * sizeof(unsigned int)) +
          align_up(h * nn * sizeof(unsigned long long)) + 3 * align_up(h * nn * sizeof(int)) + align_up(4 * sizeof(int)) +
-         align_up(h * nn * sizeof(float));
+         align_up(h * nn * sizeof(float)) + align_up(h * nn * 2 * ((g + 127) / 128) * sizeof(unsigned long long));
 }
 
-int sparsepr_test_fill(const float* D, int32_t H, int32_t n, int32_t G, int32_t cap, int32_t* labels, void* ws,
-                       sparsepr_stream_t stream) {
+static int test_fill_common(const float* D, int32_t H, int32_t n, int32_t G, int32_t cap, int32_t* labels, void* ws,
+                            sparsepr_stream_t stream, bool segmented) {
   if (!D || !labels || !ws || H < 1 || n < 1 || G < 1 || cap < 1)
     return fail(SPARSEPR_ERR_INVALID_ARG, "bad fill arguments");
   if (static_cast<long long>(G) * cap < n) return fail(SPARSEPR_ERR_INVALID_ARG, "G * cap < n");
@@ -523,10 +530,26 @@ int sparsepr_test_fill(const float* D, int32_t H, int32_t n, int32_t G, int32_t 
   fa.prop_g = at<int>(ws, take(h * nn * sizeof(int)));
   fa.list_len = at<int>(ws, take(4 * sizeof(int)));
   fa.prop_v = at<float>(ws, take(h * nn * sizeof(float)));
+  fa.nseg = 2 * spr::ceil_div(G, 128);
+  unsigned long long* seg = at<unsigned long long>(ws, take(h * nn * fa.nseg * sizeof(unsigned long long)));
+  fa.seg_min = segmented ? seg : nullptr;
   fa.hdr = header(ws);
   SPR_CUDA(cudaMemsetAsync(ws, 0, sizeof(spr::WorkspaceHeader), st), "fill: reset status");
+  if (segmented)
+    SPR_CUDA(spr::launch_segment_minima(D, G, static_cast<long long>(H) * n, G, seg, fa.nseg, &fa.hdr->status, st),
+             "segment minima");
   SPR_CUDA(spr::launch_fill(fa, st), "fill");
   return SPARSEPR_OK;
+}
+
+int sparsepr_test_fill(const float* D, int32_t H, int32_t n, int32_t G, int32_t cap, int32_t* labels, void* ws,
+                       sparsepr_stream_t stream) {
+  return test_fill_common(D, H, n, G, cap, labels, ws, stream, false);
+}
+
+int sparsepr_test_fill_segmented(const float* D, int32_t H, int32_t n, int32_t G, int32_t cap, int32_t* labels,
+                                 void* ws, sparsepr_stream_t stream) {
+  return test_fill_common(D, H, n, G, cap, labels, ws, stream, true);
 }
 
 int sparsepr_test_topk(const float* Sc, int32_t H, int32_t Gq, int32_t G, int32_t k, int32_t* route, void* ws,

@@ -5,32 +5,33 @@
 // support.  One CTA per (query block of 128 rows, head); head dim 128; key groups of 128.
 //
 // The routed tiles j = 0 .. n-1 of a block are split into two streams, even and odd j.
-// Each stream keeps its own S tile, running max / sum and O accumulator, so that the
-// two softmax warpgroups work on different tiles at the same time (one keeps the MUFU
-// busy while the other loads, reduces or stores); the two partial results are merged
-// at the end like a split-K softmax: O = (2^(m0-m) O0 + 2^(m1-m) O1) / (2^(m0-m) l0 +
-// 2^(m1-m) l1), m = max(m0, m1).
+// Each stream keeps its own S tile (TMEM), P tile (shared memory), running max / sum
+// and O accumulator (TMEM), so that the two softmax warpgroups work on different tiles
+// at the same time; the two partial results are merged at the end like a split-K
+// softmax: O = (2^(m0-m) O0 + 2^(m1-m) O1) / (2^(m0-m) l0 + 2^(m1-m) l1), m = max(m0, m1).
+// Within a stream, S is released as soon as the softmax holds it in registers, so QK of
+// the stream's next tile runs while the softmax of the current one computes P.
 //
 // Warp roles (384 threads, one CTA per SM):
-//   warps 0-1   producers, warp x feeds stream x: TMA loads of its routed groups as two
-//               64-column x 128-row boxes of the group-ordered K and V copies (sparse) or
-//               of K and V themselves (dense), into that stream's own K and V buffers;
-//               warp 0 also gathers the block's Q rows through the query permutation
-//               (tile::gather4, 4 token rows per instruction; pad rows of a short block
-//               repeat its first member).
-//   warps 2-3   MMA issuers, lane 0 of warp 2 + x drives stream x: S_x = Q K_j^T into
-//               TMEM, then O_x += P_j V_j with P read from TMEM, then S_x for the next
-//               tile of the stream.  With one issuer per stream, one stream's waits and
-//               commits overlap the other stream's MMAs.
+//   warp 0      gathers the block's Q rows through the query permutation (tile::gather4,
+//               4 token rows per instruction; pad rows of a short block repeat its first
+//               member), then loads K of every routed tile; warp 1 loads V.  Each tile is
+//               two 64-column x 128-row TMA boxes of the group-ordered K / V copies
+//               (sparse) or of K / V in token order (dense), into the buffer of its stream.
+//   warps 2-3   MMA issuers, lane 0 of warp 2 + x drives stream x: S_x = Q K^T (TMEM),
+//               and O_x += P V with P from shared memory.  With one issuer per stream,
+//               one stream's waits and commits overlap the other stream's MMAs.
 //   warps 4-7   softmax, stream 0; warps 8-11 softmax, stream 1.  Thread i of a
 //               warpgroup owns TMEM lane i (query row i); it reads S, keeps the running
-//               max / sum, writes P (bf16) back over S, rescales its O only when the row
-//               max grew by more than 2^8 (stale maxima are exact after the final
-//               division), and at the end merges the two streams for half the columns.
+//               max / sum, writes P (bf16) into the 128B-swizzled P tile, rescales its O
+//               only when the row max grew by more than 2^8 (stale maxima are exact after
+//               the final division), and at the end merges the two streams for half the
+//               columns.
 // Warps 0-3 give registers to the softmax warpgroups (setmaxnreg).
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+// Shared memory: Q, and per stream one K, one V and one P tile (7 x 32 KB).
 // Every wait is bounded; on timeout the CTA records kErrTimeout, drains its MMAs and
-// frees TMEM before exiting.
+// copies and frees TMEM before exiting.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -57,12 +58,11 @@ constexpr float kInf = __builtin_huge_valf();
 // Barriers: Q landed; per stream x (index + x): K / V tile landed, S ready (QK done,
 // which also frees the stream's K buffer), S loaded by the softmax (S may be
 // overwritten), P written to shared memory, PV done (which frees the stream's V and P
-// buffers and means O_x holds every finished tile), the other stream's exponentials
-// for the preceding tile done (kTok0: the two softmax warpgroups take turns on the
-// MUFU), drain; and the last PV of both streams.
+// buffers and means O_x holds every finished tile), drain; and the last PV of both
+// streams.
 enum : int {
-  kQFull = 0, kKFull0 = 1, kVFull0 = 3, kSFull0 = 5, kSFree0 = 7, kPFull0 = 9, kVEmpty0 = 11, kTok0 = 13,
-  kDrain0 = 15, kOFinal = 17, kNumBars = 18
+  kQFull = 0, kKFull0 = 1, kVFull0 = 3, kSFull0 = 5, kSFree0 = 7, kPFull0 = 9, kVEmpty0 = 11, kDrain0 = 13,
+  kOFinal = 15, kNumBars = 16
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -70,29 +70,6 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-
-// 2^y on the FMA pipe (a share of the exponentials, so that the MUFU is not the only
-// unit doing them).  Range reduction y = j + f, j = round(y) by the round-to-nearest
-// add of 1.5 * 2^23 (exact for |y| < 2^22), f = y - j in [-1/2, 1/2]; 2^f by a cubic
-// with p(0) = 1 whose three coefficients are a least-squares minimax fit of 2^f on
-// [-1/2, 1/2] (max relative error 1.0e-4, below the bf16 rounding of P); j is added to
-// the exponent field.  y is clamped at -127: there j = -127, f = 0, p = 1 and the
-// exponent add gives +0 exactly, so masked keys (y = -inf) still weigh nothing.
-constexpr float kExp2C1 = 0.6932829022407532f;
-constexpr float kExp2C2 = 0.2422109693288803f;
-constexpr float kExp2C3 = 0.05500893294811249f;
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
-__device__ __forceinline__ float exp2_fma(float y) {
-  y = fmaxf(y, -127.0f);
-  const float t = __fadd_rn(y, kRoundMagic);
-  const float f = __fsub_rn(y, __fsub_rn(t, kRoundMagic));
-  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, 1.0f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-// Of every 8 column pairs of a row, this many take exp2_fma, the rest the MUFU.
-constexpr int kFmaExpPairs = 0;
-// The two softmax warpgroups take turns on their exponentials (else they overlap).
-constexpr bool kAlternateExp = false;
 
 // Packed pairs of fp32 (one f32x2 instruction does two lanes' worth of FMA / add).
 __device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
@@ -169,7 +146,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc::mbar_init(bar(kSFree0 + x), 128);
       tc::mbar_init(bar(kPFull0 + x), 128);
       tc::mbar_init(bar(kVEmpty0 + x), 1);
-      tc::mbar_init(bar(kTok0 + x), 128);
       tc::mbar_init(bar(kDrain0 + x), 1);
     }
     tc::mbar_init(bar(kOFinal), 2);
@@ -350,13 +326,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         l_run *= alpha;
         m_run = mx;
       }
-      // Take turns with the other stream: tile j starts its exponentials once tile j - 1
-      // (the other stream's) has finished them, so that one warpgroup's MUFU phase runs
-      // while the other stream's MMAs do.
-      if (kAlternateExp && j >= 1 && !warp_wait(bar(kTok0 + x), (x == 1 ? it : it - 1) & 1, abort_v, status)) {
-        ok = false;
-        break;
-      }
       // The P tile is free, and O_x holds every earlier tile, once the previous PV is done.
       if (it >= 1 && !warp_wait(bar(kVEmpty0 + x), (it - 1) & 1, abort_v, status)) {
         ok = false;
@@ -386,14 +355,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int c = half * 64 + 2 * i;
           float y0, y1;
           f32x2_split(ffma2(f32x2(__uint_as_float(u[c]), __uint_as_float(u[c + 1])), sc2, nm2), y0, y1);
-          float p0, p1;
-          if ((i & 7) < kFmaExpPairs) {
-            p0 = exp2_fma(y0);
-            p1 = exp2_fma(y1);
-          } else {
-            p0 = ex2(y0);
-            p1 = ex2(y1);
-          }
+          const float p0 = ex2(y0), p1 = ex2(y1);
           acc2[i & 1] = fadd2(acc2[i & 1], f32x2(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
@@ -403,7 +365,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           st_shared_v4(sP(x) + tc::sw128_offset(r, half * 8 + c8), pk[4 * c8], pk[4 * c8 + 1], pk[4 * c8 + 2],
                        pk[4 * c8 + 3]);
       }
-      if (kAlternateExp && j + 1 < n_tiles) tc::mbar_arrive(bar(kTok0 + (x ^ 1)));
       float sum4[4];
       f32x2_split(acc2[0], sum4[0], sum4[1]);
       f32x2_split(acc2[1], sum4[2], sum4[3]);

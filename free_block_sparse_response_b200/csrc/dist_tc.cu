@@ -5,8 +5,9 @@
 // the head-dim form of the squared response-space distance used by Response-Coupled
 // Partitioning (SparsePR abstract, arXiv 2608.18484).  w_g enters as bf16 hi + lo, so
 // the cross term carries ~16-bit precision.  The full fp32 row is written (row stride
-// ldd, a multiple of 4) and its argmin (ties to the lower group) is the first proposal
-// of the capacity fill.
+// ldd, a multiple of 4), its argmin (ties to the lower group) is the first proposal of
+// the capacity fill, and the minimum of each 64-column segment is kept for the later
+// proposals.
 //
 // Persistent: one CTA per SM loops over (head, 128-item tile) work items; groups are
 // streamed in chunks of 128 (W double-buffered, cp.async into 128B-swizzled tiles); the
@@ -46,7 +47,8 @@ __global__ void __launch_bounds__(kDtThreads, 1)
     dist_tc_kernel(const __nv_bfloat16* __restrict__ X, int n, const __nv_bfloat16* __restrict__ Whi,
                    const __nv_bfloat16* __restrict__ Wlo, int ncols, int ldd, const float* __restrict__ nrm,
                    const float* __restrict__ ecol, float tau2, float* __restrict__ Dout, int* __restrict__ prop_g,
-                   float* __restrict__ prop_v, int* __restrict__ status, int heads) {
+                   float* __restrict__ prop_v, unsigned long long* __restrict__ seg_min, int nseg,
+                   int* __restrict__ status, int heads) {
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t bars[kDtBars];
   __shared__ uint32_t tmem_slot;
@@ -214,6 +216,8 @@ __global__ void __launch_bounds__(kDtThreads, 1)
         tc::mbar_arrive(bar(kAccEmpty0 + s));
         const int c0 = c * 128 + half * 64;
         const float4* e4 = reinterpret_cast<const float4*>(s_e + c0);
+        float seg_v = kDtInf;  // this 64-column segment's first minimum
+        int seg_c = -1;
 #pragma unroll
         for (int qq = 0; qq < 16; ++qq) {
           const float4 e = e4[qq];
@@ -223,12 +227,20 @@ __global__ void __launch_bounds__(kDtThreads, 1)
             const int j = 4 * qq + t;
             const float v = fmaf(m2t, __uint_as_float(u[j]), tnr) + ev[t];
             u[j] = __float_as_uint(v);
-            if (v < best_v) {
-              best_v = v;
-              best_c = c0 + j;
+            if (v < seg_v) {
+              seg_v = v;
+              seg_c = j;
             }
           }
         }
+        // segments in ascending column order: a strictly smaller minimum wins
+        if (seg_c >= 0 && seg_v < best_v) {
+          best_v = seg_v;
+          best_c = c0 + seg_c;
+        }
+        if (seg_min != nullptr && row < n)
+          seg_min[(static_cast<size_t>(head) * n + row) * nseg + 2 * c + half] =
+              seg_c >= 0 ? dist_key(seg_v, c0 + seg_c) : ~0ull;
         // transpose 32 rows x 32 columns at a time through shared memory: lane l writes its
         // row's chunk k at chunk position k ^ (l & 7) (conflict-free), then reads column l
         // of every row, so each global store covers 128 contiguous bytes of one row
@@ -311,7 +323,7 @@ cudaError_t launch_dist_tc(const RowGemmArgs& a, int ldd, cudaStream_t st) {
   const int total = a.heads * ceil_div(a.n, 128);
   kern<<<std::min(total, sms), kDtThreads, smem, st>>>(
       static_cast<const __nv_bfloat16*>(a.X), a.n, a.Bhi, a.Blo, a.ncols, ldd, a.nrm, a.ecol, a.tau2, a.Dout,
-      a.prop_g, a.prop_v, a.status, a.heads);
+      a.prop_g, a.prop_v, a.seg_min, a.nseg, a.status, a.heads);
   return counted(cudaGetLastError(), 1);
 }
 

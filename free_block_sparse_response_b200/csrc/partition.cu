@@ -548,6 +548,109 @@ __global__ void __launch_bounds__(kFillThreads, 3) fill_coop_kernel(FillArgs a) 
         __syncthreads();
         closed_all = s_closed;
       }
+      if (a.seg_min != nullptr) {
+        // Two items per warp, 16 lanes each; lane s of a half holds the minimum key of its
+        // row's 64-column segment s.  The best open group is the smallest key among the
+        // segment minima whose group is open, unless a segment whose minimum group is
+        // full still has a key below it: only such segments are read (64 values, four per
+        // lane), each read lowering the bound the remaining ones must beat.  Every key of
+        // a segment is >= its minimum key, so the result equals the argmin over the whole
+        // row's open groups.  The segment of the item's previous proposal (a group that
+        // has just filled, and the row's smallest key) is read in the same wave as the
+        // keys, since it nearly always has to be.
+        const int sub = lane & 15;
+        const unsigned int hmask = (lane & 16) ? 0xffff0000u : 0x0000ffffu;
+        for (int x0 = gwarp * 2; x0 < ncur; x0 += nwarps * 2) {
+          const int x = x0 + (lane >> 4);
+          const bool valid = x < ncur;
+          const int item = valid ? __ldcg(L + x) : 0;
+          const int h = item / n;
+          const unsigned int* closed = closed_all + static_cast<size_t>(h) * words;
+          const float* drow = a.D + static_cast<size_t>(item) * a.ldd;
+          auto is_open = [&](int g) { return !((closed[g >> 5] >> (g & 31)) & 1u); };
+          const unsigned long long key =
+              valid && sub < a.nseg ? __ldcg(a.seg_min + static_cast<size_t>(item) * a.nseg + sub) : ~0ull;
+          const int gp = (valid && round > 0) ? __ldcg(a.prop_g + item) : -1;
+          const int sp = gp >= 0 ? (gp >> 7) * 2 + ((gp >> 6) & 1) : -1;
+          float pv[4];
+          const int pcol0 = sp >= 0 ? (sp >> 1) * 128 + (sp & 1) * 64 : 0;
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int g = pcol0 + 16 * t + sub;
+            pv[t] = (sp >= 0 && g < G) ? __ldcg(drow + g) : 0.f;
+          }
+          const int kg = key != ~0ull ? static_cast<int>(key & 0xffffffffu) : -1;
+          const bool kopen = kg >= 0 && is_open(kg);
+          // a segment without a value below +inf (key ~0) is bounded below by +inf at its
+          // first column
+          const int scol0 = (sub >> 1) * 128 + (sub & 1) * 64;
+          const bool has_cols = valid && sub < a.nseg && scol0 < G;
+          const unsigned long long lb =
+              kg >= 0 ? key : (static_cast<unsigned long long>(float_order_key(__int_as_float(0x7f800000))) << 32) |
+                                  static_cast<uint32_t>(scol0);
+          unsigned long long best = kopen ? key : ~0ull;
+          bool saw_nan = false;
+          if (sp >= 0) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const int g = pcol0 + 16 * t + sub;
+              if (g < G && is_open(g)) {
+                saw_nan |= (pv[t] != pv[t]);
+                const unsigned long long kk = decision_key(pv[t], g);
+                best = kk < best ? kk : best;
+              }
+            }
+          }
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) {
+            const unsigned long long y = __shfl_xor_sync(0xffffffffu, best, o);
+            best = y < best ? y : best;
+          }
+          unsigned int need = __ballot_sync(0xffffffffu, has_cols && !kopen && sub != sp && lb < best) & hmask;
+          while (__any_sync(0xffffffffu, need != 0u)) {
+            const int sg = need != 0u ? (__ffs(need) - 1) & 15 : -1;
+            unsigned long long bb = ~0ull;
+            if (sg >= 0) {
+              const int col0 = (sg >> 1) * 128 + (sg & 1) * 64;
+              float vv[4];
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                const int g = col0 + 16 * t + sub;
+                vv[t] = g < G ? __ldcg(drow + g) : 0.f;
+              }
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                const int g = col0 + 16 * t + sub;
+                if (g < G && is_open(g)) {
+                  saw_nan |= (vv[t] != vv[t]);
+                  const unsigned long long kk = decision_key(vv[t], g);
+                  bb = kk < bb ? kk : bb;
+                }
+              }
+            }
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) {
+              const unsigned long long y = __shfl_xor_sync(0xffffffffu, bb, o);
+              bb = y < bb ? y : bb;
+            }
+            best = bb < best ? bb : best;
+            const unsigned int keep = __ballot_sync(0xffffffffu, has_cols && !kopen && sub != sp && lb < best) & hmask;
+            need = sg >= 0 ? (need & keep & ~(1u << (sg + (lane & 16)))) : 0u;
+          }
+          saw_nan = (__ballot_sync(0xffffffffu, saw_nan) & hmask) != 0u && valid;
+          if (sub == 0 && valid) {
+            if (saw_nan) record_error(&a.hdr->status, kErrNonFinite);
+            if (best == ~0ull) {
+              record_error(&a.hdr->status, kErrInvalidArg);
+            } else {
+              const int g = static_cast<int>(best & 0xffffffffu);
+              a.prop_g[item] = g;
+              a.prop_v[item] = float_from_order_key(static_cast<uint32_t>(best >> 32));
+              atomicAdd(a.cnt + static_cast<size_t>(h) * G + g, 1);
+            }
+          }
+        }
+      } else
       // One item per warp, with the item's whole distance row (up to MAXW values per
       // lane) requested before any is used; full-group bitmap words are warp-uniform.
       for (int x = gwarp; x < ncur; x += nwarps) {
@@ -672,6 +775,37 @@ __global__ void __launch_bounds__(kFillThreads, 3) fill_coop_kernel(FillArgs a) 
   }
 }
 
+// Segment minima of a row-major matrix (the convention of the tensor-core distance
+// kernel): per row and 64-column segment, the key of its first minimum among values
+// below +inf, or ~0 when it has none; a NaN is recorded as a non-finite input.  One warp
+// per (row, segment).
+__global__ void segment_minima_kernel(const float* __restrict__ D, int ldd, long long rows, int G,
+                                      unsigned long long* __restrict__ seg, int nseg, int* __restrict__ status) {
+  const int lane = threadIdx.x & 31;
+  const long long total = rows * nseg;
+  for (long long w = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5; w < total;
+       w += (static_cast<long long>(gridDim.x) * blockDim.x) >> 5) {
+    const long long row = w / nseg;
+    const int s = static_cast<int>(w - row * nseg);
+    const int col0 = (s >> 1) * 128 + (s & 1) * 64;
+    unsigned long long b = ~0ull;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int c = col0 + 32 * t + lane;
+      if (c < G) {
+        const float v = D[row * ldd + c];
+        if (v != v) record_error(status, kErrNonFinite);
+        if (v < __int_as_float(0x7f800000)) {
+          const unsigned long long k = decision_key(v, c);
+          b = k < b ? k : b;
+        }
+      }
+    }
+    b = warp_min_u64(b);
+    if (lane == 0) seg[w] = b;
+  }
+}
+
 // ----------------------------------------------------------------- labels -> permutation
 __global__ void perm_scatter_kernel(const int* __restrict__ labels, int n, int G, int cap,
                                     int* __restrict__ cursor, int* __restrict__ tmp, int heads,
@@ -740,6 +874,12 @@ __global__ void block_score_kernel(const float* __restrict__ qbar, const float* 
 }
 
 // ----------------------------------------------------------------------------- launchers
+
+cudaError_t launch_segment_minima(const float* D, int ldd, long long rows, int G, unsigned long long* seg, int nseg,
+                                  int* status, cudaStream_t st) {
+  segment_minima_kernel<<<1024, 256, 0, st>>>(D, ldd, rows, G, seg, nseg, status);
+  return counted(cudaGetLastError(), 1);
+}
 
 cudaError_t launch_midpoint_stride(int* idx, int n, int count, cudaStream_t st) {
   midpoint_stride_kernel<<<ceil_div(count, 256), 256, 0, st>>>(idx, n, count);

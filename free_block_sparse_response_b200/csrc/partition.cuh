@@ -23,6 +23,11 @@ struct RowGemmArgs {
   int ldd;                   // DIST: row stride of Dout (>= ncols)
   int* prop_g;               // DIST: [heads, n]
   float* prop_v;
+  // DIST, tensor-core path (optional): per item the minimum key of every 64-column
+  // segment of its row, [heads, n, nseg], nseg = 2 ceil(ncols / 128); ~0 for a segment
+  // without a finite value.  A key is order_key(D) << 32 | column.
+  unsigned long long* seg_min;
+  int nseg;
   float* nrm_out;            // NORM: [heads, n]
   int* status;
 };
@@ -32,6 +37,11 @@ struct FillArgs {
   int ldd;              // row stride of D (>= G)
   const int* prop_g0;   // optional first proposals [heads, n]
   const float* prop_v0;
+  // optional segment minima of every D row (see RowGemmArgs::seg_min): later proposals
+  // read those instead of the whole row, and only the segments that can still hold a
+  // better open group than the best open segment minimum
+  const unsigned long long* seg_min;
+  int nseg;
   int heads, n, G, cap;
   int* labels;          // [heads, n]
   int* room;            // [heads, G]
@@ -50,6 +60,8 @@ struct FillArgs {
 };
 
 cudaError_t launch_midpoint_stride(int* idx, int n, int count, cudaStream_t st);
+cudaError_t launch_segment_minima(const float* D, int ldd, long long rows, int G, unsigned long long* seg, int nseg,
+                                  int* status, cudaStream_t st);
 cudaError_t launch_gram(const void* X, bool f32, size_t head_stride, const int* rows, int nrows, int heads,
                         int d, float* gamma, cudaStream_t st);
 cudaError_t launch_split_bf16(const float* src, __nv_bfloat16* hi, __nv_bfloat16* lo, size_t count,

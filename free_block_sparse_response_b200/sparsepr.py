@@ -26,7 +26,7 @@ EXPORTED_SYMBOLS = (
     "sparsepr_probe_dense", "sparsepr_fit_residual", "sparsepr_apply_residual", "sparsepr_check",
     "sparsepr_last_error", "sparsepr_test_fill_workspace_size", "sparsepr_test_fill",
     "sparsepr_test_topk", "sparsepr_row_errors", "sparsepr_launch_count", "sparsepr_fit_residual_noalloc",
-    "sparsepr_kernel_timing", "sparsepr_kernel_timing_read",
+    "sparsepr_kernel_timing", "sparsepr_kernel_timing_read", "sparsepr_test_fill_segmented",
 )
 
 
@@ -97,6 +97,7 @@ def lib() -> ctypes.CDLL:
         "sparsepr_last_error": (ctypes.c_char_p, []),
         "sparsepr_test_fill_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32]),
         "sparsepr_test_fill": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+        "sparsepr_test_fill_segmented": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
         "sparsepr_test_topk": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
         "sparsepr_row_errors": (ctypes.c_int, [_vp, ctypes.c_int, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
         "sparsepr_launch_count": (ctypes.c_uint64, []),
@@ -346,13 +347,18 @@ def launch_count() -> int:
 
 # ------------------------------------------------------- decision kernels, injected input
 
-def test_fill(dist: torch.Tensor, cap: int) -> torch.Tensor:
-    """Capacity fill on injected fp32 distances [H, n, G] -> labels [H, n] int32."""
+def test_fill(dist: torch.Tensor, cap: int, segmented: bool = False) -> torch.Tensor:
+    """Capacity fill on injected fp32 distances [H, n, G] -> labels [H, n] int32.
+
+    ``segmented`` takes the proposals from the rows' 64-column segment minima (the path
+    of the bf16, d = 128 partition); the labels must not change.
+    """
     _need_cuda(dist)
     h, n, g = dist.shape
     ws = torch.empty(int(lib().sparsepr_test_fill_workspace_size(h, n, g)), dtype=torch.uint8, device=dist.device)
     labels = torch.empty(h, n, dtype=torch.int32, device=dist.device)
-    _call("sparsepr_test_fill", _p(dist), h, n, g, cap, _p(labels), _p(ws), _stream(dist))
+    _call("sparsepr_test_fill_segmented" if segmented else "sparsepr_test_fill", _p(dist), h, n, g, cap, _p(labels),
+          _p(ws), _stream(dist))
     check(ws)
     return labels
 

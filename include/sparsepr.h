@@ -228,8 +228,8 @@ SPARSEPR_API int sparsepr_kernel_timing(int enable);
 SPARSEPR_API int sparsepr_kernel_timing_read(double* ms_total, int64_t* launches);
 
 /* Wait for `stream` and return the device status word in `ws` (SPARSEPR_OK, or the
- * first device-side error since the last sparsepr_partition).  This is the only call
- * that synchronises. */
+ * first device-side error since the last sparsepr_partition).  Apart from the timing
+ * hook's read, this is the only call that synchronises. */
 SPARSEPR_API int sparsepr_check(const void* ws, sparsepr_stream_t stream);
 
 /* Message of the last host-side error on this thread ("" if none). */
@@ -238,11 +238,17 @@ SPARSEPR_API const char* sparsepr_last_error(void);
 /* ---- decision kernels on injected scores (used by the parity tests) ---------------
  * sparsepr_test_fill: the capacity-B assignment used by every k-means iteration, run
  *   on caller-supplied fp32 distances D [H, n, G] (device); labels [H, n] int32.
+ * sparsepr_test_fill_segmented: the same assignment with the proposals taken from the
+ *   minima of the rows' 64-column segments (the path the bf16, d = 128 partition runs):
+ *   the labels must equal sparsepr_test_fill's for every D.
  * sparsepr_test_topk: the routing selection on caller-supplied scores Sc [H, Gq, G];
- *   route [H, Gq, k] int32.  Both use the same kernels as the operator. */
+ *   route [H, Gq, k] int32.  All use the same kernels as the operator; the fill calls
+ *   share sparsepr_test_fill_workspace_size. */
 SPARSEPR_API size_t sparsepr_test_fill_workspace_size(int32_t H, int32_t n, int32_t G);
 SPARSEPR_API int sparsepr_test_fill(const float* D, int32_t H, int32_t n, int32_t G, int32_t cap,
                        int32_t* labels, void* ws, sparsepr_stream_t stream);
+SPARSEPR_API int sparsepr_test_fill_segmented(const float* D, int32_t H, int32_t n, int32_t G,
+                       int32_t cap, int32_t* labels, void* ws, sparsepr_stream_t stream);
 SPARSEPR_API int sparsepr_test_topk(const float* Sc, int32_t H, int32_t Gq, int32_t G, int32_t k,
                        int32_t* route, void* ws, sparsepr_stream_t stream);
 
