@@ -31,6 +31,25 @@ __device__ double block_sum_d(double v, double* red) {
   return s;
 }
 
+// Reciprocal and reciprocal square root in fp64 by Newton-Raphson refinement of the fp32
+// hardware estimates (y <- y (2 - x y), and y <- y (3 - x y^2) / 2): each step squares
+// the relative error, so two steps take the ~2^-22 seed to fp64 rounding level.  Used
+// on the latency-critical path of the Jacobi rotations, for arguments well inside the
+// fp32 range (the callers keep them there).
+__device__ __forceinline__ double rcp_nr(double x) {
+  double y = static_cast<double>(__frcp_rn(static_cast<float>(x)));
+  y = y * fma(-x, y, 2.0);
+  y = y * fma(-x, y, 2.0);
+  return y;
+}
+__device__ __forceinline__ double rsqrt_nr(double x) {
+  double y = static_cast<double>(rsqrtf(static_cast<float>(x)));
+  const double hx = 0.5 * x;
+  y = y * fma(-hx * y, y, 1.5);
+  y = y * fma(-hx * y, y, 1.5);
+  return y;
+}
+
 __host__ __device__ size_t fit_scratch_doubles(int P, int d) {
   return static_cast<size_t>(d) * d + static_cast<size_t>(P) * d + static_cast<size_t>(d) * d + 4ull * d;
 }
@@ -127,10 +146,24 @@ __global__ void __launch_bounds__(kFitThreads)
   }
   total = block_sum_d(total, red);
   const double tol2 = 1e-20 * total;  // stop at off-diagonal norm <= 1e-10 |C|
-  if (tid < D / 2) {
-    pp[tid] = 0;
-    pq[tid] = 0;
-    ps[tid] = 0.0;
+  // this thread's 2x2 blocks (a, b), a <= b, of the pair slots (fixed for all rounds)
+  constexpr int kBlocks = (D / 2) * (D / 2 + 1) / 2;
+  constexpr int kBlocksPer = (kBlocks + kFitThreads - 1) / kFitThreads;
+  int blk_a[kBlocksPer], blk_b[kBlocksPer];
+#pragma unroll
+  for (int i = 0; i < kBlocksPer; ++i) {
+    const int x = tid + i * kFitThreads;
+    blk_a[i] = -1;
+    blk_b[i] = -1;
+    if (x < kBlocks) {
+      int a = 0, first = 0;  // first = index of block (a, a)
+      while (first + (D / 2 - a) <= x) {
+        first += D / 2 - a;
+        ++a;
+      }
+      blk_a[i] = a;
+      blk_b[i] = a + (x - first);
+    }
   }
   for (int sweep = 0; sweep < 40; ++sweep) {
     double off = 0.0;
@@ -145,11 +178,6 @@ __global__ void __launch_bounds__(kFitThreads)
     if (off <= tol2 || total == 0.0) break;
     for (int round = 0; round < D - 1; ++round) {
       if (tid < D / 2) {
-        // the previous round's pair of this slot was annihilated: store exact zeros
-        if (ps[tid] != 0.0) {
-          C[pp[tid] * LD + pq[tid]] = 0.0;
-          C[pq[tid] * LD + pp[tid]] = 0.0;
-        }
         int p, q;
         if (tid == 0) {
           p = round;
@@ -167,9 +195,19 @@ __global__ void __launch_bounds__(kFitThreads)
         const double app = C[p * LD + p], aqq = C[q * LD + q];
         double c = 1.0, sn = 0.0;
         if (apq != 0.0 && apq * apq > 1e-30 * fabs(app * aqq) && apq * apq > 1e-36 * total) {
-          const double theta = (aqq - app) / (2.0 * apq);
-          const double t = (theta >= 0.0 ? 1.0 : -1.0) / (fabs(theta) + sqrt(theta * theta + 1.0));
-          c = 1.0 / sqrt(t * t + 1.0);
+          // t = tan of the annihilating angle, the smaller root of t^2 + 2 theta t - 1 = 0
+          const double den = 2.0 * apq;
+          const double theta = fabs(den) > 1e-30 && fabs(den) < 1e30 ? (aqq - app) * rcp_nr(den) : (aqq - app) / den;
+          const double at = fabs(theta);
+          double t;
+          if (at > 1e15) {
+            t = 0.5 / theta;  // sqrt(theta^2 + 1) = |theta| to fp64 precision
+          } else {
+            const double h = theta * theta + 1.0;
+            t = rcp_nr(at + h * rsqrt_nr(h));
+            if (theta < 0.0) t = -t;
+          }
+          c = rsqrt_nr(t * t + 1.0);
           sn = t * c;
         }
         pp[tid] = p;
@@ -178,41 +216,54 @@ __global__ void __launch_bounds__(kFitThreads)
         ps[tid] = sn;
       }
       __syncthreads();
-      for (int x = tid; x < (D / 2) * D; x += kFitThreads) {  // rows: J^T C, and V^T rows
+      // C <- R C R^T with R the product of this round's D/2 disjoint plane rotations
+      // (rows p, q of R: (c, -s), (s, c)), one 2x2 block {p_a, q_a} x {p_b, q_b} at a
+      // time: B <- R_a B R_b^T for a <= b, the mirror block written as its transpose;
+      // the annihilated element of a rotated pair is stored as an exact zero.
+#pragma unroll
+      for (int i = 0; i < kBlocksPer; ++i) {
+        const int a = blk_a[i], b = blk_b[i];
+        if (a < 0) continue;
+        const double sa = ps[a], sb = ps[b];
+        if (sa == 0.0 && sb == 0.0) continue;
+        const double ca = pc[a], cb = pc[b];
+        const int pa = pp[a], qa = pq[a], pb = pp[b], qb = pq[b];
+        const double b00 = C[pa * LD + pb], b01 = C[pa * LD + qb], b10 = C[qa * LD + pb], b11 = C[qa * LD + qb];
+        const double t00 = b00 * cb - b01 * sb, t01 = b00 * sb + b01 * cb;
+        const double t10 = b10 * cb - b11 * sb, t11 = b10 * sb + b11 * cb;
+        const double n00 = ca * t00 - sa * t10, n01 = ca * t01 - sa * t11;
+        const double n10 = sa * t00 + ca * t10, n11 = sa * t01 + ca * t11;
+        if (a == b) {
+          C[pa * LD + pa] = n00;
+          C[qa * LD + qa] = n11;
+          const double z = sa != 0.0 ? 0.0 : n01;
+          C[pa * LD + qa] = z;
+          C[qa * LD + pa] = z;
+        } else {
+          C[pa * LD + pb] = n00;
+          C[pa * LD + qb] = n01;
+          C[qa * LD + pb] = n10;
+          C[qa * LD + qb] = n11;
+          C[pb * LD + pa] = n00;
+          C[qb * LD + pa] = n01;
+          C[pb * LD + qa] = n10;
+          C[qb * LD + qa] = n11;
+        }
+      }
+      for (int x = tid; x < (D / 2) * D; x += kFitThreads) {  // eigenvector rows: V^T <- R V^T
         const int t = x / D, j = x % D;
         const double sn = ps[t];
         if (sn != 0.0) {
           const int p = pp[t], q = pq[t];
-          const double c = pc[t];
-          const double cp = C[p * LD + j], cq = C[q * LD + j];
-          C[p * LD + j] = c * cp - sn * cq;
-          C[q * LD + j] = sn * cp + c * cq;
-          const float cf = static_cast<float>(c), sf = static_cast<float>(sn);
+          const float cf = static_cast<float>(pc[t]), sf = static_cast<float>(sn);
           const float vp = Vt[p * D + j], vq = Vt[q * D + j];
           Vt[p * D + j] = cf * vp - sf * vq;
           Vt[q * D + j] = sf * vp + cf * vq;
         }
       }
       __syncthreads();
-      for (int x = tid; x < (D / 2) * D; x += kFitThreads) {  // columns: (J^T C) J
-        const int t = x % (D / 2), i = x / (D / 2);
-        const double sn = ps[t];
-        if (sn != 0.0) {
-          const int p = pp[t], q = pq[t];
-          const double c = pc[t];
-          const double cp = C[i * LD + p], cq = C[i * LD + q];
-          C[i * LD + p] = c * cp - sn * cq;
-          C[i * LD + q] = sn * cp + c * cq;
-        }
-      }
-      __syncthreads();
     }
   }
-  if (tid < D / 2 && ps[tid] != 0.0) {
-    C[pp[tid] * LD + pq[tid]] = 0.0;
-    C[pq[tid] * LD + pp[tid]] = 0.0;
-  }
-  __syncthreads();
   // ---- eigenvalues descending (stable on ties)
   for (int i = tid; i < D; i += kFitThreads) {
     const double li = C[i * LD + i];
