@@ -27,6 +27,8 @@ the order the pages give it:
   5. each query block keeps the k key groups with the largest centroid score,
      k set by the executed-pair density budget with probe rows counted      [abs, news]
   6. softmax attention restricted to the routed groups                       [abs]
+     (the semantic baseline partition of the comparisons replaces steps 1-4 by
+     balanced k-means on raw K and raw Q: ``partition_semantic``)
   7. exact dense attention for P probe rows                                  [abs, news]
   8. weighted ridge fit of an affine map sparse output -> residual inside the
      top-r subspace of the probe residuals                                   [abs, news]
@@ -220,6 +222,30 @@ def partition(q: np.ndarray, k: np.ndarray, tau: float, block: int, n_sampled: i
         dump["query_dist"] = qd
     return {"sample_idx": s_idx, "key_labels": key_labels, "mu": mu, "coords": coords,
             "query_labels": query_labels, "block_scores": block_scores}
+
+
+def partition_semantic(q: np.ndarray, k: np.ndarray, tau: float, block: int, iters: int,
+                       dump: Optional[dict] = None) -> dict:
+    """The semantic block partition the method is compared against ([abs]: "semantic
+    block-sparse attention without residual correction"; [news], ablations paragraph).
+    The pages do not state its rule; the reading taken is balanced k-means on the raw
+    keys and, independently, on the raw queries (squared Euclidean distance, the same
+    chunk start, fill and iteration count), with the routing scores of the response-
+    coupled partition (mean over a block's queries of tau q_i . mu_g)."""
+    n = q.shape[0]
+    g_count = n_groups(n, block)
+    kd = [] if dump is not None else None
+    key_labels, _ = balanced_kmeans(k, g_count, block, iters, kd)
+    mu = group_means(k, key_labels, g_count)
+    qd = [] if dump is not None else None
+    query_labels, _ = balanced_kmeans(q, g_count, block, iters, qd)
+    coords = tau * (q @ mu.T)
+    block_scores = group_means(coords, query_labels, g_count).astype(np.float32)
+    if dump is not None:
+        dump["key_dist"] = kd
+        dump["query_dist"] = qd
+    return {"key_labels": key_labels, "mu": mu, "coords": coords, "query_labels": query_labels,
+            "block_scores": block_scores}
 
 
 # ------------------------------------------------------------------ step 5: routing
@@ -431,10 +457,12 @@ def rel_l2_errors(o: np.ndarray, o_dense: np.ndarray, probe_idx: np.ndarray) -> 
 
 def sparsepr_head(q, k, v, *, block, n_sampled, n_probe, density, ridge_lambda, rank,
                   kmeans_iters=4, scale=None, weight_mode="inv_norm", inject=None,
-                  dump=None) -> dict:
+                  dump=None, partition_mode="response") -> dict:
     """One SparsePR call on one (batch, head).  ``inject`` may hold any of
     sample_idx, probe_idx, key_labels, query_labels, routes (e.g. the CUDA path's
-    decisions) to run the later steps on them."""
+    decisions) to run the later steps on them.  ``partition_mode`` "semantic" swaps
+    Response-Coupled Partitioning for the semantic baseline partition (the ablation);
+    the result's "S" is then the uncorrected semantic block-sparse output."""
     inject = inject or {}
     n, d = q.shape
     tau = 1.0 / math.sqrt(d) if scale is None or scale <= 0 else float(scale)
@@ -442,6 +470,8 @@ def sparsepr_head(q, k, v, *, block, n_sampled, n_probe, density, ridge_lambda, 
     if "key_labels" in inject and "query_labels" in inject:
         part = {"key_labels": np.asarray(inject["key_labels"]),
                 "query_labels": np.asarray(inject["query_labels"])}
+    elif partition_mode == "semantic":
+        part = partition_semantic(q, k, tau, block, kmeans_iters, dump)
     else:
         part = partition(q, k, tau, block, n_sampled, kmeans_iters,
                          inject.get("sample_idx"), dump)

@@ -463,3 +463,42 @@ def test_partition_and_route_follow_planted_attention():
     s = O.sparse_attention(q, k, v, tau, part["key_labels"], part["query_labels"], routes)
     dense = O.dense_attention_rows(q, k, v, tau, np.arange(n))
     assert O.rel_l2_errors(s, dense, np.array([], dtype=np.int64))["mean"] < 1e-3
+
+
+# ------------------------------------------------------------ semantic baseline partition
+
+def test_semantic_keys_equal_response_keys_when_sampled_queries_are_a_scaled_basis():
+    """With tau = 1/2 and the d sampled queries equal to 2 e_m, every key's response
+    profile is the key itself, bit for bit, so Response-Coupled Partitioning and the
+    semantic partition (k-means on raw keys) must give identical key labels and mean
+    keys; the query sides still differ in general (coordinates u vs raw q)."""
+    rng = _rng(31)
+    n, d, block = 96, 8, 16
+    q, k = rng.normal(size=(n, d)), rng.normal(size=(n, d))
+    sidx = O.midpoint_stride(n, d)
+    q[sidx] = 2.0 * np.eye(d)
+    tau = 0.5
+    assert np.array_equal(O.key_response_profiles(q, k, sidx, tau), k)
+    resp = O.partition(q, k, tau, block, n_sampled=d, iters=3)
+    sem = O.partition_semantic(q, k, tau, block, iters=3)
+    assert np.array_equal(resp["key_labels"], sem["key_labels"])
+    assert np.array_equal(resp["mu"], sem["mu"])
+
+
+def test_semantic_partition_recovers_planted_raw_clusters():
+    """Keys and queries in tight clusters of their own (in raw space): the semantic
+    partition must recover both clusterings, whatever the queries attend to."""
+    rng = _rng(32)
+    g_count, block, d = 5, 12, 10
+    n = g_count * block
+    kc = rng.normal(size=(g_count, d)) * 8
+    qc = rng.normal(size=(g_count, d)) * 8
+    key_truth = rng.permutation(np.repeat(np.arange(g_count), block))
+    query_truth = rng.permutation(np.repeat(np.arange(g_count), block))
+    k = kc[key_truth] + 0.1 * rng.normal(size=(n, d))
+    q = qc[query_truth] + 0.1 * rng.normal(size=(n, d))
+    sem = O.partition_semantic(q, k, 1 / math.sqrt(d), block, iters=3)
+    assert len(set(zip(sem["key_labels"].tolist(), key_truth.tolist()))) == g_count
+    assert len(set(zip(sem["query_labels"].tolist(), query_truth.tolist()))) == g_count
+    assert np.bincount(sem["query_labels"]).tolist() == [block] * g_count
+
