@@ -14,6 +14,7 @@ bounded sample of the same workload instead (the reference arm).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -43,6 +44,8 @@ def parse_args():
     ap.add_argument("--config", default="video")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--study", choices=["ablation", "probe-budget"], default=None,
+                    help="error studies instead of the timed run (one JSON line per variant)")
     return ap.parse_args()
 
 
@@ -410,10 +413,115 @@ def run_ours(args, w):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------- error studies
+
+def _gpu_modules():
+    import torch
+    import free_block_sparse_response_b200 as spr
+    return torch, spr
+
+
+def _err_summary(e):
+    """Head-averaged mean and p99 of the per-row errors (NaN rows = probe rows skipped)."""
+    torch, _ = _gpu_modules()
+    means, p99s = [], []
+    for b in range(e.shape[0]):
+        for hh in range(e.shape[1]):
+            x = e[b, hh]
+            x = x[~torch.isnan(x)]
+            xs, _ = torch.sort(x)
+            means.append(float(xs.double().mean()))
+            p99s.append(float(xs[max(math.ceil(0.99 * xs.numel()) - 1, 0)]))
+    return statistics.mean(means), statistics.mean(p99s)
+
+
+def _study_inputs(args, w):
+    from synthetic import make_inputs
+    torch, spr = _gpu_modules()
+    dev = torch.device("cuda", 0)
+    q, k, v = (t.to(dev) for t in make_inputs(w, args.seed))
+    bt, h, n, d = q.shape
+    dense = torch.empty(bt, h, n, d, dtype=torch.float32, device=dev)
+    spr.dense_attn(q, k, v, block=w.block, out=dense)
+    return q, k, v, dense
+
+
+def _uncorrected(q, k, v, cfg, ws):
+    """Block-sparse output without residual correction, its k from the pair budget
+    without probe rows (equal executed-pair density to the corrected call)."""
+    _, spr = _gpu_modules()
+    n = q.shape[2]
+    cfg0 = dataclasses.replace(cfg, n_probe=0)
+    part = spr.partition(q, k, cfg0, ws)
+    rt, kk, pairs = spr.route(part, n, cfg0, ws)
+    return spr.sparse_attn(q, k, v, part, rt, kk, cfg0, ws=ws), kk, pairs
+
+
+def run_study_ablation(args, w):
+    """Error of the semantic baseline and of each SparsePR component against the
+    same-family dense output: semantic partition without correction (the comparator
+    of the pages' error reduction), semantic partition + probe fit, Response-Coupled
+    Partitioning without correction, and the full method.  Errors over the rows that
+    are not probe rows of the full method; equal executed-pair density throughout."""
+    _, spr = _gpu_modules()
+    q, k, v, dense = _study_inputs(args, w)
+    bt, h, n, d = q.shape
+    base = spr.SparsePRConfig(block=w.block, n_sampled=w.n_sampled, n_probe=w.n_probe, kmeans_iters=w.kmeans_iters,
+                              rank=w.rank, density=w.density, ridge_lambda=w.ridge_lambda)
+    ws = spr.new_workspace(bt, h, n, d, base, q.device)
+    pidx = spr.probe_rows(n, w.n_probe, bt, h, q.device)
+    rows = []
+    for mode, name in ((spr.PARTITION_SEMANTIC, "semantic"), (spr.PARTITION_RESPONSE, "response-coupled")):
+        cfg = dataclasses.replace(base, partition_mode=mode)
+        s, kk0, pairs0 = _uncorrected(q, k, v, cfg, ws)
+        m, p = _err_summary(spr.row_errors(s, dense, pidx))
+        rows.append({"variant": f"{name} partition, no correction", "mean_rel_l2": m, "p99_rel_l2": p, "k": kk0,
+                     "density": float(pairs0.double().sum()) / (float(n) ** 2 * h * bt)})
+        o, parts = spr.attention(q, k, v, cfg, ws=ws, return_parts=True)
+        m, p = _err_summary(spr.row_errors(o, dense, pidx))
+        rows.append({"variant": f"{name} partition + probe-fitted correction", "mean_rel_l2": m, "p99_rel_l2": p,
+                     "k": parts["k"],
+                     "density": float(parts["executed_pairs"].double().sum()) / (float(n) ** 2 * h * bt)})
+    spr.check(ws)
+    ref = rows[0]["mean_rel_l2"]
+    for r in rows:
+        r["mean_error_reduction_vs_semantic_uncorrected"] = 1.0 - r["mean_rel_l2"] / ref
+        r.update({"study": "ablation", "workload": config_block(w, args)["workload"], "seed": args.seed,
+                  "reference": "same-family dense attention, fp32 output"})
+        print(json.dumps(r), flush=True)
+
+
+def run_study_probe_budget(args, w):
+    """Mean and p99 unprobed-row error against the probe budget P (k re-derived from
+    the pair budget for each P), with the uncorrected output at the same density."""
+    _, spr = _gpu_modules()
+    q, k, v, dense = _study_inputs(args, w)
+    bt, h, n, d = q.shape
+    for P in (32, 64, 128, 256, 512):
+        cfg = spr.SparsePRConfig(block=w.block, n_sampled=w.n_sampled, n_probe=P, kmeans_iters=w.kmeans_iters,
+                                 rank=w.rank, density=w.density, ridge_lambda=w.ridge_lambda)
+        ws = spr.new_workspace(bt, h, n, d, cfg, q.device)
+        pidx = spr.probe_rows(n, P, bt, h, q.device)
+        o, parts = spr.attention(q, k, v, cfg, ws=ws, return_parts=True)
+        m, p = _err_summary(spr.row_errors(o, dense, pidx))
+        mu, pu = _err_summary(spr.row_errors(parts["S"], dense, pidx))
+        spr.check(ws)
+        print(json.dumps({"study": "probe-budget", "workload": config_block(w, args)["workload"], "P": P,
+                          "k": parts["k"], "density": float(parts["executed_pairs"].double().sum()) /
+                          (float(n) ** 2 * h * bt), "mean_rel_l2": m, "p99_rel_l2": p,
+                          "uncorrected_mean_rel_l2": mu, "uncorrected_p99_rel_l2": pu,
+                          "mean_error_reduction": 1.0 - m / mu, "seed": args.seed}), flush=True)
+        del ws
+
+
 def main():
     args = parse_args()
     w = workload(args)
-    if args.impl == "reference":
+    if args.study == "ablation":
+        run_study_ablation(args, w)
+    elif args.study == "probe-budget":
+        run_study_probe_budget(args, w)
+    elif args.impl == "reference":
         run_reference(args, w)
     else:
         run_ours(args, w)

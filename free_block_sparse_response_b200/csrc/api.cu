@@ -183,6 +183,9 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
   if (p->kmeans_iters < 0 || p->kmeans_iters > 64) return fail(SPARSEPR_ERR_INVALID_ARG, "kmeans_iters must be in [0, 64]");
   if (spr::ceil_div(N, p->block) > 1024)
     return fail(SPARSEPR_ERR_UNSUPPORTED, "more than 1024 groups per head (N / block) is not built");
+  if (p->partition_mode != SPARSEPR_PARTITION_RESPONSE && p->partition_mode != SPARSEPR_PARTITION_SEMANTIC)
+    return fail(SPARSEPR_ERR_INVALID_ARG, "unknown partition_mode %d", p->partition_mode);
+  const bool semantic = p->partition_mode == SPARSEPR_PARTITION_SEMANTIC;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int heads = Bt * H, B = p->block, G = spr::ceil_div(N, B), S = p->n_sampled;
   const bool f32 = dtype == SPARSEPR_F32;
@@ -259,7 +262,7 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
       ra.Bf32 = wf;
       ra.nrm = nrm;
       ra.ecol = eg;
-      ra.tau2 = tau * tau;
+      ra.tau2 = semantic ? 1.0f : tau * tau;  // raw squared distances for the semantic rule
       ra.Dout = dmat;
       ra.ldd = fa.ldd;
       ra.prop_g = at<int>(ws, L.prop_g0);
@@ -279,11 +282,14 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
 
   float* cent_k = at<float>(ws, L.cent_k);
   float* cent_q = at<float>(ws, L.cent_q);
-  // keys: profiles against the sampled queries -> gamma = Q_S^T Q_S
-  SPR_CUDA(spr::launch_gram(Q, f32, static_cast<size_t>(N) * d, sidx, S, heads, d, gamma, st), "Q_S gram");
+  // keys: profiles against the sampled queries -> gamma = Q_S^T Q_S (semantic: identity)
+  if (semantic) SPR_CUDA(spr::launch_identity(gamma, heads, d, st), "identity metric");
+  else SPR_CUDA(spr::launch_gram(Q, f32, static_cast<size_t>(N) * d, sidx, S, heads, d, gamma, st), "Q_S gram");
   if ((rc = cluster(K, cent_k, key_perm, key_gsize))) return rc;
-  // queries: coordinates against the key-group mean keys -> gamma = mu^T mu
-  SPR_CUDA(spr::launch_gram(cent_k, true, static_cast<size_t>(G) * d, nullptr, G, heads, d, gamma, st), "mu gram");
+  // queries: coordinates against the key-group mean keys -> gamma = mu^T mu (semantic:
+  // the raw queries, identity)
+  if (semantic) SPR_CUDA(spr::launch_identity(gamma, heads, d, st), "identity metric");
+  else SPR_CUDA(spr::launch_gram(cent_k, true, static_cast<size_t>(G) * d, nullptr, G, heads, d, gamma, st), "mu gram");
   if ((rc = cluster(Q, cent_q, query_perm, qblock_size))) return rc;
   SPR_CUDA(spr::launch_block_scores(cent_q, cent_k, G, heads, d, tau, block_scores, st), "block scores");
   return SPARSEPR_OK;

@@ -881,6 +881,20 @@ cudaError_t launch_segment_minima(const float* D, int ldd, long long rows, int G
   return counted(cudaGetLastError(), 1);
 }
 
+__global__ void identity_kernel(float* __restrict__ gamma, int heads, int d) {
+  const size_t total = static_cast<size_t>(heads) * d * d;
+  for (size_t x = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; x < total;
+       x += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t e = x % (static_cast<size_t>(d) * d);
+    gamma[x] = (e / d == e % d) ? 1.0f : 0.0f;
+  }
+}
+
+cudaError_t launch_identity(float* gamma, int heads, int d, cudaStream_t st) {
+  identity_kernel<<<ceil_div(heads * d * d, 256), 256, 0, st>>>(gamma, heads, d);
+  return counted(cudaGetLastError(), 1);
+}
+
 cudaError_t launch_midpoint_stride(int* idx, int n, int count, cudaStream_t st) {
   midpoint_stride_kernel<<<ceil_div(count, 256), 256, 0, st>>>(idx, n, count);
   return counted(cudaGetLastError(), 1);

@@ -60,6 +60,8 @@ struct FillArgs {
 };
 
 cudaError_t launch_midpoint_stride(int* idx, int n, int count, cudaStream_t st);
+// gamma [heads, d, d] = identity (the metric of the semantic partition)
+cudaError_t launch_identity(float* gamma, int heads, int d, cudaStream_t st);
 cudaError_t launch_segment_minima(const float* D, int ldd, long long rows, int G, unsigned long long* seg, int nseg,
                                   int* status, cudaStream_t st);
 cudaError_t launch_gram(const void* X, bool f32, size_t head_stride, const int* rows, int nrows, int heads,

@@ -67,6 +67,12 @@ enum { SPARSEPR_BF16 = 0, SPARSEPR_F32 = 1 };
 
 enum { SPARSEPR_WEIGHT_INV_NORM = 0, SPARSEPR_WEIGHT_UNIFORM = 1 };
 
+/* Partition rule.  RESPONSE: Response-Coupled Partitioning (the method).  SEMANTIC: the
+ * semantic block-sparse baseline the pages compare against, read as balanced k-means on
+ * the raw keys and on the raw queries (same start, fill, iterations and routing); the
+ * pages do not state that rule. */
+enum { SPARSEPR_PARTITION_RESPONSE = 0, SPARSEPR_PARTITION_SEMANTIC = 1 };
+
 typedef struct sparsepr_params {
   int32_t block;        /* B: query-block and key-group capacity (64 or 128)            */
   int32_t n_sampled;    /* S: sampled queries that define key response profiles        */
@@ -77,6 +83,7 @@ typedef struct sparsepr_params {
   double density;       /* rho: executed-pair budget / N^2, probe rows counted          */
   double ridge_lambda;  /* lambda: ridge on the centred weighted Gram (sum w = P)       */
   float scale;          /* softmax scale tau; <= 0 selects 1/sqrt(d)                    */
+  int32_t partition_mode; /* SPARSEPR_PARTITION_*                                        */
 } sparsepr_params;
 
 /* Number of groups G = Gq = ceil(N / B): capacity-B groups that cover all N tokens. */

@@ -61,12 +61,21 @@ def test_argument_errors_return_codes_without_launching(L):
     assert rc == spr.ERR_INVALID_ARG
     rc = L.sparsepr_test_topk(None, 1, 4, 4, 5, None, None, None)
     assert rc == spr.ERR_INVALID_ARG
+    # an unknown partition rule is refused before anything is launched (the non-null
+    # pointers below are never dereferenced on the host)
+    bad = spr.SparsePRConfig(partition_mode=7).c()
+    fake = ctypes.c_void_p(256)
+    rc = L.sparsepr_partition(fake, fake, spr.BF16, 1, 1, 1024, 128, ctypes.byref(bad), None, fake, fake, fake, fake,
+                              fake, fake, None)
+    assert rc == spr.ERR_INVALID_ARG
+    assert b"partition_mode" in L.sparsepr_last_error()
 
 
 def test_params_struct_layout():
     assert ctypes.sizeof(spr.sparsepr._CParams) == 48
     assert spr.sparsepr._CParams.density.offset == 24
     assert spr.sparsepr._CParams.scale.offset == 40
+    assert spr.sparsepr._CParams.partition_mode.offset == 44
 
 
 def test_python_wrappers_refuse_cpu_tensors():

@@ -253,6 +253,26 @@ def test_partition_label_agreement_with_oracle():
     assert key_agree > 0.5
 
 
+def test_semantic_partition_call_parity():
+    """The semantic baseline partition (balanced k-means on raw K and raw Q): labels
+    agree with the oracle's semantic partition on most tokens, and the rest of the call
+    on the GPU's decisions matches the oracle as in the response-coupled calls."""
+    w = CONFIGS["small"]
+    cfg = spr_cfg(w, partition_mode=spr.PARTITION_SEMANTIC)
+    q, k, v = make_inputs(w, 0, heads=2)
+    _, parts = _check_call(w, cfg, heads=2)
+    n = w.n_tokens
+    part = parts["partition"]
+    for h in range(2):
+        kl = perm_labels(part.key_perm[0, h].cpu().numpy(), part.key_gsize[0, h].cpu().numpy(), n, w.block)
+        ql = perm_labels(part.query_perm[0, h].cpu().numpy(), part.qblock_size[0, h].cpu().numpy(), n, w.block)
+        ref = O.partition_semantic(q[0, h].double().numpy(), k[0, h].double().numpy(), 1 / math.sqrt(w.head_dim),
+                                   w.block, w.kmeans_iters)
+        key_agree, query_agree = float((kl == ref["key_labels"]).mean()), float((ql == ref["query_labels"]).mean())
+        print(f"semantic head {h}: key label agreement {key_agree:.3f}, query {query_agree:.3f}")
+        assert key_agree > 0.5 and query_agree > 0.5
+
+
 def test_nonfinite_input_is_reported():
     w = CONFIGS["tiny"].with_(dtype="bf16")
     q, k, v = make_inputs(w, 0)
