@@ -71,6 +71,24 @@ def dense_flops(w):
     return 4.0 * w.head_dim * float(w.n_tokens) ** 2 * w.heads * w.batch
 
 
+def max_over_ranks(seconds, world, device=None):
+    """The job's time: the slowest rank's (an all-reduce MAX over the process group);
+    the value itself on one rank."""
+    if world == 1:
+        return seconds
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank_step, world, steps, seconds):
+    """Whole-job aggregate (weak scaling): every rank processes the same per-step work,
+    so the job's units are units x ranks x steps over the slowest rank's time."""
+    return units_per_rank_step * world * steps / seconds
+
+
 # ------------------------------------------------------------------- CPU oracle sample
 
 def oracle_sample(w, seed=0):
@@ -294,11 +312,8 @@ def run_ours(args, w):
     launches = spr.launch_count() - launches0
     clk = clocks.stop()
     spr.check(ws)
-    elapsed = t_start.elapsed_time(t_end) / 1e3
+    elapsed = max_over_ranks(t_start.elapsed_time(t_end) / 1e3, world, dev)
     if world > 1:
-        tt = torch.tensor([elapsed], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed = float(tt.item())
         dist.barrier()
     ms_step = elapsed / args.steps * 1e3
     stage_ms = {s: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in events) for i, s in enumerate(stages)}
@@ -337,11 +352,7 @@ def run_ours(args, w):
         op.copy_(o, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
-    e2e_s = e0.elapsed_time(e1) / 1e3
-    if world > 1:
-        tt = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_s = float(tt.item())
+    e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
     d2h = o.numel() * o.element_size()
 
@@ -389,9 +400,8 @@ def run_ours(args, w):
     s_mean, s_p99 = summary(err_s)
     spr.check(ws)
 
-    total_flops = dense_flops(w) * world
-    value = total_flops * args.steps / elapsed / 1e12
-    e2e_value = total_flops * args.steps / e2e_s / 1e12
+    value = job_throughput(dense_flops(w), world, args.steps, elapsed) / 1e12
+    e2e_value = job_throughput(dense_flops(w), world, args.steps, e2e_s) / 1e12
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
