@@ -8,12 +8,14 @@
 //
 // Fit, one CTA per (batch, head), fp64 throughout:
 //   w_p (caller / 1/|d_p|^2 / uniform) scaled to sum P;  y_p = d_p - s_p;
-//   C = sum_p w_p y_p y_p^T;  eigenvectors by Jacobi with the round-robin parallel
-//   ordering (d/2 disjoint rotations per step);  U_r = top-r;  z_p = U_r^T y_p;
+//   C = sum_p w_p y_p y_p^T;  U_r = eigenvectors of the r largest eigenvalues (r <= 32:
+//   Householder tridiagonalisation, bisection and inverse iteration; larger r: cyclic
+//   Jacobi with the round-robin parallel ordering);  z_p = U_r^T y_p;
 //   A = (Z_c^T W X_c)(X_c^T W X_c + lambda I)^-1 by Cholesky;  b = zbar - A xbar;
 //   M = U_r A, beta = U_r b.
 #include "common.cuh"
 #include "fit.cuh"
+#include "tridiag_eig.cuh"
 
 namespace spr {
 
@@ -71,6 +73,8 @@ __global__ void __launch_bounds__(kFitThreads)
   __shared__ int pp[D / 2], pq[D / 2], order[D];
   __shared__ double xbar[D], zbar[D], bvec[D];
   __shared__ int s_fail;
+  __shared__ double t_dd[D], t_ee[D], t_e2[D], t_tau[D], t_evals[kTriMaxR], t_sh[8];
+  static_assert(kTriThreads == kFitThreads, "the eigensolver runs on the fit's CTA");
 
   const int head = blockIdx.x, tid = threadIdx.x;
   const float* xs = xs_all + static_cast<size_t>(head) * P * D;
@@ -135,9 +139,16 @@ __global__ void __launch_bounds__(kFitThreads)
     const int ij = tid + x * kFitThreads;
     C[(ij / D) * LD + ij % D] = acc[x];
   }
-  for (int x = tid; x < D * D; x += kFitThreads) Vt[x] = (x / D == x % D) ? 1.f : 0.f;
   __syncthreads();
 
+  // ---- eigenvectors of the R largest eigenvalues
+  const bool tri = R <= kTriMaxR;
+  if (tri) {
+    top_eigvecs_tridiagonal<D>(C, reinterpret_cast<double*>(Vt), stage, Vt, R, t_dd, t_ee, t_e2, t_tau, t_evals,
+                               t_sh);
+  } else {
+  for (int x = tid; x < D * D; x += kFitThreads) Vt[x] = (x / D == x % D) ? 1.f : 0.f;
+  __syncthreads();
   // ---- Jacobi, round-robin parallel ordering
   double total = 0.0;
   for (int x = tid; x < D * D; x += kFitThreads) {
@@ -275,11 +286,14 @@ __global__ void __launch_bounds__(kFitThreads)
     order[rank] = i;
   }
   __syncthreads();
+  }
+  // row a of U_r: the a-th largest eigenvalue's eigenvector (fp32)
+  auto urow = [&](int a) -> const float* { return tri ? Vt + a * D : Vt + static_cast<size_t>(order[a]) * D; };
 
   // ---- z_p = U_r^T y_p ; weighted means
   for (int x = tid; x < P * R; x += kFitThreads) {
     const int p = x / R, a = x % R;
-    const float* u = Vt + static_cast<size_t>(order[a]) * D;
+    const float* u = urow(a);
     double s = 0.0;
     for (int e = 0; e < D; ++e)
       s += u[e] * (static_cast<double>(dp[static_cast<size_t>(p) * D + e]) -
@@ -392,12 +406,12 @@ __global__ void __launch_bounds__(kFitThreads)
     const int i = x / D, j = x % D;
     double s = 0.0;
     for (int a = 0; a < R; ++a)
-      s += static_cast<double>(Vt[static_cast<size_t>(order[a]) * D + i]) * A[static_cast<size_t>(a) * D + j];
+      s += static_cast<double>(urow(a)[i]) * A[static_cast<size_t>(a) * D + j];
     M_out[static_cast<size_t>(head) * D * D + x] = failed ? 0.f : static_cast<float>(s);
   }
   for (int i = tid; i < D; i += kFitThreads) {
     double s = 0.0;
-    for (int a = 0; a < R; ++a) s += static_cast<double>(Vt[static_cast<size_t>(order[a]) * D + i]) * bvec[a];
+    for (int a = 0; a < R; ++a) s += static_cast<double>(urow(a)[i]) * bvec[a];
     beta_out[static_cast<size_t>(head) * D + i] = failed ? 0.f : static_cast<float>(s);
   }
   if (failed && tid == 0) record_error(status, kErrInvalidArg);

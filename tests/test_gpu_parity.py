@@ -221,11 +221,13 @@ def test_degenerate_and_variant_settings(overrides):
         assert rel(o[0, h].double().cpu().numpy(), ref["O"]) <= TOL_BF16
 
 
-def test_fit_kernel_matches_oracle_on_identical_inputs():
-    """The fp64 fit kernel alone: the GPU's probe outputs fed to both sides."""
+@pytest.mark.parametrize("rank", [16, 40])
+def test_fit_kernel_matches_oracle_on_identical_inputs(rank):
+    """The fp64 fit kernel alone: the GPU's probe outputs fed to both sides (rank 16:
+    tridiagonal eigensolver; rank 40: the Jacobi path for r > 32)."""
     w = CONFIGS["small"]
     q, k, v = make_inputs(w, 0, heads=2)
-    cfg = spr_cfg(w)
+    cfg = spr_cfg(w, rank=rank)
     _, parts = run_call(w, q, k, v, cfg)
     for h in range(2):
         xs = parts["probe_sparse"][0, h].double().cpu().numpy()
@@ -233,6 +235,30 @@ def test_fit_kernel_matches_oracle_on_identical_inputs():
         fit = O.fit_residual(xs, dp, cfg.ridge_lambda, cfg.rank)
         assert rel(parts["M"][0, h].cpu().numpy(), fit["M"]) <= 1e-5
         assert rel(parts["beta"][0, h].cpu().numpy(), fit["beta"]) <= 1e-5
+
+
+def test_fit_degenerate_residual_spectrum():
+    """Residuals along 8 orthogonal directions, 8 probes each, uniform weights: the
+    second moment has one 8-fold eigenvalue and a zero eigenvalue of multiplicity 120.
+    Eigenvectors of a cluster are arbitrary, but M and beta depend only on spans, so they
+    must match the oracle (inverse iteration must return an orthonormal basis of the
+    cluster, not 8 copies of one vector)."""
+    rng = np.random.default_rng(5)
+    P, d = 64, 128
+    dirs = np.linalg.qr(rng.normal(size=(d, d)))[0][:, :8].T
+    xs = rng.normal(size=(P, d)) * 0.3
+    y = 2.0 * dirs[np.arange(P) % 8] * (1.0 + 0.0 * rng.normal(size=(P, 1)))
+    dp = xs + y
+    xs32, dp32 = xs.astype(np.float32), dp.astype(np.float32)
+    cfg = spr.SparsePRConfig(block=128, n_probe=P, rank=16, weight_mode=spr.WEIGHT_UNIFORM)
+    ws = spr.new_workspace(1, 1, 8192, d, cfg, torch.device("cuda"))
+    m_gpu, b_gpu = spr.fit_residual(torch.from_numpy(xs32)[None, None].cuda(), torch.from_numpy(dp32)[None, None].cuda(),
+                                    cfg, ws)
+    spr.check(ws)
+    fit = O.fit_residual(xs32.astype(np.float64), dp32.astype(np.float64), cfg.ridge_lambda, cfg.rank,
+                         weight_mode="uniform")
+    assert rel(m_gpu[0, 0].cpu().numpy(), fit["M"]) <= 1e-4
+    assert rel(b_gpu[0, 0].cpu().numpy(), fit["beta"]) <= 1e-4
 
 
 def test_partition_label_agreement_with_oracle():
