@@ -15,7 +15,8 @@
 // next item -- overlaps the epilogue of chunk c).  Warps 0-1 load, warp 2 issues the
 // MMAs, warps 4-11 run the epilogue: each row is owned by two threads (columns 0-63 and
 // 64-127 of every chunk); a warp transposes its 32 rows x 32 columns through shared
-// memory so that each store instruction writes 128 contiguous bytes of one row.  The row argmin is a strict '<' scan in
+// memory so that each 16-byte-per-lane store instruction writes 128 contiguous bytes of
+// each of 4 rows.  The row argmin is a strict '<' scan in
 // ascending column order (first minimum wins, +-0 compare equal), merged across the two
 // halves at the end.  Every wait is bounded.
 #include "common.cuh"
@@ -174,7 +175,6 @@ __global__ void __launch_bounds__(kDtThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     const float m2t = -2.f * tau2;
     const uint32_t wstage = sStage + static_cast<uint32_t>(warp - 4) * kWarpStage;
-    const float* wstage_p = reinterpret_cast<const float*>(dsmem + (wstage - tc::saddr(dsmem)));
     int loaded_head = -1;
     bool aborted = false;  // after a failed wait: keep passing the named barriers, skip the work
     for (int w = blockIdx.x, it = 0; w < total; w += gridDim.x, ++it) {
@@ -195,10 +195,6 @@ __global__ void __launch_bounds__(kDtThreads, 1)
       int best_c = -1;
       const int wrow0 = row0 + (warp & 3) * 32;
       const bool full_rows = wrow0 + 32 <= n;
-      // per-lane offsets of the swizzled transpose reads, one per row phase (rr & 7)
-      int rd_off[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) rd_off[k] = (((lane >> 2) ^ k) << 2) + (lane & 3);
       for (int c = 0; c < n_chunks && !aborted; ++c) {
         const int q = it * n_chunks + c, s = q & 1;
         const bool got = tc::mbar_wait(bar(kAccFull0 + s), (q >> 1) & 1, abort_v, status);
@@ -256,20 +252,23 @@ __global__ void __launch_bounds__(kDtThreads, 1)
                          : "memory");
           }
           __syncwarp();
-          const int col = c0 + blk * 32 + lane;
+          // lane l stores 4 consecutive columns (16 B) of row rr + (l >> 3): every store
+          // instruction writes 128 contiguous bytes of each of 4 rows
+          const int col = c0 + blk * 32 + 4 * (lane & 7);
           if (col < ldd) {
-            float* dst = Dout + rowbase * ldd + col;
-            if (full_rows) {
+            const int rsub = lane >> 3;
+            float* dst = Dout + (rowbase + rsub) * ldd + col;
 #pragma unroll
-              for (int rr = 0; rr < 32; ++rr) {
-                *dst = wstage_p[rr * 32 + rd_off[rr & 7]];
-                dst += ldd;
+            for (int rr = 0; rr < 32; rr += 4) {
+              const int row_l = rr + rsub;
+              if (full_rows || wrow0 + row_l < n) {
+                float4 v;
+                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                             : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                             : "r"(wstage + row_l * 128 + (((lane & 7) ^ (row_l & 7)) << 4)));
+                *reinterpret_cast<float4*>(dst) = v;
               }
-            } else {
-              for (int rr = 0; rr < 32 && wrow0 + rr < n; ++rr) {
-                *dst = wstage_p[rr * 32 + rd_off[rr & 7]];
-                dst += ldd;
-              }
+              dst += 4 * static_cast<size_t>(ldd);
             }
           }
         }
