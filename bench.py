@@ -30,9 +30,9 @@ METRIC = "SparsePR ms/call & eff. TFLOP/s at 22% pair density; mean rel-L2 err v
 UNIT = "TFLOP/s (dense-equivalent, 4*d*N^2*H per call)"
 
 # DRAM bytes per launch of the dominant kernel from an ncu capture of the same kernel
-# build (profiles/attn_tc_kernel_video_4h.md: 367.6 MB on 4 heads), scaled by heads to
-# the 40-head launch; None whenever that kernel has changed since the capture.
-DOMINANT_TRAFFIC_BYTES = 3.676e9
+# build (profiles/), scaled by heads to the 40-head launch; None whenever that kernel
+# has changed since the capture.
+DOMINANT_TRAFFIC_BYTES = None
 
 
 def parse_args():
@@ -260,33 +260,40 @@ def run_ours(args, w):
                             rank=w.rank, density=w.density, ridge_lambda=w.ridge_lambda)
     ws = spr.new_workspace(bt, h, n, d, sc, dev)
     o = torch.empty_like(q)
-    stages = ["partition", "route", "sparse_attn", "probe_dense", "fit_residual", "apply_residual"]
+    fused = spr.fused_supported(q, sc)
+    # probe-first order with the correction fused into the attention kernel (the call
+    # spr.attention makes for this shape); the unfused order otherwise
+    stages = (["partition", "route", "probe_dense", "fit_residual", "sparse_attn_apply"] if fused else
+              ["partition", "route", "sparse_attn", "probe_dense", "fit_residual", "apply_residual"])
 
     def step(record=None):
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] if record is not None else None
-        if ev:
-            ev[0].record()
+        mark = (lambda i: ev[i].record()) if ev else (lambda i: None)
+        mark(0)
         part = spr.partition(q, k, sc, ws)
-        if ev:
-            ev[1].record()
+        mark(1)
         rt, kk, pairs = spr.route(part, n, sc, ws)
-        if ev:
-            ev[2].record()
-        s_out = spr.sparse_attn(q, k, v, part, rt, kk, sc, ws=ws)
-        if ev:
-            ev[3].record()
+        mark(2)
         pidx = spr.probe_rows(n, sc.n_probe, bt, h, dev)
-        p_out, p_sparse = spr.probe_dense(q, k, v, pidx, part, rt, kk, sc, ws)
+        if fused:
+            p_out, p_sparse = spr.probe_dense(q, k, v, pidx, part, rt, kk, sc, ws)
+            mark(3)
+            m, beta = spr.fit_residual(p_sparse, p_out, sc, ws)
+            mark(4)
+            spr.sparse_attn_apply(q, k, v, part, rt, kk, sc, m, beta, pidx, p_out, ws, out=o)
+            mark(5)
+        else:
+            s_out = spr.sparse_attn(q, k, v, part, rt, kk, sc, ws=ws)
+            mark(3)
+            p_out, p_sparse = spr.probe_dense(q, k, v, pidx, part, rt, kk, sc, ws)
+            mark(4)
+            m, beta = spr.fit_residual(p_sparse, p_out, sc, ws)
+            mark(5)
+            spr.apply_residual(s_out, m, beta, pidx, p_out, out_dtype=q.dtype, out=o)
+            mark(6)
         if ev:
-            ev[4].record()
-        m, beta = spr.fit_residual(p_sparse, p_out, sc, ws)
-        if ev:
-            ev[5].record()
-        spr.apply_residual(s_out, m, beta, pidx, p_out, out_dtype=q.dtype, out=o)
-        if ev:
-            ev[6].record()
             record.append(ev)
-        return {"S": s_out, "pidx": pidx, "pairs": pairs, "k": kk}
+        return {"part": part, "route": rt, "pidx": pidx, "pairs": pairs, "k": kk}
 
     for _ in range(args.warmup):
         step()
@@ -327,7 +334,9 @@ def run_ours(args, w):
     t_sparse = attn_kernel_ms / max(attn_kernel_n, 1) / 1e3
     peak, peak_src = measured_peak()
     achieved = sparse_flops / t_sparse / 1e12
-    roofline = {"kernel": "attn_tc_kernel<false> (block-sparse attention, tcgen05)", "bound": "tensor", "achieved": achieved,
+    kname = ("attn_tc_kernel<false, true> (block-sparse attention + fused correction, tcgen05)" if fused else
+             "attn_tc_kernel<false, false> (block-sparse attention, tcgen05)")
+    roofline = {"kernel": kname, "bound": "tensor", "achieved": achieved,
                 "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": DOMINANT_TRAFFIC_BYTES,
                 "peak_source": peak_src, "kernel_ms": t_sparse * 1e3, "kernel_launches_timed": attn_kernel_n,
                 "per_launch_flops": sparse_flops}
@@ -357,7 +366,8 @@ def run_ours(args, w):
     d2h = o.numel() * o.element_size()
 
     # ---- dense comparators and the error metric (outside the timed regions)
-    s_last = last["S"]
+    # the uncorrected sparse output of the last timed call's decisions (metric only)
+    s_last = spr.sparse_attn(q, k, v, last["part"], last["route"], last["k"], sc, ws=ws)
     dense = torch.empty(bt, h, n, d, dtype=torch.float32, device=dev)
     spr.dense_attn(q, k, v, block=w.block, out=dense)
     torch.cuda.synchronize()
@@ -512,7 +522,7 @@ def run_study_probe_budget(args, w):
                                  rank=w.rank, density=w.density, ridge_lambda=w.ridge_lambda)
         ws = spr.new_workspace(bt, h, n, d, cfg, q.device)
         pidx = spr.probe_rows(n, P, bt, h, q.device)
-        o, parts = spr.attention(q, k, v, cfg, ws=ws, return_parts=True)
+        o, parts = spr.attention(q, k, v, cfg, ws=ws, return_parts=True, fused=False)
         m, p = _err_summary(spr.row_errors(o, dense, pidx))
         mu, pu = _err_summary(spr.row_errors(parts["S"], dense, pidx))
         spr.check(ws)

@@ -52,7 +52,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct Layout {
   size_t header = 0, sample_idx, gamma, gamma_hi, gamma_lo, nrm, cent_k, cent_q, wf, whi, wlo, eg, dmat,
          prop_g0, prop_v0, labels, room, cnt, offs, cursor, closed, bucket, list0, list1, list_len, prop_g, prop_v,
-         perm_tmp, perm_cursor, qblk, partial, fit, kv_grouped, segmin, total;
+         perm_tmp, perm_cursor, qblk, partial, fit, kv_grouped, mhilo, segmin, total;
 };
 
 Layout make_layout(int heads, int N, int d, int block, int S, int P) {
@@ -67,6 +67,7 @@ Layout make_layout(int heads, int N, int d, int block, int S, int P) {
   // Regions read by the calls after partition come first, so that their offsets depend
   // only on the shapes (and P) each of those calls knows.
   L.kv_grouped = take(2 * 2 * H * G * block * D);  // K and V in key-group order, bf16
+  L.mhilo = take(2 * 2 * H * D * D);                // M as bf16 hi and lo (fused correction)
   L.partial = take(P > 0 ? spr::probe_partial_bytes(heads, P, static_cast<int>(G), d) : 0);
   L.fit = take(P > 0 ? sizeof(double) * H * spr::fit_scratch_doubles(P, d) : 0);
   L.sample_idx = take(sizeof(int) * static_cast<size_t>(S));
@@ -371,6 +372,56 @@ int sparsepr_sparse_attn(const void* Q, const void* K, const void* V, int dtype,
                          float scale, float* S_out, void* ws, sparsepr_stream_t stream) {
   return attention_common(Q, K, V, dtype, Bt, H, N, d, block, key_perm, key_gsize, query_perm, qblock_size, route, k,
                           scale, S_out, false, ws, stream);
+}
+
+int sparsepr_sparse_attn_apply(const void* Q, const void* K, const void* V, int dtype, int32_t Bt, int32_t H,
+                               int32_t N, int32_t d, int32_t block, const int32_t* key_perm, const int32_t* key_gsize,
+                               const int32_t* query_perm, const int32_t* qblock_size, const int32_t* route, int32_t k,
+                               float scale, const float* M, const float* beta, const int32_t* probe_idx, int32_t P,
+                               const float* probe_out, void* O, void* ws, sparsepr_stream_t stream) {
+  int rc;
+  if ((rc = check_shape(Bt, H, N, d)) || (rc = check_dtype(dtype)) || (rc = check_block(block))) return rc;
+  if (dtype != SPARSEPR_BF16 || d != 128 || block != 128)
+    return fail(SPARSEPR_ERR_UNSUPPORTED, "the fused correction is built for bf16, d = 128, block = 128");
+  if (!Q || !K || !V || !key_perm || !key_gsize || !query_perm || !qblock_size || !route || !M || !beta || !O || !ws)
+    return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
+  if (P < 0 || P > N || (P > 0 && (!probe_idx || !probe_out))) return fail(SPARSEPR_ERR_INVALID_ARG, "bad probe rows");
+  const int G = spr::ceil_div(N, block);
+  if (k < 1 || k > G) return fail(SPARSEPR_ERR_INVALID_ARG, "k=%d outside [1, %d]", k, G);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int heads = Bt * H;
+  const Layout L = make_layout(heads, N, d, block, 1, 0);
+  __nv_bfloat16* mh = at<__nv_bfloat16>(ws, L.mhilo);
+  SPR_CUDA(spr::launch_split_bf16(M, mh, mh + static_cast<size_t>(heads) * d * d, static_cast<size_t>(heads) * d * d, st),
+           "split M");
+  spr::AttnArgs a{};
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.f32 = false;
+  a.heads = heads;
+  a.N = N;
+  a.d = d;
+  a.block = block;
+  a.G = G;
+  a.k = k;
+  a.key_perm = key_perm;
+  a.key_gsize = key_gsize;
+  a.query_perm = query_perm;
+  a.qblock_size = qblock_size;
+  a.route = route;
+  a.scale_log2 = resolve_scale(scale, d) * kLog2e;
+  a.out = nullptr;
+  a.status = &header(ws)->status;
+  a.k_grouped = at<char>(ws, L.kv_grouped);
+  a.v_grouped = at<char>(ws, L.kv_grouped) + static_cast<size_t>(heads) * G * block * d * 2;
+  a.m_hilo = mh;
+  a.beta = beta;
+  a.out_bf16 = O;
+  SPR_CUDA(spr::launch_attention(a, false, st), "sparse attention with correction");
+  SPR_CUDA(spr::launch_probe_overwrite_bf16(probe_idx, probe_out, heads, N, P, static_cast<__nv_bfloat16*>(O), st),
+           "probe rows");
+  return SPARSEPR_OK;
 }
 
 int sparsepr_dense_attn(const void* Q, const void* K, const void* V, int dtype, int32_t Bt, int32_t H, int32_t N,

@@ -24,6 +24,12 @@ struct AttnArgs {
   // written by the sparse tensor-core path before its attention kernel; null otherwise.
   void* k_grouped;
   void* v_grouped;
+  // Fused correction (sparse, bf16, d = 128 only): when m_hilo is set the kernel writes
+  // O = S + S M^T + beta as bf16 to out_bf16 instead of S to out.  m_hilo holds M (per
+  // head [128, 128]) as bf16 hi parts for all heads, then the lo parts.
+  const void* m_hilo;
+  const float* beta;
+  void* out_bf16;
 };
 
 struct ProbeArgs {

@@ -60,9 +60,10 @@ constexpr float kInf = __builtin_huge_valf();
 // overwritten), P written to shared memory, PV done (which frees the stream's V and P
 // buffers and means O_x holds every finished tile), drain; and the last PV of both
 // streams.
+// Fused correction only: M (hi, lo) landed, the merged S tile (hi, lo) written, S M^T done.
 enum : int {
   kQFull = 0, kKFull0 = 1, kVFull0 = 3, kSFull0 = 5, kSFree0 = 7, kPFull0 = 9, kVEmpty0 = 11, kDrain0 = 13,
-  kOFinal = 15, kNumBars = 16
+  kOFinal = 15, kMFull = 16, kSFin = 17, kCorr = 18, kNumBars = 19
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -113,13 +114,16 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-template <bool DENSE>
+// FUSED (sparse only): O = S + S M^T + beta is formed in the epilogue and written as
+// bf16 to out_bf16; S itself never leaves the SM.  Otherwise S (fp32) goes to out.
+template <bool DENSE, bool FUSED>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, int N, int G, int k,
-                   const int* __restrict__ key_gsize, const int* __restrict__ query_perm,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmM, int N, int G,
+                   int k, const int* __restrict__ key_gsize, const int* __restrict__ query_perm,
                    const int* __restrict__ qblock_size, const int* __restrict__ route, float scale_log2,
-                   float* __restrict__ out, int* __restrict__ status) {
+                   float* __restrict__ out, const float* __restrict__ beta, __nv_bfloat16* __restrict__ out_bf16,
+                   int* __restrict__ status) {
   extern __shared__ uint8_t dsmem[];
   __shared__ __align__(8) uint64_t bars[kNumBars];
   __shared__ uint32_t tmem_slot;
@@ -149,6 +153,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc::mbar_init(bar(kDrain0 + x), 1);
     }
     tc::mbar_init(bar(kOFinal), 2);
+    tc::mbar_init(bar(kMFull), 1);
+    tc::mbar_init(bar(kSFin), 256);
+    tc::mbar_init(bar(kCorr), 1);
     abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -163,6 +170,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   const int row0 = head * N;  // first row of this head in the [heads * N, 128] tensor maps
   out += static_cast<size_t>(head) * N * 128;
+  if (FUSED) out_bf16 += static_cast<size_t>(head) * N * 128;
   const size_t goff = static_cast<size_t>(head) * G;
   const int nq = DENSE ? min(128, N - b * 128) : qblock_size[goff + b];
   const int* qperm = DENSE ? nullptr : query_perm + (goff + b) * 128;
@@ -228,6 +236,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (lane == 0) {
         for (int j = max(0, issued - 2); j < issued; ++j) drain_wait(bar(full0 + (j & 1)), (j >> 1) & 1);
         if (isK) drain_wait(bar(kQFull), 0);
+        // fused correction: M of this head (hi into K buffer 0, lo into K buffer 1) once
+        // every MMA of the attention is done and the K buffers are free
+        if (FUSED && isK && tc::mbar_wait(bar(kOFinal), 0, abort_v, status)) {
+          tc::mbar_arrive_expect_tx(bar(kMFull), 2 * kTile);
+          tc::tma_load_2d(sK(0), &tmM, 0, head * 128, bar(kMFull));
+          tc::tma_load_2d(sK(0) + 128 * 128, &tmM, 64, head * 128, bar(kMFull));
+          tc::tma_load_2d(sK(1), &tmM, 0, (gridDim.y + head) * 128, bar(kMFull));
+          tc::tma_load_2d(sK(1) + 128 * 128, &tmM, 64, (gridDim.y + head) * 128, bar(kMFull));
+          drain_wait(bar(kMFull), 0);  // the copies land before this thread can exit
+        }
       }
       __syncwarp();
     } else if (lane == 0) {
@@ -275,6 +293,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc::mma_commit(bar(kOFinal));
       tc::mma_commit(bar(kDrain0 + x));
       drain_wait(bar(kDrain0 + x), 0);
+      if (FUSED && x == 0 && ok && tc::mbar_wait(bar(kMFull), 0, abort_v, status) &&
+          tc::mbar_wait(bar(kSFin), 0, abort_v, status)) {
+        // S M^T into TMEM columns [0, 128) (S of stream 0, free now) in split precision:
+        // S_hi M_hi + S_hi M_lo + S_lo M_hi, S tiles in the V buffers, M tiles in the K ones
+        tc::fence_after_sync();
+        const uint32_t sA[3] = {sV(0), sV(0), sV(1)}, sB[3] = {sK(0), sK(1), sK(0)};
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            tc::mma_ss(tbase, tc::sdesc_sw128(sA[t] + koff, 16, 1024), tc::sdesc_sw128(sB[t] + koff, 16, 1024),
+                       kIdMma, (t > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc::mma_commit(bar(kCorr));
+        tc::mma_commit(bar(kDrain0));
+        drain_wait(bar(kDrain0), 1);
+      }
     }
   } else {
     // ------------------------------------------------------------------ softmax
@@ -379,6 +416,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float2* s_ml = reinterpret_cast<float2*>(gsP0);
     if (fin) s_ml[x * 128 + r] = make_float2(m_run, l_run);
     tc::named_bar_sync(1, 256);  // every softmax thread reaches this exactly once
+    float sv[FUSED ? 64 : 1];  // this thread's 64 merged S values (fused correction)
     if (fin) {
       tc::fence_after_sync();
       const float2 a0 = s_ml[r], a1 = s_ml[128 + r];
@@ -400,7 +438,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) o1[i] = 0u;
         }
-        if (tok >= 0) {
+        if (FUSED) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            sv[32 * q + i] = fmaf(__uint_as_float(o0[i]), g0, __uint_as_float(o1[i]) * g1);
+        } else if (tok >= 0) {
           float4* dst = reinterpret_cast<float4*>(out + static_cast<size_t>(tok) * 128 + col);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -409,6 +451,53 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int t = 0; t < 4; ++t)
               v[t] = fmaf(__uint_as_float(o0[4 * i + t]), g0, __uint_as_float(o1[4 * i + t]) * g1);
             dst[i] = make_float4(v[0], v[1], v[2], v[3]);
+          }
+        }
+      }
+    }
+    if (FUSED) {
+      // ---- the correction: row r of the merged S (columns [64 x, 64 x + 64)) as bf16
+      // hi and lo into the V buffers (K-major A operands), S M^T on the tensor cores,
+      // then O = S + S M^T + beta in bf16
+      if (fin) {
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float a = sv[8 * c8 + 2 * t], b2 = sv[8 * c8 + 2 * t + 1];
+            const __nv_bfloat16 ah = __float2bfloat16_rn(a), bh = __float2bfloat16_rn(b2);
+            hi[t] = pack_bf16x2(a, b2);
+            lo[t] = pack_bf16x2(a - __bfloat162float(ah), b2 - __bfloat162float(bh));
+          }
+          st_shared_v4(sV(0) + tc::sw128_offset(r, 8 * x + c8), hi[0], hi[1], hi[2], hi[3]);
+          st_shared_v4(sV(1) + tc::sw128_offset(r, 8 * x + c8), lo[0], lo[1], lo[2], lo[3]);
+        }
+      }
+      tc::fence_proxy_async();
+      tc::mbar_arrive(bar(kSFin));
+      if (fin && warp_wait(bar(kCorr), 0, abort_v, status)) {
+        tc::fence_after_sync();
+        const float* bh = beta + static_cast<size_t>(head) * 128 + 64 * x;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t c32[32];
+          tc::tmem_ld32(tbase + lane_off + 64 * x + 32 * q, c32);
+          tc::tmem_wait_ld();
+          if (tok >= 0) {
+            uint4* dst = reinterpret_cast<uint4*>(out_bf16 + static_cast<size_t>(tok) * 128 + 64 * x + 32 * q);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint32_t w[4];
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                const int c = 8 * i + 2 * t;
+                const float v0 = sv[32 * q + c] + __uint_as_float(c32[c]) + __ldg(bh + 32 * q + c);
+                const float v1 = sv[32 * q + c + 1] + __uint_as_float(c32[c + 1]) + __ldg(bh + 32 * q + c + 1);
+                w[t] = pack_bf16x2(v0, v1);
+              }
+              dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
           }
         }
       }
@@ -519,7 +608,9 @@ cudaError_t attn_timing_read(double* ms_total, long long* launches) {
 cudaError_t launch_attention_tc(const AttnArgs& a, bool dense, int* status, cudaStream_t st) {
   const size_t smem = attn_tc_smem_bytes(dense ? a.G : a.k);
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  auto kern = dense ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  const bool fused = !dense && a.m_hilo != nullptr;
+  if (fused && (a.beta == nullptr || a.out_bf16 == nullptr)) return cudaErrorInvalidValue;
+  auto kern = dense ? attn_tc_kernel<true, false> : fused ? attn_tc_kernel<false, true> : attn_tc_kernel<false, false>;
   // The register re-split must fit in what the block is launched with, or the
   // setmaxnreg.inc of the softmax warpgroups would never be granted.
   cudaFuncAttributes fa;
@@ -530,11 +621,17 @@ cudaError_t launch_attention_tc(const AttnArgs& a, bool dense, int* status, cuda
   const long long grows = static_cast<long long>(a.heads) * a.G * 128;
   if (rows > 0x7fffffffLL || grows > 0x7fffffffLL) return cudaErrorInvalidValue;  // TMA coordinates are int32
   if (!dense && (a.k_grouped == nullptr || a.v_grouped == nullptr)) return cudaErrorInvalidValue;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, tm;
   const bool maps = bf16_map(&tq, a.Q, rows, 1) &&
                     (dense ? bf16_map(&tk, a.K, rows, 128) && bf16_map(&tv, a.V, rows, 128)
                            : bf16_map(&tk, a.k_grouped, grows, 128) && bf16_map(&tv, a.v_grouped, grows, 128));
   if (!maps) return cudaErrorInvalidValue;
+  // M of every head as bf16 hi rows [0, 128 heads) then lo rows [128 heads, 256 heads)
+  if (fused) {
+    if (!bf16_map(&tm, a.m_hilo, 2LL * a.heads * 128, 128)) return cudaErrorInvalidValue;
+  } else {
+    tm = tk;  // unused
+  }
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   if (!dense) {
@@ -557,9 +654,9 @@ cudaError_t launch_attention_tc(const AttnArgs& a, bool dense, int* status, cuda
     }
   }
   if (ev.first != nullptr && (e = cudaEventRecord(ev.first, st)) != cudaSuccess) return e;
-  kern<<<dim3(a.G, a.heads), kTcThreads, smem, st>>>(tq, tk, tv, a.N, a.G, a.k, a.key_gsize,
-                                                       a.query_perm, a.qblock_size, a.route, a.scale_log2, a.out,
-                                                       status);
+  kern<<<dim3(a.G, a.heads), kTcThreads, smem, st>>>(
+      tq, tk, tv, tm, a.N, a.G, a.k, a.key_gsize, a.query_perm, a.qblock_size, a.route, a.scale_log2, a.out,
+      a.beta, static_cast<__nv_bfloat16*>(a.out_bf16), status);
   e = counted(cudaGetLastError(), 1);
   if (ev.first != nullptr) {
     cudaError_t e2 = cudaEventRecord(ev.second, st);

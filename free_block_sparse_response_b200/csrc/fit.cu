@@ -571,6 +571,13 @@ static cudaError_t launch_apply_t(const float* S, const float* M, const float* b
   return counted(cudaGetLastError(), 1);
 }
 
+cudaError_t launch_probe_overwrite_bf16(const int* probe_idx, const float* probe_out, int heads, int N, int P,
+                                       __nv_bfloat16* O, cudaStream_t st) {
+  if (P == 0) return cudaSuccess;
+  probe_overwrite_kernel<128, __nv_bfloat16><<<dim3(P, heads), 128, 0, st>>>(probe_idx, probe_out, N, P, O);
+  return counted(cudaGetLastError(), 1);
+}
+
 cudaError_t launch_apply(const float* S, const float* M, const float* beta, const int* probe_idx,
                          const float* probe_out, int heads, int N, int d, int P, void* O, bool out_f32,
                          cudaStream_t st) {

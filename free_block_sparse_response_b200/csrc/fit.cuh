@@ -1,5 +1,6 @@
 // Launch interface of the fit and apply kernels (internal to the library).
 #pragma once
+#include <cuda_bf16.h>
 
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -11,6 +12,9 @@ size_t fit_smem_bytes(int d, int P);
 cudaError_t launch_fit(const float* xs, const float* dp, const float* weights, int heads, int d, int P,
                        double lambda, int rank, int weight_mode, double* scratch, float* M, float* beta,
                        int* status, cudaStream_t st);
+// Probe rows of a bf16 output (d = 128) set to the exact probe outputs.
+cudaError_t launch_probe_overwrite_bf16(const int* probe_idx, const float* probe_out, int heads, int N, int P,
+                                       __nv_bfloat16* O, cudaStream_t st);
 cudaError_t launch_apply(const float* S, const float* M, const float* beta, const int* probe_idx,
                          const float* probe_out, int heads, int N, int d, int P, void* O, bool out_f32,
                          cudaStream_t st);

@@ -28,6 +28,7 @@ EXPORTED_SYMBOLS = (
     "sparsepr_last_error", "sparsepr_test_fill_workspace_size", "sparsepr_test_fill",
     "sparsepr_test_topk", "sparsepr_row_errors", "sparsepr_launch_count", "sparsepr_fit_residual_noalloc",
     "sparsepr_kernel_timing", "sparsepr_kernel_timing_read", "sparsepr_test_fill_segmented",
+    "sparsepr_sparse_attn_apply",
 )
 
 
@@ -89,6 +90,9 @@ def lib() -> ctypes.CDLL:
                                           _vp, _vp]),
         "sparsepr_sparse_attn": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32, _i32, _vp,
                                                 _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _vp]),
+        "sparsepr_sparse_attn_apply": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32, _i32,
+                                                      _vp, _vp, _vp, _vp, _vp, _i32, _f32, _vp, _vp, _vp, _i32,
+                                                      _vp, _vp, _vp, _vp]),
         "sparsepr_dense_attn": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32, _i32, _f32,
                                                _vp, _vp, _vp]),
         "sparsepr_probe_dense": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32, _i32, _vp,
@@ -229,6 +233,26 @@ def sparse_attn(q, k, v, part: Partition, rt: torch.Tensor, kk: int, cfg: Sparse
     return s_out
 
 
+def fused_supported(q: torch.Tensor, cfg: SparsePRConfig) -> bool:
+    """Whether the fused correction (sparse_attn_apply) is built for this shape."""
+    return q.dtype == torch.bfloat16 and q.shape[-1] == 128 and cfg.block == 128
+
+
+def sparse_attn_apply(q, k, v, part: Partition, rt: torch.Tensor, kk: int, cfg: SparsePRConfig, m: torch.Tensor,
+                      beta: torch.Tensor, probe_idx: torch.Tensor, probe_out: torch.Tensor, ws: torch.Tensor,
+                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Block-sparse attention with O = S + S M^T + beta formed in its epilogue, probe
+    rows set to probe_out; O [Bt,H,N,d] bf16 (bf16, d = 128, B = 128)."""
+    _need_cuda(q, k, v, rt, m, beta, probe_idx, probe_out, ws)
+    bt, h, n, d = q.shape
+    o = torch.empty(bt, h, n, d, dtype=torch.bfloat16, device=q.device) if out is None else out
+    p = probe_idx.shape[-1]
+    _call("sparsepr_sparse_attn_apply", _p(q), _p(k), _p(v), _dtype_code(q), bt, h, n, d, cfg.block,
+          _p(part.key_perm), _p(part.key_gsize), _p(part.query_perm), _p(part.qblock_size), _p(rt), kk,
+          cfg.scale, _p(m), _p(beta), _p(probe_idx), p, _p(probe_out), _p(o), _p(ws), _stream(q))
+    return o
+
+
 def dense_attn(q, k, v, block: int = 128, scale: float = 0.0, out: Optional[torch.Tensor] = None,
                ws: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Dense softmax attention of every row with the same kernel family (fp32 out)."""
@@ -297,21 +321,33 @@ def apply_residual(s_out, m, beta, probe_idx, probe_out, out_dtype=torch.bfloat1
 # --------------------------------------------------------------------------- the call
 
 def attention(q, k, v, cfg: SparsePRConfig, ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-              return_parts: bool = False):
-    """One SparsePR attention call: partition, route, sparse attention, probes, fit,
-    apply.  Returns O [Bt,H,N,d] in q's dtype (and the intermediates if asked).
-    Asynchronous on the current stream; ``check(ws)`` surfaces device-side errors."""
+              return_parts: bool = False, fused: Optional[bool] = None):
+    """One SparsePR attention call.  Returns O [Bt,H,N,d] in q's dtype (and the
+    intermediates if asked).  Asynchronous on the current stream; ``check(ws)`` surfaces
+    device-side errors.
+
+    fused (default: when built for the shape and no intermediates are asked for):
+    partition, route, probe rows, fit, then the sparse attention with the correction in
+    its epilogue (S never leaves the SM).  Otherwise: partition, route, sparse attention
+    (S fp32), probe rows, fit, apply."""
     _need_cuda(q, k, v)
     bt, h, n, d = q.shape
     if ws is None:
         ws = new_workspace(bt, h, n, d, cfg, q.device)
+    if fused is None:
+        fused = not return_parts and fused_supported(q, cfg)
     part = partition(q, k, cfg, ws)
     rt, kk, pairs = route(part, n, cfg, ws)
-    s_out = sparse_attn(q, k, v, part, rt, kk, cfg, ws=ws)
     pidx = probe_rows(n, cfg.n_probe, bt, h, q.device)
+    s_out = None
+    if not fused:
+        s_out = sparse_attn(q, k, v, part, rt, kk, cfg, ws=ws)
     p_out, p_sparse = probe_dense(q, k, v, pidx, part, rt, kk, cfg, ws)
     m, beta = fit_residual(p_sparse, p_out, cfg, ws)
-    o = apply_residual(s_out, m, beta, pidx, p_out, out_dtype=q.dtype, out=out)
+    if fused:
+        o = sparse_attn_apply(q, k, v, part, rt, kk, cfg, m, beta, pidx, p_out, ws, out=out)
+    else:
+        o = apply_residual(s_out, m, beta, pidx, p_out, out_dtype=q.dtype, out=out)
     if not return_parts:
         return o
     return o, {"partition": part, "route": rt, "k": kk, "executed_pairs": pairs, "S": s_out, "probe_idx": pidx,

@@ -152,6 +152,24 @@ SPARSEPR_API int sparsepr_sparse_attn(const void* Q, const void* K, const void* 
                          const int32_t* route, int32_t k, float scale, float* S_out,
                          void* ws, sparsepr_stream_t stream);
 
+/* (c + e, fused) Block-sparse attention with the residual correction applied in the
+ * attention kernel's epilogue (probe-first order: sparsepr_probe_dense and
+ * sparsepr_fit_residual run before it):
+ *   O[i] = s_i + M s_i + beta for every row, then the probe rows set to probe_out;
+ * s_i as in sparsepr_sparse_attn, never written to memory.  M s_i is formed on the
+ * tensor cores from bf16 hi + lo parts of s_i and M (three products, ~16-bit operands).
+ * O [Bt,H,N,d] bf16.  Built for dtype BF16, d = 128, block = 128 (other shapes:
+ * SPARSEPR_ERR_UNSUPPORTED; use sparsepr_sparse_attn + sparsepr_apply_residual).  The
+ * workspace is required.  Source: the abstract (the fitted map predicts each unprobed
+ * query's residual, added to its sparse output); the order of the steps is free. */
+SPARSEPR_API int sparsepr_sparse_attn_apply(const void* Q, const void* K, const void* V, int dtype,
+                         int32_t Bt, int32_t H, int32_t N, int32_t d, int32_t block,
+                         const int32_t* key_perm, const int32_t* key_gsize,
+                         const int32_t* query_perm, const int32_t* qblock_size,
+                         const int32_t* route, int32_t k, float scale, const float* M,
+                         const float* beta, const int32_t* probe_idx, int32_t P,
+                         const float* probe_out, void* O, void* ws, sparsepr_stream_t stream);
+
 /* Dense softmax attention of every row against all N keys with the same kernel
  * family (the comparator the density budget is measured against):
  *   O_out [Bt,H,N,d] fp32. */

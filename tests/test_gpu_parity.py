@@ -184,6 +184,32 @@ def test_call_bf16_d128_ragged_long_tail():
     _check_call(w, spr_cfg(w, n_sampled=128, n_probe=80, rank=8))
 
 
+@pytest.mark.parametrize("grid,heads", [(None, 3), ((5, 9, 23), 2)])
+def test_fused_correction_matches_unfused_and_oracle(grid, heads):
+    """Probe-first pipeline with O = S + S M^T + beta in the attention epilogue (S never
+    written): on the same partition, routes and fit it must equal the unfused call's O
+    (bf16 output rounding apart) and the oracle, with probe rows exact.  The second case
+    has a ragged N (last key group and query block of 11 tokens)."""
+    w = CONFIGS["small"] if grid is None else CONFIGS["small"].with_(grid=grid, heads=heads)
+    cfg = spr_cfg(w) if grid is None else spr_cfg(w, n_sampled=128, n_probe=80, rank=8)
+    q, k, v = make_inputs(w, 0, heads=heads)
+    o_ref, parts = run_call(w, q, k, v, cfg)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o = spr.sparse_attn_apply(qd, kd, vd, parts["partition"], parts["route"], parts["k"], cfg, parts["M"],
+                              parts["beta"], parts["probe_idx"], parts["probe_out"], parts["ws"])
+    spr.check(parts["ws"])
+    n = w.n_tokens
+    for h in range(heads):
+        assert rel(o[0, h].double().cpu().numpy(), o_ref[0, h].double().cpu().numpy()) <= 2e-3
+        ref = oracle_on_gpu_decisions(q, k, v, parts, h, cfg, n)
+        assert rel(o[0, h].double().cpu().numpy(), ref["O"]) <= TOL_BF16
+        want = parts["probe_out"][0, h].to(torch.bfloat16)
+        assert torch.equal(o[0, h][parts["probe_idx"][0, h].long()].cpu(), want.cpu())
+    # the default call takes the fused path and gives the same output
+    o_default = spr.attention(qd, kd, vd, cfg)
+    assert torch.equal(o_default.cpu(), o.cpu())
+
+
 def test_full_density_equals_dense():
     """k = G: sparse output is dense attention; the fitted map is ~0."""
     w = CONFIGS["small"].with_(grid=(2, 16, 32), heads=2)
