@@ -30,9 +30,9 @@ METRIC = "SparsePR ms/call & eff. TFLOP/s at 22% pair density; mean rel-L2 err v
 UNIT = "TFLOP/s (dense-equivalent, 4*d*N^2*H per call)"
 
 # DRAM bytes per launch of the dominant kernel from an ncu capture of the same kernel
-# build (profiles/), scaled by heads to the 40-head launch; None whenever that kernel
-# has changed since the capture.
-DOMINANT_TRAFFIC_BYTES = None
+# build (profiles/attn_tc_kernel_video_4h.md: 301.4 MB on 4 heads), scaled by heads to
+# the 40-head launch; None whenever that kernel has changed since the capture.
+DOMINANT_TRAFFIC_BYTES = 3.014e9
 
 
 def parse_args():
