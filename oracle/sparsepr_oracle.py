@@ -204,7 +204,8 @@ def partition(q: np.ndarray, k: np.ndarray, tau: float, block: int, n_sampled: i
     give every query the coordinates u_i[g] = tau q_i . mu_g (the response-space
     centroid of group g is tau Q_S mu_g, linear in the key); queries are then
     clustered in those coordinates.  Keys are never re-clustered afterwards.
-    Returns key/query labels, mu, the coordinates and the block scores (fp32).
+    Returns key/query labels, mu, the coordinates and the block scores (fp32; the
+    "centroid" reading of ``routing_scores``).
     """
     n = q.shape[0]
     g_count = n_groups(n, block)
@@ -246,6 +247,35 @@ def partition_semantic(q: np.ndarray, k: np.ndarray, tau: float, block: int, ite
         dump["query_dist"] = qd
     return {"key_labels": key_labels, "mu": mu, "coords": coords, "query_labels": query_labels,
             "block_scores": block_scores}
+
+
+def routing_scores(q: np.ndarray, k: np.ndarray, tau: float, key_labels: np.ndarray, query_labels: np.ndarray,
+                   g_count: int, mode: str = "centroid") -> np.ndarray:
+    """Block-routing scores Sc[b][g] (fp32) under the three readings of "routing up to
+    a target density" the comparison covers ([abs]; [news], components paragraph):
+
+    * "centroid": tau qbar_b . mu_g, the mean over block b of the query coordinates
+      (the method's reading; equals ``partition()["block_scores"]``);
+    * "size_corrected": tau qbar_b . mu_g + log n_g, the first-order log of the
+      attention mass the block's mean query puts on group g (n_g members);
+    * "lse": log sum_{j in g} exp(tau qbar_b . k_j), that mass itself.
+    qbar_b and mu_g are the member means of block b and group g (fp64)."""
+    qbar = group_means(q, query_labels, g_count)
+    mu = group_means(k, key_labels, g_count)
+    if mode == "centroid":
+        return (tau * (qbar @ mu.T)).astype(np.float32)
+    sizes = np.bincount(key_labels, minlength=g_count)
+    if mode == "size_corrected":
+        return (tau * (qbar @ mu.T) + np.log(np.maximum(sizes, 1))[None, :]).astype(np.float32)
+    if mode == "lse":
+        out = np.empty((qbar.shape[0], g_count))
+        logits = tau * (qbar @ k.T)                       # [Gq, N]
+        for g in range(g_count):
+            x = logits[:, key_labels == g]
+            m = x.max(axis=1, keepdims=True)
+            out[:, g] = (m + np.log(np.exp(x - m).sum(axis=1, keepdims=True)))[:, 0]
+        return out.astype(np.float32)
+    raise ValueError(f"unknown routing score mode {mode}")
 
 
 # ------------------------------------------------------------------ step 5: routing
@@ -457,7 +487,7 @@ def rel_l2_errors(o: np.ndarray, o_dense: np.ndarray, probe_idx: np.ndarray) -> 
 
 def sparsepr_head(q, k, v, *, block, n_sampled, n_probe, density, ridge_lambda, rank,
                   kmeans_iters=4, scale=None, weight_mode="inv_norm", inject=None,
-                  dump=None, partition_mode="response") -> dict:
+                  dump=None, partition_mode="response", route_scores="centroid") -> dict:
     """One SparsePR call on one (batch, head).  ``inject`` may hold any of
     sample_idx, probe_idx, key_labels, query_labels, routes (e.g. the CUDA path's
     decisions) to run the later steps on them.  ``partition_mode`` "semantic" swaps
@@ -479,7 +509,12 @@ def sparsepr_head(q, k, v, *, block, n_sampled, n_probe, density, ridge_lambda, 
     key_sizes = np.bincount(kl, minlength=g_count)
     block_sizes = np.bincount(ql, minlength=g_count)
     kk = route_k(n, block, density, n_probe)
-    routes = np.asarray(inject["routes"]) if "routes" in inject else route(part["block_scores"], kk)
+    if "routes" in inject:
+        routes = np.asarray(inject["routes"])
+    else:
+        scores = part["block_scores"] if route_scores == "centroid" else routing_scores(
+            q, k, tau, kl, ql, g_count, route_scores)
+        routes = route(scores, kk)
     probe_idx = np.asarray(inject["probe_idx"]) if "probe_idx" in inject else midpoint_stride(n, n_probe)
     pairs = executed_pairs(routes, key_sizes, block_sizes, probe_idx.size, n)
     s = sparse_attention(q, k, v, tau, kl, ql, routes)

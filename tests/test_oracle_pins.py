@@ -502,3 +502,36 @@ def test_semantic_partition_recovers_planted_raw_clusters():
     assert len(set(zip(sem["query_labels"].tolist(), query_truth.tolist()))) == g_count
     assert np.bincount(sem["query_labels"]).tolist() == [block] * g_count
 
+
+
+# --------------------------------------------------------------- routing score readings
+
+def test_routing_scores_bruteforce_and_jensen_bound():
+    """Each score reading against explicit loops over members; LSE >= size-corrected
+    everywhere (Jensen: log sum exp >= log n + mean), with equality for a group whose
+    keys are all equal; "centroid" equals the partition's block scores."""
+    rng = _rng(41)
+    n, d, block = 80, 6, 16
+    q, k = rng.normal(size=(n, d)), rng.normal(size=(n, d))
+    tau = 0.7
+    part = O.partition(q, k, tau, block, n_sampled=20, iters=2)
+    kl, ql = part["key_labels"], part["query_labels"]
+    g = O.n_groups(n, block)
+    k2 = k.copy()
+    k2[kl == 2] = k2[kl == 2][0]      # group 2: identical keys
+    cen = O.routing_scores(q, k, tau, kl, ql, g, "centroid")
+    assert np.array_equal(cen, part["block_scores"])
+    siz = O.routing_scores(q, k, tau, kl, ql, g, "size_corrected")
+    lse = O.routing_scores(q, k, tau, kl, ql, g, "lse")
+    for b in range(g):
+        qb = q[ql == b].mean(axis=0)
+        for gg in range(g):
+            members = np.flatnonzero(kl == gg)
+            logits = [tau * float(qb @ k[j]) for j in members]
+            mu = k[members].mean(axis=0)
+            assert siz[b, gg] == pytest.approx(tau * float(qb @ mu) + math.log(len(members)), rel=1e-6, abs=1e-6)
+            assert lse[b, gg] == pytest.approx(math.log(sum(math.exp(x) for x in logits)), rel=1e-6, abs=1e-6)
+    assert (lse >= siz - 1e-5).all()
+    lse2 = O.routing_scores(q, k2, tau, kl, ql, g, "lse")
+    siz2 = O.routing_scores(q, k2, tau, kl, ql, g, "size_corrected")
+    assert np.allclose(lse2[:, 2], siz2[:, 2], rtol=1e-6, atol=1e-5)
