@@ -44,7 +44,7 @@ def parse_args():
     ap.add_argument("--config", default="video")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--study", choices=["ablation", "probe-budget"], default=None,
+    ap.add_argument("--study", choices=["ablation", "probe-budget", "routing"], default=None,
                     help="error studies instead of the timed run (one JSON line per variant)")
     return ap.parse_args()
 
@@ -534,6 +534,31 @@ def run_study_probe_budget(args, w):
         del ws
 
 
+def run_study_routing(args, w):
+    """Error of the three block-routing score readings (centroid, size-corrected,
+    LSE) at the same uniform k, hence the same executed-pair count, with and without
+    the probe-fitted correction."""
+    _, spr = _gpu_modules()
+    q, k, v, dense = _study_inputs(args, w)
+    bt, h, n, d = q.shape
+    for mode, name in ((spr.ROUTE_CENTROID, "centroid"), (spr.ROUTE_SIZE_CORRECTED, "size-corrected"),
+                       (spr.ROUTE_LSE, "lse")):
+        cfg = spr.SparsePRConfig(block=w.block, n_sampled=w.n_sampled, n_probe=w.n_probe, kmeans_iters=w.kmeans_iters,
+                                 rank=w.rank, density=w.density, ridge_lambda=w.ridge_lambda, route_scores=mode)
+        ws = spr.new_workspace(bt, h, n, d, cfg, q.device)
+        pidx = spr.probe_rows(n, w.n_probe, bt, h, q.device)
+        o, parts = spr.attention(q, k, v, cfg, ws=ws, return_parts=True, fused=False)
+        m, p = _err_summary(spr.row_errors(o, dense, pidx))
+        mu, pu = _err_summary(spr.row_errors(parts["S"], dense, pidx))
+        spr.check(ws)
+        print(json.dumps({"study": "routing", "scores": name, "workload": config_block(w, args)["workload"],
+                          "k": parts["k"], "density": float(parts["executed_pairs"].double().sum()) /
+                          (float(n) ** 2 * h * bt), "mean_rel_l2": m, "p99_rel_l2": p,
+                          "uncorrected_mean_rel_l2": mu, "uncorrected_p99_rel_l2": pu, "seed": args.seed}),
+              flush=True)
+        del ws
+
+
 def main():
     args = parse_args()
     w = workload(args)
@@ -541,6 +566,8 @@ def main():
         run_study_ablation(args, w)
     elif args.study == "probe-budget":
         run_study_probe_budget(args, w)
+    elif args.study == "routing":
+        run_study_routing(args, w)
     elif args.impl == "reference":
         run_reference(args, w)
     else:

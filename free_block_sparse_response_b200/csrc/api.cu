@@ -187,6 +187,10 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
   if (p->partition_mode != SPARSEPR_PARTITION_RESPONSE && p->partition_mode != SPARSEPR_PARTITION_SEMANTIC)
     return fail(SPARSEPR_ERR_INVALID_ARG, "unknown partition_mode %d", p->partition_mode);
   const bool semantic = p->partition_mode == SPARSEPR_PARTITION_SEMANTIC;
+  if (p->route_scores < SPARSEPR_ROUTE_CENTROID || p->route_scores > SPARSEPR_ROUTE_LSE)
+    return fail(SPARSEPR_ERR_INVALID_ARG, "unknown route_scores %d", p->route_scores);
+  if (p->route_scores == SPARSEPR_ROUTE_LSE && (dtype == SPARSEPR_F32 || d != 128 || p->block != 128))
+    return fail(SPARSEPR_ERR_UNSUPPORTED, "LSE routing scores are built for bf16, d = 128, block = 128");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int heads = Bt * H, B = p->block, G = spr::ceil_div(N, B), S = p->n_sampled;
   const bool f32 = dtype == SPARSEPR_F32;
@@ -293,6 +297,9 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
   else SPR_CUDA(spr::launch_gram(cent_k, true, static_cast<size_t>(G) * d, nullptr, G, heads, d, gamma, st), "mu gram");
   if ((rc = cluster(Q, cent_q, query_perm, qblock_size))) return rc;
   SPR_CUDA(spr::launch_block_scores(cent_q, cent_k, G, heads, d, tau, block_scores, st), "block scores");
+  SPR_CUDA(spr::launch_route_scores(p->route_scores, block_scores, K, N, heads, G, G, key_perm, key_gsize, cent_q, tau,
+                                    st),
+           "routing scores");
   return SPARSEPR_OK;
 }
 

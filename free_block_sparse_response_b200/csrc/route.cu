@@ -5,6 +5,8 @@
 // and the executed-pair density counts the exact probe rows.  Each query block keeps the
 // k key groups with the largest score (ties to the lower group), listed in ascending
 // group order; one warp per block row selects them by radix select on 64-bit keys.
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "route.cuh"
 
@@ -104,6 +106,54 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Sc[b][g] += log n_g (size-corrected scores).
+__global__ void size_correct_kernel(float* __restrict__ sc, const int* __restrict__ key_gsize, int Gq, int G) {
+  const int head = blockIdx.y;
+  const size_t base = static_cast<size_t>(head) * Gq * G;
+  for (int x = blockIdx.x * blockDim.x + threadIdx.x; x < Gq * G; x += gridDim.x * blockDim.x) {
+    const int g = x % G;
+    sc[base + x] += logf(static_cast<float>(max(key_gsize[static_cast<size_t>(head) * G + g], 1)));
+  }
+}
+
+// Sc[b][g] = log sum_{j in g} exp(tau qbar_b . k_j): one CTA per (group, head, 256
+// blocks); the group's keys in shared memory, read by every thread at once;
+// thread = block b, its qbar_b in registers, online max / sum over the members.
+__global__ void __launch_bounds__(256) lse_scores_kernel(const __nv_bfloat16* __restrict__ K, int N, int Gq, int G,
+                                                         const int* __restrict__ key_perm,
+                                                         const int* __restrict__ key_gsize,
+                                                         const float* __restrict__ qbar, float tau,
+                                                         float* __restrict__ sc) {
+  __shared__ __nv_bfloat16 sk[128][128];  // every thread reads the same element: broadcast
+  const int g = blockIdx.x, head = blockIdx.y, b = blockIdx.z * 256 + threadIdx.x;
+  const size_t grp = static_cast<size_t>(head) * G + g;
+  const int gs = min(__ldg(key_gsize + grp), 128);
+  for (int x = threadIdx.x; x < gs * 128; x += 256) {
+    const int j = x >> 7, e = x & 127;
+    const int tok = __ldg(key_perm + grp * 128 + j);
+    sk[j][e] = K[(static_cast<size_t>(head) * N + tok) * 128 + e];
+  }
+  __syncthreads();
+  if (b >= Gq) return;
+  float qv[128];
+  const float* qb = qbar + (static_cast<size_t>(head) * Gq + b) * 128;
+#pragma unroll
+  for (int e = 0; e < 128; ++e) qv[e] = qb[e] * tau;
+  float m = -__builtin_huge_valf(), s = 0.f;
+  for (int j = 0; j < gs; ++j) {
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < 128; ++e) acc = fmaf(qv[e], __bfloat162float(sk[j][e]), acc);
+    if (acc > m) {
+      s = s * expf(m - acc) + 1.f;
+      m = acc;
+    } else {
+      s += expf(acc - m);
+    }
+  }
+  sc[(static_cast<size_t>(head) * Gq + b) * G + g] = gs > 0 ? m + logf(s) : -__builtin_huge_valf();
+}
+
 __global__ void pairs_init_kernel(unsigned long long* pairs, int heads, long long probe_pairs) {
   const int h = blockIdx.x * blockDim.x + threadIdx.x;
   if (h < heads) pairs[h] = static_cast<unsigned long long>(probe_pairs);
@@ -121,6 +171,20 @@ cudaError_t launch_route(const float* sc, int heads, int Gq, int G, int k, int* 
   route_topk_kernel<<<dim3(ceil_div(Gq, 8), heads), 256, 0, st>>>(sc, Gq, G, k, route, key_gsize, qblock_size,
                                                                    up, status);
   return counted(cudaGetLastError(), up != nullptr ? 2 : 1);
+}
+
+cudaError_t launch_route_scores(int mode, float* sc, const void* K, int N, int heads, int Gq, int G,
+                                const int* key_perm, const int* key_gsize, const float* qbar, float tau,
+                                cudaStream_t st) {
+  if (mode == 1) {
+    size_correct_kernel<<<dim3(ceil_div(Gq * G, 256), heads), 256, 0, st>>>(sc, key_gsize, Gq, G);
+  } else if (mode == 2) {
+    lse_scores_kernel<<<dim3(G, heads, ceil_div(Gq, 256)), 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(K), N, Gq, G, key_perm, key_gsize, qbar, tau, sc);
+  } else {
+    return cudaSuccess;
+  }
+  return counted(cudaGetLastError(), 1);
 }
 
 }  // namespace spr

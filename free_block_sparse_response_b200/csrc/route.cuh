@@ -9,5 +9,10 @@ namespace spr {
 cudaError_t launch_route(const float* sc, int heads, int Gq, int G, int k, int* route, const int* key_gsize,
                          const int* qblock_size, long long* pairs, long long probe_pairs, int* status,
                          cudaStream_t st);
+// Replace (LSE, mode 2) or correct (size, mode 1) the centroid block scores sc [heads,
+// Gq, G]; qbar [heads, Gq, 128] are the query-block means, K bf16 with d = 128.
+cudaError_t launch_route_scores(int mode, float* sc, const void* K, int N, int heads, int Gq, int G,
+                                const int* key_perm, const int* key_gsize, const float* qbar, float tau,
+                                cudaStream_t st);
 
 }  // namespace spr

@@ -19,6 +19,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NONFINITE = ran
 BF16, F32 = 0, 1
 WEIGHT_INV_NORM, WEIGHT_UNIFORM = 0, 1
 PARTITION_RESPONSE, PARTITION_SEMANTIC = 0, 1
+ROUTE_CENTROID, ROUTE_SIZE_CORRECTED, ROUTE_LSE = 0, 1, 2
 _DTYPE_CODE = {torch.bfloat16: BF16, torch.float32: F32}
 
 EXPORTED_SYMBOLS = (
@@ -42,14 +43,15 @@ class _CParams(ctypes.Structure):
     _fields_ = [("block", ctypes.c_int32), ("n_sampled", ctypes.c_int32), ("n_probe", ctypes.c_int32),
                 ("kmeans_iters", ctypes.c_int32), ("rank", ctypes.c_int32), ("weight_mode", ctypes.c_int32),
                 ("density", ctypes.c_double), ("ridge_lambda", ctypes.c_double), ("scale", ctypes.c_float),
-                ("partition_mode", ctypes.c_int32)]
+                ("partition_mode", ctypes.c_int32), ("route_scores", ctypes.c_int32)]
 
 
 @dataclasses.dataclass(frozen=True)
 class SparsePRConfig:
     """Parameters of one call: block B, sampled queries S, probe rows P, k-means
     iterations T, subspace rank r, probe weighting, density rho, ridge lambda, scale,
-    and the partition rule (PARTITION_RESPONSE, or the PARTITION_SEMANTIC baseline)."""
+    the partition rule (PARTITION_RESPONSE, or the PARTITION_SEMANTIC baseline) and the
+    block-routing score (ROUTE_CENTROID, ROUTE_SIZE_CORRECTED or ROUTE_LSE)."""
     block: int = 128
     n_sampled: int = 512
     n_probe: int = 256
@@ -60,10 +62,12 @@ class SparsePRConfig:
     ridge_lambda: float = 1e-3
     scale: float = 0.0
     partition_mode: int = 0
+    route_scores: int = 0
 
     def c(self) -> _CParams:
         return _CParams(self.block, self.n_sampled, self.n_probe, self.kmeans_iters, self.rank,
-                        self.weight_mode, self.density, self.ridge_lambda, self.scale, self.partition_mode)
+                        self.weight_mode, self.density, self.ridge_lambda, self.scale, self.partition_mode,
+                        self.route_scores)
 
 
 _LIB = None

@@ -73,6 +73,14 @@ enum { SPARSEPR_WEIGHT_INV_NORM = 0, SPARSEPR_WEIGHT_UNIFORM = 1 };
  * pages do not state that rule. */
 enum { SPARSEPR_PARTITION_RESPONSE = 0, SPARSEPR_PARTITION_SEMANTIC = 1 };
 
+/* Block-routing score (one uniform k either way, so the executed-pair count is the
+ * same).  CENTROID: tau qbar_b . mu_g (the method's reading).  SIZE_CORRECTED:
+ * tau qbar_b . mu_g + log n_g (first-order log attention mass of the block's mean query
+ * on group g).  LSE: log sum_{j in g} exp(tau qbar_b . k_j) (that mass itself).  The
+ * pages say "up to a target density" without the score; these are the readings the
+ * comparison covers. */
+enum { SPARSEPR_ROUTE_CENTROID = 0, SPARSEPR_ROUTE_SIZE_CORRECTED = 1, SPARSEPR_ROUTE_LSE = 2 };
+
 typedef struct sparsepr_params {
   int32_t block;        /* B: query-block and key-group capacity (64 or 128)            */
   int32_t n_sampled;    /* S: sampled queries that define key response profiles        */
@@ -84,6 +92,7 @@ typedef struct sparsepr_params {
   double ridge_lambda;  /* lambda: ridge on the centred weighted Gram (sum w = P)       */
   float scale;          /* softmax scale tau; <= 0 selects 1/sqrt(d)                    */
   int32_t partition_mode; /* SPARSEPR_PARTITION_*                                        */
+  int32_t route_scores;   /* SPARSEPR_ROUTE_*: what block_scores hold                    */
 } sparsepr_params;
 
 /* Number of groups G = Gq = ceil(N / B): capacity-B groups that cover all N tokens. */

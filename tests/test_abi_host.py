@@ -72,10 +72,11 @@ def test_argument_errors_return_codes_without_launching(L):
 
 
 def test_params_struct_layout():
-    assert ctypes.sizeof(spr.sparsepr._CParams) == 48
+    assert ctypes.sizeof(spr.sparsepr._CParams) == 56
     assert spr.sparsepr._CParams.density.offset == 24
     assert spr.sparsepr._CParams.scale.offset == 40
     assert spr.sparsepr._CParams.partition_mode.offset == 44
+    assert spr.sparsepr._CParams.route_scores.offset == 48
 
 
 def test_python_wrappers_refuse_cpu_tensors():

@@ -325,6 +325,26 @@ def test_semantic_partition_call_parity():
         assert key_agree > 0.5 and query_agree > 0.5
 
 
+@pytest.mark.parametrize("mode,name", [(1, "size_corrected"), (2, "lse")])
+def test_routing_score_readings(mode, name):
+    """Size-corrected and LSE block scores against the oracle's on the GPU's own labels
+    (fp32 on the GPU, fp64 in the oracle), and the whole call on those routes."""
+    w = CONFIGS["small"]
+    cfg = spr_cfg(w, route_scores=mode)
+    q, k, v = make_inputs(w, 0, heads=2)
+    _, parts = _check_call(w, cfg, heads=2)
+    n = w.n_tokens
+    part = parts["partition"]
+    g = spr.num_groups(n, w.block)
+    for h in range(2):
+        kl = perm_labels(part.key_perm[0, h].cpu().numpy(), part.key_gsize[0, h].cpu().numpy(), n, w.block)
+        ql = perm_labels(part.query_perm[0, h].cpu().numpy(), part.qblock_size[0, h].cpu().numpy(), n, w.block)
+        ref = O.routing_scores(q[0, h].double().numpy(), k[0, h].double().numpy(), 1 / math.sqrt(w.head_dim), kl, ql,
+                               g, name)
+        got = part.block_scores[0, h].cpu().numpy()
+        assert np.max(np.abs(got - ref)) <= 1e-4 * max(1.0, float(np.max(np.abs(ref))))
+
+
 def test_nonfinite_input_is_reported():
     w = CONFIGS["tiny"].with_(dtype="bf16")
     q, k, v = make_inputs(w, 0)
