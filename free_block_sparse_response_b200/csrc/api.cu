@@ -170,6 +170,13 @@ int sparsepr_check(const void* ws, sparsepr_stream_t stream) {
   return SPARSEPR_OK;
 }
 
+int sparsepr_reset_workspace(void* ws, sparsepr_stream_t stream) {
+  if (!ws) return fail(SPARSEPR_ERR_INVALID_ARG, "null workspace");
+  SPR_CUDA(cudaMemsetAsync(ws, 0, sizeof(spr::WorkspaceHeader), reinterpret_cast<cudaStream_t>(stream)),
+           "reset workspace");
+  return SPARSEPR_OK;
+}
+
 int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int32_t H, int32_t N, int32_t d,
                        const sparsepr_params* p, const int32_t* sample_idx, int32_t* key_perm,
                        int32_t* key_gsize, int32_t* query_perm, int32_t* qblock_size, float* block_scores,
@@ -363,6 +370,7 @@ static int attention_common(const void* Q, const void* K, const void* V, int dty
     const Layout L = make_layout(Bt * H, N, d, block, 1, 0);
     a.k_grouped = at<char>(ws, L.kv_grouped);
     a.v_grouped = at<char>(ws, L.kv_grouped) + static_cast<size_t>(Bt) * H * G * block * d * 2;
+    a.kv_tag = header(ws)->kv_tag;
   }
   if (ws != nullptr) {
     a.status = &header(ws)->status;
@@ -422,6 +430,7 @@ int sparsepr_sparse_attn_apply(const void* Q, const void* K, const void* V, int 
   a.status = &header(ws)->status;
   a.k_grouped = at<char>(ws, L.kv_grouped);
   a.v_grouped = at<char>(ws, L.kv_grouped) + static_cast<size_t>(heads) * G * block * d * 2;
+  a.kv_tag = header(ws)->kv_tag;
   a.m_hilo = mh;
   a.beta = beta;
   a.out_bf16 = O;
@@ -472,6 +481,10 @@ int sparsepr_probe_dense(const void* Q, const void* K, const void* V, int dtype,
   a.probe_sparse = probe_sparse;
   a.qblk = at<int>(ws, L.qblk);
   a.partial = at<float>(ws, L.partial);
+  a.k_grouped = at<char>(ws, L.kv_grouped);
+  a.v_grouped = at<char>(ws, L.kv_grouped) + static_cast<size_t>(Bt) * H * G * block * d * 2;
+  a.kv_tag = header(ws)->kv_tag;
+  a.status = &header(ws)->status;
   SPR_CUDA(spr::launch_probe(a, reinterpret_cast<cudaStream_t>(stream)), "probe rows");
   return SPARSEPR_OK;
 }

@@ -7,6 +7,8 @@
 // Method: the SparsePR abstract (arXiv 2608.18484, arxivdaily.com English abstract)
 // computes attention only between selected groups and exact attention on a few probe
 // rows; the routed softmax is renormalised over the routed support.
+#include <algorithm>
+
 #include "attention.cuh"
 #include "common.cuh"
 #include "warp_mma.cuh"
@@ -639,6 +641,23 @@ size_t probe_partial_bytes(int heads, int P, int G, int d) {
   return static_cast<size_t>(heads) * P * nsplit * (4 + 2 * d) * sizeof(float);
 }
 
+// Splits of the key groups for the tensor-core probe kernel (one CTA per SM): at most
+// 64 groups a split, at most max_splits (the partial buffer's room), and the count that
+// minimises waves x groups per CTA over 148 SMs, with ~4 groups of fixed cost per CTA.
+static int probe_tc_splits(int G, int units, int max_splits) {
+  const int lo = ceil_div(G, 64);
+  int best = std::max(lo, 1), best_cost = -1;
+  for (int n = std::max(lo, 1); n <= std::max(max_splits, lo); ++n) {
+    const int waves = ceil_div(units * n, 148);
+    const int cost = waves * (ceil_div(G, n) + 4);
+    if (best_cost < 0 || cost < best_cost) {
+      best = n;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
 template <int D>
 static cudaError_t launch_probe_t(const ProbeArgs& a, cudaStream_t st) {
   qblock_of_token_kernel<<<dim3(ceil_div(a.G * a.block, 256), a.heads), 256, 0, st>>>(
@@ -652,6 +671,16 @@ static cudaError_t launch_probe_t(const ProbeArgs& a, cudaStream_t st) {
   }
   const int gps = probe_groups_per_split(a.G);
   const int nsplit = ceil_div(a.G, gps);
+  if (D == 128 && a.block == 128 && a.k_grouped != nullptr && a.v_grouped != nullptr && a.status != nullptr) {
+    // tensor-core path: K / V in group order, then one CTA per (128 probe rows, split, head)
+    cudaError_t e = launch_kv_group(a.K, a.V, a.N, a.G, a.heads, a.key_perm, a.key_gsize, a.k_grouped,
+                                    a.v_grouped, a.kv_tag, st);
+    if (e != cudaSuccess) return e;
+    const int ns = probe_tc_splits(a.G, a.heads * ceil_div(a.P, 128), nsplit);
+    if ((e = launch_probe_tc(a, ns, st)) != cudaSuccess) return e;
+    probe_combine_kernel<D><<<dim3(a.P, a.heads), D, 0, st>>>(a.partial, a.P, ns, a.probe_out, a.probe_sparse);
+    return counted(cudaGetLastError(), 2);
+  }
   const size_t smem = static_cast<size_t>(kProbeRows) * D * 2 + 4ull * kProbeChunk * D * 2;
   auto kern = probe_mma_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

@@ -25,7 +25,10 @@ struct WorkspaceHeader {
   int detail;
   unsigned int barrier_count;  // grid barrier of the cooperative fill kernel
   unsigned int barrier_gen;
-  int pad[60];
+  // Source of the group-ordered K / V copy in the workspace: K, V, key_perm, key_gsize
+  // pointers, N << 32 | G, heads (all zero: no copy).  Cleared with the header.
+  unsigned long long kv_tag[6];
+  int pad[48];
 };
 static_assert(sizeof(WorkspaceHeader) == 256, "header must keep 256-byte alignment");
 

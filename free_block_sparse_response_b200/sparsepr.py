@@ -29,7 +29,7 @@ EXPORTED_SYMBOLS = (
     "sparsepr_last_error", "sparsepr_test_fill_workspace_size", "sparsepr_test_fill",
     "sparsepr_test_topk", "sparsepr_row_errors", "sparsepr_launch_count", "sparsepr_fit_residual_noalloc",
     "sparsepr_kernel_timing", "sparsepr_kernel_timing_read", "sparsepr_test_fill_segmented",
-    "sparsepr_sparse_attn_apply",
+    "sparsepr_sparse_attn_apply", "sparsepr_reset_workspace",
 )
 
 
@@ -106,6 +106,7 @@ def lib() -> ctypes.CDLL:
         "sparsepr_apply_residual": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp,
                                                    ctypes.c_int, _vp]),
         "sparsepr_check": (ctypes.c_int, [_vp, _vp]),
+        "sparsepr_reset_workspace": (ctypes.c_int, [_vp, _vp]),
         "sparsepr_last_error": (ctypes.c_char_p, []),
         "sparsepr_test_fill_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32]),
         "sparsepr_test_fill": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
@@ -185,6 +186,11 @@ def new_workspace(batch: int, heads: int, n: int, d: int, cfg: SparsePRConfig, d
 def check(ws: torch.Tensor) -> None:
     """Wait for the current stream and raise if a device-side error was recorded."""
     _call("sparsepr_check", _p(ws), _stream(ws))
+
+
+def reset_workspace(ws: torch.Tensor) -> None:
+    """Clear the workspace header (status word and the record of the key-group K/V copy)."""
+    _call("sparsepr_reset_workspace", _p(ws), _stream(ws))
 
 
 # ----------------------------------------------------------------------------- stages

@@ -35,6 +35,13 @@
  *    device (a NaN reaching a decision, a bounded wait that ran out) are recorded in a
  *    status word inside `ws`; sparsepr_check() reads it.
  *  - Partition state never persists between calls: each call's map is call-specific.
+ *  - Key-group copy (bf16, d = 128, B = 128): sparsepr_probe_dense, sparsepr_sparse_attn
+ *    and sparsepr_sparse_attn_apply gather K and V into key-group order inside `ws`.
+ *    The header records the K, V, key_perm and key_gsize pointers and the shape the
+ *    copy was made from, and a later call with the same ones reuses it instead of
+ *    copying again (the probe-first pipeline copies once).  sparsepr_partition clears
+ *    the record.  A caller that rewrites K, V, key_perm or key_gsize in place between
+ *    such calls, with no partition call in between, calls sparsepr_reset_workspace.
  */
 #ifndef SPARSEPR_H
 #define SPARSEPR_H
@@ -265,6 +272,10 @@ SPARSEPR_API int sparsepr_kernel_timing_read(double* ms_total, int64_t* launches
  * first device-side error since the last sparsepr_partition).  Apart from the timing
  * hook's read, this is the only call that synchronises. */
 SPARSEPR_API int sparsepr_check(const void* ws, sparsepr_stream_t stream);
+
+/* Zero the workspace's 256-byte header on `stream`: clears the status word and the
+ * record of the key-group copy (so the next call copies K and V again). */
+SPARSEPR_API int sparsepr_reset_workspace(void* ws, sparsepr_stream_t stream);
 
 /* Message of the last host-side error on this thread ("" if none). */
 SPARSEPR_API const char* sparsepr_last_error(void);

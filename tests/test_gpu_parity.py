@@ -210,6 +210,31 @@ def test_fused_correction_matches_unfused_and_oracle(grid, heads):
     assert torch.equal(o_default.cpu(), o.cpu())
 
 
+def test_key_group_copy_reuse_and_reset():
+    """The group-ordered K/V copy made by one call is reused by the next call on the same
+    workspace and inputs (same result bit for bit); after K changes in place,
+    reset_workspace makes the next call copy again (equal to a fresh workspace)."""
+    w = CONFIGS["small"]
+    cfg = spr_cfg(w)
+    q, k, v = make_inputs(w, 3, heads=2)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    _, parts = spr.attention(qd, kd, vd, cfg, return_parts=True)
+    ws, part, rt, kk = parts["ws"], parts["partition"], parts["route"], parts["k"]
+    s_reused = spr.sparse_attn(qd, kd, vd, part, rt, kk, cfg, ws=ws)
+    assert torch.equal(s_reused, parts["S"])
+    fresh = spr.new_workspace(1, 2, w.n_tokens, 128, cfg, qd.device)
+    assert torch.equal(spr.sparse_attn(qd, kd, vd, part, rt, kk, cfg, ws=fresh), s_reused)
+    kd.mul_(-0.5)
+    vd.mul_(2.0)
+    spr.reset_workspace(ws)
+    s_new = spr.sparse_attn(qd, kd, vd, part, rt, kk, cfg, ws=ws)
+    fresh2 = spr.new_workspace(1, 2, w.n_tokens, 128, cfg, qd.device)
+    s_fresh = spr.sparse_attn(qd, kd, vd, part, rt, kk, cfg, ws=fresh2)
+    spr.check(ws)
+    assert torch.equal(s_new, s_fresh)
+    assert not torch.equal(s_new, s_reused)
+
+
 def test_full_density_equals_dense():
     """k = G: sparse output is dense attention; the fitted map is ~0."""
     w = CONFIGS["small"].with_(grid=(2, 16, 32), heads=2)
