@@ -65,11 +65,12 @@ Layout make_layout(int heads, int N, int d, int block, int S, int P) {
     return at;
   };
   // Regions read by the calls after partition come first, so that their offsets depend
-  // only on the shapes (and P) each of those calls knows.
+  // only on the shapes (and P) each of those calls knows.  The fit's scratch comes first
+  // of all, sized for the largest P it takes: the fit call knows neither N nor the block.
+  L.fit = take(sizeof(double) * H * spr::fit_scratch_doubles(spr::fit_max_probes(d), d));
   L.kv_grouped = take(2 * 2 * H * G * block * D);  // K and V in key-group order, bf16
   L.mhilo = take(2 * 2 * H * D * D);                // M as bf16 hi and lo (fused correction)
   L.partial = take(P > 0 ? spr::probe_partial_bytes(heads, P, static_cast<int>(G), d) : 0);
-  L.fit = take(P > 0 ? sizeof(double) * H * spr::fit_scratch_doubles(P, d) : 0);
   L.sample_idx = take(sizeof(int) * static_cast<size_t>(S));
   L.gamma = take(sizeof(float) * H * D * D);
   L.gamma_hi = take(2 * H * D * D);
@@ -501,8 +502,9 @@ int sparsepr_fit_residual(const float* probe_sparse, const float* probe_out, con
     return fail(SPARSEPR_ERR_INVALID_ARG, "unknown weight_mode %d", weight_mode);
   if (!probe_sparse || !probe_out || !M || !beta || !ws) return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
   if (spr::fit_smem_bytes(d, P) > 220 * 1024) return fail(SPARSEPR_ERR_UNSUPPORTED, "P=%d too large for the fit", P);
-  // The fit's scratch starts right after the header: no partition state is live any more
-  // and sparsepr_workspace_size() covers it.
+  // The fit's scratch is the workspace's first region after the header (sized for the
+  // largest P the fit takes, so its offset needs neither N nor the block); the key-group
+  // K/V copy behind it stays intact for the attention call that follows.
   const size_t off = align_up(sizeof(spr::WorkspaceHeader));
   double* scratch = at<double>(ws, off);
   SPR_CUDA(spr::launch_fit(probe_sparse, probe_out, weights, Bt * H, d, P, ridge_lambda, rank, weight_mode, scratch, M,

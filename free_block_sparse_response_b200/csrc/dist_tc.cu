@@ -38,6 +38,26 @@ enum : int {
   kXFull0 = 0, kXEmpty0 = 2, kWFull0 = 4, kWEmpty0 = 6, kAccFull0 = 8, kAccEmpty0 = 10, kDtDrain = 12, kDtBars = 13
 };
 
+// Packed pairs of fp32: one f32x2 instruction, each lane rounded exactly as the scalar op.
+__device__ __forceinline__ uint64_t dt_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void dt_f32x2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t dt_ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t dt_fadd2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 __device__ __forceinline__ unsigned long long dist_key(float v, int idx) {
   const uint32_t ok = (v != v) ? 0xffffffffu : float_order_key(v);
   return (static_cast<unsigned long long>(ok) << 32) | static_cast<uint32_t>(idx);
@@ -212,21 +232,40 @@ __global__ void __launch_bounds__(kDtThreads, 1)
         tc::mbar_arrive(bar(kAccEmpty0 + s));
         const int c0 = c * 128 + half * 64;
         const float4* e4 = reinterpret_cast<const float4*>(s_e + c0);
-        float seg_v = kDtInf;  // this 64-column segment's first minimum
-        int seg_c = -1;
+        // this 64-column segment's first minimum: four independent strict '<' scans over
+        // the columns j = t (mod 4), each in ascending order, then merged (smaller value
+        // wins, equal values -- +-0 included -- go to the lower column), which is the
+        // first minimum of the whole segment
+        float cv[4] = {kDtInf, kDtInf, kDtInf, kDtInf};
+        int cc[4] = {-1, -1, -1, -1};
+        const uint64_t m2 = dt_f32x2(m2t, m2t), tn2 = dt_f32x2(tnr, tnr);
 #pragma unroll
         for (int qq = 0; qq < 16; ++qq) {
           const float4 e = e4[qq];
-          const float ev[4] = {e.x, e.y, e.z, e.w};
+          float v[4];
+          dt_f32x2_split(dt_fadd2(dt_ffma2(dt_f32x2(__uint_as_float(u[4 * qq]), __uint_as_float(u[4 * qq + 1])), m2, tn2),
+                                  dt_f32x2(e.x, e.y)),
+                         v[0], v[1]);
+          dt_f32x2_split(dt_fadd2(dt_ffma2(dt_f32x2(__uint_as_float(u[4 * qq + 2]), __uint_as_float(u[4 * qq + 3])), m2,
+                                           tn2),
+                                  dt_f32x2(e.z, e.w)),
+                         v[2], v[3]);
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
-            const int j = 4 * qq + t;
-            const float v = fmaf(m2t, __uint_as_float(u[j]), tnr) + ev[t];
-            u[j] = __float_as_uint(v);
-            if (v < seg_v) {
-              seg_v = v;
-              seg_c = j;
+            u[4 * qq + t] = __float_as_uint(v[t]);
+            if (v[t] < cv[t]) {
+              cv[t] = v[t];
+              cc[t] = 4 * qq + t;
             }
+          }
+        }
+        float seg_v = cv[0];
+        int seg_c = cc[0];
+#pragma unroll
+        for (int t = 1; t < 4; ++t) {
+          if (cc[t] >= 0 && (seg_c < 0 || cv[t] < seg_v || (cv[t] == seg_v && cc[t] < seg_c))) {
+            seg_v = cv[t];
+            seg_c = cc[t];
           }
         }
         // segments in ascending column order: a strictly smaller minimum wins

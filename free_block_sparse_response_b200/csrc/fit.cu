@@ -558,6 +558,11 @@ size_t fit_smem_bytes(int d, int P) {
          static_cast<size_t>(d) * d * sizeof(float);
 }
 
+int fit_max_probes(int d) {
+  const size_t base = fit_smem_bytes(d, 0), cap = 220 * 1024;
+  return base >= cap ? 0 : static_cast<int>((cap - base) / sizeof(double));
+}
+
 template <int D, typename TO>
 static cudaError_t launch_apply_t(const float* S, const float* M, const float* beta, const int* probe_idx,
                                   const float* probe_out, int heads, int N, int P, TO* O, cudaStream_t st) {

@@ -9,6 +9,8 @@ namespace spr {
 
 __host__ __device__ size_t fit_scratch_doubles(int P, int d);
 size_t fit_smem_bytes(int d, int P);
+// Largest probe count the fit kernel takes at head dimension d (its shared memory).
+int fit_max_probes(int d);
 cudaError_t launch_fit(const float* xs, const float* dp, const float* weights, int heads, int d, int P,
                        double lambda, int rank, int weight_mode, double* scratch, float* M, float* beta,
                        int* status, cudaStream_t st);

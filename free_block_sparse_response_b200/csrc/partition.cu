@@ -549,95 +549,142 @@ __global__ void __launch_bounds__(kFillThreads, 3) fill_coop_kernel(FillArgs a) 
         closed_all = s_closed;
       }
       if (a.seg_min != nullptr) {
-        // Two items per warp, 16 lanes each; lane s of a half holds the minimum key of its
-        // row's 64-column segment s.  The best open group is the smallest key among the
-        // segment minima whose group is open, unless a segment whose minimum group is
-        // full still has a key below it: only such segments are read (64 values, four per
-        // lane), each read lowering the bound the remaining ones must beat.  Every key of
-        // a segment is >= its minimum key, so the result equals the argmin over the whole
-        // row's open groups.  The segment of the item's previous proposal (a group that
-        // has just filled, and the row's smallest key) is read in the same wave as the
-        // keys, since it nearly always has to be.
-        const int sub = lane & 15;
-        const unsigned int hmask = (lane & 16) ? 0xffff0000u : 0x0000ffffu;
-        for (int x0 = gwarp * 2; x0 < ncur; x0 += nwarps * 2) {
-          const int x = x0 + (lane >> 4);
+        // Four items per warp, 8 lanes each; lane s of a quarter holds the minimum keys of
+        // its row's 64-column segments s and s + 8.  The best open group is the smallest
+        // key among the segment minima whose group is open, unless a segment whose minimum
+        // group is full still has a key below it: only such segments are read (64 values,
+        // two 16-byte loads per lane), in ascending segment order, each read lowering the
+        // bound the remaining ones must beat.  Every key of a segment is >= its minimum
+        // key, so the result equals the argmin over the whole row's open groups.  The
+        // segment of the item's previous proposal (a group that has just filled, and the
+        // row's smallest key) is read in the same wave as the keys, since it nearly always
+        // has to be.  The next batch's item indices are fetched one batch ahead.
+        const int sub = lane & 7;
+        const int qb = lane & 24;  // first lane of this item's quarter
+        const unsigned long long inf_key = static_cast<unsigned long long>(float_order_key(__int_as_float(0x7f800000)))
+                                           << 32;
+        int x = gwarp * 4 + (lane >> 3);
+        int item_next = x < ncur ? __ldcg(L + x) : 0;
+        for (int x0 = gwarp * 4; x0 < ncur; x0 += nwarps * 4, x += nwarps * 4) {
           const bool valid = x < ncur;
-          const int item = valid ? __ldcg(L + x) : 0;
+          const int item = item_next;
+          item_next = x + nwarps * 4 < ncur ? __ldcg(L + x + nwarps * 4) : 0;
           const int h = item / n;
           const unsigned int* closed = closed_all + static_cast<size_t>(h) * words;
           const float* drow = a.D + static_cast<size_t>(item) * a.ldd;
           auto is_open = [&](int g) { return !((closed[g >> 5] >> (g & 31)) & 1u); };
-          const unsigned long long key =
-              valid && sub < a.nseg ? __ldcg(a.seg_min + static_cast<size_t>(item) * a.nseg + sub) : ~0ull;
+          unsigned long long* srow = a.seg_min + static_cast<size_t>(item) * a.nseg;
+          const unsigned long long key0 = valid && sub < a.nseg ? __ldcg(srow + sub) : ~0ull;
+          const unsigned long long key1 = valid && sub + 8 < a.nseg ? __ldcg(srow + sub + 8) : ~0ull;
           const int gp = (valid && round > 0) ? __ldcg(a.prop_g + item) : -1;
           const int sp = gp >= 0 ? (gp >> 7) * 2 + ((gp >> 6) & 1) : -1;
-          float pv[4];
           const int pcol0 = sp >= 0 ? (sp >> 1) * 128 + (sp & 1) * 64 : 0;
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const int g = pcol0 + 16 * t + sub;
-            pv[t] = (sp >= 0 && g < G) ? __ldcg(drow + g) : 0.f;
+          // lane sub's 8 columns of the 64-column segment at col0: col0 + 4 sub + {0..3} and
+          // col0 + 32 + 4 sub + {0..3} (two 16-byte loads when rows are 16-byte aligned)
+          auto load8 = [&](int col0, float4& va, float4& vb) {
+            va = make_float4(0.f, 0.f, 0.f, 0.f);
+            vb = va;
+            const int c0 = col0 + 4 * sub, c1 = col0 + 32 + 4 * sub;
+            if (a.d_vec4) {
+              if (c0 < G) va = __ldcg(reinterpret_cast<const float4*>(drow + c0));
+              if (c1 < G) vb = __ldcg(reinterpret_cast<const float4*>(drow + c1));
+            } else {
+              if (c0 < G) va.x = __ldcg(drow + c0);
+              if (c0 + 1 < G) va.y = __ldcg(drow + c0 + 1);
+              if (c0 + 2 < G) va.z = __ldcg(drow + c0 + 2);
+              if (c0 + 3 < G) va.w = __ldcg(drow + c0 + 3);
+              if (c1 < G) vb.x = __ldcg(drow + c1);
+              if (c1 + 1 < G) vb.y = __ldcg(drow + c1 + 1);
+              if (c1 + 2 < G) vb.z = __ldcg(drow + c1 + 2);
+              if (c1 + 3 < G) vb.w = __ldcg(drow + c1 + 3);
+            }
+          };
+          float4 pv0, pv1;
+          if (sp >= 0) {
+            load8(pcol0, pv0, pv1);
+          } else {
+            pv0 = make_float4(0.f, 0.f, 0.f, 0.f);
+            pv1 = pv0;
           }
-          const int kg = key != ~0ull ? static_cast<int>(key & 0xffffffffu) : -1;
-          const bool kopen = kg >= 0 && is_open(kg);
+          // per segment s in {sub, sub + 8}: is its minimum group open, and its lower bound
+          const int kg0 = key0 < kSegNoOpen ? static_cast<int>(key0 & 0xffffffffu) : -1;
+          const int kg1 = key1 < kSegNoOpen ? static_cast<int>(key1 & 0xffffffffu) : -1;
+          const bool kopen0 = kg0 >= 0 && is_open(kg0);
+          const bool kopen1 = kg1 >= 0 && is_open(kg1);
+          const int scol0 = (sub >> 1) * 128 + (sub & 1) * 64;
+          const int scol1 = ((sub + 8) >> 1) * 128 + ((sub + 8) & 1) * 64;
+          const bool has0 = valid && sub < a.nseg && scol0 < G && key0 != kSegNoOpen;
+          const bool has1 = valid && sub + 8 < a.nseg && scol1 < G && key1 != kSegNoOpen;
           // a segment without a value below +inf (key ~0) is bounded below by +inf at its
           // first column
-          const int scol0 = (sub >> 1) * 128 + (sub & 1) * 64;
-          const bool has_cols = valid && sub < a.nseg && scol0 < G;
-          const unsigned long long lb =
-              kg >= 0 ? key : (static_cast<unsigned long long>(float_order_key(__int_as_float(0x7f800000))) << 32) |
-                                  static_cast<uint32_t>(scol0);
-          unsigned long long best = kopen ? key : ~0ull;
+          const unsigned long long lb0 = kg0 >= 0 ? key0 : inf_key | static_cast<uint32_t>(scol0);
+          const unsigned long long lb1 = kg1 >= 0 ? key1 : inf_key | static_cast<uint32_t>(scol1);
+          unsigned long long best = kopen0 ? key0 : ~0ull;
+          if (kopen1 && key1 < best) best = key1;
           bool saw_nan = false;
-          if (sp >= 0) {
+          auto scan8 = [&](int col0, const float4& va, const float4& vb, unsigned long long& bb) {
+            const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              const int g = pcol0 + 16 * t + sub;
+            for (int t = 0; t < 8; ++t) {
+              const int g = col0 + (t >> 2) * 32 + 4 * sub + (t & 3);
               if (g < G && is_open(g)) {
-                saw_nan |= (pv[t] != pv[t]);
-                const unsigned long long kk = decision_key(pv[t], g);
-                best = kk < best ? kk : best;
+                saw_nan |= (vv[t] != vv[t]);
+                const unsigned long long kk = decision_key(vv[t], g);
+                bb = kk < bb ? kk : bb;
               }
             }
-          }
+          };
+          unsigned long long pbest = ~0ull;  // the previous proposal's segment, open groups
+          if (sp >= 0) scan8(pcol0, pv0, pv1, pbest);
 #pragma unroll
-          for (int o = 8; o > 0; o >>= 1) {
+          for (int o = 4; o > 0; o >>= 1) {
             const unsigned long long y = __shfl_xor_sync(0xffffffffu, best, o);
             best = y < best ? y : best;
+            const unsigned long long z = __shfl_xor_sync(0xffffffffu, pbest, o);
+            pbest = z < pbest ? z : pbest;
           }
-          unsigned int need = __ballot_sync(0xffffffffu, has_cols && !kopen && sub != sp && lb < best) & hmask;
-          while (__any_sync(0xffffffffu, need != 0u)) {
-            const int sg = need != 0u ? (__ffs(need) - 1) & 15 : -1;
-            unsigned long long bb = ~0ull;
-            if (sg >= 0) {
-              const int col0 = (sg >> 1) * 128 + (sg & 1) * 64;
-              float vv[4];
+          best = pbest < best ? pbest : best;
+          if (sp >= 0 && sub == 0) srow[sp] = pbest == ~0ull ? kSegNoOpen : pbest;
+          // Segments that may still hold a better open group are read two at a time, those
+          // with the smallest lower bounds first (a lower bound is a distinct key, so it
+          // names its segment); after each pair the bound the others must beat drops.
+          bool need0 = has0 && !kopen0 && sub != sp && lb0 < best;
+          bool need1 = has1 && !kopen1 && sub + 8 != sp && lb1 < best;
+          auto quarter_min = [&](unsigned long long v) {
 #pragma unroll
-              for (int t = 0; t < 4; ++t) {
-                const int g = col0 + 16 * t + sub;
-                vv[t] = g < G ? __ldcg(drow + g) : 0.f;
-              }
-#pragma unroll
-              for (int t = 0; t < 4; ++t) {
-                const int g = col0 + 16 * t + sub;
-                if (g < G && is_open(g)) {
-                  saw_nan |= (vv[t] != vv[t]);
-                  const unsigned long long kk = decision_key(vv[t], g);
-                  bb = kk < bb ? kk : bb;
-                }
-              }
+            for (int o = 4; o > 0; o >>= 1) {
+              const unsigned long long y = __shfl_xor_sync(0xffffffffu, v, o);
+              v = y < v ? y : v;
             }
-#pragma unroll
-            for (int o = 8; o > 0; o >>= 1) {
-              const unsigned long long y = __shfl_xor_sync(0xffffffffu, bb, o);
-              bb = y < bb ? y : bb;
+            return v;
+          };
+          auto seg_col = [&](unsigned long long lbk) {
+            const int c = static_cast<int>(lbk & 0xffffffffu);
+            return (c >> 6) << 6;  // first column of the segment holding column c
+          };
+          while (__any_sync(0xffffffffu, need0 || need1)) {
+            const unsigned long long c0 = need0 ? lb0 : ~0ull, c1 = need1 ? lb1 : ~0ull;
+            const unsigned long long A = quarter_min(c0 < c1 ? c0 : c1);
+            const unsigned long long d0 = c0 == A ? ~0ull : c0, d1 = c1 == A ? ~0ull : c1;
+            const unsigned long long B = quarter_min(d0 < d1 ? d0 : d1);
+            unsigned long long ba = ~0ull, bbk = ~0ull;
+            float4 va, vb, wa, wb;
+            if (A != ~0ull) load8(seg_col(A), va, vb);
+            if (B != ~0ull) load8(seg_col(B), wa, wb);
+            if (A != ~0ull) scan8(seg_col(A), va, vb, ba);
+            if (B != ~0ull) scan8(seg_col(B), wa, wb, bbk);
+            ba = quarter_min(ba);
+            bbk = quarter_min(bbk);
+            if (sub == 0) {  // keep the segment minima current (open groups only)
+              if (A != ~0ull) srow[seg_col(A) >> 6] = ba == ~0ull ? kSegNoOpen : ba;
+              if (B != ~0ull) srow[seg_col(B) >> 6] = bbk == ~0ull ? kSegNoOpen : bbk;
             }
+            const unsigned long long bb = ba < bbk ? ba : bbk;
             best = bb < best ? bb : best;
-            const unsigned int keep = __ballot_sync(0xffffffffu, has_cols && !kopen && sub != sp && lb < best) & hmask;
-            need = sg >= 0 ? (need & keep & ~(1u << (sg + (lane & 16)))) : 0u;
+            need0 = need0 && lb0 != A && lb0 != B && lb0 < best;
+            need1 = need1 && lb1 != A && lb1 != B && lb1 < best;
           }
-          saw_nan = (__ballot_sync(0xffffffffu, saw_nan) & hmask) != 0u && valid;
+          saw_nan = ((__ballot_sync(0xffffffffu, saw_nan) >> qb) & 0xffu) != 0u && valid;
           if (sub == 0 && valid) {
             if (saw_nan) record_error(&a.hdr->status, kErrNonFinite);
             if (best == ~0ull) {
@@ -997,6 +1044,7 @@ cudaError_t launch_fill(const FillArgs& a, cudaStream_t st) {
   FillArgs args = a;
   const size_t closed_bytes = sizeof(unsigned int) * static_cast<size_t>(a.heads) * words;
   args.stage_closed = closed_bytes <= kFillStageLimit ? 1 : 0;
+  args.d_vec4 = (a.ldd % 4 == 0 && (reinterpret_cast<uintptr_t>(a.D) & 15u) == 0) ? 1 : 0;
   const size_t smem = args.stage_closed ? closed_bytes : 0;
   if (smem > 48 * 1024) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

@@ -32,6 +32,9 @@ struct RowGemmArgs {
   int* status;
 };
 
+// Segment-minimum entry of a segment whose groups are all full.
+constexpr unsigned long long kSegNoOpen = ~0ull - 1;
+
 struct FillArgs {
   const float* D;       // [heads, n, ldd]
   int ldd;              // row stride of D (>= G)
@@ -39,8 +42,10 @@ struct FillArgs {
   const float* prop_v0;
   // optional segment minima of every D row (see RowGemmArgs::seg_min): later proposals
   // read those instead of the whole row, and only the segments that can still hold a
-  // better open group than the best open segment minimum
-  const unsigned long long* seg_min;
+  // better open group than the best open segment minimum.  The fill keeps them current:
+  // a segment it reads gets the minimum over its open groups written back (or
+  // kSegNoOpen when none is open), which stays a lower bound since groups only close.
+  unsigned long long* seg_min;
   int nseg;
   int heads, n, G, cap;
   int* labels;          // [heads, n]
@@ -57,6 +62,7 @@ struct FillArgs {
   float* prop_v;
   WorkspaceHeader* hdr;
   int stage_closed;     // set by the launcher: bitmaps fit in shared memory
+  int d_vec4;           // set by the launcher: D rows start on 16-byte boundaries
 };
 
 cudaError_t launch_midpoint_stride(int* idx, int n, int count, cudaStream_t st);

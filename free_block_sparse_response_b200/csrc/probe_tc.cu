@@ -213,10 +213,15 @@ __global__ void __launch_bounds__(kPtThreads, 1)
     const int qb = __ldg(qblock_of_token + static_cast<size_t>(head) * N + tok);
     uint64_t member_bits = 0;  // bit (g - g0): group g routed to this row's query block
     {
+      // the route row is sorted ascending: eight independent loads per step
       const int* rt = route + (static_cast<size_t>(head) * G + qb) * k;
-      for (int j = 0; j < k; ++j) {
-        const int g = __ldg(rt + j);
-        if (g >= g0 && g < g1) member_bits |= 1ull << (g - g0);
+      for (int j0 = 0; j0 < k; j0 += 8) {
+        int gg[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) gg[i] = j0 + i < k ? __ldg(rt + j0 + i) : -1;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (gg[i] >= g0 && gg[i] < g1) member_bits |= 1ull << (gg[i] - g0);
       }
     }
     const int* gsz = key_gsize + static_cast<size_t>(head) * G;
@@ -276,6 +281,20 @@ __global__ void __launch_bounds__(kPtThreads, 1)
       const float csp = live_s && !far ? pt_ex2(m_d - m_s) : 0.f;
       const bool any_member = __any_sync(0xffffffffu, member);
       const bool any_far = __any_sync(0xffffffffu, far);
+      const float md_safe = m_d == -kPtInf ? 0.f : m_d;
+      const float ms_safe = m_s == -kPtInf ? 0.f : m_s;
+      float sum_d = 0.f, sum_s = 0.f;
+      if (!any_far) {
+        // dense weights in place, while the previous tile's PV products still run
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const float p0 = pt_ex2(fmaf(__uint_as_float(u[c]), scale_log2, -md_safe));
+          const float p1 = pt_ex2(fmaf(__uint_as_float(u[c + 1]), scale_log2, -md_safe));
+          u[c] = __float_as_uint(p0);
+          u[c + 1] = __float_as_uint(p1);
+          sum_d += p0 + p1;
+        }
+      }
       // P_d (TMEM), P_s (shared) and O_d / O_s are free once the previous PV is done
       if (t >= 1 && !pt_warp_wait(bar(kPPVDone), (t - 1) & 1, abort_v, status)) {
         ok = false;
@@ -299,11 +318,8 @@ __global__ void __launch_bounds__(kPtThreads, 1)
           }
         }
       }
-      const float md_safe = m_d == -kPtInf ? 0.f : m_d;
-      const float ms_safe = m_s == -kPtInf ? 0.f : m_s;
       const float mem_f = live_s ? 1.f : 0.f;
       const bool write_s = any_member || !zeroed;
-      float sum_d = 0.f, sum_s = 0.f;
       // quarters of 32 keys: 16 packed columns of P_d (hi, lo) and 4 16-byte chunks of P_s
 #pragma unroll
       for (int qt = 0; qt < 4; ++qt) {
@@ -324,15 +340,18 @@ __global__ void __launch_bounds__(kPtThreads, 1)
             pt_st_shared_v4(sPl + off, lo[4 * c4], lo[4 * c4 + 1], lo[4 * c4 + 2], lo[4 * c4 + 3]);
           }
         }
-        // dense weights, kept in u for the sparse pass
+        // dense weights (computed above unless a row of the warp is far), kept in u
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int c = qt * 32 + 2 * i;
-          const float p0 = pt_ex2(fmaf(__uint_as_float(u[c]), scale_log2, -md_safe));
-          const float p1 = pt_ex2(fmaf(__uint_as_float(u[c + 1]), scale_log2, -md_safe));
-          u[c] = __float_as_uint(p0);
-          u[c + 1] = __float_as_uint(p1);
-          sum_d += p0 + p1;
+          float p0 = __uint_as_float(u[c]), p1 = __uint_as_float(u[c + 1]);
+          if (any_far) {
+            p0 = pt_ex2(fmaf(p0, scale_log2, -md_safe));
+            p1 = pt_ex2(fmaf(p1, scale_log2, -md_safe));
+            u[c] = __float_as_uint(p0);
+            u[c + 1] = __float_as_uint(p1);
+            sum_d += p0 + p1;
+          }
           split_bf16x2(p0, p1, hi[i], lo[i]);
         }
         tc::tmem_st16(tPh + 16 * qt, hi);
