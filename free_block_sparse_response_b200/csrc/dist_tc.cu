@@ -19,6 +19,9 @@
 // each of 4 rows.  The row argmin is a strict '<' scan in
 // ascending column order (first minimum wins, +-0 compare equal), merged across the two
 // halves at the end.  Every wait is bounded.
+#include <cuda.h>
+
+#include "attention.cuh"
 #include "common.cuh"
 #include "partition.cuh"
 #include "tcgen05.cuh"
@@ -28,7 +31,6 @@ namespace spr {
 namespace {
 
 constexpr int kDtThreads = 384;
-constexpr int kDtProducers = 64;
 constexpr uint32_t kDtTile = 128 * 128 * 2;
 constexpr uint32_t kDtTmemCols = 256;
 constexpr float kDtInf = __builtin_huge_valf();
@@ -65,8 +67,8 @@ __device__ __forceinline__ unsigned long long dist_key(float v, int idx) {
 
 template <bool SPLIT>
 __global__ void __launch_bounds__(kDtThreads, 1)
-    dist_tc_kernel(const __nv_bfloat16* __restrict__ X, int n, const __nv_bfloat16* __restrict__ Whi,
-                   const __nv_bfloat16* __restrict__ Wlo, int ncols, int ldd, const float* __restrict__ nrm,
+    dist_tc_kernel(const __grid_constant__ CUtensorMap tmX, int n, const __grid_constant__ CUtensorMap tmWhi,
+                   const __grid_constant__ CUtensorMap tmWlo, int ncols, int ldd, const float* __restrict__ nrm,
                    const float* __restrict__ ecol, float tau2, float* __restrict__ Dout, int* __restrict__ prop_g,
                    float* __restrict__ prop_v, unsigned long long* __restrict__ seg_min, int nseg,
                    int* __restrict__ status, int heads) {
@@ -93,10 +95,10 @@ __global__ void __launch_bounds__(kDtThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
       if (s == 0) {
-        tc::mbar_init(bar(kXFull0), kDtProducers);
+        tc::mbar_init(bar(kXFull0), 1);
         tc::mbar_init(bar(kXEmpty0), 1);
       }
-      tc::mbar_init(bar(kWFull0 + s), kDtProducers);
+      tc::mbar_init(bar(kWFull0 + s), 1);
       tc::mbar_init(bar(kWEmpty0 + s), 1);
       tc::mbar_init(bar(kAccFull0 + s), 1);
       tc::mbar_init(bar(kAccEmpty0 + s), 256);
@@ -115,42 +117,51 @@ __global__ void __launch_bounds__(kDtThreads, 1)
   const uint32_t tbase = tmem_slot;
   volatile int* abort_v = &abort_flag;
 
-  if (warp < 2) {
-    // ------------------------------------------------------------------ producers
-    const int pt = tid, ch = pt & 15, r0 = pt >> 4;
-    bool ok = true;
-    for (int w = blockIdx.x, it = 0; ok && w < total; w += gridDim.x, ++it) {
-      const int head = w / tiles, row0 = (w - head * tiles) * 128;
-      if (it >= 1 && !tc::mbar_wait(bar(kXEmpty0), (it - 1) & 1, abort_v, status)) break;
-      const __nv_bfloat16* xh = X + static_cast<size_t>(head) * n * 128;
-#pragma unroll 4
-      for (int i = 0; i < 32; ++i) {
-        const int r = r0 + 4 * i;
-        const int row = row0 + r;
-        cp_async_16(sX + tc::sw128_offset(r, ch), row < n ? xh + static_cast<size_t>(row) * 128 + ch * 8 : xh,
-                    row < n ? 16 : 0);
-      }
-      tc::cp_async_arrive_noinc(bar(kXFull0));
-      const __nv_bfloat16* wh = Whi + static_cast<size_t>(head) * ncols * 128;
-      const __nv_bfloat16* wl = SPLIT ? Wlo + static_cast<size_t>(head) * ncols * 128 : nullptr;
-      for (int c = 0; c < n_chunks; ++c) {
-        const int q = it * n_chunks + c, s = q & 1;
-        if (q >= 2 && !tc::mbar_wait(bar(kWEmpty0 + s), ((q >> 1) - 1) & 1, abort_v, status)) {
-          ok = false;
-          break;
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    // One lane: the item tile of X (two TMA boxes of 64 columns x 128 rows), then per
+    // chunk the 128 rows of W (hi, and lo when split).  Rows past a head's n items or
+    // ncols groups come from the next head (or are zero past the tensor): they only feed
+    // rows that are never stored and columns whose e term is +inf.
+    if (lane == 0) {
+      bool ok = true;
+      int last_it = -1, last_q = -1;
+      for (int w = blockIdx.x, it = 0; ok && w < total; w += gridDim.x, ++it) {
+        const int head = w / tiles, row0 = (w - head * tiles) * 128;
+        if (it >= 1 && !tc::mbar_wait(bar(kXEmpty0), (it - 1) & 1, abort_v, status)) break;
+        tc::mbar_arrive_expect_tx(bar(kXFull0), kDtTile);
+        tc::tma_load_2d(sX, &tmX, 0, head * n + row0, bar(kXFull0));
+        tc::tma_load_2d(sX + 128 * 128, &tmX, 64, head * n + row0, bar(kXFull0));
+        last_it = it;
+        for (int c = 0; c < n_chunks; ++c) {
+          const int q = it * n_chunks + c, s = q & 1;
+          if (q >= 2 && !tc::mbar_wait(bar(kWEmpty0 + s), ((q >> 1) - 1) & 1, abort_v, status)) {
+            ok = false;
+            break;
+          }
+          const int wrow = head * ncols + c * 128;
+          tc::mbar_arrive_expect_tx(bar(kWFull0 + s), kWStage);
+          tc::tma_load_2d(sW[s], &tmWhi, 0, wrow, bar(kWFull0 + s));
+          tc::tma_load_2d(sW[s] + 128 * 128, &tmWhi, 64, wrow, bar(kWFull0 + s));
+          if (SPLIT) {
+            tc::tma_load_2d(sW[s] + kDtTile, &tmWlo, 0, wrow, bar(kWFull0 + s));
+            tc::tma_load_2d(sW[s] + kDtTile + 128 * 128, &tmWlo, 64, wrow, bar(kWFull0 + s));
+          }
+          last_q = q;
         }
-#pragma unroll 4
-        for (int i = 0; i < 32; ++i) {
-          const int r = r0 + 4 * i;
-          const int col = c * 128 + r;
-          const size_t off = col < ncols ? static_cast<size_t>(col) * 128 + ch * 8 : 0;
-          cp_async_16(sW[s] + tc::sw128_offset(r, ch), wh + off, col < ncols ? 16 : 0);
-          if (SPLIT) cp_async_16(sW[s] + kDtTile + tc::sw128_offset(r, ch), wl + off, col < ncols ? 16 : 0);
-        }
-        tc::cp_async_arrive_noinc(bar(kWFull0 + s));
       }
+      // copies still in flight after an abort land before the CTA exits (bounded waits)
+      auto drain = [&](uint32_t b, uint32_t parity) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!tc::mbar_try_wait(b, parity)) {
+          if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+        }
+      };
+      for (int q = last_q - 1; q <= last_q; ++q)
+        if (q >= 0) drain(bar(kWFull0 + (q & 1)), (q >> 1) & 1);
+      if (last_it >= 0) drain(bar(kXFull0), last_it & 1);
     }
-    cp_async_wait<0>();
+    __syncwarp();
   } else if (warp == 2) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -359,8 +370,14 @@ cudaError_t launch_dist_tc(const RowGemmArgs& a, int ldd, cudaStream_t st) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int total = a.heads * ceil_div(a.n, 128);
+  const long long xrows = static_cast<long long>(a.heads) * a.n, wrows = static_cast<long long>(a.heads) * a.ncols;
+  if (xrows > 0x7fffffffLL || wrows > 0x7fffffffLL) return cudaErrorInvalidValue;  // TMA coordinates are int32
+  CUtensorMap tx, twh, twl;
+  if (!bf16_map(&tx, a.X, xrows, 128) || !bf16_map(&twh, a.Bhi, wrows, 128) ||
+      !bf16_map(&twl, split ? static_cast<const void*>(a.Blo) : static_cast<const void*>(a.Bhi), wrows, 128))
+    return cudaErrorInvalidValue;
   kern<<<std::min(total, sms), kDtThreads, smem, st>>>(
-      static_cast<const __nv_bfloat16*>(a.X), a.n, a.Bhi, a.Blo, a.ncols, ldd, a.nrm, a.ecol, a.tau2, a.Dout,
+      tx, a.n, twh, twl, a.ncols, ldd, a.nrm, a.ecol, a.tau2, a.Dout,
       a.prop_g, a.prop_v, a.seg_min, a.nseg, a.status, a.heads);
   return counted(cudaGetLastError(), 1);
 }

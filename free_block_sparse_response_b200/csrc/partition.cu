@@ -530,13 +530,41 @@ __global__ void __launch_bounds__(kFillThreads, 3) fill_coop_kernel(FillArgs a) 
     const int ncur = __ldcg(a.list_len + cur);
     const int* L = lists[cur];
     // ---- propose
-    if (round == 0 && a.prop_g0 != nullptr) {
+    if (round == 0 && (a.prop_g0 != nullptr || a.seg_min != nullptr)) {
+      // first proposals: the row argmins, given, or the smallest segment key of the row
+      // (its first minimum among values below +inf; group 0 at +inf when it has none)
       for (int x = gthread; x < ncur; x += nthreads) {
         const int item = __ldcg(L + x);
         const int h = item / n;
-        const int g = a.prop_g0[item];
+        int g;
+        float v;
+        if (a.prop_g0 != nullptr) {
+          g = a.prop_g0[item];
+          v = a.prop_v0[item];
+        } else {
+          const ulonglong2* sk = reinterpret_cast<const ulonglong2*>(a.seg_min + static_cast<size_t>(item) * a.nseg);
+          unsigned long long key = ~0ull;
+          for (int t = 0; t < a.nseg / 2; ++t) {
+            const ulonglong2 kk = __ldcg(sk + t);
+            key = kk.x < key ? kk.x : key;
+            key = kk.y < key ? kk.y : key;
+          }
+          if (key == ~0ull) {  // no value below +inf: the whole row decides (+inf, then NaN)
+            const float* drow = a.D + static_cast<size_t>(item) * a.ldd;
+            bool saw_nan = false;
+            for (int c = 0; c < G; ++c) {
+              const float dv = __ldcg(drow + c);
+              saw_nan |= dv != dv;
+              const unsigned long long kk = decision_key(dv, c);
+              key = kk < key ? kk : key;
+            }
+            if (saw_nan) record_error(&a.hdr->status, kErrNonFinite);
+          }
+          g = static_cast<int>(key & 0xffffffffu);
+          v = float_from_order_key(static_cast<uint32_t>(key >> 32));
+        }
         a.prop_g[item] = g;
-        a.prop_v[item] = a.prop_v0[item];
+        a.prop_v[item] = v;
         atomicAdd(a.cnt + static_cast<size_t>(h) * G + g, 1);
       }
     } else {

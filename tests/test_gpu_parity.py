@@ -381,17 +381,16 @@ def test_nonfinite_input_is_reported():
 
 # ----------------------------------------------------- full size, sampled outputs (bench)
 
-def test_video_config_sampled_rows():
-    """75,600 tokens x 40 heads in the bench's launch configuration.  All heads: valid
-    partitions and exact pair counts; heads 0 and 39: sampled rows of the sparse
-    output, every probe row, and the final output on sampled rows against the oracle."""
-    w = CONFIGS["video"]
+def _full_size_sampled_rows(w, k_expected, check_heads):
+    """All heads: valid partitions and exact pair counts; the heads in check_heads:
+    sampled rows of the sparse output, every probe row, the fit and the final output on
+    sampled rows against the oracle."""
     cfg = spr_cfg(w)
     q, k, v = make_inputs(w, 0)
     o, parts = run_call(w, q, k, v, cfg)
     n, B = w.n_tokens, w.block
     kk = parts["k"]
-    assert kk == 127
+    assert kk == k_expected
     part = parts["partition"]
     pairs = parts["executed_pairs"].cpu().numpy()
     ks_all, bs_all = part.key_gsize.cpu().numpy(), part.qblock_size.cpu().numpy()
@@ -402,7 +401,7 @@ def test_video_config_sampled_rows():
         assert pairs[0, h] / n ** 2 <= w.density
     rng = np.random.default_rng(7)
     tau = 1 / math.sqrt(w.head_dim)
-    for h in (0, w.heads - 1):
+    for h in check_heads:
         qh, kh, vh = (t[0, h].double().numpy() for t in (q, k, v))
         kl = perm_labels(part.key_perm[0, h].cpu().numpy(), ks_all[0, h], n, B)
         ql = perm_labels(part.query_perm[0, h].cpu().numpy(), bs_all[0, h], n, B)
@@ -424,3 +423,16 @@ def test_video_config_sampled_rows():
         o_ref = s_ref + s_ref @ fit["M"].T + fit["beta"]
         o_gpu = o[0, h][torch.from_numpy(rows).cuda()].double().cpu().numpy()
         assert rel(o_gpu, o_ref) <= TOL_BF16
+
+
+def test_video_config_sampled_rows():
+    """75,600 tokens x 40 heads (G = 591, k = 127) in the bench's launch configuration."""
+    w = CONFIGS["video"]
+    _full_size_sampled_rows(w, 127, (0, w.heads - 1))
+
+
+def test_long_config_sampled_rows():
+    """118,800 tokens x 24 heads (G = 929, k = 202: the widest fill bitmap and 16
+    distance segments per row)."""
+    w = CONFIGS["long"]
+    _full_size_sampled_rows(w, 202, (0, w.heads - 1))
