@@ -4,10 +4,13 @@
 #include <cstdio>
 #include <atomic>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 #include <string>
 
 #include "../../include/sparsepr.h"
+
+#include <initializer_list>
 #include "attention.cuh"
 #include "common.cuh"
 #include "fit.cuh"
@@ -125,6 +128,14 @@ int check_block(int32_t block) {
   return SPARSEPR_OK;
 }
 
+// Q, K, V are read with 16-byte vector and TMA loads.
+int check_aligned(std::initializer_list<const void*> ptrs) {
+  for (const void* q : ptrs)
+    if ((reinterpret_cast<uintptr_t>(q) & 15u) != 0)
+      return fail(SPARSEPR_ERR_INVALID_ARG, "Q, K and V must start on 16-byte boundaries");
+  return SPARSEPR_OK;
+}
+
 int check_dtype(int dtype) {
   if (dtype != SPARSEPR_BF16 && dtype != SPARSEPR_F32) return fail(SPARSEPR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
   return SPARSEPR_OK;
@@ -188,6 +199,7 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
   if ((rc = check_block(p->block))) return rc;
   if (!Q || !K || !key_perm || !key_gsize || !query_perm || !qblock_size || !block_scores || !ws)
     return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
+  if ((rc = check_aligned({Q, K}))) return rc;
   if (p->n_sampled < 1 || p->n_sampled > N) return fail(SPARSEPR_ERR_INVALID_ARG, "n_sampled must be in [1, N]");
   if (p->kmeans_iters < 0 || p->kmeans_iters > 64) return fail(SPARSEPR_ERR_INVALID_ARG, "kmeans_iters must be in [0, 64]");
   if (spr::ceil_div(N, p->block) > 1024)
@@ -342,6 +354,7 @@ static int attention_common(const void* Q, const void* K, const void* V, int dty
   int rc;
   if ((rc = check_shape(Bt, H, N, d)) || (rc = check_dtype(dtype)) || (rc = check_block(block))) return rc;
   if (!Q || !K || !V || !out) return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
+  if ((rc = check_aligned({Q, K, V}))) return rc;
   const int G = spr::ceil_div(N, block);
   if (!dense) {
     if (!key_perm || !key_gsize || !query_perm || !qblock_size || !route)
@@ -401,6 +414,7 @@ int sparsepr_sparse_attn_apply(const void* Q, const void* K, const void* V, int 
     return fail(SPARSEPR_ERR_UNSUPPORTED, "the fused correction is built for bf16, d = 128, block = 128");
   if (!Q || !K || !V || !key_perm || !key_gsize || !query_perm || !qblock_size || !route || !M || !beta || !O || !ws)
     return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
+  if ((rc = check_aligned({Q, K, V}))) return rc;
   if (P < 0 || P > N || (P > 0 && (!probe_idx || !probe_out))) return fail(SPARSEPR_ERR_INVALID_ARG, "bad probe rows");
   const int G = spr::ceil_div(N, block);
   if (k < 1 || k > G) return fail(SPARSEPR_ERR_INVALID_ARG, "k=%d outside [1, %d]", k, G);
@@ -457,6 +471,7 @@ int sparsepr_probe_dense(const void* Q, const void* K, const void* V, int dtype,
   if (!Q || !K || !V || !probe_idx || !key_perm || !key_gsize || !query_perm || !route || !probe_out ||
       !probe_sparse || !ws)
     return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
+  if ((rc = check_aligned({Q, K, V}))) return rc;
   const int G = spr::ceil_div(N, block);
   if (k < 1 || k > G) return fail(SPARSEPR_ERR_INVALID_ARG, "k=%d outside [1, %d]", k, G);
   const Layout L = make_layout(Bt * H, N, d, block, 1, P);

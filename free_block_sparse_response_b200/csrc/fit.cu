@@ -111,34 +111,55 @@ __global__ void __launch_bounds__(kFitThreads)
   for (int p = tid; p < P; p += kFitThreads) w[p] *= static_cast<double>(P) / wsum;
   __syncthreads();
 
-  // ---- C = sum_p w_p y_p y_p^T
+  // ---- C = sum_p w_p y_p y_p^T.  Thread (bi, bj) accumulates rows bi + kNrb k' x columns
+  // bj + kNcb k (a kRb x kCb block, columns interleaved so that a warp's reads of a staged
+  // row hit consecutive words); the rows are staged 16 at a time as y_p and w_p y_p.
   constexpr int kPer = D * D / kFitThreads;
-  double acc[kPer];
+  constexpr int kNcb = 16, kCb = D / kNcb, kNrb = kFitThreads / kNcb, kRb = D / kNrb;
+  static_assert(kRb * kCb == kPer, "block shape");
+  const int bj = tid % kNcb, bi = tid / kNcb;
+  double acc[kRb][kCb];
+  auto acc_zero = [&]() {
 #pragma unroll
-  for (int x = 0; x < kPer; ++x) acc[x] = 0.0;
-  for (int p0 = 0; p0 < P; p0 += kStageRows) {
-    __syncthreads();
-    for (int x = tid; x < kStageRows * D; x += kFitThreads) {
-      const int p = p0 + x / D, e = x % D;
-      stage[x] = p < P ? (static_cast<double>(dp[static_cast<size_t>(p) * D + e]) -
-                          static_cast<double>(xs[static_cast<size_t>(p) * D + e])) : 0.0;
+    for (int k1 = 0; k1 < kRb; ++k1)
+#pragma unroll
+      for (int k2 = 0; k2 < kCb; ++k2) acc[k1][k2] = 0.0;
+  };
+  // acc += (w_r y_r)[rows] (y_r)[cols] for the staged rows r
+  auto acc_rows = [&](const double* wys, const double* ys, int nr) {
+    for (int r = 0; r < nr; ++r) {
+      double yi[kRb], yj[kCb];
+#pragma unroll
+      for (int k1 = 0; k1 < kRb; ++k1) yi[k1] = wys[r * D + bi + kNrb * k1];
+#pragma unroll
+      for (int k2 = 0; k2 < kCb; ++k2) yj[k2] = ys[r * D + bj + kNcb * k2];
+#pragma unroll
+      for (int k1 = 0; k1 < kRb; ++k1)
+#pragma unroll
+        for (int k2 = 0; k2 < kCb; ++k2) acc[k1][k2] = fma(yi[k1], yj[k2], acc[k1][k2]);
     }
-    __syncthreads();
-    for (int r = 0; r < kStageRows && p0 + r < P; ++r) {
-      const double wr = w[p0 + r];
-      const double* y = stage + r * D;
-#pragma unroll
-      for (int x = 0; x < kPer; ++x) {
-        const int ij = tid + x * kFitThreads;
-        acc[x] += wr * y[ij / D] * y[ij % D];
+  };
+  acc_zero();
+  {
+    double* wst = C;  // staged w_p y_p (C is written after the loop)
+    for (int p0 = 0; p0 < P; p0 += kStageRows) {
+      __syncthreads();
+      for (int x = tid; x < kStageRows * D; x += kFitThreads) {
+        const int p = p0 + x / D, e = x % D;
+        const double yv = p < P ? (static_cast<double>(dp[static_cast<size_t>(p) * D + e]) -
+                                   static_cast<double>(xs[static_cast<size_t>(p) * D + e])) : 0.0;
+        stage[x] = yv;
+        wst[x] = p < P ? w[p] * yv : 0.0;
       }
+      __syncthreads();
+      acc_rows(wst, stage, min(kStageRows, P - p0));
     }
   }
+  __syncthreads();
 #pragma unroll
-  for (int x = 0; x < kPer; ++x) {
-    const int ij = tid + x * kFitThreads;
-    C[(ij / D) * LD + ij % D] = acc[x];
-  }
+  for (int k1 = 0; k1 < kRb; ++k1)
+#pragma unroll
+    for (int k2 = 0; k2 < kCb; ++k2) C[(bi + kNrb * k1) * LD + bj + kNcb * k2] = acc[k1][k2];
   __syncthreads();
 
   // ---- eigenvectors of the R largest eigenvalues
@@ -290,124 +311,235 @@ __global__ void __launch_bounds__(kFitThreads)
   // row a of U_r: the a-th largest eigenvalue's eigenvector (fp32)
   auto urow = [&](int a) -> const float* { return tri ? Vt + a * D : Vt + static_cast<size_t>(order[a]) * D; };
 
-  // ---- z_p = U_r^T y_p ; weighted means
-  for (int x = tid; x < P * R; x += kFitThreads) {
-    const int p = x / R, a = x % R;
-    const float* u = urow(a);
-    double s = 0.0;
-    for (int e = 0; e < D; ++e)
-      s += u[e] * (static_cast<double>(dp[static_cast<size_t>(p) * D + e]) -
-                   static_cast<double>(xs[static_cast<size_t>(p) * D + e]));
-    Z[x] = s;
-  }
-  __syncthreads();
-  for (int e = tid; e < D; e += kFitThreads) {
-    double s = 0.0;
-    for (int p = 0; p < P; ++p) s += w[p] * xs[static_cast<size_t>(p) * D + e];
-    xbar[e] = s / static_cast<double>(P);
-  }
-  for (int a = tid; a < R; a += kFitThreads) {
-    double s = 0.0;
-    for (int p = 0; p < P; ++p) s += w[p] * Z[p * R + a];
-    zbar[a] = s / static_cast<double>(P);
-  }
-  __syncthreads();
-
-  // ---- Gram = X_c^T W X_c + lambda I  (into C)
-#pragma unroll
-  for (int x = 0; x < kPer; ++x) acc[x] = 0.0;
+  // ---- pass A over the probes, 16 rows at a time: z_p = U_r^T y_p (to scratch) and the
+  // per-thread parts of sum_p w_p x_p (thread tid always holds dim tid % D)
+  double xpart = 0.0;
   for (int p0 = 0; p0 < P; p0 += kStageRows) {
     __syncthreads();
     for (int x = tid; x < kStageRows * D; x += kFitThreads) {
       const int p = p0 + x / D, e = x % D;
-      stage[x] = p < P ? static_cast<double>(xs[static_cast<size_t>(p) * D + e]) - xbar[e] : 0.0;
+      double yv = 0.0;
+      if (p < P) {
+        const double xv = xs[static_cast<size_t>(p) * D + e];
+        yv = static_cast<double>(dp[static_cast<size_t>(p) * D + e]) - xv;
+        xpart += w[p] * xv;
+      }
+      stage[x] = yv;
     }
     __syncthreads();
-    for (int r = 0; r < kStageRows && p0 + r < P; ++r) {
-      const double wr = w[p0 + r];
-      const double* xc = stage + r * D;
-#pragma unroll
-      for (int x = 0; x < kPer; ++x) {
-        const int ij = tid + x * kFitThreads;
-        acc[x] += wr * xc[ij / D] * xc[ij % D];
+    // output (r, a): lanes of a warp take consecutive a, and walk the dims from (e + a) % D,
+    // so that the 32 eigenvector rows they read sit in 32 different banks
+    for (int x = tid; x < kStageRows * R; x += kFitThreads) {
+      const int r = x / R, a = x % R;
+      if (p0 + r >= P) continue;
+      const float* u = urow(a);
+      const double* y = stage + r * D;
+      double acc0 = 0.0, acc1 = 0.0;
+      for (int e0 = 0; e0 < D; e0 += 2) {
+        const int e = (e0 + a) & (D - 1), f = (e0 + 1 + a) & (D - 1);
+        acc0 = fma(static_cast<double>(u[e]), y[e], acc0);
+        acc1 = fma(static_cast<double>(u[f]), y[f], acc1);
       }
+      Z[static_cast<size_t>(p0 + r) * R + a] = acc0 + acc1;
     }
   }
   __syncthreads();
-#pragma unroll
-  for (int x = 0; x < kPer; ++x) {
-    const int ij = tid + x * kFitThreads;
-    C[(ij / D) * LD + ij % D] = acc[x] + ((ij / D == ij % D) ? lambda : 0.0);
+  {
+    double* part = C;  // free until the Gram is written
+    part[tid] = xpart;
+    __syncthreads();
+    for (int e = tid; e < D; e += kFitThreads) {
+      double sx = 0.0;
+      for (int t = e; t < kFitThreads; t += D) sx += part[t];
+      xbar[e] = sx / static_cast<double>(P);
+    }
+    __syncthreads();
+    // zbar: 16 interleaved partial sums per a, then their total
+    for (int x = tid; x < 16 * R; x += kFitThreads) {
+      const int a = x % R, prt = x / R;
+      double sz = 0.0;
+      for (int p = prt; p < P; p += 16) sz += w[p] * Z[static_cast<size_t>(p) * R + a];
+      part[x] = sz;
+    }
+    __syncthreads();
+    for (int a = tid; a < R; a += kFitThreads) {
+      double sz = 0.0;
+      for (int prt = 0; prt < 16; ++prt) sz += part[prt * R + a];
+      zbar[a] = sz / static_cast<double>(P);
+    }
+    __syncthreads();
   }
-  // cross = Z_c^T W X_c  -> A (R x D), solved in place below
-  for (int x = tid; x < R * D; x += kFitThreads) {
-    const int a = x / D, e = x % D;
-    double s = 0.0;
-    for (int p = 0; p < P; ++p)
-      s += w[p] * (Z[p * R + a] - zbar[a]) * (static_cast<double>(xs[static_cast<size_t>(p) * D + e]) - xbar[e]);
-    A[x] = s;
-  }
-  __syncthreads();
 
-  // ---- Cholesky (lower, in C)
-  for (int j = 0; j < D; ++j) {
-    if (tid < 32) {
-      double s = 0.0;
-      for (int k = tid; k < j; k += 32) s += C[j * LD + k] * C[j * LD + k];
-      s = warp_sum_d(s);
-      if (tid == 0) {
-        const double dj = C[j * LD + j] - s;
-        if (!(dj > 0.0)) {
-          s_fail = 1;
-          C[j * LD + j] = 1.0;
-        } else {
-          C[j * LD + j] = sqrt(dj);
+  // ---- pass B: Gram = X_c^T W X_c (register blocks as for C) and cross = Z_c^T W X_c
+  // (registers when R <= kTriMaxR: thread tid holds dim tid % D of rows a = tid / D + k (512 / D))
+  constexpr int kCross = kTriMaxR * D / kFitThreads;
+  const bool cross_regs = R <= kTriMaxR;
+  double cacc[kCross];
+#pragma unroll
+  for (int k = 0; k < kCross; ++k) cacc[k] = 0.0;
+  acc_zero();
+  double* wxs = C;                        // staged w_p x_c rows [16][D]
+  double* zst = C + kStageRows * D;       // staged Z_c rows [16][R]
+  for (int p0 = 0; p0 < P; p0 += kStageRows) {
+    __syncthreads();
+    for (int x = tid; x < kStageRows * D; x += kFitThreads) {
+      const int p = p0 + x / D, e = x % D;
+      const double xc = p < P ? static_cast<double>(xs[static_cast<size_t>(p) * D + e]) - xbar[e] : 0.0;
+      stage[x] = xc;
+      wxs[x] = p < P ? w[p] * xc : 0.0;
+    }
+    for (int x = tid; x < kStageRows * R; x += kFitThreads) {
+      const int p = p0 + x / R, a = x % R;
+      zst[x] = p < P ? Z[static_cast<size_t>(p) * R + a] - zbar[a] : 0.0;
+    }
+    __syncthreads();
+    const int nr = min(kStageRows, P - p0);
+    acc_rows(wxs, stage, nr);
+    if (cross_regs) {
+      for (int r = 0; r < nr; ++r) {
+        const double wx = wxs[r * D + tid % D];
+#pragma unroll
+        for (int k = 0; k < kCross; ++k) {
+          const int a = tid / D + k * (kFitThreads / D);
+          if (a < R) cacc[k] = fma(zst[r * R + a], wx, cacc[k]);
         }
       }
     }
-    __syncthreads();
-    const double ljj = C[j * LD + j];
-    for (int i = j + 1 + tid; i < D; i += kFitThreads) {
-      double s = C[i * LD + j];
-      for (int k = 0; k < j; ++k) s -= C[i * LD + k] * C[j * LD + k];
-      C[i * LD + j] = s / ljj;
-    }
-    __syncthreads();
   }
-  // ---- solve (L L^T) a_row = cross_row for every a (one warp per right-hand side)
-  const int lane = tid & 31, warp = tid >> 5;
-  for (int a = warp; a < R; a += kFitThreads / 32) {
-    double* x = A + static_cast<size_t>(a) * D;
-    for (int i = 0; i < D; ++i) {
-      double s = 0.0;
-      for (int k = lane; k < i; k += 32) s += C[i * LD + k] * x[k];
-      s = warp_sum_d(s);
-      if (lane == 0) x[i] = (x[i] - s) / C[i * LD + i];
-      __syncwarp();
+  __syncthreads();
+#pragma unroll
+  for (int k1 = 0; k1 < kRb; ++k1)
+#pragma unroll
+    for (int k2 = 0; k2 < kCb; ++k2) {
+      const int i = bi + kNrb * k1, j = bj + kNcb * k2;
+      C[i * LD + j] = acc[k1][k2] + (i == j ? lambda : 0.0);
     }
-    for (int i = D - 1; i >= 0; --i) {
-      double s = 0.0;
-      for (int k = i + 1 + lane; k < D; k += 32) s += C[k * LD + i] * x[k];
-      s = warp_sum_d(s);
-      if (lane == 0) x[i] = (x[i] - s) / C[i * LD + i];
-      __syncwarp();
+  if (cross_regs) {
+#pragma unroll
+    for (int k = 0; k < kCross; ++k) {
+      const int a = tid / D + k * (kFitThreads / D);
+      if (a < R) A[static_cast<size_t>(a) * D + tid % D] = cacc[k];
+    }
+  } else {
+    for (int x = tid; x < R * D; x += kFitThreads) {
+      const int a = x / D, e = x % D;
+      double sc = 0.0;
+      for (int p = 0; p < P; ++p)
+        sc += w[p] * (Z[static_cast<size_t>(p) * R + a] - zbar[a]) *
+              (static_cast<double>(xs[static_cast<size_t>(p) * D + e]) - xbar[e]);
+      A[x] = sc;
     }
   }
   __syncthreads();
+
+  // ---- Cholesky (lower, in C), right-looking: column j scaled, then the trailing lower
+  // triangle updated by all threads; the thread that finishes entry (j + 1, j + 1) takes
+  // its square root at once (lane 0 of warp 0)
+  const int lane = tid & 31, warp = tid >> 5;
+  double* dinv = t_dd;  // 1 / L_jj (the eigensolver's scratch is free)
+  auto take_root = [&](int j) {
+    const double dj = C[j * LD + j];
+    if (!(dj > 0.0)) {
+      s_fail = 1;
+      C[j * LD + j] = 1.0;
+      dinv[j] = 1.0;
+    } else {
+      const double l = sqrt(dj);
+      C[j * LD + j] = l;
+      dinv[j] = 1.0 / l;
+    }
+  };
+  if (tid == 0) take_root(0);
+  __syncthreads();
+  for (int j = 0; j < D; ++j) {
+    for (int i = j + 1 + tid; i < D; i += kFitThreads) C[i * LD + j] *= dinv[j];
+    __syncthreads();
+    for (int i = j + 1 + warp; i < D; i += kFitThreads / 32) {
+      const double lij = C[i * LD + j];
+      for (int k = j + 1 + lane; k <= i; k += 32) C[i * LD + k] = fma(-lij, C[k * LD + j], C[i * LD + k]);
+    }
+    if (tid == 0 && j + 1 < D) take_root(j + 1);  // row j + 1 is warp 0's, entry j + 1 lane 0's
+    __syncthreads();
+  }
+  // ---- solve (L L^T) a_row = cross_row: warp w takes right-hand sides 2 w, 2 w + 1, ...,
+  // lane l holding entries l, l + 32, ...; column-oriented substitution (the owner lane
+  // finishes entry j and broadcasts it, every lane updates its later entries)
+  constexpr int kRow = D / 32;
+  for (int a0 = 2 * warp; a0 < R; a0 += kFitThreads / 16) {
+    const bool two = a0 + 1 < R;
+    double* xg0 = A + static_cast<size_t>(a0) * D;
+    double* xg1 = A + static_cast<size_t>(two ? a0 + 1 : a0) * D;
+    double x0[kRow], x1[kRow];
+#pragma unroll
+    for (int q = 0; q < kRow; ++q) {
+      x0[q] = xg0[lane + 32 * q];
+      x1[q] = xg1[lane + 32 * q];
+    }
+#pragma unroll
+    for (int q = 0; q < kRow; ++q) {
+      for (int jl = 0; jl < 32; ++jl) {
+        const int j = 32 * q + jl;
+        if (lane == jl) {
+          x0[q] *= dinv[j];
+          x1[q] *= dinv[j];
+        }
+        const double v0 = __shfl_sync(0xffffffffu, x0[q], jl), v1 = __shfl_sync(0xffffffffu, x1[q], jl);
+#pragma unroll
+        for (int q2 = q; q2 < kRow; ++q2) {
+          const int i = lane + 32 * q2;
+          if (i > j) {
+            const double l = C[i * LD + j];
+            x0[q2] = fma(-l, v0, x0[q2]);
+            x1[q2] = fma(-l, v1, x1[q2]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int q = kRow - 1; q >= 0; --q) {
+      for (int jl = 31; jl >= 0; --jl) {
+        const int j = 32 * q + jl;
+        if (lane == jl) {
+          x0[q] *= dinv[j];
+          x1[q] *= dinv[j];
+        }
+        const double v0 = __shfl_sync(0xffffffffu, x0[q], jl), v1 = __shfl_sync(0xffffffffu, x1[q], jl);
+#pragma unroll
+        for (int q2 = 0; q2 <= q; ++q2) {
+          const int i = lane + 32 * q2;
+          if (i < j) {
+            const double l = C[j * LD + i];
+            x0[q2] = fma(-l, v0, x0[q2]);
+            x1[q2] = fma(-l, v1, x1[q2]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < kRow; ++q) {
+      xg0[lane + 32 * q] = x0[q];
+      if (two) xg1[lane + 32 * q] = x1[q];
+    }
+  }
+  __syncthreads();
+  // A (R x D) into shared memory (C is free now) for b and M
+  double* As = C;
+  for (int x = tid; x < R * D; x += kFitThreads) As[x] = A[x];
+  __syncthreads();
   for (int a = tid; a < R; a += kFitThreads) {
-    double s = 0.0;
-    for (int e = 0; e < D; ++e) s += A[static_cast<size_t>(a) * D + e] * xbar[e];
-    bvec[a] = zbar[a] - s;
+    double sb = 0.0;
+    for (int e = 0; e < D; ++e) sb += As[static_cast<size_t>(a) * D + e] * xbar[e];
+    bvec[a] = zbar[a] - sb;
   }
   __syncthreads();
   // ---- M = U_r A, beta = U_r b
   const bool failed = s_fail != 0;
   for (int x = tid; x < D * D; x += kFitThreads) {
     const int i = x / D, j = x % D;
-    double s = 0.0;
+    double sm_ = 0.0;
     for (int a = 0; a < R; ++a)
-      s += static_cast<double>(urow(a)[i]) * A[static_cast<size_t>(a) * D + j];
-    M_out[static_cast<size_t>(head) * D * D + x] = failed ? 0.f : static_cast<float>(s);
+      sm_ += static_cast<double>(urow(a)[i]) * As[static_cast<size_t>(a) * D + j];
+    M_out[static_cast<size_t>(head) * D * D + x] = failed ? 0.f : static_cast<float>(sm_);
   }
   for (int i = tid; i < D; i += kFitThreads) {
     double s = 0.0;

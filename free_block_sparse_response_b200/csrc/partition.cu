@@ -97,19 +97,63 @@ __global__ void chunk_perm_kernel(int* __restrict__ perm, int* __restrict__ size
   }
 }
 
-// c_g = fp32 mean of the members listed in perm (token order); empty groups keep c_g.
+// c_g = fp32 mean of the members listed in perm; empty groups keep c_g.  128 threads:
+// warp w sums the members j = w, w + 4, ... in list order, lane l holding dims
+// [l D/32, (l + 1) D/32) (one vector load per member), and the four partial sums are
+// added in warp order at the end.
 template <typename T, int D>
-__global__ void centroid_kernel(const T* __restrict__ X, int n, const int* __restrict__ perm,
-                                const int* __restrict__ sizes, int G, int cap, float* __restrict__ cent) {
-  const int g = blockIdx.x, head = blockIdx.y, e = threadIdx.x;
+__device__ __forceinline__ void load_dims(const T* p, float (&v)[D / 32]);
+template <>
+__device__ __forceinline__ void load_dims<__nv_bfloat16, 128>(const __nv_bfloat16* p, float (&v)[4]) {
+  const uint2 r = __ldg(reinterpret_cast<const uint2*>(p));
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+  v[0] = a.x, v[1] = a.y, v[2] = b.x, v[3] = b.y;
+}
+template <>
+__device__ __forceinline__ void load_dims<__nv_bfloat16, 64>(const __nv_bfloat16* p, float (&v)[2]) {
+  const uint32_t r = __ldg(reinterpret_cast<const unsigned int*>(p));
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r));
+  v[0] = a.x, v[1] = a.y;
+}
+template <>
+__device__ __forceinline__ void load_dims<float, 128>(const float* p, float (&v)[4]) {
+  const float4 r = __ldg(reinterpret_cast<const float4*>(p));
+  v[0] = r.x, v[1] = r.y, v[2] = r.z, v[3] = r.w;
+}
+template <>
+__device__ __forceinline__ void load_dims<float, 64>(const float* p, float (&v)[2]) {
+  const float2 r = __ldg(reinterpret_cast<const float2*>(p));
+  v[0] = r.x, v[1] = r.y;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(128) centroid_kernel(const T* __restrict__ X, int n, const int* __restrict__ perm,
+                                                       const int* __restrict__ sizes, int G, int cap,
+                                                       float* __restrict__ cent) {
+  constexpr int kPer = D / 32;
+  __shared__ float part[4][D];
+  const int g = blockIdx.x, head = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t goff = static_cast<size_t>(head) * G + g;
   const int size = sizes[goff];
   if (size <= 0) return;
-  const T* x = X + static_cast<size_t>(head) * n * D;
+  const T* x = X + static_cast<size_t>(head) * n * D + lane * kPer;
   const int* pm = perm + goff * cap;
-  float acc = 0.f;
-  for (int j = 0; j < size; ++j) acc += to_f32(x[static_cast<size_t>(__ldg(pm + j)) * D + e]);
-  cent[goff * D + e] = acc / static_cast<float>(size);
+  float acc[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
+#pragma unroll 4
+  for (int j = warp; j < size; j += 4) {
+    float v[kPer];
+    load_dims<T, D>(x + static_cast<size_t>(__ldg(pm + j)) * D, v);
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) acc[i] += v[i];
+  }
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) part[warp][lane * kPer + i] = acc[i];
+  __syncthreads();
+  for (int e = threadIdx.x; e < D; e += 128)
+    cent[goff * D + e] = (((part[0][e] + part[1][e]) + part[2][e]) + part[3][e]) / static_cast<float>(size);
 }
 
 // W = C Gamma (fp32 + bf16 hi/lo) and e_g = c_g . w_g; 8 groups per CTA, thread per dim.
@@ -1003,10 +1047,10 @@ cudaError_t launch_centroid(const void* X, bool f32, int n, const int* perm, con
                             int heads, int d, float* cent, cudaStream_t st) {
   dim3 grid(G, heads);
   if (f32) {
-    if (d == 64) centroid_kernel<float, 64><<<grid, 64, 0, st>>>(static_cast<const float*>(X), n, perm, sizes, G, cap, cent);
+    if (d == 64) centroid_kernel<float, 64><<<grid, 128, 0, st>>>(static_cast<const float*>(X), n, perm, sizes, G, cap, cent);
     else centroid_kernel<float, 128><<<grid, 128, 0, st>>>(static_cast<const float*>(X), n, perm, sizes, G, cap, cent);
   } else {
-    if (d == 64) centroid_kernel<__nv_bfloat16, 64><<<grid, 64, 0, st>>>(static_cast<const __nv_bfloat16*>(X), n, perm, sizes, G, cap, cent);
+    if (d == 64) centroid_kernel<__nv_bfloat16, 64><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(X), n, perm, sizes, G, cap, cent);
     else centroid_kernel<__nv_bfloat16, 128><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(X), n, perm, sizes, G, cap, cent);
   }
   return counted(cudaGetLastError(), 1);

@@ -48,7 +48,7 @@ __device__ __forceinline__ int tri_sturm_count(const double* dd, const double* e
 
 // C [D x (D + 1)] is destroyed.  On return U (fp32, R x D, row a = eigenvector of the
 // a-th largest eigenvalue) holds the vectors and evals[a] the eigenvalues.  Scratch:
-// pack (>= D (D - 1) / 2 doubles), stage (>= 2 D doubles and >= R D floats); C holds the
+// pack (>= D (D - 1) / 2 doubles), stage (>= D + kTriThreads doubles and >= R D floats); C holds the
 // inverse-iteration factors.  All kTriThreads threads of the CTA call it.
 template <int D>
 __device__ void top_eigvecs_tridiagonal(double* C, double* pack, double* stage, float* U, int R, double* dd,
@@ -90,31 +90,54 @@ __device__ void top_eigvecs_tridiagonal(double* C, double* pack, double* stage, 
     __syncthreads();
     const double tau = shk[0], scale = shk[1];
     if (tau == 0.0) continue;  // nothing to annihilate (the same branch for every thread)
-    for (int i = tid; i < m; i += kTriThreads) {
-      const double v = i == 0 ? 1.0 : C[(r0 + i) * LD + k] * scale;
-      vbuf[i] = v;
-      C[(r0 + i) * LD + k] = v;
-    }
-    __syncthreads();
-    for (int i = warp; i < m; i += kWarps) {  // p = tau A v, one warp per row
-      const double* row = C + (r0 + i) * LD + r0;
+    // p = tau A v in kParts column ranges: thread (part, i) sums rows j of its range of
+    // column i (A is symmetric), v_j read straight from column k (v_0 = 1)
+    {
+      constexpr int kParts = kTriThreads / D, kSpan = D / kParts;
+      const int i = tid % D, part = tid / D;
       double acc = 0.0;
-      for (int j = lane; j < m; j += 32) acc += row[j] * vbuf[j];
-      acc = warp_sum_d(acc);
-      if (lane == 0) pbuf[i] = tau * acc;
+      if (i < m) {
+        const int j1 = min(m, (part + 1) * kSpan);
+        for (int j = part * kSpan; j < j1; ++j) {
+          const double vj = j == 0 ? 1.0 : C[(r0 + j) * LD + k] * scale;
+          acc = fma(C[(r0 + j) * LD + r0 + i], vj, acc);
+        }
+        if (part == 0) vbuf[i] = i == 0 ? 1.0 : C[(r0 + i) * LD + k] * scale;
+      }
+      pbuf[part * D + i] = acc;
     }
     __syncthreads();
-    double pv = 0.0;  // every warp forms p . v itself (saves a barrier)
-    for (int j = lane; j < m; j += 32) pv += pbuf[j] * vbuf[j];
-    pv = warp_sum_d(pv);
-    const double kc = -0.5 * tau * pv;  // w = p + kc v;  A <- A - v w^T - w v^T
-    for (int i = warp; i < m; i += kWarps) {
-      double* row = C + (r0 + i) * LD + r0;
-      const double vi = vbuf[i], wi = pbuf[i] + kc * vi;
-      for (int j = lane; j < m; j += 32) {
-        const double vj = vbuf[j];
-        row[j] -= vi * (pbuf[j] + kc * vj) + wi * vj;
+    {
+      constexpr int kParts = kTriThreads / D, kT = D / 32;
+      // every warp: its lanes' p_j and v_j (j = lane + 32 t), p . v, then its rows' update
+      double pj[kT], vj[kT];
+      double pv = 0.0;
+#pragma unroll
+      for (int t = 0; t < kT; ++t) {
+        const int j = lane + 32 * t;
+        double sp = 0.0;
+#pragma unroll
+        for (int q = 0; q < kParts; ++q) sp += pbuf[q * D + j];
+        pj[t] = j < m ? tau * sp : 0.0;
+        vj[t] = j < m ? vbuf[j] : 0.0;
+        pv = fma(pj[t], vj[t], pv);
       }
+      pv = warp_sum_d(pv);
+      const double kc = -0.5 * tau * pv;  // w = p + kc v;  A <- A - v w^T - w v^T
+      for (int i = warp; i < m; i += kWarps) {
+        double pi = 0.0;
+#pragma unroll
+        for (int q = 0; q < kParts; ++q) pi += pbuf[q * D + i];
+        const double vi = vbuf[i], wi = tau * pi + kc * vi;
+        double* row = C + (r0 + i) * LD + r0;
+#pragma unroll
+        for (int t = 0; t < kT; ++t) {
+          const int j = lane + 32 * t;
+          if (j < m) row[j] -= vi * (pj[t] + kc * vj[t]) + wi * vj[t];
+        }
+      }
+      if (warp == 0)  // the reflector, kept in column k for the back-transformation
+        for (int i = lane; i < m; i += 32) C[(r0 + i) * LD + k] = vbuf[i];
     }
     __syncthreads();
   }
@@ -253,17 +276,40 @@ __device__ void top_eigvecs_tridiagonal(double* C, double* pack, double* stage, 
         const double inv = imx / sqrt(n2);
         for (int i = 0; i < D; ++i) S(i, 3) *= inv;
       }
-      // back-transformation u = H_0 H_1 ... H_{D-3} z (this thread's vector)
+    }
+    __syncthreads();
+    // back-transformation u = H_0 H_1 ... H_{D-3} z: 16 threads (half a warp) per vector,
+    // thread sub holding entries sub, sub + 16, ...
+    {
+      constexpr int kE = D / 16;
+      const int g = tid >> 4, sub = tid & 15;
+      const bool act = g < nb;
+      double z[kE];
+#pragma unroll
+      for (int q = 0; q < kE; ++q) z[q] = act ? C[((sub + 16 * q) * 4 + 3) * kBatch + g] : 0.0;
       for (int k = D - 3; k >= 0; --k) {
         const double tk = tauh[k];
         if (tk == 0.0) continue;
-        const int off = k * (D - 1) - k * (k - 1) / 2, m = D - 1 - k;
-        double s4[4] = {0.0, 0.0, 0.0, 0.0};
-        for (int i = 0; i < m; ++i) s4[i & 3] += pack[off + i] * S(k + 1 + i, 3);
-        const double s = tk * ((s4[0] + s4[1]) + (s4[2] + s4[3]));
-        for (int i = 0; i < m; ++i) S(k + 1 + i, 3) -= s * pack[off + i];
+        const int off = k * (D - 1) - k * (k - 1) / 2 - (k + 1);  // pack index of entry i: off + i
+        double part = 0.0;
+#pragma unroll
+        for (int q = 0; q < kE; ++q) {
+          const int i = sub + 16 * q;
+          if (i > k) part = fma(pack[off + i], z[q], part);
+        }
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+        const double sk = tk * part;
+#pragma unroll
+        for (int q = 0; q < kE; ++q) {
+          const int i = sub + 16 * q;
+          if (i > k) z[q] = fma(-sk, pack[off + i], z[q]);
+        }
       }
-      for (int i = 0; i < D; ++i) Us[a * D + i] = static_cast<float>(S(i, 3));
+      if (act) {
+#pragma unroll
+        for (int q = 0; q < kE; ++q) Us[(b0 + g) * D + sub + 16 * q] = static_cast<float>(z[q]);
+      }
     }
     __syncthreads();
   }

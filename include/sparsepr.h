@@ -27,6 +27,7 @@
  *    are a status header that must be zero before the first call on a new workspace
  *    (sparsepr_partition zeroes it again at the start of every call sequence).
  *  - Every call is asynchronous on `stream` (0 = legacy default stream).
+ *  - Q, K and V start on 16-byte boundaries (else SPARSEPR_ERR_INVALID_ARG).
  *  - Layouts are contiguous row-major: Q, K, V, O are [Bt, H, N, d]; per-head index
  *    arrays are [Bt, H, ...] as stated.  dtype is SPARSEPR_BF16 or SPARSEPR_F32;
  *    d is 64 or 128; block B is 64 or 128; indices are int32, pair counts int64.

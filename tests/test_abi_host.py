@@ -84,3 +84,20 @@ def test_python_wrappers_refuse_cpu_tensors():
     q = torch.zeros(1, 1, 64, 64)
     with pytest.raises(ValueError):
         spr.dense_attn(q, q, q, block=64)
+
+
+def test_misaligned_inputs_are_refused(L):
+    """Q, K and V are read with 16-byte vector and TMA loads: a start off a 16-byte
+    boundary is refused before anything is launched (pointers never dereferenced)."""
+    cfg = spr.SparsePRConfig(block=128).c()
+    ok, odd = ctypes.c_void_p(256), ctypes.c_void_p(256 + 8)
+    rc = L.sparsepr_partition(ok, odd, spr.BF16, 1, 1, 1024, 128, ctypes.byref(cfg), None, ok, ok, ok, ok, ok, ok,
+                              None)
+    assert rc == spr.ERR_INVALID_ARG
+    assert b"16-byte" in L.sparsepr_last_error()
+    rc = L.sparsepr_sparse_attn(odd, ok, ok, spr.BF16, 1, 1, 1024, 128, 128, ok, ok, ok, ok, ok, 1, 0.0, ok, ok,
+                                None)
+    assert rc == spr.ERR_INVALID_ARG
+    rc = L.sparsepr_probe_dense(ok, ok, odd, spr.BF16, 1, 1, 1024, 128, 128, ok, 8, ok, ok, ok, ok, 1, 0.0, ok, ok,
+                                ok, None)
+    assert rc == spr.ERR_INVALID_ARG
