@@ -10,5 +10,6 @@ from .sparsepr import (  # noqa: F401
     WEIGHT_INV_NORM, WEIGHT_UNIFORM, PARTITION_RESPONSE, PARTITION_SEMANTIC, ROUTE_CENTROID, ROUTE_SIZE_CORRECTED, ROUTE_LSE,
     Partition, SparsePRConfig, SparsePRError, apply_residual, attention, check,
     dense_attn, fit_residual, fit_residual_noalloc, lib, new_workspace, num_groups, partition, probe_dense, probe_rows, route, route_k,
-    sparse_attn, sparse_attn_apply, fused_supported, reset_workspace, test_fill, test_topk, workspace_size, row_errors, launch_count, kernel_timing, kernel_timing_read,
+    sparse_attn, sparse_attn_apply, fused_supported, reset_workspace, attention_call, attention_host, call_workspace,
+    host_workspace, test_fill, test_topk, workspace_size, row_errors, launch_count, kernel_timing, kernel_timing_read,
 )

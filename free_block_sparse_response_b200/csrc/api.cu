@@ -42,6 +42,14 @@ int cuda_fail(cudaError_t e, const char* where) {
   return fail(SPARSEPR_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
 }
 
+}  // namespace
+
+namespace spr {
+int api_fail(int code, const char* msg) { return fail(code, "%s", msg); }
+}  // namespace spr
+
+namespace {
+
 #define SPR_CUDA(call, where)                       \
   do {                                              \
     cudaError_t e_ = (call);                        \

@@ -29,7 +29,8 @@ EXPORTED_SYMBOLS = (
     "sparsepr_last_error", "sparsepr_test_fill_workspace_size", "sparsepr_test_fill",
     "sparsepr_test_topk", "sparsepr_row_errors", "sparsepr_launch_count", "sparsepr_fit_residual_noalloc",
     "sparsepr_kernel_timing", "sparsepr_kernel_timing_read", "sparsepr_test_fill_segmented",
-    "sparsepr_sparse_attn_apply", "sparsepr_reset_workspace",
+    "sparsepr_sparse_attn_apply", "sparsepr_reset_workspace", "sparsepr_call_workspace_size", "sparsepr_attention",
+    "sparsepr_host_workspace_size", "sparsepr_attention_host",
 )
 
 
@@ -118,6 +119,12 @@ def lib() -> ctypes.CDLL:
         "sparsepr_kernel_timing_read": (ctypes.c_int, [_vp, _vp]),
         "sparsepr_fit_residual_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, ctypes.c_double,
                                                          _i32, _i32, _vp, _vp, _vp]),
+        "sparsepr_call_workspace_size": (ctypes.c_size_t, [ctypes.c_int, _i32, _i32, _i32, _i32, P]),
+        "sparsepr_attention": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32, P, _vp, _vp,
+                                              _vp]),
+        "sparsepr_host_workspace_size": (ctypes.c_size_t, [ctypes.c_int, _i32, _i32, _i32, _i32, P, _i32]),
+        "sparsepr_attention_host": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32, P, _vp,
+                                                   _i32, _vp, _vp, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -422,3 +429,66 @@ def test_topk(scores: torch.Tensor, k: int) -> torch.Tensor:
     _call("sparsepr_test_topk", _p(scores), h, gq, g, k, _p(rt), _p(ws), _stream(scores))
     check(ws)
     return rt
+
+
+# ------------------------------------------------------------------ one-call entry points
+
+def call_workspace(q: torch.Tensor, cfg: SparsePRConfig) -> torch.Tensor:
+    """Workspace of the one-call entry ``attention_call`` (header zeroed)."""
+    bt, h, n, d = q.shape
+    size = int(lib().sparsepr_call_workspace_size(_dtype_code(q), bt, h, n, d, ctypes.byref(cfg.c())))
+    if size == 0:
+        raise SparsePRError(ERR_INVALID_ARG, "invalid sizes or parameters for the call")
+    ws = torch.empty(size, dtype=torch.uint8, device=q.device)
+    ws[:256].zero_()
+    return ws
+
+
+def attention_call(q, k, v, cfg: SparsePRConfig, ws: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The whole call as one native entry point (``sparsepr_attention``): the same stages
+    and order as ``attention``, every intermediate in ``ws``."""
+    _need_cuda(q, k, v)
+    bt, h, n, d = q.shape
+    ws = call_workspace(q, cfg) if ws is None else ws
+    o = torch.empty_like(q) if out is None else out
+    _call("sparsepr_attention", _p(q), _p(k), _p(v), _dtype_code(q), bt, h, n, d, ctypes.byref(cfg.c()), _p(o),
+          _p(ws), _stream(q))
+    return o
+
+
+_COPY_STREAMS = {}
+
+
+def host_workspace(q: torch.Tensor, cfg: SparsePRConfig, groups: int, device=None) -> torch.Tensor:
+    """Device workspace of ``attention_host`` for host tensors shaped like q."""
+    bt, h, n, d = q.shape
+    size = int(lib().sparsepr_host_workspace_size(_dtype_code(q), bt, h, n, d, ctypes.byref(cfg.c()), groups))
+    if size == 0:
+        raise SparsePRError(ERR_INVALID_ARG, "invalid sizes or parameters for the host call")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    ws = torch.empty(size, dtype=torch.uint8, device=dev)
+    ws[:256].zero_()
+    return ws
+
+
+def attention_host(q, k, v, cfg: SparsePRConfig, out: Optional[torch.Tensor] = None, groups: int = 4,
+                   ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The call from host tensors (``sparsepr_attention_host``): heads in ``groups`` groups,
+    the copies of neighbouring groups overlapping each group's compute.  q, k, v and out
+    live in page-locked host memory for the overlap; out is complete once the current
+    stream is (``torch.cuda.current_stream().synchronize()``)."""
+    for t in (q, k, v):
+        if t.is_cuda or not t.is_contiguous():
+            raise SparsePRError(ERR_INVALID_ARG, "attention_host takes contiguous host tensors")
+    bt, h, n, d = q.shape
+    ws = host_workspace(q, cfg, groups) if ws is None else ws
+    o = torch.empty(q.shape, dtype=q.dtype, pin_memory=True) if out is None else out
+    dev = ws.device
+    copy = _COPY_STREAMS.get(dev.index)
+    if copy is None:
+        copy = _COPY_STREAMS[dev.index] = torch.cuda.Stream(device=dev)
+    _call("sparsepr_attention_host", _p(q), _p(k), _p(v), _dtype_code(q), bt, h, n, d, ctypes.byref(cfg.c()),
+          _p(o), groups, _p(ws), ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream),
+          ctypes.c_void_p(copy.cuda_stream))
+    return o

@@ -187,6 +187,34 @@ SPARSEPR_API int sparsepr_sparse_attn_apply(const void* Q, const void* K, const 
                          const float* beta, const int32_t* probe_idx, int32_t P,
                          const float* probe_out, void* O, void* ws, sparsepr_stream_t stream);
 
+/* One whole SparsePR call on device tensors (S1-S10 in one entry point): partition,
+ * route, probe rows (midpoint stride), then -- for bf16, d = 128, B = 128 -- probe rows,
+ * fit and the sparse attention with the correction in its epilogue; for other shapes the
+ * sparse attention, probe rows, fit and apply.  Every intermediate lives in `ws`, of
+ * sparsepr_call_workspace_size() bytes (256-byte aligned, first 256 bytes zero before the
+ * first call); O [Bt,H,N,d] in dtype.  params->n_probe must be >= 1.  Errors as for the
+ * stage calls; sparsepr_check(ws) reads the device status. */
+SPARSEPR_API size_t sparsepr_call_workspace_size(int dtype, int32_t Bt, int32_t H, int32_t N, int32_t d,
+                                                 const sparsepr_params* params);
+SPARSEPR_API int sparsepr_attention(const void* Q, const void* K, const void* V, int dtype, int32_t Bt,
+                                    int32_t H, int32_t N, int32_t d, const sparsepr_params* params, void* O,
+                                    void* ws, sparsepr_stream_t stream);
+
+/* The same call with Q, K, V and O in HOST memory (page-locked, or the copies do not
+ * overlap).  The Bt*H heads are processed in `groups` consecutive groups (every head is
+ * an independent problem, so the result is the same for any grouping): while the group
+ * g runs on `stream`, `copy_stream` carries group g + 1 to the device and group g - 1
+ * back.  ws: sparsepr_host_workspace_size() bytes (first 256 bytes zero before the first
+ * call; sparsepr_check(ws) then reports a device error of any group).  Returns after
+ * enqueueing; the host O is complete once `stream` is.  Host calls on one device must not
+ * overlap in time (they share the device's copy events). */
+SPARSEPR_API size_t sparsepr_host_workspace_size(int dtype, int32_t Bt, int32_t H, int32_t N, int32_t d,
+                                                 const sparsepr_params* params, int32_t groups);
+SPARSEPR_API int sparsepr_attention_host(const void* Q, const void* K, const void* V, int dtype, int32_t Bt,
+                                         int32_t H, int32_t N, int32_t d, const sparsepr_params* params,
+                                         void* O, int32_t groups, void* ws, sparsepr_stream_t stream,
+                                         sparsepr_stream_t copy_stream);
+
 /* Dense softmax attention of every row against all N keys with the same kernel
  * family (the comparator the density budget is measured against):
  *   O_out [Bt,H,N,d] fp32. */

@@ -101,3 +101,21 @@ def test_misaligned_inputs_are_refused(L):
     rc = L.sparsepr_probe_dense(ok, ok, odd, spr.BF16, 1, 1, 1024, 128, 128, ok, 8, ok, ok, ok, ok, 1, 0.0, ok, ok,
                                 ok, None)
     assert rc == spr.ERR_INVALID_ARG
+
+
+def test_one_call_entries_refuse_bad_arguments(L):
+    """The one-call entries check their arguments before anything is launched."""
+    cfg = spr.SparsePRConfig(block=128, n_probe=0).c()
+    ok = ctypes.c_void_p(256)
+    assert L.sparsepr_call_workspace_size(spr.BF16, 1, 2, 1024, 128, ctypes.byref(cfg)) == 0  # n_probe = 0
+    rc = L.sparsepr_attention(ok, ok, ok, spr.BF16, 1, 2, 1024, 128, ctypes.byref(cfg), ok, ok, None)
+    assert rc == spr.ERR_INVALID_ARG
+    good = spr.SparsePRConfig(block=128, n_sampled=64, n_probe=16).c()
+    assert L.sparsepr_call_workspace_size(spr.BF16, 1, 2, 1024, 128, ctypes.byref(good)) > \
+        L.sparsepr_workspace_size(1, 2, 1024, 128, ctypes.byref(good))
+    assert L.sparsepr_host_workspace_size(spr.BF16, 1, 2, 1024, 128, ctypes.byref(good), 0) == 0
+    rc = L.sparsepr_attention_host(ok, ok, ok, spr.BF16, 1, 2, 1024, 128, ctypes.byref(good), ok, 0, ok, None, None)
+    assert rc == spr.ERR_INVALID_ARG and b"groups" in L.sparsepr_last_error()
+    s = ctypes.c_void_p(4096)
+    rc = L.sparsepr_attention_host(ok, ok, ok, spr.BF16, 1, 2, 1024, 128, ctypes.byref(good), ok, 2, ok, s, s)
+    assert rc == spr.ERR_INVALID_ARG and b"copy stream" in L.sparsepr_last_error()

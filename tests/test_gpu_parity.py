@@ -436,3 +436,33 @@ def test_long_config_sampled_rows():
     distance segments per row)."""
     w = CONFIGS["long"]
     _full_size_sampled_rows(w, 202, (0, w.heads - 1))
+
+
+@pytest.mark.parametrize("cfg_name,heads", [("small", 3), ("tiny", None)])
+def test_one_call_entry_matches_stage_pipeline(cfg_name, heads):
+    """sparsepr_attention (every stage behind one native entry, intermediates in its own
+    workspace) gives the stage pipeline's output bit for bit: the fused bf16 order and the
+    unfused fp32 order."""
+    w = CONFIGS[cfg_name]
+    cfg = spr_cfg(w)
+    q, k, v = (t.cuda() for t in make_inputs(w, 5, heads=heads))
+    o_stages = spr.attention(q, k, v, cfg)
+    ws = spr.call_workspace(q, cfg)
+    o_call = spr.attention_call(q, k, v, cfg, ws=ws)
+    spr.check(ws)
+    assert torch.equal(o_call, o_stages)
+
+
+def test_host_entry_matches_device_call():
+    """sparsepr_attention_host on pinned host tensors, heads in ragged groups (3, 3, 2),
+    equals the device call bit for bit (every head is an independent problem)."""
+    w = CONFIGS["small"]
+    cfg = spr_cfg(w)
+    q, k, v = make_inputs(w, 6)
+    qp, kp, vp = (t.contiguous().pin_memory() for t in (q, k, v))
+    o_dev = spr.attention_call(qp.cuda(), kp.cuda(), vp.cuda(), cfg)
+    ws = spr.host_workspace(qp, cfg, 3)
+    o_host = spr.attention_host(qp, kp, vp, cfg, groups=3, ws=ws)
+    torch.cuda.current_stream().synchronize()
+    spr.check(ws)
+    assert torch.equal(o_host, o_dev.cpu())
