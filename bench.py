@@ -44,6 +44,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="video")
     ap.add_argument("--heads", type=int, default=0, help="override the head count (profiling runs)")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle's CPU timing (profiling runs; cpu_baseline is then null)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--study", choices=["ablation", "probe-budget", "routing"], default=None,
                     help="error studies instead of the timed run (one JSON line per variant)")
@@ -249,7 +251,7 @@ def run_ours(args, w):
     spr.lib()
 
     cpu_base = None
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu_sec, cpu_desc, cpu_threads = oracle_sample(w, args.seed)
         cpu_base = {"value": dense_flops(w) / cpu_sec / 1e12, "unit": UNIT, "cores": cpu_threads,
                     "kind": "oracle", "sample": cpu_desc}
