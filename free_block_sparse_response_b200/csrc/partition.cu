@@ -630,17 +630,26 @@ __global__ void __launch_bounds__(kFillThreads, 3) fill_coop_kernel(FillArgs a) 
         // key, so the result equals the argmin over the whole row's open groups.  The
         // segment of the item's previous proposal (a group that has just filled, and the
         // row's smallest key) is read in the same wave as the keys, since it nearly always
-        // has to be.  The next batch's item indices are fetched one batch ahead.
+        // has to be.
         const int sub = lane & 7;
         const int qb = lane & 24;  // first lane of this item's quarter
         const unsigned long long inf_key = static_cast<unsigned long long>(float_order_key(__int_as_float(0x7f800000)))
                                            << 32;
+        // Software pipeline: the item indices two batches ahead and the previous proposal
+        // (which names the segment read with the keys) one batch ahead.
+        const int stride = nwarps * 4;
         int x = gwarp * 4 + (lane >> 3);
-        int item_next = x < ncur ? __ldcg(L + x) : 0;
-        for (int x0 = gwarp * 4; x0 < ncur; x0 += nwarps * 4, x += nwarps * 4) {
+        int item_a = x < ncur ? __ldcg(L + x) : 0;
+        int item_b = x + stride < ncur ? __ldcg(L + x + stride) : 0;
+        int gp_a = (x < ncur && round > 0) ? __ldcg(a.prop_g + item_a) : -1;
+        for (int x0 = gwarp * 4; x0 < ncur; x0 += stride, x += stride) {
           const bool valid = x < ncur;
-          const int item = item_next;
-          item_next = x + nwarps * 4 < ncur ? __ldcg(L + x + nwarps * 4) : 0;
+          const int item = item_a;
+          const int gp = gp_a;
+          const int item_c = x + 2 * stride < ncur ? __ldcg(L + x + 2 * stride) : 0;
+          gp_a = (x + stride < ncur && round > 0) ? __ldcg(a.prop_g + item_b) : -1;
+          item_a = item_b;
+          item_b = item_c;
           const int h = item / n;
           const unsigned int* closed = closed_all + static_cast<size_t>(h) * words;
           const float* drow = a.D + static_cast<size_t>(item) * a.ldd;
@@ -648,7 +657,6 @@ __global__ void __launch_bounds__(kFillThreads, 3) fill_coop_kernel(FillArgs a) 
           unsigned long long* srow = a.seg_min + static_cast<size_t>(item) * a.nseg;
           const unsigned long long key0 = valid && sub < a.nseg ? __ldcg(srow + sub) : ~0ull;
           const unsigned long long key1 = valid && sub + 8 < a.nseg ? __ldcg(srow + sub + 8) : ~0ull;
-          const int gp = (valid && round > 0) ? __ldcg(a.prop_g + item) : -1;
           const int sp = gp >= 0 ? (gp >> 7) * 2 + ((gp >> 6) & 1) : -1;
           const int pcol0 = sp >= 0 ? (sp >> 1) * 128 + (sp & 1) * 64 : 0;
           // lane sub's 8 columns of the 64-column segment at col0: col0 + 4 sub + {0..3} and
