@@ -97,6 +97,27 @@ cudaError_t host_events(HostEvents** out) {
 
 size_t elem_bytes(int dtype) { return dtype == SPARSEPR_BF16 ? 2 : 4; }
 
+// Head groups of the host call: the first about half the size of the others, so that
+// only a short copy precedes the first compute; the rest equal (the last one ragged).
+struct GroupPlan {
+  int first, rest, count, max_heads;
+  int start(int g) const { return g == 0 ? 0 : first + (g - 1) * rest; }
+};
+GroupPlan group_plan(int heads, int groups) {
+  GroupPlan gp;
+  if (groups <= 1 || heads <= 1) {
+    gp.first = gp.rest = gp.max_heads = heads;
+    gp.count = 1;
+    return gp;
+  }
+  gp.first = (heads + 2 * groups - 2) / (2 * groups - 1);
+  gp.rest = (heads - gp.first + groups - 2) / (groups - 1);
+  if (gp.rest < 1) gp.rest = 1;
+  gp.count = 1 + (heads - gp.first + gp.rest - 1) / gp.rest;
+  gp.max_heads = gp.first > gp.rest ? gp.first : gp.rest;
+  return gp;
+}
+
 }  // namespace
 
 extern "C" {
@@ -149,7 +170,7 @@ int sparsepr_attention(const void* Q, const void* K, const void* V, int dtype, i
 size_t sparsepr_host_workspace_size(int dtype, int32_t Bt, int32_t H, int32_t N, int32_t d,
                                     const sparsepr_params* params, int32_t groups) {
   if (groups < 1 || Bt < 1 || H < 1) return 0;
-  const int heads = Bt * H, hg = (heads + groups - 1) / groups;
+  const int hg = group_plan(Bt * H, groups).max_heads;
   const size_t call = sparsepr_call_workspace_size(dtype, 1, hg, N, d, params);
   if (call == 0) return 0;
   const size_t tensor = al(static_cast<size_t>(hg) * N * d * elem_bytes(dtype));
@@ -164,7 +185,9 @@ int sparsepr_attention_host(const void* Q, const void* K, const void* V, int dty
   if (stream == copy_stream) return spr::api_fail(SPARSEPR_ERR_INVALID_ARG, "the copy stream must differ from the compute stream");
   if (sparsepr_host_workspace_size(dtype, Bt, H, N, d, p, groups) == 0)
     return spr::api_fail(SPARSEPR_ERR_INVALID_ARG, "invalid sizes or parameters for the call (n_probe must be in [1, N])");
-  const int heads = Bt * H, hg = (heads + groups - 1) / groups, ng = (heads + hg - 1) / hg;
+  const int heads = Bt * H;
+  const GroupPlan plan = group_plan(heads, groups);
+  const int hg = plan.max_heads, ng = plan.count;
   const size_t call = al(sparsepr_call_workspace_size(dtype, 1, hg, N, d, p));
   const size_t per_head = static_cast<size_t>(N) * d * elem_bytes(dtype);
   const size_t tensor = al(static_cast<size_t>(hg) * per_head);
@@ -189,8 +212,15 @@ int sparsepr_attention_host(const void* Q, const void* K, const void* V, int dty
   // copy order: in(0), in(1), [done 0] out(0), in(2), [done 1] out(1), in(3), ... so that
   // group g + 1 lands during group g, and a buffer is refilled only after its last
   // group's output has been copied back
+  auto span = [&](int g, int* h0, int* nh) {
+    *h0 = plan.start(g);
+    const int want = g == 0 ? plan.first : plan.rest;
+    *nh = heads - *h0 < want ? heads - *h0 : want;
+  };
   auto copy_in = [&](int g) -> cudaError_t {
-    const int b = g & 1, h0 = g * hg, nh = heads - h0 < hg ? heads - h0 : hg;
+    int h0, nh;
+    span(g, &h0, &nh);
+    const int b = g & 1;
     const size_t off = static_cast<size_t>(h0) * per_head, bytes = static_cast<size_t>(nh) * per_head;
     cudaError_t r;
     if ((r = cudaMemcpyAsync(dbuf(b, 0), hq + off, bytes, cudaMemcpyHostToDevice, xs)) != cudaSuccess) return r;
@@ -200,7 +230,9 @@ int sparsepr_attention_host(const void* Q, const void* K, const void* V, int dty
   };
   if ((e = copy_in(0)) != cudaSuccess) return cuda_err(e);
   for (int g = 0; g < ng; ++g) {
-    const int b = g & 1, h0 = g * hg, nh = heads - h0 < hg ? heads - h0 : hg;
+    int h0, nh;
+    span(g, &h0, &nh);
+    const int b = g & 1;
     if (g + 1 < ng && (e = copy_in(g + 1)) != cudaSuccess) return cuda_err(e);
     if ((e = cudaStreamWaitEvent(cs, ev->in[b], 0)) != cudaSuccess) return cuda_err(e);
     const int rc = sparsepr_attention(dbuf(b, 0), dbuf(b, 1), dbuf(b, 2), dtype, 1, nh, N, d, p, dbuf(b, 3), cws,

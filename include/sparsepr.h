@@ -201,8 +201,9 @@ SPARSEPR_API int sparsepr_attention(const void* Q, const void* K, const void* V,
                                     void* ws, sparsepr_stream_t stream);
 
 /* The same call with Q, K, V and O in HOST memory (page-locked, or the copies do not
- * overlap).  The Bt*H heads are processed in `groups` consecutive groups (every head is
- * an independent problem, so the result is the same for any grouping): while the group
+ * overlap).  The Bt*H heads are processed in `groups` consecutive groups, the first about
+ * half the size of the others so that only a short copy precedes the first compute (every
+ * head is an independent problem, so the result is the same for any grouping): while the group
  * g runs on `stream`, `copy_stream` carries group g + 1 to the device and group g - 1
  * back.  ws: sparsepr_host_workspace_size() bytes (first 256 bytes zero before the first
  * call; sparsepr_check(ws) then reports a device error of any group).  Returns after

@@ -454,7 +454,7 @@ def test_one_call_entry_matches_stage_pipeline(cfg_name, heads):
 
 
 def test_host_entry_matches_device_call():
-    """sparsepr_attention_host on pinned host tensors, heads in ragged groups (3, 3, 2),
+    """sparsepr_attention_host on pinned host tensors, heads in ragged groups (2, 3, 3),
     equals the device call bit for bit (every head is an independent problem)."""
     w = CONFIGS["small"]
     cfg = spr_cfg(w)
