@@ -5,14 +5,15 @@
 // calibrate the correction).  The softmax weights enter the PV products as bf16 hi + lo
 // (two products each), so the fit sees ~16-bit weights.
 //
-// CTA = (128 probe rows, one split of the key groups, head); 256 threads:
+// CTA = (128 probe rows, one split of the key groups, head); 384 threads:
 //   warp 0      gathers the 128 probe rows of Q (tile::gather4), then loads each key
 //               group's K tile (two TMA boxes) from the group-ordered copy, two stages;
 //   warp 2      the same for V;
 //   warp 1      MMA issuer (one lane): S = Q K^T; once the softmax holds S the next S;
 //               then O_d += P_d,hi V + P_d,lo V (P_d from TMEM) and O_s += P_s,hi V +
 //               P_s,lo V (P_s from shared memory);
-//   warps 4-7   softmax, thread i = probe row i: running (max, sum) of the dense and of
+//   warps 4-11  softmax, two threads per probe row (columns 0-63 and 64-127 of the tile,
+//               row maxima exchanged once per tile): running (max, sum) of the dense and of
 //               the sparse state (the latter only on groups routed to the row's block;
 //               zero weights elsewhere), lazy rescaling of O_d / O_s (max grows by > 2^8).
 // The split of the key groups is at most 64 groups (membership is a 64-bit mask per row).
@@ -30,7 +31,7 @@
 namespace spr {
 namespace {
 
-constexpr int kPtThreads = 256;
+constexpr int kPtThreads = 384;
 constexpr uint32_t kPtTile = 128 * 128 * 2;
 constexpr uint32_t kPtTmemCols = 512;
 constexpr float kPtRescaleLog2 = 8.0f;
@@ -38,7 +39,7 @@ constexpr float kPtInf = __builtin_huge_valf();
 
 enum : int {
   kPQFull = 0, kPKFull0 = 1, kPVFull0 = 3, kPKEmpty0 = 5, kPVEmpty0 = 7, kPSFull = 9, kPSFree = 10,
-  kPPFull = 11, kPPVDone = 12, kPDrain = 13, kPNumBars = 14
+  kPPFull = 11, kPPVDone = 12, kPDrain = 13, kPLx = 14, kPNumBars = 15
 };
 
 __device__ __forceinline__ float pt_ex2(float x) {
@@ -94,8 +95,9 @@ __global__ void __launch_bounds__(kPtThreads, 1)
       tc::mbar_init(bar(kPVEmpty0 + s), 1);
     }
     tc::mbar_init(bar(kPSFull), 1);
-    tc::mbar_init(bar(kPSFree), 128);
-    tc::mbar_init(bar(kPPFull), 128);
+    tc::mbar_init(bar(kPSFree), 256);
+    tc::mbar_init(bar(kPPFull), 256);
+    tc::mbar_init(bar(kPLx), 256);
     tc::mbar_init(bar(kPPVDone), 1);
     tc::mbar_init(bar(kPDrain), 1);
     abort_flag = 0;
@@ -202,13 +204,20 @@ __global__ void __launch_bounds__(kPtThreads, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ softmax
-    // Thread r holds probe row r.  Both states run in log2 units (scores x scale_log2).
-    // The sparse weights reuse the dense exponentials: 2^(y - m_s) = 2^(y - m_d) 2^(m_d - m_s),
-    // which is exact unless 2^(y - m_d) underflows; a row whose sparse maximum trails the
-    // dense one by more than 2^64 takes its own exponentials instead (warp-uniform branch).
+    // Two threads per probe row: warp (quadrant q, half h) holds row 32 q + lane, columns
+    // [64 h, 64 h + 64) of S and of P, and columns [64 h, 64 h + 64) of O_d / O_s.  Each
+    // half also reads the other half of its row of S from TMEM for the row maximum (so
+    // both take the same maximum), and keeps its own partial sums, added at the end.
+    // Both states run in log2 units (scores x scale_log2).  The sparse weights reuse the
+    // dense exponentials: 2^(y - m_s) = 2^(y - m_d) 2^(m_d - m_s), exact unless
+    // 2^(y - m_d) underflows; a row whose sparse maximum trails the dense one by more than
+    // 2^64 takes its own exponentials instead (warp-uniform branch).
+    const int hf = (warp - 4) >> 2;
     const int r = 32 * (warp & 3) + lane;
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    const uint32_t tS = tbase + lane_off, tOd = tS + 128, tOs = tS + 256, tPh = tS + 384, tPl = tS + 448;
+    const uint32_t tS = tbase + lane_off + 64 * hf, tSo = tbase + lane_off + 64 * (1 - hf), tOd = tbase + lane_off + 128 + 64 * hf,
+                   tOs = tbase + lane_off + 256 + 64 * hf, tPh = tbase + lane_off + 384 + 32 * hf,
+                   tPl = tbase + lane_off + 448 + 32 * hf;
     const int tok = __ldg(pidx + prow0 + (r < nrows ? r : 0));
     const int qb = __ldg(qblock_of_token + static_cast<size_t>(head) * N + tok);
     uint64_t member_bits = 0;  // bit (g - g0): group g routed to this row's query block
@@ -225,7 +234,7 @@ __global__ void __launch_bounds__(kPtThreads, 1)
       }
     }
     const int* gsz = key_gsize + static_cast<size_t>(head) * G;
-    float m_d = -kPtInf, l_d = 0.f, m_s = -kPtInf, l_s = 0.f;
+    float m_d = -kPtInf, l_d = 0.f, m_s = -kPtInf, l_s = 0.f;  // l_*: this half's part
     bool ok = true, zeroed = false;
     int nv_next = n_tiles > 0 ? __ldg(gsz + g0) : 0;
     for (int t = 0; t < n_tiles; ++t) {
@@ -236,27 +245,35 @@ __global__ void __launch_bounds__(kPtThreads, 1)
         break;
       }
       tc::fence_after_sync();
-      uint32_t u[128];
+      uint32_t u[64];
       tc::tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
       tc::tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-      tc::tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&u[64]));
-      tc::tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&u[96]));
       tc::tmem_wait_ld();
-      tc::fence_before_sync();
-      tc::mbar_arrive(bar(kPSFree));  // S may take the next tile
       if (nvalid < 128) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= nvalid) u[c] = __float_as_uint(-kPtInf);
+        for (int c = 0; c < 64; ++c)
+          if (64 * hf + c >= nvalid) u[c] = __float_as_uint(-kPtInf);
       }
       float mx8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx8[i] = __uint_as_float(u[i]);
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(u[c]));
-      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      mx *= scale_log2;
+      for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(u[c]));
+      // the other half of the row (maximum only)
+#pragma unroll
+      for (int q2 = 0; q2 < 2; ++q2) {
+        uint32_t w32[32];
+        tc::tmem_ld32(tSo + 32 * q2, w32);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (nvalid >= 128 || 64 * (1 - hf) + 32 * q2 + c < nvalid)
+            mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(w32[c]));
+      }
+      tc::fence_before_sync();
+      tc::mbar_arrive(bar(kPSFree));  // S may take the next tile once both halves hold it
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]))) * scale_log2;
       // dense state: lazy rescale (the running max moves only when it grows by > 2^8)
       const bool grow_d = mx > m_d + kPtRescaleLog2;
       const bool need_od = grow_d && m_d != -kPtInf;
@@ -287,7 +304,7 @@ __global__ void __launch_bounds__(kPtThreads, 1)
       if (!any_far) {
         // dense weights in place, while the previous tile's PV products still run
 #pragma unroll
-        for (int c = 0; c < 128; c += 2) {
+        for (int c = 0; c < 64; c += 2) {
           const float p0 = pt_ex2(fmaf(__uint_as_float(u[c]), scale_log2, -md_safe));
           const float p1 = pt_ex2(fmaf(__uint_as_float(u[c + 1]), scale_log2, -md_safe));
           u[c] = __float_as_uint(p0);
@@ -308,7 +325,7 @@ __global__ void __launch_bounds__(kPtThreads, 1)
           if (!__any_sync(0xffffffffu, which == 0 ? need_od : need_os)) continue;
           const uint32_t ob = which == 0 ? tOd : tOs;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < 2; ++q) {
             uint32_t o[32];
             tc::tmem_ld32(ob + q * 32, o);
             tc::tmem_wait_ld();
@@ -320,10 +337,12 @@ __global__ void __launch_bounds__(kPtThreads, 1)
       }
       const float mem_f = live_s ? 1.f : 0.f;
       const bool write_s = any_member || !zeroed;
-      // quarters of 32 keys: 16 packed columns of P_d (hi, lo) and 4 16-byte chunks of P_s
+      // quarters of 32 keys of this half: 16 packed columns of P_d (hi, lo) and 4 16-byte
+      // chunks of P_s
 #pragma unroll
-      for (int qt = 0; qt < 4; ++qt) {
+      for (int qt = 0; qt < 2; ++qt) {
         uint32_t hi[16], lo[16];
+        const int ch0 = 8 * hf + 4 * qt;  // first 16-byte chunk of these keys in a P_s row
         if (any_far) {  // sparse weights from their own exponentials (before u is overwritten)
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -335,7 +354,7 @@ __global__ void __launch_bounds__(kPtThreads, 1)
           }
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
-            const uint32_t off = tc::sw128_offset(r, qt * 4 + c4);
+            const uint32_t off = tc::sw128_offset(r, ch0 + c4);
             pt_st_shared_v4(sPh + off, hi[4 * c4], hi[4 * c4 + 1], hi[4 * c4 + 2], hi[4 * c4 + 3]);
             pt_st_shared_v4(sPl + off, lo[4 * c4], lo[4 * c4 + 1], lo[4 * c4 + 2], lo[4 * c4 + 3]);
           }
@@ -364,7 +383,7 @@ __global__ void __launch_bounds__(kPtThreads, 1)
           }
 #pragma unroll
           for (int c4 = 0; c4 < 4; ++c4) {
-            const uint32_t off = tc::sw128_offset(r, qt * 4 + c4);
+            const uint32_t off = tc::sw128_offset(r, ch0 + c4);
             pt_st_shared_v4(sPh + off, hi[4 * c4], hi[4 * c4 + 1], hi[4 * c4 + 2], hi[4 * c4 + 3]);
             pt_st_shared_v4(sPl + off, lo[4 * c4], lo[4 * c4 + 1], lo[4 * c4 + 2], lo[4 * c4 + 3]);
           }
@@ -378,30 +397,43 @@ __global__ void __launch_bounds__(kPtThreads, 1)
       tc::fence_before_sync();
       tc::mbar_arrive(bar(kPPFull));
     }
-    // ---- partial records [m_d, l_d, m_s, l_s, O_d[128], O_s[128]] of this split
+    // ---- partial records [m_d, l_d, m_s, l_s, O_d[128], O_s[128]] of this split; each half
+    // writes its 64 columns of O_d and O_s, half 0 the (max, sum) header
     constexpr int kRec = 4 + 2 * 128;
     const bool have_rows = ok && n_tiles > 0 && pt_warp_wait(bar(kPPVDone), (n_tiles - 1) & 1, abort_v, status);
     float4* rec = reinterpret_cast<float4*>(
         part + ((static_cast<size_t>(head) * P + prow0 + r) * nsplit + split) * kRec);
     const bool mine = r < nrows;
     if (have_rows) {
+      // the halves' (l_d, l_s) meet in the P_s buffer, free after the last PV product
+      float2* s_l = reinterpret_cast<float2*>(dsmem + (sPh - tc::saddr(dsmem)));
+      s_l[hf * 128 + r] = make_float2(l_d, l_s);
+      tc::mbar_arrive(bar(kPLx));
+      const bool got = pt_warp_wait(bar(kPLx), 0, abort_v, status);
       tc::fence_after_sync();
-      if (mine) rec[0] = make_float4(m_d, l_d, m_s, l_s);
+      if (got && mine && hf == 0) {
+        const float2 o2 = s_l[128 + r];
+        rec[0] = make_float4(m_d, l_d + o2.x, m_s, l_s + o2.y);
+      }
 #pragma unroll 1
-      for (int q = 0; q < 8; ++q) {
+      for (int q = 0; q < 4; ++q) {
         uint32_t o[32];
-        tc::tmem_ld32((q < 4 ? tOd : tOs) + (q & 3) * 32, o);
+        tc::tmem_ld32((q < 2 ? tOd : tOs) + (q & 1) * 32, o);
         tc::tmem_wait_ld();
-        if (mine) {
+        if (got && mine) {
+          const int base = 1 + (q < 2 ? 0 : 32) + 16 * hf + 8 * (q & 1);  // float4 index in the record
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            rec[1 + q * 8 + i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                             __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+            rec[base + i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                        __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
         }
       }
     } else if (ok && n_tiles == 0 && mine) {
-      rec[0] = make_float4(-kPtInf, 0.f, -kPtInf, 0.f);
-      for (int i = 1; i < kRec / 4; ++i) rec[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (hf == 0) rec[0] = make_float4(-kPtInf, 0.f, -kPtInf, 0.f);
+      for (int i = 0; i < 16; ++i) {
+        rec[1 + 16 * hf + i] = make_float4(0.f, 0.f, 0.f, 0.f);   // O_d columns of this half
+        rec[33 + 16 * hf + i] = make_float4(0.f, 0.f, 0.f, 0.f);  // O_s columns of this half
+      }
     }
   }
   tc::fence_before_sync();
