@@ -466,3 +466,14 @@ def test_host_entry_matches_device_call():
     torch.cuda.current_stream().synchronize()
     spr.check(ws)
     assert torch.equal(o_host, o_dev.cpu())
+
+
+@pytest.mark.parametrize("grid,over", [((1, 10, 10), dict(n_sampled=32, n_probe=8, rank=4)),     # N 100: one group
+                                      ((1, 3, 43), dict(n_sampled=32, n_probe=8, rank=4)),      # N 129: last group 1 token
+                                      ((2, 8, 16), dict(n_sampled=64, n_probe=1, rank=1))])     # one probe row
+def test_edge_shapes(grid, over):
+    """Degenerate shapes of the method: a single key group and query block (N < B), a
+    last group of one token, and a single probe row (the fit's centred design is empty,
+    so M = 0 and beta carries the mean residual); full parity with the oracle."""
+    w = CONFIGS["small"].with_(grid=grid, heads=2)
+    _check_call(w, spr_cfg(w, **over))
