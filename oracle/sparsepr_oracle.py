@@ -297,12 +297,50 @@ def route(block_scores: np.ndarray, k: int) -> np.ndarray:
     return out
 
 
+def route_global(block_scores: np.ndarray, key_sizes: np.ndarray, block_sizes: np.ndarray,
+                 n: int, n_probe: int, density: float) -> list:
+    """Global budget allocation, the other reading of "routing up to a target density"
+    ([abs]): the executed-pair budget floor(rho N^2 - P N) (real sizes, probes counted)
+    is shared by all blocks of the head instead of a uniform k.  Every block keeps its
+    best group (largest fp32 score, ties -> lower group); the other (block, group) pairs
+    follow in descending score order (ties -> lower block, then lower group) and are
+    taken while the cumulative pair count n_b n_g stays within the budget (the longest
+    prefix of that order that fits).  Returns, per block, its groups in ascending order.
+    """
+    sc = np.asarray(block_scores, dtype=np.float32)
+    if np.isnan(sc).any():
+        raise NonFiniteError("NaN block score")
+    gq, g_count = sc.shape
+    budget = math.floor(density * n * n - float(n_probe * n))
+    idx = np.arange(g_count)
+    chosen = [set() for _ in range(gq)]
+    spent = 0
+    best = np.empty(gq, dtype=np.int64)
+    for b in range(gq):
+        best[b] = np.lexsort((idx, -sc[b]))[0]
+        chosen[b].add(int(best[b]))
+        spent += int(block_sizes[b]) * int(key_sizes[best[b]])
+    # candidates: descending score, then block, then group (np.lexsort: last key primary)
+    bb, gg = np.meshgrid(np.arange(gq), idx, indexing="ij")
+    mask = gg != best[:, None]
+    cb, cg = bb[mask], gg[mask]
+    order = np.lexsort((cg, cb, -sc[cb, cg]))
+    for t in order:
+        b, g = int(cb[t]), int(cg[t])
+        cost = int(block_sizes[b]) * int(key_sizes[g])
+        if spent + cost > budget:
+            break
+        spent += cost
+        chosen[b].add(g)
+    return [np.array(sorted(c), dtype=np.int64) for c in chosen]
+
+
 def executed_pairs(routes: np.ndarray, key_sizes: np.ndarray, block_sizes: np.ndarray,
                    n_probe: int, n: int) -> int:
     """Pairs the call evaluates: routed (block, group) tiles at their real sizes plus
     every probe row against all N keys ([abs]: probes are counted)."""
     total = 0
-    for b in range(routes.shape[0]):
+    for b in range(len(routes)):
         total += int(block_sizes[b]) * int(sum(int(key_sizes[g]) for g in routes[b]))
     return total + int(n_probe) * int(n)
 
@@ -319,7 +357,7 @@ def sparse_attention(q, k, v, tau, key_labels, query_labels, routes) -> np.ndarr
     """s_i = softmax over the union of the routed groups' keys of block(i) ([abs])."""
     n, d = q.shape
     out = np.zeros((n, v.shape[1]))
-    for b in range(routes.shape[0]):
+    for b in range(len(routes)):
         rows = np.flatnonzero(query_labels == b)
         if rows.size == 0:
             continue
@@ -487,12 +525,15 @@ def rel_l2_errors(o: np.ndarray, o_dense: np.ndarray, probe_idx: np.ndarray) -> 
 
 def sparsepr_head(q, k, v, *, block, n_sampled, n_probe, density, ridge_lambda, rank,
                   kmeans_iters=4, scale=None, weight_mode="inv_norm", inject=None,
-                  dump=None, partition_mode="response", route_scores="centroid") -> dict:
+                  dump=None, partition_mode="response", route_scores="centroid",
+                  route_budget="uniform") -> dict:
     """One SparsePR call on one (batch, head).  ``inject`` may hold any of
     sample_idx, probe_idx, key_labels, query_labels, routes (e.g. the CUDA path's
     decisions) to run the later steps on them.  ``partition_mode`` "semantic" swaps
     Response-Coupled Partitioning for the semantic baseline partition (the ablation);
-    the result's "S" is then the uncorrected semantic block-sparse output."""
+    the result's "S" is then the uncorrected semantic block-sparse output.
+    ``route_budget`` "global" shares the pair budget across the blocks (route_global)
+    instead of a uniform k; routes are then per-block arrays of different lengths."""
     inject = inject or {}
     n, d = q.shape
     tau = 1.0 / math.sqrt(d) if scale is None or scale <= 0 else float(scale)
@@ -510,11 +551,13 @@ def sparsepr_head(q, k, v, *, block, n_sampled, n_probe, density, ridge_lambda, 
     block_sizes = np.bincount(ql, minlength=g_count)
     kk = route_k(n, block, density, n_probe)
     if "routes" in inject:
-        routes = np.asarray(inject["routes"])
+        routes = inject["routes"]
+        routes = [np.asarray(r)[np.asarray(r) >= 0] for r in routes] if route_budget == "global" else np.asarray(routes)
     else:
         scores = part["block_scores"] if route_scores == "centroid" else routing_scores(
             q, k, tau, kl, ql, g_count, route_scores)
-        routes = route(scores, kk)
+        routes = (route_global(scores, key_sizes, block_sizes, n, n_probe, density) if route_budget == "global"
+                  else route(scores, kk))
     probe_idx = np.asarray(inject["probe_idx"]) if "probe_idx" in inject else midpoint_stride(n, n_probe)
     pairs = executed_pairs(routes, key_sizes, block_sizes, probe_idx.size, n)
     s = sparse_attention(q, k, v, tau, kl, ql, routes)

@@ -535,3 +535,56 @@ def test_routing_scores_bruteforce_and_jensen_bound():
     lse2 = O.routing_scores(q, k2, tau, kl, ql, g, "lse")
     siz2 = O.routing_scores(q, k2, tau, kl, ql, g, "size_corrected")
     assert np.allclose(lse2[:, 2], siz2[:, 2], rtol=1e-6, atol=1e-5)
+
+
+def test_route_global_hand_worked_fixture():
+    fx = json.load(open(os.path.join(GOLDEN, "route_global_hand_worked.json")))
+    sc = np.array(fx["Sc"], dtype=np.float32)
+    ks, bs = np.array(fx["key_sizes"]), np.array(fx["block_sizes"])
+    for case in fx["cases"]:
+        routes = O.route_global(sc, ks, bs, fx["n_tokens"], fx["n_probe"], case["density"])
+        assert [r.tolist() for r in routes] == case["routes"]
+        pairs = sum(int(bs[b]) * int(ks[routes[b]].sum()) for b in range(len(routes)))
+        assert pairs == case["executed_pairs"]
+
+
+def test_route_global_invariants():
+    """Every block keeps its best group; the pairs stay within the budget (unless the
+    kept best groups alone exceed it); the taken pairs precede every left-out pair in
+    (descending score, block, group) order; and the first left-out pair would not fit."""
+    rng = _rng(23)
+    for trial in range(20):
+        gq, g = int(rng.integers(2, 9)), int(rng.integers(2, 9))
+        sc = rng.integers(-3, 4, size=(gq, g)).astype(np.float32)   # many ties
+        ks, bs = rng.integers(0, 6, size=g), rng.integers(1, 6, size=gq)
+        n, probes, rho = int(bs.sum()), int(rng.integers(0, 3)), float(rng.uniform(0.05, 1.2))
+        routes = O.route_global(sc, ks, bs, n, probes, rho)
+        budget = math.floor(rho * n * n - float(probes * n))
+        best = [int(np.lexsort((np.arange(g), -sc[b]))[0]) for b in range(gq)]
+        spent = sum(int(bs[b]) * int(ks[routes[b]].sum()) for b in range(gq))
+        kept = sum(int(bs[b]) * int(ks[best[b]]) for b in range(gq))
+        assert all(best[b] in routes[b].tolist() for b in range(gq))
+        assert spent <= max(budget, kept)
+        key = lambda b, gg: (-float(sc[b, gg]), b, gg)
+        taken = [(b, int(x)) for b in range(gq) for x in routes[b] if int(x) != best[b]]
+        left = [(b, x) for b in range(gq) for x in range(g) if x not in routes[b].tolist()]
+        if taken and left:
+            assert max(key(*t) for t in taken) < min(key(*e) for e in left)
+        if left:
+            first = min(left, key=lambda e: key(*e))
+            assert spent + int(bs[first[0]]) * int(ks[first[1]]) > budget
+
+
+def test_route_global_single_block_is_uniform_topk():
+    """One block and equal group sizes: the global allocation takes the floor(budget /
+    (n_b B)) best groups, the uniform top-k route with that k."""
+    rng = _rng(29)
+    for trial in range(10):
+        g, nb, blk = int(rng.integers(3, 12)), int(rng.integers(2, 6)), int(rng.integers(2, 6))
+        sc = rng.integers(-2, 3, size=(1, g)).astype(np.float32)
+        ks, bs = np.full(g, blk), np.array([nb])
+        n, rho = 10, float(rng.uniform(0.01, 2.0))
+        budget = math.floor(rho * n * n)
+        kk = min(g, max(1, budget // (nb * blk)))
+        got = O.route_global(sc, ks, bs, n, 0, rho)
+        assert got[0].tolist() == O.route(sc, kk)[0].tolist()
