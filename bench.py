@@ -540,28 +540,41 @@ def run_study_probe_budget(args, w):
 
 
 def run_study_routing(args, w):
-    """Error of the three block-routing score readings (centroid, size-corrected,
-    LSE) at the same uniform k, hence the same executed-pair count, with and without
-    the probe-fitted correction."""
-    _, spr = _gpu_modules()
+    """Error of the three block-routing score readings (centroid, size-corrected, LSE)
+    under the two splits of the pair budget (uniform k per block; one budget per head
+    spent on the best pairs), with and without the probe-fitted correction, and the
+    device time of one whole call (the default fused order) for each."""
+    torch, spr = _gpu_modules()
     q, k, v, dense = _study_inputs(args, w)
     bt, h, n, d = q.shape
-    for mode, name in ((spr.ROUTE_CENTROID, "centroid"), (spr.ROUTE_SIZE_CORRECTED, "size-corrected"),
-                       (spr.ROUTE_LSE, "lse")):
-        cfg = spr.SparsePRConfig(block=w.block, n_sampled=w.n_sampled, n_probe=w.n_probe, kmeans_iters=w.kmeans_iters,
-                                 rank=w.rank, density=w.density, ridge_lambda=w.ridge_lambda, route_scores=mode)
-        ws = spr.new_workspace(bt, h, n, d, cfg, q.device)
-        pidx = spr.probe_rows(n, w.n_probe, bt, h, q.device)
-        o, parts = spr.attention(q, k, v, cfg, ws=ws, return_parts=True, fused=False)
-        m, p = _err_summary(spr.row_errors(o, dense, pidx))
-        mu, pu = _err_summary(spr.row_errors(parts["S"], dense, pidx))
-        spr.check(ws)
-        print(json.dumps({"study": "routing", "scores": name, "workload": config_block(w, args)["workload"],
-                          "k": parts["k"], "density": float(parts["executed_pairs"].double().sum()) /
-                          (float(n) ** 2 * h * bt), "mean_rel_l2": m, "p99_rel_l2": p,
-                          "uncorrected_mean_rel_l2": mu, "uncorrected_p99_rel_l2": pu, "seed": args.seed}),
-              flush=True)
-        del ws
+    for budget, bname in ((spr.BUDGET_UNIFORM, "uniform"), (spr.BUDGET_GLOBAL, "global")):
+        for mode, name in ((spr.ROUTE_CENTROID, "centroid"), (spr.ROUTE_SIZE_CORRECTED, "size-corrected"),
+                           (spr.ROUTE_LSE, "lse")):
+            cfg = spr.SparsePRConfig(block=w.block, n_sampled=w.n_sampled, n_probe=w.n_probe,
+                                     kmeans_iters=w.kmeans_iters, rank=w.rank, density=w.density,
+                                     ridge_lambda=w.ridge_lambda, route_scores=mode, route_budget=budget)
+            ws = spr.new_workspace(bt, h, n, d, cfg, q.device)
+            pidx = spr.probe_rows(n, w.n_probe, bt, h, q.device)
+            o, parts = spr.attention(q, k, v, cfg, ws=ws, return_parts=True, fused=False)
+            m, p = _err_summary(spr.row_errors(o, dense, pidx))
+            mu, pu = _err_summary(spr.row_errors(parts["S"], dense, pidx))
+            spr.check(ws)
+            del o, parts
+            spr.attention(q, k, v, cfg, ws=ws)  # warm
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            spr.attention(q, k, v, cfg, ws=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            spr.check(ws)
+            pairs = spr.route(spr.partition(q, k, cfg, ws), n, cfg, ws)[2]
+            print(json.dumps({"study": "routing", "scores": name, "budget": bname,
+                              "workload": config_block(w, args)["workload"],
+                              "density": float(pairs.double().sum()) / (float(n) ** 2 * h * bt),
+                              "mean_rel_l2": m, "p99_rel_l2": p, "uncorrected_mean_rel_l2": mu,
+                              "uncorrected_p99_rel_l2": pu, "call_ms": e0.elapsed_time(e1), "seed": args.seed}),
+                  flush=True)
+            del ws
 
 
 def main():

@@ -341,13 +341,28 @@ int sparsepr_route(const float* block_scores, const int32_t* key_gsize, const in
   if (!block_scores || !key_gsize || !qblock_size || !route || !ws)
     return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
   if (p->n_probe < 0 || p->n_probe > N) return fail(SPARSEPR_ERR_INVALID_ARG, "n_probe must be in [0, N]");
+  if (p->route_budget != SPARSEPR_BUDGET_UNIFORM && p->route_budget != SPARSEPR_BUDGET_GLOBAL)
+    return fail(SPARSEPR_ERR_INVALID_ARG, "unknown route_budget %d", p->route_budget);
+  if (p->route_budget == SPARSEPR_BUDGET_GLOBAL && spr::ceil_div(N, p->block) > 8192)
+    return fail(SPARSEPR_ERR_UNSUPPORTED, "more than 8192 groups per head under the global budget is not built");
   const int G = spr::ceil_div(N, p->block);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const long long probe_pairs = static_cast<long long>(p->n_probe) * N;
+  if (p->route_budget == SPARSEPR_BUDGET_GLOBAL) {
+    // floor(rho N^2 - P N) in IEEE double, in this order
+    const double budget = std::floor(p->density * static_cast<double>(N) * static_cast<double>(N) -
+                                     static_cast<double>(probe_pairs));
+    if (k_out) *k_out = G;
+    SPR_CUDA(spr::launch_route_global(block_scores, Bt * H, G, G, static_cast<long long>(budget), route, key_gsize,
+                                      qblock_size, reinterpret_cast<long long*>(executed_pairs), probe_pairs,
+                                      &header(ws)->status, st),
+             "route");
+    return SPARSEPR_OK;
+  }
   const int k = sparsepr_route_k(N, p->block, p->density, p->n_probe);
   if (k_out) *k_out = k;
   SPR_CUDA(spr::launch_route(block_scores, Bt * H, G, G, k, route, key_gsize, qblock_size,
-                             reinterpret_cast<long long*>(executed_pairs),
-                             static_cast<long long>(p->n_probe) * N, &header(ws)->status,
-                             reinterpret_cast<cudaStream_t>(stream)),
+                             reinterpret_cast<long long*>(executed_pairs), probe_pairs, &header(ws)->status, st),
            "route");
   return SPARSEPR_OK;
 }

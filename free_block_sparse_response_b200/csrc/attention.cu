@@ -70,8 +70,8 @@ __global__ void __launch_bounds__(BQ * 2, 1)
   cp_async_commit();
 
   constexpr int kCpg = BQ / kChunk;  // chunks per key group
-  const int n_chunks = k * kCpg;
   const int* my_route = DENSE ? nullptr : route + (goff + b) * k;
+  const int n_chunks = (DENSE ? k : routed_len(my_route, k)) * kCpg;
 
   auto chunk_group = [&](int t) { return DENSE ? t / kCpg : __ldg(my_route + t / kCpg); };
   auto chunk_valid = [&](int t) {
@@ -264,6 +264,7 @@ __global__ void __launch_bounds__(128)
       const int* rt = route + (goff + blk) * k;
       for (int j = 0; j < k; ++j) {
         const int g = rt[j];
+        if (g < 0) break;  // -1 padding
         if (g >= g0 && g < g1) bits |= 1u << (g - g0);
       }
     }
@@ -521,7 +522,7 @@ __global__ void attn_f32_kernel(const float* __restrict__ Q, const float* __rest
     const int tok = DENSE ? b * block + r : query_perm[(goff + b) * block + r];
     RowState<D> st;
     st.init(Q + hoff + static_cast<size_t>(tok) * D, lane);
-    const int ng = DENSE ? G : k;
+    const int ng = DENSE ? G : routed_len(route + (goff + b) * k, k);
     for (int x = 0; x < ng; ++x) {
       const int g = DENSE ? x : route[(goff + b) * k + x];
       const int gs = DENSE ? min(block, N - g * block) : key_gsize[goff + g];
@@ -557,7 +558,8 @@ __global__ void probe_f32_kernel(const float* __restrict__ Q, const float* __res
     dense.add_key(K + hoff + static_cast<size_t>(j) * D, V + hoff + static_cast<size_t>(j) * D, lane,
                   scale_log2);
   const int blk = qblock_of_token[static_cast<size_t>(head) * N + tok];
-  for (int x = 0; x < k; ++x) {
+  const int nr = routed_len(route + (goff + blk) * k, k);
+  for (int x = 0; x < nr; ++x) {
     const int g = route[(goff + blk) * k + x];
     const int gs = key_gsize[goff + g];
     for (int j = 0; j < gs; ++j) {

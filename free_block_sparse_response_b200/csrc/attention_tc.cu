@@ -174,8 +174,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const size_t goff = static_cast<size_t>(head) * G;
   const int nq = DENSE ? min(128, N - b * 128) : qblock_size[goff + b];
   const int* qperm = DENSE ? nullptr : query_perm + (goff + b) * 128;
-  const int n_tiles = DENSE ? G : k;
   const int* my_route = DENSE ? nullptr : route + (goff + b) * k;
+  const int n_tiles = DENSE ? G : routed_len(my_route, k);
   // key group of routed tile j and its number of members
   auto group_of = [&](int j) { return DENSE ? j : __ldg(my_route + j); };
   auto size_of = [&](int g) { return DENSE ? min(128, N - g * 128) : __ldg(key_gsize + goff + g); };

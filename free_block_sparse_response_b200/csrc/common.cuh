@@ -126,6 +126,21 @@ __device__ __forceinline__ float float_from_order_key(uint32_t k) {
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Number of routed groups in a route row of capacity k: rows hold ascending key groups,
+// then -1 padding when the pair budget is allocated per head rather than per block.
+__device__ __forceinline__ int routed_len(const int* __restrict__ row, int k) {
+  if (k <= 0 || __ldg(row + k - 1) >= 0) return k;
+  int lo = 0, hi = k - 1;  // row[hi] < 0; the first negative entry lies in [lo, hi]
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(row + mid) < 0)
+      hi = mid;
+    else
+      lo = mid + 1;
+  }
+  return lo;
+}
+
 // Host-side count of kernels this library has enqueued (all devices, all threads).
 void note_launches(int n);
 inline cudaError_t counted(cudaError_t e, int n) {

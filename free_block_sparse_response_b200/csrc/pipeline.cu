@@ -36,7 +36,10 @@ bool call_layout(int dtype, int32_t Bt, int32_t H, int32_t N, int32_t d, const s
   const size_t stage = sparsepr_workspace_size(Bt, H, N, d, p);
   if (stage == 0) return false;
   const size_t heads = static_cast<size_t>(Bt) * H, G = static_cast<size_t>(sparsepr_num_groups(N, p->block));
-  const size_t k = static_cast<size_t>(sparsepr_route_k(N, p->block, p->density, p->n_probe));
+  // route row capacity: k (uniform budget) or G (global budget, rows padded with -1)
+  const size_t k = p->route_budget == SPARSEPR_BUDGET_GLOBAL
+                       ? G
+                       : static_cast<size_t>(sparsepr_route_k(N, p->block, p->density, p->n_probe));
   const size_t P = static_cast<size_t>(p->n_probe), D = static_cast<size_t>(d);
   size_t off = 0;
   auto take = [&](size_t bytes) {

@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(kPtThreads, 1)
     const int qb = __ldg(qblock_of_token + static_cast<size_t>(head) * N + tok);
     uint64_t member_bits = 0;  // bit (g - g0): group g routed to this row's query block
     {
-      // the route row is sorted ascending: eight independent loads per step
+      // the route row is sorted ascending (then -1 padding): eight independent loads per step
       const int* rt = route + (static_cast<size_t>(head) * G + qb) * k;
       for (int j0 = 0; j0 < k; j0 += 8) {
         int gg[8];
@@ -231,6 +231,7 @@ __global__ void __launch_bounds__(kPtThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           if (gg[i] >= g0 && gg[i] < g1) member_bits |= 1ull << (gg[i] - g0);
+        if (gg[7] < 0 || gg[7] >= g1) break;  // -1 padding, or past this split's groups
       }
     }
     const int* gsz = key_gsize + static_cast<size_t>(head) * G;

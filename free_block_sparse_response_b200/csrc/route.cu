@@ -106,6 +106,152 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// Global budget allocation (the other reading of routing up to a target density): the
+// pair budget of a head is shared by its blocks.  Every block keeps its best group; the
+// other (block, group) pairs, ordered by descending score, then block, then group, are
+// taken while the cumulative pairs n_b n_g stay within the budget.  One CTA per head:
+// (1) the best group of every block; (2) a radix select, weighted by the pair cost, of
+// the first candidate that no longer fits (64-bit keys: inverted score order key, then
+// b G + g); (3) every block's groups in ascending order, -1 after them, and the pairs.
+constexpr int kRgThreads = 1024;
+
+__global__ void __launch_bounds__(kRgThreads)
+    route_global_kernel(const float* __restrict__ sc, int Gq, int G, long long budget, int* __restrict__ route,
+                        const int* __restrict__ key_gsize, const int* __restrict__ qblock_size,
+                        unsigned long long* __restrict__ pairs, int* __restrict__ status) {
+  extern __shared__ int s_best[];  // [Gq] best group per block
+  __shared__ unsigned long long hist[256];
+  __shared__ long long s_spent, s_below;
+  __shared__ unsigned long long s_prefix;
+  __shared__ int s_cross, s_digit;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = kRgThreads / 32;
+  const int head = blockIdx.x;
+  const float* scs = sc + static_cast<size_t>(head) * Gq * G;
+  const int* ks = key_gsize + static_cast<size_t>(head) * G;
+  const int* bs = qblock_size + static_cast<size_t>(head) * Gq;
+  if (tid == 0) {
+    s_spent = 0;
+    s_below = 0;
+    s_prefix = 0;
+    s_cross = 0;
+  }
+  __syncthreads();
+  // (1) best group of every block (smallest route key), its pairs
+  bool saw_nan = false;
+  for (int b = warp; b < Gq; b += nwarps) {
+    unsigned long long best = ~0ull;
+    for (int g = lane; g < G; g += 32) {
+      const float v = scs[static_cast<size_t>(b) * G + g];
+      saw_nan |= (v != v);
+      const unsigned long long key = route_key(v, g);
+      best = key < best ? key : best;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long y = __shfl_xor_sync(0xffffffffu, best, o);
+      best = y < best ? y : best;
+    }
+    if (lane == 0) {
+      const int g = static_cast<int>(best & 0xffffffffu);
+      s_best[b] = g;
+      atomicAdd(reinterpret_cast<unsigned long long*>(&s_spent),
+                static_cast<unsigned long long>(static_cast<long long>(bs[b]) * ks[g]));
+    }
+  }
+  __syncthreads();
+  const long long rem = budget - s_spent;  // pairs left for the other candidates
+  // (2) weighted radix select: the first candidate (ascending key) whose cumulative cost
+  // exceeds rem; every candidate before it is taken.  s_cross = 0: all candidates fit.
+  auto ckey = [&](int b, int g, float v) {
+    const uint32_t hi = (v != v) ? 0xffffffffu : ~float_order_key(v);
+    return (static_cast<unsigned long long>(hi) << 32) | static_cast<uint32_t>(b * G + g);
+  };
+  const long long cand = static_cast<long long>(Gq) * G;
+  if (rem >= 0) {
+    for (int shift = 56; shift >= 0; shift -= 8) {
+      for (int x = tid; x < 256; x += kRgThreads) hist[x] = 0;
+      __syncthreads();
+      const unsigned long long hmask = shift == 56 ? 0ull : (~0ull << (shift + 8));
+      const unsigned long long prefix = s_prefix;
+      for (long long x0 = 0; x0 < cand; x0 += kRgThreads) {
+        const long long x = x0 + tid;
+        int digit = -1, cost = 0;
+        if (x < cand) {
+          const int b = static_cast<int>(x / G), g = static_cast<int>(x - static_cast<long long>(b) * G);
+          if (g != s_best[b]) {
+            const unsigned long long key = ckey(b, g, scs[x]);
+            if ((key & hmask) == prefix) {
+              digit = static_cast<int>((key >> shift) & 255u);
+              cost = bs[b] * ks[g];
+            }
+          }
+        }
+        // lanes with the same digit add their costs once (a leader per digit)
+        const unsigned int peers = __match_any_sync(0xffffffffu, digit);
+        const int sum = __reduce_add_sync(peers, cost);
+        if (digit >= 0 && lane == __ffs(peers) - 1 && sum > 0)
+          atomicAdd(&hist[digit], static_cast<unsigned long long>(sum));
+      }
+      __syncthreads();
+      if (tid == 0) {
+        long long below = s_below;
+        int d = 0;
+        for (; d < 256; ++d) {
+          const long long hcost = static_cast<long long>(hist[d]);
+          if (below + hcost > rem) break;
+          below += hcost;
+        }
+        if (d == 256) {
+          // everything under this prefix fits (only possible at the top level: below it,
+          // the prefix was chosen because its bin crosses)
+          s_digit = -1;
+        } else {
+          s_digit = d;
+          s_below = below;
+          s_prefix = prefix | (static_cast<unsigned long long>(d) << shift);
+          s_cross = 1;
+        }
+      }
+      __syncthreads();
+      if (s_digit < 0) break;
+    }
+  }
+  const bool cross = s_cross != 0;
+  const unsigned long long kstar = s_prefix;  // the first candidate that does not fit
+  // (3) routes: every block's kept best group and the candidates before kstar
+  for (int b = warp; b < Gq; b += nwarps) {
+    int* out = route + (static_cast<size_t>(head) * Gq + b) * G;
+    int written = 0;
+    long long member_sum = 0;
+    for (int g0 = 0; g0 < G; g0 += 32) {
+      const int g = g0 + lane;
+      bool sel = false;
+      if (g < G) {
+        if (g == s_best[b]) {
+          sel = true;
+        } else if (rem >= 0) {
+          sel = !cross || ckey(b, g, scs[static_cast<size_t>(b) * G + g]) < kstar;
+        }
+      }
+      const unsigned int ball = __ballot_sync(0xffffffffu, sel);
+      const int slot = written + __popc(ball & ((1u << lane) - 1u));
+      if (sel) {
+        out[slot] = g;
+        member_sum += ks[g];
+      }
+      written += __popc(ball);
+    }
+    for (int sidx = written + lane; sidx < G; sidx += 32) out[sidx] = -1;
+    if (pairs != nullptr) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) member_sum += __shfl_xor_sync(0xffffffffu, member_sum, o);
+      if (lane == 0) atomicAdd(pairs + head, static_cast<unsigned long long>(static_cast<long long>(bs[b]) * member_sum));
+    }
+  }
+  saw_nan = __syncthreads_or(saw_nan);
+  if (tid == 0 && saw_nan) record_error(status, kErrNonFinite);
+}
+
 // Sc[b][g] += log n_g (size-corrected scores).
 __global__ void size_correct_kernel(float* __restrict__ sc, const int* __restrict__ key_gsize, int Gq, int G) {
   const int head = blockIdx.y;
@@ -170,6 +316,20 @@ cudaError_t launch_route(const float* sc, int heads, int Gq, int G, int k, int* 
   }
   route_topk_kernel<<<dim3(ceil_div(Gq, 8), heads), 256, 0, st>>>(sc, Gq, G, k, route, key_gsize, qblock_size,
                                                                    up, status);
+  return counted(cudaGetLastError(), up != nullptr ? 2 : 1);
+}
+
+cudaError_t launch_route_global(const float* sc, int heads, int Gq, int G, long long budget, int* route,
+                                const int* key_gsize, const int* qblock_size, long long* pairs, long long probe_pairs,
+                                int* status, cudaStream_t st) {
+  unsigned long long* up = reinterpret_cast<unsigned long long*>(pairs);
+  if (up != nullptr) {
+    pairs_init_kernel<<<ceil_div(heads, 256), 256, 0, st>>>(up, heads, probe_pairs);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  route_global_kernel<<<heads, kRgThreads, sizeof(int) * Gq, st>>>(sc, Gq, G, budget, route, key_gsize,
+                                                                     qblock_size, up, status);
   return counted(cudaGetLastError(), up != nullptr ? 2 : 1);
 }
 

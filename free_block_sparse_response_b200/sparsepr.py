@@ -20,6 +20,7 @@ BF16, F32 = 0, 1
 WEIGHT_INV_NORM, WEIGHT_UNIFORM = 0, 1
 PARTITION_RESPONSE, PARTITION_SEMANTIC = 0, 1
 ROUTE_CENTROID, ROUTE_SIZE_CORRECTED, ROUTE_LSE = 0, 1, 2
+BUDGET_UNIFORM, BUDGET_GLOBAL = 0, 1
 _DTYPE_CODE = {torch.bfloat16: BF16, torch.float32: F32}
 
 EXPORTED_SYMBOLS = (
@@ -44,15 +45,18 @@ class _CParams(ctypes.Structure):
     _fields_ = [("block", ctypes.c_int32), ("n_sampled", ctypes.c_int32), ("n_probe", ctypes.c_int32),
                 ("kmeans_iters", ctypes.c_int32), ("rank", ctypes.c_int32), ("weight_mode", ctypes.c_int32),
                 ("density", ctypes.c_double), ("ridge_lambda", ctypes.c_double), ("scale", ctypes.c_float),
-                ("partition_mode", ctypes.c_int32), ("route_scores", ctypes.c_int32)]
+                ("partition_mode", ctypes.c_int32), ("route_scores", ctypes.c_int32),
+                ("route_budget", ctypes.c_int32)]
 
 
 @dataclasses.dataclass(frozen=True)
 class SparsePRConfig:
     """Parameters of one call: block B, sampled queries S, probe rows P, k-means
     iterations T, subspace rank r, probe weighting, density rho, ridge lambda, scale,
-    the partition rule (PARTITION_RESPONSE, or the PARTITION_SEMANTIC baseline) and the
-    block-routing score (ROUTE_CENTROID, ROUTE_SIZE_CORRECTED or ROUTE_LSE)."""
+    the partition rule (PARTITION_RESPONSE, or the PARTITION_SEMANTIC baseline), the
+    block-routing score (ROUTE_CENTROID, ROUTE_SIZE_CORRECTED or ROUTE_LSE) and the split
+    of the pair budget (BUDGET_UNIFORM: k groups per block; BUDGET_GLOBAL: one budget
+    per head, spent on the best pairs)."""
     block: int = 128
     n_sampled: int = 512
     n_probe: int = 256
@@ -64,11 +68,12 @@ class SparsePRConfig:
     scale: float = 0.0
     partition_mode: int = 0
     route_scores: int = 0
+    route_budget: int = 0
 
     def c(self) -> _CParams:
         return _CParams(self.block, self.n_sampled, self.n_probe, self.kmeans_iters, self.rank,
                         self.weight_mode, self.density, self.ridge_lambda, self.scale, self.partition_mode,
-                        self.route_scores)
+                        self.route_scores, self.route_budget)
 
 
 _LIB = None
@@ -227,9 +232,11 @@ def partition(q, k, cfg: SparsePRConfig, ws: torch.Tensor, sample_idx: Optional[
 
 
 def route(part: Partition, n: int, cfg: SparsePRConfig, ws: torch.Tensor):
-    """Returns (route [Bt,H,G,k] int32, k, executed_pairs [Bt,H] int64)."""
+    """Returns (route [Bt,H,G,k] int32, k, executed_pairs [Bt,H] int64); under the global
+    budget k = G and each row ends with -1 after its groups."""
     bt, h, g, _ = part.block_scores.shape
-    kk = route_k(n, cfg.block, cfg.density, cfg.n_probe)
+    # row capacity: k groups per block, or G (rows padded with -1) under the global budget
+    kk = g if cfg.route_budget == BUDGET_GLOBAL else route_k(n, cfg.block, cfg.density, cfg.n_probe)
     rt = torch.empty(bt, h, g, kk, dtype=torch.int32, device=ws.device)
     pairs = torch.empty(bt, h, dtype=torch.int64, device=ws.device)
     k_out = _i32(0)

@@ -89,6 +89,14 @@ enum { SPARSEPR_PARTITION_RESPONSE = 0, SPARSEPR_PARTITION_SEMANTIC = 1 };
  * comparison covers. */
 enum { SPARSEPR_ROUTE_CENTROID = 0, SPARSEPR_ROUTE_SIZE_CORRECTED = 1, SPARSEPR_ROUTE_LSE = 2 };
 
+/* How the executed-pair budget floor(rho*N*N - P*N) is spent (SparsePR abstract: routing
+ * "up to a target density" names the budget, not its split).  UNIFORM: every query block
+ * takes the same number k of key groups (the plain reading).  GLOBAL: the head's budget
+ * is shared by its blocks: every block keeps its best group, then the remaining
+ * (block, group) pairs are taken in descending score order (ties to the lower block,
+ * then the lower group) while the cumulative n_b * n_g stays within the budget. */
+enum { SPARSEPR_BUDGET_UNIFORM = 0, SPARSEPR_BUDGET_GLOBAL = 1 };
+
 typedef struct sparsepr_params {
   int32_t block;        /* B: query-block and key-group capacity (64 or 128)            */
   int32_t n_sampled;    /* S: sampled queries that define key response profiles        */
@@ -101,6 +109,7 @@ typedef struct sparsepr_params {
   float scale;          /* softmax scale tau; <= 0 selects 1/sqrt(d)                    */
   int32_t partition_mode; /* SPARSEPR_PARTITION_*                                        */
   int32_t route_scores;   /* SPARSEPR_ROUTE_*: what block_scores hold                    */
+  int32_t route_budget;   /* SPARSEPR_BUDGET_*: uniform k per block or one budget per head */
 } sparsepr_params;
 
 /* Number of groups G = Gq = ceil(N / B): capacity-B groups that cover all N tokens. */
@@ -146,9 +155,12 @@ SPARSEPR_API int sparsepr_partition(const void* Q, const void* K, int dtype, int
                        int32_t* query_perm, int32_t* qblock_size, float* block_scores,
                        void* ws, sparsepr_stream_t stream);
 
-/* (b) Centroid routing.  For every query block: the k key groups with the largest
- * block score (ties to the lower group index), written in ascending group order, with
- * k = sparsepr_route_k(N, B, density, P) (also returned in *k_out, host memory).
+/* (b) Centroid routing.  UNIFORM budget: for every query block, the k key groups with
+ * the largest block score (ties to the lower group index), written in ascending group
+ * order, with k = sparsepr_route_k(N, B, density, P).  GLOBAL budget: the groups that
+ * the head-wide allocation (SPARSEPR_BUDGET_GLOBAL) gives each block, in ascending
+ * order, then -1 up to k = G.  The row capacity k is returned in *k_out (host memory);
+ * the attention and probe calls take it and stop at the first -1.
  *   route          [Bt,H,Gq,k] int32
  *   executed_pairs [Bt,H] int64 = sum_b qblock_size[b] * sum_{g in route(b)} key_gsize[g]
  *                  + P*N: every evaluated (query, key) pair, probe rows counted.

@@ -69,6 +69,11 @@ def test_argument_errors_return_codes_without_launching(L):
                               fake, fake, None)
     assert rc == spr.ERR_INVALID_ARG
     assert b"partition_mode" in L.sparsepr_last_error()
+    bad = spr.SparsePRConfig(route_budget=5).c()
+    k_out = ctypes.c_int32(0)
+    rc = L.sparsepr_route(fake, fake, fake, 1, 1, 1024, ctypes.byref(bad), fake, ctypes.byref(k_out), None, fake, None)
+    assert rc == spr.ERR_INVALID_ARG
+    assert b"route_budget" in L.sparsepr_last_error()
 
 
 def test_params_struct_layout():
@@ -77,6 +82,7 @@ def test_params_struct_layout():
     assert spr.sparsepr._CParams.scale.offset == 40
     assert spr.sparsepr._CParams.partition_mode.offset == 44
     assert spr.sparsepr._CParams.route_scores.offset == 48
+    assert spr.sparsepr._CParams.route_budget.offset == 52
 
 
 def test_python_wrappers_refuse_cpu_tensors():

@@ -121,6 +121,44 @@ def test_topk_bit_exact_with_ties(gq, g, k):
         assert np.array_equal(gpu[h], O.route(sc[h], k))
 
 
+def _route_rows(rt_row):
+    """Groups of one route row: entries before the first -1 (the rest must be -1)."""
+    rt_row = np.asarray(rt_row)
+    neg = np.flatnonzero(rt_row < 0)
+    n_r = int(neg[0]) if neg.size else rt_row.size
+    assert (rt_row[n_r:] == -1).all()
+    return rt_row[:n_r]
+
+
+@pytest.mark.parametrize("gq,block,density,levels", [(16, 128, 0.3, 5), (64, 128, 0.05, 3), (591, 128, 0.22, 40),
+                                                     (40, 64, 1.0, 4), (100, 64, 0.004, 7), (250, 128, 0.1, 1e9)])
+def test_route_global_bit_exact(gq, block, density, levels):
+    """Global budget allocation on injected fp32 scores with ties (and -0.0 / +0.0), random
+    block and group sizes: routes and executed pairs equal the oracle's exactly, including
+    budgets below the mandatory best groups (0.004), budgets that take everything (1.0)
+    and scores without ties (levels 1e9)."""
+    rng = np.random.default_rng(gq + int(1000 * density))
+    heads, n = 2, gq * block - 3
+    lv = int(min(levels, 1 << 20))
+    sc = (rng.integers(-lv, lv, size=(heads, gq, gq)) / 4).astype(np.float32)
+    sc[0, 0, :4] = [0.0, -0.0, 0.0, -0.0]
+    ks = rng.integers(1, block + 1, size=(heads, gq)).astype(np.int32)
+    bs = rng.integers(1, block + 1, size=(heads, gq)).astype(np.int32)
+    part = spr.Partition(None, torch.from_numpy(ks).view(1, heads, gq).cuda(), None,
+                         torch.from_numpy(bs).view(1, heads, gq).cuda(), torch.from_numpy(sc).view(1, heads, gq, gq).cuda())
+    cfg = spr.SparsePRConfig(block=block, n_probe=17, density=density, route_budget=spr.BUDGET_GLOBAL)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    rt, kk, pairs = spr.route(part, n, cfg, ws)
+    spr.check(ws)
+    assert kk == gq
+    rt, pairs = rt.cpu().numpy(), pairs.cpu().numpy()
+    for h in range(heads):
+        want = O.route_global(sc[h], ks[h], bs[h], n, 17, density)
+        for b in range(gq):
+            assert np.array_equal(_route_rows(rt[0, h, b]), want[b]), f"head {h} block {b}"
+        assert int(pairs[0, h]) == O.executed_pairs(want, ks[h], bs[h], 17, n)
+
+
 def test_nan_scores_are_reported():
     sc = np.zeros((1, 4, 8), dtype=np.float32)
     sc[0, 1, 2] = np.nan
@@ -438,19 +476,44 @@ def test_long_config_sampled_rows():
     _full_size_sampled_rows(w, 202, (0, w.heads - 1))
 
 
+def test_global_budget_call_parity():
+    """The whole call under the global pair budget: the routes are the oracle's global
+    allocation of the GPU's own block scores, the executed pairs stay within
+    floor(rho N^2) whenever the best groups fit, and the outputs match the oracle run on
+    the GPU's decisions (variable-length route rows in the attention and probe kernels)."""
+    w = CONFIGS["small"]
+    cfg = spr_cfg(w, route_budget=spr.BUDGET_GLOBAL)
+    _, parts = _check_call(w, cfg, heads=2)
+    n = w.n_tokens
+    part = parts["partition"]
+    rt = parts["route"].cpu().numpy()
+    lens = []
+    for h in range(2):
+        sc = part.block_scores[0, h].cpu().numpy()
+        ks, bs = part.key_gsize[0, h].cpu().numpy(), part.qblock_size[0, h].cpu().numpy()
+        want = O.route_global(sc, ks, bs, n, cfg.n_probe, cfg.density)
+        for b in range(len(want)):
+            got = _route_rows(rt[0, h, b])
+            assert np.array_equal(got, want[b])
+            lens.append(got.size)
+        assert int(parts["executed_pairs"][0, h]) <= math.floor(cfg.density * n * n)
+    assert min(lens) < max(lens), "the global allocation should give blocks different group counts here"
+
+
 @pytest.mark.parametrize("cfg_name,heads", [("small", 3), ("tiny", None)])
 def test_one_call_entry_matches_stage_pipeline(cfg_name, heads):
     """sparsepr_attention (every stage behind one native entry, intermediates in its own
     workspace) gives the stage pipeline's output bit for bit: the fused bf16 order and the
-    unfused fp32 order."""
+    unfused fp32 order, under both pair budgets."""
     w = CONFIGS[cfg_name]
-    cfg = spr_cfg(w)
     q, k, v = (t.cuda() for t in make_inputs(w, 5, heads=heads))
-    o_stages = spr.attention(q, k, v, cfg)
-    ws = spr.call_workspace(q, cfg)
-    o_call = spr.attention_call(q, k, v, cfg, ws=ws)
-    spr.check(ws)
-    assert torch.equal(o_call, o_stages)
+    for budget in (spr.BUDGET_UNIFORM, spr.BUDGET_GLOBAL):
+        cfg = spr_cfg(w, route_budget=budget)
+        o_stages = spr.attention(q, k, v, cfg)
+        ws = spr.call_workspace(q, cfg)
+        o_call = spr.attention_call(q, k, v, cfg, ws=ws)
+        spr.check(ws)
+        assert torch.equal(o_call, o_stages)
 
 
 def test_host_entry_matches_device_call():
