@@ -71,6 +71,7 @@ def oracle_on_gpu_decisions(q, k, v, parts, h, cfg, n):
     return O.sparsepr_head(*(t[0, h].double().numpy() for t in (q, k, v)), block=cfg.block,
                            n_sampled=cfg.n_sampled, n_probe=cfg.n_probe, density=cfg.density,
                            ridge_lambda=cfg.ridge_lambda, rank=cfg.rank, kmeans_iters=cfg.kmeans_iters,
+                           route_budget="global" if cfg.route_budget == spr.BUDGET_GLOBAL else "uniform",
                            inject={"key_labels": kl, "query_labels": ql,
                                    "routes": parts["route"][0, h].cpu().numpy(),
                                    "probe_idx": parts["probe_idx"][0, h].cpu().numpy()})
