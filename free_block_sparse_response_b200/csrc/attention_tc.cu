@@ -116,7 +116,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 
 // FUSED (sparse only): O = S + S M^T + beta is formed in the epilogue and written as
 // bf16 to out_bf16; S itself never leaves the SM.  Otherwise S (fp32) goes to out.
-template <bool DENSE, bool FUSED>
+template <bool DENSE, bool FUSED, bool VARLEN>
 __global__ void __launch_bounds__(kTcThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmM, int N, int G,
@@ -175,7 +175,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int nq = DENSE ? min(128, N - b * 128) : qblock_size[goff + b];
   const int* qperm = DENSE ? nullptr : query_perm + (goff + b) * 128;
   const int* my_route = DENSE ? nullptr : route + (goff + b) * k;
-  const int n_tiles = DENSE ? G : routed_len(my_route, k);
+  // VARLEN: route rows of capacity k = G that end with -1 (global pair budget); otherwise
+  // every row holds exactly k groups and the count stays a kernel parameter
+  const int n_tiles = DENSE ? G : VARLEN ? routed_len(my_route, k) : k;
   // key group of routed tile j and its number of members
   auto group_of = [&](int j) { return DENSE ? j : __ldg(my_route + j); };
   auto size_of = [&](int g) { return DENSE ? min(128, N - g * 128) : __ldg(key_gsize + goff + g); };
@@ -644,7 +646,10 @@ cudaError_t launch_attention_tc(const AttnArgs& a, bool dense, int* status, cuda
   if (smem > 227 * 1024) return cudaErrorInvalidValue;
   const bool fused = !dense && a.m_hilo != nullptr;
   if (fused && (a.beta == nullptr || a.out_bf16 == nullptr)) return cudaErrorInvalidValue;
-  auto kern = dense ? attn_tc_kernel<true, false> : fused ? attn_tc_kernel<false, true> : attn_tc_kernel<false, false>;
+  const bool varlen = !dense && a.k == a.G;
+  auto kern = dense    ? attn_tc_kernel<true, false, false>
+              : fused  ? (varlen ? attn_tc_kernel<false, true, true> : attn_tc_kernel<false, true, false>)
+                       : (varlen ? attn_tc_kernel<false, false, true> : attn_tc_kernel<false, false, false>);
   // The register re-split must fit in what the block is launched with, or the
   // setmaxnreg.inc of the softmax warpgroups would never be granted.
   cudaFuncAttributes fa;

@@ -110,127 +110,205 @@ __global__ void __launch_bounds__(256)
 // pair budget of a head is shared by its blocks.  Every block keeps its best group; the
 // other (block, group) pairs, ordered by descending score, then block, then group, are
 // taken while the cumulative pairs n_b n_g stay within the budget.  One CTA per head:
-// (1) the best group of every block; (2) a radix select, weighted by the pair cost, of
-// the first candidate that no longer fits (64-bit keys: inverted score order key, then
-// b G + g); (3) every block's groups in ascending order, -1 after them, and the pairs.
+//   pass 0   best group of every block (warp per block row), and the cost histogram of
+//            the top 8 bits of every pair's score key (the best pairs taken out again);
+//   pass 1-3 the next 8 bits among the pairs whose higher bits match the crossing bin:
+//            after them the score key T of the first pair that no longer fits is known;
+//   tie pass the pairs with score key T in (block, group) order, a block-wide prefix sum
+//            of their costs: the crossing pair itself;
+//   emit     every block's best group and the pairs before the crossing one, ascending,
+//            then -1, and the executed pairs.
+// Histograms are per warp (no atomics across warps; lanes with the same digit add their
+// costs once, through a warp match and reduction), summed per bin between passes.
 constexpr int kRgThreads = 1024;
+constexpr int kRgWarps = kRgThreads / 32;
+
+__device__ __forceinline__ uint32_t score_hi(float v) { return (v != v) ? 0xffffffffu : ~float_order_key(v); }
+
+__device__ __forceinline__ void warp_hist_add(unsigned long long* hw, int digit, int cost) {
+  const unsigned int peers = __match_any_sync(0xffffffffu, digit);
+  const int sum = __reduce_add_sync(peers, cost);
+  if (digit >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) hw[digit] += static_cast<unsigned long long>(sum);
+  __syncwarp();  // the next leader of this digit may be another lane
+}
 
 __global__ void __launch_bounds__(kRgThreads)
     route_global_kernel(const float* __restrict__ sc, int Gq, int G, long long budget, int* __restrict__ route,
                         const int* __restrict__ key_gsize, const int* __restrict__ qblock_size,
                         unsigned long long* __restrict__ pairs, int* __restrict__ status) {
-  extern __shared__ int s_best[];  // [Gq] best group per block
-  __shared__ unsigned long long hist[256];
+  // dynamic: per-warp histograms [kRgWarps][256] u64, then the best group of every block
+  extern __shared__ unsigned long long s_hist[];
+  int* s_best = reinterpret_cast<int*>(s_hist + kRgWarps * 256);
+  __shared__ unsigned long long s_tot[256];
+  __shared__ long long s_wsum[kRgWarps];
   __shared__ long long s_spent, s_below;
-  __shared__ unsigned long long s_prefix;
-  __shared__ int s_cross, s_digit;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = kRgThreads / 32;
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_cross, s_found;
+  __shared__ unsigned long long s_kstar;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int head = blockIdx.x;
   const float* scs = sc + static_cast<size_t>(head) * Gq * G;
   const int* ks = key_gsize + static_cast<size_t>(head) * G;
   const int* bs = qblock_size + static_cast<size_t>(head) * Gq;
+  unsigned long long* hw = s_hist + warp * 256;
   if (tid == 0) {
     s_spent = 0;
     s_below = 0;
     s_prefix = 0;
     s_cross = 0;
+    s_found = 0;
+    s_kstar = 0;
   }
+  for (int x = lane; x < 256; x += 32) hw[x] = 0;
   __syncthreads();
-  // (1) best group of every block (smallest route key), its pairs
+  // pass 0 (group and block sizes are at most B = 128: a pair costs <= 2^14, a warp's sum fits an int)
   bool saw_nan = false;
-  for (int b = warp; b < Gq; b += nwarps) {
+  for (int b = warp; b < Gq; b += kRgWarps) {
+    const float* row = scs + static_cast<size_t>(b) * G;
+    const int nb = bs[b];
     unsigned long long best = ~0ull;
-    for (int g = lane; g < G; g += 32) {
-      const float v = scs[static_cast<size_t>(b) * G + g];
-      saw_nan |= (v != v);
-      const unsigned long long key = route_key(v, g);
-      best = key < best ? key : best;
+    for (int g0 = 0; g0 < G; g0 += 32) {
+      const int g = g0 + lane;
+      int digit = -1, cost = 0;
+      if (g < G) {
+        const float v = row[g];
+        saw_nan |= (v != v);
+        const uint32_t hi = score_hi(v);
+        const unsigned long long key = (static_cast<unsigned long long>(hi) << 32) | static_cast<uint32_t>(g);
+        best = key < best ? key : best;
+        digit = static_cast<int>(hi >> 24);
+        cost = nb * ks[g];
+      }
+      warp_hist_add(hw, digit, cost);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const unsigned long long y = __shfl_xor_sync(0xffffffffu, best, o);
       best = y < best ? y : best;
     }
+    __syncwarp();
     if (lane == 0) {
       const int g = static_cast<int>(best & 0xffffffffu);
+      const unsigned long long c = static_cast<unsigned long long>(nb) * ks[g];
       s_best[b] = g;
-      atomicAdd(reinterpret_cast<unsigned long long*>(&s_spent),
-                static_cast<unsigned long long>(static_cast<long long>(bs[b]) * ks[g]));
+      hw[static_cast<uint32_t>(best >> 32) >> 24] -= c;  // the best pair is no candidate
+      atomicAdd(reinterpret_cast<unsigned long long*>(&s_spent), c);
     }
+    __syncwarp();
   }
   __syncthreads();
-  const long long rem = budget - s_spent;  // pairs left for the other candidates
-  // (2) weighted radix select: the first candidate (ascending key) whose cumulative cost
-  // exceeds rem; every candidate before it is taken.  s_cross = 0: all candidates fit.
-  auto ckey = [&](int b, int g, float v) {
-    const uint32_t hi = (v != v) ? 0xffffffffu : ~float_order_key(v);
-    return (static_cast<unsigned long long>(hi) << 32) | static_cast<uint32_t>(b * G + g);
-  };
-  const long long cand = static_cast<long long>(Gq) * G;
+  const long long rem = budget - s_spent;  // pairs left for the candidates
   if (rem >= 0) {
-    for (int shift = 56; shift >= 0; shift -= 8) {
-      for (int x = tid; x < 256; x += kRgThreads) hist[x] = 0;
-      __syncthreads();
-      const unsigned long long hmask = shift == 56 ? 0ull : (~0ull << (shift + 8));
-      const unsigned long long prefix = s_prefix;
-      for (long long x0 = 0; x0 < cand; x0 += kRgThreads) {
-        const long long x = x0 + tid;
-        int digit = -1, cost = 0;
-        if (x < cand) {
-          const int b = static_cast<int>(x / G), g = static_cast<int>(x - static_cast<long long>(b) * G);
-          if (g != s_best[b]) {
-            const unsigned long long key = ckey(b, g, scs[x]);
-            if ((key & hmask) == prefix) {
-              digit = static_cast<int>((key >> shift) & 255u);
-              cost = bs[b] * ks[g];
+    // passes 0-3: the crossing score key, 8 bits at a time
+    for (int level = 0; level < 4; ++level) {
+      const int shift = 24 - 8 * level;
+      if (level > 0) {
+        const uint32_t mask = ~0u << (shift + 8), prefix = s_prefix;
+        for (int x = lane; x < 256; x += 32) hw[x] = 0;
+        __syncwarp();
+        for (int b = warp; b < Gq; b += kRgWarps) {
+          const float* row = scs + static_cast<size_t>(b) * G;
+          const int nb = bs[b], bg = s_best[b];
+          for (int g0 = 0; g0 < G; g0 += 32) {
+            const int g = g0 + lane;
+            int digit = -1, cost = 0;
+            if (g < G && g != bg) {
+              const uint32_t hi = score_hi(row[g]);
+              if ((hi & mask) == prefix) {
+                digit = static_cast<int>((hi >> shift) & 255u);
+                cost = nb * ks[g];
+              }
             }
+            if (__any_sync(0xffffffffu, digit >= 0)) warp_hist_add(hw, digit, cost);
           }
         }
-        // lanes with the same digit add their costs once (a leader per digit)
-        const unsigned int peers = __match_any_sync(0xffffffffu, digit);
-        const int sum = __reduce_add_sync(peers, cost);
-        if (digit >= 0 && lane == __ffs(peers) - 1 && sum > 0)
-          atomicAdd(&hist[digit], static_cast<unsigned long long>(sum));
+      }
+      __syncthreads();
+      if (tid < 256) {
+        unsigned long long t = 0;
+        for (int w = 0; w < kRgWarps; ++w) t += s_hist[w * 256 + tid];
+        s_tot[tid] = t;
       }
       __syncthreads();
       if (tid == 0) {
         long long below = s_below;
         int d = 0;
         for (; d < 256; ++d) {
-          const long long hcost = static_cast<long long>(hist[d]);
-          if (below + hcost > rem) break;
-          below += hcost;
+          const long long c = static_cast<long long>(s_tot[d]);
+          if (below + c > rem) break;
+          below += c;
         }
-        if (d == 256) {
-          // everything under this prefix fits (only possible at the top level: below it,
-          // the prefix was chosen because its bin crosses)
-          s_digit = -1;
-        } else {
-          s_digit = d;
-          s_below = below;
-          s_prefix = prefix | (static_cast<unsigned long long>(d) << shift);
+        if (d < 256) {
           s_cross = 1;
+          s_below = below;
+          s_prefix |= static_cast<uint32_t>(d) << shift;
         }
+        // d == 256 only at level 0 (every candidate fits); below it the chosen bin crosses
       }
       __syncthreads();
-      if (s_digit < 0) break;
+      if (!s_cross) break;
+    }
+    if (s_cross) {
+      // tie pass: the pairs with score key T in ascending b G + g order
+      const uint32_t T = s_prefix;
+      const long long cand = static_cast<long long>(Gq) * G;
+      for (long long x0 = 0; x0 < cand; x0 += kRgThreads) {
+        const long long x = x0 + tid;
+        int cost = 0;
+        bool tie = false;
+        if (x < cand) {
+          const int b = static_cast<int>(x / G), g = static_cast<int>(x - static_cast<long long>(b) * G);
+          if (g != s_best[b] && score_hi(scs[x]) == T) {
+            tie = true;
+            cost = bs[b] * ks[g];
+          }
+        }
+        if (!__syncthreads_or(tie)) continue;
+        int incl = cost;  // warp-inclusive prefix of the tie costs
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        if (lane == 31) s_wsum[warp] = incl;
+        __syncthreads();
+        long long off = s_below;
+        for (int w = 0; w < warp; ++w) off += s_wsum[w];
+        const long long after = off + incl;
+        if (tie && after > rem && after - cost <= rem) {
+          s_kstar = (static_cast<unsigned long long>(T) << 32) | static_cast<uint32_t>(x);
+          s_found = 1;
+        }
+        __syncthreads();
+        if (s_found) break;
+        if (tid == 0) {
+          long long t = 0;
+          for (int w = 0; w < kRgWarps; ++w) t += s_wsum[w];
+          s_below += t;
+        }
+        __syncthreads();
+      }
     }
   }
   const bool cross = s_cross != 0;
-  const unsigned long long kstar = s_prefix;  // the first candidate that does not fit
-  // (3) routes: every block's kept best group and the candidates before kstar
-  for (int b = warp; b < Gq; b += nwarps) {
+  const unsigned long long kstar = s_kstar;  // the first candidate that does not fit
+  // emit: every block's best group and the candidates before kstar
+  for (int b = warp; b < Gq; b += kRgWarps) {
+    const float* row = scs + static_cast<size_t>(b) * G;
     int* out = route + (static_cast<size_t>(head) * Gq + b) * G;
+    const int bg = s_best[b];
     int written = 0;
     long long member_sum = 0;
     for (int g0 = 0; g0 < G; g0 += 32) {
       const int g = g0 + lane;
       bool sel = false;
       if (g < G) {
-        if (g == s_best[b]) {
+        if (g == bg) {
           sel = true;
         } else if (rem >= 0) {
-          sel = !cross || ckey(b, g, scs[static_cast<size_t>(b) * G + g]) < kstar;
+          const unsigned long long key =
+              (static_cast<unsigned long long>(score_hi(row[g])) << 32) | static_cast<uint32_t>(b * G + g);
+          sel = !cross || key < kstar;
         }
       }
       const unsigned int ball = __ballot_sync(0xffffffffu, sel);
@@ -245,7 +323,8 @@ __global__ void __launch_bounds__(kRgThreads)
     if (pairs != nullptr) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) member_sum += __shfl_xor_sync(0xffffffffu, member_sum, o);
-      if (lane == 0) atomicAdd(pairs + head, static_cast<unsigned long long>(static_cast<long long>(bs[b]) * member_sum));
+      if (lane == 0)
+        atomicAdd(pairs + head, static_cast<unsigned long long>(static_cast<long long>(bs[b]) * member_sum));
     }
   }
   saw_nan = __syncthreads_or(saw_nan);
@@ -328,8 +407,12 @@ cudaError_t launch_route_global(const float* sc, int heads, int Gq, int G, long 
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  route_global_kernel<<<heads, kRgThreads, sizeof(int) * Gq, st>>>(sc, Gq, G, budget, route, key_gsize,
-                                                                     qblock_size, up, status);
+  const size_t smem = sizeof(unsigned long long) * kRgWarps * 256 + sizeof(int) * Gq;
+  cudaError_t e = cudaFuncSetAttribute(route_global_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  route_global_kernel<<<heads, kRgThreads, smem, st>>>(sc, Gq, G, budget, route, key_gsize, qblock_size, up,
+                                                       status);
   return counted(cudaGetLastError(), up != nullptr ? 2 : 1);
 }
 
