@@ -125,6 +125,19 @@ constexpr int kRgWarps = kRgThreads / 32;
 
 __device__ __forceinline__ uint32_t score_hi(float v) { return (v != v) ? 0xffffffffu : ~float_order_key(v); }
 
+constexpr int kRgU = 8;  // independent loads per lane in flight
+
+// Scores and key-group sizes of groups g0 + 32 u + lane, u < kRgU, of one block row.
+__device__ __forceinline__ void load_row_chunk(const float* __restrict__ row, const int* __restrict__ ks, int G,
+                                               int g0, int lane, float (&v)[kRgU], int (&kz)[kRgU]) {
+#pragma unroll
+  for (int u = 0; u < kRgU; ++u) {
+    const int g = g0 + 32 * u + lane;
+    v[u] = g < G ? __ldg(row + g) : 0.f;
+    kz[u] = g < G ? __ldg(ks + g) : 0;
+  }
+}
+
 __device__ __forceinline__ void warp_hist_add(unsigned long long* hw, int digit, int cost) {
   const unsigned int peers = __match_any_sync(0xffffffffu, digit);
   const int sum = __reduce_add_sync(peers, cost);
@@ -167,19 +180,25 @@ __global__ void __launch_bounds__(kRgThreads)
     const float* row = scs + static_cast<size_t>(b) * G;
     const int nb = bs[b];
     unsigned long long best = ~0ull;
-    for (int g0 = 0; g0 < G; g0 += 32) {
-      const int g = g0 + lane;
-      int digit = -1, cost = 0;
-      if (g < G) {
-        const float v = row[g];
-        saw_nan |= (v != v);
-        const uint32_t hi = score_hi(v);
-        const unsigned long long key = (static_cast<unsigned long long>(hi) << 32) | static_cast<uint32_t>(g);
-        best = key < best ? key : best;
-        digit = static_cast<int>(hi >> 24);
-        cost = nb * ks[g];
+    for (int g0 = 0; g0 < G; g0 += 32 * kRgU) {
+      float v[kRgU];
+      int kz[kRgU];
+      load_row_chunk(row, ks, G, g0, lane, v, kz);
+#pragma unroll
+      for (int u = 0; u < kRgU; ++u) {
+        if (g0 + 32 * u >= G) break;
+        const int g = g0 + 32 * u + lane;
+        int digit = -1, cost = 0;
+        if (g < G) {
+          saw_nan |= (v[u] != v[u]);
+          const uint32_t hi = score_hi(v[u]);
+          const unsigned long long key = (static_cast<unsigned long long>(hi) << 32) | static_cast<uint32_t>(g);
+          best = key < best ? key : best;
+          digit = static_cast<int>(hi >> 24);
+          cost = nb * kz[u];
+        }
+        warp_hist_add(hw, digit, cost);
       }
-      warp_hist_add(hw, digit, cost);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -209,17 +228,24 @@ __global__ void __launch_bounds__(kRgThreads)
         for (int b = warp; b < Gq; b += kRgWarps) {
           const float* row = scs + static_cast<size_t>(b) * G;
           const int nb = bs[b], bg = s_best[b];
-          for (int g0 = 0; g0 < G; g0 += 32) {
-            const int g = g0 + lane;
-            int digit = -1, cost = 0;
-            if (g < G && g != bg) {
-              const uint32_t hi = score_hi(row[g]);
-              if ((hi & mask) == prefix) {
-                digit = static_cast<int>((hi >> shift) & 255u);
-                cost = nb * ks[g];
+          for (int g0 = 0; g0 < G; g0 += 32 * kRgU) {
+            float v[kRgU];
+            int kz[kRgU];
+            load_row_chunk(row, ks, G, g0, lane, v, kz);
+#pragma unroll
+            for (int u = 0; u < kRgU; ++u) {
+              if (g0 + 32 * u >= G) break;
+              const int g = g0 + 32 * u + lane;
+              int digit = -1, cost = 0;
+              if (g < G && g != bg) {
+                const uint32_t hi = score_hi(v[u]);
+                if ((hi & mask) == prefix) {
+                  digit = static_cast<int>((hi >> shift) & 255u);
+                  cost = nb * kz[u];
+                }
               }
+              if (__any_sync(0xffffffffu, digit >= 0)) warp_hist_add(hw, digit, cost);
             }
-            if (__any_sync(0xffffffffu, digit >= 0)) warp_hist_add(hw, digit, cost);
           }
         }
       }
@@ -249,22 +275,26 @@ __global__ void __launch_bounds__(kRgThreads)
       if (!s_cross) break;
     }
     if (s_cross) {
-      // tie pass: the pairs with score key T in ascending b G + g order
+      // tie pass: the pairs with score key T in ascending b G + g order; thread t takes
+      // kRgU consecutive pairs of each chunk, so chunk order = thread order = pair order
       const uint32_t T = s_prefix;
       const long long cand = static_cast<long long>(Gq) * G;
-      for (long long x0 = 0; x0 < cand; x0 += kRgThreads) {
-        const long long x = x0 + tid;
-        int cost = 0;
-        bool tie = false;
-        if (x < cand) {
-          const int b = static_cast<int>(x / G), g = static_cast<int>(x - static_cast<long long>(b) * G);
-          if (g != s_best[b] && score_hi(scs[x]) == T) {
-            tie = true;
-            cost = bs[b] * ks[g];
+      for (long long x0 = 0; x0 < cand; x0 += static_cast<long long>(kRgThreads) * kRgU) {
+        const long long xt = x0 + static_cast<long long>(tid) * kRgU;
+        int cost[kRgU];  // tie costs (0: no tie; a zero-cost tie adds nothing and never crosses)
+        int tsum = 0;
+#pragma unroll
+        for (int u = 0; u < kRgU; ++u) {
+          cost[u] = 0;
+          const long long x = xt + u;
+          if (x < cand) {
+            const int b = static_cast<int>(x / G), g = static_cast<int>(x - static_cast<long long>(b) * G);
+            if (g != s_best[b] && score_hi(__ldg(scs + x)) == T) cost[u] = bs[b] * ks[g];
           }
+          tsum += cost[u];
         }
-        if (!__syncthreads_or(tie)) continue;
-        int incl = cost;  // warp-inclusive prefix of the tie costs
+        if (!__syncthreads_or(tsum > 0)) continue;
+        int incl = tsum;  // warp-inclusive prefix of the threads' tie costs
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const int y = __shfl_up_sync(0xffffffffu, incl, o);
@@ -272,12 +302,18 @@ __global__ void __launch_bounds__(kRgThreads)
         }
         if (lane == 31) s_wsum[warp] = incl;
         __syncthreads();
-        long long off = s_below;
-        for (int w = 0; w < warp; ++w) off += s_wsum[w];
-        const long long after = off + incl;
-        if (tie && after > rem && after - cost <= rem) {
-          s_kstar = (static_cast<unsigned long long>(T) << 32) | static_cast<uint32_t>(x);
-          s_found = 1;
+        long long run = s_below;
+        for (int w = 0; w < warp; ++w) run += s_wsum[w];
+        run += incl - tsum;  // cost of the ties before this thread's first pair
+        if (tsum > 0 && run + tsum > rem) {
+#pragma unroll
+          for (int u = 0; u < kRgU; ++u) {
+            if (cost[u] > 0 && run <= rem && run + cost[u] > rem) {
+              s_kstar = (static_cast<unsigned long long>(T) << 32) | static_cast<uint32_t>(xt + u);
+              s_found = 1;
+            }
+            run += cost[u];
+          }
         }
         __syncthreads();
         if (s_found) break;
@@ -299,25 +335,32 @@ __global__ void __launch_bounds__(kRgThreads)
     const int bg = s_best[b];
     int written = 0;
     long long member_sum = 0;
-    for (int g0 = 0; g0 < G; g0 += 32) {
-      const int g = g0 + lane;
-      bool sel = false;
-      if (g < G) {
-        if (g == bg) {
-          sel = true;
-        } else if (rem >= 0) {
-          const unsigned long long key =
-              (static_cast<unsigned long long>(score_hi(row[g])) << 32) | static_cast<uint32_t>(b * G + g);
-          sel = !cross || key < kstar;
+    for (int g0 = 0; g0 < G; g0 += 32 * kRgU) {
+      float v[kRgU];
+      int kz[kRgU];
+      load_row_chunk(row, ks, G, g0, lane, v, kz);
+#pragma unroll
+      for (int u = 0; u < kRgU; ++u) {
+        if (g0 + 32 * u >= G) break;
+        const int g = g0 + 32 * u + lane;
+        bool sel = false;
+        if (g < G) {
+          if (g == bg) {
+            sel = true;
+          } else if (rem >= 0) {
+            const unsigned long long key =
+                (static_cast<unsigned long long>(score_hi(v[u])) << 32) | static_cast<uint32_t>(b * G + g);
+            sel = !cross || key < kstar;
+          }
         }
+        const unsigned int ball = __ballot_sync(0xffffffffu, sel);
+        const int slot = written + __popc(ball & ((1u << lane) - 1u));
+        if (sel) {
+          out[slot] = g;
+          member_sum += kz[u];
+        }
+        written += __popc(ball);
       }
-      const unsigned int ball = __ballot_sync(0xffffffffu, sel);
-      const int slot = written + __popc(ball & ((1u << lane) - 1u));
-      if (sel) {
-        out[slot] = g;
-        member_sum += ks[g];
-      }
-      written += __popc(ball);
     }
     for (int sidx = written + lane; sidx < G; sidx += 32) out[sidx] = -1;
     if (pairs != nullptr) {
