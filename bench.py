@@ -327,6 +327,7 @@ def run_ours(args, w):
         dist.barrier()
     ms_step = elapsed / args.steps * 1e3
     stage_ms = {s: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in events) for i, s in enumerate(stages)}
+    step_ms = [round(e[0].elapsed_time(e[-1]), 3) for e in events]  # per timed step, first stage to last
 
     # ---- dominant kernel roofline (block-sparse attention: 4*d flops per routed pair)
     pairs = last["pairs"].to(torch.float64).sum().item()
@@ -425,7 +426,7 @@ def run_ours(args, w):
                         "uncorrected_sparse_mean": s_mean, "uncorrected_sparse_p99": s_p99,
                         "reference": "same-family dense attention, fp32 output"},
                 "density": pairs / (float(n) ** 2 * h * bt), "k": last["k"],
-                "stage_ms": stage_ms, "dense_ms": dense_ms, "sdpa_ms": sdpa_ms,
+                "stage_ms": stage_ms, "step_ms": step_ms, "dense_ms": dense_ms, "sdpa_ms": sdpa_ms,
                 "speedup_vs_dense": dense_ms / ms_step,
                 "roofline": roofline, "cpu_baseline": cpu_base,
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
