@@ -9,16 +9,16 @@
 // the capacity fill, and the minimum of each 64-column segment is kept for the later
 // proposals.
 //
-// Persistent: one CTA per SM loops over (head, 128-item tile) work items; groups are
-// streamed in chunks of 128 (W double-buffered, cp.async into 128B-swizzled tiles); the
-// accumulator chunk lives in TMEM (two buffers, so the MMA of chunk c+1 -- also of the
-// next item -- overlaps the epilogue of chunk c).  Warps 0-1 load, warp 2 issues the
+// Persistent: one CTA per SM takes a contiguous run of (head, 128-item tile) work items;
+// groups are streamed in chunks of 128 (W double-buffered, TMA into 128B-swizzled tiles);
+// the accumulator chunk lives in TMEM (two buffers, so the MMA of chunk c+1 -- also of
+// the next item -- overlaps the epilogue of chunk c).  Warp 0 loads, warp 2 issues the
 // MMAs, warps 4-11 run the epilogue: each row is owned by two threads (columns 0-63 and
-// 64-127 of every chunk); a warp transposes its 32 rows x 32 columns through shared
-// memory so that each 16-byte-per-lane store instruction writes 128 contiguous bytes of
-// each of 4 rows.  The row argmin is a strict '<' scan in
-// ascending column order (first minimum wins, +-0 compare equal), merged across the two
-// halves at the end.  Every wait is bounded.
+// 64-127 of every chunk); a warp stages 32 rows x 16 columns at a time in shared memory
+// and one lane writes them to D with a tiled TMA store.  The row argmin is a strict '<'
+// scan in ascending column order (first minimum wins, +-0 compare equal), merged across
+// the two halves at the end of the item through a double-buffered slot.  Every wait is
+// bounded.
 #include <cuda.h>
 
 #include "attention.cuh"
