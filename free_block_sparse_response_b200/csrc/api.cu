@@ -50,6 +50,11 @@ int api_fail(int code, const char* msg) { return fail(code, "%s", msg); }
 
 namespace {
 
+// Row stride of the distance matrix: a whole number of 128-byte lines, so that every
+// row starts on a line and the distance kernel's 64-byte stores never split a sector.
+size_t dmat_ld(int G) { return static_cast<size_t>(G + 31) / 32 * 32; }
+
+
 #define SPR_CUDA(call, where)                       \
   do {                                              \
     cudaError_t e_ = (call);                        \
@@ -93,7 +98,7 @@ Layout make_layout(int heads, int N, int d, int block, int S, int P) {
   L.whi = take(2 * H * G * D);
   L.wlo = take(2 * H * G * D);
   L.eg = take(sizeof(float) * H * G);
-  L.dmat = take(sizeof(float) * H * n * ((G + 3) / 4 * 4));
+  L.dmat = take(sizeof(float) * H * n * dmat_ld(G));
   L.segmin = take(sizeof(unsigned long long) * H * n * 2 * ((G + 127) / 128));
   L.prop_g0 = take(sizeof(int) * H * n);
   L.prop_v0 = take(sizeof(float) * H * n);
@@ -244,7 +249,7 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
   float* dmat = at<float>(ws, L.dmat);
   spr::FillArgs fa{};
   fa.D = dmat;
-  fa.ldd = (G + 3) / 4 * 4;
+  fa.ldd = dmat_ld(G);
   fa.prop_g0 = at<int>(ws, L.prop_g0);
   fa.prop_v0 = at<float>(ws, L.prop_v0);
   // segment minima come from the tensor-core distance kernel (bf16, d = 128)

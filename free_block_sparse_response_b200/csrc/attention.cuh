@@ -62,7 +62,6 @@ cudaError_t launch_attention(const AttnArgs& a, bool dense, cudaStream_t st);
 // TMA map over a [rows, 128] bf16 tensor, 128-byte swizzle, box 64 columns x box_rows rows
 // (box_rows = 1 for row gathers); false if the driver entry point or the encode fails.
 bool bf16_map(CUtensorMap* m, const void* base, long long rows, int box_rows);
-bool f32_store_map(CUtensorMap* m, void* base, int cols, long long rows, int box_rows);
 // Group-ordered copies of K and V ([heads, G * 128, 128] bf16, pad rows zero).  With a
 // tag (the workspace header's kv_tag) the copy is skipped on the device when the tag
 // names the same K, V, key_perm, key_gsize and shape, and the tag is set afterwards.

@@ -588,21 +588,6 @@ bool bf16_map(CUtensorMap* m, const void* base, long long rows, int box_rows) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Map over a [rows, cols] fp32 tensor (row stride cols, a multiple of 4) with 64-byte
-// swizzle and a box of 16 columns x box_rows rows, for tiled stores.
-bool f32_store_map(CUtensorMap* m, void* base, int cols, long long rows, int box_rows) {
-  auto fn = encode_tiled();
-  if (fn == nullptr || (reinterpret_cast<uintptr_t>(base) & 15u) != 0 || rows <= 0 || cols <= 0 || cols % 4 != 0)
-    return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * sizeof(float)};
-  cuuint32_t box[2] = {16, static_cast<cuuint32_t>(box_rows)};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
-}
-
 namespace {
 __global__ void kv_tag_kernel(KvTag want, unsigned long long* have) {
   if (threadIdx.x < 6) have[threadIdx.x] = want.w[threadIdx.x];

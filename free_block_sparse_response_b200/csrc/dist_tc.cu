@@ -9,16 +9,16 @@
 // the capacity fill, and the minimum of each 64-column segment is kept for the later
 // proposals.
 //
-// Persistent: one CTA per SM takes a contiguous run of (head, 128-item tile) work items;
-// groups are streamed in chunks of 128 (W double-buffered, TMA into 128B-swizzled tiles);
-// the accumulator chunk lives in TMEM (two buffers, so the MMA of chunk c+1 -- also of
-// the next item -- overlaps the epilogue of chunk c).  Warp 0 loads, warp 2 issues the
+// Persistent: one CTA per SM loops over (head, 128-item tile) work items; groups are
+// streamed in chunks of 128 (W double-buffered, TMA into 128B-swizzled tiles); the
+// accumulator chunk lives in TMEM (two buffers, so the MMA of chunk c+1 -- also of the
+// next item -- overlaps the epilogue of chunk c).  Warp 0 loads, warp 2 issues the
 // MMAs, warps 4-11 run the epilogue: each row is owned by two threads (columns 0-63 and
-// 64-127 of every chunk); a warp stages 32 rows x 16 columns at a time in shared memory
-// and one lane writes them to D with a tiled TMA store.  The row argmin is a strict '<'
-// scan in ascending column order (first minimum wins, +-0 compare equal), merged across
-// the two halves at the end of the item through a double-buffered slot.  Every wait is
-// bounded.
+// 64-127 of every chunk); a warp transposes its 32 rows x 32 columns through shared
+// memory so that each 16-byte-per-lane store instruction writes 128 contiguous bytes of
+// each of 4 rows.  The row argmin is a strict '<' scan in
+// ascending column order (first minimum wins, +-0 compare equal), merged across the two
+// halves at the end.  Every wait is bounded.
 #include <cuda.h>
 
 #include "attention.cuh"
@@ -34,11 +34,10 @@ constexpr int kDtThreads = 384;
 constexpr uint32_t kDtTile = 128 * 128 * 2;
 constexpr uint32_t kDtTmemCols = 256;
 constexpr float kDtInf = __builtin_huge_valf();
-constexpr uint32_t kWarpStage = 2 * 32 * 16 * 4;  // one warp's two 32 x 16 fp32 staging blocks
+constexpr uint32_t kWarpStage = 32 * 32 * 4;  // one warp's 32 x 32 fp32 transpose block
 
 enum : int {
-  kXFull0 = 0, kXEmpty0 = 2, kWFull0 = 4, kWEmpty0 = 6, kAccFull0 = 8, kAccEmpty0 = 10, kDtDrain = 12,
-  kBestFull0 = 13, kBestEmpty0 = 15, kDtBars = 17
+  kXFull0 = 0, kXEmpty0 = 2, kWFull0 = 4, kWEmpty0 = 6, kAccFull0 = 8, kAccEmpty0 = 10, kDtDrain = 12, kDtBars = 13
 };
 
 // Packed pairs of fp32: one f32x2 instruction, each lane rounded exactly as the scalar op.
@@ -69,7 +68,7 @@ __device__ __forceinline__ unsigned long long dist_key(float v, int idx) {
 template <bool SPLIT>
 __global__ void __launch_bounds__(kDtThreads, 1)
     dist_tc_kernel(const __grid_constant__ CUtensorMap tmX, int n, const __grid_constant__ CUtensorMap tmWhi,
-                   const __grid_constant__ CUtensorMap tmWlo, const __grid_constant__ CUtensorMap tmD, int ncols, int ldd, const float* __restrict__ nrm,
+                   const __grid_constant__ CUtensorMap tmWlo, int ncols, int ldd, const float* __restrict__ nrm,
                    const float* __restrict__ ecol, float tau2, float* __restrict__ Dout, int* __restrict__ prop_g,
                    float* __restrict__ prop_v, unsigned long long* __restrict__ seg_min, int nseg,
                    int* __restrict__ status, int heads) {
@@ -77,8 +76,8 @@ __global__ void __launch_bounds__(kDtThreads, 1)
   __shared__ __align__(8) uint64_t bars[kDtBars];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
-  __shared__ float s_best_v[2][128];  // the upper half's row minimum, by item parity
-  __shared__ int s_best_c[2][128];
+  __shared__ float s_best_v[128];
+  __shared__ int s_best_c[128];
   constexpr int kWStage = kDtTile * (SPLIT ? 2 : 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -92,9 +91,6 @@ __global__ void __launch_bounds__(kDtThreads, 1)
   const int n_chunks = ceil_div(ncols, 128);
   const int tiles = ceil_div(n, 128);
   const int total = heads * tiles;
-  // each CTA takes a contiguous run of item tiles, so that it rarely changes head
-  const int w_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * total / gridDim.x);
-  const int w_end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * total / gridDim.x);
 
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -106,8 +102,6 @@ __global__ void __launch_bounds__(kDtThreads, 1)
       tc::mbar_init(bar(kWEmpty0 + s), 1);
       tc::mbar_init(bar(kAccFull0 + s), 1);
       tc::mbar_init(bar(kAccEmpty0 + s), 256);
-      tc::mbar_init(bar(kBestFull0 + s), 128);
-      tc::mbar_init(bar(kBestEmpty0 + s), 128);
     }
     tc::mbar_init(bar(kDtDrain), 1);
     abort_flag = 0;
@@ -132,7 +126,7 @@ __global__ void __launch_bounds__(kDtThreads, 1)
     if (lane == 0) {
       bool ok = true;
       int last_it = -1, last_q = -1;
-      for (int w = w_begin, it = 0; ok && w < w_end; ++w, ++it) {
+      for (int w = blockIdx.x, it = 0; ok && w < total; w += gridDim.x, ++it) {
         const int head = w / tiles, row0 = (w - head * tiles) * 128;
         if (it >= 1 && !tc::mbar_wait(bar(kXEmpty0), (it - 1) & 1, abort_v, status)) break;
         tc::mbar_arrive_expect_tx(bar(kXFull0), kDtTile);
@@ -173,7 +167,7 @@ __global__ void __launch_bounds__(kDtThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kId = tc::idesc_bf16(128, 128, false, false);
       bool ok = true;
-      for (int w = w_begin, it = 0; ok && w < w_end; ++w, ++it) {
+      for (int w = blockIdx.x, it = 0; ok && w < total; w += gridDim.x, ++it) {
         if (!tc::mbar_wait(bar(kXFull0), it & 1, abort_v, status)) break;
         tc::fence_proxy_async();
         for (int c = 0; c < n_chunks; ++c) {
@@ -213,9 +207,8 @@ __global__ void __launch_bounds__(kDtThreads, 1)
     const float m2t = -2.f * tau2;
     const uint32_t wstage = sStage + static_cast<uint32_t>(warp - 4) * kWarpStage;
     int loaded_head = -1;
-    int sbuf = 0;  // staging buffer parity
     bool aborted = false;  // after a failed wait: keep passing the named barriers, skip the work
-    for (int w = w_begin, it = 0; w < w_end; ++w, ++it) {
+    for (int w = blockIdx.x, it = 0; w < total; w += gridDim.x, ++it) {
       const int head = w / tiles, row0 = (w - head * tiles) * 128;
       if (head != loaded_head) {  // tau^2 e_g of this head, padded with +inf to whole chunks
         asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -294,62 +287,50 @@ __global__ void __launch_bounds__(kDtThreads, 1)
         if (seg_min != nullptr && row < n)
           seg_min[(static_cast<size_t>(head) * n + row) * nseg + 2 * c + half] =
               seg_c >= 0 ? dist_key(seg_v, c0 + seg_c) : ~0ull;
-        // D through shared memory: the warp stages its 32 rows x 16 columns in one of two
-        // 2 KB buffers (64-byte swizzle: lane l writes its row's 16-byte chunk k at chunk
-        // position k ^ ((l >> 1) & 3), conflict-free) and lane 0 stores the block with one
-        // tiled TMA store; a buffer is rewritten once its previous store has read it.  The
-        // last tile of a head (rows past n) is stored row by row instead.
-        if (full_rows) {
+        // transpose 32 rows x 32 columns at a time through shared memory: lane l writes its
+        // row's chunk k at chunk position k ^ (l & 7) (conflict-free), then reads column l
+        // of every row, so each global store covers 128 contiguous bytes of one row
+        const size_t rowbase = static_cast<size_t>(head) * n + wrow0;
 #pragma unroll
-          for (int blk = 0; blk < 4; ++blk) {
-            const int col = c0 + blk * 16;
-            if (col >= ldd) break;
-            const uint32_t buf = wstage + static_cast<uint32_t>(sbuf & 1) * 2048u;
-            if (lane == 0) tc::bulk_wait_read1();
-            __syncwarp();
+        for (int blk = 0; blk < 2; ++blk) {
+          __syncwarp();
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int j = blk * 16 + 4 * k;
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(buf + lane * 64 +
-                                                                           ((k ^ ((lane >> 1) & 3)) << 4)),
-                           "r"(u[j]), "r"(u[j + 1]), "r"(u[j + 2]), "r"(u[j + 3])
-                           : "memory");
-            }
-            tc::fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) {
-              tc::tma_store_2d(&tmD, buf, col, head * n + wrow0);
-              tc::bulk_commit();
-            }
-            ++sbuf;
+          for (int k = 0; k < 8; ++k) {
+            const int j = blk * 32 + 4 * k;
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(wstage + lane * 128 + ((k ^ (lane & 7)) << 4)),
+                         "r"(u[j]), "r"(u[j + 1]), "r"(u[j + 2]), "r"(u[j + 3])
+                         : "memory");
           }
-        } else if (row < n) {
-          float* drow = Dout + (static_cast<size_t>(head) * n + row) * ldd;
+          __syncwarp();
+          // lane l stores 4 consecutive columns (16 B) of row rr + (l >> 3): every store
+          // instruction writes 128 contiguous bytes of each of 4 rows
+          const int col = c0 + blk * 32 + 4 * (lane & 7);
+          if (col < ldd) {
+            const int rsub = lane >> 3;
+            float* dst = Dout + (rowbase + rsub) * ldd + col;
 #pragma unroll
-          for (int j = 0; j < 64; ++j)
-            if (c0 + j < ldd) drow[c0 + j] = __uint_as_float(u[j]);
+            for (int rr = 0; rr < 32; rr += 4) {
+              const int row_l = rr + rsub;
+              if (full_rows || wrow0 + row_l < n) {
+                float4 v;
+                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                             : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                             : "r"(wstage + row_l * 128 + (((lane & 7) ^ (row_l & 7)) << 4)));
+                *reinterpret_cast<float4*>(dst) = v;
+              }
+              dst += 4 * static_cast<size_t>(ldd);
+            }
+          }
         }
       }
-      // the halves' minima meet through a double-buffered slot (full / empty barriers of
-      // 128 arrivals), so neither half waits for the other at the end of every item
-      const int pb = it & 1;
       if (half == 1) {
-        if (!aborted && it >= 2 &&
-            !__all_sync(0xffffffffu, tc::mbar_wait(bar(kBestEmpty0 + pb), ((it >> 1) - 1) & 1, abort_v, status)))
-          aborted = true;
-        if (!aborted) {
-          s_best_v[pb][r] = best_v;
-          s_best_c[pb][r] = best_c;
-          tc::mbar_arrive(bar(kBestFull0 + pb));
-        }
-      } else if (!aborted &&
-                 !__all_sync(0xffffffffu, tc::mbar_wait(bar(kBestFull0 + pb), (it >> 1) & 1, abort_v, status))) {
-        aborted = true;
+        s_best_v[r] = best_v;
+        s_best_c[r] = best_c;
       }
-      if (half == 0 && !aborted) {
-        const float v1 = s_best_v[pb][r];
-        const int c1 = s_best_c[pb][r];
-        tc::mbar_arrive(bar(kBestEmpty0 + pb));
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (half == 0 && row < n && !aborted) {
+        const float v1 = s_best_v[r];
+        const int c1 = s_best_c[r];
         // half 0 holds the lower 64 columns of every chunk: on equal values take the
         // lower column, on a smaller value take it
         if (c1 >= 0 && (best_c < 0 || v1 < best_v || (v1 == best_v && c1 < best_c))) {
@@ -357,16 +338,13 @@ __global__ void __launch_bounds__(kDtThreads, 1)
           best_c = c1;
         }
         if (best_c < 0) best_c = 0;
-        if (row < n) {
-          const size_t o = static_cast<size_t>(head) * n + row;
-          prop_g[o] = best_c;
-          prop_v[o] = best_v;
-        }
+        const size_t o = static_cast<size_t>(head) * n + row;
+        prop_g[o] = best_c;
+        prop_v[o] = best_v;
       }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
       if (__any_sync(0xffffffffu, nonfinite && !aborted) && lane == 0) record_error(status, kErrNonFinite);
     }
-    if (lane == 0) tc::bulk_wait_all();  // this warp's D stores have landed
-    __syncwarp();
   }
 
   tc::fence_before_sync();
@@ -394,13 +372,12 @@ cudaError_t launch_dist_tc(const RowGemmArgs& a, int ldd, cudaStream_t st) {
   const int total = a.heads * ceil_div(a.n, 128);
   const long long xrows = static_cast<long long>(a.heads) * a.n, wrows = static_cast<long long>(a.heads) * a.ncols;
   if (xrows > 0x7fffffffLL || wrows > 0x7fffffffLL) return cudaErrorInvalidValue;  // TMA coordinates are int32
-  CUtensorMap tx, twh, twl, td;
+  CUtensorMap tx, twh, twl;
   if (!bf16_map(&tx, a.X, xrows, 128) || !bf16_map(&twh, a.Bhi, wrows, 128) ||
-      !bf16_map(&twl, split ? static_cast<const void*>(a.Blo) : static_cast<const void*>(a.Bhi), wrows, 128) ||
-      !f32_store_map(&td, a.Dout, ldd, xrows, 32))
+      !bf16_map(&twl, split ? static_cast<const void*>(a.Blo) : static_cast<const void*>(a.Bhi), wrows, 128))
     return cudaErrorInvalidValue;
   kern<<<std::min(total, sms), kDtThreads, smem, st>>>(
-      tx, a.n, twh, twl, td, a.ncols, ldd, a.nrm, a.ecol, a.tau2, a.Dout,
+      tx, a.n, twh, twl, a.ncols, ldd, a.nrm, a.ecol, a.tau2, a.Dout,
       a.prop_g, a.prop_v, a.seg_min, a.nseg, a.status, a.heads);
   return counted(cudaGetLastError(), 1);
 }

@@ -208,18 +208,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int 
       : "memory");
 }
 
-// TMA tiled store of the box at (col, row) of a 2-D tensor map from `src` (bulk group of
-// the issuing thread).  `col` times the element size must be a multiple of 16; the row
-// and column coordinates are never negative here.
-__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int col, int row) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
-                   reinterpret_cast<uint64_t>(tmap)),
-               "r"(col), "r"(row), "r"(src)
-               : "memory");
-}
-// Wait until at most one committed bulk group of this thread still reads shared memory.
-__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
-
 // Per-warpgroup register re-split.  Every warp of the warpgroup executes the same call;
 // the sum over warpgroups must stay within (threads x registers per thread at launch),
 // which the launcher checks against the compiled kernel before the first launch.
