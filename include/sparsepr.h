@@ -171,9 +171,12 @@ SPARSEPR_API int sparsepr_route(const float* block_scores, const int32_t* key_gs
                    int64_t* executed_pairs, void* ws, sparsepr_stream_t stream);
 
 /* (c) Block-sparse softmax attention.  Row i of query block b attends to the union of
- * the members of the k routed key groups of b, softmax renormalised over that support:
+ * the members of the routed key groups of b, softmax renormalised over that support:
  *   S_out[i] = sum_j softmax_j(tau q_i . k_j) v_j,  written fp32 in token order
- *   [Bt,H,N,d].  bf16 inputs run on tensor cores with fp32 accumulation. */
+ *   [Bt,H,N,d].  bf16 inputs run on tensor cores with fp32 accumulation.  route is
+ *   [Bt,H,Gq,k] as written by sparsepr_route (k its *k_out): every row's groups in
+ *   ascending order, each row ending at k entries or at its first -1 (global budget).
+ *   The same holds for the route argument of the calls below. */
 SPARSEPR_API int sparsepr_sparse_attn(const void* Q, const void* K, const void* V, int dtype,
                          int32_t Bt, int32_t H, int32_t N, int32_t d, int32_t block,
                          const int32_t* key_perm, const int32_t* key_gsize,

@@ -125,3 +125,19 @@ def test_one_call_entries_refuse_bad_arguments(L):
     s = ctypes.c_void_p(4096)
     rc = L.sparsepr_attention_host(ok, ok, ok, spr.BF16, 1, 2, 1024, 128, ctypes.byref(good), ok, 2, ok, s, s)
     assert rc == spr.ERR_INVALID_ARG and b"copy stream" in L.sparsepr_last_error()
+
+
+def test_call_workspace_holds_full_route_rows_under_the_global_budget():
+    """The one-call workspace sizes the route for k groups per block under the uniform
+    budget and for all G groups (rows padded with -1) under the global budget."""
+    L = spr.lib()
+    uni = spr.SparsePRConfig(block=128, n_sampled=512, n_probe=256, density=0.22)
+    glo = spr.SparsePRConfig(block=128, n_sampled=512, n_probe=256, density=0.22, route_budget=spr.BUDGET_GLOBAL)
+    n, h = 75600, 2
+    g = spr.num_groups(n, 128)
+    k = spr.route_k(n, 128, 0.22, 256)
+    a = int(L.sparsepr_call_workspace_size(spr.BF16, 1, h, n, 128, ctypes.byref(uni.c())))
+    b = int(L.sparsepr_call_workspace_size(spr.BF16, 1, h, n, 128, ctypes.byref(glo.c())))
+    assert a > 0 and b > a
+    assert b - a >= 4 * h * g * (g - k)  # the extra route columns, before alignment
+    assert b - a <= 4 * h * g * (g - k) + 4096
