@@ -485,11 +485,17 @@ def test_global_budget_call_parity():
     w = CONFIGS["small"]
     cfg = spr_cfg(w, route_budget=spr.BUDGET_GLOBAL)
     _, parts = _check_call(w, cfg, heads=2)
-    n = w.n_tokens
+    lens = _check_global_routes(parts, cfg, w.n_tokens)
+    assert min(lens) < max(lens), "the global allocation should give blocks different group counts here"
+
+
+def _check_global_routes(parts, cfg, n):
+    """Routes of every head equal the oracle's global allocation of the GPU's own block
+    scores; returns the routed-group count of every block."""
     part = parts["partition"]
     rt = parts["route"].cpu().numpy()
     lens = []
-    for h in range(2):
+    for h in range(rt.shape[1]):
         sc = part.block_scores[0, h].cpu().numpy()
         ks, bs = part.key_gsize[0, h].cpu().numpy(), part.qblock_size[0, h].cpu().numpy()
         want = O.route_global(sc, ks, bs, n, cfg.n_probe, cfg.density)
@@ -497,8 +503,23 @@ def test_global_budget_call_parity():
             got = _route_rows(rt[0, h, b])
             assert np.array_equal(got, want[b])
             lens.append(got.size)
-        assert int(parts["executed_pairs"][0, h]) <= math.floor(cfg.density * n * n)
-    assert min(lens) < max(lens), "the global allocation should give blocks different group counts here"
+    return lens
+
+
+@pytest.mark.parametrize("path", ["fp32_simt", "bf16_d64_b64"])
+def test_global_budget_other_kernel_paths(path):
+    """-1-padded route rows through the fp32 SIMT kernels (Tiny) and the bf16 mma.sync
+    kernels at d = 64, B = 64 on a ragged N: full parity with the oracle on the GPU's
+    decisions, routes equal to the oracle's global allocation."""
+    if path == "fp32_simt":
+        w = CONFIGS["tiny"]
+        cfg = spr_cfg(w, route_budget=spr.BUDGET_GLOBAL)
+        _, parts = _check_call(w, cfg, tol=TOL_F32, map_tol=1e-4)
+    else:
+        w = CONFIGS["tiny"].with_(grid=(3, 15, 22), dtype="bf16")     # N = 990
+        cfg = spr_cfg(w, n_probe=40, route_budget=spr.BUDGET_GLOBAL)
+        _, parts = _check_call(w, cfg)
+    _check_global_routes(parts, cfg, w.n_tokens)
 
 
 @pytest.mark.parametrize("cfg_name,heads", [("small", 3), ("tiny", None)])
