@@ -1,5 +1,6 @@
 // extern "C" entry points of libsparsepr (see include/sparsepr.h for the contract).
 #include <cmath>
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <atomic>
@@ -355,8 +356,11 @@ int sparsepr_route(const float* block_scores, const int32_t* key_gsize, const in
   const long long probe_pairs = static_cast<long long>(p->n_probe) * N;
   if (p->route_budget == SPARSEPR_BUDGET_GLOBAL) {
     // floor(rho N^2 - P N) in IEEE double, in this order
-    const double budget = std::floor(p->density * static_cast<double>(N) * static_cast<double>(N) -
-                                     static_cast<double>(probe_pairs));
+    if (!std::isfinite(p->density)) return fail(SPARSEPR_ERR_INVALID_ARG, "density must be finite");
+    double budget = std::floor(p->density * static_cast<double>(N) * static_cast<double>(N) -
+                               static_cast<double>(probe_pairs));
+    // a head has at most N^2 <= 2^60 pairs: clamping the budget there changes no decision
+    budget = std::min(std::max(budget, -0x1p61), 0x1p61);
     if (k_out) *k_out = G;
     SPR_CUDA(spr::launch_route_global(block_scores, Bt * H, G, G, static_cast<long long>(budget), route, key_gsize,
                                       qblock_size, reinterpret_cast<long long*>(executed_pairs), probe_pairs,

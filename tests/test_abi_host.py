@@ -74,6 +74,10 @@ def test_argument_errors_return_codes_without_launching(L):
     rc = L.sparsepr_route(fake, fake, fake, 1, 1, 1024, ctypes.byref(bad), fake, ctypes.byref(k_out), None, fake, None)
     assert rc == spr.ERR_INVALID_ARG
     assert b"route_budget" in L.sparsepr_last_error()
+    bad = spr.SparsePRConfig(route_budget=spr.BUDGET_GLOBAL, density=float("nan")).c()
+    rc = L.sparsepr_route(fake, fake, fake, 1, 1, 1024, ctypes.byref(bad), fake, ctypes.byref(k_out), None, fake, None)
+    assert rc == spr.ERR_INVALID_ARG
+    assert b"density" in L.sparsepr_last_error()
 
 
 def test_params_struct_layout():
