@@ -159,8 +159,9 @@ SPARSEPR_API int sparsepr_partition(const void* Q, const void* K, int dtype, int
  * the largest block score (ties to the lower group index), written in ascending group
  * order, with k = sparsepr_route_k(N, B, density, P).  GLOBAL budget: the groups that
  * the head-wide allocation (SPARSEPR_BUDGET_GLOBAL) gives each block, in ascending
- * order, then -1 up to k = G.  The row capacity k is returned in *k_out (host memory);
- * the attention and probe calls take it and stop at the first -1.
+ * order, then -1 up to k = G (at most 8192 groups per head, else UNSUPPORTED; density
+ * must be finite, else INVALID_ARG).  The row capacity k is returned in *k_out (host
+ * memory); the attention and probe calls take it and stop at the first -1.
  *   route          [Bt,H,Gq,k] int32
  *   executed_pairs [Bt,H] int64 = sum_b qblock_size[b] * sum_{g in route(b)} key_gsize[g]
  *                  + P*N: every evaluated (query, key) pair, probe rows counted.
