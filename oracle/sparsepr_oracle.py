@@ -36,7 +36,7 @@ the order the pages give it:
  10. metric: per-row relative L2 error against dense, mean over unprobed rows [abs];
      the p99 tail is reported too                                            [news]
 
-Readings taken where the pages are silent (each one is listed in the design doc):
+Readings taken where the pages are silent:
 
 * sample and probe rows: midpoint stride floor((2m+1) N / (2 count)) in raster order;
 * response = scaled logit tau q.k (a per-query shift would not change k-means);
@@ -49,12 +49,16 @@ Readings taken where the pages are silent (each one is listed in the design doc):
 * weights w_p = 1 / max(|d_p|^2, 1e-30) normalised to sum P, so the weighted
   least-squares objective is the summed squared relative error on the probes;
 * subspace = top-r eigenvectors of the uncentred weighted residual second moment;
-* ridge: lambda * I added to the centred weighted Gram, bias unpenalised.
+* ridge: lambda * I added to the centred weighted Gram, bias unpenalised;
+* the other split of the pair budget (``route_global``): every block keeps its best
+  group, the other (block, group) pairs follow in descending score (ties to the lower
+  block, then group) while the cumulative n_b n_g fits the head's budget.
 
 Parity pins live in tests/test_oracle_pins.py (density-100% identity, brute-force
 masked attention, library dense attention, normal-equation ridge, eigh projectors,
 planted affine residual, brute-force metric, fill invariants and brute force,
-planted clusters, route invariants).  The absolute error level at 22 % density on
+planted clusters, route invariants, the global allocation's hand-worked fixture,
+invariants and single-block reduction).  The absolute error level at 22 % density on
 synthetic inputs has no pin on the pages: parity unpinned for that number.
 """
 from __future__ import annotations
