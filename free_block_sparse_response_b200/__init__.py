@@ -12,5 +12,6 @@ from .sparsepr import (  # noqa: F401
     Partition, SparsePRConfig, SparsePRError, apply_residual, attention, check,
     dense_attn, fit_residual, fit_residual_noalloc, lib, new_workspace, num_groups, partition, probe_dense, probe_rows, route, route_k,
     sparse_attn, sparse_attn_apply, fused_supported, reset_workspace, attention_call, attention_host, call_workspace,
-    host_workspace, test_fill, test_topk, workspace_size, row_errors, launch_count, kernel_timing, kernel_timing_read,
+    host_workspace, test_fill, test_topk, test_partition_trace, load_library, workspace_size, row_errors, launch_count,
+    kernel_timing, kernel_timing_read,
 )

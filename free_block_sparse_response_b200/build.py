@@ -33,15 +33,23 @@ def _sources():
     return srcs, deps
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+# Test build: the same sources with the cooperative fill's grid-barrier wait cut to zero,
+# so that an ordinary partition call makes that bounded wait run out (its error path
+# records SPARSEPR_ERR_TIMEOUT and returns; no GPU fault, nothing left in flight).
+WAITTEST_LIB_PATH = os.path.join(PKG_DIR, "libsparsepr_waittest.so")
+VARIANTS = {None: (LIB_PATH, []), "waittest": (WAITTEST_LIB_PATH, ["-DSPR_GRID_WAIT_LIMIT_NS=0ull"])}
+
+
+def build(force: bool = False, verbose: bool = False, variant=None) -> str:
+    lib_path, defines = VARIANTS[variant]
     srcs, deps = _sources()
-    if not force and os.path.exists(LIB_PATH):
-        lib_time = os.path.getmtime(LIB_PATH)
+    if not force and os.path.exists(lib_path):
+        lib_time = os.path.getmtime(lib_path)
         if all(os.path.getmtime(p) <= lib_time for p in deps):
-            return LIB_PATH
-    tmp = LIB_PATH + ".tmp"
+            return lib_path
+    tmp = lib_path + ".tmp"
     cmd = [_nvcc(), "-std=c++17", "-O3", "-lineinfo", *ARCH_FLAGS, "-Xcompiler", "-fPIC",
-           "-Xcompiler", "-fvisibility=hidden", "-shared", "-o", tmp,
+           "-Xcompiler", "-fvisibility=hidden", "-shared", "-o", tmp, *defines,
            f"-I{os.path.join(REPO_DIR, 'include')}", *srcs]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
@@ -51,9 +59,18 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     if verbose:
         print(res.stderr, file=sys.stderr)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, lib_path)
+    return lib_path
+
+
+def build_all(force: bool = False) -> None:
+    """The library and its wait-limit test build."""
+    for variant in VARIANTS:
+        build(force=force, variant=variant)
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    if "--all" in sys.argv:
+        build_all(force="--force" in sys.argv)
+    else:
+        print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))

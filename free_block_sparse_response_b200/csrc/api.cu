@@ -203,10 +203,11 @@ int sparsepr_reset_workspace(void* ws, sparsepr_stream_t stream) {
   return SPARSEPR_OK;
 }
 
-int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int32_t H, int32_t N, int32_t d,
-                       const sparsepr_params* p, const int32_t* sample_idx, int32_t* key_perm,
-                       int32_t* key_gsize, int32_t* query_perm, int32_t* qblock_size, float* block_scores,
-                       void* ws, sparsepr_stream_t stream) {
+// The partition; `tr` (test-only, may be null) receives copies of its internal state.
+static int partition_impl(const void* Q, const void* K, int dtype, int32_t Bt, int32_t H, int32_t N, int32_t d,
+                          const sparsepr_params* p, const int32_t* sample_idx, int32_t* key_perm,
+                          int32_t* key_gsize, int32_t* query_perm, int32_t* qblock_size, float* block_scores,
+                          const sparsepr_partition_trace* tr, void* ws, sparsepr_stream_t stream) {
   int rc;
   if ((rc = check_shape(Bt, H, N, d)) || (rc = check_dtype(dtype))) return rc;
   if (p == nullptr) return fail(SPARSEPR_ERR_INVALID_ARG, "null params");
@@ -238,6 +239,12 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
     SPR_CUDA(spr::launch_midpoint_stride(at<int>(ws, L.sample_idx), N, S, st), "partition: sample");
     sidx = at<int>(ws, L.sample_idx);
   }
+  // test-only copies of the internal state (nothing below reads them)
+  auto copy_out = [&](void* dst, const void* src, size_t bytes, const char* what) -> int {
+    if (dst != nullptr) SPR_CUDA(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st), what);
+    return SPARSEPR_OK;
+  };
+  if (tr && (rc = copy_out(tr->sample_idx, sidx, sizeof(int) * S, "trace: sample"))) return rc;
   float* gamma = at<float>(ws, L.gamma);
   __nv_bfloat16* ghi = at<__nv_bfloat16>(ws, L.gamma_hi);
   __nv_bfloat16* glo = at<__nv_bfloat16>(ws, L.gamma_lo);
@@ -276,7 +283,8 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
   fa.hdr = hdr;
 
   // One side of the partition: balanced k-means of the rows of X under metric gamma.
-  auto cluster = [&](const void* X, float* cent, int32_t* perm, int32_t* sizes) -> int {
+  auto cluster = [&](const void* X, float* cent, int32_t* perm, int32_t* sizes, float* tr_dist,
+                     int32_t* tr_labels) -> int {
     spr::RowGemmArgs ra{};
     ra.X = X;
     ra.f32 = f32;
@@ -310,7 +318,16 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
       ra.nseg = fa.nseg;
       ra.nrm_out = nullptr;
       SPR_CUDA(spr::launch_rowgemm(ra, true, st), "distances");
+      if (tr_dist != nullptr)
+        SPR_CUDA(cudaMemcpy2DAsync(tr_dist + static_cast<size_t>(t) * heads * N * G, sizeof(float) * G, dmat,
+                                   sizeof(float) * fa.ldd, sizeof(float) * G, static_cast<size_t>(heads) * N,
+                                   cudaMemcpyDeviceToDevice, st),
+                 "trace: distances");
       SPR_CUDA(spr::launch_fill(fa, st), "capacity fill");
+      if (tr_labels != nullptr &&
+          (rc = copy_out(tr_labels + static_cast<size_t>(t) * heads * N, fa.labels, sizeof(int) * heads * N,
+                         "trace: labels")))
+        return rc;
       SPR_CUDA(spr::launch_build_perm(fa.labels, N, G, B, heads, at<int>(ws, L.perm_cursor), at<int>(ws, L.perm_tmp),
                                       perm, sizes, status, st),
                "permutation");
@@ -322,19 +339,45 @@ int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int3
   float* cent_k = at<float>(ws, L.cent_k);
   float* cent_q = at<float>(ws, L.cent_q);
   // keys: profiles against the sampled queries -> gamma = Q_S^T Q_S (semantic: identity)
+  const size_t gamma_bytes = sizeof(float) * heads * d * d, cent_bytes = sizeof(float) * heads * G * d;
   if (semantic) SPR_CUDA(spr::launch_identity(gamma, heads, d, st), "identity metric");
   else SPR_CUDA(spr::launch_gram(Q, f32, static_cast<size_t>(N) * d, sidx, S, heads, d, gamma, st), "Q_S gram");
-  if ((rc = cluster(K, cent_k, key_perm, key_gsize))) return rc;
+  if (tr && (rc = copy_out(tr->key_gamma, gamma, gamma_bytes, "trace: key metric"))) return rc;
+  if ((rc = cluster(K, cent_k, key_perm, key_gsize, tr ? tr->key_dist : nullptr, tr ? tr->key_labels : nullptr)))
+    return rc;
+  if (tr && (rc = copy_out(tr->mu, cent_k, cent_bytes, "trace: mu"))) return rc;
   // queries: coordinates against the key-group mean keys -> gamma = mu^T mu (semantic:
   // the raw queries, identity)
   if (semantic) SPR_CUDA(spr::launch_identity(gamma, heads, d, st), "identity metric");
   else SPR_CUDA(spr::launch_gram(cent_k, true, static_cast<size_t>(G) * d, nullptr, G, heads, d, gamma, st), "mu gram");
-  if ((rc = cluster(Q, cent_q, query_perm, qblock_size))) return rc;
+  if (tr && (rc = copy_out(tr->query_gamma, gamma, gamma_bytes, "trace: query metric"))) return rc;
+  if ((rc = cluster(Q, cent_q, query_perm, qblock_size, tr ? tr->query_dist : nullptr,
+                    tr ? tr->query_labels : nullptr)))
+    return rc;
+  if (tr && (rc = copy_out(tr->qbar, cent_q, cent_bytes, "trace: qbar"))) return rc;
   SPR_CUDA(spr::launch_block_scores(cent_q, cent_k, G, heads, d, tau, block_scores, st), "block scores");
   SPR_CUDA(spr::launch_route_scores(p->route_scores, block_scores, K, N, heads, G, G, key_perm, key_gsize, cent_q, tau,
                                     st),
            "routing scores");
   return SPARSEPR_OK;
+}
+
+int sparsepr_partition(const void* Q, const void* K, int dtype, int32_t Bt, int32_t H, int32_t N, int32_t d,
+                       const sparsepr_params* p, const int32_t* sample_idx, int32_t* key_perm,
+                       int32_t* key_gsize, int32_t* query_perm, int32_t* qblock_size, float* block_scores,
+                       void* ws, sparsepr_stream_t stream) {
+  return partition_impl(Q, K, dtype, Bt, H, N, d, p, sample_idx, key_perm, key_gsize, query_perm, qblock_size,
+                        block_scores, nullptr, ws, stream);
+}
+
+int sparsepr_test_partition_trace(const void* Q, const void* K, int dtype, int32_t Bt, int32_t H, int32_t N,
+                                  int32_t d, const sparsepr_params* p, const int32_t* sample_idx, int32_t* key_perm,
+                                  int32_t* key_gsize, int32_t* query_perm, int32_t* qblock_size,
+                                  float* block_scores, const sparsepr_partition_trace* trace, void* ws,
+                                  sparsepr_stream_t stream) {
+  if (trace == nullptr) return fail(SPARSEPR_ERR_INVALID_ARG, "null trace");
+  return partition_impl(Q, K, dtype, Bt, H, N, d, p, sample_idx, key_perm, key_gsize, query_perm, qblock_size,
+                        block_scores, trace, ws, stream);
 }
 
 int sparsepr_route(const float* block_scores, const int32_t* key_gsize, const int32_t* qblock_size, int32_t Bt,
@@ -711,19 +754,41 @@ __device__ __align__(256) unsigned char g_fit_noalloc_scratch[kNoAllocScratchByt
 
 std::mutex g_noalloc_mutex;
 void* g_noalloc_base[kNoAllocMaxDevices] = {};
+void* g_noalloc_ctx[kNoAllocMaxDevices] = {};  // context the cached address belongs to
 
-// Device address of the static scratch array on the current device (looked up once).
+// The current context of the calling thread, through the driver entry point (the
+// runtime has no call for it); nullptr when the entry point is unavailable.
+void* current_context() {
+  using GetCurrent = int (*)(void**);
+  static GetCurrent fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<GetCurrent>(p);
+  }();
+  void* ctx = nullptr;
+  if (fn == nullptr || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
+
+// Device address of the static scratch array on the current device.  Looked up once per
+// device, and again when the device's context has changed since (a cudaDeviceReset
+// unloads the module, so the old address would point outside any live allocation).
 int noalloc_scratch(void** base) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "fit_noalloc: current device");
   if (dev < 0 || dev >= kNoAllocMaxDevices) return fail(SPARSEPR_ERR_UNSUPPORTED, "device index %d too large", dev);
+  void* ctx = current_context();  // nullptr before the runtime made a context current: look up again
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_base[dev] == nullptr) {
+  if (g_noalloc_base[dev] == nullptr || ctx == nullptr || ctx != g_noalloc_ctx[dev]) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_fit_noalloc_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "fit_noalloc: scratch address");
     g_noalloc_base[dev] = ptr;
+    g_noalloc_ctx[dev] = ctx;
   }
   *base = g_noalloc_base[dev];
   return SPARSEPR_OK;
@@ -734,7 +799,7 @@ int noalloc_scratch(void** base) {
 extern "C" int sparsepr_fit_residual_noalloc(const float* probe_sparse, const float* probe_out, const float* weights,
                                              int32_t Bt, int32_t H, int32_t d, int32_t P, double ridge_lambda,
                                              int32_t rank, int32_t weight_mode, float* M, float* beta,
-                                             sparsepr_stream_t stream) {
+                                             int32_t* status, sparsepr_stream_t stream) {
   int rc;
   if ((rc = check_shape(Bt, H, 1, d))) return rc;
   if (P < 1) return fail(SPARSEPR_ERR_INVALID_ARG, "P must be >= 1");
@@ -757,5 +822,7 @@ extern "C" int sparsepr_fit_residual_noalloc(const float* probe_sparse, const fl
   SPR_CUDA(spr::launch_fit(probe_sparse, probe_out, weights, Bt * H, d, P, ridge_lambda, rank, weight_mode, scratch, M,
                            beta, static_cast<int*>(base), st),
            "fit_noalloc");
+  if (status != nullptr)
+    SPR_CUDA(cudaMemcpyAsync(status, base, sizeof(int32_t), cudaMemcpyDeviceToDevice, st), "fit_noalloc: status");
   return SPARSEPR_OK;
 }

@@ -19,6 +19,15 @@ enum : int {
 // Every bounded wait gives up after this long and records kErrTimeout.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
+// Bound of the cooperative fill's grid barrier.  A build can shorten it (e.g.
+// -DSPR_GRID_WAIT_LIMIT_NS=0) so that an ordinary call's barrier waits run out and take
+// their error path: the barrier guards no asynchronous copy or tensor-core operation,
+// so giving up early leaves nothing in flight.
+#ifndef SPR_GRID_WAIT_LIMIT_NS
+#define SPR_GRID_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr uint64_t kGridWaitLimitNs = SPR_GRID_WAIT_LIMIT_NS;
+
 // The workspace starts with this block; the rest is carved per stage.
 struct WorkspaceHeader {
   int status;    // first device-side error since the last partition call, else 0
@@ -65,7 +74,7 @@ __device__ __forceinline__ bool grid_barrier(WorkspaceHeader* hdr, unsigned int 
     } else {
       uint64_t t0 = globaltimer_ns();
       while (ld_acquire_u32(&hdr->barrier_gen) == gen) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > kGridWaitLimitNs) {
           record_error(&hdr->status, kErrTimeout);
           s_ok = 0;
           break;

@@ -31,7 +31,7 @@ EXPORTED_SYMBOLS = (
     "sparsepr_test_topk", "sparsepr_row_errors", "sparsepr_launch_count", "sparsepr_fit_residual_noalloc",
     "sparsepr_kernel_timing", "sparsepr_kernel_timing_read", "sparsepr_test_fill_segmented",
     "sparsepr_sparse_attn_apply", "sparsepr_reset_workspace", "sparsepr_call_workspace_size", "sparsepr_attention",
-    "sparsepr_host_workspace_size", "sparsepr_attention_host",
+    "sparsepr_host_workspace_size", "sparsepr_attention_host", "sparsepr_test_partition_trace",
 )
 
 
@@ -83,11 +83,17 @@ _vp, _i32, _i64p, _f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctype
 def lib() -> ctypes.CDLL:
     """Load libsparsepr.so (raises if it has not been built)."""
     global _LIB
-    if _LIB is not None:
-        return _LIB
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"{LIB_PATH} is not built; run `python -m free_block_sparse_response_b200.build`")
-    L = ctypes.CDLL(LIB_PATH)
+    if _LIB is None:
+        _LIB = load_library(LIB_PATH)
+    return _LIB
+
+
+def load_library(path: str) -> ctypes.CDLL:
+    """Open a build of the library at ``path`` with every entry point's signature set
+    (``lib()`` opens the default build; the tests also open the wait-limit build)."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is not built; run `python -m free_block_sparse_response_b200.build`")
+    L = ctypes.CDLL(path)
     P = ctypes.POINTER(_CParams)
     sig = {
         "sparsepr_num_groups": (_i32, [_i32, _i32]),
@@ -123,19 +129,20 @@ def lib() -> ctypes.CDLL:
         "sparsepr_kernel_timing": (ctypes.c_int, [ctypes.c_int]),
         "sparsepr_kernel_timing_read": (ctypes.c_int, [_vp, _vp]),
         "sparsepr_fit_residual_noalloc": (ctypes.c_int, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, ctypes.c_double,
-                                                         _i32, _i32, _vp, _vp, _vp]),
+                                                         _i32, _i32, _vp, _vp, _vp, _vp]),
         "sparsepr_call_workspace_size": (ctypes.c_size_t, [ctypes.c_int, _i32, _i32, _i32, _i32, P]),
         "sparsepr_attention": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32, P, _vp, _vp,
                                               _vp]),
         "sparsepr_host_workspace_size": (ctypes.c_size_t, [ctypes.c_int, _i32, _i32, _i32, _i32, P, _i32]),
         "sparsepr_attention_host": (ctypes.c_int, [_vp, _vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32, P, _vp,
                                                    _i32, _vp, _vp, _vp]),
+        "sparsepr_test_partition_trace": (ctypes.c_int, [_vp, _vp, ctypes.c_int, _i32, _i32, _i32, _i32, P, _vp,
+                                                         _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
         fn.restype = res
         fn.argtypes = args
-    _LIB = L
     return L
 
 
@@ -320,14 +327,15 @@ def fit_residual(probe_sparse, probe_out, cfg: SparsePRConfig, ws: torch.Tensor,
 
 
 def fit_residual_noalloc(probe_sparse, probe_out, cfg: SparsePRConfig, m: torch.Tensor, beta: torch.Tensor,
-                         weights: Optional[torch.Tensor] = None):
+                         weights: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None):
     """The fit through the allocation-free entry point, for callers that cannot
     allocate device memory during the call: results go to the caller's m [Bt,H,d,d]
-    and beta [Bt,H,d]; scratch is the library's fixed static array (no workspace)."""
-    _need_cuda(probe_sparse, probe_out, m, beta, weights)
+    and beta [Bt,H,d]; scratch is the library's fixed static array (no workspace).
+    ``status``, a one-element int32 device tensor, receives the call's device status."""
+    _need_cuda(probe_sparse, probe_out, m, beta, weights, status)
     bt, h, p, d = probe_out.shape
     _call("sparsepr_fit_residual_noalloc", _p(probe_sparse), _p(probe_out), _p(weights), bt, h, d, p,
-          cfg.ridge_lambda, cfg.rank, cfg.weight_mode, _p(m), _p(beta), _stream(probe_out))
+          cfg.ridge_lambda, cfg.rank, cfg.weight_mode, _p(m), _p(beta), _p(status), _stream(probe_out))
     return m, beta
 
 
@@ -436,6 +444,43 @@ def test_topk(scores: torch.Tensor, k: int) -> torch.Tensor:
     _call("sparsepr_test_topk", _p(scores), h, gq, g, k, _p(rt), _p(ws), _stream(scores))
     check(ws)
     return rt
+
+
+class _CTrace(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in ("sample_idx", "key_gamma", "key_dist", "key_labels", "mu",
+                                                      "query_gamma", "query_dist", "query_labels", "qbar")]
+
+
+def test_partition_trace(q, k, cfg: SparsePRConfig, ws: Optional[torch.Tensor] = None, dists: bool = True):
+    """sparsepr_partition with its internal state captured: returns (Partition, dict of
+    device tensors: sample_idx [S], key_gamma / query_gamma [Bt*H,d,d], key_dist /
+    query_dist [T,Bt*H,N,G] (only when ``dists``), key_labels / query_labels [T,Bt*H,N],
+    mu / qbar [Bt*H,G,d])."""
+    _need_cuda(q, k, ws)
+    bt, h, n, d = q.shape
+    g, t, hh, dev = num_groups(n, cfg.block), cfg.kmeans_iters, bt * h, q.device
+    ws = new_workspace(bt, h, n, d, cfg, dev) if ws is None else ws
+    f32, i32 = torch.float32, torch.int32
+    tr = {"sample_idx": torch.empty(cfg.n_sampled, dtype=i32, device=dev),
+          "key_gamma": torch.empty(hh, d, d, dtype=f32, device=dev),
+          "key_labels": torch.empty(t, hh, n, dtype=i32, device=dev),
+          "mu": torch.empty(hh, g, d, dtype=f32, device=dev),
+          "query_gamma": torch.empty(hh, d, d, dtype=f32, device=dev),
+          "query_labels": torch.empty(t, hh, n, dtype=i32, device=dev),
+          "qbar": torch.empty(hh, g, d, dtype=f32, device=dev)}
+    if dists:
+        tr["key_dist"] = torch.empty(t, hh, n, g, dtype=f32, device=dev)
+        tr["query_dist"] = torch.empty(t, hh, n, g, dtype=f32, device=dev)
+    ct = _CTrace(**{name: (tr[name].data_ptr() if name in tr and tr[name].numel() else None)
+                    for name, _ in _CTrace._fields_})
+    out = Partition(
+        torch.empty(bt, h, g * cfg.block, dtype=i32, device=dev), torch.empty(bt, h, g, dtype=i32, device=dev),
+        torch.empty(bt, h, g * cfg.block, dtype=i32, device=dev), torch.empty(bt, h, g, dtype=i32, device=dev),
+        torch.empty(bt, h, g, g, dtype=f32, device=dev))
+    _call("sparsepr_test_partition_trace", _p(q), _p(k), _dtype_code(q), bt, h, n, d, ctypes.byref(cfg.c()), None,
+          *(_p(x) for x in out), ctypes.byref(ct), _p(ws), _stream(q))
+    check(ws)
+    return out, tr
 
 
 # ------------------------------------------------------------------ one-call entry points

@@ -272,17 +272,24 @@ SPARSEPR_API int sparsepr_fit_residual(const float* probe_sparse, const float* p
  * device array inside the library, held by every GPU that loads it until the process
  * exits.  Limit: 256 + 8 * Bt*H * (2 d^2 + P d + 4 d) bytes <= 32 MiB (d = 128, P = 256:
  * 63 heads); larger calls return SPARSEPR_ERR_UNSUPPORTED without launching.  The call
- * allocates nothing (no cudaMalloc/cudaFree).  The first call on each device looks up the
+ * allocates nothing (no cudaMalloc/cudaFree).  The first call on each device (and the
+ * first after the device's context changed, e.g. after cudaDeviceReset) looks up the
  * array's device address; make that first call before any stream capture.  Every call
  * shares the one array (it keeps the last call's contents; the kernel rewrites all of it
  * before reading it), so calls that overlap on the GPU race: serialise them, e.g. on one
- * stream.  Device-side failures (non-positive weight sum, a failed Cholesky) write M = 0
- * and beta = 0 for the head. */
+ * stream.
+ *   status  optional DEVICE int32 (NULL: not reported): receives this call's device
+ *           status on `stream` after the fit, SPARSEPR_OK or the first error code.  As in
+ *           sparsepr_fit_residual, a weight sum that is not positive records
+ *           SPARSEPR_ERR_INVALID_ARG and the head is fitted with uniform weights; a ridge
+ *           system whose Cholesky fails (lambda = 0 on a singular Gram) records
+ *           SPARSEPR_ERR_INVALID_ARG and writes M = 0, beta = 0 for the head. */
 SPARSEPR_API int sparsepr_fit_residual_noalloc(const float* probe_sparse, const float* probe_out,
                                                const float* weights, int32_t Bt, int32_t H,
                                                int32_t d, int32_t P, double ridge_lambda,
                                                int32_t rank, int32_t weight_mode, float* M,
-                                               float* beta, sparsepr_stream_t stream);
+                                               float* beta, int32_t* status,
+                                               sparsepr_stream_t stream);
 
 /* (d3) Apply: O_i = S_i + M S_i + beta for unprobed rows, O_p = probe_out_p for probe
  * rows.  O [Bt,H,N,d] in out_dtype.  O may alias S_out when out_dtype is F32. */
@@ -342,6 +349,40 @@ SPARSEPR_API int sparsepr_test_fill_segmented(const float* D, int32_t H, int32_t
                        int32_t cap, int32_t* labels, void* ws, sparsepr_stream_t stream);
 SPARSEPR_API int sparsepr_test_topk(const float* Sc, int32_t H, int32_t Gq, int32_t G, int32_t k,
                        int32_t* route, void* ws, sparsepr_stream_t stream);
+
+/* sparsepr_test_partition_trace: sparsepr_partition (same arguments, same kernels, same
+ * outputs) that also copies its internal state into the caller's DEVICE buffers, so the
+ * parity tests can compare every continuous quantity of Response-Coupled Partitioning
+ * with the oracle (SparsePR abstract: keys grouped by their responses to sampled
+ * queries, queries by their responses to the key-group centroids).  Any member may be
+ * NULL (not captured).  T = params->kmeans_iters, HH = Bt*H, G = ceil(N/B):
+ *   sample_idx   [S]           sampled query tokens used (midpoint stride or the given ones)
+ *   key_gamma    [HH,d,d]      head-dim metric of the key side, Q_S^T Q_S (identity: semantic)
+ *   key_dist     [T,HH,N,G]    fp32 distances handed to each key-side capacity fill, in
+ *                              response-space units tau^2 |x - c|_Gamma^2 (semantic:
+ *                              the raw squared distances |x - c|^2)
+ *   key_labels   [T,HH,N]      key-group labels after each fill
+ *   mu           [HH,G,d]      key-group mean keys after the last key iteration
+ *   query_gamma  [HH,d,d]      metric of the query side, mu^T mu (identity: semantic)
+ *   query_dist   [T,HH,N,G], query_labels [T,HH,N]: the same for the query side
+ *   qbar         [HH,G,d]      query-block mean queries after the last query iteration
+ * The copies are asynchronous on `stream` and do not change what the call computes. */
+typedef struct sparsepr_partition_trace {
+  int32_t* sample_idx;
+  float* key_gamma;
+  float* key_dist;
+  int32_t* key_labels;
+  float* mu;
+  float* query_gamma;
+  float* query_dist;
+  int32_t* query_labels;
+  float* qbar;
+} sparsepr_partition_trace;
+SPARSEPR_API int sparsepr_test_partition_trace(const void* Q, const void* K, int dtype, int32_t Bt, int32_t H,
+                       int32_t N, int32_t d, const sparsepr_params* params,
+                       const int32_t* sample_idx, int32_t* key_perm, int32_t* key_gsize,
+                       int32_t* query_perm, int32_t* qblock_size, float* block_scores,
+                       const sparsepr_partition_trace* trace, void* ws, sparsepr_stream_t stream);
 
 #ifdef __cplusplus
 }

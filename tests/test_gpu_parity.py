@@ -18,7 +18,10 @@ from synthetic import CONFIGS, make_inputs
 pytestmark = pytest.mark.gpu
 
 TOL_BF16 = 3e-3     # per-head output rel-L2, bf16 inputs / fp32 accumulation
-TOL_F32 = 1e-4      # fp32 inputs, fp32 SIMT arithmetic; the fit at P < d+1 amplifies rounding
+TOL_F32_S = 2e-5    # fp32 inputs, fp32 SIMT arithmetic: sparse output and probe rows (measured 3e-7)
+TOL_F32 = 1e-4      # fp32 inputs: fitted map and final output.  At P = 32 < d + 1 the ridge
+                    # Gram's smallest eigenvalues are lambda = 1e-3, so the 3e-7 input error
+                    # moves M and beta by up to 4e-5 (measured) and O by up to 3e-5
 TOL_MAP = 1e-3      # fitted M and beta, relative Frobenius
 TOL_PROBE = 2e-4    # probe rows: softmax weights carried at ~16 bits
 
@@ -176,7 +179,7 @@ def test_nan_scores_are_reported():
 
 # ------------------------------------------------------------------- whole-call parity
 
-def _check_call(w, cfg, seed=0, heads=None, tol=TOL_BF16, map_tol=TOL_MAP):
+def _check_call(w, cfg, seed=0, heads=None, tol=TOL_BF16, map_tol=TOL_MAP, s_tol=None):
     q, k, v = make_inputs(w, seed, heads=heads)
     n = w.n_tokens
     o, parts = run_call(w, q, k, v, cfg)
@@ -185,17 +188,22 @@ def _check_call(w, cfg, seed=0, heads=None, tol=TOL_BF16, map_tol=TOL_MAP):
         ref = oracle_on_gpu_decisions(q, k, v, parts, h, cfg, n)
         assert int(gpu_pairs[0, h]) == ref["executed_pairs"]
         s_gpu = parts["S"][0, h].cpu().numpy()
-        assert rel(s_gpu, ref["S"]) <= tol, f"head {h}: sparse output"
         pidx = ref["probe_idx"]
-        assert rel(parts["probe_out"][0, h].cpu().numpy(), ref["probe_out"]) <= TOL_PROBE
-        assert rel(parts["probe_sparse"][0, h].cpu().numpy(), ref["S"][pidx]) <= TOL_PROBE
+        e_s = rel(s_gpu, ref["S"])
+        e_po = rel(parts["probe_out"][0, h].cpu().numpy(), ref["probe_out"])
+        e_ps = rel(parts["probe_sparse"][0, h].cpu().numpy(), ref["S"][pidx])
         m_gpu, b_gpu = parts["M"][0, h].cpu().numpy(), parts["beta"][0, h].cpu().numpy()
         fit = ref["fit"]
-        if fit["eigengap"] > 1e-6:
-            assert rel(m_gpu, fit["M"]) <= map_tol, f"head {h}: M"
-            assert rel(b_gpu, fit["beta"]) <= map_tol, f"head {h}: beta"
+        e_m, e_b = rel(m_gpu, fit["M"]), rel(b_gpu, fit["beta"])
         o_gpu = o[0, h].double().cpu().numpy()
-        assert rel(o_gpu, ref["O"]) <= tol, f"head {h}: final output"
+        e_o = rel(o_gpu, ref["O"])
+        print(f"{w.name} head {h}: S {e_s:.3g} probe {e_po:.3g}/{e_ps:.3g} M {e_m:.3g} beta {e_b:.3g} O {e_o:.3g}")
+        assert e_s <= (tol if s_tol is None else s_tol), f"head {h}: sparse output"
+        assert e_po <= min(TOL_PROBE, s_tol or 1.0) and e_ps <= min(TOL_PROBE, s_tol or 1.0)
+        if fit["eigengap"] > 1e-6:
+            assert e_m <= map_tol, f"head {h}: M"
+            assert e_b <= map_tol, f"head {h}: beta"
+        assert e_o <= tol, f"head {h}: final output"
         # probe rows of O are the probe outputs, cast to the output dtype
         want = parts["probe_out"][0, h].to(o.dtype)
         assert torch.equal(o[0, h][parts["probe_idx"][0, h].long()].cpu(), want.cpu())
@@ -204,7 +212,7 @@ def _check_call(w, cfg, seed=0, heads=None, tol=TOL_BF16, map_tol=TOL_MAP):
 
 def test_call_tiny_fp32():
     w = CONFIGS["tiny"]
-    _check_call(w, spr_cfg(w), tol=TOL_F32, map_tol=1e-4)
+    _check_call(w, spr_cfg(w), tol=TOL_F32, map_tol=TOL_F32, s_tol=TOL_F32_S)
 
 
 def test_call_small_bf16():
@@ -364,9 +372,11 @@ def test_partition_label_agreement_with_oracle():
     ql = perm_labels(part.query_perm[0, 0].cpu().numpy(), part.qblock_size[0, 0].cpu().numpy(), n, w.block)
     ref = O.partition(q[0, 0].double().numpy(), k[0, 0].double().numpy(), 1 / math.sqrt(w.head_dim), w.block,
                       w.n_sampled, w.kmeans_iters)
-    key_agree = float((kl == ref["key_labels"]).mean())
-    print(f"key label agreement {key_agree:.3f}, query {(ql == ref['query_labels']).mean():.3f}")
-    assert key_agree > 0.5
+    key_agree, query_agree = float((kl == ref["key_labels"]).mean()), float((ql == ref["query_labels"]).mean())
+    print(f"key label agreement {key_agree:.4f}, query {query_agree:.4f}")
+    # measured 1.000 / 0.999: near-ties decided on bf16 hi + lo distances may flip a few
+    # tokens, and a flip moves a centroid for the later iterations
+    assert key_agree >= 0.99 and query_agree >= 0.98
 
 
 def test_semantic_partition_call_parity():
@@ -385,14 +395,16 @@ def test_semantic_partition_call_parity():
         ref = O.partition_semantic(q[0, h].double().numpy(), k[0, h].double().numpy(), 1 / math.sqrt(w.head_dim),
                                    w.block, w.kmeans_iters)
         key_agree, query_agree = float((kl == ref["key_labels"]).mean()), float((ql == ref["query_labels"]).mean())
-        print(f"semantic head {h}: key label agreement {key_agree:.3f}, query {query_agree:.3f}")
-        assert key_agree > 0.5 and query_agree > 0.5
+        print(f"semantic head {h}: key label agreement {key_agree:.4f}, query {query_agree:.4f}")
+        # measured keys 1.000 / 0.971, queries 1.000 / 1.000 on the two heads
+        assert key_agree >= 0.95 and query_agree >= 0.98
 
 
-@pytest.mark.parametrize("mode,name", [(1, "size_corrected"), (2, "lse")])
+@pytest.mark.parametrize("mode,name", [(0, "centroid"), (1, "size_corrected"), (2, "lse")])
 def test_routing_score_readings(mode, name):
-    """Size-corrected and LSE block scores against the oracle's on the GPU's own labels
-    (fp32 on the GPU, fp64 in the oracle), and the whole call on those routes."""
+    """Centroid (the method's default), size-corrected and LSE block scores against the
+    oracle's on the GPU's own labels (fp32 on the GPU, fp64 in the oracle), and the whole
+    call on those routes."""
     w = CONFIGS["small"]
     cfg = spr_cfg(w, route_scores=mode)
     q, k, v = make_inputs(w, 0, heads=2)
@@ -407,6 +419,30 @@ def test_routing_score_readings(mode, name):
                                g, name)
         got = part.block_scores[0, h].cpu().numpy()
         assert np.max(np.abs(got - ref)) <= 1e-4 * max(1.0, float(np.max(np.abs(ref))))
+
+
+def test_row_errors_metric_matches_oracle():
+    """The error metric kernel (per-row |o - o*| / |o*|, probe rows marked NaN) against
+    the oracle's rel_l2_errors on the same bf16 output and fp32 reference (Small, 3
+    heads): every unprobed row's error, the mean and the nearest-rank p99."""
+    w = CONFIGS["small"]
+    cfg = spr_cfg(w)
+    q, k, v = make_inputs(w, 0, heads=3)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o, parts = spr.attention(qd, kd, vd, cfg, return_parts=True)
+    dense = spr.dense_attn(qd, kd, vd, block=w.block)
+    err = spr.row_errors(o, dense, parts["probe_idx"])
+    spr.check(parts["ws"])
+    for h in range(3):
+        pidx = parts["probe_idx"][0, h].cpu().numpy()
+        ref = O.rel_l2_errors(o[0, h].double().cpu().numpy(), dense[0, h].double().cpu().numpy(), pidx)
+        e = err[0, h].double().cpu().numpy()
+        assert np.isnan(e[pidx]).all() and not np.isnan(np.delete(e, pidx)).any()
+        keep = np.delete(e, pidx)
+        assert np.max(np.abs(keep - ref["errors"]) / np.maximum(ref["errors"], 1e-30)) <= 1e-5
+        assert abs(float(keep.mean()) - ref["mean"]) <= 1e-6 * ref["mean"]
+        es = np.sort(keep)
+        assert abs(float(es[int(math.ceil(0.99 * es.size)) - 1]) - ref["p99"]) <= 1e-5 * ref["p99"]
 
 
 def test_nonfinite_input_is_reported():
@@ -514,7 +550,7 @@ def test_global_budget_other_kernel_paths(path):
     if path == "fp32_simt":
         w = CONFIGS["tiny"]
         cfg = spr_cfg(w, route_budget=spr.BUDGET_GLOBAL)
-        _, parts = _check_call(w, cfg, tol=TOL_F32, map_tol=1e-4)
+        _, parts = _check_call(w, cfg, tol=TOL_F32, map_tol=TOL_F32, s_tol=TOL_F32_S)
     else:
         w = CONFIGS["tiny"].with_(grid=(3, 15, 22), dtype="bf16")     # N = 990
         cfg = spr_cfg(w, n_probe=40, route_budget=spr.BUDGET_GLOBAL)

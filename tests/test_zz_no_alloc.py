@@ -41,19 +41,46 @@ def test_noalloc_fit_matches_workspace_fit_twice():
     ws = spr.new_workspace(1, heads, 4 * p, d, cfg, torch.device("cuda"))
     m = torch.empty(1, heads, d, d, device="cuda")
     beta = torch.empty(1, heads, d, device="cuda")
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
     for call, seed in enumerate((11, 12)):
         xs, dp = _probe_problem(seed, heads, p, d)
         m_ref, b_ref = spr.fit_residual(xs, dp, cfg, ws)
         spr.check(ws)
         torch.cuda.synchronize()
         free_before = torch.cuda.mem_get_info()[0]
-        spr.fit_residual_noalloc(xs, dp, cfg, m, beta)
+        spr.fit_residual_noalloc(xs, dp, cfg, m, beta, status=status)
         torch.cuda.synchronize()
         free_after = torch.cuda.mem_get_info()[0]
         if call == 1:   # the first call may load the library module that holds the array
             assert free_after == free_before, "the no-allocation call changed free device memory"
+        assert int(status.item()) == spr.OK, f"call {call}: device status"
         assert _rel(m, m_ref) <= TOL_FIT, f"call {call}: M"
         assert _rel(beta, b_ref) <= TOL_FIT, f"call {call}: beta"
+
+
+def test_noalloc_fit_zero_weights_fall_back_to_uniform_and_report():
+    """Caller weights that sum to zero: like the workspace fit, the call records
+    INVALID_ARG in its status and fits the heads with uniform weights, so M and beta
+    equal the uniform-weight fit of the same probes."""
+    heads, p, d = 2, 128, 128
+    cfg = spr.SparsePRConfig(n_probe=p, rank=16, ridge_lambda=1e-3)
+    cfg_u = spr.SparsePRConfig(n_probe=p, rank=16, ridge_lambda=1e-3, weight_mode=spr.WEIGHT_UNIFORM)
+    xs, dp = _probe_problem(13, heads, p, d)
+    zero_w = torch.zeros(1, heads, p, device="cuda")
+    ws = spr.new_workspace(1, heads, 4 * p, d, cfg, torch.device("cuda"))
+    m_ref, b_ref = spr.fit_residual(xs, dp, cfg_u, ws)
+    spr.check(ws)
+    m = torch.empty(1, heads, d, d, device="cuda")
+    beta = torch.empty(1, heads, d, device="cuda")
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    spr.fit_residual_noalloc(xs, dp, cfg, m, beta, weights=zero_w, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == spr.ERR_INVALID_ARG
+    assert _rel(m, m_ref) <= TOL_FIT and _rel(beta, b_ref) <= TOL_FIT
+    # the next call starts from a clear status word
+    spr.fit_residual_noalloc(xs, dp, cfg_u, m, beta, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == spr.OK
 
 
 def test_noalloc_fit_rejects_sizes_beyond_its_scratch():
