@@ -3,13 +3,18 @@
 
 A step is one whole SparsePR call (partition, routing, block-sparse attention, probe
 rows, fit, apply) on the video-DiT 720p-like workload: 40 heads x 75,600 tokens
-(21x45x80 grid), head dim 128, bf16, synthetic seeded latents.  Each rank runs its own
-independent call (weak scaling, no data-path collective).
+(21x45x80 grid), head dim 128, bf16, synthetic seeded latents.  On N GPUs the call's
+heads are split into N contiguous slices, one per rank (heads are independent problems:
+no data-path collective; the output stays sharded by head, as in head-parallel DiTs);
+the call's time is the slowest rank's (strong scaling).  ``--scaling weak`` instead
+gives every rank a whole call of its own.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle on a
-bounded sample of the same workload instead (the reference arm).
+``--gpus N`` without a torchrun environment re-launches itself under
+``torch.distributed.run`` with N ranks.  Rank 0 prints one JSON line.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload instead (the reference arm; rank 0 only).
 """
 from __future__ import annotations
 
@@ -49,6 +54,8 @@ def parse_args():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--study", choices=["ablation", "probe-budget", "routing"], default=None,
                     help="error studies instead of the timed run (one JSON line per variant)")
+    ap.add_argument("--scaling", choices=["strong", "weak"], default="strong",
+                    help="strong: one call's heads split over the ranks; weak: a whole call per rank")
     return ap.parse_args()
 
 
@@ -60,13 +67,28 @@ def workload(args):
     return w
 
 
-def config_block(w, args):
+def head_slice(heads, world, rank):
+    """Contiguous heads [lo, hi) of `rank` when one call's heads are split over `world`
+    ranks; slice sizes differ by at most one."""
+    if not 1 <= world <= heads or not 0 <= rank < world:
+        raise ValueError(f"cannot split {heads} heads over {world} ranks (rank {rank})")
+    return heads * rank // world, heads * (rank + 1) // world
+
+
+def parallelism(w, world, scaling):
+    if scaling == "weak":
+        return f"independent call per rank x{world}"
+    sizes = [hi - lo for lo, hi in (head_slice(w.heads, world, r) for r in range(world))]
+    return f"heads split over {world} rank(s), contiguous slices of {sizes} heads"
+
+
+def config_block(w, args, world=1):
     t, y, x = w.grid
     return {"workload": f"{w.name}: {w.heads} heads x {w.n_tokens} tokens ({t}x{y}x{x} grid), d={w.head_dim}, "
                         f"{w.dtype}, B={w.block}, S={w.n_sampled}, P={w.n_probe}, density={w.density}, "
                         f"lambda={w.ridge_lambda}, r={w.rank}, T={w.kmeans_iters}",
             "batch": w.batch, "heads": w.heads, "tokens": w.n_tokens, "head_dim": w.head_dim,
-            "parallelism": f"independent call per rank x{args.gpus}", "seed": args.seed,
+            "parallelism": parallelism(w, world, args.scaling), "seed": args.seed,
             "l2": "inputs (3 x 774 MB bf16) larger than the 126 MB L2; no flush needed"}
 
 
@@ -92,59 +114,116 @@ def job_throughput(units_per_rank_step, world, steps, seconds):
     return units_per_rank_step * world * steps / seconds
 
 
+def sum_over_ranks(value, world, device=None):
+    """Sum of a per-rank number over the process group (the value itself on one rank)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def gather_head_stats(stats, world):
+    """Per-head statistics of every rank's slice, concatenated in head order (ranks hold
+    contiguous slices in rank order); outside the timed region."""
+    if world == 1:
+        return list(stats)
+    import torch.distributed as dist
+    parts = [None] * world
+    dist.all_gather_object(parts, list(stats))
+    return [x for part in parts for x in part]
+
+
 # ------------------------------------------------------------------- CPU oracle sample
 
-def oracle_sample(w, seed=0):
-    """Time the fp64 oracle's stages on one head of the workload restricted to its
-    first frame and extrapolate to the full call by each stage's cost order.
+def oracle_inputs(w, seed=0):
+    """The first head of the seeded workload as fp64 arrays (the oracle's inputs)."""
+    from synthetic import make_inputs
+    q, k, v = make_inputs(w, seed, heads=1)
+    return tuple(x[0, 0].double().numpy() for x in (q, k, v))
+
+
+def oracle_sample(w, seed=0, row_div=64, inputs=None):
+    """Time the fp64 oracle on one FULL head of the workload, stage by stage, and scale
+    to the whole call.  Every scale factor is an exact operation-count ratio:
+
+    * the k-means distances and the sparse attention are per-row loops: timed on a
+      uniform sample of 1/row_div of the rows (of the query blocks for the attention)
+      and scaled by rows / sampled rows;
+    * the profiles, group means, capacity fill, coordinates, routing, probe rows, fit and
+      apply run in full (the fill on a full-size distance matrix formed outside the
+      timed region; only its shape and values matter to the fill's cost);
+    * one k-means iteration per side is timed and counted T times;
+    * heads are independent problems: x heads.
     Returns (seconds per full call, description, threads)."""
     import numpy as np
 
     from oracle import sparsepr_oracle as O
-    from synthetic import make_inputs
-    t_frames, gy, gx = w.grid
-    sub = w.with_(grid=(1, gy, gx), heads=1)
-    q, k, v = make_inputs(sub, seed)
-    q, k, v = (x[0, 0].double().numpy() for x in (q, k, v))
-    n_s, n = sub.n_tokens, w.n_tokens
+    q, k, v = oracle_inputs(w, seed) if inputs is None else inputs
+    n, B, T = w.n_tokens, w.block, w.kmeans_iters
+    G = O.n_groups(n, B)
     tau = 1.0 / math.sqrt(w.head_dim)
-    s_count = min(w.n_sampled, n_s)
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(n, max(n // row_div, 1), replace=False))
+    row_scale = n / rows.size
     tm = {}
-    t0 = time.perf_counter()
-    part = O.partition(q, k, tau, w.block, s_count, w.kmeans_iters)
-    tm["partition"] = time.perf_counter() - t0
-    kk = O.route_k(n_s, w.block, w.density, w.n_probe)
-    t0 = time.perf_counter()
-    routes = O.route(part["block_scores"], kk)
-    tm["route"] = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    s = O.sparse_attention(q, k, v, tau, part["key_labels"], part["query_labels"], routes)
-    tm["sparse"] = time.perf_counter() - t0
-    pidx = O.midpoint_stride(n_s, w.n_probe)
-    t0 = time.perf_counter()
-    d_probe = O.dense_attention_rows(q, k, v, tau, pidx)
-    tm["probes"] = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    fit = O.fit_residual(s[pidx], d_probe, w.ridge_lambda, w.rank)
-    tm["fit"] = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    O.apply_residual(s, fit["M"], fit["beta"], pidx, d_probe)
-    tm["apply"] = time.perf_counter() - t0
-    r = n / n_s
-    # partition: N*G*dims with G ~ N and dims S (keys) / G (queries) -> between N^2 and N^3;
-    # take N^2 (keys dominate at S fixed).  sparse ~ N*k*B ~ N^2.  probes ~ P*N.  apply ~ N.
-    scale = {"partition": r * r, "route": r * r, "sparse": r * r, "probes": r, "fit": 1.0, "apply": r}
-    per_head = sum(tm[x] * scale[x] for x in tm)
+
+    def timed(name, fn, scale=1.0):
+        t0 = time.perf_counter()
+        out = fn()
+        tm[name] = tm.get(name, 0.0) + (time.perf_counter() - t0) * scale
+        return out
+
+    def fill_input(x, cent):   # the full fp32 distance matrix the fill takes (untimed)
+        return ((x * x).sum(1)[:, None] - 2.0 * (x @ cent.T) + (cent * cent).sum(1)[None, :]).astype(np.float32)
+
+    def kmeans_side(name, x):
+        labels = timed(f"{name} k-means", lambda: O.chunk_labels(n, B))
+        cent = timed(f"{name} k-means", lambda: O.group_means(x, labels, G))
+        if T == 0:
+            return labels
+        timed(f"{name} k-means", lambda: O.squared_distances(x[rows], cent), row_scale * T)
+        d32 = fill_input(x, cent)
+        labels = timed(f"{name} k-means", lambda: O.fill(d32, B), T)
+        timed(f"{name} k-means", lambda: O.group_means(x, labels, G, previous=cent), T)
+        return labels
+
+    sidx = O.midpoint_stride(n, w.n_sampled)
+    prof = timed("key k-means", lambda: O.key_response_profiles(q, k, sidx, tau))
+    kl = kmeans_side("key", prof)
+    mu = timed("query k-means", lambda: O.group_means(k, kl, G))
+    coords = timed("query k-means", lambda: tau * (q @ mu.T))
+    ql = kmeans_side("query", coords)
+    scores = timed("route", lambda: O.group_means(coords, ql, G).astype(np.float32))
+    kk = O.route_k(n, B, w.density, w.n_probe)
+    routes = timed("route", lambda: O.route(scores, kk))
+    blocks = np.sort(rng.choice(G, max(G // row_div, 1), replace=False))
+    brows = np.flatnonzero(np.isin(ql, blocks))
+    s_rows = timed("sparse", lambda: O.sparse_attention(q[brows], k, v, tau, kl, ql[brows], routes),
+                   n / max(brows.size, 1))
+    pidx = O.midpoint_stride(n, w.n_probe)
+    d_probe = timed("probes", lambda: O.dense_attention_rows(q, k, v, tau, pidx))
+    # the fit takes the probe rows' sparse outputs (computed untimed; the sampled
+    # attention above already counts their cost within the rows' share)
+    s_probe = O.sparse_attention(q[pidx], k, v, tau, kl, ql[pidx], routes)
+    fit = timed("fit", lambda: O.fit_residual(s_probe, d_probe, w.ridge_lambda, w.rank))
+    s_full = np.zeros((n, w.head_dim))
+    s_full[brows] = s_rows
+    timed("apply", lambda: O.apply_residual(s_full, fit["M"], fit["beta"], pidx, d_probe))
+    per_head = sum(tm.values())
     full = per_head * w.heads * w.batch
     try:
         from threadpoolctl import threadpool_info
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:  # pragma: no cover
         threads = 1
-    desc = (f"fp64 oracle, 1 head, first frame ({n_s} tokens, S={s_count}, P={w.n_probe}); stage times "
-            + ", ".join(f"{x} {tm[x]:.2f}s" for x in tm)
-            + f"; extrapolated per stage (partition, route, sparse x(N/n)^2; probes, apply x N/n; fit x1) "
-              f"and x{w.heads * w.batch} heads")
+    desc = (f"fp64 oracle on one full head ({n} tokens, G={G}, S={w.n_sampled}, P={w.n_probe}, T={T}); "
+            f"k-means distances and sparse attention timed on 1/{row_div} of the rows / query blocks and "
+            f"scaled by the exact row ratio, one k-means iteration per side x T, the rest in full; "
+            f"per-head stage seconds " + ", ".join(f"{x} {tm[x]:.1f}" for x in tm)
+            + f"; x{w.heads * w.batch} heads (independent problems)")
     return full, desc, threads
 
 
@@ -154,8 +233,9 @@ def run_reference(args, w):
         return
     times = []
     desc = threads = None
+    inputs = oracle_inputs(w, args.seed)
     for i in range(args.warmup + args.steps):
-        full, desc, threads = oracle_sample(w, args.seed)
+        full, desc, threads = oracle_sample(w, args.seed, inputs=inputs)
         if i >= args.warmup:
             times.append(full)
     sec = statistics.mean(times)
@@ -239,6 +319,11 @@ def run_ours(args, w):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: the SparsePR call needs a CUDA device (none visible); "
+                         "the CPU oracle is timed with --impl reference")
+    strong = args.scaling == "strong"
+    lo, hi = head_slice(w.heads, world, rank) if strong else (0, w.heads)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
@@ -256,7 +341,10 @@ def run_ours(args, w):
         cpu_base = {"value": dense_flops(w) / cpu_sec / 1e12, "unit": UNIT, "cores": cpu_threads,
                     "kind": "oracle", "sample": cpu_desc}
 
-    q_h, k_h, v_h = make_inputs(w, args.seed + rank)
+    if strong:   # this rank's contiguous head slice of the one seeded call
+        q_h, k_h, v_h = (t[:, lo:hi].contiguous() for t in make_inputs(w, args.seed, heads=hi))
+    else:        # a whole call of its own
+        q_h, k_h, v_h = make_inputs(w, args.seed + rank)
     q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
     bt, h, n, d = q.shape
     sc = spr.SparsePRConfig(block=w.block, n_sampled=w.n_sampled, n_probe=w.n_probe, kmeans_iters=w.kmeans_iters,
@@ -341,7 +429,8 @@ def run_ours(args, w):
     kname = ("attn_tc_kernel<false, true> (block-sparse attention + fused correction, tcgen05)" if fused else
              "attn_tc_kernel<false, false> (block-sparse attention, tcgen05)")
     roofline = {"kernel": kname, "bound": "tensor", "achieved": achieved,
-                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak if achieved is not None else None, "traffic": DOMINANT_TRAFFIC_BYTES if (args.config == "video" and not args.heads and fused) else None,
+                "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak if achieved is not None else None, "traffic": (DOMINANT_TRAFFIC_BYTES * (hi - lo) / w.heads
+                            if (args.config == "video" and not args.heads and fused) else None),
                 "peak_source": peak_src, "kernel_ms": t_sparse * 1e3, "kernel_launches_timed": attn_kernel_n,
                 "per_launch_flops": sparse_flops}
     if attn_kernel_n == 0:  # shapes outside the tensor-core kernel (fp32, d = 64, B = 64)
@@ -367,8 +456,8 @@ def run_ours(args, w):
     spr.check(ws_host)
     del ws_host
     e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
-    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
-    d2h = o.numel() * o.element_size()
+    h2d = sum_over_ranks(float(sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))), world, dev)
+    d2h = sum_over_ranks(float(o.numel() * o.element_size()), world, dev)
 
     # ---- dense comparators and the error metric (outside the timed regions)
     # the uncorrected sparse output of the last timed call's decisions (metric only)
@@ -382,7 +471,7 @@ def run_ours(args, w):
         spr.dense_attn(q, k, v, block=w.block, out=dense)
     de1.record()
     torch.cuda.synchronize()
-    dense_ms = de0.elapsed_time(de1) / 2
+    dense_ms = max_over_ranks(de0.elapsed_time(de1) / 2, world, dev)
     sdpa_ms = None
     try:
         import torch.nn.functional as F
@@ -396,37 +485,47 @@ def run_ours(args, w):
         torch.cuda.synchronize()
         sdpa_ms = se0.elapsed_time(se1) / 2
     except Exception:
-        sdpa_ms = None
+        sdpa_ms = float("nan")
+    sdpa_ms = max_over_ranks(sdpa_ms, world, dev)   # every rank takes the collective
+    sdpa_ms = None if math.isnan(sdpa_ms) else sdpa_ms
     pidx = spr.probe_rows(n, sc.n_probe, bt, h, dev)
     err = spr.row_errors(o, dense, pidx)
     err_s = spr.row_errors(s_last, dense, pidx)
 
-    def summary(e):
-        means, p99s = [], []
+    def per_head(e):
+        """(mean, nearest-rank p99) of every head's unprobed-row errors on this rank."""
+        out = []
         for hh in range(h):
             x = e[0, hh]
             x = x[~torch.isnan(x)]
             xs, _ = torch.sort(x)
-            means.append(float(xs.double().mean()))
-            p99s.append(float(xs[max(math.ceil(0.99 * xs.numel()) - 1, 0)]))
-        return statistics.mean(means), statistics.mean(p99s)
+            out.append((float(xs.double().mean()), float(xs[max(math.ceil(0.99 * xs.numel()) - 1, 0)])))
+        return out
 
-    err_mean, err_p99 = summary(err)
-    s_mean, s_p99 = summary(err_s)
+    def summary(stats):
+        return statistics.mean(m for m, _ in stats), statistics.mean(p for _, p in stats)
+
+    err_mean, err_p99 = summary(gather_head_stats(per_head(err), world))
+    s_mean, s_p99 = summary(gather_head_stats(per_head(err_s), world))
     spr.check(ws)
+    pairs_all = sum_over_ranks(pairs, world, dev)
+    heads_all = w.heads * (world if not strong else 1)
 
-    value = job_throughput(dense_flops(w), world, args.steps, elapsed) / 1e12
-    e2e_value = job_throughput(dense_flops(w), world, args.steps, e2e_s) / 1e12
+    # strong: the ranks together make one call; weak: one call per rank
+    calls = 1 if strong else world
+    value = job_throughput(dense_flops(w), calls, args.steps, elapsed) / 1e12
+    e2e_value = job_throughput(dense_flops(w), calls, args.steps, e2e_s) / 1e12
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": args.scaling,
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded video-token latents)",
-                "config": config_block(w, args),
+                "config": config_block(w, args, world),
                 "err": {"mean_rel_l2_unprobed": err_mean, "p99_rel_l2_unprobed": err_p99,
                         "uncorrected_sparse_mean": s_mean, "uncorrected_sparse_p99": s_p99,
                         "reference": "same-family dense attention, fp32 output"},
-                "density": pairs / (float(n) ** 2 * h * bt), "k": last["k"],
-                "stage_ms": stage_ms, "step_ms": step_ms, "dense_ms": dense_ms, "sdpa_ms": sdpa_ms,
+                "density": pairs_all / (float(n) ** 2 * heads_all * bt), "k": last["k"],
+                "stage_ms": stage_ms, "step_ms": step_ms, "rank0_heads": [lo, hi],
+                "dense_ms": dense_ms, "sdpa_ms": sdpa_ms,
                 "speedup_vs_dense": dense_ms / ms_step,
                 "roofline": roofline, "cpu_baseline": cpu_base,
                 "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -578,9 +677,27 @@ def run_study_routing(args, w):
             del ws
 
 
+def relaunch_under_torchrun(args):
+    """`--gpus N` (N > 1) outside a torchrun environment: run this same command line as N
+    ranks of one node (rendezvous on 127.0.0.1); returns their exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     args = parse_args()
     w = workload(args)
+    world = int(os.environ.get("WORLD_SIZE", "0"))
+    if args.impl == "ours" and args.study is None:
+        if world == 0 and args.gpus > 1:
+            sys.exit(relaunch_under_torchrun(args))
+        if world > 1 and world != args.gpus:
+            raise SystemExit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}")
     if args.study == "ablation":
         run_study_ablation(args, w)
     elif args.study == "probe-budget":

@@ -69,7 +69,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct Layout {
   size_t header = 0, sample_idx, gamma, gamma_hi, gamma_lo, nrm, cent_k, cent_q, wf, whi, wlo, eg, dmat,
          prop_g0, prop_v0, labels, room, cnt, offs, cursor, closed, bucket, list0, list1, list_len, prop_g, prop_v,
-         perm_tmp, perm_cursor, qblk, partial, fit, kv_grouped, mhilo, segmin, total;
+         perm_tmp, perm_cursor, qblk, partial, fit, kv_grouped, mhilo, segmin, ovf, total;
 };
 
 Layout make_layout(int heads, int N, int d, int block, int S, int P) {
@@ -112,12 +112,13 @@ Layout make_layout(int heads, int N, int d, int block, int S, int P) {
   L.bucket = take(sizeof(unsigned long long) * H * n);
   L.list0 = take(sizeof(int) * H * n);
   L.list1 = take(sizeof(int) * H * n);
-  L.list_len = take(sizeof(int) * 4);
+  L.list_len = take(sizeof(int) * std::max<size_t>(4, 2 * H));
   L.prop_g = take(sizeof(int) * H * n);
   L.prop_v = take(sizeof(float) * H * n);
   L.perm_tmp = take(sizeof(int) * H * G * block);
   L.perm_cursor = take(sizeof(int) * H * G);
   L.qblk = take(sizeof(int) * H * n);
+  L.ovf = take(sizeof(int) * (H * G + 2));
   L.total = off;
   return L;
 }
@@ -260,8 +261,9 @@ static int partition_impl(const void* Q, const void* K, int dtype, int32_t Bt, i
   fa.ldd = dmat_ld(G);
   fa.prop_g0 = at<int>(ws, L.prop_g0);
   fa.prop_v0 = at<float>(ws, L.prop_v0);
-  // segment minima come from the tensor-core distance kernel (bf16, d = 128)
-  const bool seg = !f32 && d == 128;
+  // bf16, d = 128: the tensor-core assignment kernel (distances and fill in one launch)
+  const bool tc_assign = !f32 && d == 128;
+  const bool seg = false;
   fa.nseg = 2 * spr::ceil_div(G, 128);
   fa.seg_min = seg ? at<unsigned long long>(ws, L.segmin) : nullptr;
   fa.heads = heads;
@@ -317,13 +319,44 @@ static int partition_impl(const void* Q, const void* K, int dtype, int32_t Bt, i
       ra.seg_min = seg ? at<unsigned long long>(ws, L.segmin) : nullptr;
       ra.nseg = fa.nseg;
       ra.nrm_out = nullptr;
-      SPR_CUDA(spr::launch_rowgemm(ra, true, st), "distances");
+      if (tc_assign) {
+        // bf16, d = 128: proposals and fill in one tensor-core kernel, no distance matrix
+        // (the parity trace has it store the first round's rows)
+        spr::AssignArgs aa{};
+        aa.heads = heads;
+        aa.n = N;
+        aa.G = G;
+        aa.cap = B;
+        aa.tau2 = ra.tau2;
+        aa.nrm = nrm;
+        aa.ecol = eg;
+        aa.labels = fa.labels;
+        aa.room = fa.room;
+        aa.cnt = fa.cnt;
+        aa.offs = fa.offs;
+        aa.cursor = fa.cursor;
+        aa.closed = fa.closed;
+        aa.bucket = fa.bucket;
+        aa.list[0] = fa.list0;
+        aa.list[1] = fa.list1;
+        aa.list_len = fa.list_len;
+        aa.prop_g = fa.prop_g;
+        aa.prop_v = fa.prop_v;
+        aa.ovf_list = at<int>(ws, L.ovf);
+        aa.ovf_total = at<int>(ws, L.ovf) + static_cast<size_t>(heads) * G;
+        aa.Dout = tr_dist != nullptr ? dmat : nullptr;
+        aa.ldd = static_cast<int>(fa.ldd);
+        aa.hdr = hdr;
+        SPR_CUDA(spr::launch_assign_tc(static_cast<const __nv_bfloat16*>(X), whi, wlo, aa, st), "assignment");
+      } else {
+        SPR_CUDA(spr::launch_rowgemm(ra, true, st), "distances");
+      }
       if (tr_dist != nullptr)
         SPR_CUDA(cudaMemcpy2DAsync(tr_dist + static_cast<size_t>(t) * heads * N * G, sizeof(float) * G, dmat,
                                    sizeof(float) * fa.ldd, sizeof(float) * G, static_cast<size_t>(heads) * N,
                                    cudaMemcpyDeviceToDevice, st),
                  "trace: distances");
-      SPR_CUDA(spr::launch_fill(fa, st), "capacity fill");
+      if (!tc_assign) SPR_CUDA(spr::launch_fill(fa, st), "capacity fill");
       if (tr_labels != nullptr &&
           (rc = copy_out(tr_labels + static_cast<size_t>(t) * heads * N, fa.labels, sizeof(int) * heads * N,
                          "trace: labels")))

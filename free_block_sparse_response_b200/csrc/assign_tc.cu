@@ -1,0 +1,686 @@
+// Balanced k-means assignment on 5th-generation tensor cores (sm_100a): the capacity-B
+// fill of one k-means iteration with every proposal round's distances recomputed on
+// tcgen05, so that no distance matrix is ever stored.
+//
+// Source: SparsePR abstract (arXiv 2608.18484): keys are grouped by their responses to
+// sampled queries, queries by their responses to the key-group centroids.  Both are the
+// balanced k-means whose assignment is the proposal-round fill: every unplaced item
+// proposes to its nearest group with room (ties to the lower group), every group takes
+// its proposers in ascending (distance, token) order while it has room.  Distances are
+//     D[i][g] = tau^2 (n_i - 2 x_i . w_g + e_g),   w_g = Gamma c_g,  e_g = c_g . w_g,
+// the head-dim form of the squared response-space distance; w_g enters as bf16 hi + lo.
+//
+// One cooperative launch per iteration, one CTA per SM, all heads.  Each round:
+//   A. proposals: the unplaced items of every head, 256 at a time, are multiplied with the
+//      head's W in chunks of 128 groups (X by TMA -- 2-D boxes in the first round,
+//      tile::gather4 rows of the unplaced list after it -- W hi and lo double-buffered and
+//      used for both 128-row halves, which halves the W traffic from L2; two accumulators
+//      per stage, double-buffered, fill the 512 TMEM columns); the epilogue forms D exactly
+//      as above and keeps the first minimum over the OPEN groups (a full group's e_g is
+//      staged as +inf, so its D never wins a strict '<' scan): the item's proposal;
+//   B. per head: groups whose proposers fit their room take them all (room and full-group
+//      bit updated here); the others get bucket offsets and join the overflow list;
+//   C. every proposer of a group that takes all is placed; the others are scattered into
+//      their group's bucket as (D, token) keys;
+//   D. every overflowing group takes its room's worth of best proposers (radix select of
+//      the kth key) and is full; the rejected join the head's list for the next round.
+// A grid barrier separates the phases.  Every item's D row is the same fp32 numbers in
+// every round (same operands, same MMA sequence, same epilogue arithmetic), so the
+// decisions are the fill's decisions on that one matrix.  Warp roles in phase A: warp 0
+// loads, warp 2 issues the MMAs, warps 4-11 run the epilogue (two threads per row pair:
+// columns 0-63 and 64-127 of every chunk, rows r and r + 128); phases B-D use all 12
+// warps.  Per-head list lengths are staged in shared memory once per round.  Every wait is
+// bounded.  With Dout set, the first round also stores every item's D row (row stride
+// ldd) for the parity tests.
+#include <cuda.h>
+
+#include "attention.cuh"
+#include "common.cuh"
+#include "fill_select.cuh"
+#include "partition.cuh"
+#include "tcgen05.cuh"
+
+namespace spr {
+namespace {
+
+constexpr int kAsThreads = 384;
+constexpr int kAsWarps = kAsThreads / 32;
+constexpr int kAsRows = 256;                 // items per work item: two 128-row halves
+constexpr uint32_t kAsTile = 128 * 128 * 2;  // 128 rows x 128 bf16: two 64-column swizzled boxes
+constexpr uint32_t kAsWStage = 2 * kAsTile;  // one chunk of W: hi and lo
+constexpr uint32_t kAsTmemCols = 512;        // 2 stages x 2 halves x 128 fp32 columns
+constexpr int kAsMaxCols = 1024;             // groups per head
+constexpr int kAsMaxHeads = 1024;            // heads per launch (the launcher splits larger calls)
+constexpr float kAsInf = __builtin_huge_valf();
+
+enum : int { kXFull = 0, kXEmpty = 1, kWFull0 = 2, kWEmpty0 = 4, kAccFull0 = 6, kAccEmpty0 = 8, kDrain = 10, kBars = 11 };
+
+__device__ __forceinline__ uint64_t as_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void as_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t as_ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t as_fadd2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// Walks the heads in order for increasing positions (work items or list entries):
+// position p -> (head, position within the head), given per-head counts in shared memory.
+struct HeadWalk {
+  int h = 0, base = 0;
+  __device__ void seek(const int* cnt, int p, int& head, int& off) {
+    while (p >= base + cnt[h]) {
+      base += cnt[h];
+      ++h;
+    }
+    head = h;
+    off = p - base;
+  }
+};
+
+// One 64-column half-chunk of a row: D from the accumulator columns u, the first minimum
+// over the open groups merged into (best_v, best_c); u is overwritten with D.
+__device__ __forceinline__ void scan_half_chunk(uint32_t (&u)[64], const float* s_e, int c0, float tnr, float m2t,
+                                                float& best_v, int& best_c) {
+  const float4* e4 = reinterpret_cast<const float4*>(s_e + c0);
+  // four interleaved first-minimum scans over the columns j = t (mod 4), merged below
+  // (smaller value wins, equal values go to the lower column)
+  float cv[4] = {kAsInf, kAsInf, kAsInf, kAsInf};
+  int cc[4] = {-1, -1, -1, -1};
+  const uint64_t m2 = as_f32x2(m2t, m2t), tn2 = as_f32x2(tnr, tnr);
+#pragma unroll
+  for (int qq = 0; qq < 16; ++qq) {
+    const float4 e = e4[qq];
+    float v[4];
+    as_split(as_fadd2(as_ffma2(as_f32x2(__uint_as_float(u[4 * qq]), __uint_as_float(u[4 * qq + 1])), m2, tn2),
+                      as_f32x2(e.x, e.y)),
+             v[0], v[1]);
+    as_split(as_fadd2(as_ffma2(as_f32x2(__uint_as_float(u[4 * qq + 2]), __uint_as_float(u[4 * qq + 3])), m2, tn2),
+                      as_f32x2(e.z, e.w)),
+             v[2], v[3]);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      u[4 * qq + t] = __float_as_uint(v[t]);
+      if (v[t] < cv[t]) {
+        cv[t] = v[t];
+        cc[t] = 4 * qq + t;
+      }
+    }
+  }
+  float seg_v = cv[0];
+  int seg_c = cc[0];
+#pragma unroll
+  for (int t = 1; t < 4; ++t) {
+    if (cc[t] >= 0 && (seg_c < 0 || cv[t] < seg_v || (cv[t] == seg_v && cc[t] < seg_c))) {
+      seg_v = cv[t];
+      seg_c = cc[t];
+    }
+  }
+  if (seg_c >= 0 && seg_v < best_v) {  // chunks in ascending order: strictly smaller wins
+    best_v = seg_v;
+    best_c = c0 + seg_c;
+  }
+}
+
+__global__ void __launch_bounds__(kAsThreads, 1)
+    assign_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmXg,
+                     const __grid_constant__ CUtensorMap tmWhi, const __grid_constant__ CUtensorMap tmWlo,
+                     AssignArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bars[kBars];
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag, s_enf, s_remaining, s_total;
+  __shared__ float s_best_v[kAsRows];
+  __shared__ int s_best_c[kAsRows];
+  __shared__ int scan_tmp[kAsThreads];
+  __shared__ unsigned int hist[kAsWarps][256];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t sbase = (tc::saddr(smem_raw) + 1023u) & ~1023u;
+  const uint32_t sX = sbase;                       // two 128-row halves
+  const uint32_t sW[2] = {sbase + 2 * kAsTile, sbase + 2 * kAsTile + kAsWStage};
+  uint8_t* sgen = smem_raw + (sbase - tc::saddr(smem_raw)) + 2 * kAsTile + 2 * kAsWStage;
+  float* s_e = reinterpret_cast<float*>(sgen);                   // [kAsMaxCols]
+  int* s_len = reinterpret_cast<int*>(sgen + 4 * kAsMaxCols);     // [kAsMaxHeads] list lengths
+  int* s_tiles = s_len + kAsMaxHeads;                             // [kAsMaxHeads] work items per head
+  auto bar = [&](int i) { return tc::saddr(&bars[i]); };
+
+  const int n = a.n, G = a.G, heads = a.heads;
+  const int n_chunks = ceil_div(G, 128);
+  const int words = ceil_div(G, 32);
+  const unsigned int nblocks = gridDim.x;
+  const int gthread = blockIdx.x * kAsThreads + tid, nthreads = nblocks * kAsThreads;
+  const int gwarp = gthread >> 5, nwarps = nthreads >> 5;
+  int* status = &a.hdr->status;
+
+  if (tid == 0) {
+    tc::mbar_init(bar(kXFull), 1);
+    tc::mbar_init(bar(kXEmpty), 1);
+    for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(bar(kWFull0 + s), 1);
+      tc::mbar_init(bar(kWEmpty0 + s), 1);
+      tc::mbar_init(bar(kAccFull0 + s), 1);
+      tc::mbar_init(bar(kAccEmpty0 + s), 256);
+    }
+    tc::mbar_init(bar(kDrain), 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 2) {
+    tc::tmem_alloc(tc::saddr(&tmem_slot), kAsTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tbase = tmem_slot;
+  volatile int* abort_v = &abort_flag;
+
+  // ---- fill state: nothing placed, every group open with room B, no lists yet
+  {
+    const size_t items = static_cast<size_t>(heads) * n, groups = static_cast<size_t>(heads) * G;
+    for (size_t x = gthread; x < items; x += nthreads) a.labels[x] = -1;
+    for (size_t x = gthread; x < groups; x += nthreads) {
+      a.room[x] = a.cap;
+      a.cnt[x] = 0;
+      a.cursor[x] = 0;
+    }
+    for (size_t x = gthread; x < static_cast<size_t>(heads) * words; x += nthreads) a.closed[x] = 0u;
+    for (int x = gthread; x < 2 * heads; x += nthreads) a.list_len[x] = 0;
+    if (gthread < 2) a.ovf_total[gthread] = 0;
+  }
+  // Grid-wide step between phases: a CTA whose bounded wait gave up raises the abort
+  // word first, so every CTA leaves the rounds together (the status word may already
+  // hold another error, which the barrier alone would not stop on).
+  auto sync_grid = [&]() -> bool {
+    __syncthreads();
+    if (tid == 0 && *abort_v) atomicExch(&a.hdr->grid_abort, 1);
+    const bool ok = grid_barrier(a.hdr, nblocks);
+    return ok && *reinterpret_cast<volatile int*>(&a.hdr->grid_abort) == 0;
+  };
+  bool alive = sync_grid();
+
+  // pipeline counters, continued across rounds: work items and W chunks seen by this CTA
+  int it_prod = 0, it_mma = 0, it_epi = 0;
+  int last_q = -1, last_it = -1;  // producer: last W chunk and X tile issued
+  const int max_rounds = n + 2;
+  int cur = 0;
+  for (int round = 0; alive; ++round) {
+    const bool first = round == 0;
+    const int* list = a.list[cur];
+    const int par = round & 1;
+    // this round's list lengths and work items per head, and their total
+    for (int h = tid; h < heads; h += kAsThreads) {
+      const int len = first ? n : __ldcg(a.list_len + cur * heads + h);
+      s_len[h] = len;
+      s_tiles[h] = ceil_div(len, kAsRows);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int t = 0;
+      for (int h = lane; h < heads; h += 32) t += s_tiles[h];
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      if (lane == 0) s_total = t;
+    }
+    __syncthreads();
+    const int total = s_total;
+
+    // ---------------------------------------------------------------- A. proposals
+    if (warp == 0) {
+      // producer: the 256 rows of X (lane 0 four 2-D boxes, or every lane four gather4 of
+      // 4 rows), then per chunk the 128 rows of W hi and lo
+      HeadWalk hw;
+      for (int w = blockIdx.x; w < total; w += nblocks, ++it_prod) {
+        int h, t;
+        hw.seek(s_tiles, w, h, t);
+        const int off = t * kAsRows;
+        int ok = 1;
+        if (lane == 0 && it_prod >= 1 && !tc::mbar_wait(bar(kXEmpty), (it_prod - 1) & 1, abort_v, status)) ok = 0;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        if (lane == 0) tc::mbar_arrive_expect_tx(bar(kXFull), 2 * kAsTile);
+        __syncwarp();
+        if (first) {
+          if (lane == 0) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              tc::tma_load_2d(sX + j * kAsTile, &tmX, 0, h * n + off + 128 * j, bar(kXFull));
+              tc::tma_load_2d(sX + j * kAsTile + 128 * 128, &tmX, 64, h * n + off + 128 * j, bar(kXFull));
+            }
+          }
+        } else {
+          const int len = s_len[h];
+          const int* hl = list + static_cast<size_t>(h) * n;
+#pragma unroll
+          for (int g4 = 0; g4 < 2; ++g4) {
+            const int row = 8 * lane + 4 * g4;  // 0..255: rows row .. row + 3
+            int r4[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int e = off + row + j;
+              // rows past the list repeat the tile's first entry (loaded, never used)
+              r4[j] = h * n + __ldcg(hl + (e < len ? e : off));
+            }
+            const uint32_t dst = sX + (row >> 7) * kAsTile + (row & 127) * 128;
+            tc::tma_gather4(dst, &tmXg, 0, r4[0], r4[1], r4[2], r4[3], bar(kXFull));
+            tc::tma_gather4(dst + 128 * 128, &tmXg, 64, r4[0], r4[1], r4[2], r4[3], bar(kXFull));
+          }
+        }
+        last_it = it_prod;
+        if (lane == 0) {
+          for (int c = 0; c < n_chunks; ++c) {
+            const int q = it_prod * n_chunks + c, s = q & 1;
+            if (q >= 2 && !tc::mbar_wait(bar(kWEmpty0 + s), ((q >> 1) - 1) & 1, abort_v, status)) {
+              ok = 0;
+              break;
+            }
+            const int wrow = h * G + c * 128;
+            tc::mbar_arrive_expect_tx(bar(kWFull0 + s), kAsWStage);
+            tc::tma_load_2d(sW[s], &tmWhi, 0, wrow, bar(kWFull0 + s));
+            tc::tma_load_2d(sW[s] + 128 * 128, &tmWhi, 64, wrow, bar(kWFull0 + s));
+            tc::tma_load_2d(sW[s] + kAsTile, &tmWlo, 0, wrow, bar(kWFull0 + s));
+            tc::tma_load_2d(sW[s] + kAsTile + 128 * 128, &tmWlo, 64, wrow, bar(kWFull0 + s));
+            last_q = q;
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      }
+    } else if (warp == 2) {
+      // MMA issuer: per chunk and half, 8 k-steps of 16, each the hi and the lo product
+      if (lane == 0) {
+        constexpr uint32_t kId = tc::idesc_bf16(128, 128, false, false);
+        for (int w = blockIdx.x; w < total; w += nblocks, ++it_mma) {
+          if (!tc::mbar_wait(bar(kXFull), it_mma & 1, abort_v, status)) break;
+          tc::fence_proxy_async();
+          bool ok = true;
+          for (int c = 0; c < n_chunks; ++c) {
+            const int q = it_mma * n_chunks + c, s = q & 1;
+            if (!tc::mbar_wait(bar(kWFull0 + s), (q >> 1) & 1, abort_v, status) ||
+                (q >= 2 && !tc::mbar_wait(bar(kAccEmpty0 + s), ((q >> 1) - 1) & 1, abort_v, status))) {
+              ok = false;
+              break;
+            }
+            tc::fence_proxy_async();
+            tc::fence_after_sync();
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const uint32_t acc = tbase + s * 256 + j * 128;
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+                const uint64_t adesc = tc::sdesc_sw128(sX + j * kAsTile + koff, 16, 1024);
+                tc::mma_ss(acc, adesc, tc::sdesc_sw128(sW[s] + koff, 16, 1024), kId, kk > 0 ? 1u : 0u);
+                tc::mma_ss(acc, adesc, tc::sdesc_sw128(sW[s] + kAsTile + koff, 16, 1024), kId, 1u);
+              }
+            }
+            tc::mma_commit(bar(kWEmpty0 + s));
+            tc::mma_commit(bar(kAccFull0 + s));
+          }
+          if (!ok) break;
+          tc::mma_commit(bar(kXEmpty));
+        }
+      }
+      __syncwarp();
+    } else if (warp >= 4) {
+      // epilogue: for rows r and r + 128, D of the row's 64 columns of every chunk and the
+      // first minimum over the open groups, halves of the columns merged at the end
+      const int r = (warp & 3) * 32 + lane;  // row within each 128-row half == TMEM lane
+      const int half = (warp - 4) >> 2;
+      const int etid = tid - 128;
+      const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+      const float tau2 = a.tau2, m2t = -2.f * tau2;
+      int loaded_head = -1;
+      bool aborted = *abort_v != 0;
+      HeadWalk hw;
+      for (int w = blockIdx.x; w < total; w += nblocks, ++it_epi) {
+        int h, t;
+        hw.seek(s_tiles, w, h, t);
+        const int off = t * kAsRows;
+        if (h != loaded_head) {  // tau^2 e_g of this head, +inf for full groups and past G
+          asm volatile("bar.sync 1, 256;" ::: "memory");
+          if (etid == 0) s_enf = 0;
+          asm volatile("bar.sync 1, 256;" ::: "memory");
+          const unsigned int* cl = a.closed + static_cast<size_t>(h) * words;
+          for (int c = etid; c < n_chunks * 128; c += 256) {
+            float v = kAsInf;
+            if (c < G) {
+              const float e = tau2 * __ldcg(a.ecol + static_cast<size_t>(h) * G + c);
+              if (!isfinite(e)) s_enf = 1;
+              if (!((__ldcg(cl + (c >> 5)) >> (c & 31)) & 1u)) v = e;
+            }
+            s_e[c] = v;
+          }
+          asm volatile("bar.sync 1, 256;" ::: "memory");
+          loaded_head = h;
+        }
+        const int len = s_len[h];
+        bool row_ok[2];
+        size_t grow[2];
+        float tnr[2], best_v[2] = {kAsInf, kAsInf};
+        int best_c[2] = {-1, -1};
+        bool nonfinite = false;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int e = off + 128 * j + r;
+          row_ok[j] = e < len;
+          const int item = row_ok[j] ? (first ? e : __ldcg(list + static_cast<size_t>(h) * n + e)) : 0;
+          grow[j] = static_cast<size_t>(h) * n + item;
+          tnr[j] = row_ok[j] ? tau2 * __ldcg(a.nrm + grow[j]) : 0.f;
+          nonfinite |= row_ok[j] && (!isfinite(tnr[j]) || s_enf != 0);
+        }
+        for (int c = 0; c < n_chunks && !aborted; ++c) {
+          const int q = it_epi * n_chunks + c, s = q & 1;
+          const bool got = tc::mbar_wait(bar(kAccFull0 + s), (q >> 1) & 1, abort_v, status);
+          if (!__all_sync(0xffffffffu, got)) {
+            aborted = true;
+            break;
+          }
+          tc::fence_after_sync();
+          const int c0 = c * 128 + half * 64;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            uint32_t u[64];
+            const uint32_t buf = tbase + lane_off + s * 256 + j * 128 + half * 64;
+            tc::tmem_ld32(buf, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+            tc::tmem_ld32(buf + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+            tc::tmem_wait_ld();
+            if (j == 1) {  // both halves read: the accumulator stage is free again
+              tc::fence_before_sync();
+              tc::mbar_arrive(bar(kAccEmpty0 + s));
+            }
+            scan_half_chunk(u, s_e, c0, tnr[j], m2t, best_v[j], best_c[j]);
+            if (first && a.Dout != nullptr && row_ok[j]) {  // parity tests: the full row of D
+              float* dst = a.Dout + grow[j] * a.ldd + c0;
+#pragma unroll
+              for (int k4 = 0; k4 < 16; ++k4) {
+                if (c0 + 4 * k4 < a.ldd)
+                  *reinterpret_cast<float4*>(dst + 4 * k4) =
+                      make_float4(__uint_as_float(u[4 * k4]), __uint_as_float(u[4 * k4 + 1]),
+                                  __uint_as_float(u[4 * k4 + 2]), __uint_as_float(u[4 * k4 + 3]));
+              }
+            }
+          }
+        }
+        if (half == 1) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            s_best_v[128 * j + r] = best_v[j];
+            s_best_c[128 * j + r] = best_c[j];
+          }
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (half == 0 && !aborted) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            if (!row_ok[j]) continue;
+            float bv = best_v[j];
+            int bc = best_c[j];
+            const float v1 = s_best_v[128 * j + r];
+            const int c1 = s_best_c[128 * j + r];
+            // half 0 holds the lower 64 columns of every chunk: equal values go to it
+            if (c1 >= 0 && (bc < 0 || v1 < bv || (v1 == bv && c1 < bc))) {
+              bv = v1;
+              bc = c1;
+            }
+            if (bc < 0) {  // every open group at +inf (or NaN): the lowest open group
+              const unsigned int* cl = a.closed + static_cast<size_t>(h) * words;
+              for (int wd = 0; wd < words && bc < 0; ++wd) {
+                const unsigned int open = ~__ldcg(cl + wd);
+                if (open != 0u) {
+                  const int g = wd * 32 + __ffs(open) - 1;
+                  if (g < G) bc = g;
+                }
+              }
+              if (bc < 0) {  // no open group: more items than room (cannot happen)
+                record_error(status, kErrInvalidArg);
+                bc = 0;
+              }
+            }
+            a.prop_g[grow[j]] = bc;
+            a.prop_v[grow[j]] = bv;
+            atomicAdd(a.cnt + static_cast<size_t>(h) * G + bc, 1);
+          }
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (__any_sync(0xffffffffu, nonfinite && !aborted) && lane == 0) record_error(status, kErrNonFinite);
+        // after an abort the loop still runs to the end, skipping the work, so that every
+        // epilogue warp passes the same named barriers
+      }
+    }
+    __syncwarp();
+    alive = sync_grid();
+    if (!alive) break;
+
+    // ---------------------------------------------------------------- B. groups
+    // A group whose proposers fit its room takes them all now; an overflowing group gets
+    // the offset of its bucket (the head's overflow proposals are packed in group order)
+    // and joins the overflow list.
+    for (int h = blockIdx.x; h < heads; h += nblocks) {
+      int* cnt = a.cnt + static_cast<size_t>(h) * G;
+      int* room = a.room + static_cast<size_t>(h) * G;
+      int* offs = a.offs + static_cast<size_t>(h) * G;
+      const int per = ceil_div(G, kAsThreads);
+      const int g0 = tid * per, g1 = min(G, g0 + per);
+      int local = 0;
+      for (int g = g0; g < g1; ++g) {
+        const int c = __ldcg(cnt + g);
+        if (c > __ldcg(room + g)) local += c;
+      }
+      scan_tmp[tid] = local;
+      __syncthreads();
+      for (int o = 1; o < kAsThreads; o <<= 1) {
+        const int y = tid >= o ? scan_tmp[tid - o] : 0;
+        __syncthreads();
+        scan_tmp[tid] += y;
+        __syncthreads();
+      }
+      int run = scan_tmp[tid] - local;
+      for (int g = g0; g < g1; ++g) {
+        const int c = __ldcg(cnt + g), rm = __ldcg(room + g);
+        if (c > rm) {
+          offs[g] = run;
+          run += c;
+          a.ovf_list[atomicAdd(a.ovf_total + par, 1)] = h * G + g;
+        } else {
+          offs[g] = -1;
+          if (c > 0) {
+            room[g] = rm - c;
+            cnt[g] = 0;
+            if (rm == c) atomicOr(a.closed + static_cast<size_t>(h) * words + g / 32, 1u << (g % 32));
+          }
+        }
+      }
+      __syncthreads();
+    }
+    alive = sync_grid();
+    if (!alive) break;
+
+    // ---------------------------------------------------------------- C. place / scatter
+    {
+      int items = 0;
+      for (int h = 0; h < heads; ++h) items += s_len[h];
+      HeadWalk hw;
+      for (int x = gthread; x < items; x += nthreads) {
+        int h, e;
+        hw.seek(s_len, x, h, e);
+        const int i = first ? e : __ldcg(list + static_cast<size_t>(h) * n + e);
+        const size_t item = static_cast<size_t>(h) * n + i;
+        const int g = __ldcg(a.prop_g + item);
+        const size_t gi = static_cast<size_t>(h) * G + g;
+        const int o = __ldcg(a.offs + gi);
+        if (o < 0) {
+          a.labels[item] = g;
+        } else {
+          const int slot = atomicAdd(a.cursor + gi, 1);
+          a.bucket[static_cast<size_t>(h) * n + o + slot] = decision_key(__ldcg(a.prop_v + item), i);
+        }
+      }
+    }
+    alive = sync_grid();
+    if (!alive) break;
+
+    // ---------------------------------------------------------------- D. overflowing groups
+    const int next = cur ^ 1;
+    {
+      const int novf = __ldcg(a.ovf_total + par);
+      for (int j = gwarp; j < novf; j += nwarps) {
+        const int x = __ldcg(a.ovf_list + j);
+        const int h = x / G, g = x - h * G;
+        const int c = __ldcg(a.cnt + x), rm = __ldcg(a.room + x);
+        const unsigned long long* bk = a.bucket + static_cast<size_t>(h) * n + __ldcg(a.offs + x);
+        int* lab = a.labels + static_cast<size_t>(h) * n;
+        int* nlist = a.list[next] + static_cast<size_t>(h) * n;
+        int* nlen = a.list_len + next * heads + h;
+        // (rm = 0 only after a recorded error: nothing is taken then)
+        const unsigned long long thr = rm == 0 ? 0ull : warp_select_kth(bk, c, rm, hist[warp]);
+        for (int e0 = 0; e0 < c; e0 += 256) {
+          unsigned long long kb[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int e = e0 + u * 32 + lane;
+            kb[u] = e < c ? __ldcg(bk + e) : ~0ull;
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const bool valid = e0 + u * 32 + lane < c;
+            const int i = static_cast<int>(kb[u] & 0xffffffffu);
+            const bool take = valid && kb[u] <= thr;
+            if (take) lab[i] = g;
+            // rejected proposers join the head's next list, one atomic per warp
+            const unsigned int rej = __ballot_sync(0xffffffffu, valid && !take);
+            if (rej != 0u) {
+              const int leader = __ffs(rej) - 1;
+              int base = 0;
+              if (lane == leader) base = atomicAdd(nlen, __popc(rej));
+              base = __shfl_sync(0xffffffffu, base, leader);
+              if (valid && !take) nlist[base + __popc(rej & ((1u << lane) - 1u))] = i;
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) {
+          a.room[x] = 0;
+          a.cnt[x] = 0;
+          a.cursor[x] = 0;
+          atomicOr(a.closed + static_cast<size_t>(h) * words + g / 32, 1u << (g % 32));
+        }
+      }
+      if (blockIdx.x == 0 && tid == 0) a.ovf_total[par ^ 1] = 0;  // the next round's list
+    }
+    alive = sync_grid();
+    if (!alive) break;
+    if (warp == 0) {
+      int rem = 0;
+      for (int h = lane; h < heads; h += 32) rem += __ldcg(a.list_len + next * heads + h);
+      for (int o = 16; o > 0; o >>= 1) rem += __shfl_xor_sync(0xffffffffu, rem, o);
+      if (lane == 0) s_remaining = rem;
+    }
+    __syncthreads();
+    if (s_remaining == 0) break;
+    if (round >= max_rounds) {
+      if (gthread == 0) record_error(status, kErrTimeout);
+      break;
+    }
+    if (blockIdx.x == 0)
+      for (int h = tid; h < heads; h += kAsThreads) a.list_len[cur * heads + h] = 0;
+    cur = next;
+  }
+
+  // ---- drain: copies still in flight after an abort land, MMAs complete, TMEM freed
+  if (warp == 0 && lane == 0) {
+    auto drain = [&](uint32_t b, uint32_t parity) {
+      const uint64_t t0 = globaltimer_ns();
+      while (!tc::mbar_try_wait(b, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+      }
+    };
+    for (int q = last_q - 1; q <= last_q; ++q)
+      if (q >= 0) drain(bar(kWFull0 + (q & 1)), (q >> 1) & 1);
+    if (last_it >= 0) drain(bar(kXFull), last_it & 1);
+  }
+  if (warp == 2 && lane == 0) {
+    tc::mma_commit(bar(kDrain));
+    const uint64_t t0 = globaltimer_ns();
+    while (!tc::mbar_try_wait(bar(kDrain), 0)) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 2) {
+    __syncwarp();
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tbase, kAsTmemCols);
+  }
+}
+
+}  // namespace
+
+size_t assign_tc_smem_bytes() {
+  return 1024 + 2 * kAsTile + 2ull * kAsWStage + sizeof(float) * kAsMaxCols + 2 * sizeof(int) * kAsMaxHeads;
+}
+
+cudaError_t launch_assign_tc(const __nv_bfloat16* X, const __nv_bfloat16* Whi, const __nv_bfloat16* Wlo,
+                             const AssignArgs& a, cudaStream_t st) {
+  if (a.G < 1 || a.G > kAsMaxCols || a.n < 1 || a.heads < 1 || a.cap < 1 || (a.Dout != nullptr && a.ldd % 4 != 0))
+    return cudaErrorInvalidValue;
+  const size_t smem = assign_tc_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, assign_tc_kernel, kAsThreads, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const int words = ceil_div(a.G, 32);
+  // at most kAsMaxHeads heads per launch: larger calls run head slices one after another
+  for (int h0 = 0; h0 < a.heads; h0 += kAsMaxHeads) {
+    const int hc = std::min(kAsMaxHeads, a.heads - h0);
+    const size_t ni = static_cast<size_t>(h0) * a.n, gi = static_cast<size_t>(h0) * a.G;
+    AssignArgs s = a;
+    s.heads = hc;
+    s.nrm = a.nrm + ni;
+    s.ecol = a.ecol + gi;
+    s.labels = a.labels + ni;
+    s.room = a.room + gi;
+    s.cnt = a.cnt + gi;
+    s.offs = a.offs + gi;
+    s.cursor = a.cursor + gi;
+    s.closed = a.closed + static_cast<size_t>(h0) * words;
+    s.bucket = a.bucket + ni;
+    s.list[0] = a.list[0] + ni;
+    s.list[1] = a.list[1] + ni;
+    s.list_len = a.list_len + 2 * h0;
+    s.prop_g = a.prop_g + ni;
+    s.prop_v = a.prop_v + ni;
+    s.ovf_list = a.ovf_list + gi;
+    s.Dout = a.Dout != nullptr ? a.Dout + ni * a.ldd : nullptr;
+    const long long xrows = static_cast<long long>(hc) * a.n, wrows = static_cast<long long>(hc) * a.G;
+    if (xrows > 0x7fffffffLL || wrows > 0x7fffffffLL) return cudaErrorInvalidValue;  // TMA coordinates are int32
+    CUtensorMap tx, txg, twh, twl;
+    const __nv_bfloat16* Xs = X + ni * 128;
+    if (!bf16_map(&tx, Xs, xrows, 128) || !bf16_map(&txg, Xs, xrows, 1) ||
+        !bf16_map(&twh, Whi + gi * 128, wrows, 128) || !bf16_map(&twl, Wlo + gi * 128, wrows, 128))
+      return cudaErrorInvalidValue;
+    e = cudaMemsetAsync(&a.hdr->barrier_count, 0, 2 * sizeof(unsigned int), st);
+    if (e != cudaSuccess) return e;
+    void* params[] = {&tx, &txg, &twh, &twl, &s};
+    e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(assign_tc_kernel), dim3(sms), dim3(kAsThreads), params,
+                                    smem, st);
+    if ((e = counted(e, 1)) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace spr

@@ -31,7 +31,7 @@ constexpr uint64_t kGridWaitLimitNs = SPR_GRID_WAIT_LIMIT_NS;
 // The workspace starts with this block; the rest is carved per stage.
 struct WorkspaceHeader {
   int status;    // first device-side error since the last partition call, else 0
-  int detail;
+  int grid_abort;  // set by a CTA of a cooperative kernel whose bounded wait gave up
   unsigned int barrier_count;  // grid barrier of the cooperative fill kernel
   unsigned int barrier_gen;
   // Source of the group-ordered K / V copy in the workspace: K, V, key_perm, key_gsize

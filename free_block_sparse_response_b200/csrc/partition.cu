@@ -13,24 +13,11 @@
 // queries (coordinates u_i = tau mu q_i); c_g is the member mean in head-dim space,
 // whose image is the profile-space centroid because both maps are linear.
 #include "common.cuh"
+#include "fill_select.cuh"
 #include "partition.cuh"
 #include "warp_mma.cuh"
 
 namespace spr {
-
-__device__ __forceinline__ unsigned long long decision_key(float v, int idx) {
-  const uint32_t ok = (v != v) ? 0xffffffffu : float_order_key(v);
-  return (static_cast<unsigned long long>(ok) << 32) | static_cast<uint32_t>(idx);
-}
-
-__device__ __forceinline__ unsigned long long warp_min_u64(unsigned long long v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long y = __shfl_xor_sync(0xffffffffu, v, o);
-    v = y < v ? y : v;
-  }
-  return v;
-}
 
 // ----------------------------------------------------------------------- small kernels
 
@@ -411,120 +398,6 @@ __global__ void __launch_bounds__(256)
 // group); each group accepts its proposers in ascending (distance, token) order while
 // it has room.  One cooperative launch runs every round for every head.  Full groups
 // are tracked in a per-head bitmap so a proposal reads only its distance row.
-
-// Key of the kth smallest (1-based) of `count` distinct 64-bit keys, by a warp: radix
-// select on 8-bit digits, starting below the bits all keys share and stopping as soon
-// as the selected digit bin holds a single key.
-__device__ unsigned long long warp_select_kth(const unsigned long long* keys, int count, int kth,
-                                              unsigned int* hist) {
-  const int lane = threadIdx.x & 31;
-  unsigned long long kmin = ~0ull, kmax = 0ull;
-  for (int e0 = 0; e0 < count; e0 += 256) {
-    unsigned long long kb[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int e = e0 + u * 32 + lane;
-      kb[u] = e < count ? __ldcg(keys + e) : 0ull;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (e0 + u * 32 + lane < count) {
-        kmin = kb[u] < kmin ? kb[u] : kmin;
-        kmax = kb[u] > kmax ? kb[u] : kmax;
-      }
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const unsigned long long a = __shfl_xor_sync(0xffffffffu, kmin, o);
-    const unsigned long long b = __shfl_xor_sync(0xffffffffu, kmax, o);
-    kmin = a < kmin ? a : kmin;
-    kmax = b > kmax ? b : kmax;
-  }
-  if (kmin == kmax) return kmin;
-  const int top = 63 - __clzll(static_cast<long long>(kmin ^ kmax));  // highest differing bit
-  int shift = (top / 8) * 8;
-  unsigned long long prefix = shift + 8 >= 64 ? 0ull : (kmin & (~0ull << (shift + 8)));
-  for (; shift >= 0; shift -= 8) {
-    for (int b = lane; b < 256; b += 32) hist[b] = 0;
-    __syncwarp();
-    const unsigned long long hmask = shift + 8 >= 64 ? 0ull : (~0ull << (shift + 8));
-    for (int e0 = 0; e0 < count; e0 += 256) {
-      unsigned long long kb[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int e = e0 + u * 32 + lane;
-        kb[u] = e < count ? __ldcg(keys + e) : ~0ull;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (e0 + u * 32 + lane < count && (kb[u] & hmask) == prefix) atomicAdd(&hist[(kb[u] >> shift) & 255u], 1u);
-      }
-    }
-    __syncwarp();
-    unsigned int local[8];
-    unsigned int tot = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      local[j] = hist[8 * lane + j];
-      tot += local[j];
-    }
-    unsigned int incl = tot;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const unsigned int excl = incl - tot;
-    const bool mine = excl < static_cast<unsigned int>(kth) && static_cast<unsigned int>(kth) <= incl;
-    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
-    int digit = 0;
-    unsigned int before = 0, in_bin = 0;
-    if (mine) {
-      unsigned int acc = excl;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (acc + local[j] >= static_cast<unsigned int>(kth)) {
-          digit = 8 * lane + j;
-          before = acc;
-          in_bin = local[j];
-          break;
-        }
-        acc += local[j];
-      }
-    }
-    digit = __shfl_sync(0xffffffffu, digit, src);
-    before = __shfl_sync(0xffffffffu, before, src);
-    in_bin = __shfl_sync(0xffffffffu, in_bin, src);
-    kth -= static_cast<int>(before);
-    prefix |= static_cast<unsigned long long>(digit) << shift;
-    __syncwarp();
-    if (in_bin == 1 || shift == 0) {
-      // the kth key is the only key with this prefix: fetch it
-      const unsigned long long pmask = ~0ull << shift;
-      unsigned long long found = ~0ull;
-      for (int e0 = 0; e0 < count; e0 += 256) {
-        unsigned long long kb[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int e = e0 + u * 32 + lane;
-          kb[u] = e < count ? __ldcg(keys + e) : ~0ull;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          if (e0 + u * 32 + lane < count && (kb[u] & pmask) == prefix) found = kb[u];
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const unsigned long long y = __shfl_xor_sync(0xffffffffu, found, o);
-        found = y < found ? y : found;
-      }
-      return found;
-    }
-  }
-  return prefix;
-}
 
 __global__ void fill_init_kernel(FillArgs a) {
   const size_t items = static_cast<size_t>(a.heads) * a.n;

@@ -65,6 +65,33 @@ struct FillArgs {
   int d_vec4;           // set by the launcher: D rows start on 16-byte boundaries
 };
 
+// One balanced k-means assignment (the capacity fill) with the distances recomputed on
+// tcgen05 in every proposal round (bf16 items, d = 128, at most 1024 groups per head).
+struct AssignArgs {
+  int heads, n, G, cap;
+  float tau2;
+  const float* nrm;             // [heads, n]  x_i^T Gamma x_i
+  const float* ecol;            // [heads, G]  c_g^T Gamma c_g
+  int* labels;                  // [heads, n]  out: the group of every item
+  int* room;                    // [heads, G]
+  int* cnt;
+  int* offs;
+  int* cursor;
+  unsigned int* closed;         // [heads, ceil(G/32)]
+  unsigned long long* bucket;   // [heads, n]
+  int* list[2];                 // [heads, n] each: per-head lists of unplaced items
+  int* list_len;                // [2, heads]
+  int* prop_g;                  // [heads, n]
+  float* prop_v;
+  int* ovf_list;                // [heads, G]: the round's groups with more proposers than room
+  int* ovf_total;               // [2]: its length, alternating between rounds
+  float* Dout;                  // optional [heads, n, ldd]: the first round's D rows
+  int ldd;
+  WorkspaceHeader* hdr;
+};
+cudaError_t launch_assign_tc(const __nv_bfloat16* X, const __nv_bfloat16* Whi, const __nv_bfloat16* Wlo,
+                             const AssignArgs& a, cudaStream_t st);
+
 cudaError_t launch_midpoint_stride(int* idx, int n, int count, cudaStream_t st);
 // gamma [heads, d, d] = identity (the metric of the semantic partition)
 cudaError_t launch_identity(float* gamma, int heads, int d, cudaStream_t st);

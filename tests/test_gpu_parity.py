@@ -589,6 +589,24 @@ def test_host_entry_matches_device_call():
     assert torch.equal(o_host, o_dev.cpu())
 
 
+@pytest.mark.parametrize("world", [3, 8])
+def test_head_slices_concatenate_to_the_full_call(world):
+    """The multi-GPU split of one call: each rank's contiguous head slice, drawn as the
+    bench draws it (the first hi heads of the seeded input, then heads lo..hi), run as its
+    own call, concatenated over the ranks in order, equals the whole call bit for bit."""
+    import bench
+    w = CONFIGS["small"]
+    cfg = spr_cfg(w)
+    q, k, v = (t.cuda() for t in make_inputs(w, 4))
+    o_full = spr.attention_call(q, k, v, cfg)
+    pieces = []
+    for r in range(world):
+        lo, hi = bench.head_slice(w.heads, world, r)
+        qs, ks, vs = (t[:, lo:hi].contiguous().cuda() for t in make_inputs(w, 4, heads=hi))
+        pieces.append(spr.attention_call(qs, ks, vs, cfg))
+    assert torch.equal(torch.cat(pieces, dim=1), o_full)
+
+
 @pytest.mark.parametrize("grid,over", [((1, 10, 10), dict(n_sampled=32, n_probe=8, rank=4)),     # N 100: one group
                                       ((1, 3, 43), dict(n_sampled=32, n_probe=8, rank=4)),      # N 129: last group 1 token
                                       ((2, 8, 16), dict(n_sampled=64, n_probe=1, rank=1))])     # one probe row
