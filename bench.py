@@ -145,13 +145,14 @@ def oracle_inputs(w, seed=0):
     return tuple(x[0, 0].double().numpy() for x in (q, k, v))
 
 
-def oracle_sample(w, seed=0, row_div=64, inputs=None):
+def oracle_sample(w, seed=0, group_sample=16, block_div=64, inputs=None):
     """Time the fp64 oracle on one FULL head of the workload, stage by stage, and scale
-    to the whole call.  Every scale factor is an exact operation-count ratio:
+    to the whole call.  Every scale factor counts identical units of work:
 
-    * the k-means distances and the sparse attention are per-row loops: timed on a
-      uniform sample of 1/row_div of the rows (of the query blocks for the attention)
-      and scaled by rows / sampled rows;
+    * the k-means distances loop over the groups, each group's pass the same full-size
+      work (all N rows): timed on `group_sample` evenly spaced groups, scaled by G / that;
+    * the sparse attention loops over query blocks of equal work: timed on 1/block_div
+      of the blocks, scaled by N / their rows;
     * the profiles, group means, capacity fill, coordinates, routing, probe rows, fit and
       apply run in full (the fill on a full-size distance matrix formed outside the
       timed region; only its shape and values matter to the fill's cost);
@@ -166,8 +167,7 @@ def oracle_sample(w, seed=0, row_div=64, inputs=None):
     G = O.n_groups(n, B)
     tau = 1.0 / math.sqrt(w.head_dim)
     rng = np.random.default_rng(seed)
-    rows = np.sort(rng.choice(n, max(n // row_div, 1), replace=False))
-    row_scale = n / rows.size
+    gsel = np.unique(np.linspace(0, G - 1, min(group_sample, G)).astype(np.int64))
     tm = {}
 
     def timed(name, fn, scale=1.0):
@@ -184,7 +184,8 @@ def oracle_sample(w, seed=0, row_div=64, inputs=None):
         cent = timed(f"{name} k-means", lambda: O.group_means(x, labels, G))
         if T == 0:
             return labels
-        timed(f"{name} k-means", lambda: O.squared_distances(x[rows], cent), row_scale * T)
+        O.squared_distances(x, cent[gsel[:2]])   # untimed: the first large allocations of a process are slower
+        timed(f"{name} k-means", lambda: O.squared_distances(x, cent[gsel]), G / gsel.size * T)
         d32 = fill_input(x, cent)
         labels = timed(f"{name} k-means", lambda: O.fill(d32, B), T)
         timed(f"{name} k-means", lambda: O.group_means(x, labels, G, previous=cent), T)
@@ -199,7 +200,7 @@ def oracle_sample(w, seed=0, row_div=64, inputs=None):
     scores = timed("route", lambda: O.group_means(coords, ql, G).astype(np.float32))
     kk = O.route_k(n, B, w.density, w.n_probe)
     routes = timed("route", lambda: O.route(scores, kk))
-    blocks = np.sort(rng.choice(G, max(G // row_div, 1), replace=False))
+    blocks = np.sort(rng.choice(G, max(G // block_div, 1), replace=False))
     brows = np.flatnonzero(np.isin(ql, blocks))
     s_rows = timed("sparse", lambda: O.sparse_attention(q[brows], k, v, tau, kl, ql[brows], routes),
                    n / max(brows.size, 1))
@@ -220,8 +221,9 @@ def oracle_sample(w, seed=0, row_div=64, inputs=None):
     except Exception:  # pragma: no cover
         threads = 1
     desc = (f"fp64 oracle on one full head ({n} tokens, G={G}, S={w.n_sampled}, P={w.n_probe}, T={T}); "
-            f"k-means distances and sparse attention timed on 1/{row_div} of the rows / query blocks and "
-            f"scaled by the exact row ratio, one k-means iteration per side x T, the rest in full; "
+            f"k-means distances timed on {gsel.size} of the {G} groups (each a full pass over the rows) and "
+            f"scaled by G/{gsel.size}, sparse attention on 1/{block_div} of the query blocks scaled by rows, "
+            f"one k-means iteration per side x T, the rest in full; "
             f"per-head stage seconds " + ", ".join(f"{x} {tm[x]:.1f}" for x in tm)
             + f"; x{w.heads * w.batch} heads (independent problems)")
     return full, desc, threads

@@ -55,6 +55,13 @@ namespace {
 // row starts on a line and the distance kernel's 64-byte stores never split a sector.
 size_t dmat_ld(int G) { return static_cast<size_t>(G + 31) / 32 * 32; }
 
+// The tensor-core fill's stored tail rows: up to 32K unplaced items (of all heads), each
+// row a whole number of 128-group chunks.
+int tail_cap(int heads, int N) {
+  return static_cast<int>(std::min<long long>(1ll << 15, static_cast<long long>(heads) * N));
+}
+int tail_ld(int G) { return (G + 127) / 128 * 128; }
+
 
 #define SPR_CUDA(call, where)                       \
   do {                                              \
@@ -69,7 +76,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct Layout {
   size_t header = 0, sample_idx, gamma, gamma_hi, gamma_lo, nrm, cent_k, cent_q, wf, whi, wlo, eg, dmat,
          prop_g0, prop_v0, labels, room, cnt, offs, cursor, closed, bucket, list0, list1, list_len, prop_g, prop_v,
-         perm_tmp, perm_cursor, qblk, partial, fit, kv_grouped, mhilo, segmin, ovf, total;
+         perm_tmp, perm_cursor, qblk, partial, fit, kv_grouped, mhilo, segmin, ovf, dtail, tailpos, total;
 };
 
 Layout make_layout(int heads, int N, int d, int block, int S, int P) {
@@ -119,6 +126,8 @@ Layout make_layout(int heads, int N, int d, int block, int S, int P) {
   L.perm_cursor = take(sizeof(int) * H * G);
   L.qblk = take(sizeof(int) * H * n);
   L.ovf = take(sizeof(int) * (H * G + 2));
+  L.dtail = take(sizeof(float) * tail_cap(heads, N) * tail_ld(static_cast<int>(G)));
+  L.tailpos = take(sizeof(int) * H * n);
   L.total = off;
   return L;
 }
@@ -300,11 +309,18 @@ static int partition_impl(const void* Q, const void* K, int dtype, int32_t Bt, i
     ra.Blo = glo;
     ra.Bf32 = gamma;
     ra.nrm_out = nrm;
-    SPR_CUDA(spr::launch_rowgemm(ra, false, st), "row norms");
+    if (tc_assign)
+      SPR_CUDA(spr::launch_row_norms_tc(static_cast<const __nv_bfloat16*>(X), ghi, glo, heads, N, nrm, hdr, st),
+               "row norms");
+    else
+      SPR_CUDA(spr::launch_rowgemm(ra, false, st), "row norms");
     SPR_CUDA(spr::launch_chunk_perm(perm, sizes, N, G, B, heads, st), "chunk start");
     SPR_CUDA(spr::launch_centroid(X, f32, N, perm, sizes, G, B, heads, d, cent, st), "centroids");
-    for (int t = 0; t < p->kmeans_iters; ++t) {
+    if (p->kmeans_iters > 0)
       SPR_CUDA(spr::launch_wmat(cent, gamma, G, heads, d, wf, whi, wlo, eg, st), "gamma centroids");
+    int* members = at<int>(ws, L.perm_tmp);
+    int* msize = at<int>(ws, L.perm_cursor);
+    for (int t = 0; t < p->kmeans_iters; ++t) {
       ra.ncols = G;
       ra.Bhi = whi;
       ra.Blo = wlo;
@@ -342,9 +358,15 @@ static int partition_impl(const void* Q, const void* K, int dtype, int32_t Bt, i
         aa.list_len = fa.list_len;
         aa.prop_g = fa.prop_g;
         aa.prop_v = fa.prop_v;
+        aa.members = members;
+        aa.msize = msize;
         aa.ovf_list = at<int>(ws, L.ovf);
         aa.ovf_total = at<int>(ws, L.ovf) + static_cast<size_t>(heads) * G;
         aa.Dout = tr_dist != nullptr ? dmat : nullptr;
+        aa.Dtail = at<float>(ws, L.dtail);
+        aa.ldt = tail_ld(G);
+        aa.tail_cap = tail_cap(heads, N);
+        aa.tailpos = at<int>(ws, L.tailpos);
         aa.ldd = static_cast<int>(fa.ldd);
         aa.hdr = hdr;
         SPR_CUDA(spr::launch_assign_tc(static_cast<const __nv_bfloat16*>(X), whi, wlo, aa, st), "assignment");
@@ -361,10 +383,13 @@ static int partition_impl(const void* Q, const void* K, int dtype, int32_t Bt, i
           (rc = copy_out(tr_labels + static_cast<size_t>(t) * heads * N, fa.labels, sizeof(int) * heads * N,
                          "trace: labels")))
         return rc;
-      SPR_CUDA(spr::launch_build_perm(fa.labels, N, G, B, heads, at<int>(ws, L.perm_cursor), at<int>(ws, L.perm_tmp),
-                                      perm, sizes, status, st),
-               "permutation");
-      SPR_CUDA(spr::launch_centroid(X, f32, N, perm, sizes, G, B, heads, d, cent, st), "centroids");
+      // members (kept by the tensor-core fill, else scattered from the labels) -> sorted
+      // permutation, the new means and the next iteration's W and e
+      if (!tc_assign)
+        SPR_CUDA(spr::launch_perm_scatter(fa.labels, N, G, B, heads, msize, members, status, st), "members");
+      SPR_CUDA(spr::launch_group_update(X, f32, N, msize, members, G, B, heads, d, gamma, perm, sizes, cent, wf, whi,
+                                        wlo, eg, st),
+               "group update");
     }
     return SPARSEPR_OK;
   };

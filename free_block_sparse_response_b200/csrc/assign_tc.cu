@@ -31,7 +31,9 @@
 // columns 0-63 and 64-127 of every chunk, rows r and r + 128); phases B-D use all 12
 // warps.  Per-head list lengths are staged in shared memory once per round.  Every wait is
 // bounded.  With Dout set, the first round also stores every item's D row (row stride
-// ldd) for the parity tests.
+// ldd) for the parity tests.  Norm mode (nrm_out set, W = Gamma, G = d): one pass over all
+// items whose epilogue forms x_i^T Gamma x_i from the accumulator row and the item's own
+// row of the X tile in shared memory, and no fill.
 #include <cuda.h>
 
 #include "attention.cuh"
@@ -78,9 +80,11 @@ __device__ __forceinline__ uint64_t as_fadd2(uint64_t a, uint64_t b) {
 // position p -> (head, position within the head), given per-head counts in shared memory.
 struct HeadWalk {
   int h = 0, base = 0;
-  __device__ void seek(const int* cnt, int p, int& head, int& off) {
+  int ibase = 0;  // list entries of the heads passed (when `lens` is given)
+  __device__ void seek(const int* cnt, int p, int& head, int& off, const int* lens = nullptr) {
     while (p >= base + cnt[h]) {
       base += cnt[h];
+      if (lens != nullptr) ibase += lens[h];
       ++h;
     }
     head = h;
@@ -186,14 +190,16 @@ __global__ void __launch_bounds__(kAsThreads, 1)
   const uint32_t tbase = tmem_slot;
   volatile int* abort_v = &abort_flag;
 
+  const bool norm_mode = a.nrm_out != nullptr;
   // ---- fill state: nothing placed, every group open with room B, no lists yet
-  {
+  if (!norm_mode) {
     const size_t items = static_cast<size_t>(heads) * n, groups = static_cast<size_t>(heads) * G;
     for (size_t x = gthread; x < items; x += nthreads) a.labels[x] = -1;
     for (size_t x = gthread; x < groups; x += nthreads) {
       a.room[x] = a.cap;
       a.cnt[x] = 0;
       a.cursor[x] = 0;
+      a.msize[x] = 0;
     }
     for (size_t x = gthread; x < static_cast<size_t>(heads) * words; x += nthreads) a.closed[x] = 0u;
     for (int x = gthread; x < 2 * heads; x += nthreads) a.list_len[x] = 0;
@@ -208,13 +214,16 @@ __global__ void __launch_bounds__(kAsThreads, 1)
     const bool ok = grid_barrier(a.hdr, nblocks);
     return ok && *reinterpret_cast<volatile int*>(&a.hdr->grid_abort) == 0;
   };
-  bool alive = sync_grid();
+  bool alive = norm_mode ? true : sync_grid();
 
   // pipeline counters, continued across rounds: work items and W chunks seen by this CTA
   int it_prod = 0, it_mma = 0, it_epi = 0;
   int last_q = -1, last_it = -1;  // producer: last W chunk and X tile issued
   const int max_rounds = n + 2;
   int cur = 0;
+  // store_rows: this round's tensor-core pass also stores the unplaced items' D rows;
+  // tail: this round proposes from the stored rows (every CTA takes the same decision)
+  bool store_rows = false, tail = false;
   for (int round = 0; alive; ++round) {
     const bool first = round == 0;
     const int* list = a.list[cur];
@@ -236,7 +245,65 @@ __global__ void __launch_bounds__(kAsThreads, 1)
     const int total = s_total;
 
     // ---------------------------------------------------------------- A. proposals
-    if (warp == 0) {
+    if (tail) {
+      // a warp per unplaced item: the first minimum over the open groups of its stored
+      // row, by the epilogue's rule (strict '<' in ascending column order, so +inf and NaN
+      // never win; none finite: the lowest open group at +inf)
+      int items = 0;
+      for (int h = 0; h < heads; ++h) items += s_len[h];
+      HeadWalk hw;
+      for (int x = gwarp; x < items; x += nwarps) {
+        int h, e;
+        hw.seek(s_len, x, h, e);
+        const int i = __ldcg(list + static_cast<size_t>(h) * n + e);
+        const size_t grow = static_cast<size_t>(h) * n + i;
+        const float* row = a.Dtail + static_cast<size_t>(__ldcg(a.tailpos + grow)) * a.ldt;
+        const unsigned int* cl = a.closed + static_cast<size_t>(h) * words;
+        unsigned long long best = ~0ull;
+        int first_open = G;
+        // 16 words of the row and of the full-group bitmap requested before any is used
+        for (int w0 = 0; w0 < words; w0 += 16) {
+          float v[16];
+          unsigned int cw[16];
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int g = (w0 + u) * 32 + lane;
+            v[u] = g < G ? __ldcg(row + g) : kAsInf;
+            cw[u] = w0 + u < words ? __ldcg(cl + w0 + u) : ~0u;
+          }
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const int g = (w0 + u) * 32 + lane;
+            const bool open = g < G && !((cw[u] >> lane) & 1u);
+            if (open && v[u] < kAsInf) {
+              const unsigned long long key = decision_key(v[u], g);
+              best = key < best ? key : best;
+            }
+            const unsigned int om = __ballot_sync(0xffffffffu, open);
+            if (first_open == G && om != 0u) first_open = (w0 + u) * 32 + __ffs(om) - 1;
+          }
+        }
+        best = warp_min_u64(best);
+        if (lane == 0) {
+          int g;
+          float v;
+          if (best != ~0ull) {
+            g = static_cast<int>(best & 0xffffffffu);
+            v = __ldcg(row + g);
+          } else if (first_open < G) {
+            g = first_open;
+            v = kAsInf;
+          } else {  // no open group: more items than room (cannot happen)
+            record_error(status, kErrInvalidArg);
+            g = 0;
+            v = kAsInf;
+          }
+          a.prop_g[grow] = g;
+          a.prop_v[grow] = v;
+          atomicAdd(a.cnt + static_cast<size_t>(h) * G + g, 1);
+        }
+      }
+    } else if (warp == 0) {
       // producer: the 256 rows of X (lane 0 four 2-D boxes, or every lane four gather4 of
       // 4 rows), then per chunk the 128 rows of W hi and lo
       HeadWalk hw;
@@ -326,7 +393,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
             tc::mma_commit(bar(kAccFull0 + s));
           }
           if (!ok) break;
-          tc::mma_commit(bar(kXEmpty));
+          if (!norm_mode) tc::mma_commit(bar(kXEmpty));  // norm mode: the epilogue frees X
         }
       }
       __syncwarp();
@@ -343,8 +410,58 @@ __global__ void __launch_bounds__(kAsThreads, 1)
       HeadWalk hw;
       for (int w = blockIdx.x; w < total; w += nblocks, ++it_epi) {
         int h, t;
-        hw.seek(s_tiles, w, h, t);
+        hw.seek(s_tiles, w, h, t, s_len);
         const int off = t * kAsRows;
+        if (norm_mode) {
+          // x_i^T Gamma x_i: this thread's 64 accumulator columns (the 64-column box
+          // `half` of its row) dotted with the same columns of x_i from the X tile
+          const uint8_t* xs = smem_raw + (sX - tc::saddr(smem_raw)) + half * (128 * 128) + r * 128;
+          float part[2] = {0.f, 0.f};
+          const bool got = !aborted && tc::mbar_wait(bar(kAccFull0 + (it_epi & 1)), (it_epi >> 1) & 1, abort_v, status);
+          if (!__all_sync(0xffffffffu, got)) {
+            aborted = true;
+          } else {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              uint32_t u[64];
+              const uint32_t buf = tbase + lane_off + (it_epi & 1) * 256 + j * 128 + half * 64;
+              tc::tmem_ld32(buf, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+              tc::tmem_ld32(buf + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+              tc::tmem_wait_ld();
+              if (j == 1) {
+                tc::fence_before_sync();
+                tc::mbar_arrive(bar(kAccEmpty0 + (it_epi & 1)));
+              }
+#pragma unroll
+              for (int ch = 0; ch < 8; ++ch) {
+                const uint4 xv = *reinterpret_cast<const uint4*>(xs + j * kAsTile + ((ch ^ (r & 7)) << 4));
+                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[k]));
+                  part[j] = fmaf(__uint_as_float(u[8 * ch + 2 * k]), xf.x, part[j]);
+                  part[j] = fmaf(__uint_as_float(u[8 * ch + 2 * k + 1]), xf.y, part[j]);
+                }
+              }
+            }
+          }
+          if (half == 1) {
+            s_best_v[r] = part[0];
+            s_best_v[128 + r] = part[1];
+          }
+          asm volatile("bar.sync 1, 256;" ::: "memory");  // every X read of this item done
+          if (etid == 0 && !aborted) tc::mbar_arrive(bar(kXEmpty));
+          if (half == 0 && !aborted) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int e = off + 128 * j + r;
+              if (e < s_len[h]) a.nrm_out[static_cast<size_t>(h) * n + e] = part[j] + s_best_v[128 * j + r];
+            }
+          }
+          asm volatile("bar.sync 1, 256;" ::: "memory");
+          continue;
+        }
         if (h != loaded_head) {  // tau^2 e_g of this head, +inf for full groups and past G
           asm volatile("bar.sync 1, 256;" ::: "memory");
           if (etid == 0) s_enf = 0;
@@ -408,6 +525,14 @@ __global__ void __launch_bounds__(kAsThreads, 1)
                                   __uint_as_float(u[4 * k4 + 2]), __uint_as_float(u[4 * k4 + 3]));
               }
             }
+            if (store_rows && row_ok[j]) {  // the tail's stored rows (ldt covers every chunk)
+              float* dst = a.Dtail + static_cast<size_t>(hw.ibase + off + 128 * j + r) * a.ldt + c0;
+#pragma unroll
+              for (int k4 = 0; k4 < 16; ++k4)
+                *reinterpret_cast<float4*>(dst + 4 * k4) =
+                    make_float4(__uint_as_float(u[4 * k4]), __uint_as_float(u[4 * k4 + 1]),
+                                __uint_as_float(u[4 * k4 + 2]), __uint_as_float(u[4 * k4 + 3]));
+            }
           }
         }
         if (half == 1) {
@@ -448,6 +573,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
             a.prop_g[grow[j]] = bc;
             a.prop_v[grow[j]] = bv;
             atomicAdd(a.cnt + static_cast<size_t>(h) * G + bc, 1);
+            if (store_rows) a.tailpos[grow[j]] = hw.ibase + off + 128 * j + r;
           }
         }
         asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -457,6 +583,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
       }
     }
     __syncwarp();
+    if (norm_mode) break;  // one pass, no fill
     alive = sync_grid();
     if (!alive) break;
 
@@ -519,6 +646,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
         const int o = __ldcg(a.offs + gi);
         if (o < 0) {
           a.labels[item] = g;
+          a.members[gi * a.cap + atomicAdd(a.msize + gi, 1)] = i;
         } else {
           const int slot = atomicAdd(a.cursor + gi, 1);
           a.bucket[static_cast<size_t>(h) * n + o + slot] = decision_key(__ldcg(a.prop_v + item), i);
@@ -554,7 +682,18 @@ __global__ void __launch_bounds__(kAsThreads, 1)
             const bool valid = e0 + u * 32 + lane < c;
             const int i = static_cast<int>(kb[u] & 0xffffffffu);
             const bool take = valid && kb[u] <= thr;
-            if (take) lab[i] = g;
+            // taken proposers join the group's member list, one atomic per warp
+            const unsigned int tk = __ballot_sync(0xffffffffu, take);
+            if (tk != 0u) {
+              const int leader = __ffs(tk) - 1;
+              int base = 0;
+              if (lane == leader) base = atomicAdd(a.msize + x, __popc(tk));
+              base = __shfl_sync(0xffffffffu, base, leader);
+              if (take) {
+                lab[i] = g;
+                a.members[static_cast<size_t>(x) * a.cap + base + __popc(tk & ((1u << lane) - 1u))] = i;
+              }
+            }
             // rejected proposers join the head's next list, one atomic per warp
             const unsigned int rej = __ballot_sync(0xffffffffu, valid && !take);
             if (rej != 0u) {
@@ -586,6 +725,12 @@ __global__ void __launch_bounds__(kAsThreads, 1)
     }
     __syncthreads();
     if (s_remaining == 0) break;
+    if (store_rows) {
+      store_rows = false;
+      tail = true;
+    } else if (!tail && s_remaining <= a.tail_cap) {
+      store_rows = true;
+    }
     if (round >= max_rounds) {
       if (gthread == 0) record_error(status, kErrTimeout);
       break;
@@ -631,7 +776,9 @@ size_t assign_tc_smem_bytes() {
 
 cudaError_t launch_assign_tc(const __nv_bfloat16* X, const __nv_bfloat16* Whi, const __nv_bfloat16* Wlo,
                              const AssignArgs& a, cudaStream_t st) {
-  if (a.G < 1 || a.G > kAsMaxCols || a.n < 1 || a.heads < 1 || a.cap < 1 || (a.Dout != nullptr && a.ldd % 4 != 0))
+  if (a.G < 1 || a.G > kAsMaxCols || a.n < 1 || a.heads < 1 || a.cap < 1 || (a.Dout != nullptr && a.ldd % 4 != 0) ||
+      (a.tail_cap > 0 && (a.Dtail == nullptr || a.tailpos == nullptr || a.ldt < ceil_div(a.G, 128) * 128 ||
+                          a.ldt % 4 != 0)))
     return cudaErrorInvalidValue;
   const size_t smem = assign_tc_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(assign_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -648,24 +795,29 @@ cudaError_t launch_assign_tc(const __nv_bfloat16* X, const __nv_bfloat16* Whi, c
   for (int h0 = 0; h0 < a.heads; h0 += kAsMaxHeads) {
     const int hc = std::min(kAsMaxHeads, a.heads - h0);
     const size_t ni = static_cast<size_t>(h0) * a.n, gi = static_cast<size_t>(h0) * a.G;
+    auto sl = [](auto* p, size_t k) { return p != nullptr ? p + k : p; };
     AssignArgs s = a;
     s.heads = hc;
-    s.nrm = a.nrm + ni;
-    s.ecol = a.ecol + gi;
-    s.labels = a.labels + ni;
-    s.room = a.room + gi;
-    s.cnt = a.cnt + gi;
-    s.offs = a.offs + gi;
-    s.cursor = a.cursor + gi;
-    s.closed = a.closed + static_cast<size_t>(h0) * words;
-    s.bucket = a.bucket + ni;
-    s.list[0] = a.list[0] + ni;
-    s.list[1] = a.list[1] + ni;
-    s.list_len = a.list_len + 2 * h0;
-    s.prop_g = a.prop_g + ni;
-    s.prop_v = a.prop_v + ni;
-    s.ovf_list = a.ovf_list + gi;
-    s.Dout = a.Dout != nullptr ? a.Dout + ni * a.ldd : nullptr;
+    s.nrm = sl(a.nrm, ni);
+    s.ecol = sl(a.ecol, gi);
+    s.labels = sl(a.labels, ni);
+    s.room = sl(a.room, gi);
+    s.cnt = sl(a.cnt, gi);
+    s.offs = sl(a.offs, gi);
+    s.cursor = sl(a.cursor, gi);
+    s.closed = sl(a.closed, static_cast<size_t>(h0) * words);
+    s.bucket = sl(a.bucket, ni);
+    s.list[0] = sl(a.list[0], ni);
+    s.list[1] = sl(a.list[1], ni);
+    s.list_len = sl(a.list_len, static_cast<size_t>(2) * h0);
+    s.prop_g = sl(a.prop_g, ni);
+    s.prop_v = sl(a.prop_v, ni);
+    s.ovf_list = sl(a.ovf_list, gi);
+    s.members = sl(a.members, gi * a.cap);
+    s.msize = sl(a.msize, gi);
+    s.tailpos = sl(a.tailpos, ni);
+    s.nrm_out = sl(a.nrm_out, ni);
+    s.Dout = sl(a.Dout, ni * a.ldd);
     const long long xrows = static_cast<long long>(hc) * a.n, wrows = static_cast<long long>(hc) * a.G;
     if (xrows > 0x7fffffffLL || wrows > 0x7fffffffLL) return cudaErrorInvalidValue;  // TMA coordinates are int32
     CUtensorMap tx, txg, twh, twl;
@@ -681,6 +833,18 @@ cudaError_t launch_assign_tc(const __nv_bfloat16* X, const __nv_bfloat16* Whi, c
     if ((e = counted(e, 1)) != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_row_norms_tc(const __nv_bfloat16* X, const __nv_bfloat16* ghi, const __nv_bfloat16* glo,
+                                int heads, int n, float* nrm, WorkspaceHeader* hdr, cudaStream_t st) {
+  AssignArgs a{};
+  a.heads = heads;
+  a.n = n;
+  a.G = 128;  // the columns of Gamma
+  a.cap = 1;
+  a.nrm_out = nrm;
+  a.hdr = hdr;
+  return launch_assign_tc(X, ghi, glo, a, st);
 }
 
 }  // namespace spr

@@ -185,6 +185,111 @@ __global__ void wmat_kernel(const float* __restrict__ cent, const float* __restr
   }
 }
 
+// One k-means iteration's group update, 8 groups of one head per CTA (256 threads): warp
+// j sorts group g0 + j's members (the unsorted lists tmp[g * cap + slot], cursor[g] of
+// them) into ascending token order by a shared-memory bitonic sort, writes perm and
+// sizes, and sums the member rows in that order for the fp32 mean c_g (an empty group
+// keeps its c_g); then W = C Gamma (fp32 and bf16 hi/lo) and e_g = c_g . w_g with the
+// arithmetic of wmat_kernel.
+template <typename T, int D>
+__global__ void __launch_bounds__(256) group_update_kernel(const T* __restrict__ X, int n,
+                                                           const int* __restrict__ cursor,
+                                                           const int* __restrict__ tmp, int G, int cap,
+                                                           const float* __restrict__ gamma, int* __restrict__ perm,
+                                                           int* __restrict__ sizes, float* __restrict__ cent,
+                                                           float* __restrict__ wf, __nv_bfloat16* __restrict__ whi,
+                                                           __nv_bfloat16* __restrict__ wlo, float* __restrict__ eg) {
+  constexpr int kPer = D / 32, kSets = 256 / D, kPerSet = 8 / kSets;
+  __shared__ int sv[8][128];
+  __shared__ float sc[8][D];
+  __shared__ float red[8][D / 32];
+  const int head = blockIdx.y, g0 = blockIdx.x * 8;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  {
+    // ---- members of group g0 + warp, sorted
+    const int g = g0 + warp;
+    const size_t gi = static_cast<size_t>(head) * G + g;
+    const int size = g < G ? min(cursor[gi], cap) : 0;
+    for (int t = lane; t < cap; t += 32) sv[warp][t] = t < size ? tmp[gi * cap + t] : 0x7fffffff;
+    __syncwarp();
+    for (int k = 2; k <= cap; k <<= 1) {
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int t = lane; t < cap; t += 32) {
+          const int p = t ^ j;
+          if (p > t) {
+            const int a = sv[warp][t], b = sv[warp][p];
+            const bool up = (t & k) == 0;
+            if ((a > b) == up) {
+              sv[warp][t] = b;
+              sv[warp][p] = a;
+            }
+          }
+        }
+        __syncwarp();
+      }
+    }
+    if (g < G) {
+      for (int t = lane; t < cap; t += 32) perm[gi * cap + t] = t < size ? sv[warp][t] : -1;
+      if (lane == 0) sizes[gi] = size;
+    }
+    // ---- c_g: lane l sums dims [l kPer, (l + 1) kPer) over the members in token order
+    float acc[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) acc[i] = 0.f;
+    const T* x = X + static_cast<size_t>(head) * n * D + lane * kPer;
+#pragma unroll 8
+    for (int j = 0; j < size; ++j) {
+      float v[kPer];
+      load_dims<T, D>(x + static_cast<size_t>(sv[warp][j]) * D, v);
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) acc[i] += v[i];
+    }
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane * kPer + i;
+      float c = 0.f;
+      if (g < G) {
+        c = size > 0 ? acc[i] / static_cast<float>(size) : cent[gi * D + e];
+        if (size > 0) cent[gi * D + e] = c;
+      }
+      sc[warp][e] = c;
+    }
+  }
+  __syncthreads();
+  // ---- W = C Gamma and e_g, thread (set, e): groups set * kPerSet + j
+  const int e = threadIdx.x % D, set = threadIdx.x / D;
+  const float* gm = gamma + static_cast<size_t>(head) * D * D;
+  float acc[kPerSet];
+#pragma unroll
+  for (int j = 0; j < kPerSet; ++j) acc[j] = 0.f;
+  for (int f = 0; f < D; ++f) {
+    const float gv = gm[f * D + e];
+#pragma unroll
+    for (int j = 0; j < kPerSet; ++j) acc[j] += sc[set * kPerSet + j][f] * gv;
+  }
+#pragma unroll
+  for (int j = 0; j < kPerSet; ++j) {
+    const float part = warp_sum(acc[j] * sc[set * kPerSet + j][e]);
+    if ((e & 31) == 0) red[set * kPerSet + j][e >> 5] = part;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kPerSet; ++j) {
+    const int gl = set * kPerSet + j, g = g0 + gl;
+    if (g >= G) break;
+    const size_t o = (static_cast<size_t>(head) * G + g) * D + e;
+    wf[o] = acc[j];
+    const __nv_bfloat16 h = __float2bfloat16_rn(acc[j]);
+    whi[o] = h;
+    wlo[o] = __float2bfloat16_rn(acc[j] - __bfloat162float(h));
+    if (e == 0) {
+      float s = 0.f;
+      for (int w = 0; w < D / 32; ++w) s += red[gl][w];
+      eg[static_cast<size_t>(head) * G + g] = s;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- row GEMM (tensor core)
 // acc[i][c] = x_i . B_c over a 128-row tile; all columns streamed in chunks of 64.
 //   NORM: out[i] = sum_c acc[i][c] * x_i[c]        (x_i^T Gamma x_i, B = Gamma)
@@ -854,23 +959,53 @@ __global__ void perm_sort_kernel(const int* __restrict__ cursor, const int* __re
   if (t == 0) sizes[gi] = size;
 }
 
-// Sc[b][g] = tau * qbar_b . mu_g  (16x16 output tile per CTA).
+// Sc[b][g] = tau * qbar_b . mu_g: a 64 x 64 output tile per CTA, 4 x 4 per thread, the
+// dimension staged 32 at a time; every dot product is summed in ascending dimension order
+// by fused multiply-adds.
 template <int D>
-__global__ void block_score_kernel(const float* __restrict__ qbar, const float* __restrict__ mu, int G,
-                                   float tau, float* __restrict__ sc) {
-  __shared__ float sa[16][D + 1], sb[16][D + 1];
+__global__ void __launch_bounds__(256) block_score_kernel(const float* __restrict__ qbar, const float* __restrict__ mu,
+                                                          int G, float tau, float* __restrict__ sc) {
+  __shared__ float sa[32][65], sb[32][65];  // [dimension][row]
   const int head = blockIdx.z;
-  const int b0 = blockIdx.y * 16, g0 = blockIdx.x * 16;
+  const int b0 = blockIdx.y * 64, g0 = blockIdx.x * 64;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  for (int x = threadIdx.x; x < 16 * D; x += 256) {
-    const int r = x / D, e = x % D;
-    sa[r][e] = b0 + r < G ? qbar[(static_cast<size_t>(head) * G + b0 + r) * D + e] : 0.f;
-    sb[r][e] = g0 + r < G ? mu[(static_cast<size_t>(head) * G + g0 + r) * D + e] : 0.f;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  for (int e0 = 0; e0 < D; e0 += 32) {
+    for (int x = threadIdx.x; x < 64 * 32; x += 256) {
+      const int r = x >> 5, e = x & 31;
+      sa[e][r] = b0 + r < G ? qbar[(static_cast<size_t>(head) * G + b0 + r) * D + e0 + e] : 0.f;
+      sb[e][r] = g0 + r < G ? mu[(static_cast<size_t>(head) * G + g0 + r) * D + e0 + e] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int e = 0; e < 32; ++e) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        av[i] = sa[e][ty + 16 * i];
+        bv[i] = sb[e][tx + 16 * i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
   }
-  __syncthreads();
-  float acc = 0.f;
-  for (int e = 0; e < D; ++e) acc += sa[ty][e] * sb[tx][e];
-  if (b0 + ty < G && g0 + tx < G) sc[(static_cast<size_t>(head) * G + b0 + ty) * G + g0 + tx] = tau * acc;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int b = b0 + ty + 16 * i;
+    if (b >= G) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int g = g0 + tx + 16 * j;
+      if (g < G) sc[(static_cast<size_t>(head) * G + b) * G + g] = tau * acc[i][j];
+    }
+  }
 }
 
 // ----------------------------------------------------------------------------- launchers
@@ -1022,9 +1157,42 @@ cudaError_t launch_build_perm(const int* labels, int n, int G, int cap, int head
   return counted(cudaGetLastError(), 2);
 }
 
+cudaError_t launch_group_update(const void* X, bool f32, int n, const int* cursor, const int* tmp, int G, int cap,
+                                int heads, int d, const float* gamma, int* perm, int* sizes, float* cent, float* wf,
+                                __nv_bfloat16* whi, __nv_bfloat16* wlo, float* eg, cudaStream_t st) {
+  if (cap > 128 || (cap & (cap - 1)) != 0) return cudaErrorInvalidValue;
+  dim3 grid(ceil_div(G, 8), heads);
+  if (f32) {
+    if (d == 64)
+      group_update_kernel<float, 64><<<grid, 256, 0, st>>>(static_cast<const float*>(X), n, cursor, tmp, G, cap, gamma,
+                                                           perm, sizes, cent, wf, whi, wlo, eg);
+    else
+      group_update_kernel<float, 128><<<grid, 256, 0, st>>>(static_cast<const float*>(X), n, cursor, tmp, G, cap,
+                                                            gamma, perm, sizes, cent, wf, whi, wlo, eg);
+  } else {
+    if (d == 64)
+      group_update_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), n, cursor,
+                                                                   tmp, G, cap, gamma, perm, sizes, cent, wf, whi,
+                                                                   wlo, eg);
+    else
+      group_update_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), n, cursor,
+                                                                    tmp, G, cap, gamma, perm, sizes, cent, wf, whi,
+                                                                    wlo, eg);
+  }
+  return counted(cudaGetLastError(), 1);
+}
+
+cudaError_t launch_perm_scatter(const int* labels, int n, int G, int cap, int heads, int* cursor, int* tmp,
+                                int* status, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(cursor, 0, static_cast<size_t>(heads) * G * sizeof(int), st);
+  if (e != cudaSuccess) return e;
+  perm_scatter_kernel<<<1024, 256, 0, st>>>(labels, n, G, cap, cursor, tmp, heads, status);
+  return counted(cudaGetLastError(), 1);
+}
+
 cudaError_t launch_block_scores(const float* qbar, const float* mu, int G, int heads, int d, float tau,
                                 float* sc, cudaStream_t st) {
-  dim3 grid(ceil_div(G, 16), ceil_div(G, 16), heads);
+  dim3 grid(ceil_div(G, 64), ceil_div(G, 64), heads);
   if (d == 64) block_score_kernel<64><<<grid, 256, 0, st>>>(qbar, mu, G, tau, sc);
   else block_score_kernel<128><<<grid, 256, 0, st>>>(qbar, mu, G, tau, sc);
   return counted(cudaGetLastError(), 1);

@@ -83,14 +83,27 @@ struct AssignArgs {
   int* list_len;                // [2, heads]
   int* prop_g;                  // [heads, n]
   float* prop_v;
+  int* members;                 // [heads, G, cap]: every group's members, in placement order
+  int* msize;                   // [heads, G]: their counts
   int* ovf_list;                // [heads, G]: the round's groups with more proposers than room
   int* ovf_total;               // [2]: its length, alternating between rounds
+  float* nrm_out;               // norm mode: [heads, n] x_i^T Gamma x_i with W = Gamma, no fill
   float* Dout;                  // optional [heads, n, ldd]: the first round's D rows
   int ldd;
+  // Tail of the fill: once at most tail_cap items are unplaced, the next round's tensor-
+  // core pass also stores each one's D row (closed groups as +inf) at Dtail[pos * ldt],
+  // pos in tailpos[item]; the rounds after it propose from the stored rows.
+  float* Dtail;                 // [tail_cap, ldt], ldt = ceil(G / 128) * 128
+  int ldt;
+  int tail_cap;
+  int* tailpos;                 // [heads, n]
   WorkspaceHeader* hdr;
 };
 cudaError_t launch_assign_tc(const __nv_bfloat16* X, const __nv_bfloat16* Whi, const __nv_bfloat16* Wlo,
                              const AssignArgs& a, cudaStream_t st);
+// nrm[h, i] = x_i^T Gamma_h x_i on the same pipeline (bf16 X, d = 128, Gamma as bf16 hi + lo)
+cudaError_t launch_row_norms_tc(const __nv_bfloat16* X, const __nv_bfloat16* ghi, const __nv_bfloat16* glo,
+                                int heads, int n, float* nrm, WorkspaceHeader* hdr, cudaStream_t st);
 
 cudaError_t launch_midpoint_stride(int* idx, int n, int count, cudaStream_t st);
 // gamma [heads, d, d] = identity (the metric of the semantic partition)
@@ -111,6 +124,14 @@ cudaError_t launch_dist_tc(const RowGemmArgs& a, int ldd, cudaStream_t st);
 cudaError_t launch_fill(const FillArgs& a, cudaStream_t st);
 cudaError_t launch_build_perm(const int* labels, int n, int G, int cap, int heads, int* cursor, int* tmp,
                               int* perm, int* sizes, int* status, cudaStream_t st);
+// Members (unsorted tmp lists, cursor counts) -> sorted perm and sizes, the member means
+// cent, and W = cent Gamma (fp32, bf16 hi/lo), e_g = c_g . w_g for the next iteration.
+cudaError_t launch_group_update(const void* X, bool f32, int n, const int* cursor, const int* tmp, int G, int cap,
+                                int heads, int d, const float* gamma, int* perm, int* sizes, float* cent, float* wf,
+                                __nv_bfloat16* whi, __nv_bfloat16* wlo, float* eg, cudaStream_t st);
+// labels -> unsorted member lists tmp[g * cap + slot] and their counts cursor[g]
+cudaError_t launch_perm_scatter(const int* labels, int n, int G, int cap, int heads, int* cursor, int* tmp,
+                                int* status, cudaStream_t st);
 cudaError_t launch_block_scores(const float* qbar, const float* mu, int G, int heads, int d, float tau,
                                 float* sc, cudaStream_t st);
 
