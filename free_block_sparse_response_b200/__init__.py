@@ -7,7 +7,7 @@ include/sparsepr.h; this package is its Python binding.
 """
 from .sparsepr import (  # noqa: F401
     BF16, ERR_CUDA, ERR_INVALID_ARG, ERR_NONFINITE, ERR_TIMEOUT, ERR_UNSUPPORTED, EXPORTED_SYMBOLS, F32, OK,
-    WEIGHT_INV_NORM, WEIGHT_UNIFORM, PARTITION_RESPONSE, PARTITION_SEMANTIC, ROUTE_CENTROID, ROUTE_SIZE_CORRECTED, ROUTE_LSE,
+    WEIGHT_INV_NORM, WEIGHT_UNIFORM, RIDGE_RELATIVE, PARTITION_RESPONSE, PARTITION_SEMANTIC, ROUTE_CENTROID, ROUTE_SIZE_CORRECTED, ROUTE_LSE,
     BUDGET_UNIFORM, BUDGET_GLOBAL,
     Partition, SparsePRConfig, SparsePRError, apply_residual, attention, check,
     dense_attn, fit_residual, fit_residual_noalloc, lib, new_workspace, num_groups, partition, probe_dense, probe_rows, route, route_k,

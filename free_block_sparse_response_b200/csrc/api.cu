@@ -76,7 +76,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct Layout {
   size_t header = 0, sample_idx, gamma, gamma_hi, gamma_lo, nrm, cent_k, cent_q, wf, whi, wlo, eg, dmat,
          prop_g0, prop_v0, labels, room, cnt, offs, cursor, closed, bucket, list0, list1, list_len, prop_g, prop_v,
-         perm_tmp, perm_cursor, qblk, partial, fit, kv_grouped, mhilo, segmin, ovf, dtail, tailpos, total;
+         perm_tmp, perm_cursor, qblk, partial, fit, kv_grouped, mhilo, ovf, dtail, tailpos, total;
 };
 
 Layout make_layout(int heads, int N, int d, int block, int S, int P) {
@@ -107,7 +107,6 @@ Layout make_layout(int heads, int N, int d, int block, int S, int P) {
   L.wlo = take(2 * H * G * D);
   L.eg = take(sizeof(float) * H * G);
   L.dmat = take(sizeof(float) * H * n * dmat_ld(G));
-  L.segmin = take(sizeof(unsigned long long) * H * n * 2 * ((G + 127) / 128));
   L.prop_g0 = take(sizeof(int) * H * n);
   L.prop_v0 = take(sizeof(float) * H * n);
   L.labels = take(sizeof(int) * H * n);
@@ -162,6 +161,16 @@ int check_aligned(std::initializer_list<const void*> ptrs) {
 
 int check_dtype(int dtype) {
   if (dtype != SPARSEPR_BF16 && dtype != SPARSEPR_F32) return fail(SPARSEPR_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  return SPARSEPR_OK;
+}
+
+static_assert(SPARSEPR_RIDGE_RELATIVE == spr::kRidgeRelative, "ridge flag of the ABI and the kernel");
+
+// Probe weights (SPARSEPR_WEIGHT_*), optionally | SPARSEPR_RIDGE_RELATIVE.
+int check_weight_mode(int weight_mode) {
+  const int w = weight_mode & ~SPARSEPR_RIDGE_RELATIVE;
+  if (w != SPARSEPR_WEIGHT_INV_NORM && w != SPARSEPR_WEIGHT_UNIFORM)
+    return fail(SPARSEPR_ERR_INVALID_ARG, "unknown weight_mode %d", weight_mode);
   return SPARSEPR_OK;
 }
 
@@ -272,9 +281,6 @@ static int partition_impl(const void* Q, const void* K, int dtype, int32_t Bt, i
   fa.prop_v0 = at<float>(ws, L.prop_v0);
   // bf16, d = 128: the tensor-core assignment kernel (distances and fill in one launch)
   const bool tc_assign = !f32 && d == 128;
-  const bool seg = false;
-  fa.nseg = 2 * spr::ceil_div(G, 128);
-  fa.seg_min = seg ? at<unsigned long long>(ws, L.segmin) : nullptr;
   fa.heads = heads;
   fa.n = N;
   fa.G = G;
@@ -332,8 +338,6 @@ static int partition_impl(const void* Q, const void* K, int dtype, int32_t Bt, i
       ra.ldd = fa.ldd;
       ra.prop_g = at<int>(ws, L.prop_g0);
       ra.prop_v = at<float>(ws, L.prop_v0);
-      ra.seg_min = seg ? at<unsigned long long>(ws, L.segmin) : nullptr;
-      ra.nseg = fa.nseg;
       ra.nrm_out = nullptr;
       if (tc_assign) {
         // bf16, d = 128: proposals and fill in one tensor-core kernel, no distance matrix
@@ -646,8 +650,7 @@ int sparsepr_fit_residual(const float* probe_sparse, const float* probe_out, con
   if (P < 1) return fail(SPARSEPR_ERR_INVALID_ARG, "P must be >= 1");
   if (rank < 1) return fail(SPARSEPR_ERR_INVALID_ARG, "rank must be >= 1");
   if (!(ridge_lambda >= 0.0)) return fail(SPARSEPR_ERR_INVALID_ARG, "ridge_lambda must be >= 0");
-  if (weight_mode != SPARSEPR_WEIGHT_INV_NORM && weight_mode != SPARSEPR_WEIGHT_UNIFORM)
-    return fail(SPARSEPR_ERR_INVALID_ARG, "unknown weight_mode %d", weight_mode);
+  if ((rc = check_weight_mode(weight_mode))) return rc;
   if (!probe_sparse || !probe_out || !M || !beta || !ws) return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
   if (spr::fit_smem_bytes(d, P) > 220 * 1024) return fail(SPARSEPR_ERR_UNSUPPORTED, "P=%d too large for the fit", P);
   // The fit's scratch is the workspace's first region after the header (sized for the
@@ -718,11 +721,11 @@ size_t sparsepr_test_fill_workspace_size(int32_t H, int32_t n, int32_t G) {
   return align_up(sizeof(spr::WorkspaceHeader)) + align_up(4 * h * g * sizeof(int)) +
          align_up(h * ((g + 31) / 32) * sizeof(unsigned int)) +
          align_up(h * nn * sizeof(unsigned long long)) + 3 * align_up(h * nn * sizeof(int)) + align_up(4 * sizeof(int)) +
-         align_up(h * nn * sizeof(float)) + align_up(h * nn * 2 * ((g + 127) / 128) * sizeof(unsigned long long));
+         align_up(h * nn * sizeof(float));
 }
 
-static int test_fill_common(const float* D, int32_t H, int32_t n, int32_t G, int32_t cap, int32_t* labels, void* ws,
-                            sparsepr_stream_t stream, bool segmented) {
+int sparsepr_test_fill(const float* D, int32_t H, int32_t n, int32_t G, int32_t cap, int32_t* labels, void* ws,
+                       sparsepr_stream_t stream) {
   if (!D || !labels || !ws || H < 1 || n < 1 || G < 1 || cap < 1)
     return fail(SPARSEPR_ERR_INVALID_ARG, "bad fill arguments");
   if (static_cast<long long>(G) * cap < n) return fail(SPARSEPR_ERR_INVALID_ARG, "G * cap < n");
@@ -757,26 +760,10 @@ static int test_fill_common(const float* D, int32_t H, int32_t n, int32_t G, int
   fa.prop_g = at<int>(ws, take(h * nn * sizeof(int)));
   fa.list_len = at<int>(ws, take(4 * sizeof(int)));
   fa.prop_v = at<float>(ws, take(h * nn * sizeof(float)));
-  fa.nseg = 2 * spr::ceil_div(G, 128);
-  unsigned long long* seg = at<unsigned long long>(ws, take(h * nn * fa.nseg * sizeof(unsigned long long)));
-  fa.seg_min = segmented ? seg : nullptr;
   fa.hdr = header(ws);
   SPR_CUDA(cudaMemsetAsync(ws, 0, sizeof(spr::WorkspaceHeader), st), "fill: reset status");
-  if (segmented)
-    SPR_CUDA(spr::launch_segment_minima(D, G, static_cast<long long>(H) * n, G, seg, fa.nseg, &fa.hdr->status, st),
-             "segment minima");
   SPR_CUDA(spr::launch_fill(fa, st), "fill");
   return SPARSEPR_OK;
-}
-
-int sparsepr_test_fill(const float* D, int32_t H, int32_t n, int32_t G, int32_t cap, int32_t* labels, void* ws,
-                       sparsepr_stream_t stream) {
-  return test_fill_common(D, H, n, G, cap, labels, ws, stream, false);
-}
-
-int sparsepr_test_fill_segmented(const float* D, int32_t H, int32_t n, int32_t G, int32_t cap, int32_t* labels,
-                                 void* ws, sparsepr_stream_t stream) {
-  return test_fill_common(D, H, n, G, cap, labels, ws, stream, true);
 }
 
 int sparsepr_test_topk(const float* Sc, int32_t H, int32_t Gq, int32_t G, int32_t k, int32_t* route, void* ws,
@@ -863,8 +850,7 @@ extern "C" int sparsepr_fit_residual_noalloc(const float* probe_sparse, const fl
   if (P < 1) return fail(SPARSEPR_ERR_INVALID_ARG, "P must be >= 1");
   if (rank < 1) return fail(SPARSEPR_ERR_INVALID_ARG, "rank must be >= 1");
   if (!(ridge_lambda >= 0.0)) return fail(SPARSEPR_ERR_INVALID_ARG, "ridge_lambda must be >= 0");
-  if (weight_mode != SPARSEPR_WEIGHT_INV_NORM && weight_mode != SPARSEPR_WEIGHT_UNIFORM)
-    return fail(SPARSEPR_ERR_INVALID_ARG, "unknown weight_mode %d", weight_mode);
+  if ((rc = check_weight_mode(weight_mode))) return rc;
   if (!probe_sparse || !probe_out || !M || !beta) return fail(SPARSEPR_ERR_INVALID_ARG, "null pointer argument");
   if (spr::fit_smem_bytes(d, P) > 220 * 1024) return fail(SPARSEPR_ERR_UNSUPPORTED, "P=%d too large for the fit", P);
   const size_t need = kNoAllocStatusBytes + sizeof(double) * static_cast<size_t>(Bt) * H * spr::fit_scratch_doubles(P, d);

@@ -45,17 +45,19 @@
 namespace spr {
 namespace {
 
-constexpr int kAsThreads = 384;
+constexpr int kAsThreads = 384;              // warp 0 loads, warp 2 issues MMAs, warps 4-11 epilogue
 constexpr int kAsWarps = kAsThreads / 32;
+constexpr int kAsEpi = kAsThreads - 128;     // epilogue threads: 2 per row, 64 columns each
 constexpr int kAsRows = 256;                 // items per work item: two 128-row halves
 constexpr uint32_t kAsTile = 128 * 128 * 2;  // 128 rows x 128 bf16: two 64-column swizzled boxes
-constexpr uint32_t kAsWStage = 2 * kAsTile;  // one chunk of W: hi and lo
+constexpr uint32_t kAsXStage = 2 * kAsTile;  // one work item's X (two buffers)
+constexpr uint32_t kAsWStage = kAsTile;      // half a chunk of W: its hi or its lo part
 constexpr uint32_t kAsTmemCols = 512;        // 2 stages x 2 halves x 128 fp32 columns
 constexpr int kAsMaxCols = 1024;             // groups per head
 constexpr int kAsMaxHeads = 1024;            // heads per launch (the launcher splits larger calls)
 constexpr float kAsInf = __builtin_huge_valf();
 
-enum : int { kXFull = 0, kXEmpty = 1, kWFull0 = 2, kWEmpty0 = 4, kAccFull0 = 6, kAccEmpty0 = 8, kDrain = 10, kBars = 11 };
+enum : int { kXFull0 = 0, kXEmpty0 = 2, kWFull0 = 4, kWEmpty0 = 6, kAccFull0 = 8, kAccEmpty0 = 10, kDrain = 12, kBars = 13 };
 
 __device__ __forceinline__ uint64_t as_f32x2(float lo, float hi) {
   uint64_t r;
@@ -144,17 +146,19 @@ __global__ void __launch_bounds__(kAsThreads, 1)
   __shared__ __align__(8) uint64_t bars[kBars];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag, s_enf, s_remaining, s_total;
-  __shared__ float s_best_v[kAsRows];
+  __shared__ float s_best_v[kAsRows];  // the upper column halves' partial results
   __shared__ int s_best_c[kAsRows];
-  __shared__ int scan_tmp[kAsThreads];
-  __shared__ unsigned int hist[kAsWarps][256];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = (tc::saddr(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sX = sbase;                       // two 128-row halves
-  const uint32_t sW[2] = {sbase + 2 * kAsTile, sbase + 2 * kAsTile + kAsWStage};
-  uint8_t* sgen = smem_raw + (sbase - tc::saddr(smem_raw)) + 2 * kAsTile + 2 * kAsWStage;
+  const uint32_t sX[2] = {sbase, sbase + kAsXStage};  // two work items, each two 128-row halves
+  const uint32_t sW[2] = {sbase + 2 * kAsXStage, sbase + 2 * kAsXStage + kAsWStage};
+  uint8_t* sgen = smem_raw + (sbase - tc::saddr(smem_raw)) + 2 * kAsXStage + 2 * kAsWStage;
   float* s_e = reinterpret_cast<float*>(sgen);                   // [kAsMaxCols]
+  // phases B-D (and the per-head rounds) run with no copy or MMA in flight: their scratch
+  // lives in the idle W stages
+  int* scan_tmp = reinterpret_cast<int*>(smem_raw + (sW[1] - tc::saddr(smem_raw)));              // [kAsThreads]
+  unsigned int (*hist)[256] = reinterpret_cast<unsigned int (*)[256]>(smem_raw + (sW[0] - tc::saddr(smem_raw)));
   int* s_len = reinterpret_cast<int*>(sgen + 4 * kAsMaxCols);     // [kAsMaxHeads] list lengths
   int* s_tiles = s_len + kAsMaxHeads;                             // [kAsMaxHeads] work items per head
   auto bar = [&](int i) { return tc::saddr(&bars[i]); };
@@ -168,13 +172,13 @@ __global__ void __launch_bounds__(kAsThreads, 1)
   int* status = &a.hdr->status;
 
   if (tid == 0) {
-    tc::mbar_init(bar(kXFull), 1);
-    tc::mbar_init(bar(kXEmpty), 1);
     for (int s = 0; s < 2; ++s) {
+      tc::mbar_init(bar(kXFull0 + s), 1);
+      tc::mbar_init(bar(kXEmpty0 + s), 1);
       tc::mbar_init(bar(kWFull0 + s), 1);
       tc::mbar_init(bar(kWEmpty0 + s), 1);
       tc::mbar_init(bar(kAccFull0 + s), 1);
-      tc::mbar_init(bar(kAccEmpty0 + s), 256);
+      tc::mbar_init(bar(kAccEmpty0 + s), kAsEpi);
     }
     tc::mbar_init(bar(kDrain), 1);
     abort_flag = 0;
@@ -246,82 +250,213 @@ __global__ void __launch_bounds__(kAsThreads, 1)
 
     // ---------------------------------------------------------------- A. proposals
     if (tail) {
-      // a warp per unplaced item: the first minimum over the open groups of its stored
-      // row, by the epilogue's rule (strict '<' in ascending column order, so +inf and NaN
-      // never win; none finite: the lowest open group at +inf)
-      int items = 0;
-      for (int h = 0; h < heads; ++h) items += s_len[h];
-      HeadWalk hw;
-      for (int x = gwarp; x < items; x += nwarps) {
-        int h, e;
-        hw.seek(s_len, x, h, e);
-        const int i = __ldcg(list + static_cast<size_t>(h) * n + e);
-        const size_t grow = static_cast<size_t>(h) * n + i;
-        const float* row = a.Dtail + static_cast<size_t>(__ldcg(a.tailpos + grow)) * a.ldt;
-        const unsigned int* cl = a.closed + static_cast<size_t>(h) * words;
-        unsigned long long best = ~0ull;
-        int first_open = G;
-        // 16 words of the row and of the full-group bitmap requested before any is used
-        for (int w0 = 0; w0 < words; w0 += 16) {
-          float v[16];
-          unsigned int cw[16];
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int g = (w0 + u) * 32 + lane;
-            v[u] = g < G ? __ldcg(row + g) : kAsInf;
-            cw[u] = w0 + u < words ? __ldcg(cl + w0 + u) : ~0u;
+      // ---- the rest of the fill, one head per CTA.  Every unplaced item's D row is stored
+      // (the previous round's tensor-core pass), and heads are independent problems, so
+      // each CTA runs its heads' remaining rounds alone: proposals from the stored rows (a
+      // warp per item: the first minimum over the open groups by the epilogue's rule --
+      // strict '<' in ascending column order, so +inf and NaN never win; none finite: the
+      // lowest open group at +inf), then the same group pass, placement and overflow
+      // selection as the grid-wide rounds, separated by __syncthreads.  The X and W
+      // buffers are idle now and hold the overflow list and the full-group bitmap.
+      int* s_ovf = reinterpret_cast<int*>(smem_raw + (sX[0] - tc::saddr(smem_raw)));           // [G]
+      unsigned int* s_cl = reinterpret_cast<unsigned int*>(smem_raw + (sX[1] - tc::saddr(smem_raw)));  // [words]
+      __shared__ int s_novf, s_nlen;
+      for (int h = blockIdx.x; h < heads; h += nblocks) {
+        int lc = cur;
+        int len = __ldcg(a.list_len + lc * heads + h);
+        int* cnt = a.cnt + static_cast<size_t>(h) * G;
+        int* room = a.room + static_cast<size_t>(h) * G;
+        int* offs = a.offs + static_cast<size_t>(h) * G;
+        int* cursor = a.cursor + static_cast<size_t>(h) * G;
+        unsigned int* cl = a.closed + static_cast<size_t>(h) * words;
+        int* lab = a.labels + static_cast<size_t>(h) * n;
+        for (int lr = 0; len > 0; ++lr) {
+          if (lr > max_rounds) {
+            if (tid == 0) record_error(status, kErrTimeout);
+            break;
           }
+          const int* hl = a.list[lc] + static_cast<size_t>(h) * n;
+          int* nl = a.list[lc ^ 1] + static_cast<size_t>(h) * n;
+          for (int wd = tid; wd < words; wd += kAsThreads) s_cl[wd] = __ldcg(cl + wd);
+          if (tid == 0) {
+            s_novf = 0;
+            s_nlen = 0;
+          }
+          __syncthreads();
+          // A. proposals
+          for (int x = warp; x < len; x += kAsWarps) {
+            const int i = __ldcg(hl + x);
+            const size_t grow = static_cast<size_t>(h) * n + i;
+            const float* row = a.Dtail + static_cast<size_t>(__ldcg(a.tailpos + grow)) * a.ldt;
+            unsigned long long best = ~0ull;
+            int first_open = G;
+            for (int w0 = 0; w0 < words; w0 += 16) {  // 16 words of the row requested at once
+              float v[16];
 #pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const int g = (w0 + u) * 32 + lane;
-            const bool open = g < G && !((cw[u] >> lane) & 1u);
-            if (open && v[u] < kAsInf) {
-              const unsigned long long key = decision_key(v[u], g);
-              best = key < best ? key : best;
+              for (int u = 0; u < 16; ++u) {
+                const int g = (w0 + u) * 32 + lane;
+                v[u] = g < G ? __ldcg(row + g) : kAsInf;
+              }
+#pragma unroll
+              for (int u = 0; u < 16; ++u) {
+                const int wd = w0 + u;
+                const int g = wd * 32 + lane;
+                const bool open = g < G && !((s_cl[wd < words ? wd : 0] >> lane) & 1u);
+                if (open && v[u] < kAsInf) {
+                  const unsigned long long key = decision_key(v[u], g);
+                  best = key < best ? key : best;
+                }
+                const unsigned int om = __ballot_sync(0xffffffffu, open);
+                if (first_open == G && om != 0u) first_open = wd * 32 + __ffs(om) - 1;
+              }
             }
-            const unsigned int om = __ballot_sync(0xffffffffu, open);
-            if (first_open == G && om != 0u) first_open = (w0 + u) * 32 + __ffs(om) - 1;
+            best = warp_min_u64(best);
+            if (lane == 0) {
+              int g;
+              float pv;
+              if (best != ~0ull) {
+                g = static_cast<int>(best & 0xffffffffu);
+                pv = __ldcg(row + g);
+              } else if (first_open < G) {
+                g = first_open;
+                pv = kAsInf;
+              } else {  // no open group: more items than room (cannot happen)
+                record_error(status, kErrInvalidArg);
+                g = 0;
+                pv = kAsInf;
+              }
+              a.prop_g[grow] = g;
+              a.prop_v[grow] = pv;
+              atomicAdd(cnt + g, 1);
+            }
           }
-        }
-        best = warp_min_u64(best);
-        if (lane == 0) {
-          int g;
-          float v;
-          if (best != ~0ull) {
-            g = static_cast<int>(best & 0xffffffffu);
-            v = __ldcg(row + g);
-          } else if (first_open < G) {
-            g = first_open;
-            v = kAsInf;
-          } else {  // no open group: more items than room (cannot happen)
-            record_error(status, kErrInvalidArg);
-            g = 0;
-            v = kAsInf;
+          __syncthreads();
+          // B. groups that take all their proposers; bucket offsets of the others
+          {
+            const int per = ceil_div(G, kAsThreads);
+            const int g0 = tid * per, g1 = min(G, g0 + per);
+            int local = 0;
+            for (int g = g0; g < g1; ++g) {
+              const int c = __ldcg(cnt + g);
+              if (c > __ldcg(room + g)) local += c;
+            }
+            scan_tmp[tid] = local;
+            __syncthreads();
+            for (int o = 1; o < kAsThreads; o <<= 1) {
+              const int y = tid >= o ? scan_tmp[tid - o] : 0;
+              __syncthreads();
+              scan_tmp[tid] += y;
+              __syncthreads();
+            }
+            int run = scan_tmp[tid] - local;
+            for (int g = g0; g < g1; ++g) {
+              const int c = __ldcg(cnt + g), rm = __ldcg(room + g);
+              if (c > rm) {
+                offs[g] = run;
+                run += c;
+                s_ovf[atomicAdd(&s_novf, 1)] = g;
+              } else {
+                offs[g] = -1;
+                if (c > 0) {
+                  room[g] = rm - c;
+                  cnt[g] = 0;
+                  if (rm == c) atomicOr(cl + g / 32, 1u << (g % 32));
+                }
+              }
+            }
           }
-          a.prop_g[grow] = g;
-          a.prop_v[grow] = v;
-          atomicAdd(a.cnt + static_cast<size_t>(h) * G + g, 1);
+          __syncthreads();
+          // C. place / scatter
+          for (int x = tid; x < len; x += kAsThreads) {
+            const int i = __ldcg(hl + x);
+            const size_t item = static_cast<size_t>(h) * n + i;
+            const int g = __ldcg(a.prop_g + item);
+            const size_t gi = static_cast<size_t>(h) * G + g;
+            const int o = __ldcg(offs + g);
+            if (o < 0) {
+              lab[i] = g;
+              a.members[gi * a.cap + atomicAdd(a.msize + gi, 1)] = i;
+            } else {
+              const int slot = atomicAdd(cursor + g, 1);
+              a.bucket[static_cast<size_t>(h) * n + o + slot] = decision_key(__ldcg(a.prop_v + item), i);
+            }
+          }
+          __syncthreads();
+          // D. overflowing groups
+          for (int j2 = warp; j2 < s_novf; j2 += kAsWarps) {
+            const int g = s_ovf[j2];
+            const size_t x = static_cast<size_t>(h) * G + g;
+            const int c = __ldcg(cnt + g), rm = __ldcg(room + g);
+            const unsigned long long* bk = a.bucket + static_cast<size_t>(h) * n + __ldcg(offs + g);
+            const unsigned long long thr = rm == 0 ? 0ull : warp_select_kth(bk, c, rm, hist[warp]);
+            for (int e0 = 0; e0 < c; e0 += 256) {
+              unsigned long long kb[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const int e = e0 + u * 32 + lane;
+                kb[u] = e < c ? __ldcg(bk + e) : ~0ull;
+              }
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const bool valid = e0 + u * 32 + lane < c;
+                const int i = static_cast<int>(kb[u] & 0xffffffffu);
+                const bool take = valid && kb[u] <= thr;
+                const unsigned int tk = __ballot_sync(0xffffffffu, take);
+                if (tk != 0u) {
+                  const int leader = __ffs(tk) - 1;
+                  int base = 0;
+                  if (lane == leader) base = atomicAdd(a.msize + x, __popc(tk));
+                  base = __shfl_sync(0xffffffffu, base, leader);
+                  if (take) {
+                    lab[i] = g;
+                    a.members[x * a.cap + base + __popc(tk & ((1u << lane) - 1u))] = i;
+                  }
+                }
+                const unsigned int rej = __ballot_sync(0xffffffffu, valid && !take);
+                if (rej != 0u) {
+                  const int leader = __ffs(rej) - 1;
+                  int base = 0;
+                  if (lane == leader) base = atomicAdd(&s_nlen, __popc(rej));
+                  base = __shfl_sync(0xffffffffu, base, leader);
+                  if (valid && !take) nl[base + __popc(rej & ((1u << lane) - 1u))] = i;
+                }
+              }
+            }
+            __syncwarp();
+            if (lane == 0) {
+              room[g] = 0;
+              cnt[g] = 0;
+              cursor[g] = 0;
+              atomicOr(cl + g / 32, 1u << (g % 32));
+            }
+          }
+          __syncthreads();
+          len = s_nlen;
+          lc ^= 1;
+          __syncthreads();
         }
       }
+      break;
     } else if (warp == 0) {
-      // producer: the 256 rows of X (lane 0 four 2-D boxes, or every lane four gather4 of
-      // 4 rows), then per chunk the 128 rows of W hi and lo
-      HeadWalk hw;
-      for (int w = blockIdx.x; w < total; w += nblocks, ++it_prod) {
-        int h, t;
-        hw.seek(s_tiles, w, h, t);
-        const int off = t * kAsRows;
+      // producer: per work item the 256 rows of X into buffer it & 1 (lane 0 four 2-D
+      // boxes, or every lane four gather4 of 4 rows), then per chunk of 128 groups its W
+      // hi part and its lo part, each one stage of a two-stage ring.  The next item's X is
+      // issued right after this item's first lo part: that stage was freed by the previous
+      // item's last MMAs, so the X buffer the next item reuses is free, and its load
+      // overlaps all of this item's MMAs.
+      auto issue_x = [&](int it, int h, int t) -> bool {
+        const int b = it & 1, off = t * kAsRows;
         int ok = 1;
-        if (lane == 0 && it_prod >= 1 && !tc::mbar_wait(bar(kXEmpty), (it_prod - 1) & 1, abort_v, status)) ok = 0;
-        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-        if (lane == 0) tc::mbar_arrive_expect_tx(bar(kXFull), 2 * kAsTile);
+        if (lane == 0 && it >= 2 && !tc::mbar_wait(bar(kXEmpty0 + b), ((it >> 1) - 1) & 1, abort_v, status)) ok = 0;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+        if (lane == 0) tc::mbar_arrive_expect_tx(bar(kXFull0 + b), kAsXStage);
         __syncwarp();
         if (first) {
           if (lane == 0) {
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              tc::tma_load_2d(sX + j * kAsTile, &tmX, 0, h * n + off + 128 * j, bar(kXFull));
-              tc::tma_load_2d(sX + j * kAsTile + 128 * 128, &tmX, 64, h * n + off + 128 * j, bar(kXFull));
+            for (int j2 = 0; j2 < 2; ++j2) {
+              tc::tma_load_2d(sX[b] + j2 * kAsTile, &tmX, 0, h * n + off + 128 * j2, bar(kXFull0 + b));
+              tc::tma_load_2d(sX[b] + j2 * kAsTile + 128 * 128, &tmX, 64, h * n + off + 128 * j2, bar(kXFull0 + b));
             }
           }
         } else {
@@ -332,68 +467,93 @@ __global__ void __launch_bounds__(kAsThreads, 1)
             const int row = 8 * lane + 4 * g4;  // 0..255: rows row .. row + 3
             int r4[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int e = off + row + j;
-              // rows past the list repeat the tile's first entry (loaded, never used)
-              r4[j] = h * n + __ldcg(hl + (e < len ? e : off));
+            for (int j2 = 0; j2 < 4; ++j2) {
+              const int e = off + row + j2;
+              // rows past the list repeat the item's first entry (loaded, never used)
+              r4[j2] = h * n + __ldcg(hl + (e < len ? e : off));
             }
-            const uint32_t dst = sX + (row >> 7) * kAsTile + (row & 127) * 128;
-            tc::tma_gather4(dst, &tmXg, 0, r4[0], r4[1], r4[2], r4[3], bar(kXFull));
-            tc::tma_gather4(dst + 128 * 128, &tmXg, 64, r4[0], r4[1], r4[2], r4[3], bar(kXFull));
+            const uint32_t dst = sX[b] + (row >> 7) * kAsTile + (row & 127) * 128;
+            tc::tma_gather4(dst, &tmXg, 0, r4[0], r4[1], r4[2], r4[3], bar(kXFull0 + b));
+            tc::tma_gather4(dst + 128 * 128, &tmXg, 64, r4[0], r4[1], r4[2], r4[3], bar(kXFull0 + b));
           }
         }
-        last_it = it_prod;
-        if (lane == 0) {
-          for (int c = 0; c < n_chunks; ++c) {
-            const int q = it_prod * n_chunks + c, s = q & 1;
-            if (q >= 2 && !tc::mbar_wait(bar(kWEmpty0 + s), ((q >> 1) - 1) & 1, abort_v, status)) {
-              ok = 0;
-              break;
+        last_it = it;
+        return true;
+      };
+      HeadWalk hw;
+      int h = 0, t = 0;
+      bool ok = true;
+      if (static_cast<int>(blockIdx.x) < total) {
+        hw.seek(s_tiles, blockIdx.x, h, t);
+        ok = issue_x(it_prod, h, t);
+      }
+      for (int w = blockIdx.x; ok && w < total; w += nblocks, ++it_prod) {
+        const int wn = w + nblocks;
+        int hn = 0, tn = 0;
+        if (wn < total) hw.seek(s_tiles, wn, hn, tn);
+        for (int c = 0; ok && c < n_chunks; ++c) {
+          for (int part = 0; ok && part < 2; ++part) {
+            int okc = 1;
+            if (lane == 0) {
+              const int q = (it_prod * n_chunks + c) * 2 + part, st = q & 1;
+              if (q >= 2 && !tc::mbar_wait(bar(kWEmpty0 + st), ((q >> 1) - 1) & 1, abort_v, status)) {
+                okc = 0;
+              } else {
+                const CUtensorMap* tm = part == 0 ? &tmWhi : &tmWlo;
+                const int wrow = h * G + c * 128;
+                tc::mbar_arrive_expect_tx(bar(kWFull0 + st), kAsWStage);
+                tc::tma_load_2d(sW[st], tm, 0, wrow, bar(kWFull0 + st));
+                tc::tma_load_2d(sW[st] + 128 * 128, tm, 64, wrow, bar(kWFull0 + st));
+                last_q = q;
+              }
             }
-            const int wrow = h * G + c * 128;
-            tc::mbar_arrive_expect_tx(bar(kWFull0 + s), kAsWStage);
-            tc::tma_load_2d(sW[s], &tmWhi, 0, wrow, bar(kWFull0 + s));
-            tc::tma_load_2d(sW[s] + 128 * 128, &tmWhi, 64, wrow, bar(kWFull0 + s));
-            tc::tma_load_2d(sW[s] + kAsTile, &tmWlo, 0, wrow, bar(kWFull0 + s));
-            tc::tma_load_2d(sW[s] + kAsTile + 128 * 128, &tmWlo, 64, wrow, bar(kWFull0 + s));
-            last_q = q;
+            ok = __shfl_sync(0xffffffffu, okc, 0) != 0;
+            if (ok && c == 0 && part == 1 && wn < total) ok = issue_x(it_prod + 1, hn, tn);
           }
         }
-        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        h = hn;
+        t = tn;
       }
     } else if (warp == 2) {
-      // MMA issuer: per chunk and half, 8 k-steps of 16, each the hi and the lo product
+      // MMA issuer: per chunk, all hi products (8 k-steps of 16, both 128-row halves),
+      // then all lo products, into the chunk's accumulator stage
       if (lane == 0) {
         constexpr uint32_t kId = tc::idesc_bf16(128, 128, false, false);
         for (int w = blockIdx.x; w < total; w += nblocks, ++it_mma) {
-          if (!tc::mbar_wait(bar(kXFull), it_mma & 1, abort_v, status)) break;
+          const int b = it_mma & 1;
+          if (!tc::mbar_wait(bar(kXFull0 + b), (it_mma >> 1) & 1, abort_v, status)) break;
           tc::fence_proxy_async();
           bool ok = true;
-          for (int c = 0; c < n_chunks; ++c) {
-            const int q = it_mma * n_chunks + c, s = q & 1;
-            if (!tc::mbar_wait(bar(kWFull0 + s), (q >> 1) & 1, abort_v, status) ||
-                (q >= 2 && !tc::mbar_wait(bar(kAccEmpty0 + s), ((q >> 1) - 1) & 1, abort_v, status))) {
+          for (int c = 0; ok && c < n_chunks; ++c) {
+            const int qc = it_mma * n_chunks + c, s = qc & 1;
+            if (qc >= 2 && !tc::mbar_wait(bar(kAccEmpty0 + s), ((qc >> 1) - 1) & 1, abort_v, status)) {
               ok = false;
               break;
             }
-            tc::fence_proxy_async();
-            tc::fence_after_sync();
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              const uint32_t acc = tbase + s * 256 + j * 128;
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-                const uint64_t adesc = tc::sdesc_sw128(sX + j * kAsTile + koff, 16, 1024);
-                tc::mma_ss(acc, adesc, tc::sdesc_sw128(sW[s] + koff, 16, 1024), kId, kk > 0 ? 1u : 0u);
-                tc::mma_ss(acc, adesc, tc::sdesc_sw128(sW[s] + kAsTile + koff, 16, 1024), kId, 1u);
+            for (int part = 0; part < 2; ++part) {
+              const int q = qc * 2 + part, st = q & 1;
+              if (!tc::mbar_wait(bar(kWFull0 + st), (q >> 1) & 1, abort_v, status)) {
+                ok = false;
+                break;
               }
+              tc::fence_proxy_async();
+              tc::fence_after_sync();
+#pragma unroll
+              for (int j = 0; j < 2; ++j) {
+                const uint32_t acc = tbase + s * 256 + j * 128;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                  const uint32_t koff = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+                  tc::mma_ss(acc, tc::sdesc_sw128(sX[b] + j * kAsTile + koff, 16, 1024),
+                             tc::sdesc_sw128(sW[st] + koff, 16, 1024), kId, (part == 0 && kk == 0) ? 0u : 1u);
+                }
+              }
+              tc::mma_commit(bar(kWEmpty0 + st));
             }
-            tc::mma_commit(bar(kWEmpty0 + s));
-            tc::mma_commit(bar(kAccFull0 + s));
+            if (ok) tc::mma_commit(bar(kAccFull0 + s));
           }
           if (!ok) break;
-          if (!norm_mode) tc::mma_commit(bar(kXEmpty));  // norm mode: the epilogue frees X
+          if (!norm_mode) tc::mma_commit(bar(kXEmpty0 + b));  // norm mode: the epilogue frees X
         }
       }
       __syncwarp();
@@ -401,7 +561,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
       // epilogue: for rows r and r + 128, D of the row's 64 columns of every chunk and the
       // first minimum over the open groups, halves of the columns merged at the end
       const int r = (warp & 3) * 32 + lane;  // row within each 128-row half == TMEM lane
-      const int half = (warp - 4) >> 2;
+      const int half = (warp - 4) >> 2;      // columns [64 half, 64 half + 64) of every chunk
       const int etid = tid - 128;
       const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
       const float tau2 = a.tau2, m2t = -2.f * tau2;
@@ -415,7 +575,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
         if (norm_mode) {
           // x_i^T Gamma x_i: this thread's 64 accumulator columns (the 64-column box
           // `half` of its row) dotted with the same columns of x_i from the X tile
-          const uint8_t* xs = smem_raw + (sX - tc::saddr(smem_raw)) + half * (128 * 128) + r * 128;
+          const uint8_t* xs = smem_raw + (sX[it_epi & 1] - tc::saddr(smem_raw)) + half * (128 * 128) + r * 128;
           float part[2] = {0.f, 0.f};
           const bool got = !aborted && tc::mbar_wait(bar(kAccFull0 + (it_epi & 1)), (it_epi >> 1) & 1, abort_v, status);
           if (!__all_sync(0xffffffffu, got)) {
@@ -451,7 +611,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
             s_best_v[128 + r] = part[1];
           }
           asm volatile("bar.sync 1, 256;" ::: "memory");  // every X read of this item done
-          if (etid == 0 && !aborted) tc::mbar_arrive(bar(kXEmpty));
+          if (etid == 0 && !aborted) tc::mbar_arrive(bar(kXEmpty0 + (it_epi & 1)));
           if (half == 0 && !aborted) {
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
@@ -467,7 +627,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
           if (etid == 0) s_enf = 0;
           asm volatile("bar.sync 1, 256;" ::: "memory");
           const unsigned int* cl = a.closed + static_cast<size_t>(h) * words;
-          for (int c = etid; c < n_chunks * 128; c += 256) {
+          for (int c = etid; c < n_chunks * 128; c += kAsEpi) {
             float v = kAsInf;
             if (c < G) {
               const float e = tau2 * __ldcg(a.ecol + static_cast<size_t>(h) * G + c);
@@ -750,7 +910,8 @@ __global__ void __launch_bounds__(kAsThreads, 1)
     };
     for (int q = last_q - 1; q <= last_q; ++q)
       if (q >= 0) drain(bar(kWFull0 + (q & 1)), (q >> 1) & 1);
-    if (last_it >= 0) drain(bar(kXFull), last_it & 1);
+    for (int it = last_it - 1; it <= last_it; ++it)
+      if (it >= 0) drain(bar(kXFull0 + (it & 1)), (it >> 1) & 1);
   }
   if (warp == 2 && lane == 0) {
     tc::mma_commit(bar(kDrain));
@@ -771,7 +932,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
 }  // namespace
 
 size_t assign_tc_smem_bytes() {
-  return 1024 + 2 * kAsTile + 2ull * kAsWStage + sizeof(float) * kAsMaxCols + 2 * sizeof(int) * kAsMaxHeads;
+  return 1024 + 2ull * kAsXStage + 2ull * kAsWStage + sizeof(float) * kAsMaxCols + 2 * sizeof(int) * kAsMaxHeads;
 }
 
 cudaError_t launch_assign_tc(const __nv_bfloat16* X, const __nv_bfloat16* Whi, const __nv_bfloat16* Wlo,

@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(kFitThreads)
     double wp = 1.0;
     if (weights != nullptr) {
       wp = weights[static_cast<size_t>(head) * P + p];
-    } else if (weight_mode == 0) {
+    } else if ((weight_mode & kWeightModeMask) == 0) {
       double n2 = 0.0;
       for (int e = 0; e < D; ++e) {
         const double v = dp[static_cast<size_t>(p) * D + e];
@@ -407,12 +407,24 @@ __global__ void __launch_bounds__(kFitThreads)
     }
   }
   __syncthreads();
+  // ridge: lambda itself, or lambda times the mean diagonal entry of X_c^T W X_c (the
+  // scale-relative reading, weight_mode | kRidgeRelative)
+  double lam = lambda;
+  if (weight_mode & kRidgeRelative) {
+    double diag = 0.0;
+#pragma unroll
+    for (int k1 = 0; k1 < kRb; ++k1)
+#pragma unroll
+      for (int k2 = 0; k2 < kCb; ++k2)
+        if (bi + kNrb * k1 == bj + kNcb * k2) diag += acc[k1][k2];
+    lam = lambda * block_sum_d(diag, red) / static_cast<double>(D);
+  }
 #pragma unroll
   for (int k1 = 0; k1 < kRb; ++k1)
 #pragma unroll
     for (int k2 = 0; k2 < kCb; ++k2) {
       const int i = bi + kNrb * k1, j = bj + kNcb * k2;
-      C[i * LD + j] = acc[k1][k2] + (i == j ? lambda : 0.0);
+      C[i * LD + j] = acc[k1][k2] + (i == j ? lam : 0.0);
     }
   if (cross_regs) {
 #pragma unroll

@@ -7,6 +7,11 @@
 
 namespace spr {
 
+// weight_mode of the fit: the probe weights in the low byte (0 inverse squared norm, 1
+// uniform), kRidgeRelative set for lambda relative to the mean diagonal of X_c^T W X_c.
+constexpr int kWeightModeMask = 0xff;
+constexpr int kRidgeRelative = 0x100;
+
 __host__ __device__ size_t fit_scratch_doubles(int P, int d);
 size_t fit_smem_bytes(int d, int P);
 // Largest probe count the fit kernel takes at head dimension d (its shared memory).

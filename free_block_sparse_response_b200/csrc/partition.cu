@@ -552,41 +552,14 @@ __global__ void __launch_bounds__(kFillThreads, 3) fill_coop_kernel(FillArgs a) 
     const int ncur = __ldcg(a.list_len + cur);
     const int* L = lists[cur];
     // ---- propose
-    if (round == 0 && (a.prop_g0 != nullptr || a.seg_min != nullptr)) {
-      // first proposals: the row argmins, given, or the smallest segment key of the row
-      // (its first minimum among values below +inf; group 0 at +inf when it has none)
+    if (round == 0 && a.prop_g0 != nullptr) {
+      // first proposals: the row argmins the distance kernel found
       for (int x = gthread; x < ncur; x += nthreads) {
         const int item = __ldcg(L + x);
         const int h = item / n;
-        int g;
-        float v;
-        if (a.prop_g0 != nullptr) {
-          g = a.prop_g0[item];
-          v = a.prop_v0[item];
-        } else {
-          const ulonglong2* sk = reinterpret_cast<const ulonglong2*>(a.seg_min + static_cast<size_t>(item) * a.nseg);
-          unsigned long long key = ~0ull;
-          for (int t = 0; t < a.nseg / 2; ++t) {
-            const ulonglong2 kk = __ldcg(sk + t);
-            key = kk.x < key ? kk.x : key;
-            key = kk.y < key ? kk.y : key;
-          }
-          if (key == ~0ull) {  // no value below +inf: the whole row decides (+inf, then NaN)
-            const float* drow = a.D + static_cast<size_t>(item) * a.ldd;
-            bool saw_nan = false;
-            for (int c = 0; c < G; ++c) {
-              const float dv = __ldcg(drow + c);
-              saw_nan |= dv != dv;
-              const unsigned long long kk = decision_key(dv, c);
-              key = kk < key ? kk : key;
-            }
-            if (saw_nan) record_error(&a.hdr->status, kErrNonFinite);
-          }
-          g = static_cast<int>(key & 0xffffffffu);
-          v = float_from_order_key(static_cast<uint32_t>(key >> 32));
-        }
+        const int g = a.prop_g0[item];
         a.prop_g[item] = g;
-        a.prop_v[item] = v;
+        a.prop_v[item] = a.prop_v0[item];
         atomicAdd(a.cnt + static_cast<size_t>(h) * G + g, 1);
       }
     } else {
@@ -598,164 +571,6 @@ __global__ void __launch_bounds__(kFillThreads, 3) fill_coop_kernel(FillArgs a) 
         __syncthreads();
         closed_all = s_closed;
       }
-      if (a.seg_min != nullptr) {
-        // Four items per warp, 8 lanes each; lane s of a quarter holds the minimum keys of
-        // its row's 64-column segments s and s + 8.  The best open group is the smallest
-        // key among the segment minima whose group is open, unless a segment whose minimum
-        // group is full still has a key below it: only such segments are read (64 values,
-        // two 16-byte loads per lane), in ascending segment order, each read lowering the
-        // bound the remaining ones must beat.  Every key of a segment is >= its minimum
-        // key, so the result equals the argmin over the whole row's open groups.  The
-        // segment of the item's previous proposal (a group that has just filled, and the
-        // row's smallest key) is read in the same wave as the keys, since it nearly always
-        // has to be.
-        const int sub = lane & 7;
-        const int qb = lane & 24;  // first lane of this item's quarter
-        const unsigned long long inf_key = static_cast<unsigned long long>(float_order_key(__int_as_float(0x7f800000)))
-                                           << 32;
-        // Software pipeline: the item indices two batches ahead and the previous proposal
-        // (which names the segment read with the keys) one batch ahead.
-        const int stride = nwarps * 4;
-        int x = gwarp * 4 + (lane >> 3);
-        int item_a = x < ncur ? __ldcg(L + x) : 0;
-        int item_b = x + stride < ncur ? __ldcg(L + x + stride) : 0;
-        int gp_a = (x < ncur && round > 0) ? __ldcg(a.prop_g + item_a) : -1;
-        for (int x0 = gwarp * 4; x0 < ncur; x0 += stride, x += stride) {
-          const bool valid = x < ncur;
-          const int item = item_a;
-          const int gp = gp_a;
-          const int item_c = x + 2 * stride < ncur ? __ldcg(L + x + 2 * stride) : 0;
-          gp_a = (x + stride < ncur && round > 0) ? __ldcg(a.prop_g + item_b) : -1;
-          item_a = item_b;
-          item_b = item_c;
-          const int h = item / n;
-          const unsigned int* closed = closed_all + static_cast<size_t>(h) * words;
-          const float* drow = a.D + static_cast<size_t>(item) * a.ldd;
-          auto is_open = [&](int g) { return !((closed[g >> 5] >> (g & 31)) & 1u); };
-          unsigned long long* srow = a.seg_min + static_cast<size_t>(item) * a.nseg;
-          const unsigned long long key0 = valid && sub < a.nseg ? __ldcg(srow + sub) : ~0ull;
-          const unsigned long long key1 = valid && sub + 8 < a.nseg ? __ldcg(srow + sub + 8) : ~0ull;
-          const int sp = gp >= 0 ? (gp >> 7) * 2 + ((gp >> 6) & 1) : -1;
-          const int pcol0 = sp >= 0 ? (sp >> 1) * 128 + (sp & 1) * 64 : 0;
-          // lane sub's 8 columns of the 64-column segment at col0: col0 + 4 sub + {0..3} and
-          // col0 + 32 + 4 sub + {0..3} (two 16-byte loads when rows are 16-byte aligned)
-          auto load8 = [&](int col0, float4& va, float4& vb) {
-            va = make_float4(0.f, 0.f, 0.f, 0.f);
-            vb = va;
-            const int c0 = col0 + 4 * sub, c1 = col0 + 32 + 4 * sub;
-            if (a.d_vec4) {
-              if (c0 < G) va = __ldcg(reinterpret_cast<const float4*>(drow + c0));
-              if (c1 < G) vb = __ldcg(reinterpret_cast<const float4*>(drow + c1));
-            } else {
-              if (c0 < G) va.x = __ldcg(drow + c0);
-              if (c0 + 1 < G) va.y = __ldcg(drow + c0 + 1);
-              if (c0 + 2 < G) va.z = __ldcg(drow + c0 + 2);
-              if (c0 + 3 < G) va.w = __ldcg(drow + c0 + 3);
-              if (c1 < G) vb.x = __ldcg(drow + c1);
-              if (c1 + 1 < G) vb.y = __ldcg(drow + c1 + 1);
-              if (c1 + 2 < G) vb.z = __ldcg(drow + c1 + 2);
-              if (c1 + 3 < G) vb.w = __ldcg(drow + c1 + 3);
-            }
-          };
-          float4 pv0, pv1;
-          if (sp >= 0) {
-            load8(pcol0, pv0, pv1);
-          } else {
-            pv0 = make_float4(0.f, 0.f, 0.f, 0.f);
-            pv1 = pv0;
-          }
-          // per segment s in {sub, sub + 8}: is its minimum group open, and its lower bound
-          const int kg0 = key0 < kSegNoOpen ? static_cast<int>(key0 & 0xffffffffu) : -1;
-          const int kg1 = key1 < kSegNoOpen ? static_cast<int>(key1 & 0xffffffffu) : -1;
-          const bool kopen0 = kg0 >= 0 && is_open(kg0);
-          const bool kopen1 = kg1 >= 0 && is_open(kg1);
-          const int scol0 = (sub >> 1) * 128 + (sub & 1) * 64;
-          const int scol1 = ((sub + 8) >> 1) * 128 + ((sub + 8) & 1) * 64;
-          const bool has0 = valid && sub < a.nseg && scol0 < G && key0 != kSegNoOpen;
-          const bool has1 = valid && sub + 8 < a.nseg && scol1 < G && key1 != kSegNoOpen;
-          // a segment without a value below +inf (key ~0) is bounded below by +inf at its
-          // first column
-          const unsigned long long lb0 = kg0 >= 0 ? key0 : inf_key | static_cast<uint32_t>(scol0);
-          const unsigned long long lb1 = kg1 >= 0 ? key1 : inf_key | static_cast<uint32_t>(scol1);
-          unsigned long long best = kopen0 ? key0 : ~0ull;
-          if (kopen1 && key1 < best) best = key1;
-          bool saw_nan = false;
-          auto scan8 = [&](int col0, const float4& va, const float4& vb, unsigned long long& bb) {
-            const float vv[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              const int g = col0 + (t >> 2) * 32 + 4 * sub + (t & 3);
-              if (g < G && is_open(g)) {
-                saw_nan |= (vv[t] != vv[t]);
-                const unsigned long long kk = decision_key(vv[t], g);
-                bb = kk < bb ? kk : bb;
-              }
-            }
-          };
-          unsigned long long pbest = ~0ull;  // the previous proposal's segment, open groups
-          if (sp >= 0) scan8(pcol0, pv0, pv1, pbest);
-#pragma unroll
-          for (int o = 4; o > 0; o >>= 1) {
-            const unsigned long long y = __shfl_xor_sync(0xffffffffu, best, o);
-            best = y < best ? y : best;
-            const unsigned long long z = __shfl_xor_sync(0xffffffffu, pbest, o);
-            pbest = z < pbest ? z : pbest;
-          }
-          best = pbest < best ? pbest : best;
-          if (sp >= 0 && sub == 0) srow[sp] = pbest == ~0ull ? kSegNoOpen : pbest;
-          // Segments that may still hold a better open group are read two at a time, those
-          // with the smallest lower bounds first (a lower bound is a distinct key, so it
-          // names its segment); after each pair the bound the others must beat drops.
-          bool need0 = has0 && !kopen0 && sub != sp && lb0 < best;
-          bool need1 = has1 && !kopen1 && sub + 8 != sp && lb1 < best;
-          auto quarter_min = [&](unsigned long long v) {
-#pragma unroll
-            for (int o = 4; o > 0; o >>= 1) {
-              const unsigned long long y = __shfl_xor_sync(0xffffffffu, v, o);
-              v = y < v ? y : v;
-            }
-            return v;
-          };
-          auto seg_col = [&](unsigned long long lbk) {
-            const int c = static_cast<int>(lbk & 0xffffffffu);
-            return (c >> 6) << 6;  // first column of the segment holding column c
-          };
-          while (__any_sync(0xffffffffu, need0 || need1)) {
-            const unsigned long long c0 = need0 ? lb0 : ~0ull, c1 = need1 ? lb1 : ~0ull;
-            const unsigned long long A = quarter_min(c0 < c1 ? c0 : c1);
-            const unsigned long long d0 = c0 == A ? ~0ull : c0, d1 = c1 == A ? ~0ull : c1;
-            const unsigned long long B = quarter_min(d0 < d1 ? d0 : d1);
-            unsigned long long ba = ~0ull, bbk = ~0ull;
-            float4 va, vb, wa, wb;
-            if (A != ~0ull) load8(seg_col(A), va, vb);
-            if (B != ~0ull) load8(seg_col(B), wa, wb);
-            if (A != ~0ull) scan8(seg_col(A), va, vb, ba);
-            if (B != ~0ull) scan8(seg_col(B), wa, wb, bbk);
-            ba = quarter_min(ba);
-            bbk = quarter_min(bbk);
-            if (sub == 0) {  // keep the segment minima current (open groups only)
-              if (A != ~0ull) srow[seg_col(A) >> 6] = ba == ~0ull ? kSegNoOpen : ba;
-              if (B != ~0ull) srow[seg_col(B) >> 6] = bbk == ~0ull ? kSegNoOpen : bbk;
-            }
-            const unsigned long long bb = ba < bbk ? ba : bbk;
-            best = bb < best ? bb : best;
-            need0 = need0 && lb0 != A && lb0 != B && lb0 < best;
-            need1 = need1 && lb1 != A && lb1 != B && lb1 < best;
-          }
-          saw_nan = ((__ballot_sync(0xffffffffu, saw_nan) >> qb) & 0xffu) != 0u && valid;
-          if (sub == 0 && valid) {
-            if (saw_nan) record_error(&a.hdr->status, kErrNonFinite);
-            if (best == ~0ull) {
-              record_error(&a.hdr->status, kErrInvalidArg);
-            } else {
-              const int g = static_cast<int>(best & 0xffffffffu);
-              a.prop_g[item] = g;
-              a.prop_v[item] = float_from_order_key(static_cast<uint32_t>(best >> 32));
-              atomicAdd(a.cnt + static_cast<size_t>(h) * G + g, 1);
-            }
-          }
-        }
-      } else
       // One item per warp, with the item's whole distance row (up to MAXW values per
       // lane) requested before any is used; full-group bitmap words are warp-uniform.
       for (int x = gwarp; x < ncur; x += nwarps) {
@@ -880,37 +695,6 @@ __global__ void __launch_bounds__(kFillThreads, 3) fill_coop_kernel(FillArgs a) 
   }
 }
 
-// Segment minima of a row-major matrix (the convention of the tensor-core distance
-// kernel): per row and 64-column segment, the key of its first minimum among values
-// below +inf, or ~0 when it has none; a NaN is recorded as a non-finite input.  One warp
-// per (row, segment).
-__global__ void segment_minima_kernel(const float* __restrict__ D, int ldd, long long rows, int G,
-                                      unsigned long long* __restrict__ seg, int nseg, int* __restrict__ status) {
-  const int lane = threadIdx.x & 31;
-  const long long total = rows * nseg;
-  for (long long w = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5; w < total;
-       w += (static_cast<long long>(gridDim.x) * blockDim.x) >> 5) {
-    const long long row = w / nseg;
-    const int s = static_cast<int>(w - row * nseg);
-    const int col0 = (s >> 1) * 128 + (s & 1) * 64;
-    unsigned long long b = ~0ull;
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int c = col0 + 32 * t + lane;
-      if (c < G) {
-        const float v = D[row * ldd + c];
-        if (v != v) record_error(status, kErrNonFinite);
-        if (v < __int_as_float(0x7f800000)) {
-          const unsigned long long k = decision_key(v, c);
-          b = k < b ? k : b;
-        }
-      }
-    }
-    b = warp_min_u64(b);
-    if (lane == 0) seg[w] = b;
-  }
-}
-
 // ----------------------------------------------------------------- labels -> permutation
 __global__ void perm_scatter_kernel(const int* __restrict__ labels, int n, int G, int cap,
                                     int* __restrict__ cursor, int* __restrict__ tmp, int heads,
@@ -1010,11 +794,6 @@ __global__ void __launch_bounds__(256) block_score_kernel(const float* __restric
 
 // ----------------------------------------------------------------------------- launchers
 
-cudaError_t launch_segment_minima(const float* D, int ldd, long long rows, int G, unsigned long long* seg, int nseg,
-                                  int* status, cudaStream_t st) {
-  segment_minima_kernel<<<1024, 256, 0, st>>>(D, ldd, rows, G, seg, nseg, status);
-  return counted(cudaGetLastError(), 1);
-}
 
 __global__ void identity_kernel(float* __restrict__ gamma, int heads, int d) {
   const size_t total = static_cast<size_t>(heads) * d * d;
@@ -1106,7 +885,6 @@ cudaError_t launch_rowgemm(const RowGemmArgs& a, bool dist, cudaStream_t st) {
     return counted(cudaGetLastError(), 1);
   }
   const bool split = a.Blo != nullptr;
-  if (dist && a.d == 128) return launch_dist_tc(a, a.ldd, st);
   if (a.d == 64) {
     if (dist) return split ? launch_rowgemm_mma_t<64, true, true>(a, st) : launch_rowgemm_mma_t<64, true, false>(a, st);
     return split ? launch_rowgemm_mma_t<64, false, true>(a, st) : launch_rowgemm_mma_t<64, false, false>(a, st);

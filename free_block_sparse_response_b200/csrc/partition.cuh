@@ -23,30 +23,15 @@ struct RowGemmArgs {
   int ldd;                   // DIST: row stride of Dout (>= ncols)
   int* prop_g;               // DIST: [heads, n]
   float* prop_v;
-  // DIST, tensor-core path (optional): per item the minimum key of every 64-column
-  // segment of its row, [heads, n, nseg], nseg = 2 ceil(ncols / 128); ~0 for a segment
-  // without a finite value.  A key is order_key(D) << 32 | column.
-  unsigned long long* seg_min;
-  int nseg;
   float* nrm_out;            // NORM: [heads, n]
   int* status;
 };
-
-// Segment-minimum entry of a segment whose groups are all full.
-constexpr unsigned long long kSegNoOpen = ~0ull - 1;
 
 struct FillArgs {
   const float* D;       // [heads, n, ldd]
   int ldd;              // row stride of D (>= G)
   const int* prop_g0;   // optional first proposals [heads, n]
   const float* prop_v0;
-  // optional segment minima of every D row (see RowGemmArgs::seg_min): later proposals
-  // read those instead of the whole row, and only the segments that can still hold a
-  // better open group than the best open segment minimum.  The fill keeps them current:
-  // a segment it reads gets the minimum over its open groups written back (or
-  // kSegNoOpen when none is open), which stays a lower bound since groups only close.
-  unsigned long long* seg_min;
-  int nseg;
   int heads, n, G, cap;
   int* labels;          // [heads, n]
   int* room;            // [heads, G]
@@ -108,8 +93,6 @@ cudaError_t launch_row_norms_tc(const __nv_bfloat16* X, const __nv_bfloat16* ghi
 cudaError_t launch_midpoint_stride(int* idx, int n, int count, cudaStream_t st);
 // gamma [heads, d, d] = identity (the metric of the semantic partition)
 cudaError_t launch_identity(float* gamma, int heads, int d, cudaStream_t st);
-cudaError_t launch_segment_minima(const float* D, int ldd, long long rows, int G, unsigned long long* seg, int nseg,
-                                  int* status, cudaStream_t st);
 cudaError_t launch_gram(const void* X, bool f32, size_t head_stride, const int* rows, int nrows, int heads,
                         int d, float* gamma, cudaStream_t st);
 cudaError_t launch_split_bf16(const float* src, __nv_bfloat16* hi, __nv_bfloat16* lo, size_t count,
@@ -120,7 +103,6 @@ cudaError_t launch_centroid(const void* X, bool f32, int n, const int* perm, con
 cudaError_t launch_wmat(const float* cent, const float* gamma, int G, int heads, int d, float* wf,
                         __nv_bfloat16* whi, __nv_bfloat16* wlo, float* eg, cudaStream_t st);
 cudaError_t launch_rowgemm(const RowGemmArgs& a, bool dist, cudaStream_t st);
-cudaError_t launch_dist_tc(const RowGemmArgs& a, int ldd, cudaStream_t st);
 cudaError_t launch_fill(const FillArgs& a, cudaStream_t st);
 cudaError_t launch_build_perm(const int* labels, int n, int G, int cap, int heads, int* cursor, int* tmp,
                               int* perm, int* sizes, int* status, cudaStream_t st);

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsparsepr
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NONFINITE = range(6)
 BF16, F32 = 0, 1
 WEIGHT_INV_NORM, WEIGHT_UNIFORM = 0, 1
+RIDGE_RELATIVE = 0x100  # weight_mode option bit: lambda relative to tr(X_c^T W X_c) / d
 PARTITION_RESPONSE, PARTITION_SEMANTIC = 0, 1
 ROUTE_CENTROID, ROUTE_SIZE_CORRECTED, ROUTE_LSE = 0, 1, 2
 BUDGET_UNIFORM, BUDGET_GLOBAL = 0, 1
@@ -29,7 +30,7 @@ EXPORTED_SYMBOLS = (
     "sparsepr_probe_dense", "sparsepr_fit_residual", "sparsepr_apply_residual", "sparsepr_check",
     "sparsepr_last_error", "sparsepr_test_fill_workspace_size", "sparsepr_test_fill",
     "sparsepr_test_topk", "sparsepr_row_errors", "sparsepr_launch_count", "sparsepr_fit_residual_noalloc",
-    "sparsepr_kernel_timing", "sparsepr_kernel_timing_read", "sparsepr_test_fill_segmented",
+    "sparsepr_kernel_timing", "sparsepr_kernel_timing_read",
     "sparsepr_sparse_attn_apply", "sparsepr_reset_workspace", "sparsepr_call_workspace_size", "sparsepr_attention",
     "sparsepr_host_workspace_size", "sparsepr_attention_host", "sparsepr_test_partition_trace",
 )
@@ -122,7 +123,6 @@ def load_library(path: str) -> ctypes.CDLL:
         "sparsepr_last_error": (ctypes.c_char_p, []),
         "sparsepr_test_fill_workspace_size": (ctypes.c_size_t, [_i32, _i32, _i32]),
         "sparsepr_test_fill": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
-        "sparsepr_test_fill_segmented": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
         "sparsepr_test_topk": (ctypes.c_int, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
         "sparsepr_row_errors": (ctypes.c_int, [_vp, ctypes.c_int, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
         "sparsepr_launch_count": (ctypes.c_uint64, []),
@@ -419,17 +419,13 @@ def launch_count() -> int:
 
 # ------------------------------------------------------- decision kernels, injected input
 
-def test_fill(dist: torch.Tensor, cap: int, segmented: bool = False) -> torch.Tensor:
-    """Capacity fill on injected fp32 distances [H, n, G] -> labels [H, n] int32.
-
-    ``segmented`` takes the proposals from the rows' 64-column segment minima (the path
-    of the bf16, d = 128 partition); the labels must not change.
-    """
+def test_fill(dist: torch.Tensor, cap: int) -> torch.Tensor:
+    """Capacity fill on injected fp32 distances [H, n, G] -> labels [H, n] int32."""
     _need_cuda(dist)
     h, n, g = dist.shape
     ws = torch.empty(int(lib().sparsepr_test_fill_workspace_size(h, n, g)), dtype=torch.uint8, device=dist.device)
     labels = torch.empty(h, n, dtype=torch.int32, device=dist.device)
-    _call("sparsepr_test_fill_segmented" if segmented else "sparsepr_test_fill", _p(dist), h, n, g, cap, _p(labels),
+    _call("sparsepr_test_fill", _p(dist), h, n, g, cap, _p(labels),
           _p(ws), _stream(dist))
     check(ws)
     return labels

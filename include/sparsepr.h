@@ -75,6 +75,14 @@ enum { SPARSEPR_BF16 = 0, SPARSEPR_F32 = 1 };
 
 enum { SPARSEPR_WEIGHT_INV_NORM = 0, SPARSEPR_WEIGHT_UNIFORM = 1 };
 
+/* Option bit of weight_mode (the fit's parameters): the ridge lambda is taken relative to
+ * the scale of the probe outputs, lambda_eff = lambda * tr(X_c^T W X_c) / d, instead of
+ * as an absolute number.  The abstract says "weighted ridge regression" without the scale
+ * of lambda; absolute lambda (the default) is the plain reading, the relative one makes
+ * the fit invariant to the scale of the outputs and is what the probe-budget study
+ * compares it with. */
+enum { SPARSEPR_RIDGE_RELATIVE = 0x100 };
+
 /* Partition rule.  RESPONSE: Response-Coupled Partitioning (the method).  SEMANTIC: the
  * semantic block-sparse baseline the pages compare against, read as balanced k-means on
  * the raw keys and on the raw queries (same start, fill, iterations and routing); the
@@ -103,7 +111,8 @@ typedef struct sparsepr_params {
   int32_t n_probe;      /* P: exact probe rows per head                                 */
   int32_t kmeans_iters; /* T: balanced k-means iterations on each side (>= 0)           */
   int32_t rank;         /* r: residual subspace rank (clamped to d)                    */
-  int32_t weight_mode;  /* SPARSEPR_WEIGHT_*: probe weights when none are supplied      */
+  int32_t weight_mode;  /* SPARSEPR_WEIGHT_* (probe weights when none are supplied),
+                           optionally | SPARSEPR_RIDGE_RELATIVE                           */
   double density;       /* rho: executed-pair budget / N^2, probe rows counted          */
   double ridge_lambda;  /* lambda: ridge on the centred weighted Gram (sum w = P)       */
   float scale;          /* softmax scale tau; <= 0 selects 1/sqrt(d)                    */
@@ -256,7 +265,8 @@ SPARSEPR_API int sparsepr_probe_dense(const void* Q, const void* K, const void* 
  *   else weight_mode (inverse squared norm of probe_out_p, or uniform), then scaled
  *   so sum_p w_p = P;  U_r = top-r eigenvectors of sum_p w_p y_p y_p^T;
  *   z_p = U_r^T y_p;  A = (Z_c^T W X_c)(X_c^T W X_c + lambda I)^-1 with X = probe_sparse
- *   centred at its weighted mean;  b = zbar - A xbar.
+ *   centred at its weighted mean (lambda times tr(X_c^T W X_c) / d when weight_mode has
+ *   SPARSEPR_RIDGE_RELATIVE);  b = zbar - A xbar.
  *   Outputs M = U_r A [Bt,H,d,d] and beta = U_r b [Bt,H,d], fp32. */
 SPARSEPR_API int sparsepr_fit_residual(const float* probe_sparse, const float* probe_out,
                           const float* weights, int32_t Bt, int32_t H, int32_t d,
@@ -334,19 +344,16 @@ SPARSEPR_API int sparsepr_reset_workspace(void* ws, sparsepr_stream_t stream);
 SPARSEPR_API const char* sparsepr_last_error(void);
 
 /* ---- decision kernels on injected scores (used by the parity tests) ---------------
- * sparsepr_test_fill: the capacity-B assignment used by every k-means iteration, run
- *   on caller-supplied fp32 distances D [H, n, G] (device); labels [H, n] int32.
- * sparsepr_test_fill_segmented: the same assignment with the proposals taken from the
- *   minima of the rows' 64-column segments (the path the bf16, d = 128 partition runs):
- *   the labels must equal sparsepr_test_fill's for every D.
+ * sparsepr_test_fill: the capacity-B assignment of a k-means iteration (the fill kernel
+ *   of the fp32 and d = 64 partitions; the bf16, d = 128 partition runs the same decision
+ *   rule inside its tensor-core assignment kernel, whose decisions the partition trace
+ *   exposes), run on caller-supplied fp32 distances D [H, n, G] (device); labels [H, n]
+ *   int32; workspace of sparsepr_test_fill_workspace_size bytes.
  * sparsepr_test_topk: the routing selection on caller-supplied scores Sc [H, Gq, G];
- *   route [H, Gq, k] int32.  All use the same kernels as the operator; the fill calls
- *   share sparsepr_test_fill_workspace_size. */
+ *   route [H, Gq, k] int32.  Both use the same kernels as the operator. */
 SPARSEPR_API size_t sparsepr_test_fill_workspace_size(int32_t H, int32_t n, int32_t G);
 SPARSEPR_API int sparsepr_test_fill(const float* D, int32_t H, int32_t n, int32_t G, int32_t cap,
                        int32_t* labels, void* ws, sparsepr_stream_t stream);
-SPARSEPR_API int sparsepr_test_fill_segmented(const float* D, int32_t H, int32_t n, int32_t G,
-                       int32_t cap, int32_t* labels, void* ws, sparsepr_stream_t stream);
 SPARSEPR_API int sparsepr_test_topk(const float* Sc, int32_t H, int32_t Gq, int32_t G, int32_t k,
                        int32_t* route, void* ws, sparsepr_stream_t stream);
 

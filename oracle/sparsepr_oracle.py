@@ -460,16 +460,21 @@ def probe_weights(d_probe: np.ndarray, mode: str = "inv_norm",
     return w * (p / total)
 
 
-def ridge_affine(x: np.ndarray, z: np.ndarray, w: np.ndarray, ridge_lambda: float):
+def ridge_affine(x: np.ndarray, z: np.ndarray, w: np.ndarray, ridge_lambda: float,
+                 ridge_mode: str = "absolute"):
     """Weighted ridge regression z ~ A x + b with an unpenalised bias ([abs]: the
     affine correction is fitted by weighted ridge regression).  Centring at the
     weighted means removes the bias from the penalised system:
-    A = (Z_c^T W X_c)(X_c^T W X_c + lambda I)^-1, b = zbar - A xbar (Cholesky)."""
+    A = (Z_c^T W X_c)(X_c^T W X_c + lambda I)^-1, b = zbar - A xbar (Cholesky).
+    ``ridge_mode`` "relative" (the other reading of the unstated lambda scale) uses
+    lambda * tr(X_c^T W X_c) / d in place of lambda."""
     wsum = w.sum()
     xbar = (w @ x) / wsum
     zbar = (w @ z) / wsum
     xc, zc = x - xbar, z - zbar
-    gram = xc.T @ (w[:, None] * xc) + ridge_lambda * np.eye(x.shape[1])
+    gram = xc.T @ (w[:, None] * xc)
+    lam = ridge_lambda * np.trace(gram) / x.shape[1] if ridge_mode == "relative" else ridge_lambda
+    gram = gram + lam * np.eye(x.shape[1])
     cross = zc.T @ (w[:, None] * xc)                 # [r, d]
     a = cholesky_solve(cholesky(gram), cross.T).T    # gram is symmetric
     return a, zbar - a @ xbar
@@ -477,7 +482,7 @@ def ridge_affine(x: np.ndarray, z: np.ndarray, w: np.ndarray, ridge_lambda: floa
 
 def fit_residual(s_probe: np.ndarray, d_probe: np.ndarray, ridge_lambda: float,
                  rank: int, weight_mode: str = "inv_norm",
-                 weights: Optional[np.ndarray] = None) -> dict:
+                 weights: Optional[np.ndarray] = None, ridge_mode: str = "absolute") -> dict:
     """Probe-Fitted Residual Reconstruction, the fit ([abs], [news]).
 
     Residual y_p = d_p - s_p of every probe; U_r = top-r eigenvectors of
@@ -494,7 +499,7 @@ def fit_residual(s_probe: np.ndarray, d_probe: np.ndarray, ridge_lambda: float,
     r = min(rank, d)
     u = evecs[:, :r]
     z = y @ u
-    a, b = ridge_affine(x, z, w, ridge_lambda)
+    a, b = ridge_affine(x, z, w, ridge_lambda, ridge_mode)
     gap = (evals[r - 1] - evals[r]) / evals[0] if r < d and evals[0] > 0 else np.inf
     return {"M": u @ a, "beta": u @ b, "U": u, "A": a, "b": b, "evals": evals,
             "weights": w, "eigengap": gap}

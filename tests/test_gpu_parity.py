@@ -93,24 +93,22 @@ def test_fill_bit_exact_on_oracle_kmeans_distances():
                     w.n_sampled, w.kmeans_iters, dump=dump)
         for dmat in dump["key_dist"] + dump["query_dist"]:
             expect = O.fill(dmat, w.block)
-            for segmented in (False, True):
-                gpu = spr.test_fill(torch.from_numpy(dmat)[None].cuda(), w.block, segmented)[0].cpu().numpy()
-                assert np.array_equal(gpu, expect), segmented
+            gpu = spr.test_fill(torch.from_numpy(dmat)[None].cuda(), w.block)[0].cpu().numpy()
+            assert np.array_equal(gpu, expect)
 
 
 @pytest.mark.parametrize("heads,n,g,cap,levels", [(1, 1000, 16, 64, 4), (3, 300, 7, 50, 3), (2, 4096, 33, 128, 1000),
                                                   (1, 64, 64, 1, 2), (2, 777, 13, 64, 0), (1, 36000, 300, 128, 1000),
                                                   (2, 9000, 300, 32, 6), (1, 5000, 200, 25, 0)])
-@pytest.mark.parametrize("segmented", [False, True])
-def test_fill_bit_exact_random_with_ties(heads, n, g, cap, levels, segmented):
+def test_fill_bit_exact_random_with_ties(heads, n, g, cap, levels):
     """Random distances with heavy ties (and signed zeros and infinities when levels = 0);
-    the larger cases fill most groups, so the segmented proposals read many segments."""
+    the larger cases fill most groups and run many proposal rounds."""
     rng = np.random.default_rng(n + g)
     if levels == 0:   # signed zeros and infinities
         dmat = rng.choice(np.array([0.0, -0.0, 1.0, np.inf], dtype=np.float32), size=(heads, n, g))
     else:
         dmat = rng.integers(0, levels, size=(heads, n, g)).astype(np.float32) * np.float32(0.5)
-    gpu = spr.test_fill(torch.from_numpy(dmat).cuda(), cap, segmented).cpu().numpy()
+    gpu = spr.test_fill(torch.from_numpy(dmat).cuda(), cap).cpu().numpy()
     for h in range(heads):
         assert np.array_equal(gpu[h], O.fill(dmat[h], cap))
 
@@ -171,10 +169,9 @@ def test_nan_scores_are_reported():
     assert ei.value.code == spr.ERR_NONFINITE
     dmat = np.ones((1, 10, 4), dtype=np.float32)
     dmat[0, 3, 1] = np.nan
-    for segmented in (False, True):
-        with pytest.raises(spr.SparsePRError) as ei:
-            spr.test_fill(torch.from_numpy(dmat).cuda(), 4, segmented)
-        assert ei.value.code == spr.ERR_NONFINITE
+    with pytest.raises(spr.SparsePRError) as ei:
+        spr.test_fill(torch.from_numpy(dmat).cuda(), 4)
+    assert ei.value.code == spr.ERR_NONFINITE
 
 
 # ------------------------------------------------------------------- whole-call parity

@@ -162,6 +162,46 @@ def test_ridge_matches_augmented_normal_equations(p, d, r, lam):
     assert np.max(np.abs(a - theta2[:d].T)) <= 1e-9 * max(1.0, np.max(np.abs(theta2)))
 
 
+@pytest.mark.parametrize("p,d,r,lam", [(40, 12, 3, 1e-3), (10, 12, 4, 1e-2), (64, 8, 8, 0.5)])
+def test_relative_ridge_matches_augmented_normal_equations(p, d, r, lam):
+    """The scale-relative reading of lambda (ridge_mode "relative"): the same augmented
+    normal equations with lambda_eff = lambda * (sum_p w_p |x_p - xbar|^2) / d, that sum
+    (the trace of the centred weighted Gram) formed here row by row in long double."""
+    rng = _rng(17)
+    x = rng.normal(size=(p, d)) * 3.0 + 0.3
+    z = rng.normal(size=(p, r))
+    w = rng.uniform(0.2, 2.0, size=p)
+    a, b = O.ridge_affine(x, z, w, lam, ridge_mode="relative")
+    xl, wl = x.astype(np.longdouble), w.astype(np.longdouble)
+    xbar = sum(wl[i] * xl[i] for i in range(p)) / sum(wl)
+    spread = sum(wl[i] * sum((xl[i, e] - xbar[e]) ** 2 for e in range(d)) for i in range(p))
+    lam_eff = float(lam * spread / d)
+    xa = np.concatenate([x, np.ones((p, 1))], axis=1)
+    lhs = xa.T @ (w[:, None] * xa)
+    lhs[:d, :d] += lam_eff * np.eye(d)
+    rhs = xa.T @ (w[:, None] * z)
+    theta = _gauss_jordan_solve(lhs, rhs).astype(np.float64)
+    assert np.max(np.abs(a - theta[:d].T)) <= 1e-10 * max(1.0, np.max(np.abs(theta)))
+    assert np.max(np.abs(b - theta[d])) <= 1e-10 * max(1.0, np.max(np.abs(theta)))
+
+
+def test_relative_ridge_makes_the_fit_scale_invariant():
+    """Scaling the sparse and the dense probe outputs by s leaves M unchanged and scales
+    beta by s under the relative lambda (weights, subspace and Gram all scale
+    consistently); under the absolute lambda M moves (lambda does not scale)."""
+    rng = _rng(18)
+    p, d, r, lam, s = 20, 16, 4, 1e-2, 1e-2
+    xs = rng.normal(size=(p, d))
+    dp = xs + 0.3 * rng.normal(size=(p, d)) @ rng.normal(size=(d, d)) * 0.2 + 0.1
+    f1 = O.fit_residual(xs, dp, lam, r, ridge_mode="relative")
+    f2 = O.fit_residual(s * xs, s * dp, lam, r, ridge_mode="relative")
+    assert np.max(np.abs(f2["M"] - f1["M"])) <= 1e-9 * np.max(np.abs(f1["M"]))
+    assert np.max(np.abs(f2["beta"] - s * f1["beta"])) <= 1e-9 * np.max(np.abs(s * f1["beta"]))
+    g1 = O.fit_residual(xs, dp, lam, r)
+    g2 = O.fit_residual(s * xs, s * dp, lam, r)
+    assert np.max(np.abs(g2["M"] - g1["M"])) > 1e-3 * np.max(np.abs(g1["M"]))
+
+
 @pytest.mark.parametrize("d,rank_c,r", [(12, 12, 4), (24, 6, 8), (32, 32, 32)])
 def test_jacobi_subspace_matches_eigh(d, rank_c, r):
     """Top-r projector and eigenvalues of the oracle's Jacobi match numpy.linalg.eigh
