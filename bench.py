@@ -620,24 +620,34 @@ def run_study_ablation(args, w):
 
 def run_study_probe_budget(args, w):
     """Mean and p99 unprobed-row error against the probe budget P (k re-derived from
-    the pair budget for each P), with the uncorrected output at the same density."""
-    _, spr = _gpu_modules()
+    the pair budget for each P), with the uncorrected output at the same density, under
+    the two readings of the ridge scale: lambda absolute (on a Gram whose weights sum to
+    P), and lambda relative to tr(X_c^T W X_c) / d (RIDGE_RELATIVE); the partition,
+    routes, probe rows and sparse output are shared, only the fit and apply differ."""
+    torch, spr = _gpu_modules()
     q, k, v, dense = _study_inputs(args, w)
     bt, h, n, d = q.shape
     for P in (32, 64, 128, 256, 512):
+        if P > n:
+            continue
         cfg = spr.SparsePRConfig(block=w.block, n_sampled=w.n_sampled, n_probe=P, kmeans_iters=w.kmeans_iters,
                                  rank=w.rank, density=w.density, ridge_lambda=w.ridge_lambda)
         ws = spr.new_workspace(bt, h, n, d, cfg, q.device)
         pidx = spr.probe_rows(n, P, bt, h, q.device)
         o, parts = spr.attention(q, k, v, cfg, ws=ws, return_parts=True, fused=False)
-        m, p = _err_summary(spr.row_errors(o, dense, pidx))
         mu, pu = _err_summary(spr.row_errors(parts["S"], dense, pidx))
-        spr.check(ws)
-        print(json.dumps({"study": "probe-budget", "workload": config_block(w, args)["workload"], "P": P,
-                          "k": parts["k"], "density": float(parts["executed_pairs"].double().sum()) /
-                          (float(n) ** 2 * h * bt), "mean_rel_l2": m, "p99_rel_l2": p,
-                          "uncorrected_mean_rel_l2": mu, "uncorrected_p99_rel_l2": pu,
-                          "mean_error_reduction": 1.0 - m / mu, "seed": args.seed}), flush=True)
+        for ridge, flag in (("absolute", 0), ("relative", spr.RIDGE_RELATIVE)):
+            rcfg = dataclasses.replace(cfg, weight_mode=cfg.weight_mode | flag)
+            m_, b_ = spr.fit_residual(parts["probe_sparse"], parts["probe_out"], rcfg, ws)
+            o_r = spr.apply_residual(parts["S"], m_, b_, parts["probe_idx"], parts["probe_out"], out_dtype=q.dtype)
+            m, p = _err_summary(spr.row_errors(o_r, dense, pidx))
+            spr.check(ws)
+            print(json.dumps({"study": "probe-budget", "workload": config_block(w, args)["workload"], "P": P,
+                              "ridge": ridge, "lambda": w.ridge_lambda,
+                              "k": parts["k"], "density": float(parts["executed_pairs"].double().sum()) /
+                              (float(n) ** 2 * h * bt), "mean_rel_l2": m, "p99_rel_l2": p,
+                              "uncorrected_mean_rel_l2": mu, "uncorrected_p99_rel_l2": pu,
+                              "mean_error_reduction": 1.0 - m / mu, "seed": args.seed}), flush=True)
         del ws
 
 

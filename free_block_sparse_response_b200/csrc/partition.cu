@@ -200,7 +200,9 @@ __global__ void __launch_bounds__(256) group_update_kernel(const T* __restrict__
                                                            float* __restrict__ wf, __nv_bfloat16* __restrict__ whi,
                                                            __nv_bfloat16* __restrict__ wlo, float* __restrict__ eg) {
   constexpr int kPer = D / 32, kSets = 256 / D, kPerSet = 8 / kSets;
+  constexpr int kGRows = 32;  // rows of Gamma staged at a time
   __shared__ int sv[8][128];
+  __shared__ float sg[kGRows][D];
   __shared__ float sc[8][D];
   __shared__ float red[8][D / 32];
   const int head = blockIdx.y, g0 = blockIdx.x * 8;
@@ -262,10 +264,16 @@ __global__ void __launch_bounds__(256) group_update_kernel(const T* __restrict__
   float acc[kPerSet];
 #pragma unroll
   for (int j = 0; j < kPerSet; ++j) acc[j] = 0.f;
-  for (int f = 0; f < D; ++f) {
-    const float gv = gm[f * D + e];
+  for (int f0 = 0; f0 < D; f0 += kGRows) {
+    for (int x = threadIdx.x; x < kGRows * D; x += 256) sg[x / D][x % D] = __ldg(gm + f0 * D + x);
+    __syncthreads();
+#pragma unroll 8
+    for (int f = 0; f < kGRows; ++f) {
+      const float gv = sg[f][e];
 #pragma unroll
-    for (int j = 0; j < kPerSet; ++j) acc[j] += sc[set * kPerSet + j][f] * gv;
+      for (int j = 0; j < kPerSet; ++j) acc[j] += sc[set * kPerSet + j][f0 + f] * gv;
+    }
+    __syncthreads();
   }
 #pragma unroll
   for (int j = 0; j < kPerSet; ++j) {

@@ -332,6 +332,27 @@ def test_fit_kernel_matches_oracle_on_identical_inputs(rank):
         assert rel(parts["beta"][0, h].cpu().numpy(), fit["beta"]) <= 1e-5
 
 
+def test_fit_relative_ridge_matches_oracle_on_identical_inputs():
+    """The scale-relative lambda (weight_mode | RIDGE_RELATIVE): the fit kernel against
+    the oracle's ridge_mode "relative" on the GPU's own probe outputs (Small, P = 64 < d,
+    where lambda matters), and the whole call with the option against the oracle."""
+    w = CONFIGS["small"]
+    q, k, v = make_inputs(w, 0, heads=2)
+    cfg = spr_cfg(w, weight_mode=spr.WEIGHT_INV_NORM | spr.RIDGE_RELATIVE, ridge_lambda=0.05)
+    o, parts = run_call(w, q, k, v, cfg)
+    for h in range(2):
+        xs = parts["probe_sparse"][0, h].double().cpu().numpy()
+        dp = parts["probe_out"][0, h].double().cpu().numpy()
+        fit = O.fit_residual(xs, dp, cfg.ridge_lambda, cfg.rank, ridge_mode="relative")
+        assert rel(parts["M"][0, h].cpu().numpy(), fit["M"]) <= 1e-5
+        assert rel(parts["beta"][0, h].cpu().numpy(), fit["beta"]) <= 1e-5
+        ref = oracle_on_gpu_decisions(q, k, v, parts, h, cfg, w.n_tokens)
+        fit_ref = O.fit_residual(ref["S"][ref["probe_idx"]], ref["probe_out"], cfg.ridge_lambda, cfg.rank,
+                                 ridge_mode="relative")
+        o_ref = O.apply_residual(ref["S"], fit_ref["M"], fit_ref["beta"], ref["probe_idx"], ref["probe_out"])
+        assert rel(o[0, h].double().cpu().numpy(), o_ref) <= TOL_BF16
+
+
 def test_fit_degenerate_residual_spectrum():
     """Residuals along 8 orthogonal directions, 8 probes each, uniform weights: the
     second moment has one 8-fold eigenvalue and a zero eigenvalue of multiplicity 120.
