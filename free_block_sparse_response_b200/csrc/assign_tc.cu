@@ -283,40 +283,65 @@ __global__ void __launch_bounds__(kAsThreads, 1)
             s_nlen = 0;
           }
           __syncthreads();
-          // A. proposals
-          for (int x = warp; x < len; x += kAsWarps) {
-            const int i = __ldcg(hl + x);
-            const size_t grow = static_cast<size_t>(h) * n + i;
-            const float* row = a.Dtail + static_cast<size_t>(__ldcg(a.tailpos + grow)) * a.ldt;
-            unsigned long long best = ~0ull;
-            int first_open = G;
-            for (int w0 = 0; w0 < words; w0 += 16) {  // 16 words of the row requested at once
-              float v[16];
+          // A. proposals, kTailItems items per warp at a time so that their row loads are in
+          // flight together; the proposal's value is the winning key's (+-0 read as +0, which
+          // the decision keys do not tell apart)
+          constexpr int kTailItems = 4;
+          for (int x0 = warp * kTailItems; x0 < len; x0 += kAsWarps * kTailItems) {
+            const int xl = x0 + lane;
+            size_t my_grow = 0;
+            long long my_row = -1;
+            if (lane < kTailItems && xl < len) {
+              my_grow = static_cast<size_t>(h) * n + __ldcg(hl + xl);
+              my_row = static_cast<long long>(__ldcg(a.tailpos + my_grow)) * a.ldt;
+            }
+            const float* rows[kTailItems];
+            unsigned long long best[kTailItems];
 #pragma unroll
-              for (int u = 0; u < 16; ++u) {
-                const int g = (w0 + u) * 32 + lane;
-                v[u] = g < G ? __ldcg(row + g) : kAsInf;
+            for (int k = 0; k < kTailItems; ++k) {
+              const long long ro = __shfl_sync(0xffffffffu, my_row, k);
+              rows[k] = ro >= 0 ? a.Dtail + ro : nullptr;
+              best[k] = ~0ull;
+            }
+            int first_open = G;
+            for (int w0 = 0; w0 < words; w0 += 16) {  // 16 words of every row requested at once
+              float v[kTailItems][16];
+#pragma unroll
+              for (int k = 0; k < kTailItems; ++k) {
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                  const int g = (w0 + u) * 32 + lane;
+                  v[k][u] = (rows[k] != nullptr && g < G) ? __ldcg(rows[k] + g) : kAsInf;
+                }
               }
 #pragma unroll
               for (int u = 0; u < 16; ++u) {
                 const int wd = w0 + u;
                 const int g = wd * 32 + lane;
                 const bool open = g < G && !((s_cl[wd < words ? wd : 0] >> lane) & 1u);
-                if (open && v[u] < kAsInf) {
-                  const unsigned long long key = decision_key(v[u], g);
-                  best = key < best ? key : best;
+#pragma unroll
+                for (int k = 0; k < kTailItems; ++k) {
+                  if (open && v[k][u] < kAsInf) {
+                    const unsigned long long key = decision_key(v[k][u], g);
+                    best[k] = key < best[k] ? key : best[k];
+                  }
                 }
                 const unsigned int om = __ballot_sync(0xffffffffu, open);
                 if (first_open == G && om != 0u) first_open = wd * 32 + __ffs(om) - 1;
               }
             }
-            best = warp_min_u64(best);
-            if (lane == 0) {
+            unsigned long long mine = ~0ull;
+#pragma unroll
+            for (int k = 0; k < kTailItems; ++k) {
+              best[k] = warp_min_u64(best[k]);
+              if (lane == k) mine = best[k];
+            }
+            if (lane < kTailItems && xl < len) {
               int g;
               float pv;
-              if (best != ~0ull) {
-                g = static_cast<int>(best & 0xffffffffu);
-                pv = __ldcg(row + g);
+              if (mine != ~0ull) {
+                g = static_cast<int>(mine & 0xffffffffu);
+                pv = float_from_order_key(static_cast<uint32_t>(mine >> 32));
               } else if (first_open < G) {
                 g = first_open;
                 pv = kAsInf;
@@ -325,8 +350,8 @@ __global__ void __launch_bounds__(kAsThreads, 1)
                 g = 0;
                 pv = kAsInf;
               }
-              a.prop_g[grow] = g;
-              a.prop_v[grow] = pv;
+              a.prop_g[my_grow] = g;
+              a.prop_v[my_grow] = pv;
               atomicAdd(cnt + g, 1);
             }
           }
@@ -568,6 +593,38 @@ __global__ void __launch_bounds__(kAsThreads, 1)
       int loaded_head = -1;
       bool aborted = *abort_v != 0;
       HeadWalk hw;
+      // The rows of the next work items are read ahead, so that no load waits at an item's
+      // start: the list entries two items ahead, the norms tau^2 n_i one item ahead (their
+      // list entries arrived during the previous item).
+      HeadWalk hwa;
+      int ah1 = 0, ah2 = 0;
+      int aidx1[2] = {0, 0}, aidx2[2] = {0, 0};
+      bool aok1[2] = {false, false}, aok2[2] = {false, false};
+      float atn1[2] = {0.f, 0.f};
+      auto fetch_idx = [&](int w, int& hh, int (&idx)[2], bool (&ok)[2]) {
+        if (w >= total) {
+          ok[0] = ok[1] = false;
+          return;
+        }
+        int tt;
+        hwa.seek(s_tiles, w, hh, tt);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int e = tt * kAsRows + 128 * j + r;
+          ok[j] = e < s_len[hh];
+          idx[j] = ok[j] ? (first ? e : __ldcg(list + static_cast<size_t>(hh) * n + e)) : 0;
+        }
+      };
+      auto fetch_nrm = [&]() {
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          atn1[j] = aok1[j] ? tau2 * __ldcg(a.nrm + static_cast<size_t>(ah1) * n + aidx1[j]) : 0.f;
+      };
+      if (!norm_mode) {
+        fetch_idx(blockIdx.x, ah1, aidx1, aok1);
+        fetch_nrm();
+        fetch_idx(blockIdx.x + nblocks, ah2, aidx2, aok2);
+      }
       for (int w = blockIdx.x; w < total; w += nblocks, ++it_epi) {
         int h, t;
         hw.seek(s_tiles, w, h, t, s_len);
@@ -639,21 +696,27 @@ __global__ void __launch_bounds__(kAsThreads, 1)
           asm volatile("bar.sync 1, 256;" ::: "memory");
           loaded_head = h;
         }
-        const int len = s_len[h];
         bool row_ok[2];
         size_t grow[2];
         float tnr[2], best_v[2] = {kAsInf, kAsInf};
         int best_c[2] = {-1, -1};
         bool nonfinite = false;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int e = off + 128 * j + r;
-          row_ok[j] = e < len;
-          const int item = row_ok[j] ? (first ? e : __ldcg(list + static_cast<size_t>(h) * n + e)) : 0;
-          grow[j] = static_cast<size_t>(h) * n + item;
-          tnr[j] = row_ok[j] ? tau2 * __ldcg(a.nrm + grow[j]) : 0.f;
+        for (int j = 0; j < 2; ++j) {  // this item's rows, read ahead (ah1 == h)
+          row_ok[j] = aok1[j];
+          grow[j] = static_cast<size_t>(h) * n + aidx1[j];
+          tnr[j] = atn1[j];
           nonfinite |= row_ok[j] && (!isfinite(tnr[j]) || s_enf != 0);
         }
+        // read ahead: the next item's norms, the list entries of the one after it
+        ah1 = ah2;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          aidx1[j] = aidx2[j];
+          aok1[j] = aok2[j];
+        }
+        fetch_nrm();
+        fetch_idx(w + 2 * static_cast<int>(nblocks), ah2, aidx2, aok2);
         for (int c = 0; c < n_chunks && !aborted; ++c) {
           const int q = it_epi * n_chunks + c, s = q & 1;
           const bool got = tc::mbar_wait(bar(kAccFull0 + s), (q >> 1) & 1, abort_v, status);
