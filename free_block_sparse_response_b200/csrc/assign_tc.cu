@@ -138,6 +138,47 @@ __device__ __forceinline__ void scan_half_chunk(uint32_t (&u)[64], const float* 
   }
 }
 
+// Of a warp's chunk of an overflowing group's bucket (key u * 32 + lane in kb[u], the
+// first valid_n valid), the keys <= thr join the group's member list and the others the
+// head's next list.  One atomic per list reserves the chunk's slots; positions follow the
+// warp's ballots.  Neither order affects a decision: the group update sorts the members,
+// and an item's next proposal is its own whatever its place in the list.
+__device__ __forceinline__ void accept_reject(const unsigned long long (&kb)[8], int valid_n, unsigned long long thr,
+                                              int g, int* lab, int* members_g, int* msize_g, int* nlist, int* nlen) {
+  const int lane = threadIdx.x & 31;
+  unsigned int tk[8], rj[8];
+  int ntk = 0, nrj = 0;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const bool valid = u * 32 + lane < valid_n;
+    const bool take = valid && kb[u] <= thr;
+    tk[u] = __ballot_sync(0xffffffffu, take);
+    rj[u] = __ballot_sync(0xffffffffu, valid && !take);
+    ntk += __popc(tk[u]);
+    nrj += __popc(rj[u]);
+  }
+  int bt = 0, br = 0;
+  if (lane == 0) {
+    if (ntk > 0) bt = atomicAdd(msize_g, ntk);
+    if (nrj > 0) br = atomicAdd(nlen, nrj);
+  }
+  bt = __shfl_sync(0xffffffffu, bt, 0);
+  br = __shfl_sync(0xffffffffu, br, 0);
+  const unsigned int lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int i = static_cast<int>(kb[u] & 0xffffffffu);
+    if ((tk[u] >> lane) & 1u) {
+      lab[i] = g;
+      members_g[bt + __popc(tk[u] & lt)] = i;
+    } else if ((rj[u] >> lane) & 1u) {
+      nlist[br + __popc(rj[u] & lt)] = i;
+    }
+    bt += __popc(tk[u]);
+    br += __popc(rj[u]);
+  }
+}
+
 __global__ void __launch_bounds__(kAsThreads, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmXg,
                      const __grid_constant__ CUtensorMap tmWhi, const __grid_constant__ CUtensorMap tmWlo,
@@ -413,39 +454,22 @@ __global__ void __launch_bounds__(kAsThreads, 1)
             const size_t x = static_cast<size_t>(h) * G + g;
             const int c = __ldcg(cnt + g), rm = __ldcg(room + g);
             const unsigned long long* bk = a.bucket + static_cast<size_t>(h) * n + __ldcg(offs + g);
-            const unsigned long long thr = rm == 0 ? 0ull : warp_select_kth(bk, c, rm, hist[warp]);
+            unsigned long long kr[8];
+            if (c <= 256) {
+#pragma unroll
+              for (int u = 0; u < 8; ++u) kr[u] = u * 32 + lane < c ? __ldcg(bk + u * 32 + lane) : ~0ull;
+            }
+            const unsigned long long thr = rm == 0 ? 0ull
+                                           : c <= 256 ? warp_select_kth_by(KeysInRegisters{kr}, c, rm, hist[warp])
+                                                      : warp_select_kth(bk, c, rm, hist[warp]);
             for (int e0 = 0; e0 < c; e0 += 256) {
               unsigned long long kb[8];
 #pragma unroll
               for (int u = 0; u < 8; ++u) {
                 const int e = e0 + u * 32 + lane;
-                kb[u] = e < c ? __ldcg(bk + e) : ~0ull;
+                kb[u] = c <= 256 ? kr[u] : (e < c ? __ldcg(bk + e) : ~0ull);
               }
-#pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                const bool valid = e0 + u * 32 + lane < c;
-                const int i = static_cast<int>(kb[u] & 0xffffffffu);
-                const bool take = valid && kb[u] <= thr;
-                const unsigned int tk = __ballot_sync(0xffffffffu, take);
-                if (tk != 0u) {
-                  const int leader = __ffs(tk) - 1;
-                  int base = 0;
-                  if (lane == leader) base = atomicAdd(a.msize + x, __popc(tk));
-                  base = __shfl_sync(0xffffffffu, base, leader);
-                  if (take) {
-                    lab[i] = g;
-                    a.members[x * a.cap + base + __popc(tk & ((1u << lane) - 1u))] = i;
-                  }
-                }
-                const unsigned int rej = __ballot_sync(0xffffffffu, valid && !take);
-                if (rej != 0u) {
-                  const int leader = __ffs(rej) - 1;
-                  int base = 0;
-                  if (lane == leader) base = atomicAdd(&s_nlen, __popc(rej));
-                  base = __shfl_sync(0xffffffffu, base, leader);
-                  if (valid && !take) nl[base + __popc(rej & ((1u << lane) - 1u))] = i;
-                }
-              }
+              accept_reject(kb, c - e0, thr, g, lab, a.members + x * a.cap, a.msize + x, nl, &s_nlen);
             }
             __syncwarp();
             if (lane == 0) {
@@ -856,23 +880,50 @@ __global__ void __launch_bounds__(kAsThreads, 1)
 
     // ---------------------------------------------------------------- C. place / scatter
     {
+      // three items per thread at a time, so that their dependent loads and atomics overlap
+      constexpr int kCI = 3;
       int items = 0;
       for (int h = 0; h < heads; ++h) items += s_len[h];
       HeadWalk hw;
-      for (int x = gthread; x < items; x += nthreads) {
-        int h, e;
-        hw.seek(s_len, x, h, e);
-        const int i = first ? e : __ldcg(list + static_cast<size_t>(h) * n + e);
-        const size_t item = static_cast<size_t>(h) * n + i;
-        const int g = __ldcg(a.prop_g + item);
-        const size_t gi = static_cast<size_t>(h) * G + g;
-        const int o = __ldcg(a.offs + gi);
-        if (o < 0) {
-          a.labels[item] = g;
-          a.members[gi * a.cap + atomicAdd(a.msize + gi, 1)] = i;
-        } else {
-          const int slot = atomicAdd(a.cursor + gi, 1);
-          a.bucket[static_cast<size_t>(h) * n + o + slot] = decision_key(__ldcg(a.prop_v + item), i);
+      for (int x0 = gthread; x0 < items; x0 += nthreads * kCI) {
+        int hh[kCI], ii[kCI], gg[kCI], oo[kCI];
+        float vv[kCI];
+#pragma unroll
+        for (int u = 0; u < kCI; ++u) {
+          const int x = x0 + u * nthreads;
+          hh[u] = -1;
+          ii[u] = 0;
+          if (x < items) {
+            int e;
+            hw.seek(s_len, x, hh[u], e);
+            ii[u] = first ? e : __ldcg(list + static_cast<size_t>(hh[u]) * n + e);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kCI; ++u) {
+          gg[u] = 0;
+          vv[u] = 0.f;
+          if (hh[u] >= 0) {
+            const size_t item = static_cast<size_t>(hh[u]) * n + ii[u];
+            gg[u] = __ldcg(a.prop_g + item);
+            vv[u] = __ldcg(a.prop_v + item);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kCI; ++u)
+          oo[u] = hh[u] >= 0 ? __ldcg(a.offs + static_cast<size_t>(hh[u]) * G + gg[u]) : 0;
+#pragma unroll
+        for (int u = 0; u < kCI; ++u) {
+          if (hh[u] < 0) continue;
+          const size_t item = static_cast<size_t>(hh[u]) * n + ii[u];
+          const size_t gi = static_cast<size_t>(hh[u]) * G + gg[u];
+          if (oo[u] < 0) {
+            a.labels[item] = gg[u];
+            a.members[gi * a.cap + atomicAdd(a.msize + gi, 1)] = ii[u];
+          } else {
+            const int slot = atomicAdd(a.cursor + gi, 1);
+            a.bucket[static_cast<size_t>(hh[u]) * n + oo[u] + slot] = decision_key(vv[u], ii[u]);
+          }
         }
       }
     }
@@ -891,42 +942,24 @@ __global__ void __launch_bounds__(kAsThreads, 1)
         int* lab = a.labels + static_cast<size_t>(h) * n;
         int* nlist = a.list[next] + static_cast<size_t>(h) * n;
         int* nlen = a.list_len + next * heads + h;
-        // (rm = 0 only after a recorded error: nothing is taken then)
-        const unsigned long long thr = rm == 0 ? 0ull : warp_select_kth(bk, c, rm, hist[warp]);
+        // (rm = 0 only after a recorded error: nothing is taken then).  A bucket of at most
+        // 256 keys is read once and selected in registers.
+        unsigned long long kr[8];
+        if (c <= 256) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) kr[u] = u * 32 + lane < c ? __ldcg(bk + u * 32 + lane) : ~0ull;
+        }
+        const unsigned long long thr = rm == 0 ? 0ull
+                                       : c <= 256 ? warp_select_kth_by(KeysInRegisters{kr}, c, rm, hist[warp])
+                                                  : warp_select_kth(bk, c, rm, hist[warp]);
         for (int e0 = 0; e0 < c; e0 += 256) {
           unsigned long long kb[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             const int e = e0 + u * 32 + lane;
-            kb[u] = e < c ? __ldcg(bk + e) : ~0ull;
+            kb[u] = c <= 256 ? kr[u] : (e < c ? __ldcg(bk + e) : ~0ull);
           }
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const bool valid = e0 + u * 32 + lane < c;
-            const int i = static_cast<int>(kb[u] & 0xffffffffu);
-            const bool take = valid && kb[u] <= thr;
-            // taken proposers join the group's member list, one atomic per warp
-            const unsigned int tk = __ballot_sync(0xffffffffu, take);
-            if (tk != 0u) {
-              const int leader = __ffs(tk) - 1;
-              int base = 0;
-              if (lane == leader) base = atomicAdd(a.msize + x, __popc(tk));
-              base = __shfl_sync(0xffffffffu, base, leader);
-              if (take) {
-                lab[i] = g;
-                a.members[static_cast<size_t>(x) * a.cap + base + __popc(tk & ((1u << lane) - 1u))] = i;
-              }
-            }
-            // rejected proposers join the head's next list, one atomic per warp
-            const unsigned int rej = __ballot_sync(0xffffffffu, valid && !take);
-            if (rej != 0u) {
-              const int leader = __ffs(rej) - 1;
-              int base = 0;
-              if (lane == leader) base = atomicAdd(nlen, __popc(rej));
-              base = __shfl_sync(0xffffffffu, base, leader);
-              if (valid && !take) nlist[base + __popc(rej & ((1u << lane) - 1u))] = i;
-            }
-          }
+          accept_reject(kb, c - e0, thr, g, lab, a.members + static_cast<size_t>(x) * a.cap, a.msize + x, nlist, nlen);
         }
         __syncwarp();
         if (lane == 0) {
