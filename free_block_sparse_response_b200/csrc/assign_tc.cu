@@ -180,7 +180,7 @@ __device__ __forceinline__ void accept_reject(const unsigned long long (&kb)[8],
 }
 
 __global__ void __launch_bounds__(kAsThreads, 1)
-    assign_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmXg,
+    assign_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                      const __grid_constant__ CUtensorMap tmWhi, const __grid_constant__ CUtensorMap tmWlo,
                      AssignArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -189,6 +189,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
   __shared__ int abort_flag, s_enf, s_remaining, s_total;
   __shared__ float s_best_v[kAsRows];  // the upper column halves' partial results
   __shared__ int s_best_c[kAsRows];
+  __shared__ int s_xidx[2][128];       // the loader warps' row items
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = (tc::saddr(smem_raw) + 1023u) & ~1023u;
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
 
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(bar(kXFull0 + s), 1);
+      tc::mbar_init(bar(kXFull0 + s), 2);  // TMA rounds: the producer twice; gathered: each loader warp
       tc::mbar_init(bar(kXEmpty0 + s), 1);
       tc::mbar_init(bar(kWFull0 + s), 1);
       tc::mbar_init(bar(kWEmpty0 + s), 1);
@@ -262,7 +263,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
   bool alive = norm_mode ? true : sync_grid();
 
   // pipeline counters, continued across rounds: work items and W chunks seen by this CTA
-  int it_prod = 0, it_mma = 0, it_epi = 0;
+  int it_prod = 0, it_mma = 0, it_epi = 0, it_x = 0;
   int last_q = -1, last_it = -1;  // producer: last W chunk and X tile issued
   const int max_rounds = n + 2;
   int cur = 0;
@@ -494,41 +495,27 @@ __global__ void __launch_bounds__(kAsThreads, 1)
       // item's last MMAs, so the X buffer the next item reuses is free, and its load
       // overlaps all of this item's MMAs.
       auto issue_x = [&](int it, int h, int t) -> bool {
+        if (!first) return true;  // the gathered rounds' X comes from the loader warps
         const int b = it & 1, off = t * kAsRows;
         int ok = 1;
         if (lane == 0 && it >= 2 && !tc::mbar_wait(bar(kXEmpty0 + b), ((it >> 1) - 1) & 1, abort_v, status)) ok = 0;
         if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
-        if (lane == 0) tc::mbar_arrive_expect_tx(bar(kXFull0 + b), kAsXStage);
-        __syncwarp();
-        if (first) {
-          if (lane == 0) {
+        if (lane == 0) {
+          tc::mbar_arrive_expect_tx(bar(kXFull0 + b), kAsXStage);
+          tc::mbar_arrive(bar(kXFull0 + b));  // the phase's second arrival (the loader warps' two otherwise)
 #pragma unroll
-            for (int j2 = 0; j2 < 2; ++j2) {
-              tc::tma_load_2d(sX[b] + j2 * kAsTile, &tmX, 0, h * n + off + 128 * j2, bar(kXFull0 + b));
-              tc::tma_load_2d(sX[b] + j2 * kAsTile + 128 * 128, &tmX, 64, h * n + off + 128 * j2, bar(kXFull0 + b));
-            }
-          }
-        } else {
-          const int len = s_len[h];
-          const int* hl = list + static_cast<size_t>(h) * n;
-#pragma unroll
-          for (int g4 = 0; g4 < 2; ++g4) {
-            const int row = 8 * lane + 4 * g4;  // 0..255: rows row .. row + 3
-            int r4[4];
-#pragma unroll
-            for (int j2 = 0; j2 < 4; ++j2) {
-              const int e = off + row + j2;
-              // rows past the list repeat the item's first entry (loaded, never used)
-              r4[j2] = h * n + __ldcg(hl + (e < len ? e : off));
-            }
-            const uint32_t dst = sX[b] + (row >> 7) * kAsTile + (row & 127) * 128;
-            tc::tma_gather4(dst, &tmXg, 0, r4[0], r4[1], r4[2], r4[3], bar(kXFull0 + b));
-            tc::tma_gather4(dst + 128 * 128, &tmXg, 64, r4[0], r4[1], r4[2], r4[3], bar(kXFull0 + b));
+          for (int j2 = 0; j2 < 2; ++j2) {
+            tc::tma_load_2d(sX[b] + j2 * kAsTile, &tmX, 0, h * n + off + 128 * j2, bar(kXFull0 + b));
+            tc::tma_load_2d(sX[b] + j2 * kAsTile + 128 * 128, &tmX, 64, h * n + off + 128 * j2, bar(kXFull0 + b));
           }
         }
+        __syncwarp();
         last_it = it;
         return true;
       };
+      // every X box of the first round has landed by now (the MMAs waited for each), and
+      // the later rounds' X is not TMA's: nothing of it is left for the final drain
+      if (!first) last_it = -1;
       HeadWalk hw;
       int h = 0, t = 0;
       bool ok = true;
@@ -562,6 +549,53 @@ __global__ void __launch_bounds__(kAsThreads, 1)
         }
         h = hn;
         t = tn;
+      }
+    } else if (warp == 1 || warp == 3) {
+      // X of the gathered rounds: the rows of the head's unplaced list, read with coalesced
+      // 16-byte loads (two rows per warp instruction, 16 instructions in flight per lane)
+      // and stored in the swizzled tile layout, warp 1 the item's rows 0-127 and warp 3
+      // rows 128-255; rows past the list are zero (never used).  The TMA engine then
+      // serves only W (the first round's contiguous rows come by TMA boxes instead).
+      const int hx = warp >> 1;
+      const int sub = lane >> 4, ch = lane & 15;  // row of the pair, 16-byte chunk of the row
+      HeadWalk hw;
+      for (int w = blockIdx.x; w < total; w += nblocks, ++it_x) {
+        if (first) continue;  // (the items are still counted: every role numbers them alike)
+        int h, t;
+        hw.seek(s_tiles, w, h, t);
+        const int b = it_x & 1, off = t * kAsRows + 128 * hx, len = s_len[h];
+        int ok = 1;
+        if (lane == 0 && it_x >= 2 && !tc::mbar_wait(bar(kXEmpty0 + b), ((it_x >> 1) - 1) & 1, abort_v, status))
+          ok = 0;
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+        int* xidx = s_xidx[hx];  // the items of this half's 128 rows
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int e = off + 32 * k + lane;
+          xidx[32 * k + lane] = e < len ? __ldcg(list + static_cast<size_t>(h) * n + e) : -1;
+        }
+        __syncwarp();
+        uint8_t* dst = smem_raw + (sX[b] - tc::saddr(smem_raw)) + hx * kAsTile + (ch >> 3) * (128 * 128);
+        const __nv_bfloat16* xh = a.x + static_cast<size_t>(h) * n * 128;
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {  // 32 rows per batch
+          uint4 v[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const int ix = xidx[32 * q + 2 * k + sub];
+            v[k] = ix >= 0 ? __ldcg(reinterpret_cast<const uint4*>(xh + static_cast<size_t>(ix) * 128) + ch)
+                           : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const int row = 32 * q + 2 * k + sub;
+            *reinterpret_cast<uint4*>(dst + row * 128 + (((ch & 7) ^ (row & 7)) << 4)) = v[k];
+          }
+        }
+        __syncwarp();  // every lane done with xidx before the next item overwrites it
+        tc::fence_proxy_async();  // the stores, before the tensor core reads the tile
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(bar(kXFull0 + b));
       }
     } else if (warp == 2) {
       // MMA issuer: per chunk, all hi products (8 k-steps of 16, both 128-row halves),
@@ -1055,6 +1089,7 @@ cudaError_t launch_assign_tc(const __nv_bfloat16* X, const __nv_bfloat16* Whi, c
     auto sl = [](auto* p, size_t k) { return p != nullptr ? p + k : p; };
     AssignArgs s = a;
     s.heads = hc;
+    s.x = X + ni * 128;
     s.nrm = sl(a.nrm, ni);
     s.ecol = sl(a.ecol, gi);
     s.labels = sl(a.labels, ni);
@@ -1077,14 +1112,14 @@ cudaError_t launch_assign_tc(const __nv_bfloat16* X, const __nv_bfloat16* Whi, c
     s.Dout = sl(a.Dout, ni * a.ldd);
     const long long xrows = static_cast<long long>(hc) * a.n, wrows = static_cast<long long>(hc) * a.G;
     if (xrows > 0x7fffffffLL || wrows > 0x7fffffffLL) return cudaErrorInvalidValue;  // TMA coordinates are int32
-    CUtensorMap tx, txg, twh, twl;
+    CUtensorMap tx, twh, twl;
     const __nv_bfloat16* Xs = X + ni * 128;
-    if (!bf16_map(&tx, Xs, xrows, 128) || !bf16_map(&txg, Xs, xrows, 1) ||
+    if (!bf16_map(&tx, Xs, xrows, 128) ||
         !bf16_map(&twh, Whi + gi * 128, wrows, 128) || !bf16_map(&twl, Wlo + gi * 128, wrows, 128))
       return cudaErrorInvalidValue;
     e = cudaMemsetAsync(&a.hdr->barrier_count, 0, 2 * sizeof(unsigned int), st);
     if (e != cudaSuccess) return e;
-    void* params[] = {&tx, &txg, &twh, &twl, &s};
+    void* params[] = {&tx, &twh, &twl, &s};
     e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(assign_tc_kernel), dim3(sms), dim3(kAsThreads), params,
                                     smem, st);
     if ((e = counted(e, 1)) != cudaSuccess) return e;

@@ -55,6 +55,7 @@ struct FillArgs {
 struct AssignArgs {
   int heads, n, G, cap;
   float tau2;
+  const __nv_bfloat16* x;       // [heads, n, 128]  the items (set by the launcher)
   const float* nrm;             // [heads, n]  x_i^T Gamma x_i
   const float* ecol;            // [heads, G]  c_g^T Gamma c_g
   int* labels;                  // [heads, n]  out: the group of every item
