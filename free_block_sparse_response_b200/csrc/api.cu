@@ -76,7 +76,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct Layout {
   size_t header = 0, sample_idx, gamma, gamma_hi, gamma_lo, nrm, cent_k, cent_q, wf, whi, wlo, eg, dmat,
          prop_g0, prop_v0, labels, room, cnt, offs, cursor, closed, bucket, list0, list1, list_len, prop_g, prop_v,
-         perm_tmp, perm_cursor, qblk, partial, fit, kv_grouped, mhilo, ovf, dtail, tailpos, total;
+         perm_tmp, perm_cursor, qblk, partial, fit, kv_grouped, mhilo, ovf, dtail, tailpos, wcomp, openg, total;
 };
 
 Layout make_layout(int heads, int N, int d, int block, int S, int P) {
@@ -127,6 +127,8 @@ Layout make_layout(int heads, int N, int d, int block, int S, int P) {
   L.ovf = take(sizeof(int) * (H * G + 2));
   L.dtail = take(sizeof(float) * tail_cap(heads, N) * tail_ld(static_cast<int>(G)));
   L.tailpos = take(sizeof(int) * H * n);
+  L.wcomp = take(2 * 2 * H * G * D);          // the open groups' W, bf16 hi and lo
+  L.openg = take(sizeof(int) * (H * G + H));  // packed column -> group, and counts
   L.total = off;
   return L;
 }
@@ -371,6 +373,10 @@ static int partition_impl(const void* Q, const void* K, int dtype, int32_t Bt, i
         aa.ldt = tail_ld(G);
         aa.tail_cap = tail_cap(heads, N);
         aa.tailpos = at<int>(ws, L.tailpos);
+        aa.wc_hi = at<__nv_bfloat16>(ws, L.wcomp);
+        aa.wc_lo = aa.wc_hi + static_cast<size_t>(heads) * G * d;
+        aa.open_g = at<int>(ws, L.openg);
+        aa.n_open = aa.open_g + static_cast<size_t>(heads) * G;
         aa.ldd = static_cast<int>(fa.ldd);
         aa.hdr = hdr;
         SPR_CUDA(spr::launch_assign_tc(static_cast<const __nv_bfloat16*>(X), whi, wlo, aa, st), "assignment");

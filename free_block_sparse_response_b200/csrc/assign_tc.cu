@@ -182,6 +182,7 @@ __device__ __forceinline__ void accept_reject(const unsigned long long (&kb)[8],
 __global__ void __launch_bounds__(kAsThreads, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                      const __grid_constant__ CUtensorMap tmWhi, const __grid_constant__ CUtensorMap tmWlo,
+                     const __grid_constant__ CUtensorMap tmWcHi, const __grid_constant__ CUtensorMap tmWcLo,
                      AssignArgs a) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars[kBars];
@@ -190,6 +191,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
   __shared__ float s_best_v[kAsRows];  // the upper column halves' partial results
   __shared__ int s_best_c[kAsRows];
   __shared__ int s_xidx[2][128];       // the loader warps' row items
+  __shared__ int s_inch[4];            // W chunks of the producer's latest work items
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t sbase = (tc::saddr(smem_raw) + 1023u) & ~1023u;
@@ -203,6 +205,8 @@ __global__ void __launch_bounds__(kAsThreads, 1)
   unsigned int (*hist)[256] = reinterpret_cast<unsigned int (*)[256]>(smem_raw + (sW[0] - tc::saddr(smem_raw)));
   int* s_len = reinterpret_cast<int*>(sgen + 4 * kAsMaxCols);     // [kAsMaxHeads] list lengths
   int* s_tiles = s_len + kAsMaxHeads;                             // [kAsMaxHeads] work items per head
+  int* s_nch = s_tiles + kAsMaxHeads;                             // [kAsMaxHeads] W chunks per head
+  int* s_g = s_nch + kAsMaxHeads;                                 // [kAsMaxCols] packed column -> group
   auto bar = [&](int i) { return tc::saddr(&bars[i]); };
 
   const int n = a.n, G = a.G, heads = a.heads;
@@ -264,6 +268,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
 
   // pipeline counters, continued across rounds: work items and W chunks seen by this CTA
   int it_prod = 0, it_mma = 0, it_epi = 0, it_x = 0;
+  int qc_prod = 0, qc_mma = 0, qc_epi = 0;  // W chunks so far (each two ring stages, one accumulator stage)
   int last_q = -1, last_it = -1;  // producer: last W chunk and X tile issued
   const int max_rounds = n + 2;
   int cur = 0;
@@ -289,6 +294,58 @@ __global__ void __launch_bounds__(kAsThreads, 1)
     }
     __syncthreads();
     const int total = s_total;
+
+    // ---- the rounds after the first multiply with the open groups' W only.  Each head's
+    // open groups (ascending) are packed into wc_hi / wc_lo at the head's offset; the
+    // round that stores the tail rows, and the tail, keep the full W.
+    const bool packed = !first && !norm_mode && !tail && !store_rows;
+    if (packed) {
+      __shared__ int s_wpre[32];
+      __shared__ int s_nopen;
+      for (int h = blockIdx.x; h < heads; h += nblocks) {
+        const unsigned int* cl = a.closed + static_cast<size_t>(h) * words;
+        if (warp == 0) {
+          unsigned int open = 0u;
+          if (lane < words) {
+            open = ~__ldcg(cl + lane);
+            if (lane == words - 1 && (G & 31) != 0) open &= (1u << (G & 31)) - 1u;
+          }
+          const int cnt = __popc(open);
+          int incl = cnt;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          s_wpre[lane] = incl - cnt;
+          if (lane == 31) s_nopen = incl;
+        }
+        __syncthreads();
+        for (int g = tid; g < G; g += kAsThreads) {
+          const unsigned int open = ~__ldcg(cl + (g >> 5));
+          if ((open >> (g & 31)) & 1u) s_g[s_wpre[g >> 5] + __popc(open & ((1u << (g & 31)) - 1u))] = g;
+        }
+        __syncthreads();
+        const int nop = s_nopen;
+        // a warp per open group: lanes 0-15 copy its hi row, lanes 16-31 its lo row
+        for (int c = warp; c < nop; c += kAsWarps) {
+          const int g = s_g[c];
+          const __nv_bfloat16* src = (lane < 16 ? a.whi : a.wlo) + (static_cast<size_t>(h) * G + g) * 128;
+          __nv_bfloat16* dst = (lane < 16 ? a.wc_hi : a.wc_lo) + (static_cast<size_t>(h) * G + c) * 128;
+          reinterpret_cast<uint4*>(dst)[lane & 15] = __ldcg(reinterpret_cast<const uint4*>(src) + (lane & 15));
+          if (lane == 0) a.open_g[static_cast<size_t>(h) * G + c] = g;
+        }
+        if (tid == 0) a.n_open[h] = nop;
+        __syncthreads();
+      }
+      // the packed rows are read by other CTAs' TMA (the async proxy) after the barrier
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      alive = sync_grid();
+      if (!alive) break;
+    }
+    for (int h = tid; h < heads; h += kAsThreads)
+      s_nch[h] = packed ? ceil_div(__ldcg(a.n_open + h), 128) : n_chunks;
+    __syncthreads();
 
     // ---------------------------------------------------------------- A. proposals
     if (tail) {
@@ -527,15 +584,17 @@ __global__ void __launch_bounds__(kAsThreads, 1)
         const int wn = w + nblocks;
         int hn = 0, tn = 0;
         if (wn < total) hw.seek(s_tiles, wn, hn, tn);
-        for (int c = 0; ok && c < n_chunks; ++c) {
+        const int nch = s_nch[h];
+        if (lane == 0) s_inch[it_prod & 3] = nch;  // for the MMA issuer (read after this item's first W stage)
+        for (int c = 0; ok && c < nch; ++c, ++qc_prod) {
           for (int part = 0; ok && part < 2; ++part) {
             int okc = 1;
             if (lane == 0) {
-              const int q = (it_prod * n_chunks + c) * 2 + part, st = q & 1;
+              const int q = qc_prod * 2 + part, st = q & 1;
               if (q >= 2 && !tc::mbar_wait(bar(kWEmpty0 + st), ((q >> 1) - 1) & 1, abort_v, status)) {
                 okc = 0;
               } else {
-                const CUtensorMap* tm = part == 0 ? &tmWhi : &tmWlo;
+                const CUtensorMap* tm = packed ? (part == 0 ? &tmWcHi : &tmWcLo) : (part == 0 ? &tmWhi : &tmWlo);
                 const int wrow = h * G + c * 128;
                 tc::mbar_arrive_expect_tx(bar(kWFull0 + st), kAsWStage);
                 tc::tma_load_2d(sW[st], tm, 0, wrow, bar(kWFull0 + st));
@@ -607,8 +666,13 @@ __global__ void __launch_bounds__(kAsThreads, 1)
           if (!tc::mbar_wait(bar(kXFull0 + b), (it_mma >> 1) & 1, abort_v, status)) break;
           tc::fence_proxy_async();
           bool ok = true;
+          // the item's chunk count, written by the producer before its first W stage (the
+          // hi part of chunk qc is ring stage 0, phase qc)
+          if (!tc::mbar_wait(bar(kWFull0), qc_mma & 1, abort_v, status)) break;
+          const int nch = s_inch[it_mma & 3];
           for (int c = 0; ok && c < n_chunks; ++c) {
-            const int qc = it_mma * n_chunks + c, s = qc & 1;
+            if (c >= nch) break;  // (a loop-invariant bound keeps the register allocation of the issue loop)
+            const int qc = qc_mma++, s = qc & 1;
             if (qc >= 2 && !tc::mbar_wait(bar(kAccEmpty0 + s), ((qc >> 1) - 1) & 1, abort_v, status)) {
               ok = false;
               break;
@@ -742,14 +806,23 @@ __global__ void __launch_bounds__(kAsThreads, 1)
           if (etid == 0) s_enf = 0;
           asm volatile("bar.sync 1, 256;" ::: "memory");
           const unsigned int* cl = a.closed + static_cast<size_t>(h) * words;
-          for (int c = etid; c < n_chunks * 128; c += kAsEpi) {
+          const int nop = packed ? __ldcg(a.n_open + h) : G;
+          for (int c = etid; c < s_nch[h] * 128; c += kAsEpi) {
             float v = kAsInf;
-            if (c < G) {
+            int g = c;
+            if (packed) {  // packed column c: the head's c-th open group
+              if (c < nop) {
+                g = __ldcg(a.open_g + static_cast<size_t>(h) * G + c);
+                v = tau2 * __ldcg(a.ecol + static_cast<size_t>(h) * G + g);
+                if (!isfinite(v)) s_enf = 1;
+              }
+            } else if (c < G) {
               const float e = tau2 * __ldcg(a.ecol + static_cast<size_t>(h) * G + c);
               if (!isfinite(e)) s_enf = 1;
               if (!((__ldcg(cl + (c >> 5)) >> (c & 31)) & 1u)) v = e;
             }
             s_e[c] = v;
+            s_g[c] = g;
           }
           asm volatile("bar.sync 1, 256;" ::: "memory");
           loaded_head = h;
@@ -775,8 +848,9 @@ __global__ void __launch_bounds__(kAsThreads, 1)
         }
         fetch_nrm();
         fetch_idx(w + 2 * static_cast<int>(nblocks), ah2, aidx2, aok2);
-        for (int c = 0; c < n_chunks && !aborted; ++c) {
-          const int q = it_epi * n_chunks + c, s = q & 1;
+        const int nch = s_nch[h];
+        for (int c = 0; c < nch && !aborted; ++c) {
+          const int q = qc_epi++, s = q & 1;
           const bool got = tc::mbar_wait(bar(kAccFull0 + s), (q >> 1) & 1, abort_v, status);
           if (!__all_sync(0xffffffffu, got)) {
             aborted = true;
@@ -837,6 +911,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
               bv = v1;
               bc = c1;
             }
+            if (bc >= 0) bc = s_g[bc];  // the column's group (packed columns ascend with it)
             if (bc < 0) {  // every open group at +inf (or NaN): the lowest open group
               const unsigned int* cl = a.closed + static_cast<size_t>(h) * words;
               for (int wd = 0; wd < words && bc < 0; ++wd) {
@@ -1062,7 +1137,8 @@ __global__ void __launch_bounds__(kAsThreads, 1)
 }  // namespace
 
 size_t assign_tc_smem_bytes() {
-  return 1024 + 2ull * kAsXStage + 2ull * kAsWStage + sizeof(float) * kAsMaxCols + 2 * sizeof(int) * kAsMaxHeads;
+  return 1024 + 2ull * kAsXStage + 2ull * kAsWStage + sizeof(float) * kAsMaxCols + 3 * sizeof(int) * kAsMaxHeads +
+         sizeof(int) * kAsMaxCols;
 }
 
 cudaError_t launch_assign_tc(const __nv_bfloat16* X, const __nv_bfloat16* Whi, const __nv_bfloat16* Wlo,
@@ -1090,6 +1166,12 @@ cudaError_t launch_assign_tc(const __nv_bfloat16* X, const __nv_bfloat16* Whi, c
     AssignArgs s = a;
     s.heads = hc;
     s.x = X + ni * 128;
+    s.whi = Whi + gi * 128;
+    s.wlo = Wlo + gi * 128;
+    s.wc_hi = sl(a.wc_hi, gi * 128);
+    s.wc_lo = sl(a.wc_lo, gi * 128);
+    s.open_g = sl(a.open_g, gi);
+    s.n_open = sl(a.n_open, static_cast<size_t>(h0));
     s.nrm = sl(a.nrm, ni);
     s.ecol = sl(a.ecol, gi);
     s.labels = sl(a.labels, ni);
@@ -1112,14 +1194,18 @@ cudaError_t launch_assign_tc(const __nv_bfloat16* X, const __nv_bfloat16* Whi, c
     s.Dout = sl(a.Dout, ni * a.ldd);
     const long long xrows = static_cast<long long>(hc) * a.n, wrows = static_cast<long long>(hc) * a.G;
     if (xrows > 0x7fffffffLL || wrows > 0x7fffffffLL) return cudaErrorInvalidValue;  // TMA coordinates are int32
-    CUtensorMap tx, twh, twl;
+    CUtensorMap tx, twh, twl, twch, twcl;
     const __nv_bfloat16* Xs = X + ni * 128;
     if (!bf16_map(&tx, Xs, xrows, 128) ||
         !bf16_map(&twh, Whi + gi * 128, wrows, 128) || !bf16_map(&twl, Wlo + gi * 128, wrows, 128))
       return cudaErrorInvalidValue;
+    // the packed open groups' W (norm mode packs nothing: the maps then name W itself)
+    if (!bf16_map(&twch, s.wc_hi != nullptr ? s.wc_hi : s.whi, wrows, 128) ||
+        !bf16_map(&twcl, s.wc_lo != nullptr ? s.wc_lo : s.wlo, wrows, 128))
+      return cudaErrorInvalidValue;
     e = cudaMemsetAsync(&a.hdr->barrier_count, 0, 2 * sizeof(unsigned int), st);
     if (e != cudaSuccess) return e;
-    void* params[] = {&tx, &twh, &twl, &s};
+    void* params[] = {&tx, &twh, &twl, &twch, &twcl, &s};
     e = cudaLaunchCooperativeKernel(reinterpret_cast<void*>(assign_tc_kernel), dim3(sms), dim3(kAsThreads), params,
                                     smem, st);
     if ((e = counted(e, 1)) != cudaSuccess) return e;

@@ -56,6 +56,8 @@ struct AssignArgs {
   int heads, n, G, cap;
   float tau2;
   const __nv_bfloat16* x;       // [heads, n, 128]  the items (set by the launcher)
+  const __nv_bfloat16* whi;     // [heads, G, 128]  W = C Gamma, bf16 hi / lo (set by the launcher)
+  const __nv_bfloat16* wlo;
   const float* nrm;             // [heads, n]  x_i^T Gamma x_i
   const float* ecol;            // [heads, G]  c_g^T Gamma c_g
   int* labels;                  // [heads, n]  out: the group of every item
@@ -83,6 +85,13 @@ struct AssignArgs {
   int ldt;
   int tail_cap;
   int* tailpos;                 // [heads, n]
+  // Rounds after the first multiply the rows with the open groups' W only: each round
+  // starts by packing every head's open groups (ascending) into wc_hi / wc_lo at the same
+  // per-head offsets, open_g mapping packed column -> group and n_open counting them.
+  __nv_bfloat16* wc_hi;         // [heads, G, 128]
+  __nv_bfloat16* wc_lo;
+  int* open_g;                  // [heads, G]
+  int* n_open;                  // [heads]
   WorkspaceHeader* hdr;
 };
 cudaError_t launch_assign_tc(const __nv_bfloat16* X, const __nv_bfloat16* Whi, const __nv_bfloat16* Wlo,
