@@ -994,7 +994,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
       int items = 0;
       for (int h = 0; h < heads; ++h) items += s_len[h];
       HeadWalk hw;
-      for (int x0 = gthread; x0 < items; x0 += nthreads * kCI) {
+      for (int x0 = gthread; x0 - lane < items; x0 += nthreads * kCI) {  // warp-uniform trip count
         int hh[kCI], ii[kCI], gg[kCI], oo[kCI];
         float vv[kCI];
 #pragma unroll
@@ -1023,14 +1023,21 @@ __global__ void __launch_bounds__(kAsThreads, 1)
           oo[u] = hh[u] >= 0 ? __ldcg(a.offs + static_cast<size_t>(hh[u]) * G + gg[u]) : 0;
 #pragma unroll
         for (int u = 0; u < kCI; ++u) {
+          // a warp's items are consecutive, often of one group: one atomic per distinct group
+          // of the warp reserves its lanes' slots (a group either places or scatters all)
+          const unsigned int act = __ballot_sync(0xffffffffu, hh[u] >= 0);
           if (hh[u] < 0) continue;
-          const size_t item = static_cast<size_t>(hh[u]) * n + ii[u];
           const size_t gi = static_cast<size_t>(hh[u]) * G + gg[u];
+          const unsigned int same = __match_any_sync(act, static_cast<unsigned long long>(gi));
+          const int leader = __ffs(same) - 1;
+          int base = 0;
+          if (lane == leader) base = atomicAdd((oo[u] < 0 ? a.msize : a.cursor) + gi, __popc(same));
+          const int slot = __shfl_sync(act, base, leader) + __popc(same & ((1u << lane) - 1u));
+          const size_t item = static_cast<size_t>(hh[u]) * n + ii[u];
           if (oo[u] < 0) {
             a.labels[item] = gg[u];
-            a.members[gi * a.cap + atomicAdd(a.msize + gi, 1)] = ii[u];
+            a.members[gi * a.cap + slot] = ii[u];
           } else {
-            const int slot = atomicAdd(a.cursor + gi, 1);
             a.bucket[static_cast<size_t>(hh[u]) * n + oo[u] + slot] = decision_key(vv[u], ii[u]);
           }
         }
