@@ -138,6 +138,33 @@ __device__ __forceinline__ void scan_half_chunk(uint32_t (&u)[64], const float* 
   }
 }
 
+// Exclusive prefix sum of one value per thread over the CTA (kAsThreads threads): warp
+// scans by shuffles, the warp totals scanned by warp 0 through `tmp` (kAsWarps ints), two
+// CTA barriers.  Every thread of the CTA calls it.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* tmp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) tmp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int t = lane < kAsWarps ? tmp[lane] : 0;
+    int ti = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, ti, o);
+      if (lane >= o) ti += y;
+    }
+    if (lane < kAsWarps) tmp[lane] = ti - t;
+  }
+  __syncthreads();
+  return tmp[warp] + incl - v;
+}
+
 // Of a warp's chunk of an overflowing group's bucket (key u * 32 + lane in kb[u], the
 // first valid_n valid), the keys <= thr join the group's member list and the others the
 // head's next list.  One atomic per list reserves the chunk's slots; positions follow the
@@ -297,7 +324,8 @@ __global__ void __launch_bounds__(kAsThreads, 1)
 
     // ---- the rounds after the first multiply with the open groups' W only.  Each head's
     // open groups (ascending) are packed into wc_hi / wc_lo at the head's offset; the
-    // round that stores the tail rows, and the tail, keep the full W.
+    // round that stores the tail rows (whose rows the tail reads by group), and the tail,
+    // keep the full W.
     const bool packed = !first && !norm_mode && !tail && !store_rows;
     if (packed) {
       __shared__ int s_wpre[32];
@@ -464,15 +492,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
               const int c = __ldcg(cnt + g);
               if (c > __ldcg(room + g)) local += c;
             }
-            scan_tmp[tid] = local;
-            __syncthreads();
-            for (int o = 1; o < kAsThreads; o <<= 1) {
-              const int y = tid >= o ? scan_tmp[tid - o] : 0;
-              __syncthreads();
-              scan_tmp[tid] += y;
-              __syncthreads();
-            }
-            int run = scan_tmp[tid] - local;
+            int run = block_exclusive_scan(local, scan_tmp);
             for (int g = g0; g < g1; ++g) {
               const int c = __ldcg(cnt + g), rm = __ldcg(room + g);
               if (c > rm) {
@@ -958,15 +978,7 @@ __global__ void __launch_bounds__(kAsThreads, 1)
         const int c = __ldcg(cnt + g);
         if (c > __ldcg(room + g)) local += c;
       }
-      scan_tmp[tid] = local;
-      __syncthreads();
-      for (int o = 1; o < kAsThreads; o <<= 1) {
-        const int y = tid >= o ? scan_tmp[tid - o] : 0;
-        __syncthreads();
-        scan_tmp[tid] += y;
-        __syncthreads();
-      }
-      int run = scan_tmp[tid] - local;
+      int run = block_exclusive_scan(local, scan_tmp);
       for (int g = g0; g < g1; ++g) {
         const int c = __ldcg(cnt + g), rm = __ldcg(room + g);
         if (c > rm) {
