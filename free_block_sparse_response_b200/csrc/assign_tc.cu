@@ -206,6 +206,85 @@ __device__ __forceinline__ void accept_reject(const unsigned long long (&kb)[8],
   }
 }
 
+// Tail proposals of the kTailItems items x0.. of head h's list hl (len items) from their
+// stored D rows, by one warp, their row loads in flight together; clw: the head's
+// full-group bitmap.  The rule is the epilogue's: the first minimum over the open groups
+// (strict '<' in ascending column order, so +inf and NaN never win; none finite: the
+// lowest open group at +inf).  The proposal's value is the winning key's (+-0 read as +0,
+// which the decision keys do not tell apart).
+constexpr int kTailItems = 4;
+__device__ __forceinline__ void tail_propose(const AssignArgs& a, int h, const int* hl, int len, int x0,
+                                             const unsigned int* clw) {
+  const int lane = threadIdx.x & 31;
+  const int n = a.n, G = a.G, words = ceil_div(G, 32);
+  const int xl = x0 + lane;
+  size_t my_grow = 0;
+  long long my_row = -1;
+  if (lane < kTailItems && xl < len) {
+    my_grow = static_cast<size_t>(h) * n + __ldcg(hl + xl);
+    my_row = static_cast<long long>(__ldcg(a.tailpos + my_grow)) * a.ldt;
+  }
+  const float* rows[kTailItems];
+  unsigned long long best[kTailItems];
+#pragma unroll
+  for (int k = 0; k < kTailItems; ++k) {
+    const long long ro = __shfl_sync(0xffffffffu, my_row, k);
+    rows[k] = ro >= 0 ? a.Dtail + ro : nullptr;
+    best[k] = ~0ull;
+  }
+  int first_open = G;
+  for (int w0 = 0; w0 < words; w0 += 16) {  // 16 words of every row requested at once
+    float v[kTailItems][16];
+#pragma unroll
+    for (int k = 0; k < kTailItems; ++k) {
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int g = (w0 + u) * 32 + lane;
+        v[k][u] = (rows[k] != nullptr && g < G) ? __ldcg(rows[k] + g) : kAsInf;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int wd = w0 + u;
+      const int g = wd * 32 + lane;
+      const bool open = g < G && !((clw[wd < words ? wd : 0] >> lane) & 1u);
+#pragma unroll
+      for (int k = 0; k < kTailItems; ++k) {
+        if (open && v[k][u] < kAsInf) {
+          const unsigned long long key = decision_key(v[k][u], g);
+          best[k] = key < best[k] ? key : best[k];
+        }
+      }
+      const unsigned int om = __ballot_sync(0xffffffffu, open);
+      if (first_open == G && om != 0u) first_open = wd * 32 + __ffs(om) - 1;
+    }
+  }
+  unsigned long long mine = ~0ull;
+#pragma unroll
+  for (int k = 0; k < kTailItems; ++k) {
+    best[k] = warp_min_u64(best[k]);
+    if (lane == k) mine = best[k];
+  }
+  if (lane < kTailItems && xl < len) {
+    int g;
+    float pv;
+    if (mine != ~0ull) {
+      g = static_cast<int>(mine & 0xffffffffu);
+      pv = float_from_order_key(static_cast<uint32_t>(mine >> 32));
+    } else if (first_open < G) {
+      g = first_open;
+      pv = kAsInf;
+    } else {  // no open group: more items than room (cannot happen)
+      record_error(&a.hdr->status, kErrInvalidArg);
+      g = 0;
+      pv = kAsInf;
+    }
+    a.prop_g[my_grow] = g;
+    a.prop_v[my_grow] = pv;
+    atomicAdd(a.cnt + static_cast<size_t>(h) * G + g, 1);
+  }
+}
+
 __global__ void __launch_bounds__(kAsThreads, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                      const __grid_constant__ CUtensorMap tmWhi, const __grid_constant__ CUtensorMap tmWlo,
@@ -388,6 +467,21 @@ __global__ void __launch_bounds__(kAsThreads, 1)
       int* s_ovf = reinterpret_cast<int*>(smem_raw + (sX[0] - tc::saddr(smem_raw)));           // [G]
       unsigned int* s_cl = reinterpret_cast<unsigned int*>(smem_raw + (sX[1] - tc::saddr(smem_raw)));  // [words]
       __shared__ int s_novf, s_nlen;
+      // The first proposals of the tail (every unplaced item once) use the whole grid,
+      // one head after the other; the per-head rounds below start from them.
+      {
+        // batches of kTailItems items, numbered across the heads; warp w takes batches
+        // w, w + nwarps, ... (its head walk moves forward only)
+        int hh = 0, bbase = 0;
+        for (int bi = gwarp;; bi += nwarps) {
+          while (hh < heads && bi >= bbase + ceil_div(s_len[hh], kTailItems)) bbase += ceil_div(s_len[hh++], kTailItems);
+          if (hh >= heads) break;
+          tail_propose(a, hh, list + static_cast<size_t>(hh) * n, s_len[hh], (bi - bbase) * kTailItems,
+                       a.closed + static_cast<size_t>(hh) * words);
+        }
+      }
+      alive = sync_grid();
+      if (!alive) break;
       for (int h = blockIdx.x; h < heads; h += nblocks) {
         int lc = cur;
         int len = __ldcg(a.list_len + lc * heads + h);
@@ -410,78 +504,9 @@ __global__ void __launch_bounds__(kAsThreads, 1)
             s_nlen = 0;
           }
           __syncthreads();
-          // A. proposals, kTailItems items per warp at a time so that their row loads are in
-          // flight together; the proposal's value is the winning key's (+-0 read as +0, which
-          // the decision keys do not tell apart)
-          constexpr int kTailItems = 4;
-          for (int x0 = warp * kTailItems; x0 < len; x0 += kAsWarps * kTailItems) {
-            const int xl = x0 + lane;
-            size_t my_grow = 0;
-            long long my_row = -1;
-            if (lane < kTailItems && xl < len) {
-              my_grow = static_cast<size_t>(h) * n + __ldcg(hl + xl);
-              my_row = static_cast<long long>(__ldcg(a.tailpos + my_grow)) * a.ldt;
-            }
-            const float* rows[kTailItems];
-            unsigned long long best[kTailItems];
-#pragma unroll
-            for (int k = 0; k < kTailItems; ++k) {
-              const long long ro = __shfl_sync(0xffffffffu, my_row, k);
-              rows[k] = ro >= 0 ? a.Dtail + ro : nullptr;
-              best[k] = ~0ull;
-            }
-            int first_open = G;
-            for (int w0 = 0; w0 < words; w0 += 16) {  // 16 words of every row requested at once
-              float v[kTailItems][16];
-#pragma unroll
-              for (int k = 0; k < kTailItems; ++k) {
-#pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                  const int g = (w0 + u) * 32 + lane;
-                  v[k][u] = (rows[k] != nullptr && g < G) ? __ldcg(rows[k] + g) : kAsInf;
-                }
-              }
-#pragma unroll
-              for (int u = 0; u < 16; ++u) {
-                const int wd = w0 + u;
-                const int g = wd * 32 + lane;
-                const bool open = g < G && !((s_cl[wd < words ? wd : 0] >> lane) & 1u);
-#pragma unroll
-                for (int k = 0; k < kTailItems; ++k) {
-                  if (open && v[k][u] < kAsInf) {
-                    const unsigned long long key = decision_key(v[k][u], g);
-                    best[k] = key < best[k] ? key : best[k];
-                  }
-                }
-                const unsigned int om = __ballot_sync(0xffffffffu, open);
-                if (first_open == G && om != 0u) first_open = wd * 32 + __ffs(om) - 1;
-              }
-            }
-            unsigned long long mine = ~0ull;
-#pragma unroll
-            for (int k = 0; k < kTailItems; ++k) {
-              best[k] = warp_min_u64(best[k]);
-              if (lane == k) mine = best[k];
-            }
-            if (lane < kTailItems && xl < len) {
-              int g;
-              float pv;
-              if (mine != ~0ull) {
-                g = static_cast<int>(mine & 0xffffffffu);
-                pv = float_from_order_key(static_cast<uint32_t>(mine >> 32));
-              } else if (first_open < G) {
-                g = first_open;
-                pv = kAsInf;
-              } else {  // no open group: more items than room (cannot happen)
-                record_error(status, kErrInvalidArg);
-                g = 0;
-                pv = kAsInf;
-              }
-              a.prop_g[my_grow] = g;
-              a.prop_v[my_grow] = pv;
-              atomicAdd(cnt + g, 1);
-            }
-          }
+          // A. proposals (the first local round's came from the whole grid above)
+          if (lr > 0)
+            for (int x0 = warp * kTailItems; x0 < len; x0 += kAsWarps * kTailItems) tail_propose(a, h, hl, len, x0, s_cl);
           __syncthreads();
           // B. groups that take all their proposers; bucket offsets of the others
           {
