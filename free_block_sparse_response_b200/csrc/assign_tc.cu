@@ -12,28 +12,34 @@
 //
 // One cooperative launch per iteration, one CTA per SM, all heads.  Each round:
 //   A. proposals: the unplaced items of every head, 256 at a time, are multiplied with the
-//      head's W in chunks of 128 groups (X by TMA -- 2-D boxes in the first round,
-//      tile::gather4 rows of the unplaced list after it -- W hi and lo double-buffered and
-//      used for both 128-row halves, which halves the W traffic from L2; two accumulators
-//      per stage, double-buffered, fill the 512 TMEM columns); the epilogue forms D exactly
-//      as above and keeps the first minimum over the OPEN groups (a full group's e_g is
-//      staged as +inf, so its D never wins a strict '<' scan): the item's proposal;
+//      head's W in chunks of 128 groups (X by four 2-D TMA boxes in the first round; in
+//      the later rounds the rows of the unplaced list, read by two loader warps with
+//      coalesced loads, and W only the head's open groups, packed at the round's start
+//      with a column -> group map; W hi and lo double-buffered and used for both 128-row
+//      halves, which halves the W traffic from L2; two accumulators per stage, double-
+//      buffered, fill the 512 TMEM columns); the epilogue forms D exactly as above and
+//      keeps the first minimum over the OPEN groups (a full group's e_g is staged as +inf,
+//      so its D never wins a strict '<' scan): the item's proposal;
 //   B. per head: groups whose proposers fit their room take them all (room and full-group
 //      bit updated here); the others get bucket offsets and join the overflow list;
 //   C. every proposer of a group that takes all is placed; the others are scattered into
-//      their group's bucket as (D, token) keys;
+//      their group's bucket as (D, token) keys (slots reserved per distinct group of a
+//      warp);
 //   D. every overflowing group takes its room's worth of best proposers (radix select of
 //      the kth key) and is full; the rejected join the head's list for the next round.
 // A grid barrier separates the phases.  Every item's D row is the same fp32 numbers in
-// every round (same operands, same MMA sequence, same epilogue arithmetic), so the
-// decisions are the fill's decisions on that one matrix.  Warp roles in phase A: warp 0
-// loads, warp 2 issues the MMAs, warps 4-11 run the epilogue (two threads per row pair:
-// columns 0-63 and 64-127 of every chunk, rows r and r + 128); phases B-D use all 12
-// warps.  Per-head list lengths are staged in shared memory once per round.  Every wait is
-// bounded.  With Dout set, the first round also stores every item's D row (row stride
-// ldd) for the parity tests.  Norm mode (nrm_out set, W = Gamma, G = d): one pass over all
-// items whose epilogue forms x_i^T Gamma x_i from the accumulator row and the item's own
-// row of the X tile in shared memory, and no fill.
+// every round (same operands, same MMA sequence, same epilogue arithmetic; a packed
+// column is computed exactly as its group's full column), so the decisions are the
+// fill's decisions on that one matrix.  Once few items are left, one round also stores
+// their D rows; the tail's first proposals then run across the grid and its later rounds
+// one head per CTA from those rows.  Warp roles in phase A: warp 0 issues the TMA loads,
+// warps 1 and 3 load the gathered rows, warp 2 issues the MMAs, warps 4-11 run the
+// epilogue (two threads per row pair: columns 0-63 and 64-127 of every chunk, rows r and
+// r + 128); phases B-D use all 12 warps.  Per-head list lengths are staged in shared
+// memory once per round.  Every wait is bounded.  With Dout set, the first round also
+// stores every item's D row (row stride ldd) for the parity tests.  Norm mode (nrm_out
+// set, W = Gamma, G = d): one pass over all items whose epilogue forms x_i^T Gamma x_i from
+// the accumulator row and the item's own row of the X tile in shared memory, and no fill.
 #include <cuda.h>
 
 #include "attention.cuh"
