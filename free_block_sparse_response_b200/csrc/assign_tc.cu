@@ -596,12 +596,12 @@ __global__ void __launch_bounds__(kAsThreads, 1)
       }
       break;
     } else if (warp == 0) {
-      // producer: per work item the 256 rows of X into buffer it & 1 (lane 0 four 2-D
-      // boxes, or every lane four gather4 of 4 rows), then per chunk of 128 groups its W
-      // hi part and its lo part, each one stage of a two-stage ring.  The next item's X is
-      // issued right after this item's first lo part: that stage was freed by the previous
-      // item's last MMAs, so the X buffer the next item reuses is free, and its load
-      // overlaps all of this item's MMAs.
+      // producer: in the first round per work item the 256 rows of X into buffer it & 1
+      // (lane 0, four 2-D boxes; the later rounds' rows come from the loader warps), then
+      // per chunk of 128 groups its W hi part and its lo part, each one stage of a two-
+      // stage ring.  The next item's X is issued right after this item's first lo part:
+      // that stage was freed by the previous item's last MMAs, so the X buffer the next
+      // item reuses is free, and its load overlaps all of this item's MMAs.
       auto issue_x = [&](int it, int h, int t) -> bool {
         if (!first) return true;  // the gathered rounds' X comes from the loader warps
         const int b = it & 1, off = t * kAsRows;
