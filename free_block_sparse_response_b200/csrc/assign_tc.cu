@@ -100,15 +100,17 @@ struct HeadWalk {
   }
 };
 
-// One 64-column half-chunk of a row: D from the accumulator columns u, the first minimum
-// over the open groups merged into (best_v, best_c); u is overwritten with D.
+// One 64-column half-chunk of a row: D from the accumulator columns u (u is overwritten
+// with D), and the first minimum over the open groups merged into (best_v, best_c).  The
+// half-chunk's minimum comes from four fminf chains (NaN never wins: fminf drops it; a
+// full group's +inf never wins either); only when it is strictly below every earlier
+// column's is the first column holding it looked for, so the result is the first minimum
+// of the row in ascending column order, as a strict '<' scan would give (+-0 compare
+// equal, so the first zero of either sign is the one kept).
 __device__ __forceinline__ void scan_half_chunk(uint32_t (&u)[64], const float* s_e, int c0, float tnr, float m2t,
                                                 float& best_v, int& best_c) {
   const float4* e4 = reinterpret_cast<const float4*>(s_e + c0);
-  // four interleaved first-minimum scans over the columns j = t (mod 4), merged below
-  // (smaller value wins, equal values go to the lower column)
-  float cv[4] = {kAsInf, kAsInf, kAsInf, kAsInf};
-  int cc[4] = {-1, -1, -1, -1};
+  float mn[4] = {kAsInf, kAsInf, kAsInf, kAsInf};
   const uint64_t m2 = as_f32x2(m2t, m2t), tn2 = as_f32x2(tnr, tnr);
 #pragma unroll
   for (int qq = 0; qq < 16; ++qq) {
@@ -123,24 +125,17 @@ __device__ __forceinline__ void scan_half_chunk(uint32_t (&u)[64], const float* 
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       u[4 * qq + t] = __float_as_uint(v[t]);
-      if (v[t] < cv[t]) {
-        cv[t] = v[t];
-        cc[t] = 4 * qq + t;
-      }
+      mn[t] = fminf(mn[t], v[t]);
     }
   }
-  float seg_v = cv[0];
-  int seg_c = cc[0];
+  const float m = fminf(fminf(mn[0], mn[1]), fminf(mn[2], mn[3]));
+  if (m < best_v) {  // chunks ascend: only a strictly smaller value can displace the best
+    int idx = 0;
 #pragma unroll
-  for (int t = 1; t < 4; ++t) {
-    if (cc[t] >= 0 && (seg_c < 0 || cv[t] < seg_v || (cv[t] == seg_v && cc[t] < seg_c))) {
-      seg_v = cv[t];
-      seg_c = cc[t];
-    }
-  }
-  if (seg_c >= 0 && seg_v < best_v) {  // chunks in ascending order: strictly smaller wins
-    best_v = seg_v;
-    best_c = c0 + seg_c;
+    for (int k = 63; k >= 0; --k)
+      if (__uint_as_float(u[k]) == m) idx = k;
+    best_v = m;
+    best_c = c0 + idx;
   }
 }
 
